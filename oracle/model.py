@@ -1,0 +1,382 @@
+"""fp64 forward and backward of the Llama-style decoder trained by MegaTrain.
+
+TEST INFRASTRUCTURE ONLY (see the package docstring). Plain numpy in float64.
+
+Model, in the notation used throughout (weights stored [out, in]):
+  x0       = E[tok]                                  embedding gather
+  per layer:
+    u      = RMSNorm(x) * g1
+    q,k,v  = u Wq^T, u Wk^T, u Wv^T ; q,k <- RoPE(q), RoPE(k)
+    a      = causal softmax(q k^T / sqrt(hd)) v      per head, GQA grouping
+    h      = x + a Wo^T
+    w      = RMSNorm(h) * g2
+    x'     = h + (silu(w Wg^T) * (w Wu^T)) Wd^T
+  n        = RMSNorm(x_L) * gf ;  z = n Whead^T
+  loss     = mean_t [ logsumexp(z_t) - z_t[y_t] ]
+
+The MegaTrain pages ("MegaTrain: Full Precision Training of 100B+ Parameter
+Large Language Models on a Single GPU", abstract; saify.me, "The memory-centric
+design") say which decoder families are trained but not their equations; the
+block above is the plain pre-norm Llama reading, and each function names the
+reading it takes.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+# Tensor ids of the arena layout (same numbering as the seeded input module,
+# restated here so the oracle depends on nothing outside numpy).
+ATTN_NORM, WQ, WK, WV, WO, MLP_NORM, WGATE, WUP, WDOWN = range(9)
+EMBED, FINAL_NORM, LM_HEAD = 100, 101, 102
+
+ALIGN_FLOATS = 64  # every tensor of the fp32 arena starts on a 256-byte boundary
+
+
+@dataclass(frozen=True)
+class OracleConfig:
+    L: int
+    d: int
+    H: int
+    Hkv: int
+    F: int
+    V: int
+    b: int
+    s: int
+    norm_eps: float = 1e-5
+    rope_base: float = 10000.0
+    lr: float = 1e-3
+    beta1: float = 0.9
+    beta2: float = 0.95
+    adam_eps: float = 1e-8
+    wd: float = 0.1
+
+    @property
+    def hd(self) -> int:
+        return self.d // self.H
+
+
+# ---------------------------------------------------------------------------
+# Host arena layout: the flat fp32 master-parameter array the caller owns.
+# ---------------------------------------------------------------------------
+
+def _layer_tensors(c: OracleConfig):
+    hd = c.hd
+    return [
+        (ATTN_NORM, (c.d,)),
+        (WQ, (c.H * hd, c.d)),
+        (WK, (c.Hkv * hd, c.d)),
+        (WV, (c.Hkv * hd, c.d)),
+        (WO, (c.d, c.H * hd)),
+        (MLP_NORM, (c.d,)),
+        (WGATE, (c.F, c.d)),
+        (WUP, (c.F, c.d)),
+        (WDOWN, (c.d, c.F)),
+    ]
+
+
+def arena_layout(c: OracleConfig):
+    """List of (layer, tensor id, offset in floats, shape) in arena order:
+    embedding, then each layer's nine tensors, then the final norm and the
+    untied LM head. Offsets are rounded up to 64 floats (256 bytes)."""
+    out = []
+    off = 0
+
+    def put(layer, tid, shape):
+        nonlocal off
+        out.append((layer, tid, off, shape))
+        n = int(np.prod(shape))
+        off += (n + ALIGN_FLOATS - 1) // ALIGN_FLOATS * ALIGN_FLOATS
+
+    put(-1, EMBED, (c.V, c.d))
+    for l in range(c.L):
+        for tid, shape in _layer_tensors(c):
+            put(l, tid, shape)
+    put(-1, FINAL_NORM, (c.d,))
+    put(-1, LM_HEAD, (c.V, c.d))
+    return out, off
+
+
+def arena_floats(c: OracleConfig) -> int:
+    return arena_layout(c)[1]
+
+
+def unpack_arena(arena: np.ndarray, c: OracleConfig, dtype=np.float64) -> dict:
+    """Views of the arena as a dict keyed by (layer, tensor id), cast to dtype."""
+    layout, total = arena_layout(c)
+    assert arena.size >= total, (arena.size, total)
+    out = {}
+    for layer, tid, off, shape in layout:
+        n = int(np.prod(shape))
+        out[(layer, tid)] = arena[off:off + n].reshape(shape).astype(dtype)
+    return out
+
+
+def pack_arena(tensors: dict, c: OracleConfig) -> np.ndarray:
+    """Inverse of unpack_arena (padding left at zero), as fp32."""
+    layout, total = arena_layout(c)
+    arena = np.zeros(total, dtype=np.float32)
+    for layer, tid, off, shape in layout:
+        t = np.asarray(tensors[(layer, tid)], dtype=np.float32).reshape(-1)
+        arena[off:off + t.size] = t
+    return arena
+
+
+# ---------------------------------------------------------------------------
+# bf16 round-to-nearest-even (the streamed copy of the master weights).
+# ---------------------------------------------------------------------------
+
+def bf16_round(x) -> np.ndarray:
+    """Round fp32 values to the nearest bfloat16 (ties to even), returned as
+    float64. bfloat16 keeps the top 16 bits of the IEEE binary32 pattern, so
+    the value is the binary32 pattern with the low 16 bits cleared after
+    adding half an ulp (0x7fff plus the kept lsb). NaN stays NaN."""
+    f = np.asarray(x, dtype=np.float32)
+    bits = f.view(np.uint32).astype(np.uint64)
+    lsb = (bits >> 16) & 1
+    rounded = ((bits + 0x7FFF + lsb) >> 16) << 16
+    out = (rounded & 0xFFFFFFFF).astype(np.uint32).view(np.float32).astype(np.float64)
+    return np.where(np.isnan(f), np.nan, out)
+
+
+# ---------------------------------------------------------------------------
+# RMSNorm. Reading: y = x / sqrt(mean(x^2) + eps) * g, eps inside the root.
+# ---------------------------------------------------------------------------
+
+def rmsnorm_fwd(x: np.ndarray, g: np.ndarray, eps: float):
+    """Returns (y, r) with r = 1/sqrt(mean(x^2, last axis) + eps)."""
+    r = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return x * r * g, r
+
+
+def rmsnorm_bwd(x: np.ndarray, g: np.ndarray, r: np.ndarray, dy: np.ndarray):
+    """Gradient of y_i = g_i x_i r with r = (sum_j x_j^2 / d + eps)^(-1/2).
+    dr/dx_j = -r^3 x_j / d, hence
+      dx_j = r g_j dy_j - (r^3 x_j / d) sum_i g_i dy_i x_i,
+      dg_i = sum over rows of dy_i x_i r.
+    Returns (dx, dg)."""
+    d = x.shape[-1]
+    gdy = g * dy
+    dot = np.sum(gdy * x, axis=-1, keepdims=True)
+    dx = r * gdy - (r ** 3) * x * dot / d
+    dg = np.sum((dy * x * r).reshape(-1, d), axis=0)
+    return dx, dg
+
+
+# ---------------------------------------------------------------------------
+# RoPE. Reading: rotate-half pairing (i, i + hd/2), theta_i = base^(-2i/hd),
+# positions 0..s-1 restarting for every sequence.
+# ---------------------------------------------------------------------------
+
+def rope_tables(s: int, hd: int, base: float):
+    """cos and sin tables of shape [s, hd/2]: angle[p, i] = p * base^(-2i/hd)."""
+    i = np.arange(hd // 2, dtype=np.float64)
+    theta = base ** (-2.0 * i / hd)
+    ang = np.arange(s, dtype=np.float64)[:, None] * theta[None, :]
+    return np.cos(ang), np.sin(ang)
+
+
+def rope_fwd(x: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """x: [b, s, heads, hd]. Rotates each pair (x_i, x_{i+hd/2}) by angle[p, i]:
+      x'_i        = x_i cos - x_{i+hd/2} sin
+      x'_{i+hd/2} = x_{i+hd/2} cos + x_i sin"""
+    half = x.shape[-1] // 2
+    c = cos[None, :, None, :]
+    s = sin[None, :, None, :]
+    x1, x2 = x[..., :half], x[..., half:]
+    return np.concatenate([x1 * c - x2 * s, x2 * c + x1 * s], axis=-1)
+
+
+def rope_bwd(dy: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
+    """Transpose of the rotation (rotation by -angle)."""
+    half = dy.shape[-1] // 2
+    c = cos[None, :, None, :]
+    s = sin[None, :, None, :]
+    d1, d2 = dy[..., :half], dy[..., half:]
+    return np.concatenate([d1 * c + d2 * s, d2 * c - d1 * s], axis=-1)
+
+
+# ---------------------------------------------------------------------------
+# Causal attention with grouped KV heads. Reading: scale 1/sqrt(hd), key j is
+# visible to query i iff j <= i (same sequence); query head h reads KV head
+# floor(h / (H / Hkv)).
+# ---------------------------------------------------------------------------
+
+def attention_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray):
+    """q: [b, s, H, hd]; k, v: [b, s, Hkv, hd]. Returns (o [b,s,H,hd], P [b,H,s,s])."""
+    b, s, H, hd = q.shape
+    Hkv = k.shape[2]
+    group = H // Hkv
+    kk = np.repeat(k, group, axis=2)  # kv head for query head h is h // group
+    vv = np.repeat(v, group, axis=2)
+    S = np.einsum("bihd,bjhd->bhij", q, kk) / np.sqrt(hd)
+    mask = np.tril(np.ones((s, s), dtype=bool))
+    S = np.where(mask[None, None], S, -np.inf)
+    S = S - S.max(axis=-1, keepdims=True)
+    P = np.exp(S)
+    P = P / P.sum(axis=-1, keepdims=True)
+    o = np.einsum("bhij,bjhd->bihd", P, vv)
+    return o, P
+
+
+def attention_bwd(q, k, v, P, do):
+    """Backward of o = P v with P = softmax(q k^T / sqrt(hd)) (causal):
+      dP = do v^T ; dv = P^T do ; dS = P * (dP - rowsum(dP * P)) ;
+      dq = dS k / sqrt(hd) ; dk = dS^T q / sqrt(hd);
+    dk, dv of a KV head sum over the query heads of its group."""
+    b, s, H, hd = q.shape
+    Hkv = k.shape[2]
+    group = H // Hkv
+    kk = np.repeat(k, group, axis=2)
+    vv = np.repeat(v, group, axis=2)
+    dP = np.einsum("bihd,bjhd->bhij", do, vv)
+    dvv = np.einsum("bhij,bihd->bjhd", P, do)
+    dS = P * (dP - np.sum(dP * P, axis=-1, keepdims=True))
+    scale = 1.0 / np.sqrt(hd)
+    dq = np.einsum("bhij,bjhd->bihd", dS, kk) * scale
+    dkk = np.einsum("bhij,bihd->bjhd", dS, q) * scale
+    dk = dkk.reshape(b, s, Hkv, group, hd).sum(axis=3)
+    dv = dvv.reshape(b, s, Hkv, group, hd).sum(axis=3)
+    return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# SwiGLU. Reading: act = silu(gate) * up, silu(z) = z * sigmoid(z).
+# ---------------------------------------------------------------------------
+
+def _sigmoid(z):
+    return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z):
+    return z * _sigmoid(z)
+
+
+def swiglu_fwd(gt, up):
+    return silu(gt) * up
+
+
+def swiglu_bwd(gt, up, dact):
+    """d/dz silu(z) = sigmoid(z) (1 + z (1 - sigmoid(z)))."""
+    sg = _sigmoid(gt)
+    dgt = dact * up * sg * (1.0 + gt * (1.0 - sg))
+    dup = dact * gt * sg
+    return dgt, dup
+
+
+# ---------------------------------------------------------------------------
+# One decoder layer.
+# ---------------------------------------------------------------------------
+
+def layer_fwd(x: np.ndarray, W: dict, c: OracleConfig, cos, sin):
+    """x: [b, s, d] -> (x_next, cache). W keys: ATTN_NORM, WQ, ..., WDOWN."""
+    b, s, d = x.shape
+    hd = c.hd
+    u, r1 = rmsnorm_fwd(x, W[ATTN_NORM], c.norm_eps)
+    q = (u @ W[WQ].T).reshape(b, s, c.H, hd)
+    k = (u @ W[WK].T).reshape(b, s, c.Hkv, hd)
+    v = (u @ W[WV].T).reshape(b, s, c.Hkv, hd)
+    qr = rope_fwd(q, cos, sin)
+    kr = rope_fwd(k, cos, sin)
+    o, P = attention_fwd(qr, kr, v)
+    a = o.reshape(b, s, c.H * hd)
+    h = x + a @ W[WO].T
+    w, r2 = rmsnorm_fwd(h, W[MLP_NORM], c.norm_eps)
+    gt = w @ W[WGATE].T
+    up = w @ W[WUP].T
+    act = swiglu_fwd(gt, up)
+    x_next = h + act @ W[WDOWN].T
+    cache = dict(x=x, u=u, r1=r1, qr=qr, kr=kr, v=v, P=P, a=a, h=h, w=w, r2=r2,
+                 gt=gt, up=up, act=act)
+    return x_next, cache
+
+
+def layer_bwd(dxn: np.ndarray, W: dict, cache: dict, c: OracleConfig, cos, sin):
+    """Gradient of a layer given dL/dx_next. Returns (dx, dW dict)."""
+    b, s, d = dxn.shape
+    hd = c.hd
+    T = b * s
+    x, u, h, w, a, act = (cache[k] for k in ("x", "u", "h", "w", "a", "act"))
+    G = {}
+    # x' = h + act Wd^T
+    G[WDOWN] = dxn.reshape(T, d).T @ act.reshape(T, c.F)
+    dact = dxn @ W[WDOWN]
+    dgt, dup = swiglu_bwd(cache["gt"], cache["up"], dact)
+    G[WGATE] = dgt.reshape(T, c.F).T @ w.reshape(T, d)
+    G[WUP] = dup.reshape(T, c.F).T @ w.reshape(T, d)
+    dw = dgt @ W[WGATE] + dup @ W[WUP]
+    dh_norm, G[MLP_NORM] = rmsnorm_bwd(h, W[MLP_NORM], cache["r2"], dw)
+    dh = dxn + dh_norm
+    # h = x + a Wo^T
+    G[WO] = dh.reshape(T, d).T @ a.reshape(T, c.H * hd)
+    da = (dh @ W[WO]).reshape(b, s, c.H, hd)
+    dqr, dkr, dv = attention_bwd(cache["qr"], cache["kr"], cache["v"], cache["P"], da)
+    dq = rope_bwd(dqr, cos, sin).reshape(T, c.H * hd)
+    dk = rope_bwd(dkr, cos, sin).reshape(T, c.Hkv * hd)
+    dv = dv.reshape(T, c.Hkv * hd)
+    uf = u.reshape(T, d)
+    G[WQ] = dq.T @ uf
+    G[WK] = dk.T @ uf
+    G[WV] = dv.T @ uf
+    du = (dq @ W[WQ] + dk @ W[WK] + dv @ W[WV]).reshape(b, s, d)
+    dx_norm, G[ATTN_NORM] = rmsnorm_bwd(x, W[ATTN_NORM], cache["r1"], du)
+    return dh + dx_norm, G
+
+
+# ---------------------------------------------------------------------------
+# Head: final norm, untied LM head, mean next-token cross-entropy.
+# ---------------------------------------------------------------------------
+
+def head_ce_fwd_bwd(xL, gf, Whead, labels, eps):
+    """xL: [T, d]; labels: [T] ints. Returns (loss, dxL, dgf, dWhead) with
+      z = RMSNorm(xL) gf Whead^T, loss = mean_t(logsumexp(z_t) - z_t[y_t]),
+      dz = (softmax(z) - onehot(y)) / T."""
+    T = xL.shape[0]
+    n, r = rmsnorm_fwd(xL, gf, eps)
+    z = n @ Whead.T
+    zmax = z.max(axis=-1, keepdims=True)
+    lse = zmax[:, 0] + np.log(np.sum(np.exp(z - zmax), axis=-1))
+    idx = np.arange(T)
+    loss = float(np.mean(lse - z[idx, labels]))
+    dz = np.exp(z - lse[:, None])
+    dz[idx, labels] -= 1.0
+    dz /= T
+    dWhead = dz.T @ n
+    dn = dz @ Whead
+    dxL, dgf = rmsnorm_bwd(xL, gf, r, dn)
+    return loss, dxL, dgf, dWhead
+
+
+# ---------------------------------------------------------------------------
+# Whole training step (loss and gradients; the update is in adamw.py).
+# ---------------------------------------------------------------------------
+
+def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
+                     c: OracleConfig):
+    """weights: dict (layer, tensor id) -> float64 array, the values the forward
+    and backward use. tokens, labels: int [b, s]. Returns (loss, grads dict)."""
+    b, s = tokens.shape
+    T = b * s
+    cos, sin = rope_tables(s, c.hd, c.rope_base)
+    E = weights[(-1, EMBED)]
+    x = E[tokens]  # [b, s, d]
+    caches = []
+    for l in range(c.L):
+        W = {tid: weights[(l, tid)] for tid in range(9)}
+        x, cache = layer_fwd(x, W, c, cos, sin)
+        caches.append(cache)
+    loss, dx, dgf, dWhead = head_ce_fwd_bwd(
+        x.reshape(T, c.d), weights[(-1, FINAL_NORM)], weights[(-1, LM_HEAD)],
+        labels.reshape(T), c.norm_eps)
+    grads = {(-1, FINAL_NORM): dgf, (-1, LM_HEAD): dWhead}
+    dx = dx.reshape(b, s, c.d)
+    for l in reversed(range(c.L)):
+        W = {tid: weights[(l, tid)] for tid in range(9)}
+        dx, G = layer_bwd(dx, W, caches[l], c, cos, sin)
+        for tid, g in G.items():
+            grads[(l, tid)] = g
+    dE = np.zeros_like(E)
+    np.add.at(dE, tokens.reshape(T), dx.reshape(T, c.d))
+    grads[(-1, EMBED)] = dE
+    return loss, grads
