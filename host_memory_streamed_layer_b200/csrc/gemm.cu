@@ -1,0 +1,403 @@
+// Persistent tcgen05 bf16 GEMM for sm_100a: C[M,N] = A[M,K] * B[N,K]^T, fp32
+// accumulation in tensor memory, operands staged by TMA (no multicast).
+//
+// This is the dense contraction of every projection in the streamed decoder
+// layer (MegaTrain, "Full Precision Training of 100B+ Parameter Large Language
+// Models on a Single GPU", abstract: each streamed layer "runs the matmuls",
+// saify.me "The memory-centric design"): the forward products u Wqkv^T, a Wo^T,
+// w Wgu^T, act Wd^T, the input-gradient products dY W and the weight-gradient
+// products dY^T X of their backward.
+//
+// Operands may be K-major (the reduction index is contiguous) or MN-major (the
+// output index is contiguous), which covers all three products without a
+// transpose kernel:
+//   forward   Y  = X  W^T : A = X  [T, in]  K-major,  B = W [out, in] K-major
+//   input grad dX = dY W   : A = dY [T, out] K-major,  B = W [out, in] MN-major
+//   weight grad dW = dY^T X: A = dY [T, out] MN-major, B = X [T, in]  MN-major
+//
+// Kernel structure (one CTA per SM, persistent over output tiles):
+//   warp 0      TMA producer: fills a ring of shared-memory stages
+//   warp 1      MMA issuer: one thread issues tcgen05.mma 128 x BN x 16
+//   warps 2..5  epilogue: tcgen05.ld from tensor memory, convert, store
+// The accumulator is double-buffered in tensor memory (2 x BN columns) so the
+// epilogue of tile i overlaps the main loop of tile i+1.
+#include <cstdio>
+#include <mutex>
+
+#include "mt_common.cuh"
+#include "mt_internal.h"
+
+namespace mt {
+
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;  // 64 bf16 = 128 bytes: one swizzle row
+constexpr int NUM_THREADS = 192;
+constexpr int GROUP_M = 16;  // tile raster: 16 M-tiles share a band of N-tiles
+
+template <int BN>
+struct Cfg {
+  static constexpr int A_BYTES = BM * BK * 2;
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr uint32_t TMEM_COLS = 2 * BN;
+};
+
+struct Params {
+  int M, N, K;
+  void* C;
+  int64_t ldc;
+  const float* R;
+  int64_t ldr;
+  int epi;
+  int* err;
+};
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
+  const int per_group = GROUP_M * num_n;
+  const int g = tile / per_group;
+  const int first_m = g * GROUP_M;
+  const int gsize = min(num_m - first_m, GROUP_M);
+  const int r = tile - g * per_group;
+  mb = first_m + r % gsize;
+  nb = r / gsize;
+}
+
+template <int BN, bool A_MN, bool B_MN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    k_gemm_bf16(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, Params p) {
+  using C = Cfg<BN>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tfull = empty + C::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_m = (p.M + BM - 1) / BM;
+  const int num_n = (p.N + BN - 1) / BN;
+  const int num_tiles = num_m * num_n;
+  const int num_kb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int last_phase[C::STAGES];
+#pragma unroll
+      for (int s = 0; s < C::STAGES; ++s) last_phase[s] = -1;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        int mb, nb;
+        tile_coords(tile, num_m, num_n, mb, nb);
+        const int m0 = mb * BM, n0 = nb * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (*abort_flag || !mbar_wait(&empty[stage], phase ^ 1)) {
+            record_error(p.err, DEV_TIMEOUT_PRODUCER);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * C::STAGE_BYTES;
+          uint8_t* sb = sa + C::A_BYTES;
+          mbar_arrive_expect_tx(&full[stage], C::STAGE_BYTES);
+          const int k0 = kb * BK;
+          if (!A_MN) {
+            tma_load_2d(sa, &tmA, &full[stage], k0, m0);
+          } else {
+#pragma unroll
+            for (int i = 0; i < BM / 64; ++i) tma_load_2d(sa + i * 8192, &tmA, &full[stage], m0 + i * 64, k0);
+          }
+          if (!B_MN) {
+            tma_load_2d(sb, &tmB, &full[stage], k0, n0);
+          } else {
+#pragma unroll
+            for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, &tmB, &full[stage], n0 + i * 64, k0);
+          }
+#pragma unroll
+          for (int s = 0; s < C::STAGES; ++s)
+            if (s == stage) last_phase[s] = (int)phase;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // Let every issued copy land before the CTA's shared memory goes away.
+#pragma unroll
+        for (int s = 0; s < C::STAGES; ++s)
+          if (last_phase[s] >= 0 && !mbar_wait(&full[s], (uint32_t)last_phase[s]))
+            record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, A_MN, B_MN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      bool issued = false;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (*abort_flag || !mbar_wait(&tempty[acc], acc_phase ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (*abort_flag || !mbar_wait(&full[stage], phase)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * C::STAGE_BYTES);
+          const uint32_t sb = sa + C::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            uint64_t ad, bd;
+            if (!A_MN)
+              ad = sdesc_sw128(sa + kk * 32, 16, 1024);
+            else
+              ad = sdesc_sw128(sa + kk * 2048, 8192, 1024);
+            if (!B_MN)
+              bd = sdesc_sw128(sb + kk * 32, 16, 1024);
+            else
+              bd = sdesc_sw128(sb + kk * 2048, 8192, 1024);
+            umma_bf16(d_tmem, ad, bd, idesc, (kb | kk) != 0);
+          }
+          issued = true;
+          umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[acc]);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      if (!ok) {
+        record_error(p.err, DEV_TIMEOUT_MMA);
+        *abort_flag = 1;
+        if (issued) {
+          umma_commit(drain);
+          if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        }
+      }
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quarter = warp & 3;  // tensor-memory lanes this warp may read
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      if (*abort_flag || !mbar_wait(&tfull[acc], acc_phase)) {
+        record_error(p.err, DEV_TIMEOUT_EPILOGUE);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      int mb, nb;
+      tile_coords(tile, num_m, num_n, mb, nb);
+      const int row = mb * BM + quarter * 32 + lane;
+      const bool row_ok = row < p.M;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_wait();
+        const int col0 = nb * BN + c * 32;
+        if (!row_ok || col0 >= p.N) continue;
+        const bool full_cols = col0 + 32 <= p.N;
+        if (p.epi == EPI_BF16) {
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(p.C) + (int64_t)row * p.ldc + col0;
+          if (full_cols) {
+            uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(r[8 * j + 0]), __uint_as_float(r[8 * j + 1]));
+              w.y = pack_bf16x2(__uint_as_float(r[8 * j + 2]), __uint_as_float(r[8 * j + 3]));
+              w.z = pack_bf16x2(__uint_as_float(r[8 * j + 4]), __uint_as_float(r[8 * j + 5]));
+              w.w = pack_bf16x2(__uint_as_float(r[8 * j + 6]), __uint_as_float(r[8 * j + 7]));
+              o4[j] = w;
+            }
+          } else {
+            const int nv = p.N - col0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nv) out[j] = __float2bfloat16_rn(__uint_as_float(r[j]));
+          }
+        } else {
+          float* out = reinterpret_cast<float*>(p.C) + (int64_t)row * p.ldc + col0;
+          const float* res = (p.epi == EPI_F32_ADD) ? p.R + (int64_t)row * p.ldr + col0 : nullptr;
+          if (full_cols) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              float4 v = make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                                     __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3]));
+              if (res) {
+                const float4 q = reinterpret_cast<const float4*>(res)[j];
+                v.x += q.x;
+                v.y += q.y;
+                v.z += q.z;
+                v.w += q.w;
+              }
+              reinterpret_cast<float4*>(out)[j] = v;
+            }
+          } else {
+            const int nv = p.N - col0;
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nv) out[j] = __uint_as_float(r[j]) + (res ? res[j] : 0.f);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side.
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2-D bf16 tensor map: inner extent `inner` (contiguous), outer extent `outer`,
+// row pitch `ld` elements, box {64, box_outer}, 128-byte swizzle, zero fill.
+bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld, int box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int g_num_sms = 0;
+
+template <int BN, bool A_MN, bool B_MN>
+int launch(const GemmDesc& g, cudaStream_t st, int* err) {
+  using C = Cfg<BN>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    if (cudaFuncSetAttribute(k_gemm_bf16<BN, A_MN, B_MN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+        cudaSuccess)
+      return MT_ERR_CUDA;
+    attr_set = true;
+  }
+  CUtensorMap ta, tb;
+  bool ok = A_MN ? make_map(&ta, g.A, g.M, g.K, g.lda, 64) : make_map(&ta, g.A, g.K, g.M, g.lda, BM);
+  ok = ok && (B_MN ? make_map(&tb, g.B, g.N, g.K, g.ldb, 64) : make_map(&tb, g.B, g.K, g.N, g.ldb, BN));
+  if (!ok) return MT_ERR_ARG;
+  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err};
+  const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
+  const int grid = tiles < g_num_sms ? tiles : g_num_sms;
+  k_gemm_bf16<BN, A_MN, B_MN><<<grid, NUM_THREADS, C::SMEM, st>>>(ta, tb, p);
+  return cudaGetLastError() == cudaSuccess ? MT_OK : MT_ERR_CUDA;
+}
+
+template <int BN>
+int dispatch_major(const GemmDesc& g, cudaStream_t st, int* err) {
+  if (!g.a_mn && !g.b_mn) return launch<BN, false, false>(g, st, err);
+  if (!g.a_mn && g.b_mn) return launch<BN, false, true>(g, st, err);
+  if (g.a_mn && !g.b_mn) return launch<BN, true, false>(g, st, err);
+  return launch<BN, true, true>(g, st, err);
+}
+
+}  // namespace
+
+int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* err) {
+  if (g.M <= 0 || g.N <= 0 || g.K <= 0) return (g.M == 0 || g.N == 0) ? MT_OK : MT_ERR_ARG;
+  if (!g.A || !g.B || !g.C) return MT_ERR_ARG;
+  if (g.epi == EPI_F32_ADD && !g.R) return MT_ERR_ARG;
+  // TMA: 16-byte aligned base and row pitch; 16-byte aligned epilogue stores.
+  auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
+  if (!al16(g.A) || !al16(g.B) || !al16(g.C) || (g.R && !al16(g.R))) return MT_ERR_ARG;
+  if ((g.lda % 8) || (g.ldb % 8) || (g.ldc % 8) || (g.R && (g.ldr % 4))) return MT_ERR_ARG;
+  if (g_num_sms == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) return MT_ERR_CUDA;
+  }
+  const int tiles256 = ((g.M + BM - 1) / BM) * ((g.N + 255) / 256);
+  if (g.N > 128 && tiles256 >= g_num_sms) return dispatch_major<256>(g, st, err);
+  return dispatch_major<128>(g, st, err);
+}
+
+}  // namespace mt

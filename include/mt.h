@@ -1,0 +1,157 @@
+/*
+ * mt.h -- C interface of the host-memory-streamed layer training library.
+ *
+ * One training step of a Llama-style decoder whose fp32 master weights and
+ * AdamW moments live in pinned host memory. Every layer's bf16 weights are
+ * streamed to the GPU, run through forward, checkpointed recompute and
+ * backward, and its fp32 gradients are streamed back to the host, where AdamW
+ * updates the master weights. The method is MegaTrain's memory-centric
+ * training: "MegaTrain: Full Precision Training of 100B+ Parameter Large
+ * Language Models on a Single GPU" (arXiv 2604.05091), abstract: parameters
+ * and optimizer states stay in host memory, the GPU is a transient compute
+ * engine, and per layer parameters stream in and gradients stream out, through
+ * a pipelined double-buffered engine on several CUDA streams with stateless
+ * layer templates.
+ *
+ * Conventions for every function below:
+ *   - return 0 (MT_OK) on success or a negative MT_ERR_* code; nothing aborts
+ *     or exits the process; mt_last_error() gives a message for the context;
+ *   - argument, configuration and token-range errors are detected on the host
+ *     before any device work and leave all state untouched;
+ *   - a context is not thread-safe: one caller thread at a time.
+ */
+#ifndef MT_H_
+#define MT_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MT_OK 0
+#define MT_ERR_ARG (-1)        /* bad pointer, size or value */
+#define MT_ERR_CONFIG (-2)     /* configuration outside what the kernels support */
+#define MT_ERR_ARENA (-3)      /* host arena too small or misaligned */
+#define MT_ERR_NOMEM (-4)      /* device or host allocation failed, or budget exceeded */
+#define MT_ERR_PIN (-5)        /* pinning the host arena failed */
+#define MT_ERR_CUDA (-6)       /* a CUDA runtime call failed */
+#define MT_ERR_TIMEOUT (-7)    /* a bounded wait (host or device) ran out */
+#define MT_ERR_NONFINITE (-8)  /* a gradient was NaN or Inf: remaining updates skipped */
+#define MT_ERR_DEVICE (-9)     /* a kernel reported an error through its error word */
+
+/* Flags (mt_config.flags). */
+#define MT_FLAG_SERIALIZE 0x1u     /* run copies and kernels on one stream (debug) */
+#define MT_FLAG_KERNEL_TIMING 0x2u /* time GEMM / attention launches with events */
+#define MT_FLAG_NO_UPDATE 0x4u     /* compute loss and gradients only, skip AdamW */
+
+/* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
+#define MT_T_ATTN_NORM 0
+#define MT_T_WQ 1
+#define MT_T_WK 2
+#define MT_T_WV 3
+#define MT_T_WO 4
+#define MT_T_MLP_NORM 5
+#define MT_T_WGATE 6
+#define MT_T_WUP 7
+#define MT_T_WDOWN 8
+#define MT_T_EMBED 100
+#define MT_T_FINAL_NORM 101
+#define MT_T_LM_HEAD 102
+
+typedef struct mt_config {
+  uint32_t struct_size; /* sizeof(mt_config); lets the layout grow */
+  int32_t L;            /* decoder layers */
+  int32_t d;            /* model width */
+  int32_t H;            /* query heads; head_dim = d / H, 64 or 128 */
+  int32_t Hkv;          /* key/value heads, divides H */
+  int32_t F;            /* SwiGLU hidden width */
+  int32_t V;            /* vocabulary */
+  int32_t b;            /* sequences per step */
+  int32_t s;            /* tokens per sequence */
+  float norm_eps;       /* RMSNorm epsilon, inside the square root */
+  float rope_base;      /* RoPE base, theta_i = base^(-2i/head_dim) */
+  float lr, beta1, beta2, adam_eps, wd; /* AdamW, decoupled decay on all tensors */
+  uint64_t seed;        /* initial weights when the library owns the arena */
+  uint32_t flags;       /* MT_FLAG_* */
+  int32_t device;       /* CUDA device ordinal */
+  int32_t host_threads; /* host AdamW threads; 0 = all cores but one */
+} mt_config;
+
+typedef struct mt_ctx mt_ctx;
+
+/* Per-step counters, filled by mt_get_stats for the last mt_train_step. */
+typedef struct mt_stats {
+  double step_ms;           /* compute-stream time of the step (device events) */
+  double fwd_ms, head_ms, bwd_ms; /* compute-stream phases */
+  double h2d_bytes, d2h_bytes;    /* bytes moved over the host link */
+  double h2d_ms, d2h_ms;          /* copy-stream busy time */
+  double wait_weights_ms;   /* compute stream idle waiting for prefetched weights */
+  double adamw_ms;          /* host optimizer busy time (wall) */
+  double adamw_bytes;       /* host DRAM bytes the optimizer touched */
+  double gemm_flops, gemm_ms; int64_t gemm_launches;  /* with MT_FLAG_KERNEL_TIMING */
+  double attn_flops, attn_ms; int64_t attn_launches;
+  int64_t kernel_launches;  /* kernels this library launched during the step */
+} mt_stats;
+
+/* Fills *cfg with the defaults (struct_size set, hyper-parameters of the
+ * workloads: eps 1e-5, RoPE base 10000, lr 1e-3, betas (0.9, 0.95), eps 1e-8,
+ * wd 0.1). Shapes are left zero. */
+int mt_config_default(mt_config* cfg);
+
+/* Bytes of the fp32 master arena for cfg: the embedding [V,d]; per layer the
+ * attention-norm gain [d], Wq [H*hd,d], Wk [Hkv*hd,d], Wv [Hkv*hd,d],
+ * Wo [d,H*hd], MLP-norm gain [d], Wgate [F,d], Wup [F,d], Wdown [d,F]; then the
+ * final-norm gain [d] and the untied LM head [V,d]. Weights are row-major
+ * [out, in]; every tensor starts on a 256-byte boundary. 0 for a bad cfg. */
+size_t mt_arena_bytes(const mt_config* cfg);
+
+/* Offset (in floats) and element count of one tensor of the arena. */
+int mt_tensor_offset(const mt_config* cfg, int layer, int tensor_id, size_t* offset_floats, size_t* numel);
+
+/* Host bytes the context holds besides the caller's arena: two fp32 Adam
+ * moments (8 B/param), the fp32 gradient arena (4 B/param) and the bf16
+ * streaming copy (2 B/param), plus padding. */
+size_t mt_host_state_bytes(const mt_config* cfg);
+
+/* Creates a context on cfg->device. host_param_arena: the caller's fp32
+ * master weights in the layout of mt_arena_bytes, at least arena_bytes long and
+ * 256-byte aligned; the library pins it (cudaHostRegister) for the context's
+ * lifetime and updates it in place every step. NULL: the library allocates the
+ * arena and fills it from cfg->seed (gains 1, matrices N(0, 0.02^2)). The
+ * library owns the moments, the gradient arena, the bf16 copy and all device
+ * memory. Fails with MT_ERR_NOMEM before allocating if the device budget does
+ * not fit. */
+int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, mt_ctx** out);
+
+/* One training step: tokens and labels are host int32 arrays of b*s ids in
+ * [0, V), sequence-major. Runs forward, loss, backward and the host AdamW
+ * update (bias correction from step 1), and writes the mean next-token
+ * cross-entropy (computed before the update) to *loss_out. Returns
+ * MT_ERR_NONFINITE if a gradient was not finite: the updates of the tensors
+ * not yet updated are skipped and the arena is partly updated. */
+int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, float* loss_out);
+
+/* Copies the fp32 gradients of the last step (taken before the update), in the
+ * arena layout, to dst (bytes >= mt_arena_bytes). */
+int mt_get_grads(mt_ctx* ctx, float* dst, size_t bytes);
+
+/* Copies the current fp32 master weights (after the last update) to dst. */
+int mt_get_params(mt_ctx* ctx, float* dst, size_t bytes);
+
+/* Counters of the last step. */
+int mt_get_stats(mt_ctx* ctx, mt_stats* out);
+
+/* Waits for the context's streams, frees its device memory and unpins or
+ * frees its host memory. NULL is ignored. */
+void mt_destroy(mt_ctx* ctx);
+
+/* Message of the last error of ctx (or of the last failed mt_create when ctx
+ * is NULL). Valid until the next call on the same context. */
+const char* mt_last_error(const mt_ctx* ctx);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MT_H_ */
