@@ -203,21 +203,39 @@ def rope_bwd(dy: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
 # floor(h / (H / Hkv)).
 # ---------------------------------------------------------------------------
 
+def _heads_first(x):
+    """[b, s, heads, hd] -> [b, heads, s, hd] (a view)."""
+    return x.transpose(0, 2, 1, 3)
+
+
+def _visible_scores(q, k):
+    """Scaled scores q_i . k_j / sqrt(hd) per query head, -inf where j > i.
+    q: [b, s, H, hd]; k: [b, s, Hkv, hd]. Returns [b, H, s, s]."""
+    b, s, H, hd = q.shape
+    kk = np.repeat(k, H // k.shape[2], axis=2)  # kv head for query head h is h // group
+    S = _heads_first(q) @ _heads_first(kk).transpose(0, 1, 3, 2) / np.sqrt(hd)
+    mask = np.tril(np.ones((s, s), dtype=bool))
+    return np.where(mask[None, None], S, -np.inf)
+
+
 def attention_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray):
     """q: [b, s, H, hd]; k, v: [b, s, Hkv, hd]. Returns (o [b,s,H,hd], P [b,H,s,s])."""
-    b, s, H, hd = q.shape
-    Hkv = k.shape[2]
-    group = H // Hkv
-    kk = np.repeat(k, group, axis=2)  # kv head for query head h is h // group
-    vv = np.repeat(v, group, axis=2)
-    S = np.einsum("bihd,bjhd->bhij", q, kk) / np.sqrt(hd)
-    mask = np.tril(np.ones((s, s), dtype=bool))
-    S = np.where(mask[None, None], S, -np.inf)
+    H = q.shape[2]
+    vv = np.repeat(v, H // v.shape[2], axis=2)
+    S = _visible_scores(q, k)
     S = S - S.max(axis=-1, keepdims=True)
     P = np.exp(S)
     P = P / P.sum(axis=-1, keepdims=True)
-    o = np.einsum("bhij,bjhd->bihd", P, vv)
+    o = _heads_first(P @ _heads_first(vv))
     return o, P
+
+
+def attention_lse(q: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """Natural log-sum-exp over visible keys of the scaled scores, [b, H, s]:
+    lse[b, h, i] = log sum_{j <= i} exp(q_i . k_j / sqrt(hd))."""
+    S = _visible_scores(q, k)
+    m = S.max(axis=-1, keepdims=True)
+    return m[..., 0] + np.log(np.sum(np.exp(S - m), axis=-1))
 
 
 def attention_bwd(q, k, v, P, do):
@@ -228,14 +246,15 @@ def attention_bwd(q, k, v, P, do):
     b, s, H, hd = q.shape
     Hkv = k.shape[2]
     group = H // Hkv
-    kk = np.repeat(k, group, axis=2)
-    vv = np.repeat(v, group, axis=2)
-    dP = np.einsum("bihd,bjhd->bhij", do, vv)
-    dvv = np.einsum("bhij,bihd->bjhd", P, do)
+    kh = _heads_first(np.repeat(k, group, axis=2))
+    vh = _heads_first(np.repeat(v, group, axis=2))
+    doh = _heads_first(do)
+    dP = doh @ vh.transpose(0, 1, 3, 2)
+    dvv = _heads_first(P.transpose(0, 1, 3, 2) @ doh)
     dS = P * (dP - np.sum(dP * P, axis=-1, keepdims=True))
     scale = 1.0 / np.sqrt(hd)
-    dq = np.einsum("bhij,bjhd->bihd", dS, kk) * scale
-    dkk = np.einsum("bhij,bihd->bjhd", dS, q) * scale
+    dq = _heads_first(dS @ kh) * scale
+    dkk = _heads_first(dS.transpose(0, 1, 3, 2) @ _heads_first(q)) * scale
     dk = dkk.reshape(b, s, Hkv, group, hd).sum(axis=3)
     dv = dvv.reshape(b, s, Hkv, group, hd).sum(axis=3)
     return dq, dk, dv
@@ -328,6 +347,20 @@ def layer_bwd(dxn: np.ndarray, W: dict, cache: dict, c: OracleConfig, cos, sin):
 # Head: final norm, untied LM head, mean next-token cross-entropy.
 # ---------------------------------------------------------------------------
 
+def softmax_ce(z, labels):
+    """Per-row cross-entropy of logits z [T, V] against integer labels:
+      loss_t = logsumexp(z_t) - z_t[y_t];  g_t = softmax(z_t) - onehot(y_t).
+    Returns (loss_t [T], g [T, V])."""
+    T = z.shape[0]
+    zmax = z.max(axis=-1, keepdims=True)
+    lse = zmax[:, 0] + np.log(np.sum(np.exp(z - zmax), axis=-1))
+    idx = np.arange(T)
+    loss_t = lse - z[idx, labels]
+    g = np.exp(z - lse[:, None])
+    g[idx, labels] -= 1.0
+    return loss_t, g
+
+
 def head_ce_fwd_bwd(xL, gf, Whead, labels, eps):
     """xL: [T, d]; labels: [T] ints. Returns (loss, dxL, dgf, dWhead) with
       z = RMSNorm(xL) gf Whead^T, loss = mean_t(logsumexp(z_t) - z_t[y_t]),
@@ -335,13 +368,9 @@ def head_ce_fwd_bwd(xL, gf, Whead, labels, eps):
     T = xL.shape[0]
     n, r = rmsnorm_fwd(xL, gf, eps)
     z = n @ Whead.T
-    zmax = z.max(axis=-1, keepdims=True)
-    lse = zmax[:, 0] + np.log(np.sum(np.exp(z - zmax), axis=-1))
-    idx = np.arange(T)
-    loss = float(np.mean(lse - z[idx, labels]))
-    dz = np.exp(z - lse[:, None])
-    dz[idx, labels] -= 1.0
-    dz /= T
+    loss_t, g = softmax_ce(z, labels)
+    loss = float(np.mean(loss_t))
+    dz = g / T
     dWhead = dz.T @ n
     dn = dz @ Whead
     dxL, dgf = rmsnorm_bwd(xL, gf, r, dn)
