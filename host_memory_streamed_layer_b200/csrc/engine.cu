@@ -1,0 +1,1092 @@
+// Pipelined, double-buffered streaming engine for one training step, and the
+// C ABI of include/mt.h.
+//
+// MegaTrain's memory-centric training (MegaTrain abstract; saify.me "The
+// memory-centric design", "Pipelined double buffering", "Stateless layer
+// templates"): parameters and optimizer state live in host memory; for each
+// layer the engine prefetches the layer's bf16 weights into one of two device
+// slots, runs the layer's kernels bound to that slot, pushes its fp32 gradients
+// back to host memory and lets the host update the layer with AdamW, so that
+// persistent device state is two weight slots, two gradient slots, the
+// layer-boundary activations and one layer's workspace.
+//
+// Streams: H2D prefetch, compute, D2H offload, ordered by per-load and
+// per-layer events. The weight loads follow the layer order of the step,
+// 0 .. L-1 (forward, keeping only boundary activations) then L-2 .. 0
+// (backward, recomputing each layer's forward from its kept input); layer L-1
+// stays resident across the turn. Load i+2 reuses the slot of load i and waits
+// for the compute stream to release it, so layer n+1 arrives while layer n
+// computes. A host optimizer thread waits on each layer's offload event and
+// updates that layer's master weights, moments and bf16 copy while the GPU
+// continues with the layers below.
+#include <math.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <chrono>
+#include <condition_variable>
+#include <deque>
+#include <mutex>
+#include <string>
+#include <thread>
+#include <vector>
+
+#include "host_adamw.h"
+#include "layout.h"
+#include "mt_internal.h"
+
+namespace mt {
+
+namespace {
+
+thread_local std::string g_create_error;
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+double now_s() {
+  return std::chrono::duration<double>(std::chrono::steady_clock::now().time_since_epoch()).count();
+}
+
+// Counter-based normal generator for library-owned arenas: splitmix64 of
+// (seed, tensor key, index) -> two uniforms -> Box-Muller.
+inline uint64_t splitmix64(uint64_t x) {
+  x += 0x9e3779b97f4a7c15ull;
+  x = (x ^ (x >> 30)) * 0xbf58476d1ce4e5b9ull;
+  x = (x ^ (x >> 27)) * 0x94d049bb133111ebull;
+  return x ^ (x >> 31);
+}
+inline float normal_at(uint64_t key, uint64_t i) {
+  const uint64_t a = splitmix64(key ^ splitmix64(2 * i));
+  const uint64_t b = splitmix64(key ^ splitmix64(2 * i + 1));
+  const double u1 = ((a >> 11) + 1.0) * (1.0 / 9007199254740993.0);  // (0, 1]
+  const double u2 = (b >> 11) * (1.0 / 9007199254740992.0);
+  return (float)(sqrt(-2.0 * log(u1)) * cos(6.283185307179586 * u2));
+}
+
+struct Job {
+  enum Kind { LAYER, HEAD, EMBED } kind;
+  int layer;
+  cudaEvent_t ready;  // offload of this job's gradients has completed
+  int flag_index;     // index in the finite-flag array
+};
+
+}  // namespace
+}  // namespace mt
+
+using namespace mt;
+
+struct mt_ctx {
+  mt_config cfg{};
+  Layout lay;
+  std::string err;
+  int device = 0;
+  int step = 0;
+
+  // ---- host memory ----
+  float* arena = nullptr;  // fp32 master
+  bool arena_owned = false;
+  float* m = nullptr;  // Adam moments (pageable, 64-byte aligned)
+  float* v = nullptr;
+  float* grad = nullptr;          // pinned fp32 gradient arena
+  uint16_t* bf_layers = nullptr;  // pinned bf16 layer blocks
+  uint16_t* bf_embed = nullptr;   // pinned bf16 embedding (read by the GPU in place)
+  uint16_t* bf_head = nullptr;    // pinned bf16 [final norm | LM head]
+  uint16_t* bf_embed_dev = nullptr;  // device alias of bf_embed
+  float* emb_rows_h = nullptr;    // pinned embedding-gradient rows [T, d]
+  int32_t* stage_i = nullptr;     // pinned: tokens[T] labels[T] offs[T+1] pos[T]
+  int32_t* flags_h = nullptr;     // pinned finite flags [L + 2]
+  float* misc_h = nullptr;        // pinned: loss sum, device error word
+  std::vector<int32_t> uniq, prev_uniq;
+  ThreadPool* pool = nullptr;
+
+  // ---- device memory ----
+  void* dmem = nullptr;
+  size_t dmem_bytes = 0;
+  cudaStream_t s_h2d = nullptr, s_comp = nullptr, s_d2h = nullptr;
+  uint16_t* wslot[2] = {nullptr, nullptr};
+  float* gslot[2] = {nullptr, nullptr};
+  uint16_t* d_head_w = nullptr;  // [gf | Whead] bf16
+  float* d_head_g = nullptr;     // [dgf | dWhead] fp32
+  float* xb = nullptr;           // boundary activations [(L+1), T, d]
+  uint16_t *u_b, *qkv_b, *ao_b, *w_b, *gu_b, *act_b, *gxb, *dact_b, *dgu_b, *dhb, *dao_b, *dqkv_b, *n_b, *dz_b;
+  float *lse, *h_f, *r1, *r2, *gx0, *gx1, *tmp_f, *dh_f, *dvec, *dqacc, *rms_part, *rf, *logits, *rowloss;
+  int32_t *d_tok, *d_lab, *d_offs, *d_pos, *d_flags, *d_err;
+  float *d_cos, *d_sin, *d_loss;
+  int Tc = 0;  // logits chunk (tokens)
+
+  // ---- events ----
+  std::vector<cudaEvent_t> ev_wready, ev_compready, ev_h2d_start, ev_slotfree;  // per weight load
+  std::vector<cudaEvent_t> ev_gready, ev_d2h_start, ev_gdrained;               // per backward layer
+  cudaEvent_t ev_head_h2d_start, ev_head_wready, ev_head_gready, ev_head_d2h_start, ev_head_drained;
+  cudaEvent_t ev_emb_ready, ev_emb_d2h_start, ev_emb_drained;
+  cudaEvent_t ev_step_start, ev_fwd_end, ev_head_end, ev_bwd_end, ev_step_end;
+  std::vector<cudaEvent_t> ev_timing;  // pool for per-kernel timing pairs
+  size_t timing_used = 0;
+  struct Timed {
+    cudaEvent_t a, b;
+    double flops;
+    int kind;  // 0 gemm, 1 attention
+  };
+  std::vector<Timed> timed;
+
+  // ---- optimizer thread ----
+  std::thread opt_thread;
+  std::mutex opt_mu;
+  std::condition_variable opt_cv, opt_done_cv;
+  std::deque<Job> jobs;
+  int jobs_pending = 0;
+  bool opt_stop = false;
+  int opt_status = MT_OK;
+  bool skip_updates = false;
+  double adamw_s = 0, adamw_bytes = 0;
+  double wait_limit_s = 600.0;
+
+  mt_stats stats{};
+  int64_t launches = 0;
+  std::vector<int> load_seq;  // layer of each weight load
+};
+
+namespace mteng {
+
+int set_err(mt_ctx* c, int code, const std::string& m) {
+  if (c)
+    c->err = m;
+  else
+    g_create_error = m;
+  return code;
+}
+
+#define CK(call)                                                                                  \
+  do {                                                                                            \
+    cudaError_t e_ = (call);                                                                      \
+    if (e_ != cudaSuccess)                                                                        \
+      return set_err(c, MT_ERR_CUDA, std::string(#call) + ": " + cudaGetErrorString(e_));          \
+  } while (0)
+#define CKM(call)               \
+  do {                          \
+    int r_ = (call);            \
+    if (r_ != MT_OK) return r_; \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// Kernel wrappers with launch counting and optional event timing.
+// ---------------------------------------------------------------------------
+cudaEvent_t timing_event(mt_ctx* c) {
+  if (c->timing_used == c->ev_timing.size()) {
+    cudaEvent_t e;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    c->ev_timing.push_back(e);
+  }
+  return c->ev_timing[c->timing_used++];
+}
+
+int gemm(mt_ctx* c, const GemmDesc& g) {
+  const bool timing = (c->cfg.flags & MT_FLAG_KERNEL_TIMING) != 0;
+  cudaEvent_t a = nullptr, b = nullptr;
+  if (timing) {
+    a = timing_event(c);
+    b = timing_event(c);
+    if (a) cudaEventRecord(a, c->s_comp);
+  }
+  int r = gemm_bf16(g, c->s_comp, c->d_err);
+  if (r != MT_OK) return set_err(c, r, "GEMM launch failed");
+  c->launches += 1;
+  if (timing && a && b) {
+    cudaEventRecord(b, c->s_comp);
+    c->timed.push_back({a, b, 2.0 * g.M * (double)g.N * g.K, 0});
+  }
+  return MT_OK;
+}
+
+GemmDesc gd_fwd(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, int epi,
+                const float* R, int M, int N, int K) {
+  return GemmDesc{A, lda, false, B, ldb, false, C, ldc, epi, R, ldc, M, N, K};
+}
+GemmDesc gd_dx(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, int epi, int M, int N,
+               int K) {
+  return GemmDesc{A, lda, false, B, ldb, true, C, ldc, epi, nullptr, 0, M, N, K};
+}
+GemmDesc gd_dw(const void* A, int64_t lda, const void* B, int64_t ldb, float* C, int64_t ldc, int epi, int M, int N,
+               int K) {
+  return GemmDesc{A, lda, true, B, ldb, true, C, ldc, epi, epi == EPI_F32_ADD ? C : nullptr, ldc, M, N, K};
+}
+
+int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
+  const bool timing = (c->cfg.flags & MT_FLAG_KERNEL_TIMING) != 0;
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if (timing) {
+    e0 = timing_event(c);
+    e1 = timing_event(c);
+    if (e0) cudaEventRecord(e0, c->s_comp);
+  }
+  int r = bwd ? attention_bwd(a, c->s_comp) : attention_fwd(a, c->s_comp);
+  if (r != MT_OK) return set_err(c, r, "attention launch failed");
+  c->launches += bwd ? 4 : 1;
+  if (timing && e0 && e1) {
+    cudaEventRecord(e1, c->s_comp);
+    // causal attention: QK^T and PV over the visible half, per query head
+    const double fwd = 2.0 * 2.0 * a.b * (double)a.s * a.s / 2.0 * a.H * a.hd;
+    c->timed.push_back({e0, e1, bwd ? 2.5 * fwd : fwd, 1});
+  }
+  return MT_OK;
+}
+
+#define KL(expr, n)                                                                              \
+  do {                                                                                           \
+    int r_ = (expr);                                                                             \
+    if (r_ != MT_OK)                                                                             \
+      return set_err(c, r_, std::string("launch: ") + #expr + ": " + last_launch_error());       \
+    c->launches += (n);                                                                          \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// Finite check of a gradient range: flag = 1 if any value is NaN or Inf.
+// ---------------------------------------------------------------------------
+__global__ void k_check_finite(const float* __restrict__ g, size_t n, int32_t* __restrict__ flag) {
+  bool bad = false;
+  const size_t n4 = n / 4;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
+    const float4 v = reinterpret_cast<const float4*>(g)[i];
+    bad |= !isfinite(v.x) || !isfinite(v.y) || !isfinite(v.z) || !isfinite(v.w);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < (n & 3)) bad |= !isfinite(g[n4 * 4 + threadIdx.x]);
+  if (__syncthreads_or(bad) && threadIdx.x == 0) *flag = 1;
+}
+
+int check_finite(mt_ctx* c, const float* g, size_t n, int idx) {
+  CK(cudaMemsetAsync(c->d_flags + idx, 0, sizeof(int32_t), c->s_comp));
+  k_check_finite<<<296, 256, 0, c->s_comp>>>(g, n, c->d_flags + idx);
+  CK(cudaGetLastError());
+  c->launches += 1;
+  return MT_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Layer forward from x = xb[l] with the weights of `slot`. With keep_out the
+// layer output goes to xb[l+1]; otherwise (recompute) the down projection is
+// skipped, since the backward only needs the intermediates.
+// ---------------------------------------------------------------------------
+int layer_fwd(mt_ctx* c, int l, int slot, bool keep_out) {
+  const Shapes& s = c->lay.sh;
+  const Layout& y = c->lay;
+  const uint16_t* W = c->wslot[slot];
+  const float* x = c->xb + (size_t)l * s.T * s.d;
+  cudaStream_t st = c->s_comp;
+  KL(launch_rmsnorm_fwd(x, W + y.bf_g1, c->u_b, c->r1, s.T, s.d, c->cfg.norm_eps, st), 1);
+  CKM(gemm(c, gd_fwd(c->u_b, s.d, W + y.bf_qkv, s.d, c->qkv_b, s.Nqkv, EPI_BF16, nullptr, s.T, s.Nqkv, s.d)));
+  KL(launch_rope(c->qkv_b, s.Nqkv, s.T, s.s, s.H, s.hd, 0, c->d_cos, c->d_sin, 1.f, st), 1);
+  KL(launch_rope(c->qkv_b, s.Nqkv, s.T, s.s, s.Hkv, s.hd, s.Hd, c->d_cos, c->d_sin, 1.f, st), 1);
+  AttnArgs a{};
+  a.q = c->qkv_b;
+  a.k = c->qkv_b + s.Hd;
+  a.v = c->qkv_b + s.Hd + s.Hkv * s.hd;
+  a.ldqkv = s.Nqkv;
+  a.o = c->ao_b;
+  a.ldo = s.Hd;
+  a.lse = c->lse;
+  a.b = s.b;
+  a.s = s.s;
+  a.H = s.H;
+  a.Hkv = s.Hkv;
+  a.hd = s.hd;
+  a.scale = 1.0f / sqrtf((float)s.hd);
+  CKM(attn(c, a, false));
+  CKM(gemm(c, gd_fwd(c->ao_b, s.Hd, W + y.bf_o, s.Hd, c->h_f, s.d, EPI_F32_ADD, x, s.T, s.d, s.Hd)));
+  KL(launch_rmsnorm_fwd(c->h_f, W + y.bf_g2, c->w_b, c->r2, s.T, s.d, c->cfg.norm_eps, st), 1);
+  CKM(gemm(c, gd_fwd(c->w_b, s.d, W + y.bf_gu, s.d, c->gu_b, 2 * s.F, EPI_BF16, nullptr, s.T, 2 * s.F, s.d)));
+  KL(launch_swiglu_fwd(c->gu_b, c->act_b, s.T, s.F, st), 1);
+  if (keep_out) {
+    float* xo = c->xb + (size_t)(l + 1) * s.T * s.d;
+    CKM(gemm(c, gd_fwd(c->act_b, s.F, W + y.bf_d, s.F, xo, s.d, EPI_F32_ADD, c->h_f, s.T, s.d, s.F)));
+  }
+  return MT_OK;
+}
+
+// Layer backward: gin = dL/dx_{l+1} (fp32), writes gout = dL/dx_l and the
+// layer's fp32 gradients into grad slot gs (arena layout of the layer).
+int layer_bwd(mt_ctx* c, int l, int slot, float* gs, const float* gin, float* gout) {
+  const Shapes& s = c->lay.sh;
+  const Layout& y = c->lay;
+  const uint16_t* W = c->wslot[slot];
+  const size_t base = y.layer_begin(l);
+  auto G = [&](int tid) { return gs + (y.t(l, tid).off - base); };
+  const float* x = c->xb + (size_t)l * s.T * s.d;
+  cudaStream_t st = c->s_comp;
+  const int T = s.T, d = s.d, F = s.F;
+
+  KL(launch_cast_f32_bf16(gin, c->gxb, (int64_t)T * d, st), 1);
+  // down projection
+  CKM(gemm(c, gd_dw(c->gxb, d, c->act_b, F, G(MT_T_WDOWN), F, EPI_F32, d, F, T)));
+  CKM(gemm(c, gd_dx(c->gxb, d, W + y.bf_d, F, c->dact_b, F, EPI_BF16, T, F, d)));
+  KL(launch_swiglu_bwd(c->gu_b, c->dact_b, c->dgu_b, T, F, st), 1);
+  // gate/up projections
+  CKM(gemm(c, gd_dw(c->dgu_b, 2 * F, c->w_b, d, G(MT_T_WGATE), d, EPI_F32, 2 * F, d, T)));
+  CKM(gemm(c, gd_dx(c->dgu_b, 2 * F, W + y.bf_gu, d, c->tmp_f, d, EPI_F32, T, d, 2 * F)));
+  KL(launch_rmsnorm_bwd(c->h_f, W + y.bf_g2, c->r2, c->tmp_f, gin, c->dh_f, c->dhb, c->rms_part, G(MT_T_MLP_NORM),
+                        T, d, st),
+     2);
+  // output projection
+  CKM(gemm(c, gd_dw(c->dhb, d, c->ao_b, s.Hd, G(MT_T_WO), s.Hd, EPI_F32, d, s.Hd, T)));
+  CKM(gemm(c, gd_dx(c->dhb, d, W + y.bf_o, s.Hd, c->dao_b, s.Hd, EPI_BF16, T, s.Hd, d)));
+  // attention
+  AttnArgs a{};
+  a.q = c->qkv_b;
+  a.k = c->qkv_b + s.Hd;
+  a.v = c->qkv_b + s.Hd + s.Hkv * s.hd;
+  a.ldqkv = s.Nqkv;
+  a.o = c->ao_b;
+  a.ldo = s.Hd;
+  a.lse = c->lse;
+  a.dout = c->dao_b;
+  a.dvec = c->dvec;
+  a.dq_acc = c->dqacc;
+  a.ldqa = s.Hd;
+  a.dq = c->dqkv_b;
+  a.lddq = s.Nqkv;
+  a.dk = c->dqkv_b + s.Hd;
+  a.dv = c->dqkv_b + s.Hd + s.Hkv * s.hd;
+  a.lddkv = s.Nqkv;
+  a.b = s.b;
+  a.s = s.s;
+  a.H = s.H;
+  a.Hkv = s.Hkv;
+  a.hd = s.hd;
+  a.scale = 1.0f / sqrtf((float)s.hd);
+  CKM(attn(c, a, true));
+  KL(launch_rope(c->dqkv_b, s.Nqkv, T, s.s, s.H, s.hd, 0, c->d_cos, c->d_sin, -1.f, st), 1);
+  KL(launch_rope(c->dqkv_b, s.Nqkv, T, s.s, s.Hkv, s.hd, s.Hd, c->d_cos, c->d_sin, -1.f, st), 1);
+  // q/k/v projections
+  CKM(gemm(c, gd_dw(c->dqkv_b, s.Nqkv, c->u_b, d, G(MT_T_WQ), d, EPI_F32, s.Nqkv, d, T)));
+  CKM(gemm(c, gd_dx(c->dqkv_b, s.Nqkv, W + y.bf_qkv, d, c->tmp_f, d, EPI_F32, T, d, s.Nqkv)));
+  KL(launch_rmsnorm_bwd(x, W + y.bf_g1, c->r1, c->tmp_f, c->dh_f, gout, nullptr, c->rms_part, G(MT_T_ATTN_NORM), T,
+                        d, st),
+     2);
+  return check_finite(c, gs, y.layer_end(l) - base, l);
+}
+
+// Final norm, LM head and cross-entropy, head gradients; writes dL/dx_L to gout.
+int head_step(mt_ctx* c, float* gout) {
+  const Shapes& s = c->lay.sh;
+  const int T = s.T, d = s.d, V = s.V;
+  cudaStream_t st = c->s_comp;
+  const size_t gf_pad = c->lay.head.off - c->lay.final_norm.off;  // floats between dgf and dWhead
+  const uint16_t* gf = c->d_head_w;
+  const uint16_t* Wh = c->d_head_w + align_up(d, 128);
+  float* dgf = c->d_head_g;
+  float* dWh = c->d_head_g + gf_pad;
+  const float* xL = c->xb + (size_t)s.L * T * d;
+  KL(launch_rmsnorm_fwd(xL, gf, c->n_b, c->rf, T, d, c->cfg.norm_eps, st), 1);
+  for (int t0 = 0; t0 < T; t0 += c->Tc) {
+    const int tc = std::min(c->Tc, T - t0);
+    const uint16_t* n_c = c->n_b + (size_t)t0 * d;
+    CKM(gemm(c, gd_fwd(n_c, d, Wh, d, c->logits, V, EPI_F32, nullptr, tc, V, d)));
+    KL(launch_softmax_ce(c->logits, V, c->d_lab + t0, c->dz_b, V, c->rowloss + t0, tc, V, 1.0f / T, st), 1);
+    CKM(gemm(c, gd_dw(c->dz_b, V, n_c, d, dWh, d, t0 == 0 ? EPI_F32 : EPI_F32_ADD, V, d, tc)));
+    CKM(gemm(c, gd_dx(c->dz_b, V, Wh, d, c->tmp_f + (size_t)t0 * d, d, EPI_F32, tc, d, V)));
+  }
+  KL(launch_sum_all(c->rowloss, T, c->d_loss, 0, st), 1);
+  KL(launch_rmsnorm_bwd(xL, gf, c->rf, c->tmp_f, nullptr, gout, nullptr, c->rms_part, dgf, T, d, st), 2);
+  return check_finite(c, c->d_head_g, gf_pad + (size_t)V * d, s.L);
+}
+
+// ---------------------------------------------------------------------------
+// Optimizer thread.
+// ---------------------------------------------------------------------------
+bool wait_event(mt_ctx* c, cudaEvent_t e) {
+  const double t0 = now_s();
+  while (true) {
+    cudaError_t r = cudaEventQuery(e);
+    if (r == cudaSuccess) return true;
+    if (r != cudaErrorNotReady) return false;
+    if (now_s() - t0 > c->wait_limit_s) return false;
+    std::this_thread::sleep_for(std::chrono::microseconds(50));
+  }
+}
+
+struct Seg {
+  size_t off, n;    // floats in the arena
+  uint16_t* bf;     // bf16 destination of element 0
+};
+
+void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
+  const AdamHyper h{c->cfg.lr, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps, c->cfg.wd};
+  const size_t chunk = 1 << 16;
+  struct Task {
+    size_t off, n;
+    uint16_t* bf;
+  };
+  std::vector<Task> tasks;
+  for (const Seg& sg : segs)
+    for (size_t i = 0; i < sg.n; i += chunk) tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf + i});
+  const int t = c->step;
+  const double t0 = now_s();
+  c->pool->run((int)tasks.size(), [&](int i) {
+    const Task& k = tasks[i];
+    adamw_chunk(c->arena + k.off, c->grad + k.off, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
+  });
+  c->adamw_s += now_s() - t0;
+  size_t n = 0;
+  for (const Seg& sg : segs) n += sg.n;
+  c->adamw_bytes += 30.0 * n;
+}
+
+void run_job(mt_ctx* c, const Job& j) {
+  const Layout& y = c->lay;
+  const Shapes& s = y.sh;
+  if (!wait_event(c, j.ready)) {
+    c->opt_status = MT_ERR_TIMEOUT;
+    c->err = "gradient offload did not complete within the wait limit";
+    c->skip_updates = true;
+    return;
+  }
+  if (j.kind == Job::EMBED) {
+    // Dense gradient of the embedding: zero last step's rows, scatter this step's.
+    float* ge = c->grad + y.embed.off;
+    const size_t d = s.d;
+    for (int32_t r : c->prev_uniq) memset(ge + (size_t)r * d, 0, d * sizeof(float));
+    bool bad = false;
+    for (size_t u = 0; u < c->uniq.size(); ++u) {
+      const float* src = c->emb_rows_h + u * d;
+      for (size_t k = 0; k < d; ++k) bad |= !std::isfinite(src[k]);
+      memcpy(ge + (size_t)c->uniq[u] * d, src, d * sizeof(float));
+    }
+    c->prev_uniq = c->uniq;
+    if (bad) c->flags_h[j.flag_index] = 1;
+  }
+  if (c->flags_h[j.flag_index] != 0) {
+    if (c->opt_status == MT_OK) {
+      c->opt_status = MT_ERR_NONFINITE;
+      c->err = "non-finite gradient; this and the remaining updates were skipped";
+    }
+    c->skip_updates = true;
+  }
+  if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
+  std::vector<Seg> segs;
+  if (j.kind == Job::LAYER) {
+    uint16_t* blk = c->bf_layers + (size_t)j.layer * y.bf_layer;
+    for (int tid = 0; tid < kLayerTensors; ++tid) {
+      const TRef& r = y.t(j.layer, tid);
+      segs.push_back({r.off, r.n, blk + y.bf_of(tid)});
+    }
+  } else if (j.kind == Job::HEAD) {
+    segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head});
+    segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(s.d, 128)});
+  } else {
+    segs.push_back({y.embed.off, y.embed.n, c->bf_embed});
+  }
+  adamw_segments(c, segs);
+}
+
+void opt_loop(mt_ctx* c) {
+  while (true) {
+    Job j;
+    {
+      std::unique_lock<std::mutex> lk(c->opt_mu);
+      c->opt_cv.wait(lk, [&] { return c->opt_stop || !c->jobs.empty(); });
+      if (c->opt_stop && c->jobs.empty()) return;
+      j = c->jobs.front();
+      c->jobs.pop_front();
+    }
+    run_job(c, j);
+    {
+      std::lock_guard<std::mutex> lk(c->opt_mu);
+      --c->jobs_pending;
+    }
+    c->opt_done_cv.notify_all();
+  }
+}
+
+void push_job(mt_ctx* c, const Job& j) {
+  {
+    std::lock_guard<std::mutex> lk(c->opt_mu);
+    c->jobs.push_back(j);
+    ++c->jobs_pending;
+  }
+  c->opt_cv.notify_one();
+}
+
+void wait_jobs(mt_ctx* c) {
+  std::unique_lock<std::mutex> lk(c->opt_mu);
+  c->opt_done_cv.wait(lk, [&] { return c->jobs_pending == 0; });
+}
+
+// ---------------------------------------------------------------------------
+// Step.
+// ---------------------------------------------------------------------------
+int issue_load(mt_ctx* c, int i) {
+  const Layout& y = c->lay;
+  const int slot = i & 1;
+  if (i >= 2) CK(cudaStreamWaitEvent(c->s_h2d, c->ev_slotfree[i - 2], 0));
+  CK(cudaEventRecord(c->ev_h2d_start[i], c->s_h2d));
+  CK(cudaMemcpyAsync(c->wslot[slot], c->bf_layers + (size_t)c->load_seq[i] * y.bf_layer, y.bf_layer * 2,
+                     cudaMemcpyHostToDevice, c->s_h2d));
+  CK(cudaEventRecord(c->ev_wready[i], c->s_h2d));
+  return MT_OK;
+}
+
+int issue_head_load(mt_ctx* c) {
+  const size_t n = align_up(c->lay.sh.d, 128) + (size_t)c->lay.sh.V * c->lay.sh.d;
+  CK(cudaEventRecord(c->ev_head_h2d_start, c->s_h2d));
+  CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, n * 2, cudaMemcpyHostToDevice, c->s_h2d));
+  CK(cudaEventRecord(c->ev_head_wready, c->s_h2d));
+  return MT_OK;
+}
+
+int offload_layer(mt_ctx* c, int l, int k) {
+  const Layout& y = c->lay;
+  const size_t b = y.layer_begin(l), e = y.layer_end(l);
+  CK(cudaEventRecord(c->ev_gready[k], c->s_comp));
+  CK(cudaStreamWaitEvent(c->s_d2h, c->ev_gready[k], 0));
+  CK(cudaEventRecord(c->ev_d2h_start[k], c->s_d2h));
+  CK(cudaMemcpyAsync(c->grad + b, c->gslot[k & 1], (e - b) * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  CK(cudaMemcpyAsync(c->flags_h + l, c->d_flags + l, 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  CK(cudaEventRecord(c->ev_gdrained[k], c->s_d2h));
+  push_job(c, Job{Job::LAYER, l, c->ev_gdrained[k], l});
+  return MT_OK;
+}
+
+int enqueue_step(mt_ctx* c, int n_unique) {
+  const Layout& y = c->lay;
+  const Shapes& s = y.sh;
+  const int L = s.L, T = s.T, d = s.d;
+  const int nloads = (int)c->load_seq.size();
+  cudaStream_t sc = c->s_comp;
+
+  CK(cudaEventRecord(c->ev_step_start, sc));
+  CK(cudaMemcpyAsync(c->d_tok, c->stage_i, (size_t)(4 * T + 1) * 4, cudaMemcpyHostToDevice, sc));
+  KL(launch_embed_fwd(c->d_tok, c->bf_embed_dev, c->xb, T, d, sc), 1);
+  CKM(issue_load(c, 0));
+  if (nloads > 1) CKM(issue_load(c, 1));
+  if (L == 1) CKM(issue_head_load(c));
+
+  float* gin = c->gx0;
+  float* gout = c->gx1;
+  for (int i = 0; i < nloads; ++i) {
+    const int slot = i & 1;
+    CK(cudaEventRecord(c->ev_compready[i], sc));
+    CK(cudaStreamWaitEvent(sc, c->ev_wready[i], 0));
+    if (i < L) {
+      const int l = i;
+      CKM(layer_fwd(c, l, slot, true));
+      if (l == L - 1) {
+        CK(cudaEventRecord(c->ev_fwd_end, sc));
+        CK(cudaStreamWaitEvent(sc, c->ev_head_wready, 0));
+        CKM(head_step(c, gin));
+        CK(cudaEventRecord(c->ev_head_gready, sc));
+        CK(cudaStreamWaitEvent(c->s_d2h, c->ev_head_gready, 0));
+        CK(cudaEventRecord(c->ev_head_d2h_start, c->s_d2h));
+        const size_t n = y.head.off + y.head.n - y.final_norm.off;
+        CK(cudaMemcpyAsync(c->grad + y.final_norm.off, c->d_head_g, n * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+        CK(cudaMemcpyAsync(c->flags_h + L, c->d_flags + L, 4, cudaMemcpyDeviceToHost, c->s_d2h));
+        CK(cudaEventRecord(c->ev_head_drained, c->s_d2h));
+        push_job(c, Job{Job::HEAD, -1, c->ev_head_drained, L});
+        CK(cudaEventRecord(c->ev_head_end, sc));
+        // backward of the last layer: its intermediates are still in the workspace
+        CKM(layer_bwd(c, l, slot, c->gslot[0], gin, gout));
+        CKM(offload_layer(c, l, 0));
+        std::swap(gin, gout);
+      }
+    } else {
+      const int k = i - (L - 1);  // backward index: layer L-1-k
+      const int l = L - 1 - k;
+      if (k >= 2) CK(cudaStreamWaitEvent(sc, c->ev_gdrained[k - 2], 0));
+      CKM(layer_fwd(c, l, slot, false));
+      CKM(layer_bwd(c, l, slot, c->gslot[k & 1], gin, gout));
+      CKM(offload_layer(c, l, k));
+      std::swap(gin, gout);
+    }
+    CK(cudaEventRecord(c->ev_slotfree[i], sc));
+    if (i + 2 < nloads) CKM(issue_load(c, i + 2));
+    if (i + 2 == L - 1 || (i == 0 && L == 2)) CKM(issue_head_load(c));
+  }
+  CK(cudaEventRecord(c->ev_bwd_end, sc));
+  // embedding gradient rows, in token order per unique id
+  KL(launch_embed_bwd(c->d_offs, c->d_pos, n_unique, gin, c->tmp_f, d, sc), 1);
+  CK(cudaEventRecord(c->ev_emb_ready, sc));
+  CK(cudaStreamWaitEvent(c->s_d2h, c->ev_emb_ready, 0));
+  CK(cudaEventRecord(c->ev_emb_d2h_start, c->s_d2h));
+  CK(cudaMemcpyAsync(c->emb_rows_h, c->tmp_f, (size_t)n_unique * d * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  CK(cudaEventRecord(c->ev_emb_drained, c->s_d2h));
+  c->flags_h[L + 1] = 0;
+  push_job(c, Job{Job::EMBED, -1, c->ev_emb_drained, L + 1});
+  CK(cudaMemcpyAsync(c->misc_h, c->d_loss, 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaEventRecord(c->ev_step_end, sc));
+  return MT_OK;
+}
+
+float ev_ms(cudaEvent_t a, cudaEvent_t b) {
+  float ms = 0.f;
+  if (cudaEventElapsedTime(&ms, a, b) != cudaSuccess) return 0.f;
+  return ms;
+}
+
+void collect_stats(mt_ctx* c) {
+  mt_stats& st = c->stats;
+  const int L = c->lay.sh.L;
+  st.step_ms = ev_ms(c->ev_step_start, c->ev_step_end);
+  st.fwd_ms = ev_ms(c->ev_step_start, c->ev_fwd_end);
+  st.head_ms = ev_ms(c->ev_fwd_end, c->ev_head_end);
+  st.bwd_ms = ev_ms(c->ev_head_end, c->ev_bwd_end);
+  double h2d = ev_ms(c->ev_head_h2d_start, c->ev_head_wready), wait = 0;
+  for (size_t i = 0; i < c->load_seq.size(); ++i) {
+    h2d += ev_ms(c->ev_h2d_start[i], c->ev_wready[i]);
+    const float w = ev_ms(c->ev_compready[i], c->ev_wready[i]);
+    if (w > 0) wait += w;
+  }
+  double d2h = ev_ms(c->ev_head_d2h_start, c->ev_head_drained) + ev_ms(c->ev_emb_d2h_start, c->ev_emb_drained);
+  for (int k = 0; k < L; ++k) d2h += ev_ms(c->ev_d2h_start[k], c->ev_gdrained[k]);
+  st.h2d_ms = h2d;
+  st.d2h_ms = d2h;
+  st.wait_weights_ms = wait;
+  const Layout& y = c->lay;
+  st.h2d_bytes = (double)c->load_seq.size() * y.bf_layer * 2 +
+                 (double)(align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d) * 2 + 4.0 * (4 * y.sh.T + 1) +
+                 (double)y.sh.T * y.sh.d * 2;  // embedding rows read in place
+  st.d2h_bytes = 4.0 * (y.head.off + y.head.n - y.final_norm.off) + 4.0 * c->uniq.size() * y.sh.d + 8.0;
+  for (int l = 0; l < L; ++l) st.d2h_bytes += 4.0 * (y.layer_end(l) - y.layer_begin(l));
+  st.adamw_ms = c->adamw_s * 1e3;
+  st.adamw_bytes = c->adamw_bytes;
+  st.gemm_flops = st.gemm_ms = st.attn_flops = st.attn_ms = 0;
+  st.gemm_launches = st.attn_launches = 0;
+  for (const auto& t : c->timed) {
+    const double ms = ev_ms(t.a, t.b);
+    if (t.kind == 0) {
+      st.gemm_flops += t.flops;
+      st.gemm_ms += ms;
+      st.gemm_launches++;
+    } else {
+      st.attn_flops += t.flops;
+      st.attn_ms += ms;
+      st.attn_launches++;
+    }
+  }
+  st.kernel_launches = c->launches;
+}
+
+// ---------------------------------------------------------------------------
+// Create / destroy helpers.
+// ---------------------------------------------------------------------------
+size_t device_bytes(const Layout& y, int Tc) {
+  const Shapes& s = y.sh;
+  const size_t T = s.T, d = s.d, F = s.F, V = s.V;
+  const size_t A = 256;
+  size_t b = 0;
+  auto add = [&](size_t bytes) { b += align_up(bytes, A); };
+  add(y.bf_layer * 2);
+  add(y.bf_layer * 2);
+  const size_t lay_f = y.layer_end(0) - y.layer_begin(0);
+  add(lay_f * 4);
+  add(lay_f * 4);
+  add((align_up(d, 128) + V * d) * 2);                     // head weights
+  add((y.head.off - y.final_norm.off + V * d) * 4);         // head grads
+  add((size_t)(s.L + 1) * T * d * 4);                       // boundary activations
+  add(T * d * 2);                                           // u
+  add(T * (size_t)s.Nqkv * 2);                              // qkv
+  add(T * (size_t)s.Hd * 2);                                // attention output
+  add((size_t)s.b * s.H * s.s * 4);                         // lse
+  add(T * d * 4);                                           // h
+  add(T * 4);                                               // r1
+  add(T * 4);                                               // r2
+  add(T * d * 2);                                           // w
+  add(T * 2 * F * 2);                                       // gate|up
+  add(T * F * 2);                                           // act
+  add(T * d * 4);                                           // gx0
+  add(T * d * 4);                                           // gx1
+  add(T * d * 2);                                           // gxb
+  add(T * F * 2);                                           // dact
+  add(T * 2 * F * 2);                                       // dgu
+  add(T * d * 4);                                           // tmp_f
+  add(T * d * 4);                                           // dh
+  add(T * d * 2);                                           // dhb
+  add(T * (size_t)s.Hd * 2);                                // dao
+  add((size_t)s.b * s.H * s.s * 4);                         // dvec
+  add(T * (size_t)s.Hd * 4);                                // dq accumulator
+  add(T * (size_t)s.Nqkv * 2);                              // dqkv
+  add((size_t)rmsnorm_bwd_blocks((int)T) * d * 4);          // RMSNorm partials
+  add(T * d * 2);                                           // n
+  add(T * 4);                                               // rf
+  add((size_t)Tc * V * 4);                                  // logits
+  add((size_t)Tc * V * 2);                                  // dz
+  add(T * 4);                                               // row loss
+  add((4 * T + 1) * 4);                                     // tokens, labels, offs, pos
+  add((size_t)(s.L + 2) * 4);                               // flags
+  add(4);                                                   // error word
+  add((size_t)s.s * (s.hd / 2) * 4 * 2);                    // cos, sin
+  add(4);                                                   // loss
+  return b + 4096;
+}
+
+void free_all(mt_ctx* c) {
+  if (!c) return;
+  if (c->opt_thread.joinable()) {
+    {
+      std::lock_guard<std::mutex> lk(c->opt_mu);
+      c->opt_stop = true;
+    }
+    c->opt_cv.notify_all();
+    c->opt_thread.join();
+  }
+  cudaSetDevice(c->device);
+  for (cudaStream_t s : {c->s_h2d, c->s_comp, c->s_d2h})
+    if (s) cudaStreamSynchronize(s);
+  auto kill = [](std::vector<cudaEvent_t>& v) {
+    for (auto e : v)
+      if (e) cudaEventDestroy(e);
+    v.clear();
+  };
+  kill(c->ev_wready);
+  kill(c->ev_compready);
+  kill(c->ev_h2d_start);
+  kill(c->ev_slotfree);
+  kill(c->ev_gready);
+  kill(c->ev_d2h_start);
+  kill(c->ev_gdrained);
+  kill(c->ev_timing);
+  for (cudaEvent_t e : {c->ev_head_h2d_start, c->ev_head_wready, c->ev_head_gready, c->ev_head_d2h_start,
+                        c->ev_head_drained, c->ev_emb_ready, c->ev_emb_d2h_start, c->ev_emb_drained,
+                        c->ev_step_start, c->ev_fwd_end, c->ev_head_end, c->ev_bwd_end, c->ev_step_end})
+    if (e) cudaEventDestroy(e);
+  // In serialized mode the three handles are one stream: destroy each once.
+  if (c->s_comp) cudaStreamDestroy(c->s_comp);
+  if (c->s_h2d && c->s_h2d != c->s_comp) cudaStreamDestroy(c->s_h2d);
+  if (c->s_d2h && c->s_d2h != c->s_comp && c->s_d2h != c->s_h2d) cudaStreamDestroy(c->s_d2h);
+  if (c->dmem) cudaFree(c->dmem);
+  for (void* p : {(void*)c->grad, (void*)c->bf_layers, (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h,
+                  (void*)c->stage_i, (void*)c->flags_h, (void*)c->misc_h})
+    if (p) cudaFreeHost(p);
+  free(c->m);
+  free(c->v);
+  if (c->arena_owned) free(c->arena);
+  delete c->pool;
+  delete c;
+}
+
+int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx** out) {
+  mt_ctx* c = nullptr;
+  std::string why;
+  int r = validate_config(cfg, &why);
+  if (r != MT_OK) return set_err(nullptr, r, why);
+  if (!out) return set_err(nullptr, MT_ERR_ARG, "out is NULL");
+  *out = nullptr;
+  Layout y = make_layout(*cfg);
+  const Shapes& s = y.sh;
+  if (arena) {
+    if (arena_bytes < y.total * 4) return set_err(nullptr, MT_ERR_ARENA, "arena smaller than mt_arena_bytes(cfg)");
+    if (reinterpret_cast<uintptr_t>(arena) & 255) return set_err(nullptr, MT_ERR_ARENA, "arena not 256-byte aligned");
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || cfg->device < 0 || cfg->device >= ndev)
+    return set_err(nullptr, MT_ERR_CUDA, "no such CUDA device");
+  if (cudaSetDevice(cfg->device) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaSetDevice failed");
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, cfg->device);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, cfg->device);
+  if (major != 10 || minor != 0) return set_err(nullptr, MT_ERR_CUDA, "this library runs on sm_100 (B200) only");
+
+  // logits chunk: at most ~4 GiB of fp32 logits + bf16 dz, multiple of 128 tokens
+  int Tc = (int)std::min<int64_t>(s.T, ((int64_t)1 << 32) / ((int64_t)s.V * 6));
+  if (Tc < s.T) Tc = std::max(128, Tc / 128 * 128);
+  const size_t need = device_bytes(y, Tc);
+  size_t free_b = 0, total_b = 0;
+  if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaMemGetInfo failed");
+  if (need + ((size_t)256 << 20) > free_b) {
+    char m[160];
+    snprintf(m, sizeof m, "device budget: need %.2f GB, %.2f GB free", need / 1e9, free_b / 1e9);
+    return set_err(nullptr, MT_ERR_NOMEM, m);
+  }
+
+  c = new mt_ctx();
+  c->cfg = *cfg;
+  c->lay = y;
+  c->device = cfg->device;
+  c->Tc = Tc;
+  int nthreads = cfg->host_threads;
+  if (nthreads <= 0) nthreads = std::max(1, (int)std::thread::hardware_concurrency() - 1);
+  c->pool = new ThreadPool(nthreads - 1);
+
+  // host memory
+  auto fail = [&](int code, const std::string& m) {
+    g_create_error = m;
+    free_all(c);
+    return code;
+  };
+  if (arena) {
+    c->arena = arena;
+  } else {
+    if (posix_memalign(reinterpret_cast<void**>(&c->arena), 256, y.total * 4)) return fail(MT_ERR_NOMEM, "arena alloc");
+    c->arena_owned = true;
+  }
+  if (posix_memalign(reinterpret_cast<void**>(&c->m), 64, y.total * 4) ||
+      posix_memalign(reinterpret_cast<void**>(&c->v), 64, y.total * 4))
+    return fail(MT_ERR_NOMEM, "host moment allocation failed");
+  const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
+  if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * 4, cudaHostAllocPortable) != cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->bf_layers), (size_t)s.L * y.bf_layer * 2, cudaHostAllocPortable) !=
+          cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->bf_embed), (size_t)s.V * s.d * 2,
+                    cudaHostAllocPortable | cudaHostAllocMapped) != cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->bf_head), head_bf * 2, cudaHostAllocPortable) != cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->emb_rows_h), (size_t)s.T * s.d * 4, cudaHostAllocPortable) !=
+          cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->stage_i), (size_t)(4 * s.T + 1) * 4, cudaHostAllocPortable) !=
+          cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->flags_h), (size_t)(s.L + 2) * 4, cudaHostAllocPortable) !=
+          cudaSuccess ||
+      cudaHostAlloc(reinterpret_cast<void**>(&c->misc_h), 64, cudaHostAllocPortable) != cudaSuccess)
+    return fail(MT_ERR_PIN, "pinned host allocation failed");
+  if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->bf_embed_dev), c->bf_embed, 0) != cudaSuccess)
+    return fail(MT_ERR_PIN, "embedding table not mapped for device access");
+  // Initialise (owned arena from seed), zero moments and gradients (parallel first touch).
+  if (c->arena_owned) {
+    auto fill = [&](const TRef& r, uint64_t key, bool gain) {
+      parallel_ranges(*c->pool, r.n, [&](size_t b, size_t e) {
+        for (size_t i = b; i < e; ++i) c->arena[r.off + i] = gain ? 1.f : 0.02f * normal_at(key, i);
+      });
+    };
+    const uint64_t seed = splitmix64(cfg->seed);
+    fill(y.embed, seed ^ 0x1000, false);
+    for (int l = 0; l < s.L; ++l)
+      for (int tid = 0; tid < kLayerTensors; ++tid)
+        fill(y.t(l, tid), seed ^ (((uint64_t)(l + 1) << 8) | tid), tid == MT_T_ATTN_NORM || tid == MT_T_MLP_NORM);
+    fill(y.final_norm, seed ^ 0x1001, true);
+    fill(y.head, seed ^ 0x1002, false);
+  }
+  parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) {
+    memset(c->m + b, 0, (e - b) * 4);
+    memset(c->v + b, 0, (e - b) * 4);
+    memset(c->grad + b, 0, (e - b) * 4);
+  });
+  // bf16 streaming copies
+  for (int l = 0; l < s.L; ++l) {
+    uint16_t* blk = c->bf_layers + (size_t)l * y.bf_layer;
+    memset(blk, 0, y.bf_layer * 2);
+    for (int tid = 0; tid < kLayerTensors; ++tid) {
+      const TRef& r = y.t(l, tid);
+      uint16_t* dst = blk + y.bf_of(tid);
+      parallel_ranges(*c->pool, r.n, [&](size_t b, size_t e) { bf16_round_chunk(c->arena + r.off + b, dst + b, e - b); });
+    }
+  }
+  parallel_ranges(*c->pool, y.embed.n,
+                  [&](size_t b, size_t e) { bf16_round_chunk(c->arena + y.embed.off + b, c->bf_embed + b, e - b); });
+  memset(c->bf_head, 0, head_bf * 2);
+  bf16_round_chunk(c->arena + y.final_norm.off, c->bf_head, s.d);
+  uint16_t* bhw = c->bf_head + align_up(s.d, 128);
+  parallel_ranges(*c->pool, y.head.n,
+                  [&](size_t b, size_t e) { bf16_round_chunk(c->arena + y.head.off + b, bhw + b, e - b); });
+
+  // device memory: one allocation carved into buffers
+  c->dmem_bytes = need;
+  if (cudaMalloc(&c->dmem, need) != cudaSuccess) return fail(MT_ERR_NOMEM, "device allocation failed");
+  uint8_t* p = static_cast<uint8_t*>(c->dmem);
+  auto carve = [&](size_t bytes) {
+    void* r = p;
+    p += align_up(bytes, 256);
+    return r;
+  };
+  const size_t T = s.T, d = s.d, F = s.F, V = s.V;
+  c->wslot[0] = (uint16_t*)carve(y.bf_layer * 2);
+  c->wslot[1] = (uint16_t*)carve(y.bf_layer * 2);
+  const size_t lay_f = y.layer_end(0) - y.layer_begin(0);
+  c->gslot[0] = (float*)carve(lay_f * 4);
+  c->gslot[1] = (float*)carve(lay_f * 4);
+  c->d_head_w = (uint16_t*)carve(head_bf * 2);
+  c->d_head_g = (float*)carve((y.head.off - y.final_norm.off + V * d) * 4);
+  c->xb = (float*)carve((size_t)(s.L + 1) * T * d * 4);
+  c->u_b = (uint16_t*)carve(T * d * 2);
+  c->qkv_b = (uint16_t*)carve(T * (size_t)s.Nqkv * 2);
+  c->ao_b = (uint16_t*)carve(T * (size_t)s.Hd * 2);
+  c->lse = (float*)carve((size_t)s.b * s.H * s.s * 4);
+  c->h_f = (float*)carve(T * d * 4);
+  c->r1 = (float*)carve(T * 4);
+  c->r2 = (float*)carve(T * 4);
+  c->w_b = (uint16_t*)carve(T * d * 2);
+  c->gu_b = (uint16_t*)carve(T * 2 * F * 2);
+  c->act_b = (uint16_t*)carve(T * F * 2);
+  c->gx0 = (float*)carve(T * d * 4);
+  c->gx1 = (float*)carve(T * d * 4);
+  c->gxb = (uint16_t*)carve(T * d * 2);
+  c->dact_b = (uint16_t*)carve(T * F * 2);
+  c->dgu_b = (uint16_t*)carve(T * 2 * F * 2);
+  c->tmp_f = (float*)carve(T * d * 4);
+  c->dh_f = (float*)carve(T * d * 4);
+  c->dhb = (uint16_t*)carve(T * d * 2);
+  c->dao_b = (uint16_t*)carve(T * (size_t)s.Hd * 2);
+  c->dvec = (float*)carve((size_t)s.b * s.H * s.s * 4);
+  c->dqacc = (float*)carve(T * (size_t)s.Hd * 4);
+  c->dqkv_b = (uint16_t*)carve(T * (size_t)s.Nqkv * 2);
+  c->rms_part = (float*)carve((size_t)rmsnorm_bwd_blocks((int)T) * d * 4);
+  c->n_b = (uint16_t*)carve(T * d * 2);
+  c->rf = (float*)carve(T * 4);
+  c->logits = (float*)carve((size_t)Tc * V * 4);
+  c->dz_b = (uint16_t*)carve((size_t)Tc * V * 2);
+  c->rowloss = (float*)carve(T * 4);
+  c->d_tok = (int32_t*)carve((4 * T + 1) * 4);
+  c->d_lab = c->d_tok + T;
+  c->d_offs = c->d_tok + 2 * T;
+  c->d_pos = c->d_tok + 3 * T + 1;
+  c->d_flags = (int32_t*)carve((size_t)(s.L + 2) * 4);
+  c->d_err = (int32_t*)carve(4);
+  c->d_cos = (float*)carve((size_t)s.s * (s.hd / 2) * 4);
+  c->d_sin = (float*)carve((size_t)s.s * (s.hd / 2) * 4);
+  c->d_loss = (float*)carve(4);
+  if ((size_t)(p - static_cast<uint8_t*>(c->dmem)) > need) return fail(MT_ERR_NOMEM, "device carve overflow");
+  if (cudaMemset(c->dmem, 0, need) != cudaSuccess) return fail(MT_ERR_CUDA, "cudaMemset failed");
+  {
+    std::vector<float> cs((size_t)s.s * (s.hd / 2)), sn(cs.size());
+    for (int pos = 0; pos < s.s; ++pos)
+      for (int i = 0; i < s.hd / 2; ++i) {
+        const double th = pow((double)cfg->rope_base, -2.0 * i / s.hd);
+        cs[(size_t)pos * (s.hd / 2) + i] = (float)cos(pos * th);
+        sn[(size_t)pos * (s.hd / 2) + i] = (float)sin(pos * th);
+      }
+    if (cudaMemcpy(c->d_cos, cs.data(), cs.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->d_sin, sn.data(), sn.size() * 4, cudaMemcpyHostToDevice) != cudaSuccess)
+      return fail(MT_ERR_CUDA, "RoPE tables");
+  }
+
+  // streams and events
+  if (cfg->flags & MT_FLAG_SERIALIZE) {
+    if (cudaStreamCreateWithFlags(&c->s_comp, cudaStreamNonBlocking) != cudaSuccess)
+      return fail(MT_ERR_CUDA, "stream");
+    c->s_h2d = c->s_d2h = c->s_comp;
+  } else {
+    if (cudaStreamCreateWithFlags(&c->s_comp, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c->s_h2d, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&c->s_d2h, cudaStreamNonBlocking) != cudaSuccess)
+      return fail(MT_ERR_CUDA, "stream");
+  }
+  // weight loads: 0..L-1 then L-2..0 (layer L-1 stays resident over the turn)
+  for (int l = 0; l < s.L; ++l) c->load_seq.push_back(l);
+  for (int l = s.L - 2; l >= 0; --l) c->load_seq.push_back(l);
+  const int nloads = (int)c->load_seq.size();
+  auto mk = [&](std::vector<cudaEvent_t>& v, int n) {
+    v.assign(n, nullptr);
+    for (auto& e : v)
+      if (cudaEventCreate(&e) != cudaSuccess) return false;
+    return true;
+  };
+  bool ok = mk(c->ev_wready, nloads) && mk(c->ev_compready, nloads) && mk(c->ev_h2d_start, nloads) &&
+            mk(c->ev_slotfree, nloads) && mk(c->ev_gready, s.L) && mk(c->ev_d2h_start, s.L) &&
+            mk(c->ev_gdrained, s.L);
+  for (cudaEvent_t* e : {&c->ev_head_h2d_start, &c->ev_head_wready, &c->ev_head_gready, &c->ev_head_d2h_start,
+                         &c->ev_head_drained, &c->ev_emb_ready, &c->ev_emb_d2h_start, &c->ev_emb_drained,
+                         &c->ev_step_start, &c->ev_fwd_end, &c->ev_head_end, &c->ev_bwd_end, &c->ev_step_end})
+    ok = ok && cudaEventCreate(e) == cudaSuccess;
+  if (!ok) return fail(MT_ERR_CUDA, "event creation failed");
+  if (const char* w = getenv("MT_WAIT_LIMIT_S")) {
+    const double lim = atof(w);
+    if (lim > 0) c->wait_limit_s = lim;
+  }
+  c->opt_thread = std::thread(opt_loop, c);
+  *out = c;
+  return MT_OK;
+}
+
+}  // namespace mteng
+using namespace mteng;
+
+// ---------------------------------------------------------------------------
+// C ABI
+// ---------------------------------------------------------------------------
+extern "C" int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, mt_ctx** out) {
+  g_create_error.clear();
+  return create_impl(cfg, host_param_arena, arena_bytes, out);
+}
+
+extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* labels, float* loss_out) {
+  if (!c) return MT_ERR_ARG;
+  if (!tokens || !labels || !loss_out) return set_err(c, MT_ERR_ARG, "tokens, labels and loss_out are required");
+  const Shapes& s = c->lay.sh;
+  const int T = s.T;
+  for (int t = 0; t < T; ++t)
+    if (tokens[t] < 0 || tokens[t] >= s.V || labels[t] < 0 || labels[t] >= s.V)
+      return set_err(c, MT_ERR_ARG, "token or label outside [0, V)");
+  CK(cudaSetDevice(c->device));
+  // Host staging: tokens, labels and the per-unique-token position lists.
+  int32_t* st = c->stage_i;
+  memcpy(st, tokens, (size_t)T * 4);
+  memcpy(st + T, labels, (size_t)T * 4);
+  std::vector<int32_t> count(s.V, 0);
+  for (int t = 0; t < T; ++t) count[tokens[t]]++;
+  c->uniq.clear();
+  std::vector<int32_t> start(s.V, 0);
+  int32_t* offs = st + 2 * T;
+  int32_t* pos = st + 3 * T + 1;
+  int32_t acc = 0;
+  for (int v = 0; v < s.V; ++v)
+    if (count[v]) {
+      offs[c->uniq.size()] = acc;
+      start[v] = acc;
+      c->uniq.push_back(v);
+      acc += count[v];
+    }
+  const int n_unique = (int)c->uniq.size();
+  offs[n_unique] = acc;
+  for (int t = 0; t < T; ++t) pos[start[tokens[t]]++] = t;  // increasing t within each token
+
+  c->step++;
+  c->opt_status = MT_OK;
+  c->skip_updates = false;
+  c->adamw_s = c->adamw_bytes = 0;
+  c->timing_used = 0;
+  c->timed.clear();
+  c->launches = 0;
+  c->err.clear();
+  int r = enqueue_step(c, n_unique);
+  if (r != MT_OK) {
+    // Let the optimizer finish the jobs already queued and the streams drain.
+    c->skip_updates = true;
+    wait_jobs(c);
+    cudaDeviceSynchronize();
+    return r;
+  }
+  wait_jobs(c);
+  if (!wait_event(c, c->ev_step_end)) return set_err(c, MT_ERR_TIMEOUT, "step did not finish within the wait limit");
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_err(c, MT_ERR_CUDA, cudaGetErrorString(e));
+  int32_t dev_err;
+  memcpy(&dev_err, c->misc_h + 1, 4);
+  if (dev_err != 0) {
+    char m[96];
+    snprintf(m, sizeof m, "kernel reported error %d (bounded wait expired)", dev_err);
+    return set_err(c, MT_ERR_DEVICE, m);
+  }
+  *loss_out = c->misc_h[0] / (float)T;
+  collect_stats(c);
+  if (c->opt_status != MT_OK) return c->opt_status;
+  return MT_OK;
+}
+
+extern "C" int mt_get_grads(mt_ctx* c, float* dst, size_t bytes) {
+  if (!c || !dst) return MT_ERR_ARG;
+  if (bytes < c->lay.total * 4) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
+  memcpy(dst, c->grad, c->lay.total * 4);
+  return MT_OK;
+}
+
+extern "C" int mt_get_params(mt_ctx* c, float* dst, size_t bytes) {
+  if (!c || !dst) return MT_ERR_ARG;
+  if (bytes < c->lay.total * 4) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
+  memcpy(dst, c->arena, c->lay.total * 4);
+  return MT_OK;
+}
+
+extern "C" int mt_get_stats(mt_ctx* c, mt_stats* out) {
+  if (!c || !out) return MT_ERR_ARG;
+  *out = c->stats;
+  return MT_OK;
+}
+
+extern "C" int mt_get_stream(mt_ctx* c, void** stream) {
+  if (!c || !stream) return MT_ERR_ARG;
+  *stream = c->s_comp;
+  return MT_OK;
+}
+
+extern "C" void mt_destroy(mt_ctx* c) { free_all(c); }
+
+extern "C" const char* mt_last_error(const mt_ctx* c) { return c ? c->err.c_str() : g_create_error.c_str(); }

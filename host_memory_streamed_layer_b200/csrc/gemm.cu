@@ -368,7 +368,7 @@ int launch(const GemmDesc& g, cudaStream_t st, int* err) {
   const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
   const int grid = tiles < g_num_sms ? tiles : g_num_sms;
   k_gemm_bf16<BN, A_MN, B_MN><<<grid, NUM_THREADS, C::SMEM, st>>>(ta, tb, p);
-  return cudaGetLastError() == cudaSuccess ? MT_OK : MT_ERR_CUDA;
+  return launch_status();
 }
 
 template <int BN>

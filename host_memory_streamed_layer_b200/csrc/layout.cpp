@@ -1,0 +1,158 @@
+// Configuration checks and the arena / layer-block layouts (see layout.h).
+#include "layout.h"
+
+#include <string.h>
+
+namespace mt {
+
+namespace {
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+}  // namespace
+
+int validate_config(const mt_config* c, std::string* why) {
+  auto fail = [&](int code, const char* m) {
+    if (why) *why = m;
+    return code;
+  };
+  if (!c) return fail(MT_ERR_ARG, "config is NULL");
+  if (c->struct_size != sizeof(mt_config)) return fail(MT_ERR_ARG, "mt_config.struct_size != sizeof(mt_config)");
+  if (c->L < 1 || c->d < 1 || c->H < 1 || c->Hkv < 1 || c->F < 1 || c->V < 1 || c->b < 1 || c->s < 1)
+    return fail(MT_ERR_CONFIG, "every shape must be positive");
+  if (c->d % 64) return fail(MT_ERR_CONFIG, "d must be a multiple of 64");
+  if (c->d > 8192) return fail(MT_ERR_CONFIG, "d must be at most 8192");
+  if (c->d % c->H) return fail(MT_ERR_CONFIG, "d must be a multiple of H");
+  const int hd = c->d / c->H;
+  if (hd != 64 && hd != 128) return fail(MT_ERR_CONFIG, "head_dim d/H must be 64 or 128");
+  if (c->H % c->Hkv) return fail(MT_ERR_CONFIG, "H must be a multiple of Hkv");
+  if (c->F % 8) return fail(MT_ERR_CONFIG, "F must be a multiple of 8");
+  if (c->V % 8) return fail(MT_ERR_CONFIG, "V must be a multiple of 8");
+  if ((int64_t)c->b * c->s > (int64_t)1 << 30) return fail(MT_ERR_CONFIG, "b*s too large");
+  if (!(c->norm_eps > 0) || !(c->rope_base > 1) || !(c->lr >= 0) || !(c->beta1 >= 0 && c->beta1 < 1) ||
+      !(c->beta2 >= 0 && c->beta2 < 1) || !(c->adam_eps > 0) || !(c->wd >= 0))
+    return fail(MT_ERR_CONFIG, "hyper-parameter out of range");
+  if (c->host_threads < 0) return fail(MT_ERR_CONFIG, "host_threads must be >= 0");
+  return MT_OK;
+}
+
+Layout make_layout(const mt_config& c) {
+  Layout y;
+  Shapes& s = y.sh;
+  s.L = c.L;
+  s.d = c.d;
+  s.H = c.H;
+  s.Hkv = c.Hkv;
+  s.F = c.F;
+  s.V = c.V;
+  s.b = c.b;
+  s.s = c.s;
+  s.hd = c.d / c.H;
+  s.T = c.b * c.s;
+  s.Nqkv = (c.H + 2 * c.Hkv) * s.hd;
+  s.Hd = c.H * s.hd;
+  size_t off = 0;
+  auto put = [&](size_t n) {
+    TRef r{off, n};
+    off += round_up(n, 64);
+    return r;
+  };
+  const size_t d = c.d, F = c.F, V = c.V;
+  y.embed = put(V * d);
+  y.layer.resize((size_t)c.L * kLayerTensors);
+  for (int l = 0; l < c.L; ++l) {
+    TRef* t = &y.layer[(size_t)l * kLayerTensors];
+    t[MT_T_ATTN_NORM] = put(d);
+    t[MT_T_WQ] = put((size_t)s.Hd * d);
+    t[MT_T_WK] = put((size_t)c.Hkv * s.hd * d);
+    t[MT_T_WV] = put((size_t)c.Hkv * s.hd * d);
+    t[MT_T_WO] = put(d * (size_t)s.Hd);
+    t[MT_T_MLP_NORM] = put(d);
+    t[MT_T_WGATE] = put(F * d);
+    t[MT_T_WUP] = put(F * d);
+    t[MT_T_WDOWN] = put(d * F);
+  }
+  y.final_norm = put(d);
+  y.head = put(V * d);
+  y.total = off;
+  // bf16 block (128 elements = 256 bytes alignment)
+  size_t b = 0;
+  auto bput = [&](size_t n) {
+    size_t r = b;
+    b += round_up(n, 128);
+    return r;
+  };
+  y.bf_g1 = bput(d);
+  y.bf_qkv = bput((size_t)s.Nqkv * d);
+  y.bf_o = bput(d * (size_t)s.Hd);
+  y.bf_g2 = bput(d);
+  y.bf_gu = bput(2 * F * d);
+  y.bf_d = bput(d * F);
+  y.bf_layer = b;
+  return y;
+}
+
+size_t Layout::bf_of(int tid) const {
+  const size_t d = sh.d;
+  switch (tid) {
+    case MT_T_ATTN_NORM: return bf_g1;
+    case MT_T_WQ: return bf_qkv;
+    case MT_T_WK: return bf_qkv + (size_t)sh.Hd * d;
+    case MT_T_WV: return bf_qkv + (size_t)(sh.Hd + sh.Hkv * sh.hd) * d;
+    case MT_T_WO: return bf_o;
+    case MT_T_MLP_NORM: return bf_g2;
+    case MT_T_WGATE: return bf_gu;
+    case MT_T_WUP: return bf_gu + (size_t)sh.F * d;
+    case MT_T_WDOWN: return bf_d;
+  }
+  return 0;
+}
+
+}  // namespace mt
+
+extern "C" int mt_config_default(mt_config* cfg) {
+  if (!cfg) return MT_ERR_ARG;
+  memset(cfg, 0, sizeof(*cfg));
+  cfg->struct_size = sizeof(mt_config);
+  cfg->norm_eps = 1e-5f;
+  cfg->rope_base = 10000.f;
+  cfg->lr = 1e-3f;
+  cfg->beta1 = 0.9f;
+  cfg->beta2 = 0.95f;
+  cfg->adam_eps = 1e-8f;
+  cfg->wd = 0.1f;
+  return MT_OK;
+}
+
+extern "C" size_t mt_arena_bytes(const mt_config* cfg) {
+  if (mt::validate_config(cfg, nullptr) != MT_OK) return 0;
+  return mt::make_layout(*cfg).total * sizeof(float);
+}
+
+extern "C" int mt_tensor_offset(const mt_config* cfg, int layer, int tid, size_t* offset_floats, size_t* numel) {
+  if (mt::validate_config(cfg, nullptr) != MT_OK) return MT_ERR_CONFIG;
+  mt::Layout y = mt::make_layout(*cfg);
+  mt::TRef r;
+  if (layer == -1) {
+    if (tid == MT_T_EMBED)
+      r = y.embed;
+    else if (tid == MT_T_FINAL_NORM)
+      r = y.final_norm;
+    else if (tid == MT_T_LM_HEAD)
+      r = y.head;
+    else
+      return MT_ERR_ARG;
+  } else {
+    if (layer < 0 || layer >= cfg->L || tid < 0 || tid >= mt::kLayerTensors) return MT_ERR_ARG;
+    r = y.t(layer, tid);
+  }
+  if (offset_floats) *offset_floats = r.off;
+  if (numel) *numel = r.n;
+  return MT_OK;
+}
+
+extern "C" size_t mt_host_state_bytes(const mt_config* cfg) {
+  if (mt::validate_config(cfg, nullptr) != MT_OK) return 0;
+  mt::Layout y = mt::make_layout(*cfg);
+  const size_t P = y.total;
+  const size_t bf = (size_t)y.sh.L * y.bf_layer + 2 * (size_t)y.sh.V * y.sh.d + y.sh.d + 256;
+  return P * 4 * 3 + bf * 2 + (size_t)y.sh.T * y.sh.d * 4;  // m, v, grads; bf16 copy; embedding staging
+}

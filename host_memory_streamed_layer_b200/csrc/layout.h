@@ -1,0 +1,58 @@
+// Host and device layouts of the streamed model.
+//
+// fp32 master arena (caller-visible, also the layout of the gradient arena):
+//   embedding [V,d]; per layer: attention-norm gain [d], Wq [H hd, d],
+//   Wk [Hkv hd, d], Wv [Hkv hd, d], Wo [d, H hd], MLP-norm gain [d],
+//   Wgate [F,d], Wup [F,d], Wdown [d,F]; final-norm gain [d]; LM head [V,d].
+//   Row-major [out, in], every tensor on a 256-byte boundary. With d a
+//   multiple of 64 no padding is needed, so Wq|Wk|Wv and Wgate|Wup are
+//   adjacent and one layer is one contiguous range.
+// bf16 layer block (host mirror and device weight slot), per layer:
+//   g1 [d] | Wqkv [(H+2Hkv) hd, d] | Wo [d, H hd] | g2 [d] | Wgu [2F, d] | Wd [d, F]
+//   each part on a 256-byte boundary.
+#pragma once
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "mt.h"
+
+namespace mt {
+
+constexpr int kLayerTensors = 9;
+
+struct TRef {
+  size_t off = 0;  // elements
+  size_t n = 0;    // elements
+};
+
+struct Shapes {
+  int L, d, H, Hkv, F, V, b, s, hd, T, Nqkv, Hd;  // Hd = H * hd
+};
+
+struct Layout {
+  Shapes sh{};
+  // fp32 arena, in floats
+  TRef embed, final_norm, head;
+  std::vector<TRef> layer;  // L * kLayerTensors
+  size_t total = 0;
+  size_t layer_begin(int l) const { return layer[(size_t)l * kLayerTensors].off; }
+  size_t layer_end(int l) const {
+    const TRef& t = layer[(size_t)l * kLayerTensors + kLayerTensors - 1];
+    return t.off + t.n;
+  }
+  const TRef& t(int l, int tid) const { return layer[(size_t)l * kLayerTensors + tid]; }
+  // bf16 layer block, in elements
+  size_t bf_g1 = 0, bf_qkv = 0, bf_o = 0, bf_g2 = 0, bf_gu = 0, bf_d = 0, bf_layer = 0;
+  // bf16 offset of arena tensor tid inside the layer block
+  size_t bf_of(int tid) const;
+};
+
+// Validates cfg (MT_OK or MT_ERR_CONFIG / MT_ERR_ARG with a message).
+int validate_config(const mt_config* cfg, std::string* why);
+Layout make_layout(const mt_config& cfg);
+
+}  // namespace mt

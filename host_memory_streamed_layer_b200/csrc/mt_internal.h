@@ -8,6 +8,11 @@
 
 namespace mt {
 
+// Status of the launch just made: MT_OK, or MT_ERR_CUDA with the CUDA message
+// kept for last_launch_error() (per thread).
+int launch_status();
+const char* last_launch_error();
+
 enum GemmEpi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_F32_ADD = 2 };
 
 // C[M,N] = A[M,K] * B[N,K]^T (+ R for EPI_F32_ADD; R may alias C).
@@ -29,5 +34,48 @@ struct GemmDesc {
 };
 
 int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
+
+// Causal attention with grouped KV heads. q, k, v: column ranges of one bf16
+// row per token (pitch ldqkv); o, dout: [T, H*hd] bf16 (pitch ldo); lse, dvec:
+// fp32 [b, H, s]; dq_acc: fp32 [T, ldqa] accumulator (zeroed by the call);
+// dq, dk, dv: bf16 outputs with pitches lddq / lddkv.
+struct AttnArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  int64_t ldqkv;
+  void* o;
+  int64_t ldo;
+  float* lse;
+  const void* dout;
+  float* dvec;
+  float* dq_acc;
+  int64_t ldqa;
+  void* dq;
+  int64_t lddq;
+  void* dk;
+  void* dv;
+  int64_t lddkv;
+  int b, s, H, Hkv, hd;
+  float scale;
+};
+int attention_fwd(const AttnArgs& a, cudaStream_t st);
+int attention_bwd(const AttnArgs& a, cudaStream_t st);
+
+int launch_rmsnorm_fwd(const float* x, const void* g, void* y, float* rstd, int T, int d, float eps, cudaStream_t st);
+int rmsnorm_bwd_blocks(int T);
+int launch_rmsnorm_bwd(const float* x, const void* g, const float* rstd, const float* dy, const float* dres,
+                       float* dx, void* dx_bf16, float* dg_part, float* dg, int T, int d, cudaStream_t st);
+int launch_rope(void* buf, int64_t ld, int T, int s, int nheads, int hd, int col0, const float* cosb,
+                const float* sinb, float sign, cudaStream_t st);
+int launch_swiglu_fwd(const void* gu, void* act, int T, int F, cudaStream_t st);
+int launch_swiglu_bwd(const void* gu, const void* dact, void* dgu, int T, int F, cudaStream_t st);
+int launch_embed_fwd(const int* tok, const void* E, float* x, int T, int d, cudaStream_t st);
+int launch_embed_bwd(const int* offs, const int* pos, int n_unique, const float* dx, float* rows, int d,
+                     cudaStream_t st);
+int launch_softmax_ce(const float* z, int64_t ldz, const int* labels, void* dz, int64_t lddz, float* row_loss,
+                      int Tc, int V, float scale, cudaStream_t st);
+int launch_sum_all(const float* v, int n, float* out, int accumulate, cudaStream_t st);
+int launch_cast_f32_bf16(const float* in, void* out, int64_t n, cudaStream_t st);
 
 }  // namespace mt

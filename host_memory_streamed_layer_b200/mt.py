@@ -30,7 +30,7 @@ class MTError(RuntimeError):
 
 def _check(rc: int, what: str = "", ctx=None):
     if rc != MT_OK:
-        msg = lib.mt_last_error(ctx).decode() if hasattr(lib, "mt_last_error") else ""
+        msg = lib.mt_last_error(ctx).decode() if ctx else ""
         raise MTError(rc, f"{what} {msg}".strip())
     return rc
 
@@ -50,3 +50,190 @@ _sig("mt_k_gemm_bf16", c_int, c_void_p, c_i64, c_int, c_void_p, c_i64, c_int, c_
 def mt_k_gemm_bf16(A, lda, a_mn, B, ldb, b_mn, C, ldc, out_kind, R, ldr, M, N, K, stream=0, dev_err=0):
     return _check(lib.mt_k_gemm_bf16(A, lda, a_mn, B, ldb, b_mn, C, ldc, out_kind, R or None, ldr, M, N, K,
                                      stream or None, dev_err or None), "mt_k_gemm_bf16")
+
+c_float, c_f = ctypes.c_float, ctypes.c_float
+
+_sig("mt_k_rmsnorm_fwd", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_float, c_void_p)
+_sig("mt_k_rmsnorm_bwd_partial_floats", c_size_t, c_int, c_int)
+_sig("mt_k_rmsnorm_bwd", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+     c_void_p, c_int, c_int, c_void_p)
+_sig("mt_k_rope", c_int, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_float, c_void_p)
+_sig("mt_k_swiglu_fwd", c_int, c_void_p, c_void_p, c_int, c_int, c_void_p)
+_sig("mt_k_swiglu_bwd", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p)
+_sig("mt_k_embed_fwd", c_int, c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p)
+_sig("mt_k_embed_bwd", c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p)
+_sig("mt_k_softmax_ce", c_int, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_int, c_int, c_float, c_void_p)
+_sig("mt_k_attn_fwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_int, c_int, c_int,
+     c_int, c_int, c_void_p)
+_sig("mt_k_attn_bwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_void_p,
+     c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p)
+
+
+def _p(x):
+    return x or None
+
+
+def mt_k_rmsnorm_fwd(x, g, y, rstd, T, d, eps, stream=0):
+    return _check(lib.mt_k_rmsnorm_fwd(x, g, y, _p(rstd), T, d, eps, _p(stream)), "mt_k_rmsnorm_fwd")
+
+
+def mt_k_rmsnorm_bwd_partial_floats(T, d):
+    return lib.mt_k_rmsnorm_bwd_partial_floats(T, d)
+
+
+def mt_k_rmsnorm_bwd(x, g, rstd, dy, dres, dx, dx_bf16, dg_part, dg, T, d, stream=0):
+    return _check(lib.mt_k_rmsnorm_bwd(x, g, rstd, dy, _p(dres), dx, _p(dx_bf16), dg_part, dg, T, d, _p(stream)),
+                  "mt_k_rmsnorm_bwd")
+
+
+def mt_k_rope(buf, ld, T, s, nheads, hd, col0, cos_tab, sin_tab, sign, stream=0):
+    return _check(lib.mt_k_rope(buf, ld, T, s, nheads, hd, col0, cos_tab, sin_tab, sign, _p(stream)), "mt_k_rope")
+
+
+def mt_k_swiglu_fwd(gu, act, T, F, stream=0):
+    return _check(lib.mt_k_swiglu_fwd(gu, act, T, F, _p(stream)), "mt_k_swiglu_fwd")
+
+
+def mt_k_swiglu_bwd(gu, dact, dgu, T, F, stream=0):
+    return _check(lib.mt_k_swiglu_bwd(gu, dact, dgu, T, F, _p(stream)), "mt_k_swiglu_bwd")
+
+
+def mt_k_embed_fwd(tok, E, x, T, d, stream=0):
+    return _check(lib.mt_k_embed_fwd(tok, E, x, T, d, _p(stream)), "mt_k_embed_fwd")
+
+
+def mt_k_embed_bwd(offs, pos, n_unique, dx, rows, d, stream=0):
+    return _check(lib.mt_k_embed_bwd(offs, pos, n_unique, dx, rows, d, _p(stream)), "mt_k_embed_bwd")
+
+
+def mt_k_softmax_ce(z, ldz, labels, dz, lddz, row_loss, Tc, V, scale, stream=0):
+    return _check(lib.mt_k_softmax_ce(z, ldz, labels, dz, lddz, row_loss, Tc, V, scale, _p(stream)),
+                  "mt_k_softmax_ce")
+
+
+def mt_k_attn_fwd(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, stream=0):
+    return _check(lib.mt_k_attn_fwd(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, _p(stream)), "mt_k_attn_fwd")
+
+
+def mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv, b, s, H, Hkv, hd,
+                  stream=0):
+    return _check(lib.mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv,
+                                    b, s, H, Hkv, hd, _p(stream)), "mt_k_attn_bwd")
+
+
+# ---------------------------------------------------------------------------
+# Engine API (include/mt.h)
+# ---------------------------------------------------------------------------
+MT_FLAG_SERIALIZE, MT_FLAG_KERNEL_TIMING, MT_FLAG_NO_UPDATE = 0x1, 0x2, 0x4
+MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
+MT_T_EMBED, MT_T_FINAL_NORM, MT_T_LM_HEAD = 100, 101, 102
+
+
+class mt_config(ctypes.Structure):
+    _fields_ = [("struct_size", ctypes.c_uint32), ("L", ctypes.c_int32), ("d", ctypes.c_int32),
+                ("H", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("F", ctypes.c_int32), ("V", ctypes.c_int32),
+                ("b", ctypes.c_int32), ("s", ctypes.c_int32), ("norm_eps", ctypes.c_float),
+                ("rope_base", ctypes.c_float), ("lr", ctypes.c_float), ("beta1", ctypes.c_float),
+                ("beta2", ctypes.c_float), ("adam_eps", ctypes.c_float), ("wd", ctypes.c_float),
+                ("seed", ctypes.c_uint64), ("flags", ctypes.c_uint32), ("device", ctypes.c_int32),
+                ("host_threads", ctypes.c_int32)]
+
+
+class mt_stats(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_double) for n in (
+        "step_ms", "fwd_ms", "head_ms", "bwd_ms", "h2d_bytes", "d2h_bytes", "h2d_ms", "d2h_ms",
+        "wait_weights_ms", "adamw_ms", "adamw_bytes", "gemm_flops", "gemm_ms")] + \
+        [("gemm_launches", ctypes.c_int64), ("attn_flops", ctypes.c_double), ("attn_ms", ctypes.c_double),
+         ("attn_launches", ctypes.c_int64), ("kernel_launches", ctypes.c_int64)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+_cfgp = ctypes.POINTER(mt_config)
+_sig("mt_config_default", c_int, _cfgp)
+_sig("mt_arena_bytes", c_size_t, _cfgp)
+_sig("mt_tensor_offset", c_int, _cfgp, c_int, c_int, ctypes.POINTER(c_size_t), ctypes.POINTER(c_size_t))
+_sig("mt_host_state_bytes", c_size_t, _cfgp)
+_sig("mt_create", c_int, _cfgp, c_void_p, c_size_t, ctypes.POINTER(c_void_p))
+_sig("mt_train_step", c_int, c_void_p, c_void_p, c_void_p, ctypes.POINTER(ctypes.c_float))
+_sig("mt_get_grads", c_int, c_void_p, c_void_p, c_size_t)
+_sig("mt_get_params", c_int, c_void_p, c_void_p, c_size_t)
+_sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
+_sig("mt_destroy", None, c_void_p)
+_sig("mt_get_stream", c_int, c_void_p, ctypes.POINTER(c_void_p))
+_sig("mt_last_error", ctypes.c_char_p, c_void_p)
+_sig("mt_k_adamw_host", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_float, c_float,
+     c_float, c_float, c_float, c_int)
+
+
+def mt_config_default(**shape) -> mt_config:
+    cfg = mt_config()
+    _check(lib.mt_config_default(ctypes.byref(cfg)), "mt_config_default")
+    for k, v in shape.items():
+        setattr(cfg, k, v)
+    return cfg
+
+
+def mt_arena_bytes(cfg: mt_config) -> int:
+    return lib.mt_arena_bytes(ctypes.byref(cfg))
+
+
+def mt_tensor_offset(cfg: mt_config, layer: int, tid: int):
+    off, n = c_size_t(), c_size_t()
+    _check(lib.mt_tensor_offset(ctypes.byref(cfg), layer, tid, ctypes.byref(off), ctypes.byref(n)),
+           "mt_tensor_offset")
+    return off.value, n.value
+
+
+def mt_host_state_bytes(cfg: mt_config) -> int:
+    return lib.mt_host_state_bytes(ctypes.byref(cfg))
+
+
+def mt_create(cfg: mt_config, arena_ptr: int = 0, arena_bytes: int = 0) -> int:
+    """Returns the context handle (an int). arena_ptr: host address or 0."""
+    ctx = c_void_p()
+    rc = lib.mt_create(ctypes.byref(cfg), arena_ptr or None, arena_bytes, ctypes.byref(ctx))
+    if rc != MT_OK:
+        raise MTError(rc, "mt_create " + lib.mt_last_error(None).decode())
+    return ctx.value
+
+
+def mt_train_step(ctx: int, tokens_ptr: int, labels_ptr: int) -> float:
+    loss = ctypes.c_float()
+    rc = lib.mt_train_step(ctx, tokens_ptr, labels_ptr, ctypes.byref(loss))
+    if rc != MT_OK:
+        raise MTError(rc, "mt_train_step " + lib.mt_last_error(ctx).decode())
+    return loss.value
+
+
+def mt_get_grads(ctx: int, dst_ptr: int, nbytes: int):
+    return _check(lib.mt_get_grads(ctx, dst_ptr, nbytes), "mt_get_grads", ctx)
+
+
+def mt_get_params(ctx: int, dst_ptr: int, nbytes: int):
+    return _check(lib.mt_get_params(ctx, dst_ptr, nbytes), "mt_get_params", ctx)
+
+
+def mt_get_stats(ctx: int) -> dict:
+    st = mt_stats()
+    _check(lib.mt_get_stats(ctx, ctypes.byref(st)), "mt_get_stats", ctx)
+    return st.as_dict()
+
+
+def mt_get_stream(ctx: int) -> int:
+    st = c_void_p()
+    _check(lib.mt_get_stream(ctx, ctypes.byref(st)), "mt_get_stream", ctx)
+    return st.value or 0
+
+
+def mt_destroy(ctx: int):
+    lib.mt_destroy(ctx)
+
+
+def mt_last_error(ctx: int = 0) -> str:
+    return lib.mt_last_error(ctx or None).decode()
+
+
+def mt_k_adamw_host(p, g, m, v, pb, n, lr, beta1, beta2, eps, wd, t):
+    return _check(lib.mt_k_adamw_host(p, g, m, v, pb or None, n, lr, beta1, beta2, eps, wd, t), "mt_k_adamw_host")

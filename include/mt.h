@@ -143,6 +143,12 @@ int mt_get_params(mt_ctx* ctx, float* dst, size_t bytes);
 /* Counters of the last step. */
 int mt_get_stats(mt_ctx* ctx, mt_stats* out);
 
+/* The context's compute stream (a cudaStream_t) in *stream, so a caller can
+ * order or time its own work against the step (for example record CUDA events
+ * around a sequence of mt_train_step calls). The stream stays owned by the
+ * context. */
+int mt_get_stream(mt_ctx* ctx, void** stream);
+
 /* Waits for the context's streams, frees its device memory and unpins or
  * frees its host memory. NULL is ignored. */
 void mt_destroy(mt_ctx* ctx);

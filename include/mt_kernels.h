@@ -47,6 +47,81 @@ int mt_k_gemm_bf16(const void* A, int64_t lda, int a_mn_major, const void* B, in
                    void* C, int64_t ldc, int out_kind, const float* R, int64_t ldr, int M, int N, int K,
                    void* stream, int32_t* dev_err);
 
+/* RMSNorm forward, one row per token (reading of the Llama block: eps inside
+ * the root): y[t] = x[t] / sqrt(mean_j x[t,j]^2 + eps) * g.
+ * x fp32 [T,d]; g bf16 [d]; y bf16 [T,d]; rstd fp32 [T] (may be NULL) receives
+ * 1/sqrt(mean x^2 + eps). d multiple of 4. */
+int mt_k_rmsnorm_fwd(const float* x, const void* g, void* y, float* rstd, int T, int d, float eps, void* stream);
+
+/* Floats of the per-block partial buffer mt_k_rmsnorm_bwd needs for T rows. */
+size_t mt_k_rmsnorm_bwd_partial_floats(int T, int d);
+
+/* RMSNorm backward (hand-written gradient, intelligentliving.co "Checkpointing,
+ * Manual Gradients, and CPU-Side Optimizer Steps"):
+ *   dx[t,j] = dres[t,j] + r g_j dy[t,j] - x[t,j] r^3 (sum_i g_i dy[t,i] x[t,i]) / d
+ *   dg[j]   = sum_t dy[t,j] x[t,j] r_t   (fixed summation order)
+ * x, dy, dres (may be NULL), dx: fp32 [T,d]; rstd fp32 [T]; g bf16 [d];
+ * dx_bf16 (may be NULL) receives a bf16 copy of dx; dg_part: caller scratch of
+ * mt_k_rmsnorm_bwd_partial_floats(T,d) floats; dg fp32 [d]. d <= 8192. */
+int mt_k_rmsnorm_bwd(const float* x, const void* g, const float* rstd, const float* dy, const float* dres, float* dx,
+                     void* dx_bf16, float* dg_part, float* dg, int T, int d, void* stream);
+
+/* RoPE in place on nheads bf16 heads of width hd starting at column col0 of a
+ * [T, ld] buffer, token t at position t % s; rotate-half pairs (i, i+hd/2)
+ * rotated by angle pos * theta_i (cos/sin tables fp32 [s, hd/2]).
+ * sign = +1 forward rotation, -1 its transpose (the backward). */
+int mt_k_rope(void* buf, int64_t ld, int T, int s, int nheads, int hd, int col0, const float* cos_tab,
+              const float* sin_tab, float sign, void* stream);
+
+/* SwiGLU: gu bf16 [T, 2F] = [gate | up]; act bf16 [T,F] = silu(gate) * up.
+ * Backward: dgu = [dact * up * s(1 + gate(1-s)) | dact * gate * s], s = sigmoid(gate).
+ * F multiple of 8. */
+int mt_k_swiglu_fwd(const void* gu, void* act, int T, int F, void* stream);
+int mt_k_swiglu_bwd(const void* gu, const void* dact, void* dgu, int T, int F, void* stream);
+
+/* Embedding gather x[t] = E[tok[t]] (bf16 table -> fp32 rows). E may be a
+ * device pointer or a mapped pinned-host pointer. d multiple of 8. */
+int mt_k_embed_fwd(const int32_t* tok, const void* E, float* x, int T, int d, void* stream);
+
+/* Embedding gradient rows: rows[u] = sum over i in [offs[u], offs[u+1]) of
+ * dx[pos[i]] in that order, for n_unique unique tokens. fp32. */
+int mt_k_embed_bwd(const int32_t* offs, const int32_t* pos, int n_unique, const float* dx, float* rows, int d,
+                   void* stream);
+
+/* Fused softmax cross-entropy over fp32 logits z [Tc, V] (pitch ldz):
+ *   row_loss[t] = logsumexp(z[t]) - z[t, labels[t]]
+ *   dz[t]       = (softmax(z[t]) - onehot(labels[t])) * scale   (bf16, pitch lddz)
+ * V multiple of 4. */
+int mt_k_softmax_ce(const float* z, int64_t ldz, const int32_t* labels, void* dz, int64_t lddz, float* row_loss,
+                    int Tc, int V, float scale, void* stream);
+
+/* Causal attention forward, scale 1/sqrt(hd), query head h reads KV head
+ * h / (H/Hkv). q, k, v: bf16 column ranges of a per-token row (pitch ldqkv),
+ * token t = bi*s + i; o bf16 [b*s, H*hd] (pitch ldo); lse fp32 [b,H,s] natural
+ * log-sum-exp of the scaled scores. hd 64 or 128. */
+int mt_k_attn_fwd(const void* q, const void* k, const void* v, int64_t ldqkv, void* o, int64_t ldo, float* lse,
+                  int b, int s, int H, int Hkv, int hd, void* stream);
+
+/* Causal attention backward from o, lse and dout (bf16, pitch ldo):
+ * dvec fp32 [b,H,s] and dq_acc fp32 [b*s, ldqa] are caller scratch (dq_acc is
+ * zeroed by the call); dq (pitch lddq), dk and dv (pitch lddkv) are bf16
+ * outputs laid out like q, k, v. dk, dv of a KV head sum over its query heads. */
+int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o, const void* dout,
+                  int64_t ldo, const float* lse, float* dvec, float* dq_acc, int64_t ldqa, void* dq, int64_t lddq,
+                  void* dk, void* dv, int64_t lddkv, int b, int s, int H, int Hkv, int hd, void* stream);
+
+/* Host AdamW over n fp32 elements, in place (HOST pointers, runs on the
+ * calling thread; the engine runs the same routine across its worker pool):
+ *   p <- p (1 - lr wd); m <- b1 m + (1-b1) g; v <- b2 v + (1-b2) g^2;
+ *   p <- p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
+ * and pb[i] <- bf16(p[i]) rounded to nearest even when pb is not NULL
+ * (the streamed copy). t >= 1 counts steps. The update is Adam (Kingma & Ba,
+ * cited by the MegaTrain paper) with decoupled decay, on the CPU as MegaTrain
+ * does (intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
+ * Optimizer Steps"). */
+int mt_k_adamw_host(float* p, const float* g, float* m, float* v, uint16_t* pb, size_t n, float lr, float beta1,
+                    float beta2, float eps, float wd, int t);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,11 +34,13 @@ from .model import (  # noqa: F401
     rope_bwd,
     attention_fwd,
     attention_bwd,
+    attention_lse,
     silu,
     swiglu_fwd,
     swiglu_bwd,
     layer_fwd,
     layer_bwd,
+    softmax_ce,
     head_ce_fwd_bwd,
     train_step_grads,
 )

@@ -80,6 +80,25 @@ def test_attention_bwd_equal_keys_give_zero_dq():
     assert np.isfinite(dk).all() and np.isfinite(dv).all()
 
 
+def test_attention_lse_closed_form_and_consistency():
+    """q = 0: every visible score is 0, so lse_i = log(i + 1). In general
+    P = exp(S / sqrt(hd) - lse) on visible entries."""
+    rng = np.random.default_rng(13)
+    s = 7
+    q0 = np.zeros((1, s, 2, 4))
+    k = rng.normal(size=(1, s, 1, 4))
+    assert np.allclose(oracle.attention_lse(q0, k)[0, 0], np.log(np.arange(1, s + 1)))
+    q = rng.normal(size=(2, s, 4, 8))
+    k = rng.normal(size=(2, s, 2, 8))
+    v = rng.normal(size=(2, s, 2, 8))
+    _, P = oracle.attention_fwd(q, k, v)
+    lse = oracle.attention_lse(q, k)
+    kk = np.repeat(k, 2, axis=2)
+    S = np.einsum("bihd,bjhd->bhij", q, kk) / np.sqrt(8)
+    vis = np.tril(np.ones((s, s), dtype=bool))
+    assert np.allclose(np.exp(S - lse[..., None])[:, :, vis], P[:, :, vis])
+
+
 def test_attention_matches_torch_sdpa():
     rng = np.random.default_rng(4)
     q = rng.normal(size=(2, 13, 6, 16))
