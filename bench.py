@@ -1,0 +1,414 @@
+#!/usr/bin/env python
+"""Benchmark of one host-memory-streamed training step (MegaTrain's method).
+
+One step = forward over every streamed layer, LM head and cross-entropy,
+checkpointed recompute and backward, gradient offload and the host AdamW
+update, on a Llama-style decoder whose fp32 master weights and Adam moments
+live in host memory. Default workload: the 1.3B decoder (24 layers, d 2048,
+16 heads, SwiGLU 5504, vocab 32000) on 8 x 2048 tokens per GPU.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   (the fp64 CPU oracle, bounded sample)
+
+Prints one JSON line on rank 0. With N > 1 (torchrun, one process per GPU)
+every rank trains an independent replica (the method runs on one GPU; no
+collective is on the data path) and `value` is the sum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "training tokens/s"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="llama-1.3b", choices=list(synth.WORKLOADS))
+    ap.add_argument("--impl", default="mt", choices=["mt", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    try:
+        return json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))), "measured"
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_desc(name, sh):
+    return (f"{name}: {sh['L']} layers, d {sh['d']}, {sh['H']} heads ({sh['Hkv']} kv), SwiGLU {sh['F']}, "
+            f"vocab {sh['V']}, {sh['b']} x {sh['s']} tokens per GPU; fp32 master + AdamW moments in host RAM, "
+            f"bf16 weights streamed per layer")
+
+
+def flops_per_step(sh):
+    """Model FLOPs (6 N T with causal attention) and the FLOPs this schedule
+    executes (forward, recompute without the down projection, backward,
+    flash-attention backward recompute, LM head)."""
+    L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
+    hd = d // H
+    T = b * s
+    Pm = d * (H + 2 * Hkv) * hd + d * H * hd + 3 * d * F
+    A = 2.0 * b * s * s * H * hd  # causal attention forward (QK^T and PV over the visible half)
+    model = L * (6.0 * T * Pm + 3 * A) + 6.0 * T * V * d
+    executed = L * (2.0 * T * Pm + A) + (L - 1) * (2.0 * T * (Pm - d * F) + A) + L * (4.0 * T * Pm + 2.5 * A) \
+        + 6.0 * T * V * d
+    return model, executed
+
+
+# ---------------------------------------------------------------------------
+# Clock sampling during the timed region.
+# ---------------------------------------------------------------------------
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        rows = []
+        for line in open(self.f.name):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on a bounded sample of the same workload.
+# ---------------------------------------------------------------------------
+def oracle_sample_tokens_per_s(sh, seed=0):
+    """Times the oracle on one 2048-token sequence (or the workload's sequence
+    length) through one decoder layer forward + backward, the final norm + LM
+    head + cross-entropy forward/backward, and AdamW over one layer's
+    parameters; scales to the full step (b sequences x L layers, AdamW over
+    all parameters). Returns (tokens/s, seconds measured, description)."""
+    import oracle
+    c = oracle.OracleConfig(**{**sh, "b": 1, "L": 1})
+    hd = c.d // c.H
+    W = {tid: synth.init_tensor(seed, 0, tid, shp).astype(np.float64)
+         for tid, shp in synth.layer_shapes(c.d, c.H, c.Hkv, c.F, hd)}
+    rng = np.random.default_rng(seed)
+    x = rng.normal(size=(1, c.s, c.d))
+    cos, sin = oracle.rope_tables(c.s, hd, c.rope_base)
+    t0 = time.perf_counter()
+    xn, cache = oracle.layer_fwd(x, W, c, cos, sin)
+    oracle.layer_bwd(rng.normal(size=x.shape), W, cache, c, cos, sin)
+    t_layer = time.perf_counter() - t0
+    Wh = synth.init_tensor(seed, -1, synth.LM_HEAD, (c.V, c.d)).astype(np.float64)
+    lab = rng.integers(0, c.V, c.s)
+    t0 = time.perf_counter()
+    oracle.head_ce_fwd_bwd(x[0], np.ones(c.d), Wh, lab, c.norm_eps)
+    t_head = time.perf_counter() - t0
+    P_layer = sum(int(np.prod(s)) for _, s in synth.layer_shapes(c.d, c.H, c.Hkv, c.F, hd))
+    params = np.concatenate([w.reshape(-1) for w in W.values()])
+    g = rng.normal(size=params.size) * 1e-4
+    t0 = time.perf_counter()
+    oracle.adamw_update(params, g, np.zeros_like(params), np.zeros_like(params), 1, c.lr, c.beta1, c.beta2,
+                        c.adam_eps, c.wd)
+    t_adam = time.perf_counter() - t0
+    P_total = sh["L"] * P_layer + 2 * sh["V"] * sh["d"] + sh["d"]
+    t_step = sh["b"] * (sh["L"] * t_layer + t_head) + t_adam * P_total / P_layer
+    T = sh["b"] * sh["s"]
+    desc = (f"oracle (fp64 numpy) on one {c.s}-token sequence: one decoder layer fwd+bwd {t_layer:.2f}s, "
+            f"head+CE fwd+bwd {t_head:.2f}s, AdamW over one layer ({P_layer/1e6:.1f}M params) {t_adam:.2f}s; "
+            f"scaled to {sh['b']} sequences x {sh['L']} layers and AdamW over {P_total/1e9:.3f}B params")
+    return T / t_step, t_layer + t_head + t_adam, desc
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# Reference arm: the oracle as it stands, bounded samples.
+# ---------------------------------------------------------------------------
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    sh = synth.WORKLOADS[args.workload]
+    for _ in range(args.warmup):
+        oracle_sample_tokens_per_s(sh)
+    vals, secs = [], 0.0
+    desc = ""
+    for _ in range(args.steps):
+        v, s, desc = oracle_sample_tokens_per_s(sh)
+        vals.append(v)
+        secs += s
+    value = statistics.median(vals)
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sh["b"] * sh["s"] / value * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(args.workload, sh), "global_batch": sh["b"], "seq_len": sh["s"],
+                   "parallelism": "none (CPU)"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# Link bandwidth (pinned 1 GiB copies, best of 3) measured in the same run.
+# ---------------------------------------------------------------------------
+def link_bandwidth(torch, dev):
+    n = 1 << 30
+    h = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    h2 = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(n, dtype=torch.uint8, device=dev)
+    d2 = torch.empty(n, dtype=torch.uint8, device=dev)
+    s1, s2 = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def best(fn):
+        b = 1e9
+        for _ in range(3):
+            torch.cuda.synchronize(dev)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize(dev)
+            b = min(b, e0.elapsed_time(e1) / 1e3)
+        return b
+
+    def h2d():
+        d.copy_(h, non_blocking=True)
+
+    def d2h():
+        h.copy_(d, non_blocking=True)
+
+    def both():
+        cur = torch.cuda.current_stream(dev)
+        s1.wait_stream(cur)
+        s2.wait_stream(cur)
+        with torch.cuda.stream(s1):
+            d.copy_(h, non_blocking=True)
+        with torch.cuda.stream(s2):
+            h2.copy_(d2, non_blocking=True)
+        cur.wait_stream(s1)
+        cur.wait_stream(s2)
+
+    r = {"h2d_gbs": n / best(h2d) / 1e9, "d2h_gbs": n / best(d2h) / 1e9, "bidir_gbs_each": n / best(both) / 1e9}
+    del h, h2, d, d2
+    torch.cuda.empty_cache()
+    return r
+
+
+# ---------------------------------------------------------------------------
+# Main arm.
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    from datetime import timedelta
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
+
+    def allmax(x):
+        if dist is None:
+            return x
+        t = torch.tensor([float(x)], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    from host_memory_streamed_layer_b200 import arena, mt
+    sh = synth.WORKLOADS[args.workload]
+    T = sh["b"] * sh["s"]
+    cfg = arena.config(sh)
+    cfg.seed = 1234 + rank
+    cfg.device = local
+    cfg.flags = mt.MT_FLAG_KERNEL_TIMING
+    ncpu = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cfg.host_threads = max(1, ncpu // world)
+
+    # Host memory: every replica holds its own master, moments, gradients and bf16 copy.
+    need = mt.mt_arena_bytes(cfg) + mt.mt_host_state_bytes(cfg)
+    try:
+        import psutil
+        avail = psutil.virtual_memory().available
+    except Exception:
+        avail = None
+    ok = 1.0 if (avail is None or need * world * 1.1 < avail) else 0.0
+    ok = -allmax(-ok) if dist is not None else ok
+    if ok < 1:
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": None, "unit": UNIT, "n_gpus": world,
+                              "error": f"host RAM: {world} replicas need {need * world / 1e9:.0f} GB, "
+                                       f"{(avail or 0) / 1e9:.0f} GB available"}), flush=True)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    link = link_bandwidth(torch, dev) if rank == 0 else None
+    ctx = mt.mt_create(cfg)
+    try:
+        nsteps = args.warmup + 2 * args.steps
+        toks = []
+        for i in range(nsteps):
+            t, l = synth.tokens_labels(sh["b"], sh["s"], sh["V"], seed=rank, step=i)
+            tt = torch.from_numpy(t).pin_memory()
+            ll = torch.from_numpy(l).pin_memory()
+            toks.append((tt, ll))
+        for i in range(args.warmup):
+            mt.mt_train_step(ctx, toks[i][0].data_ptr(), toks[i][1].data_ptr())
+        stream = torch.cuda.ExternalStream(mt.mt_get_stream(ctx), device=dev)
+
+        # -------- timed region: device events on the engine's compute stream --------
+        clocks = Clocks(local)
+        clocks.start()
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        stats = []
+        losses = []
+        for i in range(args.warmup, args.warmup + args.steps):
+            losses.append(mt.mt_train_step(ctx, toks[i][0].data_ptr(), toks[i][1].data_ptr()))
+            stats.append(mt.mt_get_stats(ctx))
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        clk = clocks.stop()
+        t_dev = allmax(e0.elapsed_time(e1) / 1e3)
+
+        # -------- end-to-end: host clock around the public call, host buffers --------
+        barrier()
+        torch.cuda.synchronize(dev)
+        w0 = time.perf_counter()
+        for i in range(args.warmup + args.steps, nsteps):
+            losses.append(mt.mt_train_step(ctx, toks[i][0].data_ptr(), toks[i][1].data_ptr()))
+        w1 = time.perf_counter()
+        barrier()
+        t_e2e = allmax(w1 - w0)
+    finally:
+        mt.mt_destroy(ctx)
+
+    if rank == 0:
+        P, ptype = peaks()
+        model_f, exec_f = flops_per_step(sh)
+        K = args.steps
+        value = world * T * K / t_dev
+        ms = t_dev / K * 1e3
+        g_fl = sum(s["gemm_flops"] for s in stats)
+        g_ms = sum(s["gemm_ms"] for s in stats)
+        g_n = sum(s["gemm_launches"] for s in stats)
+        a_fl = sum(s["attn_flops"] for s in stats)
+        a_ms = sum(s["attn_ms"] for s in stats)
+        achieved = g_fl / (g_ms / 1e3) / 1e12 if g_ms > 0 else None
+        peak = P["bf16_tflops_sustained"]
+        mean = lambda k: sum(s[k] for s in stats) / len(stats)  # noqa: E731
+        h2d_b, d2h_b = mean("h2d_bytes"), mean("d2h_bytes")
+        t_compute = exec_f / (peak * 1e12)
+        t_h2d = h2d_b / (link["h2d_gbs"] * 1e9)
+        t_d2h = d2h_b / (link["d2h_gbs"] * 1e9)
+        t_bound = max(t_compute, t_h2d, t_d2h)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic (uniform random tokens from seed, N(0,0.02) weights)",
+            "config": {"workload": workload_desc(args.workload, sh), "global_batch": sh["b"] * world,
+                       "seq_len": sh["s"], "parallelism": "replicas" if world > 1 else "single GPU",
+                       "l2": "no flush needed: every step streams all weights (>1 GB) through HBM from host"},
+            "model_tflops": model_f * world / (t_dev / K) / 1e12,
+            "executed_tflops": exec_f * world / (t_dev / K) / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "tcgen05 bf16 GEMM (all projections, fwd/dX/dW)",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": (achieved / peak) if achieved else None, "traffic": None,
+                         "peak_kind": f"bf16_tflops_sustained ({ptype})",
+                         "launches_per_step": g_n / K, "gemm_ms_per_step": g_ms / K},
+            "step_roofline": {"compute_ms": t_compute * 1e3, "h2d_ms": t_h2d * 1e3, "d2h_ms": t_d2h * 1e3,
+                              "bound_ms": t_bound * 1e3, "frac": t_bound / (t_dev / K),
+                              "link_measured": link, "h2d_bytes": h2d_b, "d2h_bytes": d2h_b,
+                              "attention_tflops": a_fl / (a_ms / 1e3) / 1e12 if a_ms > 0 else None,
+                              "attention_ms_per_step": a_ms / K,
+                              "gpu_step_ms": mean("step_ms"), "fwd_ms": mean("fwd_ms"), "head_ms": mean("head_ms"),
+                              "bwd_ms": mean("bwd_ms"), "wait_weights_ms": mean("wait_weights_ms"),
+                              "host_adamw_ms": mean("adamw_ms"), "host_adamw_gbs": mean("adamw_bytes") /
+                              max(mean("adamw_ms"), 1e-9) / 1e6, "host_threads": cfg.host_threads},
+            "loss": losses[-1],
+            "clocks": clk,
+            "e2e": {"value": world * T * K / t_e2e, "unit": UNIT, "h2d_bytes_per_step": 2 * T * 4,
+                    "d2h_bytes_per_step": 4, "timing": "host wall clock around mt_train_step (public C API)"},
+            "gpu_launches": int(sum(s["kernel_launches"] for s in stats)),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, secs, desc = oracle_sample_tokens_per_s(sh)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                    "sample": desc, "seconds": secs}
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
