@@ -452,3 +452,63 @@ int launch_cast_f32_bf16(const float* in, void* out, int64_t n, cudaStream_t st)
 }
 
 }  // namespace mt
+
+// ---------------------------------------------------------------------------
+// RMSNorm backward without any allocation by caller or library.
+//
+// The per-block partial sums of dg live in this fixed device array instead of
+// a caller buffer. Host code must not pass the array's name to a kernel (in
+// host code it is only a stand-in for the device symbol): the device address
+// is looked up once per device with cudaGetSymbolAddress and cached.
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+namespace mt {
+namespace {
+
+constexpr int kNoAllocScratchFloats = 1 << 20;  // 4 MiB per device that loads the library
+static __device__ __align__(256) float g_rmsnorm_scratch[kNoAllocScratchFloats];
+
+constexpr int kMaxDevices = 64;
+float* g_scratch_addr[kMaxDevices] = {};
+std::mutex g_scratch_mu;
+
+// Address of the scratch array on the current device (set up on first use).
+int scratch_address(float** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MT_ERR_CUDA;
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_rmsnorm_scratch) != cudaSuccess || !p) return MT_ERR_CUDA;
+    g_scratch_addr[dev] = static_cast<float*>(p);
+  }
+  *out = g_scratch_addr[dev];
+  return MT_OK;
+}
+
+}  // namespace
+}  // namespace mt
+
+extern "C" int mt_k_rmsnorm_bwd_noalloc(const float* x, const void* g, const float* rstd, const float* dy,
+                                        const float* dres, float* dx, void* dx_bf16, float* dg, int T, int d,
+                                        void* stream) {
+  using namespace mt;
+  if (!x || !g || !rstd || !dy || !dx || !dg || T < 0 || d <= 0 || (d % 4)) return MT_ERR_ARG;
+  if (d > 256 * 4 * RMS_KMAX) return MT_ERR_ARG;  // beyond the widest row the kernel (and scratch) supports
+  if (T == 0) return MT_OK;
+  float* part = nullptr;
+  if (scratch_address(&part) != MT_OK) return MT_ERR_CUDA;
+  // As many row blocks as the regular entry point uses, capped so that
+  // blocks x d partials fit in the fixed scratch array.
+  int nb = rmsnorm_bwd_blocks(T);
+  const int cap = kNoAllocScratchFloats / d;
+  if (nb > cap) nb = cap;
+  const int rpb = (T + nb - 1) / nb;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // Every block writes its own partial row (zeros when it owns no rows), so
+  // stale contents from an earlier call are never read.
+  k_rmsnorm_bwd<<<nb, 256, 0, st>>>(x, (const bf16*)g, rstd, dy, dres, dx, (bf16*)dx_bf16, part, T, d, rpb);
+  k_sum_rows<<<nblk(d, 256), 256, 0, st>>>(part, nb, d, dg);
+  return launch_status();
+}

@@ -69,6 +69,10 @@ _sig("mt_k_attn_bwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_vo
      c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p)
 
 
+_sig("mt_k_rmsnorm_bwd_noalloc", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+     c_void_p, c_int, c_int, c_void_p)
+
+
 def _p(x):
     return x or None
 
@@ -84,6 +88,11 @@ def mt_k_rmsnorm_bwd_partial_floats(T, d):
 def mt_k_rmsnorm_bwd(x, g, rstd, dy, dres, dx, dx_bf16, dg_part, dg, T, d, stream=0):
     return _check(lib.mt_k_rmsnorm_bwd(x, g, rstd, dy, _p(dres), dx, _p(dx_bf16), dg_part, dg, T, d, _p(stream)),
                   "mt_k_rmsnorm_bwd")
+
+
+def mt_k_rmsnorm_bwd_noalloc(x, g, rstd, dy, dres, dx, dx_bf16, dg, T, d, stream=0):
+    return _check(lib.mt_k_rmsnorm_bwd_noalloc(x, g, rstd, dy, _p(dres), dx, _p(dx_bf16), dg, T, d, _p(stream)),
+                  "mt_k_rmsnorm_bwd_noalloc")
 
 
 def mt_k_rope(buf, ld, T, s, nheads, hd, col0, cos_tab, sin_tab, sign, stream=0):

@@ -66,6 +66,26 @@ size_t mt_k_rmsnorm_bwd_partial_floats(int T, int d);
 int mt_k_rmsnorm_bwd(const float* x, const void* g, const float* rstd, const float* dy, const float* dres, float* dx,
                      void* dx_bf16, float* dg_part, float* dg, int T, int d, void* stream);
 
+/* RMSNorm backward that allocates nothing and takes no scratch buffer: the
+ * same outputs as mt_k_rmsnorm_bwd (dx, optional dx_bf16, dg) for callers that
+ * cannot call cudaMalloc at this point -- for example code whose device memory
+ * was all handed to another allocator up front, hot loops that cannot absorb
+ * the device-wide synchronisation an allocation may cause, or plugin hosts
+ * that forbid allocation after start-up. The method's pages have no
+ * counterpart: this is a convenience of this library.
+ * The partial sums live in one fixed 4 MiB device array inside the library
+ * (1M floats, held on every GPU that loads the library until the process
+ * exits); the block count is reduced when needed so that blocks x d partials
+ * fit. Limits: d <= 8192 and d % 4 == 0, else MT_ERR_ARG. The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture. Each
+ * device has its own copy of the array, and every call on that device shares
+ * it, which keeps the last call's contents: two calls whose executions overlap
+ * on the GPU (for example on two streams with no ordering between them) race
+ * on it and give wrong dg. Calls ordered on one stream are safe. */
+int mt_k_rmsnorm_bwd_noalloc(const float* x, const void* g, const float* rstd, const float* dy, const float* dres,
+                             float* dx, void* dx_bf16, float* dg, int T, int d, void* stream);
+
 /* RoPE in place on nheads bf16 heads of width hd starting at column col0 of a
  * [T, ld] buffer, token t at position t % s; rotate-half pairs (i, i+hd/2)
  * rotated by angle pos * theta_i (cos/sin tables fp32 [s, hd/2]).
