@@ -45,6 +45,7 @@ def parse():
     ap.add_argument("--workload", default="llama-1.3b", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="mt", choices=["mt", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--host-threads", type=int, default=0, help="host optimizer threads per replica (0: cores / N)")
     return ap.parse_args()
 
 
@@ -287,7 +288,7 @@ def main():
     cfg.device = local
     cfg.flags = mt.MT_FLAG_KERNEL_TIMING
     ncpu = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    cfg.host_threads = max(1, ncpu // world)
+    cfg.host_threads = args.host_threads or max(1, ncpu // world)
 
     # Host memory: every replica holds its own master, moments, gradients and bf16 copy.
     need = mt.mt_arena_bytes(cfg) + mt.mt_host_state_bytes(cfg)
@@ -393,7 +394,9 @@ def main():
                               "gpu_step_ms": mean("step_ms"), "fwd_ms": mean("fwd_ms"), "head_ms": mean("head_ms"),
                               "bwd_ms": mean("bwd_ms"), "wait_weights_ms": mean("wait_weights_ms"),
                               "host_adamw_ms": mean("adamw_ms"), "host_adamw_gbs": mean("adamw_bytes") /
-                              max(mean("adamw_ms"), 1e-9) / 1e6, "host_threads": cfg.host_threads},
+                              max(mean("adamw_ms"), 1e-9) / 1e6, "host_threads": cfg.host_threads,
+                              "host_step_ms": mean("host_step_ms"), "adamw_first_ms": mean("adamw_first_ms"),
+                              "adamw_last_ms": mean("adamw_last_ms"), "enqueue_ms": mean("enqueue_ms")},
             "loss": losses[-1],
             "clocks": clk,
             "e2e": {"value": world * T * K / t_e2e, "unit": UNIT, "h2d_bytes_per_step": 2 * T * 4,

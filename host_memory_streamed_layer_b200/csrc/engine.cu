@@ -142,6 +142,7 @@ struct mt_ctx {
   int opt_status = MT_OK;
   bool skip_updates = false;
   double adamw_s = 0, adamw_bytes = 0;
+  double call_t0 = 0, adamw_first = 0, adamw_last = 0, enqueue_s = 0;
   double wait_limit_s = 600.0;
 
   mt_stats stats{};
@@ -222,7 +223,7 @@ int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
     e1 = timing_event(c);
     if (e0) cudaEventRecord(e0, c->s_comp);
   }
-  int r = bwd ? attention_bwd(a, c->s_comp) : attention_fwd(a, c->s_comp);
+  int r = bwd ? attention_bwd(a, c->s_comp) : attention_fwd_tc(a, c->s_comp, c->d_err);
   if (r != MT_OK) return set_err(c, r, "attention launch failed");
   c->launches += bwd ? 4 : 1;
   if (timing && e0 && e1) {
@@ -423,11 +424,13 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
     for (size_t i = 0; i < sg.n; i += chunk) tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf + i});
   const int t = c->step;
   const double t0 = now_s();
+  if (c->adamw_first == 0) c->adamw_first = t0;
   c->pool->run((int)tasks.size(), [&](int i) {
     const Task& k = tasks[i];
     adamw_chunk(c->arena + k.off, c->grad + k.off, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
   });
-  c->adamw_s += now_s() - t0;
+  c->adamw_last = now_s();
+  c->adamw_s += c->adamw_last - t0;
   size_t n = 0;
   for (const Seg& sg : segs) n += sg.n;
   c->adamw_bytes += 30.0 * n;
@@ -443,18 +446,30 @@ void run_job(mt_ctx* c, const Job& j) {
     return;
   }
   if (j.kind == Job::EMBED) {
-    // Dense gradient of the embedding: zero last step's rows, scatter this step's.
+    // Dense gradient of the embedding: zero last step's rows, then scatter this
+    // step's rows (checking them for NaN/Inf), both across the worker pool.
     float* ge = c->grad + y.embed.off;
     const size_t d = s.d;
-    for (int32_t r : c->prev_uniq) memset(ge + (size_t)r * d, 0, d * sizeof(float));
-    bool bad = false;
-    for (size_t u = 0; u < c->uniq.size(); ++u) {
-      const float* src = c->emb_rows_h + u * d;
-      for (size_t k = 0; k < d; ++k) bad |= !std::isfinite(src[k]);
-      memcpy(ge + (size_t)c->uniq[u] * d, src, d * sizeof(float));
-    }
+    const int nt = c->pool->size() * 4;
+    const size_t np = c->prev_uniq.size(), nu = c->uniq.size();
+    c->pool->run(nt, [&](int i) {
+      for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k) memset(ge + (size_t)c->prev_uniq[k] * d, 0, d * 4);
+    });
+    std::vector<char> bad(nt, 0);
+    c->pool->run(nt, [&](int i) {
+      bool b = false;
+      for (size_t u = nu * i / nt; u < nu * (i + 1) / nt; ++u) {
+        const float* src = c->emb_rows_h + u * d;
+        float acc = 0.f;
+        for (size_t k = 0; k < d; ++k) acc += src[k] * 0.f;  // NaN or Inf anywhere makes acc NaN
+        b |= !(acc == 0.f);
+        memcpy(ge + (size_t)c->uniq[u] * d, src, d * sizeof(float));
+      }
+      bad[i] = b;
+    });
     c->prev_uniq = c->uniq;
-    if (bad) c->flags_h[j.flag_index] = 1;
+    for (char b : bad)
+      if (b) c->flags_h[j.flag_index] = 1;
   }
   if (c->flags_h[j.flag_index] != 0) {
     if (c->opt_status == MT_OK) {
@@ -1028,6 +1043,8 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   offs[n_unique] = acc;
   for (int t = 0; t < T; ++t) pos[start[tokens[t]]++] = t;  // increasing t within each token
 
+  c->call_t0 = now_s();
+  c->adamw_first = c->adamw_last = 0;
   c->step++;
   c->opt_status = MT_OK;
   c->skip_updates = false;
@@ -1036,7 +1053,9 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   c->timed.clear();
   c->launches = 0;
   c->err.clear();
+  const double te0 = now_s();
   int r = enqueue_step(c, n_unique);
+  c->enqueue_s = now_s() - te0;
   if (r != MT_OK) {
     // Let the optimizer finish the jobs already queued and the streams drain.
     c->skip_updates = true;
@@ -1057,6 +1076,10 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   }
   *loss_out = c->misc_h[0] / (float)T;
   collect_stats(c);
+  c->stats.host_step_ms = (now_s() - c->call_t0) * 1e3;
+  c->stats.enqueue_ms = c->enqueue_s * 1e3;
+  c->stats.adamw_first_ms = c->adamw_first > 0 ? (c->adamw_first - c->call_t0) * 1e3 : 0;
+  c->stats.adamw_last_ms = c->adamw_last > 0 ? (c->adamw_last - c->call_t0) * 1e3 : 0;
   if (c->opt_status != MT_OK) return c->opt_status;
   return MT_OK;
 }

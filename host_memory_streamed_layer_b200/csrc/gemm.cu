@@ -333,9 +333,12 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+}  // namespace
+
 // 2-D bf16 tensor map: inner extent `inner` (contiguous), outer extent `outer`,
 // row pitch `ld` elements, box {64, box_outer}, 128-byte swizzle, zero fill.
-bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld, int box_outer) {
+bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                             int box_outer) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
@@ -347,6 +350,8 @@ bool make_map(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, in
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+namespace {
 
 int g_num_sms = 0;
 
@@ -361,8 +366,10 @@ int launch(const GemmDesc& g, cudaStream_t st, int* err) {
     attr_set = true;
   }
   CUtensorMap ta, tb;
-  bool ok = A_MN ? make_map(&ta, g.A, g.M, g.K, g.lda, 64) : make_map(&ta, g.A, g.K, g.M, g.lda, BM);
-  ok = ok && (B_MN ? make_map(&tb, g.B, g.N, g.K, g.ldb, 64) : make_map(&tb, g.B, g.K, g.N, g.ldb, BN));
+  bool ok = A_MN ? make_tensor_map_2d_bf16(&ta, g.A, g.M, g.K, g.lda, 64)
+              : make_tensor_map_2d_bf16(&ta, g.A, g.K, g.M, g.lda, BM);
+  ok = ok && (B_MN ? make_tensor_map_2d_bf16(&tb, g.B, g.N, g.K, g.ldb, 64)
+                    : make_tensor_map_2d_bf16(&tb, g.B, g.K, g.N, g.ldb, BN));
   if (!ok) return MT_ERR_ARG;
   Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err};
   const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);

@@ -46,9 +46,12 @@ __attribute__((target("avx512f,avx512bw"))) inline __m256i bf16x16_rne(__m512 x)
   return _mm512_cvtepi32_epi16(r);
 }
 
+// The bf16 copy is only written (the next step's H2D reads it), so it is
+// stored with non-temporal stores when 32-byte aligned: no read-for-ownership.
 __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const float* g, float* m, float* v,
                                                               uint16_t* pb, size_t n, float decay, float b1, float b2,
                                                               float step, float inv_sqrt_bc2, float eps) {
+  const bool nt = pb && ((reinterpret_cast<uintptr_t>(pb) & 31) == 0);
   const __m512 vb1 = _mm512_set1_ps(b1), vc1 = _mm512_set1_ps(1.f - b1);
   const __m512 vb2 = _mm512_set1_ps(b2), vc2 = _mm512_set1_ps(1.f - b2);
   const __m512 vdec = _mm512_set1_ps(decay), vstep = _mm512_set1_ps(step);
@@ -64,8 +67,12 @@ __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const fl
     _mm512_storeu_ps(m + i, mi);
     _mm512_storeu_ps(v + i, vi);
     _mm512_storeu_ps(p + i, pi);
-    if (pb) _mm256_storeu_si256(reinterpret_cast<__m256i*>(pb + i), bf16x16_rne(pi));
+    if (nt)
+      _mm256_stream_si256(reinterpret_cast<__m256i*>(pb + i), bf16x16_rne(pi));
+    else if (pb)
+      _mm256_storeu_si256(reinterpret_cast<__m256i*>(pb + i), bf16x16_rne(pi));
   }
+  if (nt) _mm_sfence();
   if (i < n) adamw_scalar(p + i, g + i, m + i, v + i, pb ? pb + i : nullptr, n - i, decay, b1, b2, step, inv_sqrt_bc2, eps);
 }
 

@@ -99,3 +99,14 @@ extern "C" int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_
   a.lddkv = lddkv; a.b = b; a.s = s; a.H = H; a.Hkv = Hkv; a.hd = hd; a.scale = 1.0f / std::sqrt((float)hd);
   return mt::attention_bwd(a, S(stream));
 }
+
+extern "C" int mt_k_attn_fwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv, void* o, int64_t ldo,
+                                float* lse, int b, int s, int H, int Hkv, int hd, void* stream, int32_t* dev_err) {
+  if (!q || !k || !v || !o || !lse || b < 0 || s < 0 || H <= 0 || Hkv <= 0 || (H % Hkv)) return MT_ERR_ARG;
+  if (hd != 64 && hd != 128) return MT_ERR_CONFIG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || (ldqkv % 8) || (ldo % 8)) return MT_ERR_ARG;
+  mt::AttnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.ldqkv = ldqkv; a.o = o; a.ldo = ldo; a.lse = lse;
+  a.b = b; a.s = s; a.H = H; a.Hkv = Hkv; a.hd = hd; a.scale = 1.0f / std::sqrt((float)hd);
+  return mt::attention_fwd_tc(a, S(stream), dev_err);
+}

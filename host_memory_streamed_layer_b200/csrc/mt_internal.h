@@ -1,6 +1,7 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,6 +36,11 @@ struct GemmDesc {
 
 int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
 
+// 2-D bf16 TMA map: inner (contiguous) extent, outer extent, row pitch ld
+// (elements), box {64, box_outer}, 128-byte swizzle, zero fill out of bounds.
+bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                             int box_outer);
+
 // Causal attention with grouped KV heads. q, k, v: column ranges of one bf16
 // row per token (pitch ldqkv); o, dout: [T, H*hd] bf16 (pitch ldo); lse, dvec:
 // fp32 [b, H, s]; dq_acc: fp32 [T, ldqa] accumulator (zeroed by the call);
@@ -61,6 +67,8 @@ struct AttnArgs {
 };
 int attention_fwd(const AttnArgs& a, cudaStream_t st);
 int attention_bwd(const AttnArgs& a, cudaStream_t st);
+// Forward on the tcgen05 tensor cores (same outputs as attention_fwd).
+int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
 
 int launch_rmsnorm_fwd(const float* x, const void* g, void* y, float* rstd, int T, int d, float eps, cudaStream_t st);
 int rmsnorm_bwd_blocks(int T);

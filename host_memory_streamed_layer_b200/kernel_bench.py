@@ -1,0 +1,136 @@
+"""Micro-benchmark of single hot-path kernels through the C ABI.
+
+    python -m host_memory_streamed_layer_b200.kernel_bench gemm [--shape NAME] [--iters N]
+    python -m host_memory_streamed_layer_b200.kernel_bench attn [--fwd-only] [--iters N]
+    python -m host_memory_streamed_layer_b200.kernel_bench rmsnorm_bwd [--iters N]
+
+Times each launch with CUDA events on the launching stream after warm-up and
+prints achieved TFLOP/s (tensor-bound kernels) or GB/s of algorithmic bytes
+(memory-bound kernels). With --iters 1 --warmup 0 it launches exactly once,
+which is what an ncu capture of one launch wants. Shapes are those of the
+llama-1.3b workload (T = 8 x 2048 tokens, d 2048, FFN 5504, 16 heads).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+
+import torch
+
+from . import mt
+
+T, D, F, V, H, HD, B, S = 16384, 2048, 5504, 32000, 16, 128, 8, 2048
+GEMMS = {  # name: (M, N, K, form)
+    "qkv_fwd": (T, 3 * D, D, "fwd"), "o_fwd": (T, D, D, "fwd"), "gu_fwd": (T, 2 * F, D, "fwd"),
+    "down_fwd": (T, D, F, "fwd"), "down_dx": (T, F, D, "dx"), "gu_dx": (T, D, 2 * F, "dx"),
+    "qkv_dx": (T, D, 3 * D, "dx"), "o_dx": (T, D, D, "dx"), "down_dw": (D, F, T, "dw"), "gu_dw": (2 * F, D, T, "dw"),
+    "qkv_dw": (3 * D, D, T, "dw"), "o_dw": (D, D, T, "dw"), "head_fwd": (T, V, D, "fwd"),
+}
+
+
+def timed(fn, iters, warmup):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    if iters == 0:
+        return 0.0
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters / 1e3
+
+
+def bench_gemm(names, iters, warmup):
+    st = torch.cuda.current_stream().cuda_stream
+    out = []
+    for name in names:
+        M, N, K, form = GEMMS[name]
+        A = torch.randn(M * K, device="cuda").to(torch.bfloat16)
+        Bm = torch.randn(N * K, device="cuda").to(torch.bfloat16)
+        C = torch.empty(M * N, device="cuda", dtype=torch.float32 if form == "dw" else torch.bfloat16)
+        if form == "fwd":
+            a = (A.data_ptr(), K, 0, Bm.data_ptr(), K, 0)
+        elif form == "dx":
+            a = (A.data_ptr(), K, 0, Bm.data_ptr(), N, 1)
+        else:
+            a = (A.data_ptr(), M, 1, Bm.data_ptr(), N, 1)
+        kind = mt.GEMM_OUT_F32 if form == "dw" else mt.GEMM_OUT_BF16
+        sec = timed(lambda: mt.mt_k_gemm_bf16(*a, C.data_ptr(), N, kind, 0, 0, M, N, K, st, 0), iters, warmup)
+        fl = 2.0 * M * N * K
+        out.append({"kernel": "gemm", "shape": name, "M": M, "N": N, "K": K, "us": sec * 1e6,
+                    "tflops": fl / sec / 1e12 if sec else None})
+    return out
+
+
+def bench_attn(iters, warmup, fwd_only, impl="tc"):
+    st = torch.cuda.current_stream().cuda_stream
+    ld = 3 * H * HD
+    qkv = torch.randn(T, ld, device="cuda").to(torch.bfloat16)
+    o = torch.empty(T, H * HD, device="cuda", dtype=torch.bfloat16)
+    lse = torch.empty(B, H, S, device="cuda")
+    p = qkv.data_ptr()
+    pk, pv = p + 2 * H * HD, p + 4 * H * HD
+    if impl == "tc":
+        fwd = lambda: mt.mt_k_attn_fwd_tc(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, H, HD,  # noqa
+                                          st)
+    else:
+        fwd = lambda: mt.mt_k_attn_fwd(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, H, HD, st)  # noqa
+    fl = 2.0 * B * H * S * S * HD
+    res = [{"kernel": f"attn_fwd_{impl}", "us": 0, "tflops": None}]
+    sec = timed(fwd, iters, warmup)
+    res[0].update(us=sec * 1e6, tflops=fl / sec / 1e12 if sec else None)
+    if not fwd_only:
+        fwd()
+        do = torch.randn(T, H * HD, device="cuda").to(torch.bfloat16)
+        dvec = torch.empty(B, H, S, device="cuda")
+        dqa = torch.empty(T, H * HD, device="cuda")
+        dqkv = torch.empty(T, ld, device="cuda", dtype=torch.bfloat16)
+        dp = dqkv.data_ptr()
+        bwd = lambda: mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(),  # noqa
+                                       dvec.data_ptr(), dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD,
+                                       dp + 4 * H * HD, ld, B, S, H, H, HD, st)
+        sec = timed(bwd, iters, warmup)
+        res.append({"kernel": "attn_bwd", "us": sec * 1e6, "tflops": 2.5 * fl / sec / 1e12 if sec else None})
+    return res
+
+
+def bench_rmsnorm_bwd(iters, warmup):
+    st = torch.cuda.current_stream().cuda_stream
+    x, dy, dres, dx = (torch.randn(T, D, device="cuda") for _ in range(4))
+    g = torch.ones(D, device="cuda", dtype=torch.bfloat16)
+    r = torch.ones(T, device="cuda")
+    dxb = torch.empty(T, D, device="cuda", dtype=torch.bfloat16)
+    part = torch.empty(mt.mt_k_rmsnorm_bwd_partial_floats(T, D), device="cuda")
+    dg = torch.empty(D, device="cuda")
+    sec = timed(lambda: mt.mt_k_rmsnorm_bwd(x.data_ptr(), g.data_ptr(), r.data_ptr(), dy.data_ptr(), dres.data_ptr(),
+                                            dx.data_ptr(), dxb.data_ptr(), part.data_ptr(), dg.data_ptr(), T, D, st),
+                iters, warmup)
+    byt = 18.0 * T * D
+    return [{"kernel": "rmsnorm_bwd", "us": sec * 1e6, "gbs": byt / sec / 1e9 if sec else None}]
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kernel", choices=["gemm", "attn", "rmsnorm_bwd"])
+    ap.add_argument("--shape", default="all")
+    ap.add_argument("--iters", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--fwd-only", action="store_true")
+    ap.add_argument("--impl", default="tc", choices=["tc", "mma"])
+    a = ap.parse_args()
+    if a.kernel == "gemm":
+        names = list(GEMMS) if a.shape == "all" else a.shape.split(",")
+        res = bench_gemm(names, a.iters, a.warmup)
+    elif a.kernel == "attn":
+        res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl)
+    else:
+        res = bench_rmsnorm_bwd(a.iters, a.warmup)
+    for r in res:
+        print(json.dumps(r))
+
+
+if __name__ == "__main__":
+    main()

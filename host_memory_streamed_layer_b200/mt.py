@@ -65,6 +65,8 @@ _sig("mt_k_embed_bwd", c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_i
 _sig("mt_k_softmax_ce", c_int, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_int, c_int, c_float, c_void_p)
 _sig("mt_k_attn_fwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_int, c_int, c_int,
      c_int, c_int, c_void_p)
+_sig("mt_k_attn_fwd_tc", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_int, c_int,
+     c_int, c_int, c_int, c_void_p, c_void_p)
 _sig("mt_k_attn_bwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_void_p,
      c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p)
 
@@ -124,6 +126,11 @@ def mt_k_attn_fwd(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, stream=0):
     return _check(lib.mt_k_attn_fwd(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, _p(stream)), "mt_k_attn_fwd")
 
 
+def mt_k_attn_fwd_tc(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, stream=0, dev_err=0):
+    return _check(lib.mt_k_attn_fwd_tc(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, _p(stream), _p(dev_err)),
+                  "mt_k_attn_fwd_tc")
+
+
 def mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv, b, s, H, Hkv, hd,
                   stream=0):
     return _check(lib.mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv,
@@ -153,7 +160,8 @@ class mt_stats(ctypes.Structure):
         "step_ms", "fwd_ms", "head_ms", "bwd_ms", "h2d_bytes", "d2h_bytes", "h2d_ms", "d2h_ms",
         "wait_weights_ms", "adamw_ms", "adamw_bytes", "gemm_flops", "gemm_ms")] + \
         [("gemm_launches", ctypes.c_int64), ("attn_flops", ctypes.c_double), ("attn_ms", ctypes.c_double),
-         ("attn_launches", ctypes.c_int64), ("kernel_launches", ctypes.c_int64)]
+         ("attn_launches", ctypes.c_int64), ("kernel_launches", ctypes.c_int64), ("host_step_ms", ctypes.c_double),
+         ("adamw_first_ms", ctypes.c_double), ("adamw_last_ms", ctypes.c_double), ("enqueue_ms", ctypes.c_double)]
 
     def as_dict(self):
         return {n: getattr(self, n) for n, _ in self._fields_}

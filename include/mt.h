@@ -93,6 +93,10 @@ typedef struct mt_stats {
   double gemm_flops, gemm_ms; int64_t gemm_launches;  /* with MT_FLAG_KERNEL_TIMING */
   double attn_flops, attn_ms; int64_t attn_launches;
   int64_t kernel_launches;  /* kernels this library launched during the step */
+  double host_step_ms;      /* wall time of mt_train_step */
+  double adamw_first_ms;    /* host optimizer's first update began, ms after the call started */
+  double adamw_last_ms;     /* host optimizer's last update ended, ms after the call started */
+  double enqueue_ms;        /* host time spent enqueueing the step's GPU work */
 } mt_stats;
 
 /* Fills *cfg with the defaults (struct_size set, hyper-parameters of the

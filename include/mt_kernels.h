@@ -122,6 +122,13 @@ int mt_k_softmax_ce(const float* z, int64_t ldz, const int32_t* labels, void* dz
 int mt_k_attn_fwd(const void* q, const void* k, const void* v, int64_t ldqkv, void* o, int64_t ldo, float* lse,
                   int b, int s, int H, int Hkv, int hd, void* stream);
 
+/* The same causal attention forward (same arguments, outputs and layout) on the
+ * tcgen05 tensor cores: 128-query x 128-key tiles, S and P V in tensor memory,
+ * TMA loads. Additionally needs q, k, v and o 16-byte aligned. dev_err:
+ * optional device int32 set when a bounded wait inside the kernel runs out. */
+int mt_k_attn_fwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv, void* o, int64_t ldo, float* lse,
+                     int b, int s, int H, int Hkv, int hd, void* stream, int32_t* dev_err);
+
 /* Causal attention backward from o, lse and dout (bf16, pitch ldo):
  * dvec fp32 [b,H,s] and dq_acc fp32 [b*s, ldqa] are caller scratch (dq_acc is
  * zeroed by the call); dq (pitch lddq), dk and dv (pitch lddkv) are bf16

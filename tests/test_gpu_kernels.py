@@ -178,7 +178,8 @@ def test_softmax_ce(T, V):
     assert np.all(np.abs(np64(dz) - ref) <= 2 ** -8 * np.abs(ref) + 1e-7 * scale)
 
 
-ATTN = [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 8, 1, 200, 1), (64, 2, 2, 1, 2), (128, 4, 4, 64, 1)]
+ATTN = [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 8, 1, 200, 1), (64, 2, 2, 1, 2), (128, 4, 4, 64, 1),
+        (128, 2, 2, 384, 2), (64, 4, 1, 300, 2)]
 
 
 def _attn_inputs(hd, H, Hkv, s, b, seed):
@@ -193,17 +194,24 @@ def _attn_inputs(hd, H, Hkv, s, b, seed):
     return qkv, q, k, v, ld
 
 
+@pytest.mark.parametrize("impl", ["mma", "tc"])
 @pytest.mark.parametrize("hd,H,Hkv,s,b", ATTN)
-def test_attention_fwd(hd, H, Hkv, s, b):
+def test_attention_fwd(hd, H, Hkv, s, b, impl):
     mt = _mt()
     qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, hd + s)
     T = b * s
     o = torch.empty(T, H * hd, dtype=torch.bfloat16, device=DEV)
     lse = torch.empty(b, H, s, device=DEV)
     p = qkv.data_ptr()
-    mt.mt_k_attn_fwd(p, p + 2 * H * hd, p + 2 * (H + Hkv) * hd, ld, o.data_ptr(), H * hd, lse.data_ptr(),
-                     b, s, H, Hkv, hd)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    if impl == "mma":
+        mt.mt_k_attn_fwd(p, p + 2 * H * hd, p + 2 * (H + Hkv) * hd, ld, o.data_ptr(), H * hd, lse.data_ptr(),
+                         b, s, H, Hkv, hd)
+    else:
+        mt.mt_k_attn_fwd_tc(p, p + 2 * H * hd, p + 2 * (H + Hkv) * hd, ld, o.data_ptr(), H * hd, lse.data_ptr(),
+                            b, s, H, Hkv, hd, 0, err.data_ptr())
     sync()
+    assert err.item() == 0
     ro, _ = oracle.attention_fwd(q, k, v)
     got = np64(o).reshape(b, s, H, hd)
     assert rel_l2(got, ro) < 4e-3
