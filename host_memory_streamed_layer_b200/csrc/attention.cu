@@ -258,7 +258,8 @@ __global__ void __launch_bounds__(128) k_flash_bwd(const bf16* __restrict__ Q, c
                                                    const float* __restrict__ LSE, const float* __restrict__ Dv,
                                                    float* __restrict__ dQacc, int64_t ldqa, bf16* __restrict__ dK,
                                                    bf16* __restrict__ dV, int64_t lddkv, int s, int H, int Hkv,
-                                                   float scale) {
+                                                   float scale, const float* __restrict__ rcos,
+                                                   const float* __restrict__ rsin) {
   constexpr int BKV = 64, BQ = 32;
   extern __shared__ __align__(128) uint8_t smraw[];
   bf16* sK = reinterpret_cast<bf16*>(smraw);
@@ -451,28 +452,65 @@ __global__ void __launch_bounds__(128) k_flash_bwd(const bf16* __restrict__ Q, c
     if (kj < s) {
       bf16* kr = dK + (tb + kj) * lddkv + kvh * HD + 2 * tq;
       bf16* vr = dV + (tb + kj) * lddkv + kvh * HD + 2 * tq;
+      if (rcos) {
+        // gradient w.r.t. k before RoPE: transposed rotation of the pair
+        // (i, i + HD/2); this thread holds both, in n-tiles n and n + HD/16.
+        const float* cs = rcos + (int64_t)kj * (HD / 2);
+        const float* sn = rsin + (int64_t)kj * (HD / 2);
 #pragma unroll
-      for (int n = 0; n < HD / 8; ++n) {
-        *reinterpret_cast<uint32_t*>(kr + n * 8) = pack_bf16x2(dk[n][2 * r] * scale, dk[n][2 * r + 1] * scale);
-        *reinterpret_cast<uint32_t*>(vr + n * 8) = pack_bf16x2(dv[n][2 * r], dv[n][2 * r + 1]);
+        for (int n = 0; n < HD / 16; ++n) {
+          const int i0 = n * 8 + 2 * tq;
+          float a[2], bb[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float x1 = dk[n][2 * r + e] * scale, x2 = dk[n + HD / 16][2 * r + e] * scale;
+            a[e] = x1 * cs[i0 + e] + x2 * sn[i0 + e];
+            bb[e] = x2 * cs[i0 + e] - x1 * sn[i0 + e];
+          }
+          *reinterpret_cast<uint32_t*>(kr + n * 8) = pack_bf16x2(a[0], a[1]);
+          *reinterpret_cast<uint32_t*>(kr + (n + HD / 16) * 8) = pack_bf16x2(bb[0], bb[1]);
+        }
+      } else {
+#pragma unroll
+        for (int n = 0; n < HD / 8; ++n)
+          *reinterpret_cast<uint32_t*>(kr + n * 8) = pack_bf16x2(dk[n][2 * r] * scale, dk[n][2 * r + 1] * scale);
       }
+#pragma unroll
+      for (int n = 0; n < HD / 8; ++n)
+        *reinterpret_cast<uint32_t*>(vr + n * 8) = pack_bf16x2(dv[n][2 * r], dv[n][2 * r + 1]);
     }
   }
 }
 
-// dQ (fp32 [T, H*hd], pitch ldqa) -> bf16 columns of dqkv (pitch ld).
+// dQ (fp32 [T, H*hd], pitch ldqa) -> bf16 columns of dqkv (pitch ld). With
+// RoPE tables the transposed rotation is applied on the way (pairs (i, i+hd/2)
+// of each head at position t % s). Thread = 4 consecutive pairs.
 __global__ void k_dq_cast(const float* __restrict__ dq, int64_t ldqa, bf16* __restrict__ out, int64_t ld, int T,
-                          int w) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // 4 elements each
-  const int w4 = w >> 2;
-  if (i >= (int64_t)T * w4) return;
-  const int64_t t = i / w4;
-  const int c = (int)(i % w4) * 4;
-  const float4 v = *reinterpret_cast<const float4*>(dq + t * ldqa + c);
-  uint2 u;
-  u.x = pack_bf16x2(v.x, v.y);
-  u.y = pack_bf16x2(v.z, v.w);
-  *reinterpret_cast<uint2*>(out + t * ld + c) = u;
+                          int H, int hd, int s, const float* __restrict__ rcos, const float* __restrict__ rsin) {
+  const int half = hd >> 1;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int per_row = H * (half >> 2);
+  if (i >= (int64_t)T * per_row) return;
+  const int64_t t = i / per_row;
+  const int k = (int)(i % per_row);
+  const int h = k / (half >> 2);
+  const int c = (k % (half >> 2)) * 4;  // pair index 0..half-1
+  const float* src = dq + t * ldqa + h * hd;
+  float4 a = *reinterpret_cast<const float4*>(src + c);
+  float4 b = *reinterpret_cast<const float4*>(src + c + half);
+  if (rcos) {
+    const int pos = (int)(t % s);
+    const float4 cs = *reinterpret_cast<const float4*>(rcos + (int64_t)pos * half + c);
+    const float4 sn = *reinterpret_cast<const float4*>(rsin + (int64_t)pos * half + c);
+    const float4 a0 = a, b0 = b;
+    a = make_float4(a0.x * cs.x + b0.x * sn.x, a0.y * cs.y + b0.y * sn.y, a0.z * cs.z + b0.z * sn.z,
+                    a0.w * cs.w + b0.w * sn.w);
+    b = make_float4(b0.x * cs.x - a0.x * sn.x, b0.y * cs.y - a0.y * sn.y, b0.z * cs.z - a0.z * sn.z,
+                    b0.w * cs.w - a0.w * sn.w);
+  }
+  bf16* o = out + t * ld + h * hd;
+  *reinterpret_cast<uint2*>(o + c) = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  *reinterpret_cast<uint2*>(o + c + half) = make_uint2(pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
 }
 
 template <int HD>
@@ -507,10 +545,11 @@ int bwd_impl(const AttnArgs& a, cudaStream_t st) {
   dim3 grid((a.s + 63) / 64, a.Hkv, a.b);
   k_flash_bwd<HD><<<grid, 128, SMEM, st>>>((const bf16*)a.q, (const bf16*)a.k, (const bf16*)a.v, a.ldqkv,
                                            (const bf16*)a.dout, a.ldo, a.lse, a.dvec, a.dq_acc, a.ldqa,
-                                           (bf16*)a.dk, (bf16*)a.dv, a.lddkv, a.s, a.H, a.Hkv, a.scale);
-  const int w = a.H * HD;
-  const int64_t n4 = (int64_t)T * (w / 4);
-  k_dq_cast<<<(int)((n4 + 255) / 256), 256, 0, st>>>(a.dq_acc, a.ldqa, (bf16*)a.dq, a.lddq, T, w);
+                                           (bf16*)a.dk, (bf16*)a.dv, a.lddkv, a.s, a.H, a.Hkv, a.scale, a.rope_cos,
+                                           a.rope_sin);
+  const int64_t nthr = (int64_t)T * a.H * (HD / 8);
+  k_dq_cast<<<(int)((nthr + 255) / 256), 256, 0, st>>>(a.dq_acc, a.ldqa, (bf16*)a.dq, a.lddq, T, a.H, HD, a.s,
+                                                       a.rope_cos, a.rope_sin);
   return launch_status();
 }
 

@@ -204,15 +204,16 @@ int gemm(mt_ctx* c, const GemmDesc& g) {
 
 GemmDesc gd_fwd(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, int epi,
                 const float* R, int M, int N, int K) {
-  return GemmDesc{A, lda, false, B, ldb, false, C, ldc, epi, R, ldc, M, N, K};
+  return GemmDesc{A, lda, false, B, ldb, false, C, ldc, epi, R, ldc, M, N, K, RopeDesc{}};
 }
 GemmDesc gd_dx(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, int epi, int M, int N,
                int K) {
-  return GemmDesc{A, lda, false, B, ldb, true, C, ldc, epi, nullptr, 0, M, N, K};
+  return GemmDesc{A, lda, false, B, ldb, true, C, ldc, epi, nullptr, 0, M, N, K, RopeDesc{}};
 }
 GemmDesc gd_dw(const void* A, int64_t lda, const void* B, int64_t ldb, float* C, int64_t ldc, int epi, int M, int N,
                int K) {
-  return GemmDesc{A, lda, true, B, ldb, true, C, ldc, epi, epi == EPI_F32_ADD ? C : nullptr, ldc, M, N, K};
+  return GemmDesc{A, lda, true, B, ldb, true, C, ldc, epi, epi == EPI_F32_ADD ? C : nullptr, ldc, M, N, K,
+                  RopeDesc{}};
 }
 
 int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
@@ -277,9 +278,12 @@ int layer_fwd(mt_ctx* c, int l, int slot, bool keep_out) {
   const float* x = c->xb + (size_t)l * s.T * s.d;
   cudaStream_t st = c->s_comp;
   KL(launch_rmsnorm_fwd(x, W + y.bf_g1, c->u_b, c->r1, s.T, s.d, c->cfg.norm_eps, st), 1);
-  CKM(gemm(c, gd_fwd(c->u_b, s.d, W + y.bf_qkv, s.d, c->qkv_b, s.Nqkv, EPI_BF16, nullptr, s.T, s.Nqkv, s.d)));
-  KL(launch_rope(c->qkv_b, s.Nqkv, s.T, s.s, s.H, s.hd, 0, c->d_cos, c->d_sin, 1.f, st), 1);
-  KL(launch_rope(c->qkv_b, s.Nqkv, s.T, s.s, s.Hkv, s.hd, s.Hd, c->d_cos, c->d_sin, 1.f, st), 1);
+  {
+    // q, k, v projection with RoPE on the q and k heads in the epilogue
+    GemmDesc g = gd_fwd(c->u_b, s.d, W + y.bf_qkv, s.d, c->qkv_b, s.Nqkv, EPI_BF16_ROPE, nullptr, s.T, s.Nqkv, s.d);
+    g.rope = RopeDesc{c->d_cos, c->d_sin, s.Hd + s.Hkv * s.hd, s.hd, s.s};
+    CKM(gemm(c, g));
+  }
   AttnArgs a{};
   a.q = c->qkv_b;
   a.k = c->qkv_b + s.Hd;
@@ -356,9 +360,9 @@ int layer_bwd(mt_ctx* c, int l, int slot, float* gs, const float* gin, float* go
   a.Hkv = s.Hkv;
   a.hd = s.hd;
   a.scale = 1.0f / sqrtf((float)s.hd);
+  a.rope_cos = c->d_cos;  // dq, dk come back with respect to the pre-RoPE projections
+  a.rope_sin = c->d_sin;
   CKM(attn(c, a, true));
-  KL(launch_rope(c->dqkv_b, s.Nqkv, T, s.s, s.H, s.hd, 0, c->d_cos, c->d_sin, -1.f, st), 1);
-  KL(launch_rope(c->dqkv_b, s.Nqkv, T, s.s, s.Hkv, s.hd, s.Hd, c->d_cos, c->d_sin, -1.f, st), 1);
   // q/k/v projections
   CKM(gemm(c, gd_dw(c->dqkv_b, s.Nqkv, c->u_b, d, G(MT_T_WQ), d, EPI_F32, s.Nqkv, d, T)));
   CKM(gemm(c, gd_dx(c->dqkv_b, s.Nqkv, W + y.bf_qkv, d, c->tmp_f, d, EPI_F32, T, d, s.Nqkv)));

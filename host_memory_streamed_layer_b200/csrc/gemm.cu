@@ -55,6 +55,7 @@ struct Params {
   int64_t ldr;
   int epi;
   int* err;
+  RopeDesc rope;
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
@@ -243,10 +244,55 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tile_coords(tile, num_m, num_n, mb, nb);
       const int row = mb * BM + quarter * 32 + lane;
       const bool row_ok = row < p.M;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      if (p.epi == EPI_BF16_ROPE) {
+        // Heads of width hd tile BN exactly; rotate-half pairs live in 32-column
+        // chunks a and a + hd/64 of the same head.
+        const int hd = p.rope.hd;
+        const int pos = row_ok ? row % p.rope.seq : 0;
+        const float* cs = p.rope.cos + (int64_t)pos * (hd >> 1);
+        const float* sn = p.rope.sin + (int64_t)pos * (hd >> 1);
+#pragma unroll 1
+        for (int h0 = 0; h0 < BN; h0 += hd) {
+#pragma unroll 1
+          for (int a = 0; a < hd / 64; ++a) {
+            uint32_t x1[32], x2[32];
+            tmem_ld_32x32b_x32(tbase + h0 + a * 32, x1);
+            tmem_ld_32x32b_x32(tbase + h0 + a * 32 + hd / 2, x2);
+            tmem_ld_wait();
+            const int c1 = nb * BN + h0 + a * 32;
+            const int c2 = c1 + hd / 2;
+            if (!row_ok || c2 >= p.N) continue;  // N is a multiple of hd: the pair is whole or absent
+            __nv_bfloat16* o1 = reinterpret_cast<__nv_bfloat16*>(p.C) + (int64_t)row * p.ldc + c1;
+            __nv_bfloat16* o2 = o1 + hd / 2;
+            const bool rot = c1 < p.rope.cols;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              float y1[8], y2[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float a1 = __uint_as_float(x1[8 * j + e]), a2 = __uint_as_float(x2[8 * j + e]);
+                if (rot) {
+                  const float cv = cs[a * 32 + 8 * j + e], sv = sn[a * 32 + 8 * j + e];
+                  y1[e] = a1 * cv - a2 * sv;
+                  y2[e] = a2 * cv + a1 * sv;
+                } else {
+                  y1[e] = a1;
+                  y2[e] = a2;
+                }
+              }
+              reinterpret_cast<uint4*>(o1)[j] = make_uint4(pack_bf16x2(y1[0], y1[1]), pack_bf16x2(y1[2], y1[3]),
+                                                           pack_bf16x2(y1[4], y1[5]), pack_bf16x2(y1[6], y1[7]));
+              reinterpret_cast<uint4*>(o2)[j] = make_uint4(pack_bf16x2(y2[0], y2[1]), pack_bf16x2(y2[2], y2[3]),
+                                                           pack_bf16x2(y2[4], y2[5]), pack_bf16x2(y2[6], y2[7]));
+            }
+          }
+        }
+      } else {
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN + c * 32, r);
+        tmem_ld_32x32b_x32(tbase + c * 32, r);
         tmem_ld_wait();
         const int col0 = nb * BN + c * 32;
         if (!row_ok || col0 >= p.N) continue;
@@ -294,6 +340,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               if (j < nv) out[j] = __uint_as_float(r[j]) + (res ? res[j] : 0.f);
           }
         }
+      }
       }
       tc_fence_before();
       __syncwarp();
@@ -371,7 +418,7 @@ int launch(const GemmDesc& g, cudaStream_t st, int* err) {
   ok = ok && (B_MN ? make_tensor_map_2d_bf16(&tb, g.B, g.N, g.K, g.ldb, 64)
                     : make_tensor_map_2d_bf16(&tb, g.B, g.K, g.N, g.ldb, BN));
   if (!ok) return MT_ERR_ARG;
-  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err};
+  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err, g.rope};
   const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
   const int grid = tiles < g_num_sms ? tiles : g_num_sms;
   k_gemm_bf16<BN, A_MN, B_MN><<<grid, NUM_THREADS, C::SMEM, st>>>(ta, tb, p);
@@ -392,6 +439,10 @@ int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* err) {
   if (g.M <= 0 || g.N <= 0 || g.K <= 0) return (g.M == 0 || g.N == 0) ? MT_OK : MT_ERR_ARG;
   if (!g.A || !g.B || !g.C) return MT_ERR_ARG;
   if (g.epi == EPI_F32_ADD && !g.R) return MT_ERR_ARG;
+  if (g.epi == EPI_BF16_ROPE) {
+    const RopeDesc& r = g.rope;
+    if (!r.cos || !r.sin || (r.hd != 64 && r.hd != 128) || r.seq <= 0 || (g.N % r.hd) || r.cols < 0) return MT_ERR_ARG;
+  }
   // TMA: 16-byte aligned base and row pitch; 16-byte aligned epilogue stores.
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(g.A) || !al16(g.B) || !al16(g.C) || (g.R && !al16(g.R))) return MT_ERR_ARG;

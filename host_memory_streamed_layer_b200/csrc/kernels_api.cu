@@ -7,7 +7,7 @@ extern "C" int mt_k_gemm_bf16(const void* A, int64_t lda, int a_mn_major, const 
                               int M, int N, int K, void* stream, int32_t* dev_err) {
   if (out_kind < MT_GEMM_OUT_BF16 || out_kind > MT_GEMM_OUT_F32_ADD) return MT_ERR_ARG;
   if (M < 0 || N < 0 || K < 0) return MT_ERR_ARG;
-  mt::GemmDesc g{A, lda, a_mn_major != 0, B, ldb, b_mn_major != 0, C, ldc, out_kind, R, ldr, M, N, K};
+  mt::GemmDesc g{A, lda, a_mn_major != 0, B, ldb, b_mn_major != 0, C, ldc, out_kind, R, ldr, M, N, K, mt::RopeDesc{}};
   return mt::gemm_bf16(g, static_cast<cudaStream_t>(stream), dev_err);
 }
 
@@ -86,7 +86,8 @@ extern "C" int mt_k_attn_fwd(const void* q, const void* k, const void* v, int64_
 extern "C" int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o,
                              const void* dout, int64_t ldo, const float* lse, float* dvec, float* dq_acc,
                              int64_t ldqa, void* dq, int64_t lddq, void* dk, void* dv, int64_t lddkv, int b, int s,
-                             int H, int Hkv, int hd, void* stream) {
+                             int H, int Hkv, int hd, const float* cos_tab, const float* sin_tab, void* stream) {
+  if ((cos_tab == nullptr) != (sin_tab == nullptr)) return MT_ERR_ARG;
   if (!q || !k || !v || !o || !dout || !lse || !dvec || !dq_acc || !dq || !dk || !dv) return MT_ERR_ARG;
   if (b < 0 || s < 0 || H <= 0 || Hkv <= 0 || (H % Hkv)) return MT_ERR_ARG;
   if (hd != 64 && hd != 128) return MT_ERR_CONFIG;
@@ -97,6 +98,7 @@ extern "C" int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_
   a.q = q; a.k = k; a.v = v; a.ldqkv = ldqkv; a.o = const_cast<void*>(o); a.ldo = ldo; a.lse = const_cast<float*>(lse);
   a.dout = dout; a.dvec = dvec; a.dq_acc = dq_acc; a.ldqa = ldqa; a.dq = dq; a.lddq = lddq; a.dk = dk; a.dv = dv;
   a.lddkv = lddkv; a.b = b; a.s = s; a.H = H; a.Hkv = Hkv; a.hd = hd; a.scale = 1.0f / std::sqrt((float)hd);
+  a.rope_cos = cos_tab; a.rope_sin = sin_tab;
   return mt::attention_bwd(a, S(stream));
 }
 
@@ -109,4 +111,13 @@ extern "C" int mt_k_attn_fwd_tc(const void* q, const void* k, const void* v, int
   a.q = q; a.k = k; a.v = v; a.ldqkv = ldqkv; a.o = o; a.ldo = ldo; a.lse = lse;
   a.b = b; a.s = s; a.H = H; a.Hkv = Hkv; a.hd = hd; a.scale = 1.0f / std::sqrt((float)hd);
   return mt::attention_fwd_tc(a, S(stream), dev_err);
+}
+
+extern "C" int mt_k_gemm_bf16_rope(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, int M,
+                                   int N, int K, int rope_cols, int hd, int s, const float* cos_tab,
+                                   const float* sin_tab, void* stream, int32_t* dev_err) {
+  if (M < 0 || N < 0 || K < 0 || !cos_tab || !sin_tab) return MT_ERR_ARG;
+  mt::GemmDesc g{A, lda, false, B, ldb, false, C, ldc, mt::EPI_BF16_ROPE, nullptr, 0, M, N, K,
+                 mt::RopeDesc{cos_tab, sin_tab, rope_cols, hd, s}};
+  return mt::gemm_bf16(g, static_cast<cudaStream_t>(stream), dev_err);
 }

@@ -14,7 +14,17 @@ namespace mt {
 int launch_status();
 const char* last_launch_error();
 
-enum GemmEpi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_F32_ADD = 2 };
+enum GemmEpi : int { EPI_BF16 = 0, EPI_F32 = 1, EPI_F32_ADD = 2, EPI_BF16_ROPE = 3 };
+
+// RoPE applied in the epilogue (EPI_BF16_ROPE): columns [0, cols) hold heads of
+// width hd whose rotate-half pairs (i, i + hd/2) are rotated by the angle of
+// position (row % seq) with fp32 tables cos/sin [seq, hd/2]; other columns are
+// stored unrotated.
+struct RopeDesc {
+  const float* cos;
+  const float* sin;
+  int cols, hd, seq;
+};
 
 // C[M,N] = A[M,K] * B[N,K]^T (+ R for EPI_F32_ADD; R may alias C).
 //   A K-major: element (m,k) at A[m*lda + k];  A MN-major: at A[k*lda + m]
@@ -32,6 +42,7 @@ struct GemmDesc {
   const float* R;
   int64_t ldr;
   int M, N, K;
+  RopeDesc rope;
 };
 
 int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
@@ -64,6 +75,10 @@ struct AttnArgs {
   int64_t lddkv;
   int b, s, H, Hkv, hd;
   float scale;
+  // When set, the backward returns gradients with respect to q and k before
+  // RoPE (the transposed rotation is applied to dQ and dK on output).
+  const float* rope_cos;
+  const float* rope_sin;
 };
 int attention_fwd(const AttnArgs& a, cudaStream_t st);
 int attention_bwd(const AttnArgs& a, cudaStream_t st);

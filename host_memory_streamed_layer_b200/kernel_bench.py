@@ -91,7 +91,7 @@ def bench_attn(iters, warmup, fwd_only, impl="tc"):
         dp = dqkv.data_ptr()
         bwd = lambda: mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(),  # noqa
                                        dvec.data_ptr(), dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD,
-                                       dp + 4 * H * HD, ld, B, S, H, H, HD, st)
+                                       dp + 4 * H * HD, ld, B, S, H, H, HD, 0, 0, st)
         sec = timed(bwd, iters, warmup)
         res.append({"kernel": "attn_bwd", "us": sec * 1e6, "tflops": 2.5 * fl / sec / 1e12 if sec else None})
     return res

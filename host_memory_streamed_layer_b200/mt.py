@@ -68,7 +68,10 @@ _sig("mt_k_attn_fwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_i6
 _sig("mt_k_attn_fwd_tc", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_int, c_int,
      c_int, c_int, c_int, c_void_p, c_void_p)
 _sig("mt_k_attn_bwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_void_p,
-     c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p)
+     c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p,
+     c_void_p, c_void_p)
+_sig("mt_k_gemm_bf16_rope", c_int, c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_i64, c_int, c_int, c_int, c_int,
+     c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p)
 
 
 _sig("mt_k_rmsnorm_bwd_noalloc", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
@@ -132,9 +135,14 @@ def mt_k_attn_fwd_tc(q, k, v, ldqkv, o, ldo, lse, b, s, H, Hkv, hd, stream=0, de
 
 
 def mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv, b, s, H, Hkv, hd,
-                  stream=0):
+                  cos_tab=0, sin_tab=0, stream=0):
     return _check(lib.mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv,
-                                    b, s, H, Hkv, hd, _p(stream)), "mt_k_attn_bwd")
+                                    b, s, H, Hkv, hd, _p(cos_tab), _p(sin_tab), _p(stream)), "mt_k_attn_bwd")
+
+
+def mt_k_gemm_bf16_rope(A, lda, B, ldb, C, ldc, M, N, K, rope_cols, hd, s, cos_tab, sin_tab, stream=0, dev_err=0):
+    return _check(lib.mt_k_gemm_bf16_rope(A, lda, B, ldb, C, ldc, M, N, K, rope_cols, hd, s, cos_tab, sin_tab,
+                                          _p(stream), _p(dev_err)), "mt_k_gemm_bf16_rope")
 
 
 # ---------------------------------------------------------------------------

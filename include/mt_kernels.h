@@ -132,10 +132,25 @@ int mt_k_attn_fwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv,
 /* Causal attention backward from o, lse and dout (bf16, pitch ldo):
  * dvec fp32 [b,H,s] and dq_acc fp32 [b*s, ldqa] are caller scratch (dq_acc is
  * zeroed by the call); dq (pitch lddq), dk and dv (pitch lddkv) are bf16
- * outputs laid out like q, k, v. dk, dv of a KV head sum over its query heads. */
+ * outputs laid out like q, k, v. dk, dv of a KV head sum over its query heads.
+ * When cos_tab/sin_tab (fp32 [s, hd/2], as for mt_k_rope) are given, q and k
+ * are taken to be post-RoPE and dq, dk are returned with respect to the
+ * pre-RoPE values (the transposed rotation is applied on output); NULL
+ * returns gradients with respect to q and k as given. */
 int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o, const void* dout,
                   int64_t ldo, const float* lse, float* dvec, float* dq_acc, int64_t ldqa, void* dq, int64_t lddq,
-                  void* dk, void* dv, int64_t lddkv, int b, int s, int H, int Hkv, int hd, void* stream);
+                  void* dk, void* dv, int64_t lddkv, int b, int s, int H, int Hkv, int hd, const float* cos_tab,
+                  const float* sin_tab, void* stream);
+
+/* Forward projection with RoPE fused into the epilogue: C bf16 [M,N] =
+ * rope(A[M,K] B[N,K]^T), both operands K-major as in mt_k_gemm_bf16. Columns
+ * [0, rope_cols) are heads of width hd (64 or 128) whose rotate-half pairs are
+ * rotated in fp32 by the angle of position (row % s) from the fp32 tables
+ * cos_tab/sin_tab [s, hd/2] before the single rounding to bf16; columns from
+ * rope_cols on are stored unrotated. N must be a multiple of hd. */
+int mt_k_gemm_bf16_rope(const void* A, int64_t lda, const void* B, int64_t ldb, void* C, int64_t ldc, int M, int N,
+                        int K, int rope_cols, int hd, int s, const float* cos_tab, const float* sin_tab, void* stream,
+                        int32_t* dev_err);
 
 /* Host AdamW over n fp32 elements, in place (HOST pointers, runs on the
  * calling thread; the engine runs the same routine across its worker pool):

@@ -247,3 +247,67 @@ def test_attention_bwd(hd, H, Hkv, s, b):
     assert rel_l2(g[:, :H * hd].reshape(b, s, H, hd), rdq, floor) < 1e-2
     assert rel_l2(g[:, H * hd:(H + Hkv) * hd].reshape(b, s, Hkv, hd), rdk, floor) < 1e-2
     assert rel_l2(g[:, (H + Hkv) * hd:].reshape(b, s, Hkv, hd), rdv) < 1e-2
+
+
+@pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 16, 16, 256, 1)])
+def test_qkv_gemm_with_rope_epilogue(hd, H, Hkv, s, b):
+    """q, k, v projection with RoPE fused in the epilogue = oracle RoPE of the
+    fp64 product (v columns unrotated), rounded once to bf16."""
+    mt = _mt()
+    rng = np.random.default_rng(hd * s)
+    T, d = b * s, 256
+    N = (H + 2 * Hkv) * hd
+    A = bf(rng.normal(size=(T, d)))
+    Bw = bf(rng.normal(size=(N, d)) * 0.05)
+    cos, sin = oracle.rope_tables(s, hd, 10000.0)
+    c32, s32 = f32(cos), f32(sin)
+    C = torch.empty(T, N, dtype=torch.bfloat16, device=DEV)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    mt.mt_k_gemm_bf16_rope(A.data_ptr(), d, Bw.data_ptr(), d, C.data_ptr(), N, T, N, d, (H + Hkv) * hd, hd, s,
+                           c32.data_ptr(), s32.data_ptr(), 0, err.data_ptr())
+    sync()
+    assert err.item() == 0
+    prod = np64(A) @ np64(Bw).T
+    q = oracle.rope_fwd(prod[:, :H * hd].reshape(b, s, H, hd), cos, sin).reshape(T, -1)
+    k = oracle.rope_fwd(prod[:, H * hd:(H + Hkv) * hd].reshape(b, s, Hkv, hd), cos, sin).reshape(T, -1)
+    ref = np.concatenate([q, k, prod[:, (H + Hkv) * hd:]], axis=1)
+    got = np64(C)
+    scale = np.abs(np64(A)) @ np.abs(np64(Bw)).T  # bound of |products| per element
+    pair = np.concatenate([scale[:, :H * hd].reshape(T, H, hd), scale[:, H * hd:(H + Hkv) * hd].reshape(T, Hkv, hd)],
+                          axis=1)
+    pair = (pair + np.roll(pair, hd // 2, axis=-1)).reshape(T, -1)
+    bound = 2 ** -8 * np.abs(ref) + 1e-5 * np.concatenate([pair, scale[:, (H + Hkv) * hd:]], axis=1)
+    assert np.all(np.abs(got - ref) <= bound)
+
+
+@pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3)])
+def test_attention_bwd_returns_pre_rope_gradients(hd, H, Hkv, s, b):
+    """With the RoPE tables the backward returns dL/d(pre-RoPE q, k): the
+    oracle's attention backward followed by its rope_bwd."""
+    mt = _mt()
+    qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, 11 * hd + s)
+    T = b * s
+    rng = np.random.default_rng(5 * s)
+    do = bf(rng.normal(size=(T, H * hd)))
+    o = torch.empty(T, H * hd, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(b, H, s, device=DEV)
+    p = qkv.data_ptr()
+    pk, pv = p + 2 * H * hd, p + 2 * (H + Hkv) * hd
+    mt.mt_k_attn_fwd_tc(p, pk, pv, ld, o.data_ptr(), H * hd, lse.data_ptr(), b, s, H, Hkv, hd)
+    cos, sin = oracle.rope_tables(s, hd, 10000.0)
+    c32, s32 = f32(cos), f32(sin)
+    dvec = torch.empty(b, H, s, device=DEV)
+    dqa = torch.empty(T, H * hd, device=DEV)
+    dqkv = torch.zeros(T, ld, dtype=torch.bfloat16, device=DEV)
+    dp = dqkv.data_ptr()
+    mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(), dvec.data_ptr(),
+                     dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd, dp + 2 * (H + Hkv) * hd, ld, b, s, H, Hkv, hd,
+                     c32.data_ptr(), s32.data_ptr())
+    sync()
+    _, P = oracle.attention_fwd(q, k, v)
+    rdq, rdk, rdv = oracle.attention_bwd(q, k, v, P, np64(do).reshape(b, s, H, hd))
+    rdq, rdk = oracle.rope_bwd(rdq, cos, sin), oracle.rope_bwd(rdk, cos, sin)
+    g = np64(dqkv)
+    assert rel_l2(g[:, :H * hd].reshape(b, s, H, hd), rdq) < 1e-2
+    assert rel_l2(g[:, H * hd:(H + Hkv) * hd].reshape(b, s, Hkv, hd), rdk) < 1e-2
+    assert rel_l2(g[:, (H + Hkv) * hd:].reshape(b, s, Hkv, hd), rdv) < 1e-2
