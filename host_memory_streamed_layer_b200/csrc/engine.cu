@@ -67,7 +67,7 @@ inline float normal_at(uint64_t key, uint64_t i) {
 }
 
 struct Job {
-  enum Kind { LAYER, HEAD, EMBED } kind;
+  enum Kind { LAYER, HEAD, EMBED, EMBED_UNTOUCHED } kind;
   int layer;
   cudaEvent_t ready;  // offload of this job's gradients has completed
   int flag_index;     // index in the finite-flag array
@@ -401,6 +401,7 @@ int head_step(mt_ctx* c, float* gout) {
 // Optimizer thread.
 // ---------------------------------------------------------------------------
 bool wait_event(mt_ctx* c, cudaEvent_t e) {
+  if (!e) return true;
   const double t0 = now_s();
   while (true) {
     cudaError_t r = cudaEventQuery(e);
@@ -417,6 +418,8 @@ struct Seg {
 };
 
 void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
+  // 64K-element pieces handed out dynamically: a worker slowed by other
+  // activity on its core (the enqueueing thread, DMA) does not hold the job up.
   const AdamHyper h{c->cfg.lr, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps, c->cfg.wd};
   const size_t chunk = 1 << 16;
   struct Task {
@@ -424,8 +427,13 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
     uint16_t* bf;
   };
   std::vector<Task> tasks;
-  for (const Seg& sg : segs)
-    for (size_t i = 0; i < sg.n; i += chunk) tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf + i});
+  size_t total = 0;
+  for (const Seg& sg : segs) {
+    for (size_t i = 0; i < sg.n; i += chunk)
+      tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf ? sg.bf + i : nullptr});
+    total += sg.n;
+  }
+  if (tasks.empty()) return;
   const int t = c->step;
   const double t0 = now_s();
   if (c->adamw_first == 0) c->adamw_first = t0;
@@ -435,9 +443,7 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
   });
   c->adamw_last = now_s();
   c->adamw_s += c->adamw_last - t0;
-  size_t n = 0;
-  for (const Seg& sg : segs) n += sg.n;
-  c->adamw_bytes += 30.0 * n;
+  c->adamw_bytes += 30.0 * total;
 }
 
 void run_job(mt_ctx* c, const Job& j) {
@@ -449,16 +455,38 @@ void run_job(mt_ctx* c, const Job& j) {
     c->skip_updates = true;
     return;
   }
-  if (j.kind == Job::EMBED) {
-    // Dense gradient of the embedding: zero last step's rows, then scatter this
-    // step's rows (checking them for NaN/Inf), both across the worker pool.
+  if (j.kind == Job::EMBED_UNTOUCHED) {
+    // Rows no token of this batch touches have a zero gradient, so their update
+    // does not depend on this step's backward and runs while the GPU is in the
+    // forward sweep (the gather reads only the touched rows). Zero last step's
+    // touched gradient rows first: every row's gradient this step is then 0
+    // until the touched rows are scattered at the end.
     float* ge = c->grad + y.embed.off;
     const size_t d = s.d;
     const int nt = c->pool->size() * 4;
-    const size_t np = c->prev_uniq.size(), nu = c->uniq.size();
+    const size_t np = c->prev_uniq.size();
     c->pool->run(nt, [&](int i) {
       for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k) memset(ge + (size_t)c->prev_uniq[k] * d, 0, d * 4);
     });
+    c->prev_uniq = c->uniq;
+    if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
+    std::vector<Seg> segs;
+    int32_t next = 0;  // first row of the current untouched run
+    for (size_t u = 0; u <= c->uniq.size(); ++u) {
+      const int32_t stop = u < c->uniq.size() ? c->uniq[u] : s.V;
+      if (stop > next)
+        segs.push_back({y.embed.off + (size_t)next * d, (size_t)(stop - next) * d, c->bf_embed + (size_t)next * d});
+      next = stop + 1;
+    }
+    adamw_segments(c, segs);
+    return;
+  }
+  if (j.kind == Job::EMBED) {
+    // Touched rows: scatter this step's gradient rows (checking for NaN/Inf).
+    float* ge = c->grad + y.embed.off;
+    const size_t d = s.d;
+    const int nt = c->pool->size() * 4;
+    const size_t nu = c->uniq.size();
     std::vector<char> bad(nt, 0);
     c->pool->run(nt, [&](int i) {
       bool b = false;
@@ -471,7 +499,6 @@ void run_job(mt_ctx* c, const Job& j) {
       }
       bad[i] = b;
     });
-    c->prev_uniq = c->uniq;
     for (char b : bad)
       if (b) c->flags_h[j.flag_index] = 1;
   }
@@ -494,7 +521,7 @@ void run_job(mt_ctx* c, const Job& j) {
     segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head});
     segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(s.d, 128)});
   } else {
-    segs.push_back({y.embed.off, y.embed.n, c->bf_embed});
+    for (int32_t r : c->uniq) segs.push_back({y.embed.off + (size_t)r * s.d, (size_t)s.d, c->bf_embed + (size_t)r * s.d});
   }
   adamw_segments(c, segs);
 }
@@ -1057,6 +1084,7 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   c->timed.clear();
   c->launches = 0;
   c->err.clear();
+  push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, s.L + 1});
   const double te0 = now_s();
   int r = enqueue_step(c, n_unique);
   c->enqueue_s = now_s() - te0;
