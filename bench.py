@@ -249,6 +249,25 @@ def link_bandwidth(torch, dev):
     return r
 
 
+def host_optimizer_bandwidth(mt, threads, n=1 << 28):
+    """GB/s (30 B/param accounting) of the library's host AdamW on its own
+    worker pool over 4 x 1 GiB fp32 arrays, best of 3: the host-DRAM ceiling
+    the optimizer can reach when nothing else uses memory."""
+    return mt.mt_host_optimizer_gbs(n, threads)
+
+
+def phase_flops(sh):
+    """(forward + head FLOPs, backward-phase FLOPs) of the schedule."""
+    L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
+    hd = d // H
+    T = b * s
+    Pm = d * (H + 2 * Hkv) * hd + d * H * hd + 3 * d * F
+    A = 2.0 * b * s * s * H * hd
+    fwd = L * (2.0 * T * Pm + A) + 6.0 * T * V * d
+    bwd = (L - 1) * (2.0 * T * (Pm - d * F) + A) + L * (4.0 * T * Pm + 2.5 * A)
+    return fwd, bwd
+
+
 # ---------------------------------------------------------------------------
 # Main arm.
 # ---------------------------------------------------------------------------
@@ -309,6 +328,7 @@ def main():
         return
 
     link = link_bandwidth(torch, dev) if rank == 0 else None
+    host_bw = host_optimizer_bandwidth(mt, cfg.host_threads) if rank == 0 else None
     ctx = mt.mt_create(cfg)
     try:
         nsteps = args.warmup + 2 * args.steps
@@ -371,7 +391,18 @@ def main():
         t_compute = exec_f / (peak * 1e12)
         t_h2d = h2d_b / (link["h2d_gbs"] * 1e9)
         t_d2h = d2h_b / (link["d2h_gbs"] * 1e9)
-        t_bound = max(t_compute, t_h2d, t_d2h)
+        # Phase bound of this method's dependency structure: the forward sweep
+        # and head (GPU compute or weight H2D, whichever is slower) must finish
+        # before any gradient exists; then the backward (GPU compute, D2H) runs
+        # alongside the host optimizer, which with the concurrent DMA is bound
+        # by host DRAM bandwidth.
+        f_fl, b_fl = phase_flops(sh)
+        L = sh["L"]
+        t_fwd_b = max(f_fl / (peak * 1e12), h2d_b * L / (2 * L - 1) / (link["h2d_gbs"] * 1e9))
+        host_bytes = mean("adamw_bytes") + d2h_b + h2d_b * (L - 1) / (2 * L - 1)
+        t_host_b = host_bytes / (host_bw * 1e9)
+        t_bwd_b = max(b_fl / (peak * 1e12), t_d2h, t_host_b)
+        t_bound = t_fwd_b + t_bwd_b
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -386,8 +417,11 @@ def main():
                          "frac": (achieved / peak) if achieved else None, "traffic": None,
                          "peak_kind": f"bf16_tflops_sustained ({ptype})",
                          "launches_per_step": g_n / K, "gemm_ms_per_step": g_ms / K},
-            "step_roofline": {"compute_ms": t_compute * 1e3, "h2d_ms": t_h2d * 1e3, "d2h_ms": t_d2h * 1e3,
-                              "bound_ms": t_bound * 1e3, "frac": t_bound / (t_dev / K),
+            "step_roofline": {"bound_ms": t_bound * 1e3, "frac": t_bound / (t_dev / K),
+                              "fwd_bound_ms": t_fwd_b * 1e3, "bwd_bound_ms": t_bwd_b * 1e3,
+                              "host_bytes": host_bytes, "host_bound_ms": t_host_b * 1e3,
+                              "host_optimizer_gbs_measured": host_bw,
+                              "compute_ms": t_compute * 1e3, "h2d_ms": t_h2d * 1e3, "d2h_ms": t_d2h * 1e3,
                               "link_measured": link, "h2d_bytes": h2d_b, "d2h_bytes": d2h_b,
                               "attention_tflops": a_fl / (a_ms / 1e3) / 1e12 if a_ms > 0 else None,
                               "attention_ms_per_step": a_ms / K,

@@ -836,6 +836,10 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   // logits chunk: at most ~4 GiB of fp32 logits + bf16 dz, multiple of 128 tokens
   int Tc = (int)std::min<int64_t>(s.T, ((int64_t)1 << 32) / ((int64_t)s.V * 6));
   if (Tc < s.T) Tc = std::max(128, Tc / 128 * 128);
+  if (const char* e = getenv("MT_LOGITS_CHUNK")) {  // smaller chunks (multiple of 128 tokens), e.g. for tests
+    const int want = atoi(e);
+    if (want >= 128 && want % 128 == 0 && want < Tc) Tc = want;
+  }
   const size_t need = device_bytes(y, Tc);
   size_t free_b = 0, total_b = 0;
   if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaMemGetInfo failed");

@@ -1,11 +1,18 @@
 // Host AdamW (AVX-512 with a portable fallback) and the worker pool.
 #include "host_adamw.h"
 
+#include "mt.h"
 #include "mt_kernels.h"
+
+#include <algorithm>
 
 #include <immintrin.h>
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
+
+#include <chrono>
+#include <thread>
 
 namespace mt {
 
@@ -205,4 +212,39 @@ extern "C" int mt_k_adamw_host(float* p, const float* g, float* m, float* v, uin
   if (t < 1 || !(eps > 0) || !(beta1 >= 0 && beta1 < 1) || !(beta2 >= 0 && beta2 < 1)) return MT_ERR_ARG;
   mt::adamw_chunk(p, g, m, v, pb, n, mt::AdamHyper{lr, beta1, beta2, eps, wd}, t);
   return MT_OK;
+}
+
+extern "C" double mt_host_optimizer_gbs(size_t n, int threads) {
+  if (n < (1u << 16)) return MT_ERR_ARG;
+  if (threads <= 0) threads = std::max(1, (int)std::thread::hardware_concurrency() - 1);
+  float* a[4] = {};
+  uint16_t* pb = nullptr;
+  for (auto& x : a)
+    if (posix_memalign(reinterpret_cast<void**>(&x), 64, n * 4)) x = nullptr;
+  if (posix_memalign(reinterpret_cast<void**>(&pb), 64, n * 2)) pb = nullptr;
+  double best = 0;
+  if (a[0] && a[1] && a[2] && a[3] && pb) {
+    mt::ThreadPool pool(threads - 1);
+    const size_t chunk = 1 << 16;
+    const int tasks = (int)((n + chunk - 1) / chunk);
+    pool.run(tasks, [&](int i) {  // parallel first touch
+      const size_t b = (size_t)i * chunk, m = std::min(chunk, n - b);
+      for (int k = 0; k < 4; ++k)
+        for (size_t j = 0; j < m; ++j) a[k][b + j] = 1e-3f;
+      memset(pb + b, 0, m * 2);
+    });
+    const mt::AdamHyper h{1e-3f, 0.9f, 0.95f, 1e-8f, 0.1f};
+    for (int rep = 0; rep < 3; ++rep) {
+      const auto t0 = std::chrono::steady_clock::now();
+      pool.run(tasks, [&](int i) {
+        const size_t b = (size_t)i * chunk, m = std::min(chunk, n - b);
+        mt::adamw_chunk(a[0] + b, a[1] + b, a[2] + b, a[3] + b, pb + b, m, h, 1);
+      });
+      const double sec = std::chrono::duration<double>(std::chrono::steady_clock::now() - t0).count();
+      best = std::max(best, 30.0 * n / sec / 1e9);
+    }
+  }
+  for (auto& x : a) free(x);
+  free(pb);
+  return best > 0 ? best : MT_ERR_NOMEM;
 }

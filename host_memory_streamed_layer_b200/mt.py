@@ -187,6 +187,7 @@ _sig("mt_get_params", c_int, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
 _sig("mt_destroy", None, c_void_p)
 _sig("mt_get_stream", c_int, c_void_p, ctypes.POINTER(c_void_p))
+_sig("mt_host_optimizer_gbs", ctypes.c_double, c_size_t, c_int)
 _sig("mt_last_error", ctypes.c_char_p, c_void_p)
 _sig("mt_k_adamw_host", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_float, c_float,
      c_float, c_float, c_float, c_int)
@@ -262,3 +263,10 @@ def mt_last_error(ctx: int = 0) -> str:
 
 def mt_k_adamw_host(p, g, m, v, pb, n, lr, beta1, beta2, eps, wd, t):
     return _check(lib.mt_k_adamw_host(p, g, m, v, pb or None, n, lr, beta1, beta2, eps, wd, t), "mt_k_adamw_host")
+
+
+def mt_host_optimizer_gbs(n: int = 1 << 28, threads: int = 0) -> float:
+    r = lib.mt_host_optimizer_gbs(n, threads)
+    if r < 0:
+        raise MTError(int(r), "mt_host_optimizer_gbs")
+    return r

@@ -153,6 +153,14 @@ int mt_get_stats(mt_ctx* ctx, mt_stats* out);
  * context. */
 int mt_get_stream(mt_ctx* ctx, void** stream);
 
+/* Host-memory ceiling of the optimizer: runs the library's host AdamW (the
+ * same routine, worker pool and chunking the engine uses) over four fp32
+ * arrays of n elements with `threads` threads (0 = all cores but one), best
+ * of 3 passes, and returns GB/s counted as 30 bytes per element (read p, g,
+ * m, v; write p, m, v and the bf16 copy). Allocates and frees its own host
+ * buffers; no GPU needed. Returns a negative MT_ERR_* on failure. */
+double mt_host_optimizer_gbs(size_t n, int threads);
+
 /* Waits for the context's streams, frees its device memory and unpins or
  * frees its host memory. NULL is ignored. */
 void mt_destroy(mt_ctx* ctx);

@@ -168,3 +168,15 @@ def test_library_owned_arena_initialisation():
         assert abs(loss - (math.log(shape["V"]) + 0.0004 * shape["d"] / 2)) < 0.1
     finally:
         mt.mt_destroy(ctx)
+
+
+def test_chunked_head_matches_oracle(monkeypatch):
+    """LM head processed in token chunks (dW_head accumulated across chunks)."""
+    monkeypatch.setenv("MT_LOGITS_CHUNK", "128")
+    shape = SHAPES["gqa_ragged"]  # T = 300 tokens -> chunks of 128, 128, 44
+    c = oracle.OracleConfig(**shape)
+    g = run_gpu(shape, 1)[0]
+    r = oracle_steps(shape, 1)[0]
+    assert abs(g["loss"] - r["loss"]) <= 1e-2
+    G = oracle.unpack_arena(g["G"], c)
+    assert max(rel(G[k], r["G"][k]) for k in r["G"]) <= 2e-2
