@@ -65,6 +65,12 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// Bounded wait whose result is the same on every lane of the warp, so that a
+// timeout can never split a warp in front of a warp-collective tcgen05.ld.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity));
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -250,7 +256,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
 
     auto accumulate_o = [&](int i, float corr) -> bool {
       const int ob = i & 1;
-      if (*abort_flag || !mbar_wait(&o_full[ob], (i >> 1) & 1)) return false;
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[ob], (i >> 1) & 1)) return false;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < HH / 16; ++c) {
@@ -269,7 +275,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     for (int j = 0; j < nkv; ++j) {
       const int sb = j & 1;
       const uint32_t ph = (j >> 1) & 1;
-      if (*abort_flag || !mbar_wait(&s_full[sb], ph)) {
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&s_full[sb], ph)) {
         ok = false;
         break;
       }
@@ -405,6 +411,468 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   if (a.hd == 64) return launch_fa<64>(a, st, err);
   if (a.hd == 128) return launch_fa<128>(a, st, err);
   return MT_ERR_CONFIG;
+}
+
+
+// ===========================================================================
+// Backward on the tcgen05 tensor cores (head_dim 128).
+//
+// One CTA per (128-key block, KV head, sequence); it loops over every query
+// head of the group and every 64-query block at or after its keys:
+//   S^T  = K Q^T,   dP^T = V dO^T          (128 keys x 64 queries, TMEM)
+//   P^T  = exp(S^T / sqrt(hd) - LSE),  dS^T = P^T (dP^T - D)   (softmax warps,
+//          one key row per thread, bf16 into 128-byte-swizzled tiles)
+//   dV  += P^T dO,  dK += dS^T Q            (128 keys x hd, TMEM, whole CTA)
+//   dQ^T = K^T dS^T                          (hd x 64 queries, TMEM), read out
+//          one head column per thread into an fp32 staging tile in shared
+//          memory, then added to the fp32 dQ accumulator with TMA bulk
+//          reduce-add (four 64 x 32 boxes per tile)
+// The K tile serves both as the K-major A operand of S^T (keys x hd) and as
+// the MN-major A operand of dQ^T (hd x keys); the dS^T tile both as the
+// K-major A operand of dK and the MN-major B operand of dQ^T.
+// ===========================================================================
+namespace {
+
+constexpr int FB_BKV = 128, FB_BQ = 64, FB_HD = 128;
+constexpr int FB_THREADS = 320;  // producer, MMA, 8 gradient warps (two per tensor-memory lane quarter)
+
+struct FbCfg {
+  static constexpr int KV_BYTES = FB_BKV * FB_HD * 2;  // 32 KB
+  static constexpr int QT_BYTES = FB_BQ * FB_HD * 2;   // 16 KB (Q or dO tile)
+  static constexpr int T_BYTES = FB_BKV * FB_BQ * 2;   // 16 KB (P^T or dS^T)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_BYTES;
+  static constexpr int OFF_Q = OFF_V + KV_BYTES;        // [2] stages
+  static constexpr int OFF_DO = OFF_Q + 2 * QT_BYTES;   // [2]
+  static constexpr int OFF_PT = OFF_DO + 2 * QT_BYTES;
+  static constexpr int OFF_DST = OFF_PT + T_BYTES;
+  static constexpr int OFF_DQS = OFF_DST + T_BYTES;     // dQ staging: 4 boxes [64 q][32 hd] fp32
+  static constexpr int DQS_BYTES = FB_BQ * FB_HD * 4;    // 32 KB
+  static constexpr int OFF_BAR = OFF_DQS + DQS_BYTES;
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  // tensor-memory columns: dK, dV, then two buffers of [S^T (64) | dP^T (64)];
+  // dQ^T of an iteration reuses the S^T columns of its buffer once consumed.
+  static constexpr uint32_t C_DK = 0, C_DV = 128, C_BUF = 256, BUF_COLS = 128, C_DP_OFF = 64;
+};
+
+struct FbParams {
+  const float* LSE;
+  const float* Dv;
+  float* dQacc;
+  int64_t ldqa;
+  __nv_bfloat16* dK;
+  __nv_bfloat16* dV;
+  int64_t lddkv;
+  int s, H, Hkv;
+  float scale;
+  const float* rcos;
+  const float* rsin;
+  int* err;
+};
+
+__global__ void __launch_bounds__(FB_THREADS, 1)
+    k_flash_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const __grid_constant__ CUtensorMap tmDQ, FbParams p) {
+  using C = FbCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sdO = smem + C::OFF_DO;
+  uint8_t* sPt = smem + C::OFF_PT;
+  uint8_t* sdSt = smem + C::OFF_DST;
+  float* sDQ = reinterpret_cast<float*>(smem + C::OFF_DQS);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bar + 0;
+  uint64_t* q_full = bar + 1;    // [2]
+  uint64_t* q_empty = bar + 3;   // [2]
+  uint64_t* s_full = bar + 5;    // [2] S^T, dP^T of a buffer ready
+  uint64_t* p_full = bar + 7;    // P^T, dS^T tiles written
+  uint64_t* mma_done = bar + 8;  // dV, dK, dQ^T of an iteration done
+  uint64_t* dq_empty = bar + 9;  // [2] dQ^T of a buffer read out
+  uint64_t* drain = bar + 11;
+  uint64_t* dq_staged = bar + 12;  // staging tile written
+  uint64_t* dq_free = bar + 13;    // the previous reduce has read the staging tile
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 14);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 15);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kvb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int group = p.H / p.Hkv;
+  const int kv0 = kvb * FB_BKV;
+  const int row0 = b * p.s;
+  const int nqb = (p.s + FB_BQ - 1) / FB_BQ;
+  const int qb_first = kv0 / FB_BQ;
+  const int per_head = nqb - qb_first;
+  const int n_it = group * per_head;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&dq_empty[i], 8);
+    }
+    mbar_init(p_full, 8);
+    mbar_init(mma_done, 1);
+    mbar_init(drain, 1);
+    mbar_init(dq_staged, 8);
+    mbar_init(dq_free, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmDQ);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int q_last[2] = {-1, -1};
+      bool ok = true;
+      mbar_arrive_expect_tx(kv_full, 2 * C::KV_BYTES);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_2d(sK + c * 16384, &tmK, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+        tma_load_2d(sV + c * 16384, &tmV, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+      }
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const int h = kvh * group + it / per_head;
+        const int q0 = (qb_first + it % per_head) * FB_BQ;
+        if (*abort_flag || !mbar_wait(&q_empty[st], ph ^ 1)) {
+          record_error(p.err, 100 + (it & 63));
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[st], 2 * C::QT_BYTES);
+        for (int c = 0; c < 2; ++c) {
+          tma_load_2d(sQ + st * C::QT_BYTES + c * 8192, &tmQ, &q_full[st], h * FB_HD + c * 64, row0 + q0);
+          tma_load_2d(sdO + st * C::QT_BYTES + c * 8192, &tmO, &q_full[st], h * FB_HD + c * 64, row0 + q0);
+        }
+        q_last[st] = (int)ph;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (!mbar_wait(kv_full, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        for (int s2 = 0; s2 < 2; ++s2)
+          if (q_last[s2] >= 0 && !mbar_wait(&q_full[s2], (uint32_t)q_last[s2])) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      // Order per iteration: S(it+1), dP(it+1) into the other buffer, then
+      // dV(it), dK(it), dQ^T(it); the tensor core works on the next scores
+      // while the gradient warps form P(it) and drain dQ^T(it-1).
+      constexpr uint32_t id_s = idesc_bf16_f32(FB_BKV, FB_BQ, false, false);   // keys x queries, K = hd
+      constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, FB_HD, false, true);   // keys x hd, K = queries
+      constexpr uint32_t id_dq = idesc_bf16_f32(FB_HD, FB_BQ, true, true);     // hd x queries, K = keys
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPt = smem_u32(sPt), adSt = smem_u32(sdSt);
+      bool issued = false;
+      auto issue_s = [&](int it) -> bool {
+        const int st = it & 1;
+        if (*abort_flag || !mbar_wait(&q_full[st], (it >> 1) & 1)) {
+          record_error(p.err, 210 + (it & 63));
+          return false;
+        }
+        if (it >= 2 && !mbar_wait(&dq_empty[st], ((it - 2) >> 1) & 1)) {  // buffer st drained by iteration it-2
+          record_error(p.err, 250 + (it & 31));
+          return false;
+        }
+        tc_fence_after();
+        const uint32_t bQ = smem_u32(sQ + st * C::QT_BYTES), bO = smem_u32(sdO + st * C::QT_BYTES);
+        const uint32_t cs = tmem + C::C_BUF + st * C::BUF_COLS;
+#pragma unroll
+        for (int kk = 0; kk < FB_HD / 16; ++kk) {
+          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32, kb = (kk >> 2) * 8192 + (kk & 3) * 32;
+          umma_bf16(cs, sdesc_sw128(aK + ka, 16, 1024), sdesc_sw128(bQ + kb, 16, 1024), id_s, kk != 0);
+          umma_bf16(cs + C::C_DP_OFF, sdesc_sw128(aV + ka, 16, 1024), sdesc_sw128(bO + kb, 16, 1024), id_s, kk != 0);
+        }
+        issued = true;
+        umma_commit(&s_full[st]);
+        return true;
+      };
+      bool ok = mbar_wait(kv_full, 0) && !*abort_flag;
+      if (!ok) record_error(p.err, 200);
+      if (ok && n_it > 0) ok = issue_s(0);
+      for (int it = 0; it < n_it && ok; ++it) {
+        const int st = it & 1;
+        if (it + 1 < n_it && !issue_s(it + 1)) {
+          ok = false;
+          break;
+        }
+        if (*abort_flag || !mbar_wait(p_full, it & 1)) {
+          record_error(p.err, 280 + (it & 15));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t bQ = smem_u32(sQ + st * C::QT_BYTES), bO = smem_u32(sdO + st * C::QT_BYTES);
+        // dV += P^T dO, dK += dS^T Q (K = 64 queries: 4 steps; B MN-major over hd, 8 KB between hd chunks)
+#pragma unroll
+        for (int kk = 0; kk < FB_BQ / 16; ++kk) {
+          const bool acc = (it > 0) || (kk > 0);
+          umma_bf16(tmem + C::C_DV, sdesc_sw128(aPt + kk * 32, 16, 1024), sdesc_sw128(bO + kk * 2048, 8192, 1024),
+                    id_kv, acc);
+          umma_bf16(tmem + C::C_DK, sdesc_sw128(adSt + kk * 32, 16, 1024), sdesc_sw128(bQ + kk * 2048, 8192, 1024),
+                    id_kv, acc);
+        }
+        // dQ^T = K^T dS^T (K = 128 keys: 8 steps; A MN-major over hd, 16 KB between hd chunks) into the
+        // S^T columns of this iteration's buffer
+#pragma unroll
+        for (int kk = 0; kk < FB_BKV / 16; ++kk)
+          umma_bf16(tmem + C::C_BUF + st * C::BUF_COLS, sdesc_sw128(aK + kk * 2048, 16384, 1024),
+                    sdesc_sw128(adSt + kk * 2048, 8192, 1024), id_dq, kk != 0);
+        umma_commit(mma_done);
+        umma_commit(&q_empty[st]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (issued) {
+          umma_commit(drain);
+          if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        }
+      }
+    }
+  } else {
+    // ---------------- gradient warps (2..9) ----------------
+    const int wg = (warp - 2) >> 2;     // query columns [32 wg, 32 wg + 32) of each block
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key row == tensor-memory lane (the head column for dQ^T)
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale * 1.4426950408889634f;
+    const int key = kv0 + r;
+    const bool issuer = (warp == 2 && lane == 0);  // issues the dQ reductions
+    bool ok = true;
+
+    // Reads dQ^T(it) (already complete: the caller waited for it), stages it
+    // and lets the issuer add it to the accumulator.
+    auto flush_dq = [&](int it) -> bool {
+      const int bf = it & 1;
+      if (it > 0) {
+        // the staging tile is reused: the previous reduce must have read it
+        if (issuer) {
+          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+          mbar_arrive(dq_free);
+        }
+        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(dq_free, (it - 1) & 1)) {
+          record_error(p.err, 600 + (it & 63));
+          return false;
+        }
+      }
+      float* col = sDQ + (r >> 5) * (FB_BQ * 32) + (r & 31);  // box r/32: [64 queries][32 head columns]
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + wg * 32 + c * 16, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) col[(wg * 32 + c * 16 + e) * 32] = __uint_as_float(v[e]) * p.scale;
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&dq_empty[bf]);
+        mbar_arrive(dq_staged);
+      }
+      if (issuer) {
+        if (!mbar_wait(dq_staged, it & 1)) {
+          record_error(p.err, 700 + (it & 63));
+          return false;
+        }
+        const int h = kvh * group + it / per_head;
+        const int q0 = (qb_first + it % per_head) * FB_BQ;
+#pragma unroll
+        for (int bx = 0; bx < 4; ++bx)
+          asm volatile(
+              "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                  reinterpret_cast<uint64_t>(&tmDQ)),
+              "r"(smem_u32(sDQ + bx * FB_BQ * 32)), "r"(h * FB_HD + bx * 32), "r"(row0 + q0)
+              : "memory");
+        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+      }
+      return true;
+    };
+
+    for (int it = 0; it < n_it; ++it) {
+      const int bf = it & 1;
+      const int h = kvh * group + it / per_head;
+      const int q0 = (qb_first + it % per_head) * FB_BQ;
+      const float* lse = p.LSE + ((int64_t)b * p.H + h) * p.s + q0 + wg * 32;
+      const float* dd = p.Dv + ((int64_t)b * p.H + h) * p.s + q0 + wg * 32;
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&s_full[bf], (it >> 1) & 1)) {
+        record_error(p.err, 300 + (it & 63));
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // P^T and dS^T of this key row for this warpgroup's 32 queries (bf16 pairs)
+      uint32_t pp[16], ds[16];
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t sv[16], dv[16];
+        const uint32_t cb = tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + wg * 32 + c * 16;
+        tmem_ld_32x32b_x16(cb, sv);
+        tmem_ld_32x32b_x16(cb + C::C_DP_OFF, dv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 16; e += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int cq = c * 16 + e + u;
+            const int qi = q0 + wg * 32 + cq;
+            const bool vis = key <= qi && qi < p.s && key < p.s;
+            const float pr = vis ? ex2(__uint_as_float(sv[e + u]) * sl2 - __ldg(lse + cq) * 1.4426950408889634f) : 0.f;
+            pv[u] = pr;
+            dsv[u] = vis ? pr * (__uint_as_float(dv[e + u]) - __ldg(dd + cq)) : 0.f;
+          }
+          pp[(c * 16 + e) >> 1] = pack_bf16x2(pv[0], pv[1]);
+          ds[(c * 16 + e) >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+        }
+      }
+      // dV, dK, dQ^T of the previous iteration must be done with the tiles
+      if (it > 0 && (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1))) {
+        record_error(p.err, 400 + (it & 63));
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int c8 = 0; c8 < 4; ++c8) {
+        const int chunk = wg * 4 + c8;
+        const int off = r * 128 + ((chunk ^ (r & 7)) << 4);
+        *reinterpret_cast<uint4*>(sPt + off) = make_uint4(pp[4 * c8], pp[4 * c8 + 1], pp[4 * c8 + 2], pp[4 * c8 + 3]);
+        *reinterpret_cast<uint4*>(sdSt + off) = make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]);
+      }
+      tc_fence_before();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+      if (it > 0 && !flush_dq(it - 1)) {
+        ok = false;
+        break;
+      }
+    }
+    if (ok && n_it > 0) {
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (n_it - 1) & 1)) {
+        record_error(p.err, 450);
+        ok = false;
+      } else if (!flush_dq(n_it - 1)) {
+        ok = false;
+      }
+    }
+    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (!ok) {
+      *abort_flag = 1;
+    } else if (n_it > 0) {
+      // tcgen05.ld is warp-collective: every lane loads, only keys inside the
+      // sequence store. Warpgroup 0 writes dK (scaled, transposed RoPE),
+      // warpgroup 1 writes dV.
+      const bool store = key < p.s;
+      if (wg == 0) {
+        __nv_bfloat16* kr = p.dK + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
+        const float* cs = (p.rcos && store) ? p.rcos + (int64_t)key * (FB_HD / 2) : nullptr;
+        const float* sn = (p.rsin && store) ? p.rsin + (int64_t)key * (FB_HD / 2) : nullptr;
+#pragma unroll
+        for (int c = 0; c < FB_HD / 2 / 16; ++c) {  // pairs (i, i + 64), 16 at a time
+          uint32_t a[16], bb[16];
+          tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + c * 16, a);
+          tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + 64 + c * 16, bb);
+          tmem_ld_wait();
+          uint32_t w1[8], w2[8];
+#pragma unroll
+          for (int e = 0; e < 16; e += 2) {
+            float y1[2], y2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const float x1 = __uint_as_float(a[e + u]) * p.scale, x2 = __uint_as_float(bb[e + u]) * p.scale;
+              if (cs) {
+                const int i = c * 16 + e + u;
+                y1[u] = x1 * cs[i] + x2 * sn[i];
+                y2[u] = x2 * cs[i] - x1 * sn[i];
+              } else {
+                y1[u] = x1;
+                y2[u] = x2;
+              }
+            }
+            w1[e >> 1] = pack_bf16x2(y1[0], y1[1]);
+            w2[e >> 1] = pack_bf16x2(y2[0], y2[1]);
+          }
+          if (store) {
+            reinterpret_cast<uint4*>(kr + c * 16)[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+            reinterpret_cast<uint4*>(kr + c * 16)[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+            reinterpret_cast<uint4*>(kr + 64 + c * 16)[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+            reinterpret_cast<uint4*>(kr + 64 + c * 16)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+          }
+        }
+      } else {
+        __nv_bfloat16* vr = p.dV + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
+#pragma unroll
+        for (int c = 0; c < FB_HD / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem + lane_base + C::C_DV + c * 16, v);
+          tmem_ld_wait();
+          uint32_t w[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          if (store) {
+            reinterpret_cast<uint4*>(vr + c * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            reinterpret_cast<uint4*>(vr + c * 16)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// Backward with head_dim 128 on the tensor cores. a.dvec must already hold
+// D = rowsum(dO * O) and a.dq_acc must be zeroed; the caller casts dQ.
+int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
+  using C = FbCfg;
+  if (a.hd != FB_HD) return MT_ERR_CONFIG;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_flash_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return MT_ERR_CUDA;
+    attr = true;
+  }
+  const int64_t T = (int64_t)a.b * a.s;
+  CUtensorMap mq, mk, mv, mo, mdq;
+  if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * FB_HD, T, a.ldqkv, FB_BQ) ||
+      !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
+      !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ) ||
+      !make_tensor_map_2d_f32(&mdq, a.dq_acc, (int64_t)a.H * FB_HD, T, a.ldqa, 32, FB_BQ))
+    return MT_ERR_ARG;
+  FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
+             a.scale, a.rope_cos, a.rope_sin, err};
+  dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
+  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, p);
+  return launch_status();
 }
 
 }  // namespace mt

@@ -224,7 +224,8 @@ int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
     e1 = timing_event(c);
     if (e0) cudaEventRecord(e0, c->s_comp);
   }
-  int r = bwd ? attention_bwd(a, c->s_comp) : attention_fwd_tc(a, c->s_comp, c->d_err);
+  int r = bwd ? (a.hd == 128 ? attention_bwd_tc(a, c->s_comp, c->d_err) : attention_bwd(a, c->s_comp))
+              : attention_fwd_tc(a, c->s_comp, c->d_err);
   if (r != MT_OK) return set_err(c, r, "attention launch failed");
   c->launches += bwd ? 4 : 1;
   if (timing && e0 && e1) {
@@ -1131,6 +1132,49 @@ extern "C" int mt_get_params(mt_ctx* c, float* dst, size_t bytes) {
   if (!c || !dst) return MT_ERR_ARG;
   if (bytes < c->lay.total * 4) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
   memcpy(dst, c->arena, c->lay.total * 4);
+  return MT_OK;
+}
+
+extern "C" int mt_get_opt_state(mt_ctx* c, float* m_dst, float* v_dst, size_t bytes_each, int64_t* step) {
+  if (!c) return MT_ERR_ARG;
+  const size_t need = c->lay.total * 4;
+  if ((m_dst || v_dst) && bytes_each < need) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
+  if (m_dst) memcpy(m_dst, c->m, need);
+  if (v_dst) memcpy(v_dst, c->v, need);
+  if (step) *step = c->step;
+  return MT_OK;
+}
+
+extern "C" int mt_set_state(mt_ctx* c, const float* params, const float* m, const float* v, size_t bytes_each,
+                            int64_t step) {
+  if (!c) return MT_ERR_ARG;
+  const Layout& y = c->lay;
+  const Shapes& s = y.sh;
+  const size_t need = y.total * 4;
+  if ((params || m || v) && bytes_each < need) return set_err(c, MT_ERR_ARG, "source smaller than the arena");
+  if (step < 0 || step > (int64_t)1 << 30) return set_err(c, MT_ERR_ARG, "step out of range");
+  if (m) memcpy(c->m, m, need);
+  if (v) memcpy(c->v, v, need);
+  c->step = (int)step;
+  if (params) {
+    memcpy(c->arena, params, need);
+    // rebuild the bf16 streaming copies from the new master
+    for (int l = 0; l < s.L; ++l) {
+      uint16_t* blk = c->bf_layers + (size_t)l * y.bf_layer;
+      for (int tid = 0; tid < kLayerTensors; ++tid) {
+        const TRef& r = y.t(l, tid);
+        uint16_t* dst = blk + y.bf_of(tid);
+        parallel_ranges(*c->pool, r.n,
+                        [&](size_t b, size_t e) { bf16_round_chunk(c->arena + r.off + b, dst + b, e - b); });
+      }
+    }
+    parallel_ranges(*c->pool, y.embed.n,
+                    [&](size_t b, size_t e) { bf16_round_chunk(c->arena + y.embed.off + b, c->bf_embed + b, e - b); });
+    bf16_round_chunk(c->arena + y.final_norm.off, c->bf_head, s.d);
+    uint16_t* bhw = c->bf_head + align_up(s.d, 128);
+    parallel_ranges(*c->pool, y.head.n,
+                    [&](size_t b, size_t e) { bf16_round_chunk(c->arena + y.head.off + b, bhw + b, e - b); });
+  }
   return MT_OK;
 }
 

@@ -121,3 +121,23 @@ extern "C" int mt_k_gemm_bf16_rope(const void* A, int64_t lda, const void* B, in
                  mt::RopeDesc{cos_tab, sin_tab, rope_cols, hd, s}};
   return mt::gemm_bf16(g, static_cast<cudaStream_t>(stream), dev_err);
 }
+
+extern "C" int mt_k_attn_bwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o,
+                                const void* dout, int64_t ldo, const float* lse, float* dvec, float* dq_acc,
+                                int64_t ldqa, void* dq, int64_t lddq, void* dk, void* dv, int64_t lddkv, int b, int s,
+                                int H, int Hkv, int hd, const float* cos_tab, const float* sin_tab, void* stream,
+                                int32_t* dev_err) {
+  if ((cos_tab == nullptr) != (sin_tab == nullptr)) return MT_ERR_ARG;
+  if (!q || !k || !v || !o || !dout || !lse || !dvec || !dq_acc || !dq || !dk || !dv) return MT_ERR_ARG;
+  if (b < 0 || s < 0 || H <= 0 || Hkv <= 0 || (H % Hkv)) return MT_ERR_ARG;
+  if (hd != 128) return MT_ERR_CONFIG;
+  if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al16(dout) || !al16(dq_acc) || (ldqkv % 8) || (ldo % 8) ||
+      (ldqa % 4) || (lddq % 4) || (lddkv % 8) || ldqa < (int64_t)H * hd)
+    return MT_ERR_ARG;
+  mt::AttnArgs a{};
+  a.q = q; a.k = k; a.v = v; a.ldqkv = ldqkv; a.o = const_cast<void*>(o); a.ldo = ldo; a.lse = const_cast<float*>(lse);
+  a.dout = dout; a.dvec = dvec; a.dq_acc = dq_acc; a.ldqa = ldqa; a.dq = dq; a.lddq = lddq; a.dk = dk; a.dv = dv;
+  a.lddkv = lddkv; a.b = b; a.s = s; a.H = H; a.Hkv = Hkv; a.hd = hd; a.scale = 1.0f / std::sqrt((float)hd);
+  a.rope_cos = cos_tab; a.rope_sin = sin_tab;
+  return mt::attention_bwd_tc(a, S(stream), dev_err);
+}

@@ -51,6 +51,9 @@ int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
 // (elements), box {64, box_outer}, 128-byte swizzle, zero fill out of bounds.
 bool make_tensor_map_2d_bf16(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
                              int box_outer);
+// 2-D fp32 TMA map without swizzle, box {box_inner, box_outer}.
+bool make_tensor_map_2d_f32(CUtensorMap* m, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                            int box_inner, int box_outer);
 
 // Causal attention with grouped KV heads. q, k, v: column ranges of one bf16
 // row per token (pitch ldqkv); o, dout: [T, H*hd] bf16 (pitch ldo); lse, dvec:
@@ -84,6 +87,10 @@ int attention_fwd(const AttnArgs& a, cudaStream_t st);
 int attention_bwd(const AttnArgs& a, cudaStream_t st);
 // Forward on the tcgen05 tensor cores (same outputs as attention_fwd).
 int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
+// Backward on the tcgen05 tensor cores for head_dim 128 (same outputs as
+// attention_bwd); _main is the tensor-core kernel alone.
+int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
+int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* dev_err);
 
 int launch_rmsnorm_fwd(const float* x, const void* g, void* y, float* rstd, int T, int d, float eps, cudaStream_t st);
 int rmsnorm_bwd_blocks(int T);

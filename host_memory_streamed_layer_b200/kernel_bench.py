@@ -89,11 +89,12 @@ def bench_attn(iters, warmup, fwd_only, impl="tc"):
         dqa = torch.empty(T, H * HD, device="cuda")
         dqkv = torch.empty(T, ld, device="cuda", dtype=torch.bfloat16)
         dp = dqkv.data_ptr()
-        bwd = lambda: mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(),  # noqa
-                                       dvec.data_ptr(), dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD,
-                                       dp + 4 * H * HD, ld, B, S, H, H, HD, 0, 0, st)
+        fn = mt.mt_k_attn_bwd_tc if impl == "tc" else mt.mt_k_attn_bwd
+        bwd = lambda: fn(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(),  # noqa
+                         dvec.data_ptr(), dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD,
+                         dp + 4 * H * HD, ld, B, S, H, H, HD, 0, 0, st)
         sec = timed(bwd, iters, warmup)
-        res.append({"kernel": "attn_bwd", "us": sec * 1e6, "tflops": 2.5 * fl / sec / 1e12 if sec else None})
+        res.append({"kernel": f"attn_bwd_{impl}", "us": sec * 1e6, "tflops": 2.5 * fl / sec / 1e12 if sec else None})
     return res
 
 

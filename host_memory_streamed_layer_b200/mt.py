@@ -70,6 +70,9 @@ _sig("mt_k_attn_fwd_tc", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c
 _sig("mt_k_attn_bwd", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_void_p,
      c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p,
      c_void_p, c_void_p)
+_sig("mt_k_attn_bwd_tc", c_int, c_void_p, c_void_p, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_void_p, c_void_p,
+     c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_void_p, c_i64, c_int, c_int, c_int, c_int, c_int, c_void_p,
+     c_void_p, c_void_p, c_void_p)
 _sig("mt_k_gemm_bf16_rope", c_int, c_void_p, c_i64, c_void_p, c_i64, c_void_p, c_i64, c_int, c_int, c_int, c_int,
      c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p)
 
@@ -140,6 +143,13 @@ def mt_k_attn_bwd(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, ldd
                                     b, s, H, Hkv, hd, _p(cos_tab), _p(sin_tab), _p(stream)), "mt_k_attn_bwd")
 
 
+def mt_k_attn_bwd_tc(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv, b, s, H, Hkv,
+                     hd, cos_tab=0, sin_tab=0, stream=0, dev_err=0):
+    return _check(lib.mt_k_attn_bwd_tc(q, k, v, ldqkv, o, dout, ldo, lse, dvec, dq_acc, ldqa, dq, lddq, dk, dv, lddkv,
+                                       b, s, H, Hkv, hd, _p(cos_tab), _p(sin_tab), _p(stream), _p(dev_err)),
+                  "mt_k_attn_bwd_tc")
+
+
 def mt_k_gemm_bf16_rope(A, lda, B, ldb, C, ldc, M, N, K, rope_cols, hd, s, cos_tab, sin_tab, stream=0, dev_err=0):
     return _check(lib.mt_k_gemm_bf16_rope(A, lda, B, ldb, C, ldc, M, N, K, rope_cols, hd, s, cos_tab, sin_tab,
                                           _p(stream), _p(dev_err)), "mt_k_gemm_bf16_rope")
@@ -188,6 +198,8 @@ _sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
 _sig("mt_destroy", None, c_void_p)
 _sig("mt_get_stream", c_int, c_void_p, ctypes.POINTER(c_void_p))
 _sig("mt_host_optimizer_gbs", ctypes.c_double, c_size_t, c_int)
+_sig("mt_get_opt_state", c_int, c_void_p, c_void_p, c_void_p, c_size_t, ctypes.POINTER(ctypes.c_int64))
+_sig("mt_set_state", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, ctypes.c_int64)
 _sig("mt_last_error", ctypes.c_char_p, c_void_p)
 _sig("mt_k_adamw_host", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_float, c_float,
      c_float, c_float, c_float, c_int)
@@ -270,3 +282,15 @@ def mt_host_optimizer_gbs(n: int = 1 << 28, threads: int = 0) -> float:
     if r < 0:
         raise MTError(int(r), "mt_host_optimizer_gbs")
     return r
+
+
+def mt_get_opt_state(ctx: int, m_ptr: int, v_ptr: int, nbytes: int) -> int:
+    step = ctypes.c_int64()
+    _check(lib.mt_get_opt_state(ctx, m_ptr or None, v_ptr or None, nbytes, ctypes.byref(step)), "mt_get_opt_state",
+           ctx)
+    return step.value
+
+
+def mt_set_state(ctx: int, params_ptr: int, m_ptr: int, v_ptr: int, nbytes: int, step: int):
+    return _check(lib.mt_set_state(ctx, params_ptr or None, m_ptr or None, v_ptr or None, nbytes, step),
+                  "mt_set_state", ctx)

@@ -144,6 +144,18 @@ int mt_get_grads(mt_ctx* ctx, float* dst, size_t bytes);
 /* Copies the current fp32 master weights (after the last update) to dst. */
 int mt_get_params(mt_ctx* ctx, float* dst, size_t bytes);
 
+/* Checkpoint: copies the fp32 Adam moments m and v (arena layout, each at
+ * least mt_arena_bytes long) and the number of completed steps. The master
+ * weights come from mt_get_params. The host arena is the whole training state
+ * (MegaTrain keeps parameters and optimizer state in host memory). */
+int mt_get_opt_state(mt_ctx* ctx, float* m_dst, float* v_dst, size_t bytes_each, int64_t* step);
+
+/* Resume: replaces the master weights, both moments and the step counter
+ * (bias correction continues from step + 1) and rebuilds the bf16 streaming
+ * copies. Any pointer may be NULL to keep that part. Nothing runs on the GPU. */
+int mt_set_state(mt_ctx* ctx, const float* params, const float* m, const float* v, size_t bytes_each,
+                 int64_t step);
+
 /* Counters of the last step. */
 int mt_get_stats(mt_ctx* ctx, mt_stats* out);
 

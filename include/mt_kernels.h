@@ -142,6 +142,16 @@ int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_t ldqkv, co
                   void* dk, void* dv, int64_t lddkv, int b, int s, int H, int Hkv, int hd, const float* cos_tab,
                   const float* sin_tab, void* stream);
 
+/* The same backward (same arguments and outputs as mt_k_attn_bwd) on the
+ * tcgen05 tensor cores, head_dim 128 only (MT_ERR_CONFIG otherwise): one CTA
+ * per 128-key block accumulates dK and dV in tensor memory over the group's
+ * query heads and 64-query blocks; dQ goes through the fp32 accumulator.
+ * q, k, v, o, dout 16-byte aligned; dev_err as for mt_k_attn_fwd_tc. */
+int mt_k_attn_bwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o, const void* dout,
+                     int64_t ldo, const float* lse, float* dvec, float* dq_acc, int64_t ldqa, void* dq, int64_t lddq,
+                     void* dk, void* dv, int64_t lddkv, int b, int s, int H, int Hkv, int hd, const float* cos_tab,
+                     const float* sin_tab, void* stream, int32_t* dev_err);
+
 /* Forward projection with RoPE fused into the epilogue: C bf16 [M,N] =
  * rope(A[M,K] B[N,K]^T), both operands K-major as in mt_k_gemm_bf16. Columns
  * [0, rope_cols) are heads of width hd (64 or 128) whose rotate-half pairs are

@@ -73,7 +73,8 @@ def test_gemm_full_shape_sampled(name, M, N, K, form):
     assert np.all(np.abs(got - ref) <= bound), np.max(np.abs(got - ref) / bound)
 
 
-def test_attention_full_shape_sampled():
+@pytest.mark.parametrize("impl", ["mma", "tc"])
+def test_attention_full_shape_sampled(impl):
     mt = _mt()
     g = torch.Generator(device=DEV).manual_seed(7)
     ld = 3 * H * HD
@@ -89,8 +90,9 @@ def test_attention_full_shape_sampled():
     dqa = torch.empty(T, H * HD, device=DEV)
     dqkv = torch.empty(T, ld, device=DEV, dtype=torch.bfloat16)
     dp = dqkv.data_ptr()
-    mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(), dvec.data_ptr(),
-                     dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD, dp + 4 * H * HD, ld, B, S, H, H, HD)
+    bwd = mt.mt_k_attn_bwd if impl == "mma" else mt.mt_k_attn_bwd_tc
+    bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(), dvec.data_ptr(),
+        dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD, dp + 4 * H * HD, ld, B, S, H, H, HD)
     torch.cuda.synchronize()
     assert err.item() == 0
     Q = qkv.view(B, S, 3, H, HD)

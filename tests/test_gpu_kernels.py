@@ -219,8 +219,11 @@ def test_attention_fwd(hd, H, Hkv, s, b, impl):
     assert np.allclose(np64(lse), oracle.attention_lse(q, k), rtol=1e-4, atol=1e-4)
 
 
+@pytest.mark.parametrize("impl", ["mma", "tc"])
 @pytest.mark.parametrize("hd,H,Hkv,s,b", ATTN)
-def test_attention_bwd(hd, H, Hkv, s, b):
+def test_attention_bwd(hd, H, Hkv, s, b, impl):
+    if impl == "tc" and hd != 128:
+        pytest.skip("tensor-core backward is for head_dim 128")
     mt = _mt()
     qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, 7 * hd + s)
     T = b * s
@@ -235,9 +238,13 @@ def test_attention_bwd(hd, H, Hkv, s, b):
     dqa = torch.empty(T, H * hd, device=DEV)
     dqkv = torch.zeros(T, ld, dtype=torch.bfloat16, device=DEV)
     dp = dqkv.data_ptr()
-    mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(), dvec.data_ptr(),
-                     dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd, dp + 2 * (H + Hkv) * hd, ld, b, s, H, Hkv, hd)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    bwd = mt.mt_k_attn_bwd if impl == "mma" else mt.mt_k_attn_bwd_tc
+    kw = {} if impl == "mma" else {"dev_err": err.data_ptr()}
+    bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(), dvec.data_ptr(),
+        dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd, dp + 2 * (H + Hkv) * hd, ld, b, s, H, Hkv, hd, **kw)
     sync()
+    assert err.item() == 0
     ro, P = oracle.attention_fwd(q, k, v)
     rdq, rdk, rdv = oracle.attention_bwd(q, k, v, P, np64(do).reshape(b, s, H, hd))
     g = np64(dqkv)
@@ -280,8 +287,11 @@ def test_qkv_gemm_with_rope_epilogue(hd, H, Hkv, s, b):
     assert np.all(np.abs(got - ref) <= bound)
 
 
-@pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3)])
-def test_attention_bwd_returns_pre_rope_gradients(hd, H, Hkv, s, b):
+@pytest.mark.parametrize("impl", ["mma", "tc"])
+@pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 2, 1, 300, 2)])
+def test_attention_bwd_returns_pre_rope_gradients(hd, H, Hkv, s, b, impl):
+    if impl == "tc" and hd != 128:
+        pytest.skip("tensor-core backward is for head_dim 128")
     """With the RoPE tables the backward returns dL/d(pre-RoPE q, k): the
     oracle's attention backward followed by its rope_bwd."""
     mt = _mt()
@@ -300,9 +310,10 @@ def test_attention_bwd_returns_pre_rope_gradients(hd, H, Hkv, s, b):
     dqa = torch.empty(T, H * hd, device=DEV)
     dqkv = torch.zeros(T, ld, dtype=torch.bfloat16, device=DEV)
     dp = dqkv.data_ptr()
-    mt.mt_k_attn_bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(), dvec.data_ptr(),
-                     dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd, dp + 2 * (H + Hkv) * hd, ld, b, s, H, Hkv, hd,
-                     c32.data_ptr(), s32.data_ptr())
+    bwd = mt.mt_k_attn_bwd if impl == "mma" else mt.mt_k_attn_bwd_tc
+    bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(), dvec.data_ptr(),
+        dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd, dp + 2 * (H + Hkv) * hd, ld, b, s, H, Hkv, hd,
+        c32.data_ptr(), s32.data_ptr())
     sync()
     _, P = oracle.attention_fwd(q, k, v)
     rdq, rdk, rdv = oracle.attention_bwd(q, k, v, P, np64(do).reshape(b, s, H, hd))

@@ -180,3 +180,35 @@ def test_chunked_head_matches_oracle(monkeypatch):
     assert abs(g["loss"] - r["loss"]) <= 1e-2
     G = oracle.unpack_arena(g["G"], c)
     assert max(rel(G[k], r["G"][k]) for k in r["G"]) <= 2e-2
+
+
+def test_checkpoint_resume_continues_the_trajectory():
+    """Train two steps in one context; in a second context restore the state
+    saved after step 1 and run step 2: same loss and same updated master."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    shape = SHAPES["tiny"]
+    cfg = arena.config(shape)
+    A = arena.pack(cfg, synth.init_weights(shape, 0))
+    n = A.size
+    toks = [synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, k) for k in range(2)]
+    ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+    try:
+        mt.mt_train_step(ctx, toks[0][0].ctypes.data, toks[0][1].ctypes.data)
+        P1 = A.copy()
+        M1, V1 = np.empty(n, np.float32), np.empty(n, np.float32)
+        step = mt.mt_get_opt_state(ctx, M1.ctypes.data, V1.ctypes.data, M1.nbytes)
+        loss2 = mt.mt_train_step(ctx, toks[1][0].ctypes.data, toks[1][1].ctypes.data)
+        P2 = A.copy()
+    finally:
+        mt.mt_destroy(ctx)
+    assert step == 1 and np.abs(M1).max() > 0 and np.abs(V1).max() > 0
+    B = arena.pack(cfg, synth.init_weights(shape, 42))  # different start, overwritten by the restore
+    ctx = mt.mt_create(cfg, B.ctypes.data, B.nbytes)
+    try:
+        mt.mt_set_state(ctx, P1.ctypes.data, M1.ctypes.data, V1.ctypes.data, P1.nbytes, step)
+        loss2b = mt.mt_train_step(ctx, toks[1][0].ctypes.data, toks[1][1].ctypes.data)
+        P2b = B.copy()
+    finally:
+        mt.mt_destroy(ctx)
+    assert abs(loss2 - loss2b) <= 1e-5
+    assert rel(P2b, P2) <= 1e-5
