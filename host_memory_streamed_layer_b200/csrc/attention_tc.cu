@@ -22,6 +22,8 @@
 //
 // Every mbarrier wait is bounded (mt_common.cuh); on expiry the kernel records
 // an error code, drains its copies and MMAs (bounded) and returns.
+#include <type_traits>
+
 #include "mt_common.cuh"
 #include "mt_internal.h"
 
@@ -280,52 +282,61 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         break;
       }
       tc_fence_after();
-      const bool diag = (j == nkv - 1);
       const uint32_t sbase = tmem + lane_base + C::S_COL + sb * FA_BKV;
-      // pass 1: row max of the visible scores (whole row)
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < FA_BKV / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(sbase + c * 16, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float x = __uint_as_float(v[e]);
-          if (!diag || c * 16 + e <= r) mx = fmaxf(mx, x);
-        }
-      }
-      const float mnew = fmaxf(m, mx);
-      const float corr = (m == -INFINITY) ? 0.f : ex2((m - mnew) * sl2);
-      const float mb = mnew * sl2;
-      // pass 2: this warpgroup's 64 keys -> probabilities, partial row sum,
-      // bf16 P into swizzle sub-tile wg of the A operand
       uint8_t* prow = sP + sb * C::P_BYTES + wg * 16384 + r * 128;
-      float rs = 0.f;
+      float corr, rs;
+      // The causal mask only touches the diagonal block: the other blocks run
+      // an instantiation without any per-element test.
+      auto block = [&](auto diag_tag) {
+        constexpr bool DIAG = decltype(diag_tag)::value;
+        // pass 1: row max of the visible scores (whole row)
+        float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(sbase + wg * 64 + c * 16, v);
-        tmem_ld_wait();
+        for (int c = 0; c < FA_BKV / 16; ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(sbase + c * 16, v);
+          tmem_ld_wait();
 #pragma unroll
-        for (int q = 0; q < 2; ++q) {  // two 16-byte chunks of 8 keys
-          uint32_t pk[4];
-#pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const int col = wg * 64 + c * 16 + q * 8 + e;
-            float p0 = ex2(__uint_as_float(v[q * 8 + e]) * sl2 - mb);
-            float p1 = ex2(__uint_as_float(v[q * 8 + e + 1]) * sl2 - mb);
-            if (diag && col > r) p0 = 0.f;
-            if (diag && col + 1 > r) p1 = 0.f;
-            rs += p0 + p1;
-            pk[e >> 1] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 16; ++e) {
+            const float x = __uint_as_float(v[e]);
+            if (!DIAG || c * 16 + e <= r) mx = fmaxf(mx, x);
           }
-          const int chunk = c * 2 + q;  // 0..7 inside the 64-key sub-tile
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
-      }
+        const float mnew = fmaxf(m, mx);
+        corr = (m == -INFINITY) ? 0.f : ex2((m - mnew) * sl2);
+        const float mb = mnew * sl2;
+        m = mnew;
+        // pass 2: this warpgroup's 64 keys -> probabilities, partial row sum,
+        // bf16 P into swizzle sub-tile wg of the A operand
+        rs = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(sbase + wg * 64 + c * 16, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {  // two 16-byte chunks of 8 keys
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+              const int col = wg * 64 + c * 16 + q * 8 + e;
+              float p0 = ex2(fmaf(__uint_as_float(v[q * 8 + e]), sl2, -mb));
+              float p1 = ex2(fmaf(__uint_as_float(v[q * 8 + e + 1]), sl2, -mb));
+              if (DIAG && col > r) p0 = 0.f;
+              if (DIAG && col + 1 > r) p1 = 0.f;
+              rs += p0 + p1;
+              pk[e >> 1] = pack_bf16x2(p0, p1);
+            }
+            const int chunk = c * 2 + q;  // 0..7 inside the 64-key sub-tile
+            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      };
+      if (j == nkv - 1)
+        block(std::true_type{});
+      else
+        block(std::false_type{});
       l = l * corr + rs;
-      m = mnew;
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
@@ -721,31 +732,41 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         break;
       }
       tc_fence_after();
-      // P^T and dS^T of this key row for this warpgroup's 32 queries (bf16 pairs)
+      // P^T and dS^T of this key row for this warpgroup's 32 queries (bf16 pairs).
+      // Only blocks that touch the diagonal or a sequence end need the mask.
       uint32_t pp[16], ds[16];
+      auto grads = [&](auto mask_tag) {
+        constexpr bool MASK = decltype(mask_tag)::value;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t sv[16], dv[16];
-        const uint32_t cb = tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + wg * 32 + c * 16;
-        tmem_ld_32x32b_x16(cb, sv);
-        tmem_ld_32x32b_x16(cb + C::C_DP_OFF, dv);
-        tmem_ld_wait();
+        for (int c = 0; c < 2; ++c) {
+          uint32_t sv[16], dv[16];
+          const uint32_t cb = tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + wg * 32 + c * 16;
+          tmem_ld_32x32b_x16(cb, sv);
+          tmem_ld_32x32b_x16(cb + C::C_DP_OFF, dv);
+          tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; e += 2) {
-          float pv[2], dsv[2];
+          for (int e = 0; e < 16; e += 2) {
+            float pv[2], dsv[2];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int cq = c * 16 + e + u;
-            const int qi = q0 + wg * 32 + cq;
-            const bool vis = key <= qi && qi < p.s && key < p.s;
-            const float pr = vis ? ex2(__uint_as_float(sv[e + u]) * sl2 - __ldg(lse + cq) * 1.4426950408889634f) : 0.f;
-            pv[u] = pr;
-            dsv[u] = vis ? pr * (__uint_as_float(dv[e + u]) - __ldg(dd + cq)) : 0.f;
+            for (int u = 0; u < 2; ++u) {
+              const int cq = c * 16 + e + u;
+              const int qi = q0 + wg * 32 + cq;
+              const bool vis = !MASK || (key <= qi && qi < p.s && key < p.s);
+              const float pr =
+                  vis ? ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -__ldg(lse + cq) * 1.4426950408889634f)) : 0.f;
+              pv[u] = pr;
+              dsv[u] = vis ? pr * (__uint_as_float(dv[e + u]) - __ldg(dd + cq)) : 0.f;
+            }
+            pp[(c * 16 + e) >> 1] = pack_bf16x2(pv[0], pv[1]);
+            ds[(c * 16 + e) >> 1] = pack_bf16x2(dsv[0], dsv[1]);
           }
-          pp[(c * 16 + e) >> 1] = pack_bf16x2(pv[0], pv[1]);
-          ds[(c * 16 + e) >> 1] = pack_bf16x2(dsv[0], dsv[1]);
         }
-      }
+      };
+      const bool need_mask = (q0 + wg * 32 < kv0 + FB_BKV) || (q0 + FB_BQ > p.s) || (kv0 + FB_BKV > p.s);
+      if (need_mask)
+        grads(std::true_type{});
+      else
+        grads(std::false_type{});
       // dV, dK, dQ^T of the previous iteration must be done with the tiles
       if (it > 0 && (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1))) {
         record_error(p.err, 400 + (it & 63));
