@@ -76,22 +76,28 @@ __global__ void k_rmsnorm_fwd(const float* __restrict__ x, const bf16* __restric
 // RMSNorm backward. For y_j = g_j x_j r, r = (mean x^2 + eps)^-1/2:
 //   dx_j = dres_j + r g_j dy_j - x_j r^3 (sum_i g_i dy_i x_i) / d
 //   dg_j = sum over rows of dy_j x_j r      (per-block partials, fixed order)
-// Block of 256 threads owns a contiguous chunk of rows; thread t owns the
-// float4 column groups t, t+256, ... (d <= 256 * 4 * KMAX).
+// A block of 256 threads owns a contiguous chunk of rows and takes them R at a
+// time; thread t owns the float4 column groups t, t + 256, ... (K4 of them,
+// d <= 1024 K4). The R rows' dot products are reduced together, with one
+// barrier per group, so that R rows of loads are in flight per block; the
+// reduction buffer alternates between two halves so the next group's writes
+// cannot race this group's reads. Two blocks fit an SM.
 // ---------------------------------------------------------------------------
 constexpr int RMS_KMAX = 8;
 
-__global__ void __launch_bounds__(256) k_rmsnorm_bwd(const float* __restrict__ x, const bf16* __restrict__ g,
-                                                     const float* __restrict__ rstd, const float* __restrict__ dy,
-                                                     const float* __restrict__ dres, float* __restrict__ dx,
-                                                     bf16* __restrict__ dx_bf16, float* __restrict__ dg_part,
-                                                     int T, int d, int rows_per_block) {
-  __shared__ float sh[8];
+template <int K4, int R>
+__global__ void __launch_bounds__(256, 2) k_rmsnorm_bwd(const float* __restrict__ x, const bf16* __restrict__ g,
+                                                        const float* __restrict__ rstd, const float* __restrict__ dy,
+                                                        const float* __restrict__ dres, float* __restrict__ dx,
+                                                        bf16* __restrict__ dx_bf16, float* __restrict__ dg_part,
+                                                        int T, int d, int rows_per_block) {
+  __shared__ float red[2][8][R];
   const int n4 = d >> 2;
-  float gv[RMS_KMAX][4];
-  float acc[RMS_KMAX][4];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float gv[K4][4];
+  float acc[K4][4];
 #pragma unroll
-  for (int k = 0; k < RMS_KMAX; ++k) {
+  for (int k = 0; k < K4; ++k) {
     const int c = threadIdx.x + k * 256;
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[k][e] = 0.f;
@@ -104,55 +110,106 @@ __global__ void __launch_bounds__(256) k_rmsnorm_bwd(const float* __restrict__ x
   }
   const int r0 = blockIdx.x * rows_per_block;
   const int r1 = min(T, r0 + rows_per_block);
-  for (int row = r0; row < r1; ++row) {
-    const float4* xr = reinterpret_cast<const float4*>(x + (int64_t)row * d);
-    const float4* dyr = reinterpret_cast<const float4*>(dy + (int64_t)row * d);
-    const float r = rstd[row];
-    float4 xv[RMS_KMAX], dv[RMS_KMAX];
-    float dot = 0.f;
+  int half = 0;
+  for (int row0 = r0; row0 < r1; row0 += R, half ^= 1) {
+    float4 xv[R][K4], dv[R][K4];
+    float rr[R], dot[R];
 #pragma unroll
-    for (int k = 0; k < RMS_KMAX; ++k) {
-      const int c = threadIdx.x + k * 256;
-      if (c < n4) {
-        xv[k] = xr[c];
-        dv[k] = dyr[c];
-        dot += gv[k][0] * dv[k].x * xv[k].x + gv[k][1] * dv[k].y * xv[k].y + gv[k][2] * dv[k].z * xv[k].z +
-               gv[k][3] * dv[k].w * xv[k].w;
+    for (int q = 0; q < R; ++q) {
+      const int row = row0 + q;
+      const bool ok = row < r1;
+      rr[q] = ok ? rstd[row] : 0.f;
+      dot[q] = 0.f;
+#pragma unroll
+      for (int k = 0; k < K4; ++k) {
+        const int c = threadIdx.x + k * 256;
+        if (ok && c < n4) {
+          xv[q][k] = reinterpret_cast<const float4*>(x + (int64_t)row * d)[c];
+          dv[q][k] = reinterpret_cast<const float4*>(dy + (int64_t)row * d)[c];
+        } else {
+          xv[q][k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          dv[q][k] = xv[q][k];
+        }
       }
     }
-    dot = block_sum_256(dot, sh);
-    const float c3 = r * r * r * dot / (float)d;
 #pragma unroll
-    for (int k = 0; k < RMS_KMAX; ++k) {
-      const int c = threadIdx.x + k * 256;
-      if (c < n4) {
-        float4 o;
-        o.x = r * gv[k][0] * dv[k].x - xv[k].x * c3;
-        o.y = r * gv[k][1] * dv[k].y - xv[k].y * c3;
-        o.z = r * gv[k][2] * dv[k].z - xv[k].z * c3;
-        o.w = r * gv[k][3] * dv[k].w - xv[k].w * c3;
-        if (dres) {
-          const float4 q = reinterpret_cast<const float4*>(dres + (int64_t)row * d)[c];
-          o.x += q.x;
-          o.y += q.y;
-          o.z += q.z;
-          o.w += q.w;
+    for (int q = 0; q < R; ++q) {
+#pragma unroll
+      for (int k = 0; k < K4; ++k)
+        dot[q] += gv[k][0] * dv[q][k].x * xv[q][k].x + gv[k][1] * dv[q][k].y * xv[q][k].y +
+                  gv[k][2] * dv[q][k].z * xv[q][k].z + gv[k][3] * dv[q][k].w * xv[q][k].w;
+      dot[q] = warp_sum(dot[q]);
+    }
+    if (lane == 0) {
+#pragma unroll
+      for (int q = 0; q < R; ++q) red[half][warp][q] = dot[q];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < R; ++q) {
+      const int row = row0 + q;
+      if (row >= r1) break;
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) tot += red[half][w][q];
+      const float r = rr[q];
+      const float c3 = r * r * r * tot / (float)d;
+#pragma unroll
+      for (int k = 0; k < K4; ++k) {
+        const int c = threadIdx.x + k * 256;
+        if (c < n4) {
+          const float4 dq = dv[q][k], xq = xv[q][k];
+          float4 o;
+          o.x = r * gv[k][0] * dq.x - xq.x * c3;
+          o.y = r * gv[k][1] * dq.y - xq.y * c3;
+          o.z = r * gv[k][2] * dq.z - xq.z * c3;
+          o.w = r * gv[k][3] * dq.w - xq.w * c3;
+          if (dres) {
+            const float4 s = reinterpret_cast<const float4*>(dres + (int64_t)row * d)[c];
+            o.x += s.x;
+            o.y += s.y;
+            o.z += s.z;
+            o.w += s.w;
+          }
+          reinterpret_cast<float4*>(dx + (int64_t)row * d)[c] = o;
+          if (dx_bf16) store_bf16x4(dx_bf16 + (int64_t)row * d + 4 * c, o.x, o.y, o.z, o.w);
+          acc[k][0] += dq.x * xq.x * r;
+          acc[k][1] += dq.y * xq.y * r;
+          acc[k][2] += dq.z * xq.z * r;
+          acc[k][3] += dq.w * xq.w * r;
         }
-        reinterpret_cast<float4*>(dx + (int64_t)row * d)[c] = o;
-        if (dx_bf16) store_bf16x4(dx_bf16 + (int64_t)row * d + 4 * c, o.x, o.y, o.z, o.w);
-        acc[k][0] += dv[k].x * xv[k].x * r;
-        acc[k][1] += dv[k].y * xv[k].y * r;
-        acc[k][2] += dv[k].z * xv[k].z * r;
-        acc[k][3] += dv[k].w * xv[k].w * r;
       }
     }
   }
 #pragma unroll
-  for (int k = 0; k < RMS_KMAX; ++k) {
+  for (int k = 0; k < K4; ++k) {
     const int c = threadIdx.x + k * 256;
     if (c < n4)
       reinterpret_cast<float4*>(dg_part + (int64_t)blockIdx.x * d)[c] =
           make_float4(acc[k][0], acc[k][1], acc[k][2], acc[k][3]);
+  }
+}
+
+// Rows in flight per block: as many as keep the loads of a group within ~64
+// registers per thread.
+template <int K4>
+void rmsnorm_bwd_k4(int nb, const float* x, const bf16* g, const float* rstd, const float* dy, const float* dres,
+                    float* dx, bf16* dxb, float* part, int T, int d, int rpb, cudaStream_t st) {
+  constexpr int R = K4 >= 5 ? 1 : 8 / K4;
+  k_rmsnorm_bwd<K4, R><<<nb, 256, 0, st>>>(x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb);
+}
+
+void rmsnorm_bwd_kernel(int nb, const float* x, const bf16* g, const float* rstd, const float* dy, const float* dres,
+                        float* dx, bf16* dxb, float* part, int T, int d, int rpb, cudaStream_t st) {
+  switch (((d >> 2) + 255) / 256) {
+    case 1: rmsnorm_bwd_k4<1>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    case 2: rmsnorm_bwd_k4<2>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    case 3: rmsnorm_bwd_k4<3>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    case 4: rmsnorm_bwd_k4<4>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    case 5: rmsnorm_bwd_k4<5>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    case 6: rmsnorm_bwd_k4<6>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    case 7: rmsnorm_bwd_k4<7>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
+    default: rmsnorm_bwd_k4<8>(nb, x, g, rstd, dy, dres, dx, dxb, part, T, d, rpb, st); break;
   }
 }
 
@@ -393,7 +450,7 @@ int launch_rmsnorm_bwd(const float* x, const void* g, const float* rstd, const f
   if (d > 256 * 4 * RMS_KMAX) return MT_ERR_CONFIG;
   const int nb = rmsnorm_bwd_blocks(T);
   const int rpb = (T + nb - 1) / nb;
-  k_rmsnorm_bwd<<<nb, 256, 0, st>>>(x, (const bf16*)g, rstd, dy, dres, dx, (bf16*)dx_bf16, dg_part, T, d, rpb);
+  rmsnorm_bwd_kernel(nb, x, (const bf16*)g, rstd, dy, dres, dx, (bf16*)dx_bf16, dg_part, T, d, rpb, st);
   k_sum_rows<<<nblk(d, 256), 256, 0, st>>>(dg_part, nb, d, dg);
   return launch_status();
 }
@@ -508,7 +565,7 @@ extern "C" int mt_k_rmsnorm_bwd_noalloc(const float* x, const void* g, const flo
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // Every block writes its own partial row (zeros when it owns no rows), so
   // stale contents from an earlier call are never read.
-  k_rmsnorm_bwd<<<nb, 256, 0, st>>>(x, (const bf16*)g, rstd, dy, dres, dx, (bf16*)dx_bf16, part, T, d, rpb);
+  rmsnorm_bwd_kernel(nb, x, (const bf16*)g, rstd, dy, dres, dx, (bf16*)dx_bf16, part, T, d, rpb, st);
   k_sum_rows<<<nblk(d, 256), 256, 0, st>>>(part, nb, d, dg);
   return launch_status();
 }

@@ -69,8 +69,9 @@ inline float normal_at(uint64_t key, uint64_t i) {
 struct Job {
   enum Kind { LAYER, HEAD, EMBED, EMBED_UNTOUCHED } kind;
   int layer;
-  cudaEvent_t ready;  // offload of this job's gradients has completed
-  int flag_index;     // index in the finite-flag array
+  cudaEvent_t ready;         // offload of this job's gradients has completed
+  int flag_index;            // index in the finite-flag array
+  const float* g = nullptr;  // LAYER: host gradient of the layer's first element
 };
 
 }  // namespace
@@ -90,7 +91,10 @@ struct mt_ctx {
   bool arena_owned = false;
   float* m = nullptr;  // Adam moments (pageable, 64-byte aligned)
   float* v = nullptr;
-  float* grad = nullptr;          // pinned fp32 gradient arena
+  float* grad = nullptr;          // pinned fp32 gradient arena (not with MT_FLAG_GRAD_RING)
+  float* ring = nullptr;          // pinned gradient ring of MT_GRAD_RING_SLOTS layer slots
+  float* grad_head = nullptr;     // [final norm | LM head] gradients: inside grad, or own buffer
+  size_t layer_f = 0;             // floats of one layer's gradient block
   uint16_t* bf_layers = nullptr;  // pinned bf16 layer blocks
   uint16_t* bf_embed = nullptr;   // pinned bf16 embedding (read by the GPU in place)
   uint16_t* bf_head = nullptr;    // pinned bf16 [final norm | LM head]
@@ -138,6 +142,7 @@ struct mt_ctx {
   std::condition_variable opt_cv, opt_done_cv;
   std::deque<Job> jobs;
   int jobs_pending = 0;
+  int layer_jobs_done = 0;  // LAYER jobs finished this step: ring slots released
   bool opt_stop = false;
   int opt_status = MT_OK;
   bool skip_updates = false;
@@ -414,8 +419,9 @@ bool wait_event(mt_ctx* c, cudaEvent_t e) {
 }
 
 struct Seg {
-  size_t off, n;    // floats in the arena
-  uint16_t* bf;     // bf16 destination of element 0
+  size_t off, n;       // floats in the arena
+  uint16_t* bf;        // bf16 destination of element 0
+  const float* g;      // gradient of element 0; nullptr: zero gradient
 };
 
 void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
@@ -426,12 +432,13 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
   struct Task {
     size_t off, n;
     uint16_t* bf;
+    const float* g;
   };
   std::vector<Task> tasks;
   size_t total = 0;
   for (const Seg& sg : segs) {
     for (size_t i = 0; i < sg.n; i += chunk)
-      tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf ? sg.bf + i : nullptr});
+      tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf ? sg.bf + i : nullptr, sg.g ? sg.g + i : nullptr});
     total += sg.n;
   }
   if (tasks.empty()) return;
@@ -440,7 +447,7 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
   if (c->adamw_first == 0) c->adamw_first = t0;
   c->pool->run((int)tasks.size(), [&](int i) {
     const Task& k = tasks[i];
-    adamw_chunk(c->arena + k.off, c->grad + k.off, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
+    adamw_chunk(c->arena + k.off, k.g, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
   });
   c->adamw_last = now_s();
   c->adamw_s += c->adamw_last - t0;
@@ -459,16 +466,19 @@ void run_job(mt_ctx* c, const Job& j) {
   if (j.kind == Job::EMBED_UNTOUCHED) {
     // Rows no token of this batch touches have a zero gradient, so their update
     // does not depend on this step's backward and runs while the GPU is in the
-    // forward sweep (the gather reads only the touched rows). Zero last step's
-    // touched gradient rows first: every row's gradient this step is then 0
-    // until the touched rows are scattered at the end.
-    float* ge = c->grad + y.embed.off;
+    // forward sweep (the gather reads only the touched rows); it reads no
+    // gradient at all. With a gradient arena, zero last step's touched rows
+    // first: every row's stored gradient is then 0 until the touched rows are
+    // scattered at the end.
     const size_t d = s.d;
-    const int nt = c->pool->size() * 4;
-    const size_t np = c->prev_uniq.size();
-    c->pool->run(nt, [&](int i) {
-      for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k) memset(ge + (size_t)c->prev_uniq[k] * d, 0, d * 4);
-    });
+    if (c->grad) {
+      float* ge = c->grad + y.embed.off;
+      const int nt = c->pool->size() * 4;
+      const size_t np = c->prev_uniq.size();
+      c->pool->run(nt, [&](int i) {
+        for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k) memset(ge + (size_t)c->prev_uniq[k] * d, 0, d * 4);
+      });
+    }
     c->prev_uniq = c->uniq;
     if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
     std::vector<Seg> segs;
@@ -476,15 +486,18 @@ void run_job(mt_ctx* c, const Job& j) {
     for (size_t u = 0; u <= c->uniq.size(); ++u) {
       const int32_t stop = u < c->uniq.size() ? c->uniq[u] : s.V;
       if (stop > next)
-        segs.push_back({y.embed.off + (size_t)next * d, (size_t)(stop - next) * d, c->bf_embed + (size_t)next * d});
+        segs.push_back(
+            {y.embed.off + (size_t)next * d, (size_t)(stop - next) * d, c->bf_embed + (size_t)next * d, nullptr});
       next = stop + 1;
     }
     adamw_segments(c, segs);
     return;
   }
   if (j.kind == Job::EMBED) {
-    // Touched rows: scatter this step's gradient rows (checking for NaN/Inf).
-    float* ge = c->grad + y.embed.off;
+    // Touched rows: check this step's gradient rows for NaN/Inf (and scatter
+    // them into the gradient arena when there is one). The update reads them
+    // from the staging rows.
+    float* ge = c->grad ? c->grad + y.embed.off : nullptr;
     const size_t d = s.d;
     const int nt = c->pool->size() * 4;
     const size_t nu = c->uniq.size();
@@ -496,7 +509,7 @@ void run_job(mt_ctx* c, const Job& j) {
         float acc = 0.f;
         for (size_t k = 0; k < d; ++k) acc += src[k] * 0.f;  // NaN or Inf anywhere makes acc NaN
         b |= !(acc == 0.f);
-        memcpy(ge + (size_t)c->uniq[u] * d, src, d * sizeof(float));
+        if (ge) memcpy(ge + (size_t)c->uniq[u] * d, src, d * sizeof(float));
       }
       bad[i] = b;
     });
@@ -516,13 +529,16 @@ void run_job(mt_ctx* c, const Job& j) {
     uint16_t* blk = c->bf_layers + (size_t)j.layer * y.bf_layer;
     for (int tid = 0; tid < kLayerTensors; ++tid) {
       const TRef& r = y.t(j.layer, tid);
-      segs.push_back({r.off, r.n, blk + y.bf_of(tid)});
+      segs.push_back({r.off, r.n, blk + y.bf_of(tid), j.g + (r.off - y.layer_begin(j.layer))});
     }
   } else if (j.kind == Job::HEAD) {
-    segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head});
-    segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(s.d, 128)});
+    segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head, c->grad_head});
+    segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(s.d, 128), c->grad_head + (y.head.off - y.final_norm.off)});
   } else {
-    for (int32_t r : c->uniq) segs.push_back({y.embed.off + (size_t)r * s.d, (size_t)s.d, c->bf_embed + (size_t)r * s.d});
+    for (size_t u = 0; u < c->uniq.size(); ++u) {
+      const size_t r = (size_t)c->uniq[u];
+      segs.push_back({y.embed.off + r * s.d, (size_t)s.d, c->bf_embed + r * s.d, c->emb_rows_h + u * s.d});
+    }
   }
   adamw_segments(c, segs);
 }
@@ -541,6 +557,7 @@ void opt_loop(mt_ctx* c) {
     {
       std::lock_guard<std::mutex> lk(c->opt_mu);
       --c->jobs_pending;
+      if (j.kind == Job::LAYER) ++c->layer_jobs_done;
     }
     c->opt_done_cv.notify_all();
   }
@@ -582,16 +599,27 @@ int issue_head_load(mt_ctx* c) {
   return MT_OK;
 }
 
+// Backward index k (layer l = L-1-k): D2H of the layer's gradients into the
+// gradient arena, or into ring slot k mod MT_GRAD_RING_SLOTS once the update
+// of backward index k - MT_GRAD_RING_SLOTS (the slot's previous user) is done.
 int offload_layer(mt_ctx* c, int l, int k) {
   const Layout& y = c->lay;
   const size_t b = y.layer_begin(l), e = y.layer_end(l);
+  float* dst = c->grad ? c->grad + b : c->ring + (size_t)(k % MT_GRAD_RING_SLOTS) * c->layer_f;
+  if (!c->grad && k >= MT_GRAD_RING_SLOTS) {
+    std::unique_lock<std::mutex> lk(c->opt_mu);
+    const int need = k - MT_GRAD_RING_SLOTS + 1;
+    if (!c->opt_done_cv.wait_for(lk, std::chrono::duration<double>(c->wait_limit_s),
+                                 [&] { return c->layer_jobs_done >= need; }))
+      return set_err(c, MT_ERR_TIMEOUT, "gradient ring: no slot was released within the wait limit");
+  }
   CK(cudaEventRecord(c->ev_gready[k], c->s_comp));
   CK(cudaStreamWaitEvent(c->s_d2h, c->ev_gready[k], 0));
   CK(cudaEventRecord(c->ev_d2h_start[k], c->s_d2h));
-  CK(cudaMemcpyAsync(c->grad + b, c->gslot[k & 1], (e - b) * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  CK(cudaMemcpyAsync(dst, c->gslot[k & 1], (e - b) * 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaMemcpyAsync(c->flags_h + l, c->d_flags + l, 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaEventRecord(c->ev_gdrained[k], c->s_d2h));
-  push_job(c, Job{Job::LAYER, l, c->ev_gdrained[k], l});
+  push_job(c, Job{Job::LAYER, l, c->ev_gdrained[k], l, dst});
   return MT_OK;
 }
 
@@ -626,7 +654,7 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         CK(cudaStreamWaitEvent(c->s_d2h, c->ev_head_gready, 0));
         CK(cudaEventRecord(c->ev_head_d2h_start, c->s_d2h));
         const size_t n = y.head.off + y.head.n - y.final_norm.off;
-        CK(cudaMemcpyAsync(c->grad + y.final_norm.off, c->d_head_g, n * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+        CK(cudaMemcpyAsync(c->grad_head, c->d_head_g, n * 4, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaMemcpyAsync(c->flags_h + L, c->d_flags + L, 4, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaEventRecord(c->ev_head_drained, c->s_d2h));
         push_job(c, Job{Job::HEAD, -1, c->ev_head_drained, L});
@@ -802,8 +830,9 @@ void free_all(mt_ctx* c) {
   if (c->s_h2d && c->s_h2d != c->s_comp) cudaStreamDestroy(c->s_h2d);
   if (c->s_d2h && c->s_d2h != c->s_comp && c->s_d2h != c->s_h2d) cudaStreamDestroy(c->s_d2h);
   if (c->dmem) cudaFree(c->dmem);
-  for (void* p : {(void*)c->grad, (void*)c->bf_layers, (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h,
-                  (void*)c->stage_i, (void*)c->flags_h, (void*)c->misc_h})
+  for (void* p : {(void*)c->grad, (void*)c->ring, (void*)(c->grad ? nullptr : c->grad_head), (void*)c->bf_layers,
+                  (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h, (void*)c->stage_i, (void*)c->flags_h,
+                  (void*)c->misc_h})
     if (p) cudaFreeHost(p);
   free(c->m);
   free(c->v);
@@ -875,8 +904,21 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
       posix_memalign(reinterpret_cast<void**>(&c->v), 64, y.total * 4))
     return fail(MT_ERR_NOMEM, "host moment allocation failed");
   const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
-  if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * 4, cudaHostAllocPortable) != cudaSuccess ||
-      cudaHostAlloc(reinterpret_cast<void**>(&c->bf_layers), (size_t)s.L * y.bf_layer * 2, cudaHostAllocPortable) !=
+  const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
+  c->layer_f = y.layer_end(0) - y.layer_begin(0);
+  for (int l = 1; l < s.L; ++l)
+    if (y.layer_end(l) - y.layer_begin(l) != c->layer_f) return fail(MT_ERR_CONFIG, "layer blocks differ in size");
+  if (cfg->flags & MT_FLAG_GRAD_RING) {
+    if (cudaHostAlloc(reinterpret_cast<void**>(&c->ring), (size_t)MT_GRAD_RING_SLOTS * c->layer_f * 4,
+                      cudaHostAllocPortable) != cudaSuccess ||
+        cudaHostAlloc(reinterpret_cast<void**>(&c->grad_head), head_f * 4, cudaHostAllocPortable) != cudaSuccess)
+      return fail(MT_ERR_PIN, "pinned gradient ring allocation failed");
+  } else {
+    if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * 4, cudaHostAllocPortable) != cudaSuccess)
+      return fail(MT_ERR_PIN, "pinned gradient arena allocation failed");
+    c->grad_head = c->grad + y.final_norm.off;
+  }
+  if (cudaHostAlloc(reinterpret_cast<void**>(&c->bf_layers), (size_t)s.L * y.bf_layer * 2, cudaHostAllocPortable) !=
           cudaSuccess ||
       cudaHostAlloc(reinterpret_cast<void**>(&c->bf_embed), (size_t)s.V * s.d * 2,
                     cudaHostAllocPortable | cudaHostAllocMapped) != cudaSuccess ||
@@ -909,8 +951,13 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) {
     memset(c->m + b, 0, (e - b) * 4);
     memset(c->v + b, 0, (e - b) * 4);
-    memset(c->grad + b, 0, (e - b) * 4);
+    if (c->grad) memset(c->grad + b, 0, (e - b) * 4);
   });
+  if (c->ring) {
+    const size_t nr = (size_t)MT_GRAD_RING_SLOTS * c->layer_f;
+    parallel_ranges(*c->pool, nr, [&](size_t b, size_t e) { memset(c->ring + b, 0, (e - b) * 4); });
+    parallel_ranges(*c->pool, head_f, [&](size_t b, size_t e) { memset(c->grad_head + b, 0, (e - b) * 4); });
+  }
   // bf16 streaming copies
   for (int l = 0; l < s.L; ++l) {
     uint16_t* blk = c->bf_layers + (size_t)l * y.bf_layer;
@@ -1089,6 +1136,10 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   c->timed.clear();
   c->launches = 0;
   c->err.clear();
+  {
+    std::lock_guard<std::mutex> lk(c->opt_mu);
+    c->layer_jobs_done = 0;
+  }
   push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, s.L + 1});
   const double te0 = now_s();
   int r = enqueue_step(c, n_unique);
@@ -1123,6 +1174,7 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
 
 extern "C" int mt_get_grads(mt_ctx* c, float* dst, size_t bytes) {
   if (!c || !dst) return MT_ERR_ARG;
+  if (!c->grad) return set_err(c, MT_ERR_CONFIG, "created with MT_FLAG_GRAD_RING: no gradient arena is kept");
   if (bytes < c->lay.total * 4) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
   memcpy(dst, c->grad, c->lay.total * 4);
   return MT_OK;

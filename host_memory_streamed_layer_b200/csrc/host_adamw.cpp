@@ -30,7 +30,7 @@ void adamw_scalar(float* p, const float* g, float* m, float* v, uint16_t* pb, si
                   float b2, float step, float inv_sqrt_bc2, float eps) {
   const float c1 = 1.f - b1, c2 = 1.f - b2;
   for (size_t i = 0; i < n; ++i) {
-    const float gi = g[i];
+    const float gi = g ? g[i] : 0.f;
     const float mi = b1 * m[i] + c1 * gi;
     const float vi = b2 * v[i] + c2 * gi * gi;
     const float pi = p[i] * decay - step * mi / (sqrtf(vi) * inv_sqrt_bc2 + eps);
@@ -55,6 +55,10 @@ __attribute__((target("avx512f,avx512bw"))) inline __m256i bf16x16_rne(__m512 x)
 
 // The bf16 copy is only written (the next step's H2D reads it), so it is
 // stored with non-temporal stores when 32-byte aligned: no read-for-ownership.
+// HAS_G = false is the update of a zero gradient (embedding rows no token of
+// the batch touches): the moments only decay and no gradient is read; the
+// result is bit-identical to reading zeros (b m + 0 rounds like b m).
+template <bool HAS_G>
 __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const float* g, float* m, float* v,
                                                               uint16_t* pb, size_t n, float decay, float b1, float b2,
                                                               float step, float inv_sqrt_bc2, float eps) {
@@ -65,9 +69,15 @@ __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const fl
   const __m512 vibc2 = _mm512_set1_ps(inv_sqrt_bc2), veps = _mm512_set1_ps(eps);
   size_t i = 0;
   for (; i + 16 <= n; i += 16) {
-    const __m512 gi = _mm512_loadu_ps(g + i);
-    const __m512 mi = _mm512_fmadd_ps(vb1, _mm512_loadu_ps(m + i), _mm512_mul_ps(vc1, gi));
-    const __m512 vi = _mm512_fmadd_ps(vb2, _mm512_loadu_ps(v + i), _mm512_mul_ps(vc2, _mm512_mul_ps(gi, gi)));
+    __m512 mi, vi;
+    if (HAS_G) {
+      const __m512 gi = _mm512_loadu_ps(g + i);
+      mi = _mm512_fmadd_ps(vb1, _mm512_loadu_ps(m + i), _mm512_mul_ps(vc1, gi));
+      vi = _mm512_fmadd_ps(vb2, _mm512_loadu_ps(v + i), _mm512_mul_ps(vc2, _mm512_mul_ps(gi, gi)));
+    } else {
+      mi = _mm512_mul_ps(vb1, _mm512_loadu_ps(m + i));
+      vi = _mm512_mul_ps(vb2, _mm512_loadu_ps(v + i));
+    }
     const __m512 den = _mm512_fmadd_ps(_mm512_sqrt_ps(vi), vibc2, veps);
     const __m512 pi = _mm512_sub_ps(_mm512_mul_ps(_mm512_loadu_ps(p + i), vdec),
                                     _mm512_div_ps(_mm512_mul_ps(vstep, mi), den));
@@ -80,7 +90,9 @@ __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const fl
       _mm256_storeu_si256(reinterpret_cast<__m256i*>(pb + i), bf16x16_rne(pi));
   }
   if (nt) _mm_sfence();
-  if (i < n) adamw_scalar(p + i, g + i, m + i, v + i, pb ? pb + i : nullptr, n - i, decay, b1, b2, step, inv_sqrt_bc2, eps);
+  if (i < n)
+    adamw_scalar(p + i, HAS_G ? g + i : nullptr, m + i, v + i, pb ? pb + i : nullptr, n - i, decay, b1, b2, step,
+                 inv_sqrt_bc2, eps);
 }
 
 __attribute__((target("avx512f,avx512bw"))) void round_avx512(const float* x, uint16_t* out, size_t n) {
@@ -108,8 +120,10 @@ void adamw_chunk(float* p, const float* g, float* m, float* v, uint16_t* pb, siz
   const float decay = 1.f - h.lr * h.wd;
   const float step = (float)(h.lr / bc1);
   const float inv_sqrt_bc2 = (float)(1.0 / sqrt(bc2));
-  if (adamw_uses_avx512())
-    adamw_avx512(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
+  if (adamw_uses_avx512() && g)
+    adamw_avx512<true>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
+  else if (adamw_uses_avx512())
+    adamw_avx512<false>(p, nullptr, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
   else
     adamw_scalar(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
 }
@@ -208,7 +222,7 @@ void parallel_ranges(ThreadPool& pool, size_t n, const std::function<void(size_t
 
 extern "C" int mt_k_adamw_host(float* p, const float* g, float* m, float* v, uint16_t* pb, size_t n, float lr,
                                float beta1, float beta2, float eps, float wd, int t) {
-  if ((!p || !g || !m || !v) && n) return MT_ERR_ARG;
+  if ((!p || !m || !v) && n) return MT_ERR_ARG;
   if (t < 1 || !(eps > 0) || !(beta1 >= 0 && beta1 < 1) || !(beta2 >= 0 && beta2 < 1)) return MT_ERR_ARG;
   mt::adamw_chunk(p, g, m, v, pb, n, mt::AdamHyper{lr, beta1, beta2, eps, wd}, t);
   return MT_OK;

@@ -28,6 +28,7 @@ struct AdamHyper {
 //   p <- p (1 - lr wd); m <- b1 m + (1 - b1) g; v <- b2 v + (1 - b2) g^2;
 //   p <- p - (lr / (1 - b1^t)) m / (sqrt(v) / sqrt(1 - b2^t) + eps)
 // and pb[i] <- bf16(p[i]) (round to nearest even) when pb is not null.
+// g == nullptr means a zero gradient (nothing is read).
 void adamw_chunk(float* p, const float* g, float* m, float* v, uint16_t* pb, size_t n, const AdamHyper& h, int t);
 
 // Round-to-nearest-even fp32 -> bf16 over n elements (NaN stays NaN).

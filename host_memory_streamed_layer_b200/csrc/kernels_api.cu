@@ -11,6 +11,11 @@ extern "C" int mt_k_gemm_bf16(const void* A, int64_t lda, int a_mn_major, const 
   return mt::gemm_bf16(g, static_cast<cudaStream_t>(stream), dev_err);
 }
 
+extern "C" int mt_k_gemm_variant(int variant) {
+  if (variant < 0 || variant > 2) return MT_ERR_ARG;
+  return mt::gemm_variant(variant);
+}
+
 #include <cmath>
 
 namespace {

@@ -46,6 +46,8 @@ struct GemmDesc {
 };
 
 int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
+// Kernel family for later GEMMs: 0 automatic, 1 single-CTA, 2 CTA pairs; returns the previous one.
+int gemm_variant(int v);
 
 // 2-D bf16 TMA map: inner (contiguous) extent, outer extent, row pitch ld
 // (elements), box {64, box_outer}, 128-byte swizzle, zero fill out of bounds.

@@ -51,6 +51,19 @@ def mt_k_gemm_bf16(A, lda, a_mn, B, ldb, b_mn, C, ldc, out_kind, R, ldr, M, N, K
     return _check(lib.mt_k_gemm_bf16(A, lda, a_mn, B, ldb, b_mn, C, ldc, out_kind, R or None, ldr, M, N, K,
                                      stream or None, dev_err or None), "mt_k_gemm_bf16")
 
+
+_sig("mt_k_gemm_variant", c_int, c_int)
+GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
+
+
+def mt_k_gemm_variant(variant: int) -> int:
+    """Selects the GEMM kernel family for later calls; returns the previous one."""
+    rc = lib.mt_k_gemm_variant(variant)
+    if rc < 0:
+        raise MTError(rc, "mt_k_gemm_variant")
+    return rc
+
+
 c_float, c_f = ctypes.c_float, ctypes.c_float
 
 _sig("mt_k_rmsnorm_fwd", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_float, c_void_p)
@@ -158,7 +171,8 @@ def mt_k_gemm_bf16_rope(A, lda, B, ldb, C, ldc, M, N, K, rope_cols, hd, s, cos_t
 # ---------------------------------------------------------------------------
 # Engine API (include/mt.h)
 # ---------------------------------------------------------------------------
-MT_FLAG_SERIALIZE, MT_FLAG_KERNEL_TIMING, MT_FLAG_NO_UPDATE = 0x1, 0x2, 0x4
+MT_FLAG_SERIALIZE, MT_FLAG_KERNEL_TIMING, MT_FLAG_NO_UPDATE, MT_FLAG_GRAD_RING = 0x1, 0x2, 0x4, 0x8
+MT_GRAD_RING_SLOTS = 3
 MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
 MT_T_EMBED, MT_T_FINAL_NORM, MT_T_LM_HEAD = 100, 101, 102
 
@@ -274,7 +288,8 @@ def mt_last_error(ctx: int = 0) -> str:
 
 
 def mt_k_adamw_host(p, g, m, v, pb, n, lr, beta1, beta2, eps, wd, t):
-    return _check(lib.mt_k_adamw_host(p, g, m, v, pb or None, n, lr, beta1, beta2, eps, wd, t), "mt_k_adamw_host")
+    return _check(lib.mt_k_adamw_host(p, g or None, m, v, pb or None, n, lr, beta1, beta2, eps, wd, t),
+                  "mt_k_adamw_host")
 
 
 def mt_host_optimizer_gbs(n: int = 1 << 28, threads: int = 0) -> float:

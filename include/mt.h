@@ -45,6 +45,15 @@ extern "C" {
 #define MT_FLAG_SERIALIZE 0x1u     /* run copies and kernels on one stream (debug) */
 #define MT_FLAG_KERNEL_TIMING 0x2u /* time GEMM / attention launches with events */
 #define MT_FLAG_NO_UPDATE 0x4u     /* compute loss and gradients only, skip AdamW */
+/* Gradients stream through a ring of MT_GRAD_RING_SLOTS layer-sized pinned
+ * host slots (plus one buffer for the final norm and LM head) instead of a
+ * full fp32 gradient arena: host memory drops from 18 to about 14 bytes per
+ * parameter, and the gradient of every layer is consumed by its AdamW update
+ * as it lands. When the optimizer falls that many layers behind the backward,
+ * the next gradient offload waits for a slot (bounded by the context's wait
+ * limit). mt_get_grads is not available in this mode. */
+#define MT_FLAG_GRAD_RING 0x8u
+#define MT_GRAD_RING_SLOTS 3
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0
@@ -115,18 +124,21 @@ size_t mt_arena_bytes(const mt_config* cfg);
 int mt_tensor_offset(const mt_config* cfg, int layer, int tensor_id, size_t* offset_floats, size_t* numel);
 
 /* Host bytes the context holds besides the caller's arena: two fp32 Adam
- * moments (8 B/param), the fp32 gradient arena (4 B/param) and the bf16
- * streaming copy (2 B/param), plus padding. */
+ * moments (8 B/param), the bf16 streaming copy (2 B/param) and the staging of
+ * the embedding-gradient rows, plus the fp32 gradients: the whole gradient
+ * arena (4 B/param), or with MT_FLAG_GRAD_RING in cfg->flags the ring of
+ * MT_GRAD_RING_SLOTS layer slots and the final-norm + LM-head gradient. */
 size_t mt_host_state_bytes(const mt_config* cfg);
 
 /* Creates a context on cfg->device. host_param_arena: the caller's fp32
  * master weights in the layout of mt_arena_bytes, at least arena_bytes long and
- * 256-byte aligned; the library pins it (cudaHostRegister) for the context's
- * lifetime and updates it in place every step. NULL: the library allocates the
+ * 256-byte aligned; the library updates it in place every step and keeps the
+ * pointer for the context's lifetime. Only host threads touch it (the GPU reads
+ * the bf16 copies), so it need not be pinned. NULL: the library allocates the
  * arena and fills it from cfg->seed (gains 1, matrices N(0, 0.02^2)). The
- * library owns the moments, the gradient arena, the bf16 copy and all device
- * memory. Fails with MT_ERR_NOMEM before allocating if the device budget does
- * not fit. */
+ * library owns the moments, the gradient buffers, the bf16 copy (pinned) and
+ * all device memory. Fails with MT_ERR_NOMEM before allocating if the device
+ * budget does not fit. */
 int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, mt_ctx** out);
 
 /* One training step: tokens and labels are host int32 arrays of b*s ids in
@@ -138,7 +150,8 @@ int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes,
 int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, float* loss_out);
 
 /* Copies the fp32 gradients of the last step (taken before the update), in the
- * arena layout, to dst (bytes >= mt_arena_bytes). */
+ * arena layout, to dst (bytes >= mt_arena_bytes). MT_ERR_CONFIG for a context
+ * created with MT_FLAG_GRAD_RING, which keeps no gradient arena. */
 int mt_get_grads(mt_ctx* ctx, float* dst, size_t bytes);
 
 /* Copies the current fp32 master weights (after the last update) to dst. */

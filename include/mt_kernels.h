@@ -162,12 +162,21 @@ int mt_k_gemm_bf16_rope(const void* A, int64_t lda, const void* B, int64_t ldb, 
                         int K, int rope_cols, int hd, int s, const float* cos_tab, const float* sin_tab, void* stream,
                         int32_t* dev_err);
 
+/* Selects the GEMM kernel family for later calls in this process: 0 automatic
+ * (the default, or MT_GEMM_VARIANT=auto), 1 single-CTA tiles only (=single),
+ * 2 CTA-pair tiles (tcgen05 cta_group::2, 256-row tiles) wherever a problem
+ * has at least one pair tile per SM pair (=pair). Both families compute the
+ * same product; this exists for measurement and tests. Returns the previous
+ * family, or MT_ERR_ARG for another value (nothing changes). No GPU work. */
+int mt_k_gemm_variant(int variant);
+
 /* Host AdamW over n fp32 elements, in place (HOST pointers, runs on the
  * calling thread; the engine runs the same routine across its worker pool):
  *   p <- p (1 - lr wd); m <- b1 m + (1-b1) g; v <- b2 v + (1-b2) g^2;
  *   p <- p - lr (m / (1 - b1^t)) / (sqrt(v / (1 - b2^t)) + eps)
  * and pb[i] <- bf16(p[i]) rounded to nearest even when pb is not NULL
- * (the streamed copy). t >= 1 counts steps. The update is Adam (Kingma & Ba,
+ * (the streamed copy). g may be NULL for a zero gradient (nothing is read:
+ * the embedding rows a batch does not touch). t >= 1 counts steps. The update is Adam (Kingma & Ba,
  * cited by the MegaTrain paper) with decoupled decay, on the CPU as MegaTrain
  * does (intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
  * Optimizer Steps"). */

@@ -61,6 +61,62 @@ def test_host_state_accounting():
     assert 14 * P <= extra <= 14.2 * P
 
 
+@pytest.mark.parametrize("name", ["llama-1.3b", "llama-7b", "gqa-14b"])
+def test_host_state_with_gradient_ring(name):
+    """With the gradient ring the fp32 gradient arena (4 B/param) is replaced by
+    MT_GRAD_RING_SLOTS layer-sized slots plus the final-norm + LM-head
+    gradient: master + state is then about 14 B/param, which is what lets the
+    14B workload (12.57 B parameters) fit a host with under 200 GB of RAM."""
+    mt = _mt()
+    shape = synth.WORKLOADS[name]
+    cfg = mt.mt_config_default(**shape)
+    full = mt.mt_host_state_bytes(cfg)
+    cfg.flags = mt.MT_FLAG_GRAD_RING
+    ring = mt.mt_host_state_bytes(cfg)
+    P = mt.mt_arena_bytes(cfg) // 4
+    c = oracle.OracleConfig(**shape)
+    layout, _ = oracle.arena_layout(c)
+    first = {}
+    for layer, tid, off, shp in layout:
+        first[(layer, tid)] = (off, int(np.prod(shp)))
+    # one layer's gradient block: from its first tensor to the next layer's first tensor
+    layer_f = first[(1, mt.MT_T_ATTN_NORM)][0] - first[(0, mt.MT_T_ATTN_NORM)][0]
+    fn_off = first[(-1, mt.MT_T_FINAL_NORM)][0]
+    head_off, head_n = first[(-1, mt.MT_T_LM_HEAD)]
+    head_f = head_off + head_n - fn_off
+    assert ring == full - 4 * P + 4 * (mt.MT_GRAD_RING_SLOTS * layer_f + head_f)
+    # the fixed buffers weigh less as models grow: ~14.9 B/param at 1.3B, ~14.5 at 14B
+    assert ring + 4 * P <= (15.0 if P < 5e9 else 14.6) * P
+
+
+def test_host_adamw_zero_gradient_reads_nothing():
+    """g = NULL is the update of a zero gradient: bit-identical to passing
+    zeros, and equal to the oracle's AdamW with g = 0 (decay and moment decay
+    only)."""
+    mt = _mt()
+    rng = np.random.default_rng(3)
+    n = 4099
+    p0 = (rng.normal(size=n) * 0.02).astype(np.float32)
+    m0 = (rng.normal(size=n) * 1e-3).astype(np.float32)
+    v0 = (np.abs(rng.normal(size=n)) * 1e-6).astype(np.float32)
+    hyper = dict(lr=1e-3, beta1=0.9, beta2=0.95, eps=1e-8, wd=0.1)
+    outs = []
+    for g in (None, np.zeros(n, dtype=np.float32)):
+        p, m, v = p0.copy(), m0.copy(), v0.copy()
+        pb = np.zeros(n, dtype=np.uint16)
+        mt.mt_k_adamw_host(p.ctypes.data, 0 if g is None else g.ctypes.data, m.ctypes.data, v.ctypes.data,
+                           pb.ctypes.data, n, hyper["lr"], hyper["beta1"], hyper["beta2"], hyper["eps"],
+                           hyper["wd"], 3)
+        outs.append((p, m, v, pb))
+    for a, b in zip(outs[0], outs[1]):
+        assert np.array_equal(a, b)
+    rp, rm, rv = oracle.adamw_update(p0.astype(np.float64), np.zeros(n), m0.astype(np.float64),
+                                     v0.astype(np.float64), 3, **hyper)
+    assert np.all(np.abs(outs[0][0] - rp) <= 2e-8 + 1e-6 * np.abs(rp))
+    assert np.allclose(outs[0][1], 0.9 * m0.astype(np.float64), rtol=1e-6, atol=0)
+    assert np.allclose(outs[0][2], 0.95 * v0.astype(np.float64), rtol=1e-6, atol=0)
+
+
 @pytest.mark.parametrize("bad", [dict(d=100), dict(H=3), dict(Hkv=3), dict(F=689), dict(V=1001), dict(L=0),
                                  dict(d=512, H=2), dict(b=0)])
 def test_invalid_config_rejected(bad):

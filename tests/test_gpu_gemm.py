@@ -1,6 +1,7 @@
 """Parity of the tcgen05 GEMM (through the C ABI) with an fp64 CPU product of
 the same bf16 inputs, in the three operand forms the layer uses, across
-ragged sizes (M, N, K not multiples of the tile) and both tile widths."""
+ragged sizes (M, N, K not multiples of the tile), both tile widths of the
+single-CTA kernel and both tile widths of the CTA-pair kernel."""
 import numpy as np
 import pytest
 import torch
@@ -17,17 +18,30 @@ def _ref(A, B):  # fp64 product of the exact bf16 values
     return A.double().cpu() @ B.double().cpu().T
 
 
-CASES = [
-    (128, 256, 64), (256, 512, 128), (300, 200, 100), (1000, 768, 688), (64, 48, 40),
-    (4096, 2304, 512), (257, 1376, 256), (2048, 4096, 1024),
-]
+SMALL = [(128, 256, 64), (256, 512, 128), (300, 200, 100), (1000, 768, 688), (64, 48, 40), (257, 1376, 256)]
+# Large enough for the CTA-pair kernel (at least one 256-row tile per SM pair
+# of a 148-SM part); the last three are ragged in M, N and K and take 256-wide
+# pair tiles, 128-wide pair tiles (they quantize into waves better), and
+# 128-wide pair tiles because 256-wide ones would not fill every pair.
+LARGE = [(4096, 2304, 512), (2048, 4096, 1024), (2200, 5504, 200), (4000, 2344, 328), (2304, 2048, 4160)]
+CASES = [(*c, "auto") for c in SMALL] + [(*c, v) for c in LARGE for v in ("auto", "single", "pair")]
 
 
-@pytest.mark.parametrize("M,N,K", CASES)
+@pytest.mark.parametrize("M,N,K,variant", CASES)
 @pytest.mark.parametrize("form", ["fwd", "dx", "dw"])
 @pytest.mark.parametrize("out", ["bf16", "f32", "f32_add"])
-def test_gemm_matches_fp64(M, N, K, form, out):
+def test_gemm_matches_fp64(M, N, K, variant, form, out):
+    """variant: the GEMM kernel family (auto; single-CTA tiles only; CTA-pair
+    tiles wherever the problem has one per SM pair)."""
     mt = _mt()
+    prev = mt.mt_k_gemm_variant({"auto": mt.GEMM_AUTO, "single": mt.GEMM_SINGLE, "pair": mt.GEMM_PAIR}[variant])
+    try:
+        _gemm_case(mt, M, N, K, form, out)
+    finally:
+        mt.mt_k_gemm_variant(prev)
+
+
+def _gemm_case(mt, M, N, K, form, out):
     g = torch.Generator(device="cpu").manual_seed(M * 7 + N * 3 + K)
     A = torch.randn(M, K, generator=g).to(torch.bfloat16)
     B = torch.randn(N, K, generator=g).to(torch.bfloat16)

@@ -256,11 +256,23 @@ def test_attention_bwd(hd, H, Hkv, s, b, impl):
     assert rel_l2(g[:, (H + Hkv) * hd:].reshape(b, s, Hkv, hd), rdv) < 1e-2
 
 
-@pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 16, 16, 256, 1)])
-def test_qkv_gemm_with_rope_epilogue(hd, H, Hkv, s, b):
+@pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 16, 16, 256, 1),
+                                         # large enough for the CTA-pair kernel (256- and 128-wide tiles)
+                                         (128, 16, 16, 2048, 2), (64, 16, 4, 1024, 4)])
+@pytest.mark.parametrize("variant", [0, 1, 2])
+def test_qkv_gemm_with_rope_epilogue(hd, H, Hkv, s, b, variant):
     """q, k, v projection with RoPE fused in the epilogue = oracle RoPE of the
-    fp64 product (v columns unrotated), rounded once to bf16."""
+    fp64 product (v columns unrotated), rounded once to bf16; through each GEMM
+    kernel family (automatic, single-CTA, CTA pairs)."""
     mt = _mt()
+    prev = mt.mt_k_gemm_variant(variant)
+    try:
+        _qkv_rope_case(mt, hd, H, Hkv, s, b)
+    finally:
+        mt.mt_k_gemm_variant(prev)
+
+
+def _qkv_rope_case(mt, hd, H, Hkv, s, b):
     rng = np.random.default_rng(hd * s)
     T, d = b * s, 256
     N = (H + 2 * Hkv) * hd

@@ -212,3 +212,42 @@ def test_checkpoint_resume_continues_the_trajectory():
         mt.mt_destroy(ctx)
     assert abs(loss2 - loss2b) <= 1e-5
     assert rel(P2b, P2) <= 1e-5
+
+
+def test_gradient_ring_matches_full_arena_and_oracle():
+    """MT_FLAG_GRAD_RING: layer gradients pass through MT_GRAD_RING_SLOTS host
+    slots (5 layers > slots, so offloads wait for released slots) and the
+    untouched embedding rows take the zero-gradient update. Two steps follow
+    the run with the full gradient arena (same tokens and initial master) and
+    the first step's update is within the end-to-end bar of the oracle's."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    shape = dict(L=5, d=256, H=4, Hkv=4, F=688, V=1024, b=2, s=128)
+    assert shape["L"] > mt.MT_GRAD_RING_SLOTS
+    c = oracle.OracleConfig(**shape)
+    full = run_gpu(shape, 2)
+    cfg = arena.config(shape)
+    cfg.flags = mt.MT_FLAG_GRAD_RING
+    cfg.host_threads = 4
+    A = arena.pack(cfg, synth.init_weights(shape, 0))
+    ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+    ring = []
+    try:
+        for step in range(2):
+            tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, step)
+            loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+            ring.append(dict(loss=loss, P=A.copy()))
+        with pytest.raises(mt.MTError) as e:
+            G = np.empty_like(A)
+            mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
+        assert e.value.code == -2
+    finally:
+        mt.mt_destroy(ctx)
+    for f, r in zip(full, ring):
+        assert abs(f["loss"] - r["loss"]) <= 1e-4
+        assert rel(r["P"], f["P"]) <= 2e-3
+    o = oracle_steps(shape, 1)[0]
+    P = oracle.unpack_arena(ring[0]["P"], c)
+    num = sum(float(np.sum((P[k] - o["P"][k]) ** 2)) for k in P)
+    den = sum(float(np.sum(o["P"][k] ** 2)) for k in P)
+    assert abs(ring[0]["loss"] - o["loss"]) <= 1e-2
+    assert math.sqrt(num / den) <= 5e-3
