@@ -187,7 +187,13 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc_s = idesc_bf16_f32(FA_BQ, FA_BKV, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(FA_BQ, HD, false, true);
-      const uint32_t aQ = smem_u32(sQ);
+      // Descriptors of the first k-step of each operand; k-steps, stages and
+      // 64-column sub-tiles only move the start-address field (address / 16),
+      // so the loops add constants (the MMAs are 64 cycles each).
+      const uint64_t dQ0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dP0 = sdesc_sw128(smem_u32(sP), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
       bool ok = mbar_wait(q_full, 0) && !*abort_flag;
       bool issued = false;
       auto issue_pv = [&](int i) -> bool {
@@ -197,14 +203,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
             !mbar_wait(&o_empty[pb], ph ^ 1))
           return false;
         tc_fence_after();
-        const uint32_t aP = smem_u32(sP + pb * C::P_BYTES);
-        const uint32_t bV = smem_u32(sV + (i & 1) * C::KV_BYTES);
+        const uint64_t aP = dP0 + ((pb * C::P_BYTES) >> 4), bV = dV0 + (((i & 1) * C::KV_BYTES) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < FA_BKV / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(aP + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(bV + kk * 2048, 16384, 1024);
-          umma_bf16(tmem + C::O_COL + pb * HD, ad, bd, idesc_o, kk != 0);
-        }
+        for (int kk = 0; kk < FA_BKV / 16; ++kk)
+          umma_bf16(tmem + C::O_COL + pb * HD, aP + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), bV + ((kk * 2048) >> 4),
+                    idesc_o, kk != 0);
         umma_commit(&o_full[pb]);
         umma_commit(&v_empty[pb]);
         return true;
@@ -217,12 +220,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t bK = smem_u32(sK + st * C::KV_BYTES);
+        const uint64_t bK = dK0 + ((st * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(aQ + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(bK + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024);
-          umma_bf16(tmem + C::S_COL + st * FA_BKV, ad, bd, idesc_s, kk != 0);
+          const uint32_t step = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + C::S_COL + st * FA_BKV, dQ0 + step, bK + step, idesc_s, kk != 0);
         }
         issued = true;
         umma_commit(&s_full[st]);
@@ -445,7 +447,9 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
 namespace {
 
 constexpr int FB_BKV = 128, FB_BQ = 64, FB_HD = 128;
-constexpr int FB_THREADS = 320;  // producer, MMA, 8 gradient warps (two per tensor-memory lane quarter)
+constexpr int FB_GWARPS = 16;                     // gradient warps: four per tensor-memory lane quarter
+constexpr int FB_QW = FB_BQ / (FB_GWARPS / 4);    // queries per gradient warp (16)
+constexpr int FB_THREADS = 64 + 32 * FB_GWARPS;   // producer, MMA, gradient warps
 
 struct FbCfg {
   static constexpr int KV_BYTES = FB_BKV * FB_HD * 2;  // 32 KB
@@ -479,6 +483,7 @@ struct FbParams {
   const float* rcos;
   const float* rsin;
   int* err;
+  int vec_lse;  // LSE and D rows start 16-byte aligned: s % 4 == 0 and aligned bases
 };
 
 __global__ void __launch_bounds__(FB_THREADS, 1)
@@ -525,12 +530,12 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&dq_empty[i], 8);
+      mbar_init(&dq_empty[i], FB_GWARPS);
     }
-    mbar_init(p_full, 8);
+    mbar_init(p_full, FB_GWARPS);
     mbar_init(mma_done, 1);
     mbar_init(drain, 1);
-    mbar_init(dq_staged, 8);
+    mbar_init(dq_staged, FB_GWARPS);
     mbar_init(dq_free, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -559,11 +564,15 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         tma_load_2d(sK + c * 16384, &tmK, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
         tma_load_2d(sV + c * 16384, &tmV, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
       }
+      int h = kvh * group, qb = qb_first;  // head and query block of iteration it
       for (int it = 0; it < n_it; ++it) {
         const int st = it & 1;
         const uint32_t ph = (it >> 1) & 1;
-        const int h = kvh * group + it / per_head;
-        const int q0 = (qb_first + it % per_head) * FB_BQ;
+        const int q0 = qb * FB_BQ, hq = h;
+        if (++qb == nqb) {
+          qb = qb_first;
+          ++h;
+        }
         if (*abort_flag || !mbar_wait(&q_empty[st], ph ^ 1)) {
           record_error(p.err, 100 + (it & 63));
           ok = false;
@@ -571,8 +580,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         }
         mbar_arrive_expect_tx(&q_full[st], 2 * C::QT_BYTES);
         for (int c = 0; c < 2; ++c) {
-          tma_load_2d(sQ + st * C::QT_BYTES + c * 8192, &tmQ, &q_full[st], h * FB_HD + c * 64, row0 + q0);
-          tma_load_2d(sdO + st * C::QT_BYTES + c * 8192, &tmO, &q_full[st], h * FB_HD + c * 64, row0 + q0);
+          tma_load_2d(sQ + st * C::QT_BYTES + c * 8192, &tmQ, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
+          tma_load_2d(sdO + st * C::QT_BYTES + c * 8192, &tmO, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
         }
         q_last[st] = (int)ph;
       }
@@ -592,7 +601,13 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       constexpr uint32_t id_s = idesc_bf16_f32(FB_BKV, FB_BQ, false, false);   // keys x queries, K = hd
       constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, FB_HD, false, true);   // keys x hd, K = queries
       constexpr uint32_t id_dq = idesc_bf16_f32(FB_HD, FB_BQ, true, true);     // hd x queries, K = keys
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aPt = smem_u32(sPt), adSt = smem_u32(sdSt);
+      // Descriptors of the first k-step of each operand form; the loops add
+      // start-address steps (address / 16) instead of rebuilding them.
+      const uint64_t dK_km = sdesc_sw128(smem_u32(sK), 16, 1024), dV_km = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dQ_km = sdesc_sw128(smem_u32(sQ), 16, 1024), dO_km = sdesc_sw128(smem_u32(sdO), 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 8192, 1024), dO_mn = sdesc_sw128(smem_u32(sdO), 8192, 1024);
+      const uint64_t dPt_km = sdesc_sw128(smem_u32(sPt), 16, 1024), ddSt_km = sdesc_sw128(smem_u32(sdSt), 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024), ddSt_mn = sdesc_sw128(smem_u32(sdSt), 8192, 1024);
       bool issued = false;
       auto issue_s = [&](int it) -> bool {
         const int st = it & 1;
@@ -605,13 +620,13 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           return false;
         }
         tc_fence_after();
-        const uint32_t bQ = smem_u32(sQ + st * C::QT_BYTES), bO = smem_u32(sdO + st * C::QT_BYTES);
+        const uint32_t so = (st * C::QT_BYTES) >> 4;
         const uint32_t cs = tmem + C::C_BUF + st * C::BUF_COLS;
 #pragma unroll
         for (int kk = 0; kk < FB_HD / 16; ++kk) {
-          const uint32_t ka = (kk >> 2) * 16384 + (kk & 3) * 32, kb = (kk >> 2) * 8192 + (kk & 3) * 32;
-          umma_bf16(cs, sdesc_sw128(aK + ka, 16, 1024), sdesc_sw128(bQ + kb, 16, 1024), id_s, kk != 0);
-          umma_bf16(cs + C::C_DP_OFF, sdesc_sw128(aV + ka, 16, 1024), sdesc_sw128(bO + kb, 16, 1024), id_s, kk != 0);
+          const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, kb = so + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
+          umma_bf16(cs, dK_km + ka, dQ_km + kb, id_s, kk != 0);
+          umma_bf16(cs + C::C_DP_OFF, dV_km + ka, dO_km + kb, id_s, kk != 0);
         }
         issued = true;
         umma_commit(&s_full[st]);
@@ -632,22 +647,20 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t bQ = smem_u32(sQ + st * C::QT_BYTES), bO = smem_u32(sdO + st * C::QT_BYTES);
+        const uint32_t so = (st * C::QT_BYTES) >> 4;
         // dV += P^T dO, dK += dS^T Q (K = 64 queries: 4 steps; B MN-major over hd, 8 KB between hd chunks)
 #pragma unroll
         for (int kk = 0; kk < FB_BQ / 16; ++kk) {
           const bool acc = (it > 0) || (kk > 0);
-          umma_bf16(tmem + C::C_DV, sdesc_sw128(aPt + kk * 32, 16, 1024), sdesc_sw128(bO + kk * 2048, 8192, 1024),
-                    id_kv, acc);
-          umma_bf16(tmem + C::C_DK, sdesc_sw128(adSt + kk * 32, 16, 1024), sdesc_sw128(bQ + kk * 2048, 8192, 1024),
-                    id_kv, acc);
+          umma_bf16(tmem + C::C_DV, dPt_km + ((kk * 32) >> 4), dO_mn + so + ((kk * 2048) >> 4), id_kv, acc);
+          umma_bf16(tmem + C::C_DK, ddSt_km + ((kk * 32) >> 4), dQ_mn + so + ((kk * 2048) >> 4), id_kv, acc);
         }
         // dQ^T = K^T dS^T (K = 128 keys: 8 steps; A MN-major over hd, 16 KB between hd chunks) into the
         // S^T columns of this iteration's buffer
 #pragma unroll
         for (int kk = 0; kk < FB_BKV / 16; ++kk)
-          umma_bf16(tmem + C::C_BUF + st * C::BUF_COLS, sdesc_sw128(aK + kk * 2048, 16384, 1024),
-                    sdesc_sw128(adSt + kk * 2048, 8192, 1024), id_dq, kk != 0);
+          umma_bf16(tmem + C::C_BUF + st * C::BUF_COLS, dK_mn + ((kk * 2048) >> 4), ddSt_mn + ((kk * 2048) >> 4),
+                    id_dq, kk != 0);
         umma_commit(mma_done);
         umma_commit(&q_empty[st]);
       }
@@ -660,19 +673,25 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       }
     }
   } else {
-    // ---------------- gradient warps (2..9) ----------------
-    const int wg = (warp - 2) >> 2;     // query columns [32 wg, 32 wg + 32) of each block
+    // ---------------- gradient warps (2 .. 2 + FB_GWARPS) ----------------
+    // Warp w owns tensor-memory lane quarter w mod 4 (32 key rows) and query
+    // columns [FB_QW qg, FB_QW qg + FB_QW) of each 64-query block: four warps
+    // per quarter keep enough independent work in flight to hide the latency
+    // of the tensor-memory loads and the exponentials.
+    const int qg = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row == tensor-memory lane (the head column for dQ^T)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale * 1.4426950408889634f;
     const int key = kv0 + r;
     const bool issuer = (warp == 2 && lane == 0);  // issues the dQ reductions
+    const bool vec_ok = p.vec_lse != 0;            // LSE / D rows 16-byte aligned
     bool ok = true;
 
-    // Reads dQ^T(it) (already complete: the caller waited for it), stages it
-    // and lets the issuer add it to the accumulator.
-    auto flush_dq = [&](int it) -> bool {
+    // Reads dQ^T of the iteration with head hq and query block start q0
+    // (already complete: the caller waited for it), stages it and lets the
+    // issuer add it to the accumulator.
+    auto flush_dq = [&](int it, int hq, int q0) -> bool {
       const int bf = it & 1;
       if (it > 0) {
         // the staging tile is reused: the previous reduce must have read it
@@ -686,13 +705,12 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         }
       }
       float* col = sDQ + (r >> 5) * (FB_BQ * 32) + (r & 31);  // box r/32: [64 queries][32 head columns]
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      {
         uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + wg * 32 + c * 16, v);
+        tmem_ld_32x32b_x16(tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + qg * FB_QW, v);
         tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) col[(wg * 32 + c * 16 + e) * 32] = __uint_as_float(v[e]) * p.scale;
+        for (int e = 0; e < 16; ++e) col[(qg * FB_QW + e) * 32] = __uint_as_float(v[e]) * p.scale;
       }
       tc_fence_before();
       fence_proxy_async_smem();
@@ -706,67 +724,94 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           record_error(p.err, 700 + (it & 63));
           return false;
         }
-        const int h = kvh * group + it / per_head;
-        const int q0 = (qb_first + it % per_head) * FB_BQ;
 #pragma unroll
         for (int bx = 0; bx < 4; ++bx)
           asm volatile(
               "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
                   reinterpret_cast<uint64_t>(&tmDQ)),
-              "r"(smem_u32(sDQ + bx * FB_BQ * 32)), "r"(h * FB_HD + bx * 32), "r"(row0 + q0)
+              "r"(smem_u32(sDQ + bx * FB_BQ * 32)), "r"(hq * FB_HD + bx * 32), "r"(row0 + q0)
               : "memory");
         asm volatile("cp.async.bulk.commit_group;" ::: "memory");
       }
       return true;
     };
 
+    int h = kvh * group, qb = qb_first;  // head and query block of iteration it
+    int h_prev = h, q0_prev = 0;         // those of iteration it - 1
     for (int it = 0; it < n_it; ++it) {
       const int bf = it & 1;
-      const int h = kvh * group + it / per_head;
-      const int q0 = (qb_first + it % per_head) * FB_BQ;
-      const float* lse = p.LSE + ((int64_t)b * p.H + h) * p.s + q0 + wg * 32;
-      const float* dd = p.Dv + ((int64_t)b * p.H + h) * p.s + q0 + wg * 32;
+      const int q0 = qb * FB_BQ, hq = h;
+      if (++qb == nqb) {
+        qb = qb_first;
+        ++h;
+      }
+      const int qc = q0 + qg * FB_QW;  // first query of this warp's columns
+      const float* lse = p.LSE + ((int64_t)b * p.H + hq) * p.s + qc;
+      const float* dd = p.Dv + ((int64_t)b * p.H + hq) * p.s + qc;
+      // Only blocks that touch the diagonal or a sequence end need the mask.
+      const bool need_mask = (qc < kv0 + FB_BKV) || (q0 + FB_BQ > p.s) || (kv0 + FB_BKV > p.s);
+      // this warp's 16 LSE and D values (the same for every lane), loaded
+      // before the wait: broadcast float4 loads where the columns lie inside
+      // the sequence and rows start 16-byte aligned, else guarded scalar loads
+      float lv[FB_QW], dvv[FB_QW];
+      if (!need_mask && vec_ok) {
+#pragma unroll
+        for (int i = 0; i < FB_QW / 4; ++i) {
+          const float4 a4 = __ldg(reinterpret_cast<const float4*>(lse) + i);
+          const float4 d4 = __ldg(reinterpret_cast<const float4*>(dd) + i);
+          lv[4 * i] = a4.x * 1.4426950408889634f;
+          lv[4 * i + 1] = a4.y * 1.4426950408889634f;
+          lv[4 * i + 2] = a4.z * 1.4426950408889634f;
+          lv[4 * i + 3] = a4.w * 1.4426950408889634f;
+          dvv[4 * i] = d4.x;
+          dvv[4 * i + 1] = d4.y;
+          dvv[4 * i + 2] = d4.z;
+          dvv[4 * i + 3] = d4.w;
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < FB_QW; ++i) {
+          const bool in = qc + i < p.s;
+          lv[i] = in ? __ldg(lse + i) * 1.4426950408889634f : 0.f;
+          dvv[i] = in ? __ldg(dd + i) : 0.f;
+        }
+      }
       if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&s_full[bf], (it >> 1) & 1)) {
         record_error(p.err, 300 + (it & 63));
         ok = false;
         break;
       }
       tc_fence_after();
-      // P^T and dS^T of this key row for this warpgroup's 32 queries (bf16 pairs).
-      // Only blocks that touch the diagonal or a sequence end need the mask.
-      uint32_t pp[16], ds[16];
-      auto grads = [&](auto mask_tag) {
-        constexpr bool MASK = decltype(mask_tag)::value;
+      // P^T and dS^T of this key row for this warp's 16 queries (bf16 pairs).
+      uint32_t pp[FB_QW / 2], ds[FB_QW / 2];
+      {
+        uint32_t sv[16], dv[16];
+        const uint32_t cb = tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + qg * FB_QW;
+        tmem_ld_32x32b_x16(cb, sv);
+        tmem_ld_32x32b_x16(cb + C::C_DP_OFF, dv);
+        tmem_ld_wait();
+        auto grads = [&](auto mask_tag) {
+          constexpr bool MASK = decltype(mask_tag)::value;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
-          uint32_t sv[16], dv[16];
-          const uint32_t cb = tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + wg * 32 + c * 16;
-          tmem_ld_32x32b_x16(cb, sv);
-          tmem_ld_32x32b_x16(cb + C::C_DP_OFF, dv);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
+          for (int e = 0; e < FB_QW; e += 2) {
             float pv[2], dsv[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const int cq = c * 16 + e + u;
-              const int qi = q0 + wg * 32 + cq;
+              const int qi = qc + e + u;
               const bool vis = !MASK || (key <= qi && qi < p.s && key < p.s);
-              const float pr =
-                  vis ? ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -__ldg(lse + cq) * 1.4426950408889634f)) : 0.f;
+              const float pr = vis ? ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lv[e + u])) : 0.f;
               pv[u] = pr;
-              dsv[u] = vis ? pr * (__uint_as_float(dv[e + u]) - __ldg(dd + cq)) : 0.f;
+              dsv[u] = vis ? pr * (__uint_as_float(dv[e + u]) - dvv[e + u]) : 0.f;
             }
-            pp[(c * 16 + e) >> 1] = pack_bf16x2(pv[0], pv[1]);
-            ds[(c * 16 + e) >> 1] = pack_bf16x2(dsv[0], dsv[1]);
+            pp[e >> 1] = pack_bf16x2(pv[0], pv[1]);
+            ds[e >> 1] = pack_bf16x2(dsv[0], dsv[1]);
           }
-        }
-      };
-      const bool need_mask = (q0 + wg * 32 < kv0 + FB_BKV) || (q0 + FB_BQ > p.s) || (kv0 + FB_BKV > p.s);
-      if (need_mask)
-        grads(std::true_type{});
-      else
-        grads(std::false_type{});
+        };
+        if (need_mask)
+          grads(std::true_type{});
+        else
+          grads(std::false_type{});
+      }
       // dV, dK, dQ^T of the previous iteration must be done with the tiles
       if (it > 0 && (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1))) {
         record_error(p.err, 400 + (it & 63));
@@ -774,8 +819,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         break;
       }
 #pragma unroll
-      for (int c8 = 0; c8 < 4; ++c8) {
-        const int chunk = wg * 4 + c8;
+      for (int c8 = 0; c8 < FB_QW / 8; ++c8) {
+        const int chunk = qg * (FB_QW / 8) + c8;  // 16-byte chunk of the 128-byte swizzled row
         const int off = r * 128 + ((chunk ^ (r & 7)) << 4);
         *reinterpret_cast<uint4*>(sPt + off) = make_uint4(pp[4 * c8], pp[4 * c8 + 1], pp[4 * c8 + 2], pp[4 * c8 + 3]);
         *reinterpret_cast<uint4*>(sdSt + off) = make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]);
@@ -784,16 +829,18 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      if (it > 0 && !flush_dq(it - 1)) {
+      if (it > 0 && !flush_dq(it - 1, h_prev, q0_prev)) {
         ok = false;
         break;
       }
+      h_prev = hq;
+      q0_prev = q0;
     }
     if (ok && n_it > 0) {
       if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (n_it - 1) & 1)) {
         record_error(p.err, 450);
         ok = false;
-      } else if (!flush_dq(n_it - 1)) {
+      } else if (!flush_dq(n_it - 1, h_prev, q0_prev)) {
         ok = false;
       }
     }
@@ -802,15 +849,17 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       *abort_flag = 1;
     } else if (n_it > 0) {
       // tcgen05.ld is warp-collective: every lane loads, only keys inside the
-      // sequence store. Warpgroup 0 writes dK (scaled, transposed RoPE),
-      // warpgroup 1 writes dV.
+      // sequence store. Warps of query group 0 and 1 write dK (scaled,
+      // transposed RoPE; rotate-half pairs (i, i + 64) for i in [32 qg, 32 qg + 32)),
+      // groups 2 and 3 write dV columns [64 (qg - 2), 64 (qg - 2) + 64).
       const bool store = key < p.s;
-      if (wg == 0) {
+      if (qg < 2) {
         __nv_bfloat16* kr = p.dK + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
         const float* cs = (p.rcos && store) ? p.rcos + (int64_t)key * (FB_HD / 2) : nullptr;
         const float* sn = (p.rsin && store) ? p.rsin + (int64_t)key * (FB_HD / 2) : nullptr;
 #pragma unroll
-        for (int c = 0; c < FB_HD / 2 / 16; ++c) {  // pairs (i, i + 64), 16 at a time
+        for (int cc = 0; cc < 2; ++cc) {  // pairs (i, i + 64), 16 at a time
+          const int c = qg * 2 + cc;
           uint32_t a[16], bb[16];
           tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + c * 16, a);
           tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + 64 + c * 16, bb);
@@ -844,7 +893,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       } else {
         __nv_bfloat16* vr = p.dV + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
 #pragma unroll
-        for (int c = 0; c < FB_HD / 16; ++c) {
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = (qg - 2) * 4 + cc;
           uint32_t v[16];
           tmem_ld_32x32b_x16(tmem + lane_base + C::C_DV + c * 16, v);
           tmem_ld_wait();
@@ -889,8 +939,9 @@ int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
       !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ) ||
       !make_tensor_map_2d_f32(&mdq, a.dq_acc, (int64_t)a.H * FB_HD, T, a.ldqa, 32, FB_BQ))
     return MT_ERR_ARG;
+  const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
-             a.scale, a.rope_cos, a.rope_sin, err};
+             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
   k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, p);
   return launch_status();

@@ -1172,6 +1172,37 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   return MT_OK;
 }
 
+extern "C" int mt_layer_fwd_bwd(mt_ctx* c, int l, const float* x_in, const float* dx_out, float* x_out,
+                                float* dx_in, float* grads, size_t grads_bytes) {
+  if (!c) return MT_ERR_ARG;
+  if (!x_in || !dx_out || !x_out || !dx_in || !grads) return set_err(c, MT_ERR_ARG, "NULL argument");
+  const Layout& y = c->lay;
+  const Shapes& s = y.sh;
+  if (l < 0 || l >= s.L) return set_err(c, MT_ERR_ARG, "layer outside [0, L)");
+  if (grads_bytes < c->layer_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than one layer's block");
+  CK(cudaSetDevice(c->device));
+  const size_t n = (size_t)s.T * s.d;
+  cudaStream_t sc = c->s_comp;
+  c->timing_used = 0;
+  c->timed.clear();
+  c->err.clear();
+  // the layer's streamed bf16 weights into slot 0, x_l into its boundary slot
+  CK(cudaMemcpyAsync(c->wslot[0], c->bf_layers + (size_t)l * y.bf_layer, y.bf_layer * 2, cudaMemcpyHostToDevice, sc));
+  CK(cudaMemcpyAsync(c->xb + (size_t)l * n, x_in, n * 4, cudaMemcpyHostToDevice, sc));
+  CK(cudaMemcpyAsync(c->gx0, dx_out, n * 4, cudaMemcpyHostToDevice, sc));
+  CKM(layer_fwd(c, l, 0, true));
+  CKM(layer_bwd(c, l, 0, c->gslot[0], c->gx0, c->gx1));
+  CK(cudaMemcpyAsync(x_out, c->xb + (size_t)(l + 1) * n, n * 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(dx_in, c->gx1, n * 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(grads, c->gslot[0], c->layer_f * 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaStreamSynchronize(sc));
+  int32_t dev_err;
+  memcpy(&dev_err, c->misc_h + 1, 4);
+  if (dev_err != 0) return set_err(c, MT_ERR_DEVICE, "kernel reported an error (bounded wait expired)");
+  return MT_OK;
+}
+
 extern "C" int mt_get_grads(mt_ctx* c, float* dst, size_t bytes) {
   if (!c || !dst) return MT_ERR_ARG;
   if (!c->grad) return set_err(c, MT_ERR_CONFIG, "created with MT_FLAG_GRAD_RING: no gradient arena is kept");

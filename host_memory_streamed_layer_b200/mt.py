@@ -207,6 +207,7 @@ _sig("mt_host_state_bytes", c_size_t, _cfgp)
 _sig("mt_create", c_int, _cfgp, c_void_p, c_size_t, ctypes.POINTER(c_void_p))
 _sig("mt_train_step", c_int, c_void_p, c_void_p, c_void_p, ctypes.POINTER(ctypes.c_float))
 _sig("mt_get_grads", c_int, c_void_p, c_void_p, c_size_t)
+_sig("mt_layer_fwd_bwd", c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_params", c_int, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
 _sig("mt_destroy", None, c_void_p)
@@ -261,6 +262,12 @@ def mt_train_step(ctx: int, tokens_ptr: int, labels_ptr: int) -> float:
 
 def mt_get_grads(ctx: int, dst_ptr: int, nbytes: int):
     return _check(lib.mt_get_grads(ctx, dst_ptr, nbytes), "mt_get_grads", ctx)
+
+
+def mt_layer_fwd_bwd(ctx: int, layer: int, x_in: int, dx_out: int, x_out: int, dx_in: int, grads: int,
+                     grads_bytes: int):
+    return _check(lib.mt_layer_fwd_bwd(ctx, layer, x_in, dx_out, x_out, dx_in, grads, grads_bytes),
+                  "mt_layer_fwd_bwd", ctx)
 
 
 def mt_get_params(ctx: int, dst_ptr: int, nbytes: int):

@@ -154,6 +154,23 @@ int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, flo
  * created with MT_FLAG_GRAD_RING, which keeps no gradient arena. */
 int mt_get_grads(mt_ctx* ctx, float* dst, size_t bytes);
 
+/* One decoder layer through the engine's own stateless layer template, with
+ * no optimizer step: the layer's current bf16 streamed weights, the forward
+ * from x_in = x_l, the backward from dx_out = dL/dx_{l+1}, on the context's
+ * compute stream and workspace (the same kernels and launches as in
+ * mt_train_step). MegaTrain's per-layer unit of work (MegaTrain abstract:
+ * parameters stream in, gradients stream out; intelligentliving.co,
+ * "Leveraging Double-Buffered Pipelining and Stateless Layer Templates").
+ * x_in, dx_out: HOST fp32 [b*s, d]; writes x_out = x_{l+1} and dx_in = dL/dx_l
+ * (HOST fp32 [b*s, d]) and the layer's fp32 gradients into grads, laid out as
+ * the layer's block of the arena: grads[i] is the gradient of arena element
+ * (offset of the layer's attention-norm gain) + i, for the floats between it
+ * and the next layer's attention-norm gain (grads_bytes at least that many
+ * times 4). Synchronous; the master arena and the moments are unchanged.
+ * MT_ERR_DEVICE if a kernel's bounded wait expired. */
+int mt_layer_fwd_bwd(mt_ctx* ctx, int layer, const float* x_in, const float* dx_out, float* x_out, float* dx_in,
+                     float* grads, size_t grads_bytes);
+
 /* Copies the current fp32 master weights (after the last update) to dst. */
 int mt_get_params(mt_ctx* ctx, float* dst, size_t bytes);
 

@@ -163,3 +163,39 @@ def test_full_step_properties():
     pa, _, _ = oracle.adamw_update(P0[idx], G[idx], 0, 0, 1, 1e-3, 0.9, 0.95, 1e-8, 0.1)
     assert np.allclose(P1[idx], pa, rtol=0, atol=2e-8 + 1e-6 * np.abs(pa))
     assert st["wait_weights_ms"] < 0.1 * st["step_ms"]  # prefetch keeps the compute stream fed
+
+
+@pytest.mark.parametrize("layer", [0, SH["L"] - 1])
+def test_layer_local_parity_full_shape(layer):
+    """Layer-local parity at the full 1.3B shape, in the launch configuration of
+    the training step: mt_layer_fwd_bwd runs the engine's layer forward and
+    backward on all 8 x 2048 tokens; the upstream gradient is nonzero only for
+    sequences 0 and 1, so the other sequences' input gradients are exactly
+    zero and every weight gradient is the sum over those two sequences, which
+    the oracle recomputes in fp64 (x_{l+1} and dx_l of sequences 0 and 1, all
+    nine weight gradients)."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    from layer_parity import layer_check
+    cfg = arena.config(SH)
+    cfg.seed = 5
+    ctx = mt.mt_create(cfg)
+    try:
+        n = mt.mt_arena_bytes(cfg) // 4
+        P = np.empty(n, dtype=np.float32)
+        mt.mt_get_params(ctx, P.ctypes.data, P.nbytes)
+        c = oracle.OracleConfig(**SH)
+        shapes = {tid: shp for lay, tid, _, shp in oracle.arena_layout(c)[0] if lay == layer}
+        W = {}
+        for tid in range(9):
+            o, k = mt.mt_tensor_offset(cfg, layer, tid)
+            W[tid] = oracle.bf16_round(P[o:o + k]).astype(np.float64).reshape(shapes[tid])
+        del P
+        rng = np.random.default_rng(layer)
+        x = rng.normal(size=(T, D)).astype(np.float32)
+        dxn = np.zeros((T, D), dtype=np.float32)
+        dxn[:2 * S] = rng.normal(size=(2 * S, D)).astype(np.float32)
+        xo, dxi, _ = layer_check(mt, ctx, cfg, SH, layer, W, x, dxn, [0, 1])
+        assert np.all(dxi[2 * S:] == 0.0)
+        assert np.isfinite(xo).all()
+    finally:
+        mt.mt_destroy(ctx)

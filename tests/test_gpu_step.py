@@ -14,6 +14,7 @@ import pytest
 
 import oracle
 import synth
+from layer_parity import layer_check
 
 pytestmark = pytest.mark.gpu
 
@@ -251,3 +252,28 @@ def test_gradient_ring_matches_full_arena_and_oracle():
     den = sum(float(np.sum(o["P"][k] ** 2)) for k in P)
     assert abs(ring[0]["loss"] - o["loss"]) <= 1e-2
     assert math.sqrt(num / den) <= 5e-3
+
+
+@pytest.mark.parametrize("name", ["gqa_ragged", "hd128"])
+def test_layer_template_matches_oracle(name):
+    """mt_layer_fwd_bwd (the engine's per-layer forward + backward on supplied
+    boundary activations) against the oracle's layer, for every layer."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    shape = SHAPES[name]
+    cfg = arena.config(shape)
+    init = synth.init_weights(shape, 3)
+    A = arena.pack(cfg, init)
+    ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+    rng = np.random.default_rng(11)
+    T, d = shape["b"] * shape["s"], shape["d"]
+    try:
+        for layer in range(shape["L"]):
+            W = {tid: oracle.bf16_round(init[(layer, tid)].astype(np.float32)).astype(np.float64) for tid in range(9)}
+            x = rng.normal(size=(T, d)).astype(np.float32)
+            dxn = rng.normal(size=(T, d)).astype(np.float32)
+            layer_check(mt, ctx, cfg, shape, layer, W, x, dxn, list(range(shape["b"])))
+        P = np.empty_like(A)
+        mt.mt_get_params(ctx, P.ctypes.data, P.nbytes)
+        assert np.array_equal(P, A)  # no optimizer step
+    finally:
+        mt.mt_destroy(ctx)
