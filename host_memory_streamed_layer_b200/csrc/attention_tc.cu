@@ -431,43 +431,42 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
 // Backward on the tcgen05 tensor cores (head_dim 128).
 //
 // One CTA per (128-key block, KV head, sequence); it loops over every query
-// head of the group and every 64-query block at or after its keys:
-//   S^T  = K Q^T,   dP^T = V dO^T          (128 keys x 64 queries, TMEM)
-//   P^T  = exp(S^T / sqrt(hd) - LSE),  dS^T = P^T (dP^T - D)   (softmax warps,
-//          one key row per thread, bf16 into 128-byte-swizzled tiles)
-//   dV  += P^T dO,  dK += dS^T Q            (128 keys x hd, TMEM, whole CTA)
-//   dQ^T = K^T dS^T                          (hd x 64 queries, TMEM), read out
-//          one head column per thread into an fp32 staging tile in shared
-//          memory, then added to the fp32 dQ accumulator with TMA bulk
-//          reduce-add (four 64 x 32 boxes per tile)
-// The K tile serves both as the K-major A operand of S^T (keys x hd) and as
-// the MN-major A operand of dQ^T (hd x keys); the dS^T tile both as the
-// K-major A operand of dK and the MN-major B operand of dQ^T.
+// head of the group and every 128-query block at or after its keys:
+//   S^T  = K Q^T,   dP^T = V dO^T            (128 keys x 128 queries, TMEM)
+//   P^T  = exp(S^T / sqrt(hd) - LSE),  dS^T = P^T (dP^T - D)   (gradient
+//          warps, one key row per thread; P^T and dS^T go back into the S^T
+//          columns as bf16 pairs, 16 queries' P^T then their dS^T in the 16
+//          columns those queries' scores came from, where dV and dK read them
+//          as their A operand; dS^T also into a 128-byte-swizzled shared tile)
+//   dV  += P^T dO,  dK += dS^T Q              (128 keys x hd, TMEM, A from TMEM)
+//   dQ^T = K^T dS^T                            (hd x 128 queries, into the
+//          dP^T columns), read out one head column per thread and added to
+//          the fp32 dQ accumulator with global reductions from registers
+// Every product is N = 128 wide: 64-wide products run the tensor core at
+// little more than half rate (55 instead of 32 cycles per 128 x 64 x 16 MMA,
+// measured), which bounded the 64-query form of this kernel.
+// Tensor memory: dK [0,128), dV [128,256), S^T / P^T|dS^T [256,384),
+// dP^T / dQ^T [384,512). Shared memory: K, V, two Q and two dO stages and the
+// dS^T tile, 32 KB each (224 KB).
 // ===========================================================================
 namespace {
 
-constexpr int FB_BKV = 128, FB_BQ = 64, FB_HD = 128;
-constexpr int FB_GWARPS = 16;                     // gradient warps: four per tensor-memory lane quarter
-constexpr int FB_QW = FB_BQ / (FB_GWARPS / 4);    // queries per gradient warp (16)
-constexpr int FB_THREADS = 64 + 32 * FB_GWARPS;   // producer, MMA, gradient warps
+constexpr int FB_BKV = 128, FB_BQ = 128, FB_HD = 128;
+constexpr int FB_GWARPS = 16;                   // gradient warps: four per tensor-memory lane quarter
+constexpr int FB_QW = FB_BQ / (FB_GWARPS / 4);  // queries per gradient warp (32)
+constexpr int FB_THREADS = 64 + 32 * FB_GWARPS; // producer, MMA, gradient warps
 
 struct FbCfg {
-  static constexpr int KV_BYTES = FB_BKV * FB_HD * 2;  // 32 KB
-  static constexpr int QT_BYTES = FB_BQ * FB_HD * 2;   // 16 KB (Q or dO tile)
-  static constexpr int T_BYTES = FB_BKV * FB_BQ * 2;   // 16 KB (P^T or dS^T)
+  static constexpr int TILE = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16 as two 64-column sub-tiles
+  static constexpr int SUB = 128 * 128;       // 16 KB: one 64-column sub-tile (128 rows x 128 B)
   static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + KV_BYTES;
-  static constexpr int OFF_Q = OFF_V + KV_BYTES;        // [2] stages
-  static constexpr int OFF_DO = OFF_Q + 2 * QT_BYTES;   // [2]
-  static constexpr int OFF_PT = OFF_DO + 2 * QT_BYTES;
-  static constexpr int OFF_DST = OFF_PT + T_BYTES;
-  static constexpr int OFF_DQS = OFF_DST + T_BYTES;     // dQ staging: 4 boxes [64 q][32 hd] fp32
-  static constexpr int DQS_BYTES = FB_BQ * FB_HD * 4;    // 32 KB
-  static constexpr int OFF_BAR = OFF_DQS + DQS_BYTES;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;       // [2] stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // [2]
+  static constexpr int OFF_DST = OFF_DO + 2 * TILE;
+  static constexpr int OFF_BAR = OFF_DST + TILE;
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
-  // tensor-memory columns: dK, dV, then two buffers of [S^T (64) | dP^T (64)];
-  // dQ^T of an iteration reuses the S^T columns of its buffer once consumed.
-  static constexpr uint32_t C_DK = 0, C_DV = 128, C_BUF = 256, BUF_COLS = 128, C_DP_OFF = 64;
+  static constexpr uint32_t C_DK = 0, C_DV = 128, C_S = 256, C_DP = 384;
 };
 
 struct FbParams {
@@ -486,10 +485,16 @@ struct FbParams {
   int vec_lse;  // LSE and D rows start 16-byte aligned: s % 4 == 0 and aligned bases
 };
 
+// Start-address step (address / 16) of k-step kk (16 elements of the
+// contraction) inside a K-major 128-row tile made of two 64-column sub-tiles.
+__device__ __forceinline__ uint32_t km_step(int kk) {
+  return (uint32_t)(((kk >> 2) * FbCfg::SUB + (kk & 3) * 32) >> 4);
+}
+
 __global__ void __launch_bounds__(FB_THREADS, 1)
     k_flash_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const __grid_constant__ CUtensorMap tmDQ, FbParams p) {
+                   FbParams p) {
   using C = FbCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -497,22 +502,19 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   uint8_t* sV = smem + C::OFF_V;
   uint8_t* sQ = smem + C::OFF_Q;
   uint8_t* sdO = smem + C::OFF_DO;
-  uint8_t* sPt = smem + C::OFF_PT;
   uint8_t* sdSt = smem + C::OFF_DST;
-  float* sDQ = reinterpret_cast<float*>(smem + C::OFF_DQS);
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   uint64_t* kv_full = bar + 0;
   uint64_t* q_full = bar + 1;    // [2]
   uint64_t* q_empty = bar + 3;   // [2]
-  uint64_t* s_full = bar + 5;    // [2] S^T, dP^T of a buffer ready
-  uint64_t* p_full = bar + 7;    // P^T, dS^T tiles written
-  uint64_t* mma_done = bar + 8;  // dV, dK, dQ^T of an iteration done
-  uint64_t* dq_empty = bar + 9;  // [2] dQ^T of a buffer read out
-  uint64_t* drain = bar + 11;
-  uint64_t* dq_staged = bar + 12;  // staging tile written
-  uint64_t* dq_free = bar + 13;    // the previous reduce has read the staging tile
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 14);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 15);
+  uint64_t* s_full = bar + 5;    // S^T and dP^T of an iteration ready
+  uint64_t* p_full = bar + 6;    // P^T, dS^T written (tensor and shared memory)
+  uint64_t* pdone = bar + 7;     // dV, dK of an iteration done (S^T columns free)
+  uint64_t* mma_done = bar + 8;  // dQ^T of an iteration done (and the dS^T tile read)
+  uint64_t* dq_empty = bar + 9;  // dQ^T read out (dP^T columns free)
+  uint64_t* drain = bar + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -529,21 +531,19 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&dq_empty[i], FB_GWARPS);
     }
+    mbar_init(s_full, 1);
     mbar_init(p_full, FB_GWARPS);
+    mbar_init(pdone, 1);
     mbar_init(mma_done, 1);
+    mbar_init(dq_empty, FB_GWARPS);
     mbar_init(drain, 1);
-    mbar_init(dq_staged, FB_GWARPS);
-    mbar_init(dq_free, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmO);
-    tma_prefetch_desc(&tmDQ);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -559,10 +559,10 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       // ---------------- TMA producer ----------------
       int q_last[2] = {-1, -1};
       bool ok = true;
-      mbar_arrive_expect_tx(kv_full, 2 * C::KV_BYTES);
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
       for (int c = 0; c < 2; ++c) {
-        tma_load_2d(sK + c * 16384, &tmK, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
-        tma_load_2d(sV + c * 16384, &tmV, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+        tma_load_2d(sK + c * C::SUB, &tmK, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+        tma_load_2d(sV + c * C::SUB, &tmV, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
       }
       int h = kvh * group, qb = qb_first;  // head and query block of iteration it
       for (int it = 0; it < n_it; ++it) {
@@ -578,10 +578,10 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&q_full[st], 2 * C::QT_BYTES);
+        mbar_arrive_expect_tx(&q_full[st], 2 * C::TILE);
         for (int c = 0; c < 2; ++c) {
-          tma_load_2d(sQ + st * C::QT_BYTES + c * 8192, &tmQ, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
-          tma_load_2d(sdO + st * C::QT_BYTES + c * 8192, &tmO, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
+          tma_load_2d(sQ + st * C::TILE + c * C::SUB, &tmQ, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
+          tma_load_2d(sdO + st * C::TILE + c * C::SUB, &tmO, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
         }
         q_last[st] = (int)ph;
       }
@@ -595,72 +595,69 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      // Order per iteration: S(it+1), dP(it+1) into the other buffer, then
-      // dV(it), dK(it), dQ^T(it); the tensor core works on the next scores
-      // while the gradient warps form P(it) and drain dQ^T(it-1).
-      constexpr uint32_t id_s = idesc_bf16_f32(FB_BKV, FB_BQ, false, false);   // keys x queries, K = hd
-      constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, FB_HD, false, true);   // keys x hd, K = queries
-      constexpr uint32_t id_dq = idesc_bf16_f32(FB_HD, FB_BQ, true, true);     // hd x queries, K = keys
+      constexpr uint32_t id_s = idesc_bf16_f32(FB_BKV, FB_BQ, false, false);  // keys x queries, K = hd
+      constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, FB_HD, false, true);  // keys x hd, K = queries (A in TMEM)
+      constexpr uint32_t id_dq = idesc_bf16_f32(FB_HD, FB_BQ, true, true);    // hd x queries, K = keys
       // Descriptors of the first k-step of each operand form; the loops add
-      // start-address steps (address / 16) instead of rebuilding them.
+      // start-address steps (address / 16).
       const uint64_t dK_km = sdesc_sw128(smem_u32(sK), 16, 1024), dV_km = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dQ_km = sdesc_sw128(smem_u32(sQ), 16, 1024), dO_km = sdesc_sw128(smem_u32(sdO), 16, 1024);
-      const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), 8192, 1024), dO_mn = sdesc_sw128(smem_u32(sdO), 8192, 1024);
-      const uint64_t dPt_km = sdesc_sw128(smem_u32(sPt), 16, 1024), ddSt_km = sdesc_sw128(smem_u32(sdSt), 16, 1024);
-      const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), 16384, 1024), ddSt_mn = sdesc_sw128(smem_u32(sdSt), 8192, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), C::SUB, 1024), dO_mn = sdesc_sw128(smem_u32(sdO), C::SUB, 1024);
+      const uint64_t dK_mn = sdesc_sw128(smem_u32(sK), C::SUB, 1024), ddSt_mn = sdesc_sw128(smem_u32(sdSt), C::SUB, 1024);
+      constexpr uint32_t kStage = C::TILE >> 4, kMn = 2048 >> 4;  // one stage; 16 rows of a 128-byte-row tile
       bool issued = false;
-      auto issue_s = [&](int it) -> bool {
+      bool ok = mbar_wait(kv_full, 0) && !*abort_flag;
+      if (!ok) record_error(p.err, 200);
+      for (int it = 0; it < n_it && ok; ++it) {
         const int st = it & 1;
         if (*abort_flag || !mbar_wait(&q_full[st], (it >> 1) & 1)) {
           record_error(p.err, 210 + (it & 63));
-          return false;
-        }
-        if (it >= 2 && !mbar_wait(&dq_empty[st], ((it - 2) >> 1) & 1)) {  // buffer st drained by iteration it-2
-          record_error(p.err, 250 + (it & 31));
-          return false;
-        }
-        tc_fence_after();
-        const uint32_t so = (st * C::QT_BYTES) >> 4;
-        const uint32_t cs = tmem + C::C_BUF + st * C::BUF_COLS;
-#pragma unroll
-        for (int kk = 0; kk < FB_HD / 16; ++kk) {
-          const uint32_t ka = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4, kb = so + (((kk >> 2) * 8192 + (kk & 3) * 32) >> 4);
-          umma_bf16(cs, dK_km + ka, dQ_km + kb, id_s, kk != 0);
-          umma_bf16(cs + C::C_DP_OFF, dV_km + ka, dO_km + kb, id_s, kk != 0);
-        }
-        issued = true;
-        umma_commit(&s_full[st]);
-        return true;
-      };
-      bool ok = mbar_wait(kv_full, 0) && !*abort_flag;
-      if (!ok) record_error(p.err, 200);
-      if (ok && n_it > 0) ok = issue_s(0);
-      for (int it = 0; it < n_it && ok; ++it) {
-        const int st = it & 1;
-        if (it + 1 < n_it && !issue_s(it + 1)) {
           ok = false;
           break;
         }
+        // S^T columns hold P^T | dS^T of the previous iteration until its dV, dK finish
+        if (it > 0 && !mbar_wait(pdone, (it - 1) & 1)) {
+          record_error(p.err, 230 + (it & 15));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < FB_HD / 16; ++kk)
+          umma_bf16(tmem + C::C_S, dK_km + km_step(kk), dQ_km + st * kStage + km_step(kk), id_s, kk != 0);
+        issued = true;
+        // dP^T columns hold dQ^T of the previous iteration until it is read out
+        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1)) {
+          record_error(p.err, 250 + (it & 15));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < FB_HD / 16; ++kk)
+          umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
+        umma_commit(s_full);
         if (*abort_flag || !mbar_wait(p_full, it & 1)) {
           record_error(p.err, 280 + (it & 15));
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t so = (st * C::QT_BYTES) >> 4;
-        // dV += P^T dO, dK += dS^T Q (K = 64 queries: 4 steps; B MN-major over hd, 8 KB between hd chunks)
+        // dV += P^T dO, dK += dS^T Q: K = 128 queries in 8 steps; query step kk
+        // (queries [16 kk, 16 kk + 16)) of P^T sits in columns C_S + 16 kk,
+        // its dS^T in the next 8 columns
 #pragma unroll
         for (int kk = 0; kk < FB_BQ / 16; ++kk) {
           const bool acc = (it > 0) || (kk > 0);
-          umma_bf16(tmem + C::C_DV, dPt_km + ((kk * 32) >> 4), dO_mn + so + ((kk * 2048) >> 4), id_kv, acc);
-          umma_bf16(tmem + C::C_DK, ddSt_km + ((kk * 32) >> 4), dQ_mn + so + ((kk * 2048) >> 4), id_kv, acc);
+          const uint32_t ap = tmem + C::C_S + 16 * kk;
+          umma_bf16_ts(tmem + C::C_DV, ap, dO_mn + st * kStage + kk * kMn, id_kv, acc);
+          umma_bf16_ts(tmem + C::C_DK, ap + 8, dQ_mn + st * kStage + kk * kMn, id_kv, acc);
         }
-        // dQ^T = K^T dS^T (K = 128 keys: 8 steps; A MN-major over hd, 16 KB between hd chunks) into the
-        // S^T columns of this iteration's buffer
+        umma_commit(pdone);
+        // dQ^T = K^T dS^T (K = 128 keys in 8 steps) into the dP^T columns
 #pragma unroll
         for (int kk = 0; kk < FB_BKV / 16; ++kk)
-          umma_bf16(tmem + C::C_BUF + st * C::BUF_COLS, dK_mn + ((kk * 2048) >> 4), ddSt_mn + ((kk * 2048) >> 4),
-                    id_dq, kk != 0);
+          umma_bf16(tmem + C::C_DP, dK_mn + kk * kMn, ddSt_mn + kk * kMn, id_dq, kk != 0);
         umma_commit(mma_done);
         umma_commit(&q_empty[st]);
       }
@@ -674,130 +671,107 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     }
   } else {
     // ---------------- gradient warps (2 .. 2 + FB_GWARPS) ----------------
-    // Warp w owns tensor-memory lane quarter w mod 4 (32 key rows) and query
-    // columns [FB_QW qg, FB_QW qg + FB_QW) of each 64-query block: four warps
-    // per quarter keep enough independent work in flight to hide the latency
-    // of the tensor-memory loads and the exponentials.
+    // Warp w owns tensor-memory lane quarter w mod 4 (32 key rows, or 32 head
+    // columns of dQ^T) and query columns [32 qg, 32 qg + 32) of each block.
     const int qg = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row == tensor-memory lane (the head column for dQ^T)
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const float sl2 = p.scale * 1.4426950408889634f;
     const int key = kv0 + r;
-    const bool issuer = (warp == 2 && lane == 0);  // issues the dQ reductions
-    const bool vec_ok = p.vec_lse != 0;            // LSE / D rows 16-byte aligned
+    const bool vec_ok = p.vec_lse != 0;  // LSE / D rows 16-byte aligned
     bool ok = true;
 
-    // Reads dQ^T of the iteration with head hq and query block start q0
-    // (already complete: the caller waited for it), stages it and lets the
-    // issuer add it to the accumulator.
-    auto flush_dq = [&](int it, int hq, int q0) -> bool {
-      const int bf = it & 1;
-      if (it > 0) {
-        // the staging tile is reused: the previous reduce must have read it
-        if (issuer) {
-          asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-          mbar_arrive(dq_free);
-        }
-        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(dq_free, (it - 1) & 1)) {
-          record_error(p.err, 600 + (it & 63));
-          return false;
-        }
-      }
-      float* col = sDQ + (r >> 5) * (FB_BQ * 32) + (r & 31);  // box r/32: [64 queries][32 head columns]
-      {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + qg * FB_QW, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) col[(qg * FB_QW + e) * 32] = __uint_as_float(v[e]) * p.scale;
-      }
+    // dQ^T of an iteration (complete: the caller waited for mma_done): this
+    // warp's 32 query columns for head column r, added to the fp32 dQ
+    // accumulator with reductions from registers (a warp's 32 lanes are 32
+    // consecutive head columns of one query row: 128 coalesced bytes).
+    auto flush_dq = [&](int hq, int q0) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tmem + lane_base + C::C_DP + qg * FB_QW, v);
+      tmem_ld_wait();
       tc_fence_before();
-      fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&dq_empty[bf]);
-        mbar_arrive(dq_staged);
-      }
-      if (issuer) {
-        if (!mbar_wait(dq_staged, it & 1)) {
-          record_error(p.err, 700 + (it & 63));
-          return false;
-        }
+      if (lane == 0) mbar_arrive(dq_empty);
+      const int qf = q0 + qg * FB_QW;
+      float* dst = p.dQacc + (int64_t)(row0 + qf) * p.ldqa + (int64_t)hq * FB_HD + r;
 #pragma unroll
-        for (int bx = 0; bx < 4; ++bx)
-          asm volatile(
-              "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                  reinterpret_cast<uint64_t>(&tmDQ)),
-              "r"(smem_u32(sDQ + bx * FB_BQ * 32)), "r"(hq * FB_HD + bx * 32), "r"(row0 + q0)
-              : "memory");
-        asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-      }
-      return true;
+      for (int e = 0; e < FB_QW; ++e)
+        if (qf + e < p.s)
+          asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + (int64_t)e * p.ldqa), "f"(__uint_as_float(v[e]) * p.scale)
+                       : "memory");
     };
 
     int h = kvh * group, qb = qb_first;  // head and query block of iteration it
     int h_prev = h, q0_prev = 0;         // those of iteration it - 1
     for (int it = 0; it < n_it; ++it) {
-      const int bf = it & 1;
       const int q0 = qb * FB_BQ, hq = h;
       if (++qb == nqb) {
         qb = qb_first;
         ++h;
+      }
+      // dQ^T of the previous iteration first: its columns take this iteration's dP^T
+      if (it > 0) {
+        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1)) {
+          record_error(p.err, 400 + (it & 63));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        flush_dq(h_prev, q0_prev);
       }
       const int qc = q0 + qg * FB_QW;  // first query of this warp's columns
       const float* lse = p.LSE + ((int64_t)b * p.H + hq) * p.s + qc;
       const float* dd = p.Dv + ((int64_t)b * p.H + hq) * p.s + qc;
       // Only blocks that touch the diagonal or a sequence end need the mask.
       const bool need_mask = (qc < kv0 + FB_BKV) || (q0 + FB_BQ > p.s) || (kv0 + FB_BKV > p.s);
-      // this warp's 16 LSE and D values (the same for every lane), loaded
-      // before the wait: broadcast float4 loads where the columns lie inside
-      // the sequence and rows start 16-byte aligned, else guarded scalar loads
-      float lv[FB_QW], dvv[FB_QW];
-      if (!need_mask && vec_ok) {
-#pragma unroll
-        for (int i = 0; i < FB_QW / 4; ++i) {
-          const float4 a4 = __ldg(reinterpret_cast<const float4*>(lse) + i);
-          const float4 d4 = __ldg(reinterpret_cast<const float4*>(dd) + i);
-          lv[4 * i] = a4.x * 1.4426950408889634f;
-          lv[4 * i + 1] = a4.y * 1.4426950408889634f;
-          lv[4 * i + 2] = a4.z * 1.4426950408889634f;
-          lv[4 * i + 3] = a4.w * 1.4426950408889634f;
-          dvv[4 * i] = d4.x;
-          dvv[4 * i + 1] = d4.y;
-          dvv[4 * i + 2] = d4.z;
-          dvv[4 * i + 3] = d4.w;
-        }
-      } else {
-#pragma unroll
-        for (int i = 0; i < FB_QW; ++i) {
-          const bool in = qc + i < p.s;
-          lv[i] = in ? __ldg(lse + i) * 1.4426950408889634f : 0.f;
-          dvv[i] = in ? __ldg(dd + i) : 0.f;
-        }
-      }
-      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&s_full[bf], (it >> 1) & 1)) {
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(s_full, it & 1)) {
         record_error(p.err, 300 + (it & 63));
         ok = false;
         break;
       }
       tc_fence_after();
-      // P^T and dS^T of this key row for this warp's 16 queries (bf16 pairs).
-      uint32_t pp[FB_QW / 2], ds[FB_QW / 2];
-      {
+      // Two halves of 16 queries: S^T, dP^T -> P^T, dS^T (bf16 pairs) back into
+      // this warp's own S^T columns (the ones it has just read) and into the
+      // shared dS^T tile.
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        float lv[16], dvv[16];
+        if (!need_mask && vec_ok) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float4 a4 = __ldg(reinterpret_cast<const float4*>(lse + hf * 16) + i);
+            const float4 d4 = __ldg(reinterpret_cast<const float4*>(dd + hf * 16) + i);
+            lv[4 * i] = a4.x * 1.4426950408889634f;
+            lv[4 * i + 1] = a4.y * 1.4426950408889634f;
+            lv[4 * i + 2] = a4.z * 1.4426950408889634f;
+            lv[4 * i + 3] = a4.w * 1.4426950408889634f;
+            dvv[4 * i] = d4.x;
+            dvv[4 * i + 1] = d4.y;
+            dvv[4 * i + 2] = d4.z;
+            dvv[4 * i + 3] = d4.w;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const bool in = qc + hf * 16 + i < p.s;
+            lv[i] = in ? __ldg(lse + hf * 16 + i) * 1.4426950408889634f : 0.f;
+            dvv[i] = in ? __ldg(dd + hf * 16 + i) : 0.f;
+          }
+        }
         uint32_t sv[16], dv[16];
-        const uint32_t cb = tmem + lane_base + C::C_BUF + bf * C::BUF_COLS + qg * FB_QW;
-        tmem_ld_32x32b_x16(cb, sv);
-        tmem_ld_32x32b_x16(cb + C::C_DP_OFF, dv);
+        tmem_ld_32x32b_x16(tmem + lane_base + C::C_S + qg * FB_QW + hf * 16, sv);
+        tmem_ld_32x32b_x16(tmem + lane_base + C::C_DP + qg * FB_QW + hf * 16, dv);
         tmem_ld_wait();
+        uint32_t pp[8], ds[8];
         auto grads = [&](auto mask_tag) {
           constexpr bool MASK = decltype(mask_tag)::value;
 #pragma unroll
-          for (int e = 0; e < FB_QW; e += 2) {
+          for (int e = 0; e < 16; e += 2) {
             float pv[2], dsv[2];
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
-              const int qi = qc + e + u;
+              const int qi = qc + hf * 16 + e + u;
               const bool vis = !MASK || (key <= qi && qi < p.s && key < p.s);
               const float pr = vis ? ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lv[e + u])) : 0.f;
               pv[u] = pr;
@@ -811,28 +785,24 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           grads(std::true_type{});
         else
           grads(std::false_type{});
-      }
-      // dV, dK, dQ^T of the previous iteration must be done with the tiles
-      if (it > 0 && (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1))) {
-        record_error(p.err, 400 + (it & 63));
-        ok = false;
-        break;
-      }
+        // P^T of queries [32 qg + 16 hf, +16) -> columns C_S + 32 qg + 16 hf, dS^T in the
+        // next 8: exactly the 16 columns this half has just read, so no warp
+        // overwrites scores another warp (or its own next half) still needs
+        tmem_st_32x32b_x8(tmem + lane_base + C::C_S + qg * FB_QW + hf * 16, pp);
+        tmem_st_32x32b_x8(tmem + lane_base + C::C_S + qg * FB_QW + hf * 16 + 8, ds);
+        // dS^T row r, queries [32 qg + 16 hf, +16): sub-tile qg / 2, 16-byte chunks 4 (qg % 2) + 2 hf, +1
 #pragma unroll
-      for (int c8 = 0; c8 < FB_QW / 8; ++c8) {
-        const int chunk = qg * (FB_QW / 8) + c8;  // 16-byte chunk of the 128-byte swizzled row
-        const int off = r * 128 + ((chunk ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(sPt + off) = make_uint4(pp[4 * c8], pp[4 * c8 + 1], pp[4 * c8 + 2], pp[4 * c8 + 3]);
-        *reinterpret_cast<uint4*>(sdSt + off) = make_uint4(ds[4 * c8], ds[4 * c8 + 1], ds[4 * c8 + 2], ds[4 * c8 + 3]);
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int chunk = 4 * (qg & 1) + 2 * hf + c2;
+          const int off = (qg >> 1) * C::SUB + r * 128 + ((chunk ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(sdSt + off) = make_uint4(ds[4 * c2], ds[4 * c2 + 1], ds[4 * c2 + 2], ds[4 * c2 + 3]);
+        }
       }
+      tmem_st_wait();
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(p_full);
-      if (it > 0 && !flush_dq(it - 1, h_prev, q0_prev)) {
-        ok = false;
-        break;
-      }
       h_prev = hq;
       q0_prev = q0;
     }
@@ -840,11 +810,11 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (n_it - 1) & 1)) {
         record_error(p.err, 450);
         ok = false;
-      } else if (!flush_dq(n_it - 1, h_prev, q0_prev)) {
-        ok = false;
+      } else {
+        tc_fence_after();
+        flush_dq(h_prev, q0_prev);
       }
     }
-    if (issuer) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     if (!ok) {
       *abort_flag = 1;
     } else if (n_it > 0) {
@@ -932,18 +902,17 @@ int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
     attr = true;
   }
   const int64_t T = (int64_t)a.b * a.s;
-  CUtensorMap mq, mk, mv, mo, mdq;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * FB_HD, T, a.ldqkv, FB_BQ) ||
       !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
       !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
-      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ) ||
-      !make_tensor_map_2d_f32(&mdq, a.dq_acc, (int64_t)a.H * FB_HD, T, a.ldqa, 32, FB_BQ))
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ))
     return MT_ERR_ARG;
   const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
              a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
-  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, p);
+  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
 
