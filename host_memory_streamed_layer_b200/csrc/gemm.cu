@@ -325,7 +325,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
+          // No tcgen05 fence here: the stage's bytes were written by TMA and
+          // published through this mbarrier, which orders them for the MMAs'
+          // shared-memory reads. A fence per k-block measurably stalled the
+          // tensor pipe (a 64-deep k-block took ~690 instead of 512 cycles).
           const uint64_t ad = a0 + stage * kStage, bd = b0 + stage * kStage;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) umma_bf16(d_tmem, ad + kk * kAStep, bd + kk * kBStep, idesc, (kb | kk) != 0);
@@ -556,7 +559,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
+          // No tcgen05 fence here: the stage's bytes were written by TMA and
+          // published through this mbarrier, which orders them for the MMAs'
+          // shared-memory reads. A fence per k-block measurably stalled the
+          // tensor pipe (a 64-deep k-block took ~690 instead of 512 cycles).
           const uint64_t ad = a0 + stage * kStage, bd = b0 + stage * kStage;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
@@ -778,10 +784,11 @@ int dispatch_pair(const GemmDesc& g, int max_pairs, cudaStream_t st, int* err) {
 
 // Automatic choice of the pair kernel. Measured on the decoder layer's shapes
 // (B200): pairs are 2-8 % faster than single-CTA tiles for every product whose
-// A operand is K-major (forward and input-gradient products, LM head); for the
-// weight gradients (both operands MN-major) they tie or lose, most where the
-// 128-wide pair tile is chosen, so those stay on single-CTA tiles.
-bool use_pair_auto(const GemmDesc& g) { return !g.a_mn; }
+// A operand is K-major (forward and input-gradient products, LM head). For the
+// weight gradients (both operands MN-major) 256-wide pair tiles tie or win
+// (q,k,v and gate|up), while 128-wide pair tiles lose by 20-30 % (down and O
+// projections): those stay on single-CTA tiles.
+bool use_pair_auto(const GemmDesc& g, bool pair_tile_256) { return !g.a_mn || pair_tile_256; }
 
 // Fraction of the pairs' time spent on real tiles when `tiles` tiles are dealt
 // round-robin to `pairs` persistent pairs.
@@ -820,10 +827,11 @@ int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* err) {
   const int max_pairs = g_num_sms / 2;
   const int tm = (g.M + 2 * BM - 1) / (2 * BM);
   const int t256 = tm * ((g.N + 255) / 256), t128 = tm * ((g.N + 127) / 128);
-  const bool pair_ok = g_variant == 2 || (g_variant == 0 && use_pair_auto(g));
-  if (pair_ok && g.N > 128 && t256 >= max_pairs) {
-    if (wave_efficiency(t128, max_pairs) > wave_efficiency(t256, max_pairs) + 0.08)
-      return dispatch_pair<128>(g, max_pairs, st, err);
+  const bool fits256 = g.N > 128 && t256 >= max_pairs;
+  const bool prefer256 = fits256 && wave_efficiency(t128, max_pairs) <= wave_efficiency(t256, max_pairs) + 0.08;
+  const bool pair_ok = g_variant == 2 || (g_variant == 0 && use_pair_auto(g, prefer256));
+  if (pair_ok && fits256) {
+    if (!prefer256) return dispatch_pair<128>(g, max_pairs, st, err);
     return dispatch_pair<256>(g, max_pairs, st, err);
   }
   if (pair_ok && t128 >= max_pairs) return dispatch_pair<128>(g, max_pairs, st, err);
