@@ -53,6 +53,8 @@ def parse():
     ap.add_argument("--workload", default="llama-1.3b", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="mt", choices=["mt", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--timeline", default="", metavar="PATH",
+                    help="write the last step's copy/compute timeline (Markdown) to PATH")
     ap.add_argument("--grads", default="ring", choices=["ring", "arena"],
                     help="host gradients: ring of layer slots (14 B/param of host memory) or a full arena (18)")
     ap.add_argument("--host-threads", type=int, default=0, help="host optimizer threads per replica (0: cores / N)")
@@ -271,6 +273,39 @@ def host_optimizer_bandwidth(mt, threads, n=1 << 28):
     return mt.mt_host_optimizer_gbs(n, threads)
 
 
+def write_timeline(tl, path, workload):
+    """Markdown timeline of one step: weight loads against the compute stream,
+    gradient offloads, and the host optimizer jobs."""
+    ph = tl["phases"]
+    out = [f"# Step timeline: {workload}, 1 B200", "",
+           "Device times in ms from the step's start on the compute stream (CUDA events); host optimizer",
+           "times in ms of host clock from the mt_train_step call (the two origins agree to tens of us).", "",
+           f"Phases: forward ends {ph['fwd_end']:.2f}, head ends {ph['head_end']:.2f}, backward ends "
+           f"{ph['bwd_end']:.2f}, step ends {ph['step_end']:.2f}.", "",
+           "## Weight loads (H2D stream) against the compute stream", "",
+           "| load | layer | H2D start | weights ready | compute reaches its wait | compute waits | slot released |",
+           "|---:|---:|---:|---:|---:|---:|---:|"]
+    wait_total = 0.0
+    for i, ld in enumerate(tl["loads"]):
+        w = max(0.0, ld["ready"] - ld["compute_arrives"])
+        wait_total += w
+        out.append(f"| {i} | {ld['layer']} | {ld['h2d_start']:.2f} | {ld['ready']:.2f} | {ld['compute_arrives']:.2f} "
+                   f"| {w:.3f} | {ld['released']:.2f} |")
+    out += ["", f"Compute stream waiting for weights in this step: {wait_total:.3f} ms.", "",
+            "## Gradient offloads (D2H stream)", "",
+            "| layer | gradients ready | D2H start | D2H done |", "|---:|---:|---:|---:|"]
+    for o in tl["offload"]:
+        out.append(f"| {o['layer']} | {o['grads_ready']:.2f} | {o['d2h_start']:.2f} | {o['d2h_done']:.2f} |")
+    kinds = {0: "layer", 1: "LM head", 2: "embedding (touched rows)", 3: "embedding (untouched rows)"}
+    out += ["", "## Host optimizer jobs (host clock)", "",
+            "| job | layer | gradients available | update done |", "|---|---:|---:|---:|"]
+    for j in tl["jobs"]:
+        out.append(f"| {kinds.get(j['kind'], j['kind'])} | {j['layer'] if j['kind'] == 0 else ''} "
+                   f"| {j['ready_ms']:.2f} | {j['done_ms']:.2f} |")
+    with open(path, "w") as f:
+        f.write("\n".join(out) + "\n")
+
+
 def phase_flops(sh):
     """(forward + head FLOPs, backward-phase FLOPs) of the schedule."""
     L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
@@ -388,6 +423,8 @@ def main():
         w1 = time.perf_counter()
         barrier()
         t_e2e = allmax(w1 - w0)
+        if args.timeline and rank == 0:
+            write_timeline(mt.mt_get_timeline(ctx), args.timeline, args.workload)
     finally:
         mt.mt_destroy(ctx)
 

@@ -143,6 +143,11 @@ struct mt_ctx {
   std::deque<Job> jobs;
   int jobs_pending = 0;
   int layer_jobs_done = 0;  // LAYER jobs finished this step: ring slots released
+  struct JobTime {
+    int kind, layer;
+    double ready, done;  // host seconds: gradients landed (wait ended), update finished
+  };
+  std::vector<JobTime> job_times;  // this step's optimizer jobs, in execution order
   bool opt_stop = false;
   int opt_status = MT_OK;
   bool skip_updates = false;
@@ -454,15 +459,23 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
   c->adamw_bytes += 30.0 * total;
 }
 
+void run_job_body(mt_ctx* c, const Job& j);
+
 void run_job(mt_ctx* c, const Job& j) {
-  const Layout& y = c->lay;
-  const Shapes& s = y.sh;
   if (!wait_event(c, j.ready)) {
     c->opt_status = MT_ERR_TIMEOUT;
     c->err = "gradient offload did not complete within the wait limit";
     c->skip_updates = true;
     return;
   }
+  const double t0 = now_s();
+  run_job_body(c, j);
+  c->job_times.push_back({(int)j.kind, j.layer, t0, now_s()});
+}
+
+void run_job_body(mt_ctx* c, const Job& j) {
+  const Layout& y = c->lay;
+  const Shapes& s = y.sh;
   if (j.kind == Job::EMBED_UNTOUCHED) {
     // Rows no token of this batch touches have a zero gradient, so their update
     // does not depend on this step's backward and runs while the GPU is in the
@@ -1140,6 +1153,7 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
     std::lock_guard<std::mutex> lk(c->opt_mu);
     c->layer_jobs_done = 0;
   }
+  c->job_times.clear();
   push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, s.L + 1});
   const double te0 = now_s();
   int r = enqueue_step(c, n_unique);
@@ -1264,6 +1278,48 @@ extern "C" int mt_set_state(mt_ctx* c, const float* params, const float* m, cons
 extern "C" int mt_get_stats(mt_ctx* c, mt_stats* out) {
   if (!c || !out) return MT_ERR_ARG;
   *out = c->stats;
+  return MT_OK;
+}
+
+extern "C" int mt_get_timeline(mt_ctx* c, float* out, size_t cap_floats, size_t* n_floats) {
+  if (!c || !n_floats) return MT_ERR_ARG;
+  const int L = c->lay.sh.L;
+  const size_t nloads = c->load_seq.size();
+  const size_t nj = c->job_times.size();
+  const size_t need = 3 + 5 * nloads + 4 * (size_t)L + 4 + 4 * nj;
+  *n_floats = need;
+  if (!out) return MT_OK;
+  if (cap_floats < need) return set_err(c, MT_ERR_ARG, "timeline buffer too small");
+  if (c->step == 0) return set_err(c, MT_ERR_ARG, "no step has run");
+  CK(cudaSetDevice(c->device));
+  auto t = [&](cudaEvent_t e) { return ev_ms(c->ev_step_start, e); };
+  size_t k = 0;
+  out[k++] = (float)nloads;
+  out[k++] = (float)L;
+  out[k++] = (float)nj;
+  for (size_t i = 0; i < nloads; ++i) {
+    out[k++] = (float)c->load_seq[i];
+    out[k++] = t(c->ev_h2d_start[i]);
+    out[k++] = t(c->ev_wready[i]);
+    out[k++] = t(c->ev_compready[i]);
+    out[k++] = t(c->ev_slotfree[i]);
+  }
+  for (int b = 0; b < L; ++b) {
+    out[k++] = (float)(L - 1 - b);
+    out[k++] = t(c->ev_gready[b]);
+    out[k++] = t(c->ev_d2h_start[b]);
+    out[k++] = t(c->ev_gdrained[b]);
+  }
+  out[k++] = t(c->ev_fwd_end);
+  out[k++] = t(c->ev_head_end);
+  out[k++] = t(c->ev_bwd_end);
+  out[k++] = t(c->ev_step_end);
+  for (const auto& jt : c->job_times) {
+    out[k++] = (float)jt.kind;
+    out[k++] = (float)jt.layer;
+    out[k++] = (float)((jt.ready - c->call_t0) * 1e3);
+    out[k++] = (float)((jt.done - c->call_t0) * 1e3);
+  }
   return MT_OK;
 }
 

@@ -207,6 +207,7 @@ _sig("mt_host_state_bytes", c_size_t, _cfgp)
 _sig("mt_create", c_int, _cfgp, c_void_p, c_size_t, ctypes.POINTER(c_void_p))
 _sig("mt_train_step", c_int, c_void_p, c_void_p, c_void_p, ctypes.POINTER(ctypes.c_float))
 _sig("mt_get_grads", c_int, c_void_p, c_void_p, c_size_t)
+_sig("mt_get_timeline", c_int, c_void_p, c_void_p, c_size_t, ctypes.POINTER(c_size_t))
 _sig("mt_layer_fwd_bwd", c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_params", c_int, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
@@ -268,6 +269,28 @@ def mt_layer_fwd_bwd(ctx: int, layer: int, x_in: int, dx_out: int, x_out: int, d
                      grads_bytes: int):
     return _check(lib.mt_layer_fwd_bwd(ctx, layer, x_in, dx_out, x_out, dx_in, grads, grads_bytes),
                   "mt_layer_fwd_bwd", ctx)
+
+
+def mt_get_timeline(ctx: int) -> dict:
+    """Timeline of the last step (see include/mt.h), as a dict of lists."""
+    n = c_size_t(0)
+    _check(lib.mt_get_timeline(ctx, None, 0, ctypes.byref(n)), "mt_get_timeline", ctx)
+    buf = (ctypes.c_float * n.value)()
+    _check(lib.mt_get_timeline(ctx, buf, n.value, ctypes.byref(n)), "mt_get_timeline", ctx)
+    v = list(buf)
+    nl, L, nj = int(v[0]), int(v[1]), int(v[2])
+    k = 3
+    loads = [dict(layer=int(v[k + 5 * i]), h2d_start=v[k + 5 * i + 1], ready=v[k + 5 * i + 2],
+                  compute_arrives=v[k + 5 * i + 3], released=v[k + 5 * i + 4]) for i in range(nl)]
+    k += 5 * nl
+    offload = [dict(layer=int(v[k + 4 * i]), grads_ready=v[k + 4 * i + 1], d2h_start=v[k + 4 * i + 2],
+                    d2h_done=v[k + 4 * i + 3]) for i in range(L)]
+    k += 4 * L
+    phases = dict(fwd_end=v[k], head_end=v[k + 1], bwd_end=v[k + 2], step_end=v[k + 3])
+    k += 4
+    jobs = [dict(kind=int(v[k + 4 * i]), layer=int(v[k + 4 * i + 1]), ready_ms=v[k + 4 * i + 2],
+                 done_ms=v[k + 4 * i + 3]) for i in range(nj)]
+    return dict(loads=loads, offload=offload, phases=phases, jobs=jobs)
 
 
 def mt_get_params(ctx: int, dst_ptr: int, nbytes: int):

@@ -189,6 +189,23 @@ int mt_set_state(mt_ctx* ctx, const float* params, const float* m, const float* 
 /* Counters of the last step. */
 int mt_get_stats(mt_ctx* ctx, mt_stats* out);
 
+/* Timeline of the last step, for seeing the copy/compute overlap of the
+ * pipeline (a profiler-free trace). Writes *n_floats; with out == NULL only
+ * the size. Layout (floats):
+ *   [0] n_loads (2L-1 weight loads), [1] L, [2] n_jobs;
+ *   per weight load i: layer, H2D start, weights ready, compute stream
+ *     reaches its wait for them, compute stream releases the slot;
+ *   per backward layer (order L-1 .. 0): layer, gradients ready on the
+ *     compute stream, D2H start, D2H done;
+ *   forward end, head end, backward end, step end;
+ *   per host optimizer job (execution order): kind (0 layer, 1 LM head,
+ *     2 touched embedding rows, 3 untouched embedding rows), layer (-1 for
+ *     the others), gradients available, update finished.
+ * Device times are ms from the step's start on the compute stream (CUDA
+ * events); host job times are ms of host clock from the mt_train_step call,
+ * a separate clock whose origin is within a few tens of microseconds of it. */
+int mt_get_timeline(mt_ctx* ctx, float* out, size_t cap_floats, size_t* n_floats);
+
 /* The context's compute stream (a cudaStream_t) in *stream, so a caller can
  * order or time its own work against the step (for example record CUDA events
  * around a sequence of mt_train_step calls). The stream stays owned by the

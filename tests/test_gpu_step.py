@@ -277,3 +277,38 @@ def test_layer_template_matches_oracle(name):
         assert np.array_equal(P, A)  # no optimizer step
     finally:
         mt.mt_destroy(ctx)
+
+
+def test_step_timeline_is_consistent():
+    """mt_get_timeline after a step: 2L-1 weight loads in the order 0..L-1,
+    L-2..0; every load's H2D precedes its readiness and every offload follows
+    its gradients; the backward offloads run L-1..0; the host ran one job per
+    layer plus the head and both embedding jobs, each after its data."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    shape = dict(L=4, d=256, H=4, Hkv=4, F=688, V=1024, b=2, s=128)
+    cfg = arena.config(shape)
+    cfg.host_threads = 4
+    ctx = mt.mt_create(cfg)
+    try:
+        tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0)
+        for _ in range(2):
+            mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+        tl = mt.mt_get_timeline(ctx)
+    finally:
+        mt.mt_destroy(ctx)
+    L = shape["L"]
+    assert [x["layer"] for x in tl["loads"]] == list(range(L)) + list(range(L - 2, -1, -1))
+    eps = 1e-3
+    for ld in tl["loads"]:
+        assert 0 - eps <= ld["h2d_start"] <= ld["ready"] + eps
+        assert ld["ready"] <= ld["released"] + eps and ld["compute_arrives"] <= ld["released"] + eps
+    assert [o["layer"] for o in tl["offload"]] == list(range(L - 1, -1, -1))
+    for o in tl["offload"]:
+        assert o["grads_ready"] <= o["d2h_start"] + eps <= o["d2h_done"] + 2 * eps
+        assert o["d2h_done"] <= tl["phases"]["step_end"] + eps
+    ph = tl["phases"]
+    assert ph["fwd_end"] <= ph["head_end"] <= ph["bwd_end"] <= ph["step_end"]
+    kinds = sorted(j["kind"] for j in tl["jobs"])
+    assert kinds == [0] * L + [1, 2, 3]
+    assert sorted(j["layer"] for j in tl["jobs"] if j["kind"] == 0) == list(range(L))
+    assert all(j["ready_ms"] <= j["done_ms"] for j in tl["jobs"])
