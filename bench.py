@@ -319,6 +319,42 @@ def phase_flops(sh):
 
 
 # ---------------------------------------------------------------------------
+# Cross-rank helpers: one process per GPU, replicas with no data-path
+# collective. NCCL on the GPU run; the CPU tests drive the same code on gloo.
+# ---------------------------------------------------------------------------
+class Ranks:
+    def __init__(self, torch, dist=None, device=None):
+        self.torch, self.dist, self.device = torch, dist, device
+
+    def allmax(self, x: float) -> float:
+        """Maximum of x over the ranks (the timed region is the slowest rank's)."""
+        if self.dist is None:
+            return float(x)
+        t = self.torch.tensor([float(x)], device=self.device, dtype=self.torch.float64)
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def all_ok(self, ok: bool) -> bool:
+        """True only if every rank passes ok=True: every rank takes the same branch."""
+        return -self.allmax(-1.0 if ok else 0.0) >= 1.0
+
+    def barrier(self):
+        if self.dist is not None:
+            self.dist.barrier()
+
+
+def host_ram_fits(need_bytes: int, world: int, avail_bytes, margin_bytes: int = 6 << 30) -> bool:
+    """Every replica holds its own host state: N replicas fit when N times one
+    replica's bytes plus a margin stay under the host's available memory."""
+    return avail_bytes is None or need_bytes * world + margin_bytes < avail_bytes
+
+
+def weak_value(tokens_per_rank_step: int, world: int, steps: int, t_max_s: float) -> float:
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank_step * world * steps / t_max_s
+
+
+# ---------------------------------------------------------------------------
 # Main arm.
 # ---------------------------------------------------------------------------
 def main():
@@ -338,16 +374,8 @@ def main():
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=timedelta(seconds=600), device_id=dev)
 
-    def allmax(x):
-        if dist is None:
-            return x
-        t = torch.tensor([float(x)], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    def barrier():
-        if dist is not None:
-            dist.barrier()
+    ranks = Ranks(torch, dist, dev)
+    allmax, barrier = ranks.allmax, ranks.barrier
 
     from host_memory_streamed_layer_b200 import arena, mt
     sh = synth.WORKLOADS[args.workload]
@@ -369,9 +397,7 @@ def main():
         avail = psutil.virtual_memory().available
     except Exception:
         avail = None
-    ok = 1.0 if (avail is None or need * world + (6 << 30) < avail) else 0.0
-    ok = -allmax(-ok) if dist is not None else ok
-    if ok < 1:
+    if not ranks.all_ok(host_ram_fits(need, world, avail)):
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": None, "unit": UNIT, "n_gpus": world,
                               "error": f"host RAM: {world} replicas need {need * world / 1e9:.0f} GB, "
@@ -432,7 +458,7 @@ def main():
         P, ptype = peaks()
         model_f, exec_f = flops_per_step(sh)
         K = args.steps
-        value = world * T * K / t_dev
+        value = weak_value(T, world, K, t_dev)
         ms = t_dev / K * 1e3
         g_fl = sum(s["gemm_flops"] for s in stats)
         g_ms = sum(s["gemm_ms"] for s in stats)
@@ -495,7 +521,7 @@ def main():
                               "adamw_last_ms": mean("adamw_last_ms"), "enqueue_ms": mean("enqueue_ms")},
             "loss": losses[-1],
             "clocks": clk,
-            "e2e": {"value": world * T * K / t_e2e, "unit": UNIT, "h2d_bytes_per_step": 2 * T * 4,
+            "e2e": {"value": weak_value(T, world, K, t_e2e), "unit": UNIT, "h2d_bytes_per_step": 2 * T * 4,
                     "d2h_bytes_per_step": 4, "timing": "host wall clock around mt_train_step (public C API)"},
             "gpu_launches": int(sum(s["kernel_launches"] for s in stats)),
         }
