@@ -1217,6 +1217,39 @@ extern "C" int mt_layer_fwd_bwd(mt_ctx* c, int l, const float* x_in, const float
   return MT_OK;
 }
 
+extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* labels, float* loss_out, float* dx_L,
+                               float* grads, size_t grads_bytes) {
+  if (!c) return MT_ERR_ARG;
+  if (!x_L || !labels || !loss_out || !dx_L || !grads) return set_err(c, MT_ERR_ARG, "NULL argument");
+  const Layout& y = c->lay;
+  const Shapes& s = y.sh;
+  const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
+  if (grads_bytes < head_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than the final-norm + head block");
+  for (int t = 0; t < s.T; ++t)
+    if (labels[t] < 0 || labels[t] >= s.V) return set_err(c, MT_ERR_ARG, "label outside [0, V)");
+  CK(cudaSetDevice(c->device));
+  const size_t n = (size_t)s.T * s.d;
+  cudaStream_t sc = c->s_comp;
+  c->timing_used = 0;
+  c->timed.clear();
+  c->err.clear();
+  const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
+  CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, head_bf * 2, cudaMemcpyHostToDevice, sc));
+  CK(cudaMemcpyAsync(c->xb + (size_t)s.L * n, x_L, n * 4, cudaMemcpyHostToDevice, sc));
+  CK(cudaMemcpyAsync(c->d_lab, labels, (size_t)s.T * 4, cudaMemcpyHostToDevice, sc));
+  CKM(head_step(c, c->gx0));
+  CK(cudaMemcpyAsync(c->misc_h, c->d_loss, 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(dx_L, c->gx0, n * 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(grads, c->d_head_g, head_f * 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
+  CK(cudaStreamSynchronize(sc));
+  int32_t dev_err;
+  memcpy(&dev_err, c->misc_h + 1, 4);
+  if (dev_err != 0) return set_err(c, MT_ERR_DEVICE, "kernel reported an error (bounded wait expired)");
+  *loss_out = c->misc_h[0] / (float)s.T;
+  return MT_OK;
+}
+
 extern "C" int mt_get_grads(mt_ctx* c, float* dst, size_t bytes) {
   if (!c || !dst) return MT_ERR_ARG;
   if (!c->grad) return set_err(c, MT_ERR_CONFIG, "created with MT_FLAG_GRAD_RING: no gradient arena is kept");

@@ -208,6 +208,7 @@ _sig("mt_create", c_int, _cfgp, c_void_p, c_size_t, ctypes.POINTER(c_void_p))
 _sig("mt_train_step", c_int, c_void_p, c_void_p, c_void_p, ctypes.POINTER(ctypes.c_float))
 _sig("mt_get_grads", c_int, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_timeline", c_int, c_void_p, c_void_p, c_size_t, ctypes.POINTER(c_size_t))
+_sig("mt_head_fwd_bwd", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t)
 _sig("mt_layer_fwd_bwd", c_int, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_params", c_int, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
@@ -269,6 +270,13 @@ def mt_layer_fwd_bwd(ctx: int, layer: int, x_in: int, dx_out: int, x_out: int, d
                      grads_bytes: int):
     return _check(lib.mt_layer_fwd_bwd(ctx, layer, x_in, dx_out, x_out, dx_in, grads, grads_bytes),
                   "mt_layer_fwd_bwd", ctx)
+
+
+def mt_head_fwd_bwd(ctx: int, x_L: int, labels: int, dx_L: int, grads: int, grads_bytes: int) -> float:
+    loss = ctypes.c_float(0.0)
+    _check(lib.mt_head_fwd_bwd(ctx, x_L, labels, ctypes.byref(loss), dx_L, grads, grads_bytes),
+           "mt_head_fwd_bwd", ctx)
+    return loss.value
 
 
 def mt_get_timeline(ctx: int) -> dict:

@@ -171,6 +171,19 @@ int mt_get_grads(mt_ctx* ctx, float* dst, size_t bytes);
 int mt_layer_fwd_bwd(mt_ctx* ctx, int layer, const float* x_in, const float* dx_out, float* x_out, float* dx_in,
                      float* grads, size_t grads_bytes);
 
+/* The head of the step on its own, with no optimizer step: final RMSNorm,
+ * LM-head logits, cross-entropy against labels (mean over the b*s tokens)
+ * and its backward, through the same kernels, token chunks and launches as
+ * mt_train_step, with the current bf16 streamed final gain and head.
+ * x_L: HOST fp32 [b*s, d] (the last layer's output); labels: HOST int32
+ * [b*s] in [0, V) (MT_ERR_ARG otherwise, checked first). Writes the loss,
+ * dx_L = dL/dx_L (HOST fp32 [b*s, d]) and the gradients of the final gain and
+ * the LM head into grads, laid out as the arena from the final gain's offset
+ * on (grads_bytes at least 4 * (LM head offset + V*d - final gain offset)).
+ * Synchronous; the master arena and the moments are unchanged. */
+int mt_head_fwd_bwd(mt_ctx* ctx, const float* x_L, const int32_t* labels, float* loss_out, float* dx_L,
+                    float* grads, size_t grads_bytes);
+
 /* Copies the current fp32 master weights (after the last update) to dst. */
 int mt_get_params(mt_ctx* ctx, float* dst, size_t bytes);
 

@@ -40,3 +40,38 @@ def layer_check(mt, ctx, cfg, shape, layer, W, x, dxn, seqs, tol=2e-2):
     assert max(worst.values()) <= tol, worst
     return xo, dxi, g
 
+
+
+def head_check(mt, ctx, cfg, shape, x, labels, chunk=None, tol=2e-2):
+    """Runs mt_head_fwd_bwd on x ([b*s, d] fp32) and labels and compares the
+    loss, dx_L and the final-gain and LM-head gradients with the oracle's head
+    on the bf16 streamed weights, token-chunked (each chunk's mean loss and
+    gradients rescaled to the mean over all tokens)."""
+    T, d, V = shape["b"] * shape["s"], shape["d"], shape["V"]
+    n = mt.mt_arena_bytes(cfg) // 4
+    P = np.empty(n, dtype=np.float32)
+    mt.mt_get_params(ctx, P.ctypes.data, P.nbytes)
+    fo, _ = mt.mt_tensor_offset(cfg, -1, mt.MT_T_FINAL_NORM)
+    ho, hn = mt.mt_tensor_offset(cfg, -1, mt.MT_T_LM_HEAD)
+    gf = oracle.bf16_round(P[fo:fo + d]).astype(np.float64)
+    Wh = oracle.bf16_round(P[ho:ho + hn]).astype(np.float64).reshape(V, d)
+    del P
+    dx = np.empty_like(x)
+    g = np.empty(ho + hn - fo, dtype=np.float32)
+    loss = mt.mt_head_fwd_bwd(ctx, x.ctypes.data, labels.ctypes.data, dx.ctypes.data, g.ctypes.data, g.nbytes)
+    chunk = chunk or T
+    rl, rdx, rdgf, rdW = 0.0, np.empty((T, d)), np.zeros(d), np.zeros((V, d))
+    eps = oracle.OracleConfig(**shape).norm_eps
+    for t0 in range(0, T, chunk):
+        t1 = min(T, t0 + chunk)
+        w = (t1 - t0) / T
+        l_c, dx_c, dgf_c, dW_c = oracle.head_ce_fwd_bwd(x[t0:t1].astype(np.float64), gf, Wh, labels[t0:t1], eps)
+        rl += w * l_c
+        rdx[t0:t1] = w * dx_c
+        rdgf += w * dgf_c
+        rdW += w * dW_c
+    assert abs(loss - rl) <= 1e-2, (loss, rl)
+    assert rel(dx, rdx) <= tol
+    assert rel(g[:d], rdgf) <= tol
+    assert rel(g[ho - fo:].reshape(V, d), rdW) <= tol
+    return loss

@@ -199,3 +199,20 @@ def test_layer_local_parity_full_shape(layer):
         assert np.isfinite(xo).all()
     finally:
         mt.mt_destroy(ctx)
+
+
+def test_head_parity_full_shape():
+    """Head + cross-entropy parity at the full 1.3B shape (8 x 2048 tokens,
+    vocab 32000) through mt_head_fwd_bwd, against the oracle token-chunked."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    from layer_parity import head_check
+    cfg = arena.config(SH)
+    cfg.seed = 9
+    ctx = mt.mt_create(cfg)
+    try:
+        x = np.random.default_rng(3).normal(size=(T, D)).astype(np.float32)
+        _, lab = synth.tokens_labels(B, S, V, 4)
+        loss = head_check(mt, ctx, cfg, SH, x, np.ascontiguousarray(lab.reshape(-1)).astype(np.int32), chunk=2048)
+        assert abs(loss - (math.log(V) + 0.0004 * D / 2)) < 0.15  # unit-RMS inputs: the closed form holds
+    finally:
+        mt.mt_destroy(ctx)

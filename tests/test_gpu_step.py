@@ -312,3 +312,26 @@ def test_step_timeline_is_consistent():
     assert kinds == [0] * L + [1, 2, 3]
     assert sorted(j["layer"] for j in tl["jobs"] if j["kind"] == 0) == list(range(L))
     assert all(j["ready_ms"] <= j["done_ms"] for j in tl["jobs"])
+
+
+def test_head_matches_oracle(monkeypatch):
+    """mt_head_fwd_bwd (final norm, LM head in token chunks, CE and its
+    backward, as in the step) against the oracle's head."""
+    monkeypatch.setenv("MT_LOGITS_CHUNK", "128")  # T = 300: chunks of 128, 128, 44
+    from host_memory_streamed_layer_b200 import arena, mt
+    from layer_parity import head_check
+    shape = SHAPES["gqa_ragged"]
+    cfg = arena.config(shape)
+    ctx = mt.mt_create(cfg)
+    try:
+        T = shape["b"] * shape["s"]
+        x = np.random.default_rng(5).normal(size=(T, shape["d"])).astype(np.float32)
+        _, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 2)
+        head_check(mt, ctx, cfg, shape, x, np.ascontiguousarray(lab.reshape(-1)).astype(np.int32))
+        with pytest.raises(mt.MTError) as e:
+            bad = np.full(T, shape["V"], dtype=np.int32)
+            g = np.empty(1 << 22, dtype=np.float32)
+            mt.mt_head_fwd_bwd(ctx, x.ctypes.data, bad.ctypes.data, x.ctypes.data, g.ctypes.data, g.nbytes)
+        assert e.value.code == -1
+    finally:
+        mt.mt_destroy(ctx)
