@@ -3,6 +3,7 @@
     python -m host_memory_streamed_layer_b200.kernel_bench gemm [--shape NAME] [--iters N]
     python -m host_memory_streamed_layer_b200.kernel_bench attn [--fwd-only] [--iters N]
     python -m host_memory_streamed_layer_b200.kernel_bench rmsnorm_bwd [--iters N]
+    python -m host_memory_streamed_layer_b200.kernel_bench elementwise [--iters N]
 
 Times each launch with CUDA events on the launching stream after warm-up and
 prints achieved TFLOP/s (tensor-bound kernels) or GB/s of algorithmic bytes
@@ -113,9 +114,52 @@ def bench_rmsnorm_bwd(iters, warmup):
     return [{"kernel": "rmsnorm_bwd", "us": sec * 1e6, "gbs": byt / sec / 1e9 if sec else None}]
 
 
+def bench_elementwise(iters, warmup):
+    """The HBM-bound kernels of the layer at the 1.3B shape, each against its
+    algorithmic bytes (every input read once, every output written once)."""
+    st = torch.cuda.current_stream().cuda_stream
+    dev = "cuda"
+    out = []
+
+    def rec(name, fn, nbytes):
+        sec = timed(fn, iters, warmup)
+        out.append({"kernel": name, "us": sec * 1e6, "bytes": nbytes, "gbs": nbytes / sec / 1e9 if sec else None})
+
+    x = torch.randn(T, D, device=dev)
+    g = torch.ones(D, device=dev, dtype=torch.bfloat16)
+    y = torch.empty(T, D, device=dev, dtype=torch.bfloat16)
+    rstd = torch.empty(T, device=dev)
+    rec("rmsnorm_fwd", lambda: mt.mt_k_rmsnorm_fwd(x.data_ptr(), g.data_ptr(), y.data_ptr(), rstd.data_ptr(), T, D,
+                                                   1e-5, st), T * (6 * D + 4))
+    gu = torch.randn(T, 2 * F, device=dev).to(torch.bfloat16)
+    act = torch.empty(T, F, device=dev, dtype=torch.bfloat16)
+    rec("swiglu_fwd", lambda: mt.mt_k_swiglu_fwd(gu.data_ptr(), act.data_ptr(), T, F, st), T * 6 * F)
+    dact = torch.randn(T, F, device=dev).to(torch.bfloat16)
+    dgu = torch.empty(T, 2 * F, device=dev, dtype=torch.bfloat16)
+    rec("swiglu_bwd", lambda: mt.mt_k_swiglu_bwd(gu.data_ptr(), dact.data_ptr(), dgu.data_ptr(), T, F, st),
+        T * 10 * F)
+    del gu, act, dact, dgu
+    Tc = 4096
+    z = torch.randn(Tc, V, device=dev)
+    lab = torch.randint(0, V, (Tc,), device=dev, dtype=torch.int32)
+    dz = torch.empty(Tc, V, device=dev, dtype=torch.bfloat16)
+    rl = torch.empty(Tc, device=dev)
+    rec("softmax_ce", lambda: mt.mt_k_softmax_ce(z.data_ptr(), V, lab.data_ptr(), dz.data_ptr(), V, rl.data_ptr(), Tc,
+                                                 V, 1.0 / T, st), Tc * 6 * V)
+    del z, dz
+    E = torch.randn(V, D, device=dev).to(torch.bfloat16)
+    tok = torch.randint(0, V, (T,), device=dev, dtype=torch.int32)
+    xe = torch.empty(T, D, device=dev)
+    rec("embed_fwd (table in HBM)", lambda: mt.mt_k_embed_fwd(tok.data_ptr(), E.data_ptr(), xe.data_ptr(), T, D, st),
+        T * 6 * D)
+    out += bench_rmsnorm_bwd(iters, warmup)
+    out[-1]["bytes"] = 18.0 * T * D
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["gemm", "attn", "rmsnorm_bwd"])
+    ap.add_argument("kernel", choices=["gemm", "attn", "rmsnorm_bwd", "elementwise"])
     ap.add_argument("--shape", default="all")
     ap.add_argument("--iters", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
@@ -127,6 +171,8 @@ def main():
         res = bench_gemm(names, a.iters, a.warmup)
     elif a.kernel == "attn":
         res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl)
+    elif a.kernel == "elementwise":
+        res = bench_elementwise(a.iters, a.warmup)
     else:
         res = bench_rmsnorm_bwd(a.iters, a.warmup)
     for r in res:
