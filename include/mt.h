@@ -19,6 +19,16 @@
  *   - argument, configuration and token-range errors are detected on the host
  *     before any device work and leave all state untouched;
  *   - a context is not thread-safe: one caller thread at a time.
+ *
+ * Environment read by mt_create:
+ *   MT_WAIT_LIMIT_S  limit, in seconds, of every host wait on GPU work and of
+ *                    a gradient-ring slot (default 600); past it a call
+ *                    returns MT_ERR_TIMEOUT;
+ *   MT_LOGITS_CHUNK  tokens per LM-head chunk, a multiple of 128 below the
+ *                    default (the default keeps fp32 logits + bf16 dz of a
+ *                    chunk under ~4 GiB); smaller chunks use less device
+ *                    memory and compute the same result.
+ * and by the GEMM launcher: MT_GEMM_VARIANT (see mt_kernels.h).
  */
 #ifndef MT_H_
 #define MT_H_
