@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--grads", default="ring", choices=["ring", "arena"],
                     help="host gradients: ring of layer slots (14 B/param of host memory) or a full arena (18)")
     ap.add_argument("--host-threads", type=int, default=0, help="host optimizer threads per replica (0: cores / N)")
+    ap.add_argument("--no-defer", action="store_true",
+                    help="run every update inside its own step (no MT_FLAG_DEFER_UPDATES)")
     return ap.parse_args()
 
 
@@ -296,14 +298,38 @@ def write_timeline(tl, path, workload):
             "| layer | gradients ready | D2H start | D2H done |", "|---:|---:|---:|---:|"]
     for o in tl["offload"]:
         out.append(f"| {o['layer']} | {o['grads_ready']:.2f} | {o['d2h_start']:.2f} | {o['d2h_done']:.2f} |")
-    kinds = {0: "layer", 1: "LM head", 2: "embedding (touched rows)", 3: "embedding (untouched rows)"}
+    kinds = {0: "layer", 1: "LM head", 2: "embedding (touched rows)", 3: "embedding (untouched rows)",
+             4: "LM head, previous step's deferred update", 5: "layer, previous step's deferred update"}
+    deferred = {j["layer"] for j in tl["jobs"] if j["kind"] == 5}
+    has_head = any(j["kind"] == 4 for j in tl["jobs"])
     out += ["", "## Host optimizer jobs (host clock)", "",
             "| job | layer | gradients available | update done |", "|---|---:|---:|---:|"]
     for j in tl["jobs"]:
-        out.append(f"| {kinds.get(j['kind'], j['kind'])} | {j['layer'] if j['kind'] == 0 else ''} "
+        name = kinds.get(j["kind"], j["kind"])
+        if (j["kind"] == 0 and j["layer"] in deferred) or (j["kind"] == 1 and has_head):
+            name += " (finite check; update deferred)"
+        out.append(f"| {name} | {j['layer'] if j['kind'] in (0, 5) else ''} "
                    f"| {j['ready_ms']:.2f} | {j['done_ms']:.2f} |")
     with open(path, "w") as f:
         f.write("\n".join(out) + "\n")
+
+
+def defer_layers(sh):
+    """Deferred layers as the library reads them (MT_DEFER_LAYERS, default 1)."""
+    try:
+        n = int(os.environ.get("MT_DEFER_LAYERS", "1"))
+    except ValueError:
+        n = 1
+    return min(max(n, 0), sh["L"] - 1)
+
+
+def layer_params(sh):
+    hd = sh["d"] // sh["H"]
+    return sh["d"] * (sh["H"] + 2 * sh["Hkv"]) * hd + sh["d"] * sh["H"] * hd + 3 * sh["d"] * sh["F"] + 2 * sh["d"]
+
+
+def head_params(sh):
+    return sh["d"] + sh["V"] * sh["d"]
 
 
 def phase_flops(sh):
@@ -386,7 +412,10 @@ def main():
     # Gradients stream through a ring of host slots (14 instead of 18 B/param of
     # host memory): the 14B workload then fits a ~200 GB host, and so do eight
     # 1.3B replicas.
-    cfg.flags = mt.MT_FLAG_KERNEL_TIMING | (mt.MT_FLAG_GRAD_RING if args.grads == "ring" else 0)
+    # The LM head's and the last layer's updates overlap the next forward sweep
+    # (MT_FLAG_DEFER_UPDATES), when the host optimizer is otherwise idle.
+    cfg.flags = (mt.MT_FLAG_KERNEL_TIMING | (mt.MT_FLAG_GRAD_RING if args.grads == "ring" else 0) |
+                 (0 if args.no_defer else mt.MT_FLAG_DEFER_UPDATES))
     ncpu = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cfg.host_threads = args.host_threads or max(1, ncpu // world)
 
@@ -417,6 +446,9 @@ def main():
             tt = torch.from_numpy(t).pin_memory()
             ll = torch.from_numpy(l).pin_memory()
             toks.append((tt, ll))
+        # distinct token ids of a timed step: the embedding rows that get a gradient
+        n_uniq = sum(int(torch.unique(toks[i][0]).numel())
+                     for i in range(args.warmup, args.warmup + args.steps)) / args.steps
         for i in range(args.warmup):
             mt.mt_train_step(ctx, toks[i][0].data_ptr(), toks[i][1].data_ptr())
         stream = torch.cuda.ExternalStream(mt.mt_get_stream(ctx), device=dev)
@@ -434,6 +466,9 @@ def main():
         for i in range(args.warmup, args.warmup + args.steps):
             losses.append(mt.mt_train_step(ctx, toks[i][0].data_ptr(), toks[i][1].data_ptr()))
             stats.append(mt.mt_get_stats(ctx))
+        # the last step's deferred updates run inside the timed region (the
+        # first timed step already ran the last warm-up step's)
+        mt.mt_flush(ctx)
         e1.record(stream)
         torch.cuda.synchronize(dev)
         barrier()
@@ -446,6 +481,7 @@ def main():
         w0 = time.perf_counter()
         for i in range(args.warmup + args.steps, nsteps):
             losses.append(mt.mt_train_step(ctx, toks[i][0].data_ptr(), toks[i][1].data_ptr()))
+        mt.mt_flush(ctx)
         w1 = time.perf_counter()
         barrier()
         t_e2e = allmax(w1 - w0)
@@ -472,17 +508,27 @@ def main():
         t_compute = exec_f / (peak * 1e12)
         t_h2d = h2d_b / (link["h2d_gbs"] * 1e9)
         t_d2h = d2h_b / (link["d2h_gbs"] * 1e9)
-        # Phase bound of this method's dependency structure: the forward sweep
-        # and head (GPU compute or weight H2D, whichever is slower) must finish
-        # before any gradient exists; then the backward (GPU compute, D2H over
-        # the link) runs alongside the host optimizer, whose bytes move at most
-        # at the rate the same AdamW routine reaches alone on this host (the
-        # DMA engines' traffic is bounded by the link terms instead).
+        # Phase bound of this method's dependency structure. The forward sweep
+        # and head must finish before any gradient of the step exists; then the
+        # backward runs alongside the host optimizer. Each phase takes at least
+        # the longest of its GPU compute, its copies over the host link, and
+        # the host DRAM traffic it needs at the rate the library's AdamW
+        # reaches alone on this host: the optimizer's bytes plus the copies'
+        # (pinned host memory is read by every H2D and written by every D2H).
+        # The forward phase's optimizer bytes are the untouched embedding rows
+        # and, when deferred, the previous step's LM-head and last-layer
+        # updates; the backward phase has the rest.
         f_fl, b_fl = phase_flops(sh)
         L = sh["L"]
-        t_fwd_b = max(f_fl / (peak * 1e12), h2d_b * L / (2 * L - 1) / (link["h2d_gbs"] * 1e9))
+        h2d_fwd = h2d_b * L / (2 * L - 1)
         host_bytes = mean("adamw_bytes")
-        t_host_b = host_bytes / (host_bw * 1e9)
+        upd_fwd = 30.0 * (sh["V"] - n_uniq) * sh["d"]
+        if not args.no_defer:
+            upd_fwd += 30.0 * (head_params(sh) + defer_layers(sh) * layer_params(sh))
+        dram_fwd = upd_fwd + h2d_fwd
+        dram_bwd = host_bytes - upd_fwd + (h2d_b - h2d_fwd) + d2h_b
+        t_fwd_b = max(f_fl / (peak * 1e12), h2d_fwd / (link["h2d_gbs"] * 1e9), dram_fwd / (host_bw * 1e9))
+        t_host_b = dram_bwd / (host_bw * 1e9)
         t_bwd_b = max(b_fl / (peak * 1e12), t_d2h, t_host_b)
         t_bound = t_fwd_b + t_bwd_b
         line = {
@@ -492,6 +538,9 @@ def main():
             "config": {"workload": workload_desc(args.workload, sh), "global_batch": sh["b"] * world,
                        "seq_len": sh["s"], "parallelism": "replicas" if world > 1 else "single GPU",
                        "l2": "no flush needed: every step streams all weights (>1 GB) through HBM from host",
+                       "deferred_updates": (None if args.no_defer else
+                                            f"LM head + last {defer_layers(sh)} layer(s) updated during the next "
+                                            "forward sweep; the timed region ends after mt_flush"),
                        "grads": (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
                                  if args.grads == "ring" else "full fp32 gradient arena in pinned host memory")},
             "model_tflops": model_f * world / (t_dev / K) / 1e12,
@@ -508,6 +557,7 @@ def main():
                               "compute_link_frac": max(t_compute, t_h2d, t_d2h) / (t_dev / K),
                               "fwd_bound_ms": t_fwd_b * 1e3, "bwd_bound_ms": t_bwd_b * 1e3,
                               "host_bytes": host_bytes, "host_bound_ms": t_host_b * 1e3,
+                              "host_dram_bytes_fwd": dram_fwd, "host_dram_bytes_bwd": dram_bwd,
                               "host_optimizer_gbs_measured": host_bw,
                               "compute_ms": t_compute * 1e3, "h2d_ms": t_h2d * 1e3, "d2h_ms": t_d2h * 1e3,
                               "link_measured": link, "h2d_bytes": h2d_b, "d2h_bytes": d2h_b,

@@ -25,6 +25,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <chrono>
 #include <condition_variable>
@@ -67,11 +68,15 @@ inline float normal_at(uint64_t key, uint64_t i) {
 }
 
 struct Job {
-  enum Kind { LAYER, HEAD, EMBED, EMBED_UNTOUCHED } kind;
+  // HEAD_PREV / LAYER_PREV: an update deferred from the previous step
+  // (MT_FLAG_DEFER_UPDATES), its gradients already checked.
+  enum Kind { LAYER, HEAD, EMBED, EMBED_UNTOUCHED, HEAD_PREV, LAYER_PREV } kind;
   int layer;
   cudaEvent_t ready;         // offload of this job's gradients has completed
   int flag_index;            // index in the finite-flag array
   const float* g = nullptr;  // LAYER: host gradient of the layer's first element
+  bool defer = false;        // HEAD / LAYER: check now, update at the next step
+  int step = 0;              // *_PREV: the AdamW step (bias correction) of the update
 };
 
 }  // namespace
@@ -143,6 +148,16 @@ struct mt_ctx {
   std::deque<Job> jobs;
   int jobs_pending = 0;
   int layer_jobs_done = 0;  // LAYER jobs finished this step: ring slots released
+  // MT_FLAG_DEFER_UPDATES: checked updates waiting for the next step, which
+  // queued ones have not finished (index l for layer l, L for the LM head),
+  // the deferred layer count, the pinned gradient buffers of the deferred
+  // layers (ring mode) and the threads of the updates that overlap the
+  // forward sweep.
+  std::vector<Job> deferred;
+  std::vector<char> prev_pending;
+  int defer_layers = 0;
+  float* defer_g = nullptr;
+  int overlap_threads = 0;
   struct JobTime {
     int kind, layer;
     double ready, done;  // host seconds: gradients landed (wait ended), update finished
@@ -429,7 +444,9 @@ struct Seg {
   const float* g;      // gradient of element 0; nullptr: zero gradient
 };
 
-void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
+// AdamW step t over the segments. threads > 0 caps the threads that work on
+// it (the others of the pool stay idle).
+void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs, int t, int threads = 0) {
   // 64K-element pieces handed out dynamically: a worker slowed by other
   // activity on its core (the enqueueing thread, DMA) does not hold the job up.
   const AdamHyper h{c->cfg.lr, c->cfg.beta1, c->cfg.beta2, c->cfg.adam_eps, c->cfg.wd};
@@ -447,13 +464,20 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs) {
     total += sg.n;
   }
   if (tasks.empty()) return;
-  const int t = c->step;
   const double t0 = now_s();
   if (c->adamw_first == 0) c->adamw_first = t0;
-  c->pool->run((int)tasks.size(), [&](int i) {
+  auto one = [&](size_t i) {
     const Task& k = tasks[i];
     adamw_chunk(c->arena + k.off, k.g, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
-  });
+  };
+  if (threads <= 0 || threads >= c->pool->size()) {
+    c->pool->run((int)tasks.size(), [&](int i) { one((size_t)i); });
+  } else {
+    std::atomic<size_t> next{0};
+    c->pool->run(threads, [&](int) {
+      for (size_t i = next.fetch_add(1); i < tasks.size(); i = next.fetch_add(1)) one(i);
+    });
+  }
   c->adamw_last = now_s();
   c->adamw_s += c->adamw_last - t0;
   c->adamw_bytes += 30.0 * total;
@@ -473,9 +497,35 @@ void run_job(mt_ctx* c, const Job& j) {
   c->job_times.push_back({(int)j.kind, j.layer, t0, now_s()});
 }
 
+// AdamW segments of decoder layer l (gradient block g) or, for l < 0, of the
+// final norm and LM head (gradients in grad_head).
+std::vector<Seg> layer_or_head_segs(mt_ctx* c, int l, const float* g) {
+  const Layout& y = c->lay;
+  std::vector<Seg> segs;
+  if (l >= 0) {
+    uint16_t* blk = c->bf_layers + (size_t)l * y.bf_layer;
+    for (int tid = 0; tid < kLayerTensors; ++tid) {
+      const TRef& r = y.t(l, tid);
+      segs.push_back({r.off, r.n, blk + y.bf_of(tid), g + (r.off - y.layer_begin(l))});
+    }
+  } else {
+    segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head, c->grad_head});
+    segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(y.sh.d, 128),
+                    c->grad_head + (y.head.off - y.final_norm.off)});
+  }
+  return segs;
+}
+
 void run_job_body(mt_ctx* c, const Job& j) {
   const Layout& y = c->lay;
   const Shapes& s = y.sh;
+  if (j.kind == Job::HEAD_PREV || j.kind == Job::LAYER_PREV) {
+    // Checked in its own step; it belongs to that step's update, so this
+    // step's skip state does not apply to it.
+    adamw_segments(c, layer_or_head_segs(c, j.kind == Job::HEAD_PREV ? -1 : j.layer, j.g), j.step,
+                   c->overlap_threads);
+    return;
+  }
   if (j.kind == Job::EMBED_UNTOUCHED) {
     // Rows no token of this batch touches have a zero gradient, so their update
     // does not depend on this step's backward and runs while the GPU is in the
@@ -494,6 +544,7 @@ void run_job_body(mt_ctx* c, const Job& j) {
     }
     c->prev_uniq = c->uniq;
     if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
+    const int threads = (c->cfg.flags & MT_FLAG_DEFER_UPDATES) ? c->overlap_threads : 0;
     std::vector<Seg> segs;
     int32_t next = 0;  // first row of the current untouched run
     for (size_t u = 0; u <= c->uniq.size(); ++u) {
@@ -503,7 +554,7 @@ void run_job_body(mt_ctx* c, const Job& j) {
             {y.embed.off + (size_t)next * d, (size_t)(stop - next) * d, c->bf_embed + (size_t)next * d, nullptr});
       next = stop + 1;
     }
-    adamw_segments(c, segs);
+    adamw_segments(c, segs, c->step, threads);
     return;
   }
   if (j.kind == Job::EMBED) {
@@ -537,23 +588,26 @@ void run_job_body(mt_ctx* c, const Job& j) {
     c->skip_updates = true;
   }
   if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
+  if (j.defer) {
+    // Gradients are finite: the update runs at the start of the next step.
+    Job p = j;
+    p.kind = j.kind == Job::HEAD ? Job::HEAD_PREV : Job::LAYER_PREV;
+    p.ready = nullptr;
+    p.defer = false;
+    p.step = c->step;
+    c->deferred.push_back(p);
+    return;
+  }
   std::vector<Seg> segs;
-  if (j.kind == Job::LAYER) {
-    uint16_t* blk = c->bf_layers + (size_t)j.layer * y.bf_layer;
-    for (int tid = 0; tid < kLayerTensors; ++tid) {
-      const TRef& r = y.t(j.layer, tid);
-      segs.push_back({r.off, r.n, blk + y.bf_of(tid), j.g + (r.off - y.layer_begin(j.layer))});
-    }
-  } else if (j.kind == Job::HEAD) {
-    segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head, c->grad_head});
-    segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(s.d, 128), c->grad_head + (y.head.off - y.final_norm.off)});
+  if (j.kind == Job::LAYER || j.kind == Job::HEAD) {
+    segs = layer_or_head_segs(c, j.kind == Job::HEAD ? -1 : j.layer, j.g);
   } else {
     for (size_t u = 0; u < c->uniq.size(); ++u) {
       const size_t r = (size_t)c->uniq[u];
       segs.push_back({y.embed.off + r * s.d, (size_t)s.d, c->bf_embed + r * s.d, c->emb_rows_h + u * s.d});
     }
   }
-  adamw_segments(c, segs);
+  adamw_segments(c, segs, c->step);
 }
 
 void opt_loop(mt_ctx* c) {
@@ -571,6 +625,8 @@ void opt_loop(mt_ctx* c) {
       std::lock_guard<std::mutex> lk(c->opt_mu);
       --c->jobs_pending;
       if (j.kind == Job::LAYER) ++c->layer_jobs_done;
+      if (j.kind == Job::HEAD_PREV) c->prev_pending[c->lay.sh.L] = 0;
+      if (j.kind == Job::LAYER_PREV) c->prev_pending[j.layer] = 0;
     }
     c->opt_done_cv.notify_all();
   }
@@ -590,12 +646,52 @@ void wait_jobs(mt_ctx* c) {
   c->opt_done_cv.wait(lk, [&] { return c->jobs_pending == 0; });
 }
 
+// Queues the updates deferred by the last step in the order the forward sweep
+// streams their weights again (layers ascending, then the LM head); they touch
+// disjoint tensors, so any order gives the same result. Called between steps,
+// when the optimizer is idle.
+void queue_deferred(mt_ctx* c) {
+  if (c->deferred.empty()) return;
+  std::sort(c->deferred.begin(), c->deferred.end(), [](const Job& a, const Job& b) {
+    const int ka = a.kind == Job::HEAD_PREV ? INT32_MAX : a.layer, kb = b.kind == Job::HEAD_PREV ? INT32_MAX : b.layer;
+    return ka < kb;
+  });
+  {
+    std::lock_guard<std::mutex> lk(c->opt_mu);
+    for (const Job& j : c->deferred) {
+      c->jobs.push_back(j);
+      c->prev_pending[j.kind == Job::HEAD_PREV ? c->lay.sh.L : j.layer] = 1;
+    }
+    c->jobs_pending += (int)c->deferred.size();
+  }
+  c->deferred.clear();
+  c->opt_cv.notify_one();
+}
+
+// Applies pending deferred updates before the state is read or replaced.
+void flush_deferred(mt_ctx* c) {
+  if (c->deferred.empty()) return;
+  queue_deferred(c);
+  wait_jobs(c);
+}
+
+// Bounded host wait for the deferred update of layer l (l = L: the LM head)
+// queued at the start of this step: its weights are about to be streamed again.
+int await_deferred(mt_ctx* c, int l) {
+  std::unique_lock<std::mutex> lk(c->opt_mu);
+  if (!c->opt_done_cv.wait_for(lk, std::chrono::duration<double>(c->wait_limit_s),
+                               [&] { return c->prev_pending[l] == 0; }))
+    return set_err(c, MT_ERR_TIMEOUT, "a deferred update did not finish within the wait limit");
+  return MT_OK;
+}
+
 // ---------------------------------------------------------------------------
 // Step.
 // ---------------------------------------------------------------------------
 int issue_load(mt_ctx* c, int i) {
   const Layout& y = c->lay;
   const int slot = i & 1;
+  if (i < y.sh.L && i >= y.sh.L - c->defer_layers) CKM(await_deferred(c, i));  // forward load of a deferred layer
   if (i >= 2) CK(cudaStreamWaitEvent(c->s_h2d, c->ev_slotfree[i - 2], 0));
   CK(cudaEventRecord(c->ev_h2d_start[i], c->s_h2d));
   CK(cudaMemcpyAsync(c->wslot[slot], c->bf_layers + (size_t)c->load_seq[i] * y.bf_layer, y.bf_layer * 2,
@@ -606,6 +702,7 @@ int issue_load(mt_ctx* c, int i) {
 
 int issue_head_load(mt_ctx* c) {
   const size_t n = align_up(c->lay.sh.d, 128) + (size_t)c->lay.sh.V * c->lay.sh.d;
+  CKM(await_deferred(c, c->lay.sh.L));
   CK(cudaEventRecord(c->ev_head_h2d_start, c->s_h2d));
   CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, n * 2, cudaMemcpyHostToDevice, c->s_h2d));
   CK(cudaEventRecord(c->ev_head_wready, c->s_h2d));
@@ -613,13 +710,19 @@ int issue_head_load(mt_ctx* c) {
 }
 
 // Backward index k (layer l = L-1-k): D2H of the layer's gradients into the
-// gradient arena, or into ring slot k mod MT_GRAD_RING_SLOTS once the update
-// of backward index k - MT_GRAD_RING_SLOTS (the slot's previous user) is done.
+// gradient arena or, in ring mode, into deferred-layer buffer k for the first
+// defer_layers indices (their update runs at the next step), else into ring
+// slot (k - defer_layers) mod MT_GRAD_RING_SLOTS once the update of backward
+// index k - MT_GRAD_RING_SLOTS (the slot's previous user) is done: the layer
+// jobs finish in backward order, so that is when layer_jobs_done passes it.
 int offload_layer(mt_ctx* c, int l, int k) {
   const Layout& y = c->lay;
   const size_t b = y.layer_begin(l), e = y.layer_end(l);
-  float* dst = c->grad ? c->grad + b : c->ring + (size_t)(k % MT_GRAD_RING_SLOTS) * c->layer_f;
-  if (!c->grad && k >= MT_GRAD_RING_SLOTS) {
+  const int nd = c->defer_layers;
+  float* dst = c->grad ? c->grad + b
+               : k < nd ? c->defer_g + (size_t)k * c->layer_f
+                        : c->ring + (size_t)((k - nd) % MT_GRAD_RING_SLOTS) * c->layer_f;
+  if (!c->grad && k >= nd + MT_GRAD_RING_SLOTS) {
     std::unique_lock<std::mutex> lk(c->opt_mu);
     const int need = k - MT_GRAD_RING_SLOTS + 1;
     if (!c->opt_done_cv.wait_for(lk, std::chrono::duration<double>(c->wait_limit_s),
@@ -632,7 +735,9 @@ int offload_layer(mt_ctx* c, int l, int k) {
   CK(cudaMemcpyAsync(dst, c->gslot[k & 1], (e - b) * 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaMemcpyAsync(c->flags_h + l, c->d_flags + l, 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaEventRecord(c->ev_gdrained[k], c->s_d2h));
-  push_job(c, Job{Job::LAYER, l, c->ev_gdrained[k], l, dst});
+  Job j{Job::LAYER, l, c->ev_gdrained[k], l, dst};
+  j.defer = k < nd;
+  push_job(c, j);
   return MT_OK;
 }
 
@@ -670,7 +775,9 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         CK(cudaMemcpyAsync(c->grad_head, c->d_head_g, n * 4, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaMemcpyAsync(c->flags_h + L, c->d_flags + L, 4, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaEventRecord(c->ev_head_drained, c->s_d2h));
-        push_job(c, Job{Job::HEAD, -1, c->ev_head_drained, L});
+        Job hj{Job::HEAD, -1, c->ev_head_drained, L};
+        hj.defer = (c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !(c->cfg.flags & MT_FLAG_NO_UPDATE);
+        push_job(c, hj);
         CK(cudaEventRecord(c->ev_head_end, sc));
         // backward of the last layer: its intermediates are still in the workspace
         CKM(layer_bwd(c, l, slot, c->gslot[0], gin, gout));
@@ -687,8 +794,12 @@ int enqueue_step(mt_ctx* c, int n_unique) {
       std::swap(gin, gout);
     }
     CK(cudaEventRecord(c->ev_slotfree[i], sc));
+    // The head's weights follow the last forward load on the H2D stream, ahead
+    // of the first backward load. Issued here, after layer L-2's forward is
+    // queued, a wait for its deferred update holds back no forward layer but
+    // the last one.
+    if (i + 2 == L) CKM(issue_head_load(c));
     if (i + 2 < nloads) CKM(issue_load(c, i + 2));
-    if (i + 2 == L - 1 || (i == 0 && L == 2)) CKM(issue_head_load(c));
   }
   CK(cudaEventRecord(c->ev_bwd_end, sc));
   // embedding gradient rows, in token order per unique id
@@ -843,7 +954,8 @@ void free_all(mt_ctx* c) {
   if (c->s_h2d && c->s_h2d != c->s_comp) cudaStreamDestroy(c->s_h2d);
   if (c->s_d2h && c->s_d2h != c->s_comp && c->s_d2h != c->s_h2d) cudaStreamDestroy(c->s_d2h);
   if (c->dmem) cudaFree(c->dmem);
-  for (void* p : {(void*)c->grad, (void*)c->ring, (void*)(c->grad ? nullptr : c->grad_head), (void*)c->bf_layers,
+  for (void* p : {(void*)c->grad, (void*)c->ring, (void*)c->defer_g, (void*)(c->grad ? nullptr : c->grad_head),
+                  (void*)c->bf_layers,
                   (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h, (void*)c->stage_i, (void*)c->flags_h,
                   (void*)c->misc_h})
     if (p) cudaFreeHost(p);
@@ -921,11 +1033,22 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->layer_f = y.layer_end(0) - y.layer_begin(0);
   for (int l = 1; l < s.L; ++l)
     if (y.layer_end(l) - y.layer_begin(l) != c->layer_f) return fail(MT_ERR_CONFIG, "layer blocks differ in size");
+  c->defer_layers = defer_layer_count(*cfg);
+  c->prev_pending.assign((size_t)s.L + 1, 0);
+  c->overlap_threads = std::max(1, c->pool->size() / 2);
+  if (const char* e = getenv("MT_OVERLAP_THREADS")) {
+    const int n = atoi(e);
+    if (n > 0) c->overlap_threads = std::min(n, c->pool->size());
+  }
   if (cfg->flags & MT_FLAG_GRAD_RING) {
     if (cudaHostAlloc(reinterpret_cast<void**>(&c->ring), (size_t)MT_GRAD_RING_SLOTS * c->layer_f * 4,
                       cudaHostAllocPortable) != cudaSuccess ||
         cudaHostAlloc(reinterpret_cast<void**>(&c->grad_head), head_f * 4, cudaHostAllocPortable) != cudaSuccess)
       return fail(MT_ERR_PIN, "pinned gradient ring allocation failed");
+    if (c->defer_layers > 0 && cudaHostAlloc(reinterpret_cast<void**>(&c->defer_g),
+                                             (size_t)c->defer_layers * c->layer_f * 4,
+                                             cudaHostAllocPortable) != cudaSuccess)
+      return fail(MT_ERR_PIN, "pinned deferred-layer gradient allocation failed");
   } else {
     if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * 4, cudaHostAllocPortable) != cudaSuccess)
       return fail(MT_ERR_PIN, "pinned gradient arena allocation failed");
@@ -969,6 +1092,9 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   if (c->ring) {
     const size_t nr = (size_t)MT_GRAD_RING_SLOTS * c->layer_f;
     parallel_ranges(*c->pool, nr, [&](size_t b, size_t e) { memset(c->ring + b, 0, (e - b) * 4); });
+    if (c->defer_g)
+      parallel_ranges(*c->pool, (size_t)c->defer_layers * c->layer_f,
+                      [&](size_t b, size_t e) { memset(c->defer_g + b, 0, (e - b) * 4); });
     parallel_ranges(*c->pool, head_f, [&](size_t b, size_t e) { memset(c->grad_head + b, 0, (e - b) * 4); });
   }
   // bf16 streaming copies
@@ -1154,6 +1280,7 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
     c->layer_jobs_done = 0;
   }
   c->job_times.clear();
+  queue_deferred(c);  // the last step's deferred updates overlap this forward sweep
   push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, s.L + 1});
   const double te0 = now_s();
   int r = enqueue_step(c, n_unique);
@@ -1194,6 +1321,7 @@ extern "C" int mt_layer_fwd_bwd(mt_ctx* c, int l, const float* x_in, const float
   const Shapes& s = y.sh;
   if (l < 0 || l >= s.L) return set_err(c, MT_ERR_ARG, "layer outside [0, L)");
   if (grads_bytes < c->layer_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than one layer's block");
+  flush_deferred(c);
   CK(cudaSetDevice(c->device));
   const size_t n = (size_t)s.T * s.d;
   cudaStream_t sc = c->s_comp;
@@ -1227,6 +1355,7 @@ extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* label
   if (grads_bytes < head_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than the final-norm + head block");
   for (int t = 0; t < s.T; ++t)
     if (labels[t] < 0 || labels[t] >= s.V) return set_err(c, MT_ERR_ARG, "label outside [0, V)");
+  flush_deferred(c);
   CK(cudaSetDevice(c->device));
   const size_t n = (size_t)s.T * s.d;
   cudaStream_t sc = c->s_comp;
@@ -1261,6 +1390,7 @@ extern "C" int mt_get_grads(mt_ctx* c, float* dst, size_t bytes) {
 extern "C" int mt_get_params(mt_ctx* c, float* dst, size_t bytes) {
   if (!c || !dst) return MT_ERR_ARG;
   if (bytes < c->lay.total * 4) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
+  flush_deferred(c);
   memcpy(dst, c->arena, c->lay.total * 4);
   return MT_OK;
 }
@@ -1269,6 +1399,7 @@ extern "C" int mt_get_opt_state(mt_ctx* c, float* m_dst, float* v_dst, size_t by
   if (!c) return MT_ERR_ARG;
   const size_t need = c->lay.total * 4;
   if ((m_dst || v_dst) && bytes_each < need) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
+  flush_deferred(c);
   if (m_dst) memcpy(m_dst, c->m, need);
   if (v_dst) memcpy(v_dst, c->v, need);
   if (step) *step = c->step;
@@ -1283,6 +1414,7 @@ extern "C" int mt_set_state(mt_ctx* c, const float* params, const float* m, cons
   const size_t need = y.total * 4;
   if ((params || m || v) && bytes_each < need) return set_err(c, MT_ERR_ARG, "source smaller than the arena");
   if (step < 0 || step > (int64_t)1 << 30) return set_err(c, MT_ERR_ARG, "step out of range");
+  flush_deferred(c);  // the pending updates belong to the state being replaced
   if (m) memcpy(c->m, m, need);
   if (v) memcpy(c->v, v, need);
   c->step = (int)step;
@@ -1362,6 +1494,15 @@ extern "C" int mt_get_stream(mt_ctx* c, void** stream) {
   return MT_OK;
 }
 
-extern "C" void mt_destroy(mt_ctx* c) { free_all(c); }
+extern "C" int mt_flush(mt_ctx* c) {
+  if (!c) return MT_ERR_ARG;
+  flush_deferred(c);
+  return MT_OK;
+}
+
+extern "C" void mt_destroy(mt_ctx* c) {
+  if (c) flush_deferred(c);
+  free_all(c);
+}
 
 extern "C" const char* mt_last_error(const mt_ctx* c) { return c ? c->err.c_str() : g_create_error.c_str(); }

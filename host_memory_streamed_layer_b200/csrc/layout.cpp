@@ -1,7 +1,10 @@
 // Configuration checks and the arena / layer-block layouts (see layout.h).
 #include "layout.h"
 
+#include <stdlib.h>
 #include <string.h>
+
+#include <algorithm>
 
 namespace mt {
 
@@ -149,6 +152,13 @@ extern "C" int mt_tensor_offset(const mt_config* cfg, int layer, int tid, size_t
   return MT_OK;
 }
 
+int mt::defer_layer_count(const mt_config& cfg) {
+  if (!(cfg.flags & MT_FLAG_DEFER_UPDATES) || (cfg.flags & MT_FLAG_NO_UPDATE)) return 0;
+  long n = 1;
+  if (const char* e = getenv("MT_DEFER_LAYERS")) n = strtol(e, nullptr, 10);
+  return (int)std::min<long>(std::max<long>(n, 0), std::max(cfg.L - 1, 0));
+}
+
 extern "C" size_t mt_host_state_bytes(const mt_config* cfg) {
   if (mt::validate_config(cfg, nullptr) != MT_OK) return 0;
   mt::Layout y = mt::make_layout(*cfg);
@@ -158,5 +168,5 @@ extern "C" size_t mt_host_state_bytes(const mt_config* cfg) {
   if (!(cfg->flags & MT_FLAG_GRAD_RING)) return common + P * 4;          // whole gradient arena
   const size_t layer_f = y.layer_end(0) - y.layer_begin(0);
   const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
-  return common + ((size_t)MT_GRAD_RING_SLOTS * layer_f + head_f) * 4;
+  return common + ((size_t)(MT_GRAD_RING_SLOTS + mt::defer_layer_count(*cfg)) * layer_f + head_f) * 4;
 }

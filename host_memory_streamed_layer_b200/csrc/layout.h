@@ -55,4 +55,9 @@ struct Layout {
 int validate_config(const mt_config* cfg, std::string* why);
 Layout make_layout(const mt_config& cfg);
 
+// Layers whose update MT_FLAG_DEFER_UPDATES defers to the next step: 0 without
+// the flag or with MT_FLAG_NO_UPDATE, else MT_DEFER_LAYERS (default 1) clamped
+// to [0, L-1].
+int defer_layer_count(const mt_config& cfg);
+
 }  // namespace mt

@@ -172,6 +172,7 @@ def mt_k_gemm_bf16_rope(A, lda, B, ldb, C, ldc, M, N, K, rope_cols, hd, s, cos_t
 # Engine API (include/mt.h)
 # ---------------------------------------------------------------------------
 MT_FLAG_SERIALIZE, MT_FLAG_KERNEL_TIMING, MT_FLAG_NO_UPDATE, MT_FLAG_GRAD_RING = 0x1, 0x2, 0x4, 0x8
+MT_FLAG_DEFER_UPDATES = 0x10
 MT_GRAD_RING_SLOTS = 3
 MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
 MT_T_EMBED, MT_T_FINAL_NORM, MT_T_LM_HEAD = 100, 101, 102
@@ -206,6 +207,7 @@ _sig("mt_tensor_offset", c_int, _cfgp, c_int, c_int, ctypes.POINTER(c_size_t), c
 _sig("mt_host_state_bytes", c_size_t, _cfgp)
 _sig("mt_create", c_int, _cfgp, c_void_p, c_size_t, ctypes.POINTER(c_void_p))
 _sig("mt_train_step", c_int, c_void_p, c_void_p, c_void_p, ctypes.POINTER(ctypes.c_float))
+_sig("mt_flush", c_int, c_void_p)
 _sig("mt_get_grads", c_int, c_void_p, c_void_p, c_size_t)
 _sig("mt_get_timeline", c_int, c_void_p, c_void_p, c_size_t, ctypes.POINTER(c_size_t))
 _sig("mt_head_fwd_bwd", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t)
@@ -260,6 +262,10 @@ def mt_train_step(ctx: int, tokens_ptr: int, labels_ptr: int) -> float:
     if rc != MT_OK:
         raise MTError(rc, "mt_train_step " + lib.mt_last_error(ctx).decode())
     return loss.value
+
+
+def mt_flush(ctx: int):
+    return _check(lib.mt_flush(ctx), "mt_flush", ctx)
 
 
 def mt_get_grads(ctx: int, dst_ptr: int, nbytes: int):

@@ -27,7 +27,15 @@
  *   MT_LOGITS_CHUNK  tokens per LM-head chunk, a multiple of 128 below the
  *                    default (the default keeps fp32 logits + bf16 dz of a
  *                    chunk under ~4 GiB); smaller chunks use less device
- *                    memory and compute the same result.
+ *                    memory and compute the same result;
+ *   MT_DEFER_LAYERS  with MT_FLAG_DEFER_UPDATES, how many of the last layers
+ *                    have their update deferred (default 1; clamped to
+ *                    [0, L-1]; mt_host_state_bytes reads it too);
+ *   MT_OVERLAP_THREADS  with MT_FLAG_DEFER_UPDATES, host threads of the
+ *                    updates that overlap the forward sweep (deferred ones and
+ *                    the untouched embedding rows; default half the pool), so
+ *                    that the weight copies keep their share of host memory
+ *                    bandwidth.
  * and by the GEMM launcher: MT_GEMM_VARIANT (see mt_kernels.h).
  */
 #ifndef MT_H_
@@ -64,6 +72,22 @@ extern "C" {
  * limit). mt_get_grads is not available in this mode. */
 #define MT_FLAG_GRAD_RING 0x8u
 #define MT_GRAD_RING_SLOTS 3
+/* Overlap part of each step's host update with the next step's forward sweep,
+ * when the host optimizer is otherwise idle. The updates of the final norm and
+ * LM head and of the last MT_DEFER_LAYERS decoder layers (environment variable,
+ * default 1, at most L-1) are checked for non-finite gradients in their own
+ * step as usual; their AdamW update is then run at the start of the next
+ * mt_train_step, which waits (bounded by the wait limit) for it before
+ * streaming those weights again. Every update still uses its own step's
+ * gradient and bias correction and completes before its weights are next
+ * read, so the trajectory is that of the undeferred step. Until a pending
+ * update has run, the caller's arena holds those tensors' previous values:
+ * mt_flush applies pending updates, and so does every call that reads or
+ * writes the training state (mt_get_params, mt_get_opt_state, mt_set_state,
+ * mt_layer_fwd_bwd, mt_head_fwd_bwd, mt_destroy). With MT_FLAG_GRAD_RING the
+ * deferred layers keep their gradients in MT_DEFER_LAYERS extra pinned
+ * layer-sized buffers. Ignored with MT_FLAG_NO_UPDATE. */
+#define MT_FLAG_DEFER_UPDATES 0x10u
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0
@@ -137,7 +161,8 @@ int mt_tensor_offset(const mt_config* cfg, int layer, int tensor_id, size_t* off
  * moments (8 B/param), the bf16 streaming copy (2 B/param) and the staging of
  * the embedding-gradient rows, plus the fp32 gradients: the whole gradient
  * arena (4 B/param), or with MT_FLAG_GRAD_RING in cfg->flags the ring of
- * MT_GRAD_RING_SLOTS layer slots and the final-norm + LM-head gradient. */
+ * MT_GRAD_RING_SLOTS layer slots and the final-norm + LM-head gradient (and,
+ * with MT_FLAG_DEFER_UPDATES too, MT_DEFER_LAYERS more layer slots). */
 size_t mt_host_state_bytes(const mt_config* cfg);
 
 /* Creates a context on cfg->device. host_param_arena: the caller's fp32
@@ -156,8 +181,15 @@ int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes,
  * update (bias correction from step 1), and writes the mean next-token
  * cross-entropy (computed before the update) to *loss_out. Returns
  * MT_ERR_NONFINITE if a gradient was not finite: the updates of the tensors
- * not yet updated are skipped and the arena is partly updated. */
+ * not yet updated are skipped and the arena is partly updated. With
+ * MT_FLAG_DEFER_UPDATES some of this step's updates are still pending when it
+ * returns (see the flag). */
 int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, float* loss_out);
+
+/* Runs the updates that MT_FLAG_DEFER_UPDATES left pending, and returns when
+ * the arena, the moments and the bf16 copies hold the state after the last
+ * step. A no-op without pending updates. */
+int mt_flush(mt_ctx* ctx);
 
 /* Copies the fp32 gradients of the last step (taken before the update), in the
  * arena layout, to dst (bytes >= mt_arena_bytes). MT_ERR_CONFIG for a context
@@ -222,8 +254,11 @@ int mt_get_stats(mt_ctx* ctx, mt_stats* out);
  *     compute stream, D2H start, D2H done;
  *   forward end, head end, backward end, step end;
  *   per host optimizer job (execution order): kind (0 layer, 1 LM head,
- *     2 touched embedding rows, 3 untouched embedding rows), layer (-1 for
- *     the others), gradients available, update finished.
+ *     2 touched embedding rows, 3 untouched embedding rows, 4 LM head and
+ *     5 layer deferred from the previous step by MT_FLAG_DEFER_UPDATES; with
+ *     the flag, kinds 0 and 1 of the deferred tensors only check their
+ *     gradients), layer (-1 for the others), gradients available, update
+ *     finished.
  * Device times are ms from the step's start on the compute stream (CUDA
  * events); host job times are ms of host clock from the mt_train_step call,
  * a separate clock whose origin is within a few tens of microseconds of it. */
@@ -243,8 +278,8 @@ int mt_get_stream(mt_ctx* ctx, void** stream);
  * buffers; no GPU needed. Returns a negative MT_ERR_* on failure. */
 double mt_host_optimizer_gbs(size_t n, int threads);
 
-/* Waits for the context's streams, frees its device memory and unpins or
- * frees its host memory. NULL is ignored. */
+/* Applies pending deferred updates, waits for the context's streams, frees
+ * its device memory and unpins or frees its host memory. NULL is ignored. */
 void mt_destroy(mt_ctx* ctx);
 
 /* Message of the last error of ctx (or of the last failed mt_create when ctx

@@ -89,6 +89,32 @@ def test_host_state_with_gradient_ring(name):
     assert ring + 4 * P <= (15.0 if P < 5e9 else 14.6) * P
 
 
+def test_host_state_with_deferred_updates(monkeypatch):
+    """MT_FLAG_DEFER_UPDATES with the ring adds one layer-sized gradient buffer
+    per deferred layer (MT_DEFER_LAYERS, default 1, clamped to [0, L-1]); the
+    full gradient arena already holds every layer's gradient, and with
+    MT_FLAG_NO_UPDATE nothing is deferred."""
+    mt = _mt()
+    shape = dict(L=4, d=256, H=4, Hkv=4, F=688, V=1024, b=2, s=128)
+    cfg = mt.mt_config_default(**shape)
+    full = mt.mt_host_state_bytes(cfg)
+    cfg.flags = mt.MT_FLAG_GRAD_RING
+    ring = mt.mt_host_state_bytes(cfg)
+    first = [mt.mt_tensor_offset(cfg, layer, mt.MT_T_ATTN_NORM)[0] for layer in (0, 1)]
+    layer_bytes = 4 * (first[1] - first[0])
+    cfg.flags = mt.MT_FLAG_GRAD_RING | mt.MT_FLAG_DEFER_UPDATES
+    monkeypatch.delenv("MT_DEFER_LAYERS", raising=False)
+    assert mt.mt_host_state_bytes(cfg) == ring + layer_bytes
+    for env, nd in (("0", 0), ("2", 2), ("99", shape["L"] - 1), ("-3", 0)):
+        monkeypatch.setenv("MT_DEFER_LAYERS", env)
+        assert mt.mt_host_state_bytes(cfg) == ring + nd * layer_bytes, env
+    monkeypatch.setenv("MT_DEFER_LAYERS", "2")
+    cfg.flags = mt.MT_FLAG_GRAD_RING | mt.MT_FLAG_DEFER_UPDATES | mt.MT_FLAG_NO_UPDATE
+    assert mt.mt_host_state_bytes(cfg) == ring
+    cfg.flags = mt.MT_FLAG_DEFER_UPDATES
+    assert mt.mt_host_state_bytes(cfg) == full
+
+
 def test_host_adamw_zero_gradient_reads_nothing():
     """g = NULL is the update of a zero gradient: bit-identical to passing
     zeros, and equal to the oracle's AdamW with g = 0 (decay and moment decay

@@ -335,3 +335,73 @@ def test_head_matches_oracle(monkeypatch):
         assert e.value.code == -1
     finally:
         mt.mt_destroy(ctx)
+
+
+def test_deferred_updates_follow_the_undeferred_trajectory(monkeypatch):
+    """MT_FLAG_DEFER_UPDATES (2 deferred layers of 6, plus the LM head): three
+    steps with no flush between them, so each step's deferred updates run in
+    the next step's forward sweep and the weight loads wait for them. Each
+    step's loss and gradients match the undeferred run's (stale weights in a
+    load would change them), the state after mt_flush is AdamW replayed on the
+    engine's own gradients with each step's bias correction (relative 1e-6),
+    mt_get_params flushes, the deferred jobs appear in the timeline and finish
+    before their layer's forward load starts, and the gradient ring with
+    deferral reaches the same master."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    monkeypatch.setenv("MT_DEFER_LAYERS", "2")
+    shape = dict(L=6, d=256, H=4, Hkv=2, F=688, V=1024, b=2, s=128)
+    L, nd, n_steps = shape["L"], 2, 3
+    toks = [synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, k) for k in range(n_steps)]
+
+    def run(flags, grads):
+        cfg = arena.config(shape)
+        cfg.flags = flags
+        cfg.host_threads = 4
+        A = arena.pack(cfg, synth.init_weights(shape, 0))
+        P0 = A.copy()
+        ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+        losses, Gs = [], []
+        try:
+            for tok, lab in toks:
+                losses.append(mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data))
+                if grads:
+                    G = np.empty_like(A)
+                    mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
+                    Gs.append(G)
+            tl = mt.mt_get_timeline(ctx)
+            P = np.empty_like(A)
+            mt.mt_get_params(ctx, P.ctypes.data, P.nbytes)
+            assert np.array_equal(P, A)  # the pending updates were applied first
+            mt.mt_flush(ctx)  # nothing left: a no-op
+            M, V = np.empty_like(A), np.empty_like(A)
+            assert mt.mt_get_opt_state(ctx, M.ctypes.data, V.ctypes.data, M.nbytes) == n_steps
+        finally:
+            mt.mt_destroy(ctx)
+        return dict(P0=P0, P=P, M=M, V=V, losses=losses, G=Gs, tl=tl)
+
+    base = run(0, True)
+    dfr = run(mt.MT_FLAG_DEFER_UPDATES, True)
+    c = oracle.OracleConfig(**shape)
+    for k in range(n_steps):
+        assert abs(dfr["losses"][k] - base["losses"][k]) <= 1e-5, k
+        Gd, Gb = oracle.unpack_arena(dfr["G"][k], c), oracle.unpack_arena(base["G"][k], c)
+        assert max(rel(Gd[t], Gb[t]) for t in Gb) <= 1e-3, k
+    p, m, v = dfr["P0"].astype(np.float64), 0.0, 0.0
+    for k in range(n_steps):
+        p, m, v = oracle.adamw_update(p, dfr["G"][k], m, v, k + 1, **HYP)
+    for got, want in ((dfr["P"], p), (dfr["M"], m), (dfr["V"], v)):
+        assert rel(got.astype(np.float64), want) <= 1e-6
+    # timeline of the last step: one check job per layer and for the head, the
+    # two embedding jobs, and the previous step's deferred head and layers
+    jobs = dfr["tl"]["jobs"]
+    assert sorted(j["kind"] for j in jobs) == [0] * L + [1, 2, 3, 4] + [5] * nd
+    assert sorted(j["layer"] for j in jobs if j["kind"] == 5) == list(range(L - nd, L))
+    loads = dfr["tl"]["loads"]
+    for j in jobs:
+        if j["kind"] == 5:
+            assert j["done_ms"] <= loads[j["layer"]]["h2d_start"] + 1.0
+    # gradient ring + deferral: 2 deferred buffers, ring waits from backward index 5
+    ring = run(mt.MT_FLAG_DEFER_UPDATES | mt.MT_FLAG_GRAD_RING, False)
+    for a, b in zip(ring["losses"], dfr["losses"]):
+        assert abs(a - b) <= 1e-4
+    assert rel(ring["P"], dfr["P"]) <= 2e-3
