@@ -314,6 +314,43 @@ def write_timeline(tl, path, workload):
         f.write("\n".join(out) + "\n")
 
 
+def step_bounds(sh, *, peak_tflops, link, host_gbs, h2d_bytes, d2h_bytes, update_bytes, n_unique,
+                deferred_layers=None):
+    """Phase bound of this method's dependency structure (seconds).
+
+    The forward sweep and head (GPU compute or weight H2D, whichever is slower)
+    must finish before any gradient of the step exists. The backward (GPU
+    compute, D2H over the link) then runs alongside the host updates that need
+    this step's gradients, whose bytes move at most at host_gbs, the rate the
+    library's AdamW reaches alone on this host. The untouched embedding rows
+    and, with deferral (deferred_layers not None), the previous step's LM-head
+    and last-layer updates run during the forward sweep instead; all of the
+    step's update bytes at host_gbs bound the step as well.
+
+    "model" is not a bound: it adds the copies' host DRAM traffic (pinned memory
+    is read by every H2D and written by every D2H) to the optimizer's at the
+    same rate, and measured steps beat it where DMA and CPU traffic together
+    draw more from host DRAM than the CPU alone."""
+    f_fl, b_fl = phase_flops(sh)
+    L = sh["L"]
+    peak = peak_tflops * 1e12
+    h2d_fwd = h2d_bytes * L / (2 * L - 1)
+    upd_fwd = 30.0 * (sh["V"] - n_unique) * sh["d"]
+    if deferred_layers is not None:
+        upd_fwd += 30.0 * (head_params(sh) + deferred_layers * layer_params(sh))
+    upd_bwd = update_bytes - upd_fwd
+    t_d2h = d2h_bytes / (link["d2h_gbs"] * 1e9)
+    fwd = max(f_fl / peak, h2d_fwd / (link["h2d_gbs"] * 1e9))
+    host_bwd = upd_bwd / (host_gbs * 1e9)
+    bwd = max(b_fl / peak, t_d2h, host_bwd)
+    dram_fwd = upd_fwd + h2d_fwd
+    dram_bwd = upd_bwd + (h2d_bytes - h2d_fwd) + d2h_bytes
+    model = max(fwd, dram_fwd / (host_gbs * 1e9)) + max(b_fl / peak, t_d2h, dram_bwd / (host_gbs * 1e9))
+    return dict(fwd=fwd, bwd=bwd, host_bwd=host_bwd, bound=max(fwd + bwd, update_bytes / (host_gbs * 1e9)),
+                update_bytes=update_bytes, update_bytes_fwd=upd_fwd, update_bytes_bwd=upd_bwd,
+                model=model, dram_fwd=dram_fwd, dram_bwd=dram_bwd)
+
+
 def defer_layers(sh):
     """Deferred layers as the library reads them (MT_DEFER_LAYERS, default 1)."""
     try:
@@ -508,29 +545,12 @@ def main():
         t_compute = exec_f / (peak * 1e12)
         t_h2d = h2d_b / (link["h2d_gbs"] * 1e9)
         t_d2h = d2h_b / (link["d2h_gbs"] * 1e9)
-        # Phase bound of this method's dependency structure. The forward sweep
-        # and head must finish before any gradient of the step exists; then the
-        # backward runs alongside the host optimizer. Each phase takes at least
-        # the longest of its GPU compute, its copies over the host link, and
-        # the host DRAM traffic it needs at the rate the library's AdamW
-        # reaches alone on this host: the optimizer's bytes plus the copies'
-        # (pinned host memory is read by every H2D and written by every D2H).
-        # The forward phase's optimizer bytes are the untouched embedding rows
-        # and, when deferred, the previous step's LM-head and last-layer
-        # updates; the backward phase has the rest.
-        f_fl, b_fl = phase_flops(sh)
-        L = sh["L"]
-        h2d_fwd = h2d_b * L / (2 * L - 1)
-        host_bytes = mean("adamw_bytes")
-        upd_fwd = 30.0 * (sh["V"] - n_uniq) * sh["d"]
-        if not args.no_defer:
-            upd_fwd += 30.0 * (head_params(sh) + defer_layers(sh) * layer_params(sh))
-        dram_fwd = upd_fwd + h2d_fwd
-        dram_bwd = host_bytes - upd_fwd + (h2d_b - h2d_fwd) + d2h_b
-        t_fwd_b = max(f_fl / (peak * 1e12), h2d_fwd / (link["h2d_gbs"] * 1e9), dram_fwd / (host_bw * 1e9))
-        t_host_b = dram_bwd / (host_bw * 1e9)
-        t_bwd_b = max(b_fl / (peak * 1e12), t_d2h, t_host_b)
-        t_bound = t_fwd_b + t_bwd_b
+        sb = step_bounds(sh, peak_tflops=peak, link=link, host_gbs=host_bw, h2d_bytes=h2d_b, d2h_bytes=d2h_b,
+                         update_bytes=mean("adamw_bytes"), n_unique=n_uniq,
+                         deferred_layers=None if args.no_defer else defer_layers(sh))
+        host_bytes, upd_fwd, upd_bwd = sb["update_bytes"], sb["update_bytes_fwd"], sb["update_bytes_bwd"]
+        t_fwd_b, t_bwd_b, t_host_b, t_bound = sb["fwd"], sb["bwd"], sb["host_bwd"], sb["bound"]
+        t_model, dram_fwd, dram_bwd = sb["model"], sb["dram_fwd"], sb["dram_bwd"]
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -557,7 +577,10 @@ def main():
                               "compute_link_frac": max(t_compute, t_h2d, t_d2h) / (t_dev / K),
                               "fwd_bound_ms": t_fwd_b * 1e3, "bwd_bound_ms": t_bwd_b * 1e3,
                               "host_bytes": host_bytes, "host_bound_ms": t_host_b * 1e3,
-                              "host_dram_bytes_fwd": dram_fwd, "host_dram_bytes_bwd": dram_bwd,
+                              "update_bytes_fwd": upd_fwd, "update_bytes_bwd": upd_bwd,
+                              "n_unique_tokens": n_uniq,
+                              "host_dram_model": {"ms": t_model * 1e3, "ratio": t_model / (t_dev / K),
+                                                  "bytes_fwd": dram_fwd, "bytes_bwd": dram_bwd},
                               "host_optimizer_gbs_measured": host_bw,
                               "compute_ms": t_compute * 1e3, "h2d_ms": t_h2d * 1e3, "d2h_ms": t_d2h * 1e3,
                               "link_measured": link, "h2d_bytes": h2d_b, "d2h_bytes": d2h_b,

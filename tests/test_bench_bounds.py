@@ -1,0 +1,63 @@
+"""The bench's phase bound (bench.step_bounds) on made-up rates: which term
+binds in each phase, how deferral moves update bytes into the forward phase,
+that the whole step's update bytes bound it too, and that the DRAM model only
+adds traffic. No GPU: the inputs are plain numbers."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+import synth  # noqa: E402
+
+SH = synth.WORKLOADS["llama-1.3b"]
+LINK = {"h2d_gbs": 50.0, "d2h_gbs": 50.0}
+
+
+def params(sh):
+    L = sh["L"]
+    return L * bench.layer_params(sh) + 2 * bench.head_params(sh) - sh["d"]  # embedding has no final-norm gain
+
+
+def test_parameter_counts_match_the_arena():
+    from host_memory_streamed_layer_b200 import arena, mt
+    cfg = arena.config(SH)
+    first = [mt.mt_tensor_offset(cfg, layer, mt.MT_T_ATTN_NORM)[0] for layer in (0, 1)]
+    n_layer = sum(mt.mt_tensor_offset(cfg, 0, t)[1] for t in range(9))
+    assert bench.layer_params(SH) == n_layer <= first[1] - first[0]
+    fn = mt.mt_tensor_offset(cfg, -1, mt.MT_T_FINAL_NORM)[1]
+    head = mt.mt_tensor_offset(cfg, -1, mt.MT_T_LM_HEAD)[1]
+    assert bench.head_params(SH) == fn + head
+
+
+def test_host_bound_phase_structure():
+    n_unique = 12000
+    upd = 30.0 * params(SH)
+    kw = dict(peak_tflops=1000.0, link=LINK, h2d_bytes=5e9, d2h_bytes=5e9, update_bytes=upd, n_unique=n_unique)
+    slow = bench.step_bounds(SH, host_gbs=100.0, **kw)
+    untouched = 30.0 * (SH["V"] - n_unique) * SH["d"]
+    assert slow["update_bytes_fwd"] == pytest.approx(untouched)
+    assert slow["update_bytes_bwd"] == pytest.approx(upd - untouched)
+    # a slow host: the backward is the optimizer's bytes at the host rate
+    assert slow["bwd"] == pytest.approx((upd - untouched) / 100e9)
+    f_fl, b_fl = bench.phase_flops(SH)
+    L = SH["L"]
+    assert slow["fwd"] == pytest.approx(max(f_fl / 1e15, 5e9 * L / (2 * L - 1) / 50e9))
+    assert slow["bound"] == pytest.approx(max(slow["fwd"] + slow["bwd"], upd / 100e9))
+    # a fast host: the backward is the GPU's or the D2H's
+    fast = bench.step_bounds(SH, host_gbs=1e6, **kw)
+    assert fast["bwd"] == pytest.approx(max(b_fl / 1e15, 5e9 / 50e9))
+    # deferral moves the LM head and the deferred layers into the forward phase
+    d1 = bench.step_bounds(SH, host_gbs=100.0, deferred_layers=1, **kw)
+    moved = 30.0 * (bench.head_params(SH) + bench.layer_params(SH))
+    assert d1["update_bytes_fwd"] - slow["update_bytes_fwd"] == pytest.approx(moved)
+    assert d1["bwd"] == pytest.approx(slow["bwd"] - moved / 100e9)
+    assert d1["fwd"] == slow["fwd"]
+    # however the updates are split, the step needs all of them at the host rate
+    assert d1["bound"] >= upd / 100e9 - 1e-12
+    # the DRAM model adds the copies' traffic, so it never undercuts the bound's phases
+    for r in (slow, fast, d1):
+        assert r["model"] >= r["fwd"] + r["bwd"] - 1e-12
+        assert r["dram_fwd"] + r["dram_bwd"] == pytest.approx(upd + 5e9 + 5e9)
