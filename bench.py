@@ -20,6 +20,7 @@ import argparse
 import json
 import math
 import os
+import platform
 import statistics
 import subprocess
 import sys
@@ -179,6 +180,30 @@ def oracle_sample_tokens_per_s(sh, seed=0):
     return T / t_step, t_layer + t_head + t_adam, desc
 
 
+def cpu_model() -> str:
+    """The host CPU's model name, as the kernel reports it."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
+
+
+def step_spread(stats):
+    """Min and median over the timed steps of each step's host wall time
+    (the mt_train_step call) and compute-stream time (device events)."""
+    out = {}
+    for key, name in (("host_step_ms", "host_ms"), ("step_ms", "device_ms")):
+        v = [float(st[key]) for st in stats]
+        if v:
+            out[name + "_min"] = min(v)
+            out[name + "_median"] = statistics.median(v)
+    return out
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -210,7 +235,8 @@ def run_reference(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_desc(args.workload, sh), "global_batch": sh["b"], "seq_len": sh["s"],
                    "parallelism": "none (CPU)"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "cpu_model": cpu_model(), "kind": "oracle",
+                         "sample": desc},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -597,11 +623,12 @@ def main():
             "e2e": {"value": weak_value(T, world, K, t_e2e), "unit": UNIT, "h2d_bytes_per_step": 2 * T * 4,
                     "d2h_bytes_per_step": 4, "timing": "host wall clock around mt_train_step (public C API)"},
             "gpu_launches": int(sum(s["kernel_launches"] for s in stats)),
+            "per_step": step_spread(stats),
         }
         if world == 1 and not args.no_cpu_baseline:
             v, secs, desc = oracle_sample_tokens_per_s(sh)
-            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                                    "sample": desc, "seconds": secs}
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": blas_threads(), "cpu_model": cpu_model(),
+                                    "kind": "oracle", "sample": desc, "seconds": secs}
         print(json.dumps(line), flush=True)
     if dist is not None:
         barrier()

@@ -61,3 +61,11 @@ def test_host_bound_phase_structure():
     for r in (slow, fast, d1):
         assert r["model"] >= r["fwd"] + r["bwd"] - 1e-12
         assert r["dram_fwd"] + r["dram_bwd"] == pytest.approx(upd + 5e9 + 5e9)
+
+
+def test_step_spread_and_cpu_model():
+    stats = [dict(host_step_ms=h, step_ms=d) for h, d in ((320.0, 290.0), (318.0, 288.0), (330.0, 291.0))]
+    sp = bench.step_spread(stats)
+    assert sp == dict(host_ms_min=318.0, host_ms_median=320.0, device_ms_min=288.0, device_ms_median=290.0)
+    assert bench.step_spread([]) == {}
+    assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
