@@ -21,6 +21,7 @@ import json
 import math
 import os
 import platform
+import re
 import statistics
 import subprocess
 import sys
@@ -378,11 +379,14 @@ def step_bounds(sh, *, peak_tflops, link, host_gbs, h2d_bytes, d2h_bytes, update
 
 
 def defer_layers(sh):
-    """Deferred layers as the library reads them (MT_DEFER_LAYERS, default 1)."""
-    try:
-        n = int(os.environ.get("MT_DEFER_LAYERS", "1"))
-    except ValueError:
+    """Deferred layers as the library reads them: MT_DEFER_LAYERS (default 1)
+    parsed like strtol (leading integer, else 0), clamped to [0, L-1]."""
+    env = os.environ.get("MT_DEFER_LAYERS")
+    if env is None:
         n = 1
+    else:
+        m = re.match(r"\s*([+-]?\d+)", env)
+        n = int(m.group(1)) if m else 0
     return min(max(n, 0), sh["L"] - 1)
 
 

@@ -69,3 +69,21 @@ def test_step_spread_and_cpu_model():
     assert sp == dict(host_ms_min=318.0, host_ms_median=320.0, device_ms_min=288.0, device_ms_median=290.0)
     assert bench.step_spread([]) == {}
     assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
+
+
+@pytest.mark.parametrize("env", [None, "0", "2", " 3", "2x", "abc", "-4", "99"])
+def test_deferred_layer_count_matches_the_library(monkeypatch, env):
+    """bench.defer_layers reads MT_DEFER_LAYERS as the library does: its
+    host-memory accounting grows by one layer-sized buffer per deferred layer."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    sh = dict(L=5, d=256, H=4, Hkv=4, F=688, V=1024, b=2, s=128)
+    if env is None:
+        monkeypatch.delenv("MT_DEFER_LAYERS", raising=False)
+    else:
+        monkeypatch.setenv("MT_DEFER_LAYERS", env)
+    cfg = arena.config(sh)
+    cfg.flags = mt.MT_FLAG_GRAD_RING
+    ring = mt.mt_host_state_bytes(cfg)
+    cfg.flags |= mt.MT_FLAG_DEFER_UPDATES
+    layer_bytes = 4 * (mt.mt_tensor_offset(cfg, 1, 0)[0] - mt.mt_tensor_offset(cfg, 0, 0)[0])
+    assert mt.mt_host_state_bytes(cfg) - ring == bench.defer_layers(sh) * layer_bytes

@@ -199,3 +199,13 @@ def test_host_adamw_rejects_bad_step():
     with pytest.raises(mt.MTError):
         mt.mt_k_adamw_host(x.ctypes.data, x.ctypes.data, x.ctypes.data, x.ctypes.data, 0, 4, 1e-3, 0.9, 0.95,
                            1e-8, 0.1, 0)
+
+
+def test_null_context_calls_are_rejected():
+    """Every context call given NULL returns MT_ERR_ARG (mt_destroy ignores it)."""
+    mt = _mt()
+    assert mt.lib.mt_flush(None) == -1
+    assert mt.lib.mt_get_params(None, None, 0) == -1
+    assert mt.lib.mt_get_grads(None, None, 0) == -1
+    assert mt.lib.mt_get_opt_state(None, None, None, 0, None) == -1
+    mt.lib.mt_destroy(None)
