@@ -50,7 +50,7 @@ GEMM_TRAFFIC_PER_LAUNCH = {"llama-1.3b": 561.8e6}
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="llama-1.3b", choices=list(synth.WORKLOADS))
     ap.add_argument("--impl", default="mt", choices=["mt", "reference"])
