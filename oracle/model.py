@@ -200,7 +200,9 @@ def rope_bwd(dy: np.ndarray, cos: np.ndarray, sin: np.ndarray) -> np.ndarray:
 # ---------------------------------------------------------------------------
 # Causal attention with grouped KV heads. Reading: scale 1/sqrt(hd), key j is
 # visible to query i iff j <= i (same sequence); query head h reads KV head
-# floor(h / (H / Hkv)).
+# floor(h / (H / Hkv)). The query rows may be a block of the sequence: rows at
+# positions q_offset .. q_offset + r - 1 against keys 0 .. s_k - 1 (the same
+# visibility rule, so a long sequence can be checked a few rows at a time).
 # ---------------------------------------------------------------------------
 
 def _heads_first(x):
@@ -208,21 +210,25 @@ def _heads_first(x):
     return x.transpose(0, 2, 1, 3)
 
 
-def _visible_scores(q, k):
-    """Scaled scores q_i . k_j / sqrt(hd) per query head, -inf where j > i.
-    q: [b, s, H, hd]; k: [b, s, Hkv, hd]. Returns [b, H, s, s]."""
-    b, s, H, hd = q.shape
+def _visible_scores(q, k, q_offset=0):
+    """Scaled scores q_i . k_j / sqrt(hd) per query head, -inf where key j comes
+    after query i. q: [b, r, H, hd], row i at position q_offset + i;
+    k: [b, s_k, Hkv, hd] from position 0. Returns [b, H, r, s_k]."""
+    b, r, H, hd = q.shape
+    sk = k.shape[1]
     kk = np.repeat(k, H // k.shape[2], axis=2)  # kv head for query head h is h // group
     S = _heads_first(q) @ _heads_first(kk).transpose(0, 1, 3, 2) / np.sqrt(hd)
-    mask = np.tril(np.ones((s, s), dtype=bool))
+    mask = np.arange(sk)[None, :] <= (q_offset + np.arange(r))[:, None]
     return np.where(mask[None, None], S, -np.inf)
 
 
-def attention_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray):
-    """q: [b, s, H, hd]; k, v: [b, s, Hkv, hd]. Returns (o [b,s,H,hd], P [b,H,s,s])."""
+def attention_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray, q_offset: int = 0):
+    """q: [b, r, H, hd] (rows at positions q_offset ..); k, v: [b, s_k, Hkv, hd].
+    Returns (o [b,r,H,hd], P [b,H,r,s_k]); r = s_k and q_offset = 0 is the
+    whole sequence."""
     H = q.shape[2]
     vv = np.repeat(v, H // v.shape[2], axis=2)
-    S = _visible_scores(q, k)
+    S = _visible_scores(q, k, q_offset)
     S = S - S.max(axis=-1, keepdims=True)
     P = np.exp(S)
     P = P / P.sum(axis=-1, keepdims=True)
@@ -230,10 +236,10 @@ def attention_fwd(q: np.ndarray, k: np.ndarray, v: np.ndarray):
     return o, P
 
 
-def attention_lse(q: np.ndarray, k: np.ndarray) -> np.ndarray:
-    """Natural log-sum-exp over visible keys of the scaled scores, [b, H, s]:
-    lse[b, h, i] = log sum_{j <= i} exp(q_i . k_j / sqrt(hd))."""
-    S = _visible_scores(q, k)
+def attention_lse(q: np.ndarray, k: np.ndarray, q_offset: int = 0) -> np.ndarray:
+    """Natural log-sum-exp over visible keys of the scaled scores, [b, H, r]:
+    lse[b, h, i] = log sum_{j <= q_offset + i} exp(q_i . k_j / sqrt(hd))."""
+    S = _visible_scores(q, k, q_offset)
     m = S.max(axis=-1, keepdims=True)
     return m[..., 0] + np.log(np.sum(np.exp(S - m), axis=-1))
 
@@ -242,8 +248,11 @@ def attention_bwd(q, k, v, P, do):
     """Backward of o = P v with P = softmax(q k^T / sqrt(hd)) (causal):
       dP = do v^T ; dv = P^T do ; dS = P * (dP - rowsum(dP * P)) ;
       dq = dS k / sqrt(hd) ; dk = dS^T q / sqrt(hd);
-    dk, dv of a KV head sum over the query heads of its group."""
-    b, s, H, hd = q.shape
+    dk, dv of a KV head sum over the query heads of its group. With a block of
+    query rows (P from attention_fwd with q_offset), dk and dv [b, s_k, ...]
+    are those rows' contributions."""
+    b, r, H, hd = q.shape
+    sk = k.shape[1]
     Hkv = k.shape[2]
     group = H // Hkv
     kh = _heads_first(np.repeat(k, group, axis=2))
@@ -255,8 +264,8 @@ def attention_bwd(q, k, v, P, do):
     scale = 1.0 / np.sqrt(hd)
     dq = _heads_first(dS @ kh) * scale
     dkk = _heads_first(dS.transpose(0, 1, 3, 2) @ _heads_first(q)) * scale
-    dk = dkk.reshape(b, s, Hkv, group, hd).sum(axis=3)
-    dv = dvv.reshape(b, s, Hkv, group, hd).sum(axis=3)
+    dk = dkk.reshape(b, sk, Hkv, group, hd).sum(axis=3)
+    dv = dvv.reshape(b, sk, Hkv, group, hd).sum(axis=3)
     return dq, dk, dv
 
 

@@ -47,6 +47,86 @@ def test_attention_brute_force_gqa():
     assert np.all(np.triu(P[0, 0], 1) == 0)  # nothing above the diagonal
 
 
+def _brute_attention_rows(q, k, v, q_offset):
+    """Scalar loops for query rows at positions q_offset + i against keys
+    0 .. s_k - 1: softmax over j <= q_offset + i; also the log-sum-exp."""
+    b, r, H, hd = q.shape
+    group = H // k.shape[2]
+    o = np.zeros_like(q)
+    lse = np.zeros((b, H, r))
+    for bi in range(b):
+        for h in range(H):
+            g = h // group
+            for i in range(r):
+                last = q_offset + i
+                sc = [sum(q[bi, i, h, e] * k[bi, j, g, e] for e in range(hd)) / math.sqrt(hd)
+                      for j in range(last + 1)]
+                mx = max(sc)
+                ex = [math.exp(x - mx) for x in sc]
+                z = sum(ex)
+                lse[bi, h, i] = mx + math.log(z)
+                for e in range(hd):
+                    o[bi, i, h, e] = sum(ex[j] * v[bi, j, g, e] for j in range(last + 1)) / z
+    return o, lse
+
+
+def test_attention_query_block_brute_force_gqa():
+    """A block of query rows at positions q_offset .. against the whole key
+    prefix (how the long-context parity tests sample rows) follows the same
+    causal rule, checked by scalar loops."""
+    rng = np.random.default_rng(5)
+    sk, r, off = 11, 3, 6
+    q = rng.normal(size=(2, r, 4, 4))
+    k = rng.normal(size=(2, sk, 2, 4))
+    v = rng.normal(size=(2, sk, 2, 4))
+    o, P = oracle.attention_fwd(q, k, v, q_offset=off)
+    ro, rlse = _brute_attention_rows(q, k, v, off)
+    assert np.allclose(o, ro, rtol=1e-12, atol=1e-12)
+    assert np.allclose(oracle.attention_lse(q, k, q_offset=off), rlse, rtol=1e-12, atol=1e-12)
+    assert P.shape == (2, 4, r, sk) and np.allclose(P.sum(-1), 1.0)
+    for i in range(r):
+        assert np.all(P[:, :, i, off + i + 1:] == 0)  # keys after the row's position are invisible
+
+
+def test_attention_query_block_zero_query_is_prefix_mean():
+    rng = np.random.default_rng(6)
+    sk, r, off = 12, 4, 8
+    q = np.zeros((1, r, 2, 8))
+    k = rng.normal(size=(1, sk, 1, 8))
+    v = rng.normal(size=(1, sk, 1, 8))
+    o, _ = oracle.attention_fwd(q, k, v, q_offset=off)
+    for i in range(r):
+        assert np.allclose(o[0, i, 0], v[0, :off + i + 1, 0].mean(axis=0))
+
+
+def test_attention_query_block_backward_central_differences():
+    """dq of the block's rows and the block's contribution to dk and dv, for
+    L = sum(o * W), against central differences in fp64."""
+    rng = np.random.default_rng(7)
+    sk, r, off, hd = 7, 3, 4, 4
+    q = rng.normal(size=(1, r, 2, hd))
+    k = rng.normal(size=(1, sk, 1, hd))
+    v = rng.normal(size=(1, sk, 1, hd))
+    Wt = rng.normal(size=(1, r, 2, hd))
+    o, P = oracle.attention_fwd(q, k, v, q_offset=off)
+    dq, dk, dv = oracle.attention_bwd(q, k, v, P, Wt)
+    h = 1e-6
+
+    def loss(q_, k_, v_):
+        return float(np.sum(oracle.attention_fwd(q_, k_, v_, q_offset=off)[0] * Wt))
+
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        fd = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = [xp if a is x else a for a in (q, k, v)]
+            argm = [xm if a is x else a for a in (q, k, v)]
+            fd[idx] = (loss(*args) - loss(*argm)) / (2 * h)
+        assert np.allclose(g, fd, rtol=1e-6, atol=1e-8)
+
+
 def test_attention_zero_query_is_prefix_mean():
     rng = np.random.default_rng(1)
     s = 9

@@ -79,6 +79,13 @@ def _rope_fwd_pairs_adjacent(x, cos, sin):
     return out
 
 
+_orig_scores = M._visible_scores
+
+
+def _scores_see_next_key(q, k, q_offset=0):
+    return _orig_scores(q, k, q_offset + 1)  # causal mask off by one: key i + 1 visible to query i
+
+
 @pytest.mark.parametrize("name,fn", [
     ("rope_bwd", _rope_bwd_wrong_sign),
     ("rmsnorm_bwd", _rms_bwd_dropped_term),
@@ -87,6 +94,7 @@ def _rope_fwd_pairs_adjacent(x, cos, sin):
     ("head_ce_fwd_bwd", _head_not_mean),
     ("rope_fwd", _rope_fwd_pairs_adjacent),
     ("attention_fwd", _attn_fwd_wrong_group),
+    ("_visible_scores", _scores_see_next_key),
 ])
 def test_planted_mistake_is_caught(monkeypatch, name, fn):
     monkeypatch.setattr(M, name, fn)
