@@ -209,3 +209,27 @@ def test_null_context_calls_are_rejected():
     assert mt.lib.mt_get_grads(None, None, 0) == -1
     assert mt.lib.mt_get_opt_state(None, None, None, 0, None) == -1
     mt.lib.mt_destroy(None)
+
+
+def _declared_param_counts():
+    """Parameter count of every function the headers declare."""
+    out = {}
+    for h in ("mt.h", "mt_kernels.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(mt_\w+)\s*\(([^)]*)\)\s*;", src, flags=re.M | re.S):
+            params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
+            out[m.group(1)] = len(params)
+    return out
+
+
+def test_binding_signatures_match_the_headers():
+    """Every function the Python binding declares takes as many arguments as its
+    C declaration, and the binding covers every declared function."""
+    mt = _mt()
+    counts = _declared_param_counts()
+    assert set(counts) == _declared_functions()
+    for name, n in sorted(counts.items()):
+        fn = getattr(mt.lib, name)
+        assert fn.argtypes is not None, f"{name} has no ctypes signature"
+        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
