@@ -211,25 +211,51 @@ def test_null_context_calls_are_rejected():
     mt.lib.mt_destroy(None)
 
 
-def _declared_param_counts():
-    """Parameter count of every function the headers declare."""
+def _declared_params():
+    """Parameter declarations of every function the headers declare."""
     out = {}
     for h in ("mt.h", "mt_kernels.h"):
         src = open(os.path.join(ROOT, "include", h)).read()
         src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(mt_\w+)\s*\(([^)]*)\)\s*;", src, flags=re.M | re.S):
-            params = [p for p in m.group(2).split(",") if p.strip() and p.strip() != "void"]
-            out[m.group(1)] = len(params)
+        for m in re.finditer(r"^([A-Za-z_][\w\s\*]*?)\b(mt_\w+)\s*\(([^)]*)\)\s*;", src, flags=re.M | re.S):
+            params = [p.strip() for p in m.group(3).split(",") if p.strip() and p.strip() != "void"]
+            out[m.group(2)] = (m.group(1).strip(), params)
     return out
 
 
+# scalar C types of the headers: (is floating point, bytes)
+_C_SCALARS = {"int": (False, 4), "int32_t": (False, 4), "uint32_t": (False, 4), "int64_t": (False, 8),
+              "size_t": (False, 8), "float": (True, 4), "double": (True, 8)}
+
+
+def _kind_of_ctype(t):
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return "pointer"
+    return (t in (ctypes.c_float, ctypes.c_double), ctypes.sizeof(t))
+
+
+def _kind_of_param(decl):
+    if "*" in decl:
+        return "pointer"
+    ctype = decl.replace("const ", "").split()[0]
+    return _C_SCALARS[ctype]
+
+
 def test_binding_signatures_match_the_headers():
-    """Every function the Python binding declares takes as many arguments as its
-    C declaration, and the binding covers every declared function."""
+    """Every function the Python binding declares takes the arguments and
+    returns the type of its C declaration: as many arguments, each a pointer
+    where the header has one, else a scalar of the same kind (integer or
+    floating point) and width; and the binding covers every declared function."""
     mt = _mt()
-    counts = _declared_param_counts()
-    assert set(counts) == _declared_functions()
-    for name, n in sorted(counts.items()):
+    decls = _declared_params()
+    assert set(decls) == _declared_functions()
+    for name, (ret, params) in sorted(decls.items()):
         fn = getattr(mt.lib, name)
         assert fn.argtypes is not None, f"{name} has no ctypes signature"
-        assert len(fn.argtypes) == n, (name, len(fn.argtypes), n)
+        if ret == "void":
+            assert fn.restype is None, name
+        else:
+            assert _kind_of_ctype(fn.restype) == _kind_of_param(ret), (name, ret, fn.restype)
+        assert len(fn.argtypes) == len(params), (name, len(fn.argtypes), len(params))
+        for i, (t, decl) in enumerate(zip(fn.argtypes, params)):
+            assert _kind_of_ctype(t) == _kind_of_param(decl), (name, i, decl, t)
