@@ -8,6 +8,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 import synth
@@ -191,6 +192,34 @@ def test_host_adamw_matches_oracle_over_steps():
         # the streamed copy is exactly the round-to-nearest-even of the new master
         ref_bits = (oracle.bf16_round(p).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
         assert np.array_equal(pb, ref_bits)
+
+
+def test_host_bf16_copy_special_values_match_torch():
+    """With lr = 0 and wd = 0 the master is unchanged and the streamed bf16 copy
+    is the library's own round-to-nearest-even of it: ties to even and to odd,
+    just below and above a tie, a carry into the next exponent, the overflow to
+    infinity of float32's largest value, subnormals, signed zeros and
+    infinities bit-exact against torch's conversion, NaN kept NaN, in the
+    16-wide vector loop and in the scalar tail."""
+    mt = _mt()
+    bits = [0x3F808000, 0x3F818000, 0x3F807FFF, 0x3F808001, 0x3F7FFFFF, 0x7F7FFFFF, 0xFF7FFFFF, 0x00000001,
+            0x000FFFFF, 0x80008000, 0x00000000, 0x80000000, 0x7F800000, 0xFF800000, 0x3F800000, 0xBF818000,
+            0x7FC00000, 0xFFC12345, 0x7F800001]
+    vals = np.array(bits, dtype=np.uint32).view(np.float32)
+    p = np.concatenate([vals, vals, vals[:15]]).copy()  # 53 = 3 x 16 + 5: vector lanes and a scalar tail
+    n = p.size
+    p0 = p.copy()
+    g, m, v = np.zeros(n, np.float32), np.zeros(n, np.float32), np.zeros(n, np.float32)
+    pb = np.zeros(n, dtype=np.uint16)
+    mt.mt_k_adamw_host(p.ctypes.data, g.ctypes.data, m.ctypes.data, v.ctypes.data, pb.ctypes.data, n,
+                       0.0, 0.9, 0.95, 1e-8, 0.0, 1)
+    nan = np.isnan(p0)
+    assert np.array_equal(p.view(np.uint32)[~nan], p0.view(np.uint32)[~nan]) and np.isnan(p[nan]).all()
+    ref = torch.from_numpy(p0).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got_f = (pb.astype(np.uint32) << 16).view(np.float32)
+    assert np.array_equal(pb[~nan], ref[~nan]), [(hex(b), hex(a), hex(r)) for b, a, r in
+                                                 zip(p0.view(np.uint32), pb, ref) if a != r]
+    assert np.isnan(got_f[nan]).all()
 
 
 def test_host_adamw_rejects_bad_step():
