@@ -145,7 +145,7 @@ int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_t ldqkv, co
 /* The same backward (same arguments and outputs as mt_k_attn_bwd) on the
  * tcgen05 tensor cores, head_dim 128 only (MT_ERR_CONFIG otherwise): one CTA
  * per 128-key block accumulates dK and dV in tensor memory over the group's
- * query heads and 64-query blocks; dQ goes through the fp32 accumulator.
+ * query heads and 128-query blocks; dQ goes through the fp32 accumulator.
  * q, k, v, o, dout 16-byte aligned; dev_err as for mt_k_attn_fwd_tc. */
 int mt_k_attn_bwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o, const void* dout,
                      int64_t ldo, const float* lse, float* dvec, float* dq_acc, int64_t ldqa, void* dq, int64_t lddq,
