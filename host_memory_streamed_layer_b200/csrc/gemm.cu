@@ -3,10 +3,10 @@
 //
 // This is the dense contraction of every projection in the streamed decoder
 // layer (MegaTrain, "Full Precision Training of 100B+ Parameter Large Language
-// Models on a Single GPU", abstract: each streamed layer "runs the matmuls",
-// saify.me "The memory-centric design"): the forward products u Wqkv^T, a Wo^T,
-// w Wgu^T, act Wd^T, the input-gradient products dY W and the weight-gradient
-// products dY^T X of their backward.
+// Models on a Single GPU", abstract; saify.me, "The memory-centric design":
+// each streamed layer's matrix products run on the GPU): the forward products
+// u Wqkv^T, a Wo^T, w Wgu^T, act Wd^T, the input-gradient products dY W and
+// the weight-gradient products dY^T X of their backward.
 //
 // Operands may be K-major (the reduction index is contiguous) or MN-major (the
 // output index is contiguous), which covers all three products without a

@@ -35,9 +35,8 @@ extern "C" {
 
 /* Dense product C[M,N] = A[M,K] B[N,K]^T with bf16 inputs and fp32
  * accumulation on the tcgen05 tensor cores: the matmuls a streamed layer runs
- * (MegaTrain abstract; saify.me, "The memory-centric design": "runs the
- * matmuls"), in forward (X W^T), input-gradient (dY W) and weight-gradient
- * (dY^T X) form.
+ * (MegaTrain abstract; saify.me, "The memory-centric design"), in forward
+ * (X W^T), input-gradient (dY W) and weight-gradient (dY^T X) form.
  *   A: a_mn_major = 0: element (m,k) at A[m*lda + k]; = 1: at A[k*lda + m]
  *   B: b_mn_major = 0: element (n,k) at B[n*ldb + k]; = 1: at B[k*ldb + n]
  *   C: element (m,n) at C[m*ldc + n]; R likewise with ldr.
