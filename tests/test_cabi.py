@@ -288,3 +288,29 @@ def test_binding_signatures_match_the_headers():
         assert len(fn.argtypes) == len(params), (name, len(fn.argtypes), len(params))
         for i, (t, decl) in enumerate(zip(fn.argtypes, params)):
             assert _kind_of_ctype(t) == _kind_of_param(decl), (name, i, decl, t)
+
+
+@pytest.mark.parametrize("shape", [synth.WORKLOADS["tiny"], dict(L=3, d=320, H=5, Hkv=1, F=712, V=1000, b=1, s=64)])
+def test_arena_pack_round_trips_through_the_oracle_layout(shape):
+    """arena.pack places every tensor where the oracle's independent reading of
+    the layout expects it, 256-byte aligned, with zero padding between
+    tensors; a tensor of the wrong size is rejected."""
+    from host_memory_streamed_layer_b200 import arena
+    cfg = arena.config(shape, lr=2e-3)
+    assert abs(cfg.lr - 2e-3) < 1e-9
+    W = synth.init_weights(shape, 4)
+    A = arena.pack(cfg, W)
+    assert A.ctypes.data % 256 == 0 and A.dtype == np.float32
+    c = oracle.OracleConfig(**shape)
+    U = oracle.unpack_arena(A, c, dtype=np.float32)
+    for k, w in W.items():
+        assert np.array_equal(U[k], np.asarray(w, dtype=np.float32).reshape(U[k].shape)), k
+    used = np.zeros(A.size, dtype=bool)
+    for layer, tid, off, shp in oracle.arena_layout(c)[0]:
+        used[off:off + int(np.prod(shp))] = True
+    assert np.all(A[~used] == 0)
+    bad = dict(W)
+    k0 = next(iter(bad))
+    bad[k0] = np.zeros(np.asarray(bad[k0]).size + 1, dtype=np.float32)
+    with pytest.raises(ValueError):
+        arena.pack(cfg, bad)
