@@ -516,31 +516,22 @@ int launch_cast_f32_bf16(const float* in, void* out, int64_t n, cudaStream_t st)
 // The per-block partial sums of dg live in this fixed device array instead of
 // a caller buffer. Host code must not pass the array's name to a kernel (in
 // host code it is only a stand-in for the device symbol): the device address
-// is looked up once per device with cudaGetSymbolAddress and cached.
+// is looked up with cudaGetSymbolAddress on every call, with the caller's
+// device current. Nothing is cached, so the address stays right after a
+// device reset or a context re-creation, which may reload the module at
+// another address.
 // ---------------------------------------------------------------------------
-#include <mutex>
-
 namespace mt {
 namespace {
 
 constexpr int kNoAllocScratchFloats = 1 << 20;  // 4 MiB per device that loads the library
 static __device__ __align__(256) float g_rmsnorm_scratch[kNoAllocScratchFloats];
 
-constexpr int kMaxDevices = 64;
-float* g_scratch_addr[kMaxDevices] = {};
-std::mutex g_scratch_mu;
-
-// Address of the scratch array on the current device (set up on first use).
+// Address of the scratch array on the current device.
 int scratch_address(float** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MT_ERR_CUDA;
-  std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_rmsnorm_scratch) != cudaSuccess || !p) return MT_ERR_CUDA;
-    g_scratch_addr[dev] = static_cast<float*>(p);
-  }
-  *out = g_scratch_addr[dev];
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_rmsnorm_scratch) != cudaSuccess || !p) return MT_ERR_CUDA;
+  *out = static_cast<float*>(p);
   return MT_OK;
 }
 

@@ -75,9 +75,11 @@ int mt_k_rmsnorm_bwd(const float* x, const void* g, const float* rstd, const flo
  * The partial sums live in one fixed 4 MiB device array inside the library
  * (1M floats, held on every GPU that loads the library until the process
  * exits); the block count is reduced when needed so that blocks x d partials
- * fit. Limits: d <= 8192 and d % 4 == 0, else MT_ERR_ARG. The first call on a
- * device looks up the array's device address (cudaGetSymbolAddress) with that
- * device current; make that first call before any stream capture. Each
+ * fit. Limits: d <= 8192 and d % 4 == 0, else MT_ERR_ARG. Every call looks
+ * up the array's device address (cudaGetSymbolAddress) on the current device
+ * and caches nothing, so a device reset between calls is harmless; the first
+ * call on a device also loads the library's module there, so make that first
+ * call before any stream capture. Each
  * device has its own copy of the array, and every call on that device shares
  * it, which keeps the last call's contents: two calls whose executions overlap
  * on the GPU (for example on two streams with no ordering between them) race
