@@ -25,6 +25,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <iterator>
 #include <atomic>
 #include <cmath>
 #include <chrono>
@@ -69,8 +70,11 @@ inline float normal_at(uint64_t key, uint64_t i) {
 
 struct Job {
   // HEAD_PREV / LAYER_PREV: an update deferred from the previous step
-  // (MT_FLAG_DEFER_UPDATES), its gradients already checked.
-  enum Kind { LAYER, HEAD, EMBED, EMBED_UNTOUCHED, HEAD_PREV, LAYER_PREV } kind;
+  // (MT_FLAG_DEFER_UPDATES), its gradients already checked. EMBED_UNTOUCHED:
+  // the zero-gradient update of the embedding rows no token of the step
+  // touched, run once every gradient of the step has passed its checks;
+  // EMBED_UNTOUCHED_PREV: the same update deferred into the next step.
+  enum Kind { LAYER, HEAD, EMBED, EMBED_UNTOUCHED, HEAD_PREV, LAYER_PREV, EMBED_UNTOUCHED_PREV } kind;
   int layer;
   cudaEvent_t ready;         // offload of this job's gradients has completed
   int flag_index;            // index in the finite-flag array
@@ -109,6 +113,12 @@ struct mt_ctx {
   int32_t* flags_h = nullptr;     // pinned finite flags [L + 2]
   float* misc_h = nullptr;        // pinned: loss sum, device error word
   std::vector<int32_t> uniq, prev_uniq;
+  // MT_FLAG_DEFER_UPDATES: the zero-gradient update of the embedding rows that
+  // step `untouched_step` did not touch (its touched rows: untouched_of) is
+  // pending; `untouched_skip` lists the rows the queued remainder leaves out.
+  bool untouched_pending = false;
+  int untouched_step = 0;
+  std::vector<int32_t> untouched_of, untouched_skip;
   ThreadPool* pool = nullptr;
 
   // ---- device memory ----
@@ -271,9 +281,15 @@ int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
   } while (0)
 
 // ---------------------------------------------------------------------------
-// Finite check of a gradient range: flag = 1 if any value is NaN or Inf.
+// Check of a gradient range before its host update: flag bit 0 is set if any
+// value is NaN or Inf, bit 1 if any kernel so far in the step has reported a
+// bounded wait that ran out (its outputs, and so these gradients, are then
+// undefined even when finite).
 // ---------------------------------------------------------------------------
-__global__ void k_check_finite(const float* __restrict__ g, size_t n, int32_t* __restrict__ flag) {
+constexpr int32_t kFlagNonFinite = 1, kFlagDeviceError = 2;
+
+__global__ void k_check_finite(const float* __restrict__ g, size_t n, const int32_t* __restrict__ dev_err,
+                               int32_t* __restrict__ flag) {
   bool bad = false;
   const size_t n4 = n / 4;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4; i += (size_t)gridDim.x * blockDim.x) {
@@ -281,12 +297,13 @@ __global__ void k_check_finite(const float* __restrict__ g, size_t n, int32_t* _
     bad |= !isfinite(v.x) || !isfinite(v.y) || !isfinite(v.z) || !isfinite(v.w);
   }
   if (blockIdx.x == 0 && threadIdx.x < (n & 3)) bad |= !isfinite(g[n4 * 4 + threadIdx.x]);
-  if (__syncthreads_or(bad) && threadIdx.x == 0) *flag = 1;
+  if (__syncthreads_or(bad) && threadIdx.x == 0) atomicOr(flag, kFlagNonFinite);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && *dev_err != 0) atomicOr(flag, kFlagDeviceError);
 }
 
 int check_finite(mt_ctx* c, const float* g, size_t n, int idx) {
   CK(cudaMemsetAsync(c->d_flags + idx, 0, sizeof(int32_t), c->s_comp));
-  k_check_finite<<<296, 256, 0, c->s_comp>>>(g, n, c->d_flags + idx);
+  k_check_finite<<<296, 256, 0, c->s_comp>>>(g, n, c->d_err, c->d_flags + idx);
   CK(cudaGetLastError());
   c->launches += 1;
   return MT_OK;
@@ -516,6 +533,38 @@ std::vector<Seg> layer_or_head_segs(mt_ctx* c, int l, const float* g) {
   return segs;
 }
 
+// Segments of the zero-gradient update of every embedding row not listed in
+// skip (sorted, distinct row ids): the rows no token of a step touched.
+std::vector<Seg> untouched_segs(mt_ctx* c, const std::vector<int32_t>& skip) {
+  const Layout& y = c->lay;
+  const size_t d = y.sh.d;
+  std::vector<Seg> segs;
+  int32_t next = 0;  // first row of the current untouched run
+  for (size_t u = 0; u <= skip.size(); ++u) {
+    const int32_t stop = u < skip.size() ? skip[u] : y.sh.V;
+    if (stop > next)
+      segs.push_back({y.embed.off + (size_t)next * d, (size_t)(stop - next) * d, c->bf_embed + (size_t)next * d,
+                      nullptr});
+    next = stop + 1;
+  }
+  return segs;
+}
+
+// Records the outcome of a job's gradient checks (flag bits of k_check_finite)
+// and returns true while updates may still run this step: after a failed check
+// this and every later update of the step are skipped.
+bool passes_checks(mt_ctx* c, int32_t flag) {
+  if ((flag & kFlagDeviceError) && c->opt_status == MT_OK) {
+    c->opt_status = MT_ERR_DEVICE;
+    c->err = "a kernel's bounded wait ran out; this and the remaining updates were skipped";
+  } else if ((flag & kFlagNonFinite) && c->opt_status == MT_OK) {
+    c->opt_status = MT_ERR_NONFINITE;
+    c->err = "non-finite gradient; this and the remaining updates were skipped";
+  }
+  if (flag & (kFlagDeviceError | kFlagNonFinite)) c->skip_updates = true;
+  return !c->skip_updates;
+}
+
 void run_job_body(mt_ctx* c, const Job& j) {
   const Layout& y = c->lay;
   const Shapes& s = y.sh;
@@ -526,44 +575,34 @@ void run_job_body(mt_ctx* c, const Job& j) {
                    c->overlap_threads);
     return;
   }
+  if (j.kind == Job::EMBED_UNTOUCHED_PREV) {
+    // The rest of the previous step's untouched-row update (that step passed
+    // every check): rows this step does not touch either, so neither the GPU
+    // nor this step's updates read them meanwhile.
+    adamw_segments(c, untouched_segs(c, c->untouched_skip), j.step, c->overlap_threads);
+    return;
+  }
   if (j.kind == Job::EMBED_UNTOUCHED) {
-    // Rows no token of this batch touches have a zero gradient, so their update
-    // does not depend on this step's backward and runs while the GPU is in the
-    // forward sweep (the gather reads only the touched rows); it reads no
-    // gradient at all. With a gradient arena, zero last step's touched rows
-    // first: every row's stored gradient is then 0 until the touched rows are
-    // scattered at the end.
+    // Queued after the step's last checked job: runs only if every check passed.
+    if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
+    adamw_segments(c, untouched_segs(c, c->uniq), c->step);
+    return;
+  }
+  if (j.kind == Job::EMBED) {
+    // Touched rows: check this step's gradient rows for NaN/Inf and, with a
+    // gradient arena, put last step's touched rows back to zero and scatter
+    // this step's rows in (every other row's stored gradient is 0). The update
+    // reads them from the staging rows.
+    float* ge = c->grad ? c->grad + y.embed.off : nullptr;
     const size_t d = s.d;
-    if (c->grad) {
-      float* ge = c->grad + y.embed.off;
-      const int nt = c->pool->size() * 4;
+    const int nt = c->pool->size() * 4;
+    if (ge) {
       const size_t np = c->prev_uniq.size();
       c->pool->run(nt, [&](int i) {
         for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k) memset(ge + (size_t)c->prev_uniq[k] * d, 0, d * 4);
       });
     }
     c->prev_uniq = c->uniq;
-    if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
-    const int threads = (c->cfg.flags & MT_FLAG_DEFER_UPDATES) ? c->overlap_threads : 0;
-    std::vector<Seg> segs;
-    int32_t next = 0;  // first row of the current untouched run
-    for (size_t u = 0; u <= c->uniq.size(); ++u) {
-      const int32_t stop = u < c->uniq.size() ? c->uniq[u] : s.V;
-      if (stop > next)
-        segs.push_back(
-            {y.embed.off + (size_t)next * d, (size_t)(stop - next) * d, c->bf_embed + (size_t)next * d, nullptr});
-      next = stop + 1;
-    }
-    adamw_segments(c, segs, c->step, threads);
-    return;
-  }
-  if (j.kind == Job::EMBED) {
-    // Touched rows: check this step's gradient rows for NaN/Inf (and scatter
-    // them into the gradient arena when there is one). The update reads them
-    // from the staging rows.
-    float* ge = c->grad ? c->grad + y.embed.off : nullptr;
-    const size_t d = s.d;
-    const int nt = c->pool->size() * 4;
     const size_t nu = c->uniq.size();
     std::vector<char> bad(nt, 0);
     c->pool->run(nt, [&](int i) {
@@ -578,16 +617,13 @@ void run_job_body(mt_ctx* c, const Job& j) {
       bad[i] = b;
     });
     for (char b : bad)
-      if (b) c->flags_h[j.flag_index] = 1;
+      if (b) c->flags_h[j.flag_index] |= kFlagNonFinite;
+    int32_t dev_err = 0;  // device error word as of the embedding backward
+    memcpy(&dev_err, c->misc_h + 2, 4);
+    if (dev_err != 0) c->flags_h[j.flag_index] |= kFlagDeviceError;
   }
-  if (c->flags_h[j.flag_index] != 0) {
-    if (c->opt_status == MT_OK) {
-      c->opt_status = MT_ERR_NONFINITE;
-      c->err = "non-finite gradient; this and the remaining updates were skipped";
-    }
-    c->skip_updates = true;
-  }
-  if (c->skip_updates || (c->cfg.flags & MT_FLAG_NO_UPDATE)) return;
+  if (!passes_checks(c, c->flags_h[j.flag_index])) return;
+  if (c->cfg.flags & MT_FLAG_NO_UPDATE) return;
   if (j.defer) {
     // Gradients are finite: the update runs at the start of the next step.
     Job p = j;
@@ -608,6 +644,14 @@ void run_job_body(mt_ctx* c, const Job& j) {
     }
   }
   adamw_segments(c, segs, c->step);
+  if (j.kind == Job::EMBED && (c->cfg.flags & MT_FLAG_DEFER_UPDATES)) {
+    // The step's last job: every gradient passed its checks, so the
+    // zero-gradient update of the rows it did not touch is due. It runs with
+    // the next step (or at the next flush), overlapping its GPU work.
+    c->untouched_pending = true;
+    c->untouched_step = c->step;
+    c->untouched_of = c->uniq;
+  }
 }
 
 void opt_loop(mt_ctx* c) {
@@ -647,20 +691,22 @@ void wait_jobs(mt_ctx* c) {
 }
 
 // Queues the updates deferred by the last step in the order the forward sweep
-// streams their weights again (layers ascending, then the LM head); they touch
-// disjoint tensors, so any order gives the same result. Called between steps,
-// when the optimizer is idle.
+// streams their weights again (layers ascending, then the LM head), then the
+// rest of the untouched embedding rows, which nothing of the step reads; they
+// touch disjoint tensors, so any order gives the same result. Called between
+// steps, when the optimizer is idle.
 void queue_deferred(mt_ctx* c) {
   if (c->deferred.empty()) return;
-  std::sort(c->deferred.begin(), c->deferred.end(), [](const Job& a, const Job& b) {
-    const int ka = a.kind == Job::HEAD_PREV ? INT32_MAX : a.layer, kb = b.kind == Job::HEAD_PREV ? INT32_MAX : b.layer;
-    return ka < kb;
-  });
+  auto key = [](const Job& j) {
+    return j.kind == Job::EMBED_UNTOUCHED_PREV ? INT32_MAX : j.kind == Job::HEAD_PREV ? INT32_MAX - 1 : j.layer;
+  };
+  std::sort(c->deferred.begin(), c->deferred.end(), [&](const Job& a, const Job& b) { return key(a) < key(b); });
   {
     std::lock_guard<std::mutex> lk(c->opt_mu);
     for (const Job& j : c->deferred) {
       c->jobs.push_back(j);
-      c->prev_pending[j.kind == Job::HEAD_PREV ? c->lay.sh.L : j.layer] = 1;
+      if (j.kind == Job::HEAD_PREV) c->prev_pending[c->lay.sh.L] = 1;
+      if (j.kind == Job::LAYER_PREV) c->prev_pending[j.layer] = 1;
     }
     c->jobs_pending += (int)c->deferred.size();
   }
@@ -668,11 +714,43 @@ void queue_deferred(mt_ctx* c) {
   c->opt_cv.notify_one();
 }
 
+// Queues the remainder of a pending untouched-row update: every row outside
+// `skip` (sorted, distinct). Called between steps.
+void defer_untouched_rest(mt_ctx* c, std::vector<int32_t> skip) {
+  c->untouched_skip = std::move(skip);
+  Job j{Job::EMBED_UNTOUCHED_PREV, -1, nullptr, 0};
+  j.step = c->untouched_step;
+  c->deferred.push_back(j);
+  c->untouched_pending = false;
+}
+
 // Applies pending deferred updates before the state is read or replaced.
 void flush_deferred(mt_ctx* c) {
+  if (c->untouched_pending) defer_untouched_rest(c, c->untouched_of);
   if (c->deferred.empty()) return;
   queue_deferred(c);
   wait_jobs(c);
+}
+
+// Start of a step with a pending untouched-row update from the last step: the
+// rows this step's batch gathers (and later updates) get it first, on every
+// host thread, before any GPU work of the step is enqueued; the other rows
+// follow in the background. Called with the optimizer idle.
+void start_untouched_prev(mt_ctx* c) {
+  const Layout& y = c->lay;
+  const size_t d = y.sh.d;
+  const std::vector<int32_t>& was = c->untouched_of;  // touched by the last step
+  std::vector<Seg> first;
+  std::vector<int32_t> both;
+  both.reserve(was.size() + c->uniq.size());
+  std::set_union(was.begin(), was.end(), c->uniq.begin(), c->uniq.end(), std::back_inserter(both));
+  for (int32_t r : c->uniq)
+    if (!std::binary_search(was.begin(), was.end(), r))
+      first.push_back({y.embed.off + (size_t)r * d, d, c->bf_embed + (size_t)r * d, nullptr});
+  const double t0 = now_s();
+  adamw_segments(c, first, c->untouched_step);
+  c->job_times.push_back({7, -1, t0, now_s()});
+  defer_untouched_rest(c, std::move(both));
 }
 
 // Bounded host wait for the deferred update of layer l (l = L: the LM head)
@@ -749,6 +827,7 @@ int enqueue_step(mt_ctx* c, int n_unique) {
   cudaStream_t sc = c->s_comp;
 
   CK(cudaEventRecord(c->ev_step_start, sc));
+  CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));  // error word of this step's kernels
   CK(cudaMemcpyAsync(c->d_tok, c->stage_i, (size_t)(4 * T + 1) * 4, cudaMemcpyHostToDevice, sc));
   KL(launch_embed_fwd(c->d_tok, c->bf_embed_dev, c->xb, T, d, sc), 1);
   CKM(issue_load(c, 0));
@@ -808,9 +887,12 @@ int enqueue_step(mt_ctx* c, int n_unique) {
   CK(cudaStreamWaitEvent(c->s_d2h, c->ev_emb_ready, 0));
   CK(cudaEventRecord(c->ev_emb_d2h_start, c->s_d2h));
   CK(cudaMemcpyAsync(c->emb_rows_h, c->tmp_f, (size_t)n_unique * d * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  CK(cudaMemcpyAsync(c->misc_h + 2, c->d_err, 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaEventRecord(c->ev_emb_drained, c->s_d2h));
   c->flags_h[L + 1] = 0;
   push_job(c, Job{Job::EMBED, -1, c->ev_emb_drained, L + 1});
+  // Without deferral the untouched rows' update follows the step's last check.
+  if (!(c->cfg.flags & MT_FLAG_DEFER_UPDATES)) push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, L + 1});
   CK(cudaMemcpyAsync(c->misc_h, c->d_loss, 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaEventRecord(c->ev_step_end, sc));
@@ -919,6 +1001,18 @@ size_t device_bytes(const Layout& y, int Tc) {
   return b + 4096;
 }
 
+// Tokens per LM-head chunk: at most ~4 GiB of fp32 logits + bf16 dz, a
+// multiple of 128 tokens; MT_LOGITS_CHUNK may ask for smaller chunks.
+int logits_chunk(const Shapes& s) {
+  int Tc = (int)std::min<int64_t>(s.T, ((int64_t)1 << 32) / ((int64_t)s.V * 6));
+  if (Tc < s.T) Tc = std::max(128, Tc / 128 * 128);
+  if (const char* e = getenv("MT_LOGITS_CHUNK")) {
+    const int want = atoi(e);
+    if (want >= 128 && want % 128 == 0 && want < Tc) Tc = want;
+  }
+  return Tc;
+}
+
 void free_all(mt_ctx* c) {
   if (!c) return;
   if (c->opt_thread.joinable()) {
@@ -988,13 +1082,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, cfg->device);
   if (major != 10 || minor != 0) return set_err(nullptr, MT_ERR_CUDA, "this library runs on sm_100 (B200) only");
 
-  // logits chunk: at most ~4 GiB of fp32 logits + bf16 dz, multiple of 128 tokens
-  int Tc = (int)std::min<int64_t>(s.T, ((int64_t)1 << 32) / ((int64_t)s.V * 6));
-  if (Tc < s.T) Tc = std::max(128, Tc / 128 * 128);
-  if (const char* e = getenv("MT_LOGITS_CHUNK")) {  // smaller chunks (multiple of 128 tokens), e.g. for tests
-    const int want = atoi(e);
-    if (want >= 128 && want % 128 == 0 && want < Tc) Tc = want;
-  }
+  const int Tc = logits_chunk(s);
   const size_t need = device_bytes(y, Tc);
   size_t free_b = 0, total_b = 0;
   if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaMemGetInfo failed");
@@ -1280,8 +1368,8 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
     c->layer_jobs_done = 0;
   }
   c->job_times.clear();
+  if (c->untouched_pending) start_untouched_prev(c);
   queue_deferred(c);  // the last step's deferred updates overlap this forward sweep
-  push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, s.L + 1});
   const double te0 = now_s();
   int r = enqueue_step(c, n_unique);
   c->enqueue_s = now_s() - te0;
@@ -1299,8 +1387,10 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   int32_t dev_err;
   memcpy(&dev_err, c->misc_h + 1, 4);
   if (dev_err != 0) {
-    char m[96];
-    snprintf(m, sizeof m, "kernel reported error %d (bounded wait expired)", dev_err);
+    char m[160];
+    snprintf(m, sizeof m,
+             "kernel reported error %d (bounded wait expired); the step's updates from that point on were skipped",
+             dev_err);
     return set_err(c, MT_ERR_DEVICE, m);
   }
   *loss_out = c->misc_h[0] / (float)T;
@@ -1328,6 +1418,7 @@ extern "C" int mt_layer_fwd_bwd(mt_ctx* c, int l, const float* x_in, const float
   c->timing_used = 0;
   c->timed.clear();
   c->err.clear();
+  CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));
   // the layer's streamed bf16 weights into slot 0, x_l into its boundary slot
   CK(cudaMemcpyAsync(c->wslot[0], c->bf_layers + (size_t)l * y.bf_layer, y.bf_layer * 2, cudaMemcpyHostToDevice, sc));
   CK(cudaMemcpyAsync(c->xb + (size_t)l * n, x_in, n * 4, cudaMemcpyHostToDevice, sc));
@@ -1363,6 +1454,7 @@ extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* label
   c->timed.clear();
   c->err.clear();
   const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
+  CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));
   CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, head_bf * 2, cudaMemcpyHostToDevice, sc));
   CK(cudaMemcpyAsync(c->xb + (size_t)s.L * n, x_L, n * 4, cudaMemcpyHostToDevice, sc));
   CK(cudaMemcpyAsync(c->d_lab, labels, (size_t)s.T * 4, cudaMemcpyHostToDevice, sc));
@@ -1491,6 +1583,28 @@ extern "C" int mt_get_timeline(mt_ctx* c, float* out, size_t cap_floats, size_t*
 extern "C" int mt_get_stream(mt_ctx* c, void** stream) {
   if (!c || !stream) return MT_ERR_ARG;
   *stream = c->s_comp;
+  return MT_OK;
+}
+
+extern "C" size_t mt_device_bytes(const mt_config* cfg) {
+  if (validate_config(cfg, nullptr) != MT_OK) return 0;
+  const Layout y = make_layout(*cfg);
+  return device_bytes(y, logits_chunk(y.sh));
+}
+
+namespace {
+void CUDART_CB host_sleep(void* ms) {
+  std::this_thread::sleep_for(std::chrono::milliseconds((int64_t)(intptr_t)ms));
+}
+}  // namespace
+
+extern "C" int mt_inject_host_stall(mt_ctx* c, int stream, int ms) {
+  if (!c) return MT_ERR_ARG;
+  if (stream < 0 || stream > 2 || ms < 0 || ms > 60000)
+    return set_err(c, MT_ERR_ARG, "stream must be 0, 1 or 2 and ms in [0, 60000]");
+  CK(cudaSetDevice(c->device));
+  cudaStream_t st = stream == 0 ? c->s_h2d : stream == 1 ? c->s_comp : c->s_d2h;
+  CK(cudaLaunchHostFunc(st, host_sleep, (void*)(intptr_t)ms));
   return MT_OK;
 }
 

@@ -64,6 +64,9 @@ struct Params {
   int epi;
   int* err;
   RopeDesc rope;
+  // Limit of the single-CTA kernel's main-loop waits (ns; 0: give up at the
+  // first incomplete poll). Waits that let the CTA exit safely use kWaitLimitNs.
+  uint64_t wait_ns;
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int& mb, int& nb) {
@@ -240,7 +243,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tile_coords(tile, num_m, num_n, mb, nb);
         const int m0 = mb * BM, n0 = nb * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (*abort_flag || !mbar_wait(&empty[stage], phase ^ 1)) {
+          if (*abort_flag || !mbar_wait(&empty[stage], phase ^ 1, p.wait_ns)) {
             record_error(p.err, DEV_TIMEOUT_PRODUCER);
             *abort_flag = 1;
             ok = false;
@@ -271,18 +274,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       if (ok) {
         // Producer tail: wait until the MMA has released every stage, so that no
-        // commit-arrive on this CTA's barriers is in flight when it exits.
-        for (int i = 0; i < C::STAGES; ++i) {
-          if (!mbar_wait(&empty[stage], phase ^ 1)) {
-            record_error(p.err, DEV_TIMEOUT_TEARDOWN);
-            break;
+        // commit-arrive on this CTA's barriers is in flight when it exits. If
+        // another role gives up meanwhile, the MMA may never release them:
+        // drain this CTA's copies instead (below).
+        for (int i = 0; i < C::STAGES && ok; ++i) {
+          const uint64_t t0 = globaltimer();
+          while (!mbar_wait(&empty[stage], phase ^ 1, 0)) {
+            if (*abort_flag) {
+              ok = false;
+              break;
+            }
+            if (globaltimer() - t0 > kWaitLimitNs) {
+              record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
           }
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-      } else {
+      }
+      if (!ok) {
         // Let every issued copy land before the CTA's shared memory goes away:
         // stage s was last filled by fill number s + STAGES * q (largest below
         // `issued`), in phase q mod 2.
@@ -313,7 +328,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool ok = true;
       bool issued = false;
       for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        if (*abort_flag || !mbar_wait(&tempty[acc], acc_phase ^ 1)) {
+        if (*abort_flag || !mbar_wait(&tempty[acc], acc_phase ^ 1, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -321,7 +336,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < num_kb; ++kb) {
           // A stalled producer shows up here as a wait that runs out.
-          if (!mbar_wait_u32(full0 + 8 * stage, phase)) {
+          if (!mbar_wait_u32(full0 + 8 * stage, phase, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -349,10 +364,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) {
         record_error(p.err, DEV_TIMEOUT_MMA);
         *abort_flag = 1;
-        if (issued) {
-          umma_commit(drain);
-          if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
-        }
+      }
+      // Every MMA issued here completes before tensor memory is freed, also
+      // when the epilogue gave up on an accumulator it will never read.
+      if (issued) {
+        umma_commit(drain);
+        if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
       }
     }
   } else {
@@ -362,7 +379,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       // warp-uniform outcome: the tcgen05.ld below is warp-collective
-      if (__any_sync(0xffffffffu, *abort_flag) || !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase))) {
+      if (__any_sync(0xffffffffu, *abort_flag) ||
+          !__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase, p.wait_ns))) {
         record_error(p.err, DEV_TIMEOUT_EPILOGUE);
         *abort_flag = 1;
         break;
@@ -587,10 +605,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) {
         record_error(p.err, DEV_TIMEOUT_MMA);
         *abort_flag = 1;
-        if (issued) {
-          umma_commit_pair(smem_u32(drain));
-          if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
-        }
+      }
+      if (issued) {
+        umma_commit_pair(smem_u32(drain));
+        if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
       }
     }
   } else {
@@ -692,6 +710,8 @@ bool make_tensor_map_2d_f32(CUtensorMap* m, const void* base, int64_t inner, int
 namespace {
 
 int g_num_sms = 0;
+// Main-loop wait limit of the single-CTA kernel for later launches (ns).
+uint64_t g_wait_ns = kWaitLimitNs;
 // Kernel family: 0 automatic, 1 single-CTA only, 2 CTA pairs wherever they fit
 // (MT_GEMM_VARIANT = auto | single | pair, read once; for A/B measurements).
 int g_variant = -1;
@@ -712,7 +732,7 @@ int launch(const GemmDesc& g, cudaStream_t st, int* err) {
   ok = ok && (B_MN ? make_tensor_map_2d_bf16(&tb, g.B, g.N, g.K, g.ldb, 64)
                     : make_tensor_map_2d_bf16(&tb, g.B, g.K, g.N, g.ldb, BN));
   if (!ok) return MT_ERR_ARG;
-  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err, g.rope};
+  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err, g.rope, g_wait_ns};
   const int tiles = ((g.M + BM - 1) / BM) * ((g.N + BN - 1) / BN);
   const int grid = tiles < g_num_sms ? tiles : g_num_sms;
   k_gemm_bf16<BN, A_MN, B_MN><<<grid, NUM_THREADS, C::SMEM, st>>>(ta, tb, p);
@@ -743,7 +763,9 @@ int launch_pair(const GemmDesc& g, int max_pairs, cudaStream_t st, int* err) {
   ok = ok && (B_MN ? make_tensor_map_2d_bf16(&tb, g.B, g.N, g.K, g.ldb, 64)
                    : make_tensor_map_2d_bf16(&tb, g.B, g.K, g.N, g.ldb, BN / 2));
   if (!ok) return MT_ERR_ARG;
-  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err, g.rope};
+  // The pair kernel keeps the fixed limit: its two producers would have to
+  // agree on the last stage filled before a shorter wait could unwind it.
+  Params p{g.M, g.N, g.K, g.C, g.ldc, g.R, g.ldr, g.epi, err, g.rope, kWaitLimitNs};
   const int tiles = ((g.M + C::TILE_M - 1) / C::TILE_M) * ((g.N + BN - 1) / BN);
   cudaLaunchConfig_t cfg = {};
   cfg.blockDim = dim3(NUM_THREADS, 1, 1);
@@ -838,6 +860,12 @@ int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* err) {
   const int tiles256 = ((g.M + BM - 1) / BM) * ((g.N + 255) / 256);
   if (g.N > 128 && tiles256 >= g_num_sms) return dispatch_major<256>(g, st, err);
   return dispatch_major<128>(g, st, err);
+}
+
+uint64_t gemm_wait_limit_ns(uint64_t ns) {
+  const uint64_t prev = g_wait_ns;
+  g_wait_ns = ns;
+  return prev;
 }
 
 int gemm_variant(int v) {

@@ -11,6 +11,15 @@ extern "C" int mt_k_gemm_bf16(const void* A, int64_t lda, int a_mn_major, const 
   return mt::gemm_bf16(g, static_cast<cudaStream_t>(stream), dev_err);
 }
 
+extern "C" int64_t mt_k_gemm_wait_limit_ns(int64_t ns) {
+  if (ns < 0) {
+    const uint64_t cur = mt::gemm_wait_limit_ns(0);
+    mt::gemm_wait_limit_ns(cur);
+    return (int64_t)cur;
+  }
+  return (int64_t)mt::gemm_wait_limit_ns((uint64_t)ns);
+}
+
 extern "C" int mt_k_gemm_variant(int variant) {
   if (variant < 0 || variant > 2) return MT_ERR_ARG;
   return mt::gemm_variant(variant);

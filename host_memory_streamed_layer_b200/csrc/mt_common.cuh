@@ -26,7 +26,11 @@ enum DeviceError : int {
   DEV_TIMEOUT_TEARDOWN = 4,
 };
 
-// Limit of any single wait on an mbarrier, in nanoseconds of %globaltimer.
+// Default limit of a single wait on an mbarrier, in nanoseconds of
+// %globaltimer. Waits that let a CTA exit safely (its own copies and MMAs in
+// flight) always use this limit; a kernel's main-loop waits may take a shorter
+// one from its parameters, where 0 means: give up at the first poll that finds
+// the phase incomplete.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -69,27 +73,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed. Returns false if
-// the wait exceeded kWaitLimitNs (the caller records an error and unwinds).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
-  const uint32_t addr = smem_u32(bar);
+// the wait exceeded limit_ns (the caller records an error and unwinds).
+__device__ __forceinline__ bool mbar_wait_u32(uint32_t addr, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(addr, parity)) return true;
+  if (limit_ns == 0) return false;
   const uint64_t t0 = globaltimer();
   while (true) {
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait(addr, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
 }
 
-// Same, for a barrier given by its shared-memory address.
-__device__ __forceinline__ bool mbar_wait_u32(uint32_t addr, uint32_t parity) {
-  if (mbar_try_wait(addr, parity)) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-    for (int i = 0; i < 256; ++i)
-      if (mbar_try_wait(addr, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
-  }
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
+  return mbar_wait_u32(smem_u32(bar), parity, limit_ns);
 }
 
 __device__ __forceinline__ void record_error(int* err, int code) {
@@ -260,14 +257,15 @@ __device__ __forceinline__ bool mbar_try_wait_acq_cluster(uint32_t addr, uint32_
 }
 // Bounded wait with cluster-scope acquire: for barriers that threads of the
 // peer CTA arrive on.
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t addr = smem_u32(bar);
   if (mbar_try_wait_acq_cluster(addr, parity)) return true;
+  if (limit_ns == 0) return false;
   const uint64_t t0 = globaltimer();
   while (true) {
     for (int i = 0; i < 256; ++i)
       if (mbar_try_wait_acq_cluster(addr, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    if (globaltimer() - t0 > limit_ns) return false;
   }
 }
 // 2-D tiled load into this CTA's shared memory whose completion is counted on

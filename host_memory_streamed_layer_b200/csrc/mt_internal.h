@@ -48,6 +48,8 @@ struct GemmDesc {
 int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
 // Kernel family for later GEMMs: 0 automatic, 1 single-CTA, 2 CTA pairs; returns the previous one.
 int gemm_variant(int v);
+// Main-loop wait limit (ns) of later single-CTA GEMM launches; returns the previous one.
+uint64_t gemm_wait_limit_ns(uint64_t ns);
 
 // 2-D bf16 TMA map: inner (contiguous) extent, outer extent, row pitch ld
 // (elements), box {64, box_outer}, 128-byte swizzle, zero fill out of bounds.

@@ -9,7 +9,10 @@ Times each launch with CUDA events on the launching stream after warm-up and
 prints achieved TFLOP/s (tensor-bound kernels) or GB/s of algorithmic bytes
 (memory-bound kernels). With --iters 1 --warmup 0 it launches exactly once,
 which is what an ncu capture of one launch wants. Shapes are those of the
-llama-1.3b workload (T = 8 x 2048 tokens, d 2048, FFN 5504, 16 heads).
+llama-1.3b workload (T = 8 x 2048 tokens, d 2048, FFN 5504, 16 heads); for
+the GEMMs, --workload NAME takes every GEMM shape of that workload's training
+step instead, and each result line carries the shape's launches per step
+(so per-shape ncu figures can be weighted into a per-launch step average).
 """
 from __future__ import annotations
 
@@ -29,6 +32,35 @@ GEMMS = {  # name: (M, N, K, form)
 }
 
 
+def step_gemms(sh):
+    """Every GEMM shape of one training step of workload sh, as the engine
+    launches them: name -> (M, N, K, form, launches per step). Forward per
+    layer; recompute (no down projection) for all layers but the last; the
+    backward's input- and weight-gradient products per layer; the LM head per
+    token chunk (chunks of at most ~4 GiB of fp32 logits + bf16 dz, multiples
+    of 128 tokens)."""
+    L, d, H, Hkv, Fh, Vh, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
+    hd = d // H
+    Tt, Nqkv, Hd = b * s, (H + 2 * Hkv) * hd, H * hd
+    tc = min(Tt, (1 << 32) // (Vh * 6))
+    if tc < Tt:
+        tc = max(128, tc // 128 * 128)
+    chunks = [min(tc, Tt - t0) for t0 in range(0, Tt, tc)]
+    g = {
+        "qkv_fwd": (Tt, Nqkv, d, "fwd", 2 * L - 1), "o_fwd": (Tt, d, Hd, "fwd", 2 * L - 1),
+        "gu_fwd": (Tt, 2 * Fh, d, "fwd", 2 * L - 1), "down_fwd": (Tt, d, Fh, "fwd", L),
+        "down_dw": (d, Fh, Tt, "dw", L), "down_dx": (Tt, Fh, d, "dx", L), "gu_dw": (2 * Fh, d, Tt, "dw", L),
+        "gu_dx": (Tt, d, 2 * Fh, "dx", L), "o_dw": (d, Hd, Tt, "dw", L), "o_dx": (Tt, Hd, d, "dx", L),
+        "qkv_dw": (Nqkv, d, Tt, "dw", L), "qkv_dx": (Tt, d, Nqkv, "dx", L),
+    }
+    for c in sorted(set(chunks)):
+        n = chunks.count(c)
+        g[f"head_fwd_{c}"] = (c, Vh, d, "fwd32", n)
+        g[f"head_dw_{c}"] = (Vh, d, c, "dw", n)
+        g[f"head_dx_{c}"] = (c, d, Vh, "dx32", n)
+    return g
+
+
 def timed(fn, iters, warmup):
     for _ in range(warmup):
         fn()
@@ -44,25 +76,36 @@ def timed(fn, iters, warmup):
     return e0.elapsed_time(e1) / iters / 1e3
 
 
-def bench_gemm(names, iters, warmup):
+def bench_gemm(names, iters, warmup, table=None):
+    """Times each named GEMM; `table` maps name -> (M, N, K, form[, launches
+    per step]) (default: the 1.3B shapes). Forms: fwd (bf16 out), fwd32 (fp32
+    out, the LM head's logits), dx (B MN-major; bf16 out), dx32 (fp32 out),
+    dw (both operands MN-major, fp32 out)."""
+    table = table or GEMMS
     st = torch.cuda.current_stream().cuda_stream
     out = []
     for name in names:
-        M, N, K, form = GEMMS[name]
+        M, N, K, form = table[name][:4]
         A = torch.randn(M * K, device="cuda").to(torch.bfloat16)
         Bm = torch.randn(N * K, device="cuda").to(torch.bfloat16)
-        C = torch.empty(M * N, device="cuda", dtype=torch.float32 if form == "dw" else torch.bfloat16)
-        if form == "fwd":
+        f32 = form in ("dw", "fwd32", "dx32")
+        C = torch.empty(M * N, device="cuda", dtype=torch.float32 if f32 else torch.bfloat16)
+        if form.startswith("fwd"):
             a = (A.data_ptr(), K, 0, Bm.data_ptr(), K, 0)
-        elif form == "dx":
+        elif form.startswith("dx"):
             a = (A.data_ptr(), K, 0, Bm.data_ptr(), N, 1)
         else:
             a = (A.data_ptr(), M, 1, Bm.data_ptr(), N, 1)
-        kind = mt.GEMM_OUT_F32 if form == "dw" else mt.GEMM_OUT_BF16
+        kind = mt.GEMM_OUT_F32 if f32 else mt.GEMM_OUT_BF16
         sec = timed(lambda: mt.mt_k_gemm_bf16(*a, C.data_ptr(), N, kind, 0, 0, M, N, K, st, 0), iters, warmup)
         fl = 2.0 * M * N * K
-        out.append({"kernel": "gemm", "shape": name, "M": M, "N": N, "K": K, "us": sec * 1e6,
-                    "tflops": fl / sec / 1e12 if sec else None})
+        r = {"kernel": "gemm", "shape": name, "M": M, "N": N, "K": K, "us": sec * 1e6,
+             "tflops": fl / sec / 1e12 if sec else None}
+        if len(table[name]) > 4:
+            r["launches_per_step"] = table[name][4]
+        out.append(r)
+        del A, Bm, C
+        torch.cuda.empty_cache()
     return out
 
 
@@ -165,10 +208,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--impl", default="tc", choices=["tc", "mma"])
+    ap.add_argument("--workload", default=None, help="GEMMs: every shape of this workload's training step")
     a = ap.parse_args()
     if a.kernel == "gemm":
-        names = list(GEMMS) if a.shape == "all" else a.shape.split(",")
-        res = bench_gemm(names, a.iters, a.warmup)
+        table = None
+        if a.workload:
+            import synth
+            table = step_gemms(synth.WORKLOADS[a.workload])
+        names = list(table or GEMMS) if a.shape == "all" else a.shape.split(",")
+        res = bench_gemm(names, a.iters, a.warmup, table)
     elif a.kernel == "attn":
         res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl)
     elif a.kernel == "elementwise":

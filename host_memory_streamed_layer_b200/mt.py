@@ -64,6 +64,17 @@ def mt_k_gemm_variant(variant: int) -> int:
     return rc
 
 
+_sig("mt_k_gemm_wait_limit_ns", c_i64, c_i64)
+DEV_TIMEOUT_PRODUCER, DEV_TIMEOUT_MMA, DEV_TIMEOUT_EPILOGUE, DEV_TIMEOUT_TEARDOWN = 1, 2, 3, 4
+GEMM_WAIT_DEFAULT_NS = 1_000_000_000
+
+
+def mt_k_gemm_wait_limit_ns(ns: int) -> int:
+    """Sets the main-loop wait limit of later single-CTA GEMM launches (ns < 0
+    only queries); returns the previous limit."""
+    return lib.mt_k_gemm_wait_limit_ns(ns)
+
+
 c_float, c_f = ctypes.c_float, ctypes.c_float
 
 _sig("mt_k_rmsnorm_fwd", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int, c_float, c_void_p)
@@ -220,6 +231,8 @@ _sig("mt_host_optimizer_gbs", ctypes.c_double, c_size_t, c_int)
 _sig("mt_get_opt_state", c_int, c_void_p, c_void_p, c_void_p, c_size_t, ctypes.POINTER(ctypes.c_int64))
 _sig("mt_set_state", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, ctypes.c_int64)
 _sig("mt_last_error", ctypes.c_char_p, c_void_p)
+_sig("mt_device_bytes", c_size_t, _cfgp)
+_sig("mt_inject_host_stall", c_int, c_void_p, c_int, c_int)
 _sig("mt_k_adamw_host", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_float, c_float,
      c_float, c_float, c_float, c_int)
 
@@ -321,6 +334,16 @@ def mt_get_stream(ctx: int) -> int:
     st = c_void_p()
     _check(lib.mt_get_stream(ctx, ctypes.byref(st)), "mt_get_stream", ctx)
     return st.value or 0
+
+
+def mt_device_bytes(cfg: mt_config) -> int:
+    return lib.mt_device_bytes(ctypes.byref(cfg))
+
+
+def mt_inject_host_stall(ctx: int, stream: int, ms: int):
+    """Test aid: a host function sleeping ms milliseconds on one of the
+    context's streams (0 prefetch, 1 compute, 2 offload)."""
+    return _check(lib.mt_inject_host_stall(ctx, stream, ms), "mt_inject_host_stall", ctx)
 
 
 def mt_destroy(ctx: int):

@@ -165,6 +165,16 @@ int mt_tensor_offset(const mt_config* cfg, int layer, int tensor_id, size_t* off
  * with MT_FLAG_DEFER_UPDATES too, MT_DEFER_LAYERS more layer slots). */
 size_t mt_host_state_bytes(const mt_config* cfg);
 
+/* Device bytes mt_create allocates for cfg, in one allocation, 0 for a bad
+ * cfg: two bf16 layer-weight slots and two fp32 layer-gradient slots (the
+ * double-buffered layer pair of saify.me, "The memory-centric design":
+ * persistent GPU state stays at about one layer's footprint), the LM head's
+ * weights and gradients, the boundary activations x_0..x_L (fp32 [b*s, d]
+ * each, the only per-layer state kept: intelligentliving.co, "Checkpointing,
+ * Manual Gradients, and CPU-Side Optimizer Steps") and one layer's workspace.
+ * Only the boundary activations grow with L. No GPU needed. */
+size_t mt_device_bytes(const mt_config* cfg);
+
 /* Creates a context on cfg->device. host_param_arena: the caller's fp32
  * master weights in the layout of mt_arena_bytes, at least arena_bytes long and
  * 256-byte aligned; the library updates it in place every step and keeps the
@@ -179,11 +189,17 @@ int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes,
 /* One training step: tokens and labels are host int32 arrays of b*s ids in
  * [0, V), sequence-major. Runs forward, loss, backward and the host AdamW
  * update (bias correction from step 1), and writes the mean next-token
- * cross-entropy (computed before the update) to *loss_out. Returns
- * MT_ERR_NONFINITE if a gradient was not finite: the updates of the tensors
- * not yet updated are skipped and the arena is partly updated. With
- * MT_FLAG_DEFER_UPDATES some of this step's updates are still pending when it
- * returns (see the flag). */
+ * cross-entropy (computed before the update) to *loss_out. Each tensor's
+ * gradients are checked on the GPU before its host update (intelligentliving.co,
+ * "Checkpointing, Manual Gradients, and CPU-Side Optimizer Steps": updates run
+ * on the CPU as the gradients arrive). Returns MT_ERR_NONFINITE if a gradient
+ * was not finite, and MT_ERR_DEVICE if a kernel of the step reported a bounded
+ * wait that ran out (its outputs are then undefined): in both cases the
+ * updates of the tensors not yet updated are skipped and the arena is partly
+ * updated; the embedding rows no token of the step touched are updated only
+ * after every check of the step has passed. The next step starts afresh (the
+ * device error word is cleared at its start). With MT_FLAG_DEFER_UPDATES some
+ * of this step's updates are still pending when it returns (see the flag). */
 int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, float* loss_out);
 
 /* Runs the updates that MT_FLAG_DEFER_UPDATES left pending, and returns when
@@ -241,6 +257,18 @@ int mt_get_opt_state(mt_ctx* ctx, float* m_dst, float* v_dst, size_t bytes_each,
 int mt_set_state(mt_ctx* ctx, const float* params, const float* m, const float* v, size_t bytes_each,
                  int64_t step);
 
+/* Fault injection for tests of the host-side waits: enqueues on the
+ * context's stream `stream` (0 weight prefetch, 1 compute, 2 gradient
+ * offload) a host function that sleeps `ms` milliseconds (0..60000), so that
+ * the work queued after it starts late. The GPU itself is untouched: nothing
+ * faults, traps or spins on it. With MT_WAIT_LIMIT_S below the stall, the
+ * next mt_train_step returns MT_ERR_TIMEOUT with its remaining updates
+ * skipped, and the context can still be used or destroyed (mt_destroy waits
+ * for the stall to end). The pages give no failure model beyond fewer
+ * crashes and out-of-memory errors (intelligentliving.co, "Leveraging
+ * Double-Buffered Pipelining and Stateless Layer Templates"). */
+int mt_inject_host_stall(mt_ctx* ctx, int stream, int ms);
+
 /* Counters of the last step. */
 int mt_get_stats(mt_ctx* ctx, mt_stats* out);
 
@@ -255,10 +283,12 @@ int mt_get_stats(mt_ctx* ctx, mt_stats* out);
  *   forward end, head end, backward end, step end;
  *   per host optimizer job (execution order): kind (0 layer, 1 LM head,
  *     2 touched embedding rows, 3 untouched embedding rows, 4 LM head and
- *     5 layer deferred from the previous step by MT_FLAG_DEFER_UPDATES; with
- *     the flag, kinds 0 and 1 of the deferred tensors only check their
- *     gradients), layer (-1 for the others), gradients available, update
- *     finished.
+ *     5 layer deferred from the previous step by MT_FLAG_DEFER_UPDATES,
+ *     6 the previous step's untouched embedding rows deferred by the flag,
+ *     7 those of them this step's batch gathers, updated before the step's
+ *     GPU work is enqueued; with the flag, kinds 0 and 1 of the deferred
+ *     tensors only check their gradients), layer (-1 for the others),
+ *     gradients available, update finished.
  * Device times are ms from the step's start on the compute stream (CUDA
  * events); host job times are ms of host clock from the mt_train_step call,
  * a separate clock whose origin is within a few tens of microseconds of it. */

@@ -163,6 +163,27 @@ int mt_k_gemm_bf16_rope(const void* A, int64_t lda, const void* B, int64_t ldb, 
                         int K, int rope_cols, int hd, int s, const float* cos_tab, const float* sin_tab, void* stream,
                         int32_t* dev_err);
 
+/* Codes a kernel writes into dev_err when one of its bounded waits runs out
+ * (the first code recorded wins). */
+#define MT_DEV_TIMEOUT_PRODUCER 1 /* the copy producer waited too long for a free stage */
+#define MT_DEV_TIMEOUT_MMA 2      /* the MMA issuer waited too long for operands or an accumulator */
+#define MT_DEV_TIMEOUT_EPILOGUE 3 /* the epilogue waited too long for a finished accumulator */
+#define MT_DEV_TIMEOUT_TEARDOWN 4 /* a wait for the CTA's own copies or MMAs before exit ran out */
+
+/* Limit, in nanoseconds, of each main-loop wait of the single-CTA GEMM kernel
+ * for later launches in this process (mt_k_gemm_bf16, mt_k_gemm_bf16_rope and
+ * the engine's GEMMs alike); returns the previous limit. ns < 0 only queries.
+ * Default 1e9 (1 s). With 0 a wait gives up at its first poll that finds the
+ * stage or accumulator not ready, so a test can make a kernel take its
+ * bounded-wait exit without any fault: the kernel records an
+ * MT_DEV_TIMEOUT_* code in dev_err, lets its own copies and MMAs finish,
+ * frees its tensor memory and returns; outputs are then undefined, and the
+ * context stays usable. The waits that let a CTA exit safely keep 1 s, and so
+ * does every wait of the CTA-pair kernel (used for problems with at least one
+ * 256-row tile per SM pair). Host-side only; not thread-safe against
+ * concurrent GEMM launches. */
+int64_t mt_k_gemm_wait_limit_ns(int64_t ns);
+
 /* Selects the GEMM kernel family for later calls in this process: 0 automatic
  * (the default, or MT_GEMM_VARIANT=auto), 1 single-CTA tiles only (=single),
  * 2 CTA-pair tiles (tcgen05 cta_group::2, 256-row tiles) wherever a problem

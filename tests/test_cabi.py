@@ -314,3 +314,22 @@ def test_arena_pack_round_trips_through_the_oracle_layout(shape):
     bad[k0] = np.zeros(np.asarray(bad[k0]).size + 1, dtype=np.float32)
     with pytest.raises(ValueError):
         arena.pack(cfg, bad)
+
+
+def test_device_bytes_grow_only_by_the_boundary_activations():
+    """mt_device_bytes: two bf16 weight slots, two fp32 gradient slots, the head,
+    one workspace and the L+1 boundary activations; one more layer adds exactly
+    one fp32 [b*s, d] boundary activation and nothing else (the persistent
+    state of saify.me, "The memory-centric design")."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    for base in (dict(d=1024, H=8, Hkv=8, F=2752, V=4096, b=4, s=1024),
+                 dict(d=5120, H=40, Hkv=8, F=13824, V=152064, b=2, s=4096)):
+        T, d = base["b"] * base["s"], base["d"]
+        sizes = [mt.mt_device_bytes(arena.config(dict(base, L=L))) for L in (1, 2, 5, 40)]
+        for (La, a), (Lb, b) in zip(zip((1, 2, 5, 40), sizes), zip((2, 5, 40), sizes[1:])):
+            assert b - a == (Lb - La) * T * d * 4
+        cfg = arena.config(dict(base, L=2))
+        P_layer = sum(mt.mt_tensor_offset(cfg, 0, t)[1] for t in range(9))
+        assert sizes[1] > 2 * 2 * P_layer + 2 * 4 * P_layer + 3 * T * d * 4
+    bad = arena.config(dict(L=2, d=100, H=2, Hkv=2, F=64, V=64, b=1, s=8))
+    assert mt.mt_device_bytes(bad) == 0

@@ -215,6 +215,66 @@ def test_checkpoint_resume_continues_the_trajectory():
     assert rel(P2b, P2) <= 1e-5
 
 
+def test_resume_follows_the_oracle_from_the_restored_state():
+    """Checkpoint after step 1 (master, moments, step counter), restore into a
+    fresh context and run step 2 there: the loss and gradients are the
+    oracle's on the restored master, the update is AdamW at t = 2 from the
+    restored moments (relative 1e-6 on the engine's own gradients), and the
+    updated master, m and v are within the end-to-end bars of the oracle's
+    own step-2 update from the same restored state."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    shape = SHAPES["gqa_ragged"]
+    c = oracle.OracleConfig(**shape)
+    cfg = arena.config(shape)
+    cfg.host_threads = 4
+    A = arena.pack(cfg, synth.init_weights(shape, 0))
+    n = A.size
+    toks = [synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, k) for k in range(2)]
+    ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+    try:
+        mt.mt_train_step(ctx, toks[0][0].ctypes.data, toks[0][1].ctypes.data)
+        P1 = A.copy()
+        M1, V1 = np.empty(n, np.float32), np.empty(n, np.float32)
+        step = mt.mt_get_opt_state(ctx, M1.ctypes.data, V1.ctypes.data, M1.nbytes)
+    finally:
+        mt.mt_destroy(ctx)
+    assert step == 1
+    B = arena.pack(cfg, synth.init_weights(shape, 7))
+    ctx = mt.mt_create(cfg, B.ctypes.data, B.nbytes)
+    try:
+        mt.mt_set_state(ctx, P1.ctypes.data, M1.ctypes.data, V1.ctypes.data, P1.nbytes, step)
+        loss2 = mt.mt_train_step(ctx, toks[1][0].ctypes.data, toks[1][1].ctypes.data)
+        G2 = np.empty_like(B)
+        mt.mt_get_grads(ctx, G2.ctypes.data, G2.nbytes)
+        M2, V2 = np.empty(n, np.float32), np.empty(n, np.float32)
+        assert mt.mt_get_opt_state(ctx, M2.ctypes.data, V2.ctypes.data, M2.nbytes) == 2
+        P2 = B.copy()
+    finally:
+        mt.mt_destroy(ctx)
+    Wb = {k: oracle.bf16_round(w.astype(np.float32)) for k, w in oracle.unpack_arena(P1, c).items()}
+    rloss, RG = oracle.train_step_grads(Wb, toks[1][0], toks[1][1], c)
+    assert abs(loss2 - rloss) <= 1e-2
+    G = oracle.unpack_arena(G2, c)
+    assert max(rel(G[k], RG[k]) for k in RG) <= 2e-2
+    # the host update from the restored state, on the engine's own gradients
+    p, m, v = oracle.adamw_update(P1.astype(np.float64), G2.astype(np.float64), M1.astype(np.float64),
+                                  V1.astype(np.float64), 2, **HYP)
+    for got, want in ((P2, p), (M2, m), (V2, v)):
+        assert rel(got.astype(np.float64), want) <= 1e-6
+    # end to end against the oracle's step-2 update from the same restored state
+    Pu, Mu, Vu = oracle.unpack_arena(P1, c), oracle.unpack_arena(M1, c), oracle.unpack_arena(V1, c)
+    P2d, M2d, V2d = oracle.unpack_arena(P2, c), oracle.unpack_arena(M2, c), oracle.unpack_arena(V2, c)
+    num = den = 0.0
+    for k in RG:
+        po, mo, vo = oracle.adamw_update(Pu[k].astype(np.float64), RG[k], Mu[k].astype(np.float64),
+                                         Vu[k].astype(np.float64), 2, **HYP)
+        num += float(np.sum((P2d[k] - po) ** 2))
+        den += float(np.sum(po ** 2))
+        assert rel(M2d[k].astype(np.float64), mo) <= 2e-2, k
+        assert rel(V2d[k].astype(np.float64), vo) <= 4e-2, k
+    assert math.sqrt(num / den) <= 5e-3, math.sqrt(num / den)
+
+
 def test_gradient_ring_matches_full_arena_and_oracle():
     """MT_FLAG_GRAD_RING: layer gradients pass through MT_GRAD_RING_SLOTS host
     slots (5 layers > slots, so offloads wait for released slots) and the
@@ -392,9 +452,10 @@ def test_deferred_updates_follow_the_undeferred_trajectory(monkeypatch):
     for got, want in ((dfr["P"], p), (dfr["M"], m), (dfr["V"], v)):
         assert rel(got.astype(np.float64), want) <= 1e-6
     # timeline of the last step: one check job per layer and for the head, the
-    # two embedding jobs, and the previous step's deferred head and layers
+    # touched embedding rows, and the previous step's deferred head, layers and
+    # untouched embedding rows (those this step gathers first, then the rest)
     jobs = dfr["tl"]["jobs"]
-    assert sorted(j["kind"] for j in jobs) == [0] * L + [1, 2, 3, 4] + [5] * nd
+    assert sorted(j["kind"] for j in jobs) == [0] * L + [1, 2, 4, 6, 7] + [5] * nd
     assert sorted(j["layer"] for j in jobs if j["kind"] == 5) == list(range(L - nd, L))
     loads = dfr["tl"]["loads"]
     for j in jobs:
