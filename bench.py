@@ -606,6 +606,8 @@ def main():
 
     link = link_bandwidth(torch, dev) if rank == 0 else None
     host_bw = host_optimizer_bandwidth(mt, cfg.host_threads) if rank == 0 else None
+    # independent host-DRAM ceiling: STREAM triad (12 B/element, non-temporal stores)
+    triad = mt.mt_host_triad_gbs(1 << 28, cfg.host_threads) if rank == 0 else None
     ctx = mt.mt_create(cfg)
     try:
         n_e2e = max(3, (args.steps + 1) // 2)
@@ -716,6 +718,9 @@ def main():
                               "host_dram_model": {"ms": t_model * 1e3, "ratio": t_model / (t_dev / K),
                                                   "bytes_fwd": dram_fwd, "bytes_bwd": dram_bwd},
                               "host_optimizer_gbs_measured": host_bw,
+                              "host_triad_gbs": triad,
+                              "host_adamw_frac_of_triad": (mean("adamw_bytes") / max(mean("adamw_ms"), 1e-9) / 1e6
+                                                           / triad) if triad else None,
                               "compute_ms": t_compute * 1e3, "h2d_ms": t_h2d * 1e3, "d2h_ms": t_d2h * 1e3,
                               "link_measured": link, "h2d_bytes": h2d_b, "d2h_bytes": d2h_b,
                               "attention_tflops": a_fl / (a_ms / 1e3) / 1e12 if a_ms > 0 else None,
@@ -727,6 +732,10 @@ def main():
                               "host_step_ms": mean("host_step_ms"), "adamw_first_ms": mean("adamw_first_ms"),
                               "adamw_last_ms": mean("adamw_last_ms"), "enqueue_ms": mean("enqueue_ms")},
             "loss": losses[-1],
+            "parity": {"loss_abs": 1e-2, "grad_rel_l2": 2e-2, "updated_param_rel_l2": {
+                "target": 1e-3, "met": False, "tested": 5e-3,
+                "why": "the first Adam step is ~lr*sign(g); bf16 operands put its floor at ~2.5e-3 and every bf16 "
+                       "rounding point alone (stored activations, stored gradients, attention P/dS) exceeds 1e-3"}},
             "clocks": clk,
             "e2e": {"value": weak_value(T, world, n_e2e, t_e2e), "unit": UNIT, "h2d_bytes_per_step": 2 * T * 4,
                     "d2h_bytes_per_step": 4, "steps": n_e2e,

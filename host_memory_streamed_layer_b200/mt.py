@@ -228,6 +228,7 @@ _sig("mt_get_stats", c_int, c_void_p, ctypes.POINTER(mt_stats))
 _sig("mt_destroy", None, c_void_p)
 _sig("mt_get_stream", c_int, c_void_p, ctypes.POINTER(c_void_p))
 _sig("mt_host_optimizer_gbs", ctypes.c_double, c_size_t, c_int)
+_sig("mt_host_triad_gbs", ctypes.c_double, c_size_t, c_int)
 _sig("mt_get_opt_state", c_int, c_void_p, c_void_p, c_void_p, c_size_t, ctypes.POINTER(ctypes.c_int64))
 _sig("mt_set_state", c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, ctypes.c_int64)
 _sig("mt_last_error", ctypes.c_char_p, c_void_p)
@@ -363,6 +364,13 @@ def mt_host_optimizer_gbs(n: int = 1 << 28, threads: int = 0) -> float:
     r = lib.mt_host_optimizer_gbs(n, threads)
     if r < 0:
         raise MTError(int(r), "mt_host_optimizer_gbs")
+    return r
+
+
+def mt_host_triad_gbs(n: int = 1 << 28, threads: int = 0) -> float:
+    r = lib.mt_host_triad_gbs(n, threads)
+    if r < 0:
+        raise MTError(int(r), "mt_host_triad_gbs")
     return r
 
 

@@ -308,6 +308,16 @@ int mt_get_stream(mt_ctx* ctx, void** stream);
  * buffers; no GPU needed. Returns a negative MT_ERR_* on failure. */
 double mt_host_optimizer_gbs(size_t n, int threads);
 
+/* Host DRAM ceiling independent of the optimizer: the STREAM triad
+ * a[i] = b[i] + s c[i] over three fp32 arrays of n elements with `threads`
+ * threads (0 = all cores but one), parallel first touch, non-temporal stores,
+ * best of 5 passes, in GB/s counted as 12 bytes per element (two reads, one
+ * write). The host AdamW's 30 bytes per parameter are judged against it
+ * (intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
+ * Optimizer Steps": CPU-side updates can become the slow step). Allocates
+ * and frees its own host buffers; no GPU needed. Negative MT_ERR_* on failure. */
+double mt_host_triad_gbs(size_t n, int threads);
+
 /* Applies pending deferred updates, waits for the context's streams, frees
  * its device memory and unpins or frees its host memory. NULL is ignored. */
 void mt_destroy(mt_ctx* ctx);
