@@ -144,21 +144,31 @@ typedef struct mt_stats {
 
 /* Fills *cfg with the defaults (struct_size set, hyper-parameters of the
  * workloads: eps 1e-5, RoPE base 10000, lr 1e-3, betas (0.9, 0.95), eps 1e-8,
- * wd 0.1). Shapes are left zero. */
+ * wd 0.1). Shapes are left zero. The pages fix none of these values: AdamW is
+ * the optimizer of the paper's references (mlsanity.com index, "Builds on":
+ * Adam), the rest are the usual Llama-style settings. */
 int mt_config_default(mt_config* cfg);
 
-/* Bytes of the fp32 master arena for cfg: the embedding [V,d]; per layer the
+/* Bytes of the fp32 master arena for cfg, the parameters that live in host
+ * memory (MegaTrain abstract: parameters and optimizer states are stored in
+ * host memory; intelligentliving.co, "Implementing Host Memory Offloading
+ * for Persistent Model State"): the embedding [V,d]; per layer the
  * attention-norm gain [d], Wq [H*hd,d], Wk [Hkv*hd,d], Wv [Hkv*hd,d],
  * Wo [d,H*hd], MLP-norm gain [d], Wgate [F,d], Wup [F,d], Wdown [d,F]; then the
  * final-norm gain [d] and the untied LM head [V,d]. Weights are row-major
  * [out, in]; every tensor starts on a 256-byte boundary. 0 for a bad cfg. */
 size_t mt_arena_bytes(const mt_config* cfg);
 
-/* Offset (in floats) and element count of one tensor of the arena. */
+/* Offset (in floats) and element count of one tensor of the arena (the
+ * layout of mt_arena_bytes; tensor_id MT_T_*, layer -1 for the embedding,
+ * final norm and LM head). MT_ERR_ARG for an unknown tensor or layer. */
 int mt_tensor_offset(const mt_config* cfg, int layer, int tensor_id, size_t* offset_floats, size_t* numel);
 
-/* Host bytes the context holds besides the caller's arena: two fp32 Adam
- * moments (8 B/param), the bf16 streaming copy (2 B/param) and the staging of
+/* Host bytes the context holds besides the caller's arena (the pages budget
+ * ~12 GB of host memory per 1B parameters for the full-precision state:
+ * saify.me, "Who this is actually for"; intelligentliving.co, FAQ, minimum
+ * RAM): two fp32 Adam moments (8 B/param, with the caller's 4 B/param master
+ * the 12), the bf16 streaming copy (2 B/param) and the staging of
  * the embedding-gradient rows, plus the fp32 gradients: the whole gradient
  * arena (4 B/param), or with MT_FLAG_GRAD_RING in cfg->flags the ring of
  * MT_GRAD_RING_SLOTS layer slots and the final-norm + LM-head gradient (and,
@@ -175,7 +185,10 @@ size_t mt_host_state_bytes(const mt_config* cfg);
  * Only the boundary activations grow with L. No GPU needed. */
 size_t mt_device_bytes(const mt_config* cfg);
 
-/* Creates a context on cfg->device. host_param_arena: the caller's fp32
+/* Creates a context on cfg->device: the host-resident state and the small,
+ * fixed device footprint of MegaTrain's memory-centric design (MegaTrain
+ * abstract: GPUs are transient compute engines; saify.me, "The memory-centric
+ * design"). host_param_arena: the caller's fp32
  * master weights in the layout of mt_arena_bytes, at least arena_bytes long and
  * 256-byte aligned; the library updates it in place every step and keeps the
  * pointer for the context's lifetime. Only host threads touch it (the GPU reads
@@ -204,12 +217,17 @@ int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, flo
 
 /* Runs the updates that MT_FLAG_DEFER_UPDATES left pending, and returns when
  * the arena, the moments and the bf16 copies hold the state after the last
- * step. A no-op without pending updates. */
+ * step. A no-op without pending updates. (The host optimizer step of
+ * intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
+ * Optimizer Steps", moved in time, not changed.) */
 int mt_flush(mt_ctx* ctx);
 
 /* Copies the fp32 gradients of the last step (taken before the update), in the
- * arena layout, to dst (bytes >= mt_arena_bytes). MT_ERR_CONFIG for a context
- * created with MT_FLAG_GRAD_RING, which keeps no gradient arena. */
+ * arena layout, to dst (bytes >= mt_arena_bytes): the gradients each layer
+ * pushed back to host memory (MegaTrain abstract: per layer, gradients stream
+ * out; intelligentliving.co, "Quantifying Host Memory Requirements...": the
+ * stream immediately pushes gradients back to the host). MT_ERR_CONFIG for a
+ * context created with MT_FLAG_GRAD_RING, which keeps no gradient arena. */
 int mt_get_grads(mt_ctx* ctx, float* dst, size_t bytes);
 
 /* One decoder layer through the engine's own stateless layer template, with
@@ -242,7 +260,11 @@ int mt_layer_fwd_bwd(mt_ctx* ctx, int layer, const float* x_in, const float* dx_
 int mt_head_fwd_bwd(mt_ctx* ctx, const float* x_L, const int32_t* labels, float* loss_out, float* dx_L,
                     float* grads, size_t grads_bytes);
 
-/* Copies the current fp32 master weights (after the last update) to dst. */
+/* Copies the current fp32 master weights (after the last update) to dst
+ * (bytes >= mt_arena_bytes), applying pending deferred updates first. The
+ * master lives in host memory and is the state the host AdamW updates
+ * (intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
+ * Optimizer Steps": FP32 master weights and optimizer moments live in RAM). */
 int mt_get_params(mt_ctx* ctx, float* dst, size_t bytes);
 
 /* Checkpoint: copies the fp32 Adam moments m and v (arena layout, each at
@@ -269,7 +291,10 @@ int mt_set_state(mt_ctx* ctx, const float* params, const float* m, const float* 
  * Double-Buffered Pipelining and Stateless Layer Templates"). */
 int mt_inject_host_stall(mt_ctx* ctx, int stream, int ms);
 
-/* Counters of the last step. */
+/* Counters of the last step: the copy/compute overlap and optimizer-latency
+ * figures that the pages ask a profile of this method to report
+ * (intelligentliving.co, "Limitations of Current Throughput Metrics...":
+ * CPU-to-GPU transfer overlap and optimizer update latencies). */
 int mt_get_stats(mt_ctx* ctx, mt_stats* out);
 
 /* Timeline of the last step, for seeing the copy/compute overlap of the
@@ -294,13 +319,17 @@ int mt_get_stats(mt_ctx* ctx, mt_stats* out);
  * a separate clock whose origin is within a few tens of microseconds of it. */
 int mt_get_timeline(mt_ctx* ctx, float* out, size_t cap_floats, size_t* n_floats);
 
-/* The context's compute stream (a cudaStream_t) in *stream, so a caller can
+/* The context's compute stream (one of the several CUDA streams of the
+ * pipelined engine, saify.me "Pipelined double buffering") as a cudaStream_t
+ * in *stream, so a caller can
  * order or time its own work against the step (for example record CUDA events
  * around a sequence of mt_train_step calls). The stream stays owned by the
  * context. */
 int mt_get_stream(mt_ctx* ctx, void** stream);
 
-/* Host-memory ceiling of the optimizer: runs the library's host AdamW (the
+/* Host-memory ceiling of the optimizer (intelligentliving.co, "Checkpointing,
+ * Manual Gradients, and CPU-Side Optimizer Steps": CPU-side updates can
+ * become the slow step): runs the library's host AdamW (the
  * same routine, worker pool and chunking the engine uses) over four fp32
  * arrays of n elements with `threads` threads (0 = all cores but one), best
  * of 3 passes, and returns GB/s counted as 30 bytes per element (read p, g,
@@ -319,11 +348,17 @@ double mt_host_optimizer_gbs(size_t n, int threads);
 double mt_host_triad_gbs(size_t n, int threads);
 
 /* Applies pending deferred updates, waits for the context's streams, frees
- * its device memory and unpins or frees its host memory. NULL is ignored. */
+ * its device memory and unpins or frees its host memory. NULL is ignored.
+ * The caller's arena then holds the final master weights (MegaTrain abstract:
+ * the host holds the parameters; the GPU kept only transient state). */
 void mt_destroy(mt_ctx* ctx);
 
 /* Message of the last error of ctx (or of the last failed mt_create when ctx
- * is NULL). Valid until the next call on the same context. */
+ * is NULL). Valid until the next call on the same context. The pages describe
+ * no error interface; this is the library's own (every call reports instead
+ * of aborting, so that out-of-memory and stalls surface as codes:
+ * intelligentliving.co, "Leveraging Double-Buffered Pipelining and Stateless
+ * Layer Templates", on avoiding unpredictable OOM errors). */
 const char* mt_last_error(const mt_ctx* ctx);
 
 #ifdef __cplusplus
