@@ -46,7 +46,7 @@ UNIT = "tokens/s"
 # --iters 1 --warmup 0`, at most a few GB on the device), never from a
 # full-size training run. Workloads without a capture report null, and so does
 # a workload whose GEMM kernels changed after its capture.
-GEMM_TRAFFIC_PER_LAUNCH = {}
+GEMM_TRAFFIC_PER_LAUNCH = {"gqa-14b": 1257.6e6, "llama-1.3b": 497.3e6}
 
 
 def parse():
@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--grads", default="ring", choices=["ring", "arena"],
                     help="host gradients: ring of layer slots (14 B/param of host memory) or a full arena (18)")
     ap.add_argument("--host-threads", type=int, default=0, help="host optimizer threads per replica (0: cores / N)")
+    ap.add_argument("--grad-dtype", default="fp32", choices=["fp32", "bf16"],
+                    help="dtype of the offloaded gradients (bf16: MT_FLAG_BF16_GRADS, a measured variant)")
     ap.add_argument("--no-defer", action="store_true",
                     help="run every update inside its own step (no MT_FLAG_DEFER_UPDATES)")
     return ap.parse_args()
@@ -584,7 +586,8 @@ def main():
     # The LM head's and the last layer's updates overlap the next forward sweep
     # (MT_FLAG_DEFER_UPDATES), when the host optimizer is otherwise idle.
     cfg.flags = (mt.MT_FLAG_KERNEL_TIMING | (mt.MT_FLAG_GRAD_RING if args.grads == "ring" else 0) |
-                 (0 if args.no_defer else mt.MT_FLAG_DEFER_UPDATES))
+                 (0 if args.no_defer else mt.MT_FLAG_DEFER_UPDATES) |
+                 (mt.MT_FLAG_BF16_GRADS if args.grad_dtype == "bf16" else 0))
     ncpu = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cfg.host_threads = args.host_threads or max(1, ncpu // world)
 
@@ -697,8 +700,9 @@ def main():
                        "deferred_updates": (None if args.no_defer else
                                             f"LM head + last {defer_layers(sh)} layer(s) updated during the next "
                                             "forward sweep; the timed region ends after mt_flush"),
-                       "grads": (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
-                                 if args.grads == "ring" else "full fp32 gradient arena in pinned host memory")},
+                       "grads": (f"{args.grad_dtype} gradients offloaded; " +
+                                 (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
+                                  if args.grads == "ring" else "full gradient arena in pinned host memory"))},
             "model_tflops": model_f * world / (t_dev / K) / 1e12,
             "executed_tflops": exec_f * world / (t_dev / K) / 1e12,
             "roofline": {"bound": "tensor", "kernel": "tcgen05 bf16 GEMM (all projections, fwd/dX/dW)",

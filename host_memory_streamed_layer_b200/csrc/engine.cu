@@ -78,7 +78,7 @@ struct Job {
   int layer;
   cudaEvent_t ready;         // offload of this job's gradients has completed
   int flag_index;            // index in the finite-flag array
-  const float* g = nullptr;  // LAYER: host gradient of the layer's first element
+  const uint8_t* g = nullptr;  // LAYER: host gradient of the layer's first element (gsz bytes each)
   bool defer = false;        // HEAD / LAYER: check now, update at the next step
   int step = 0;              // *_PREV: the AdamW step (bias correction) of the update
 };
@@ -100,9 +100,11 @@ struct mt_ctx {
   bool arena_owned = false;
   float* m = nullptr;  // Adam moments (pageable, 64-byte aligned)
   float* v = nullptr;
-  float* grad = nullptr;          // pinned fp32 gradient arena (not with MT_FLAG_GRAD_RING)
-  float* ring = nullptr;          // pinned gradient ring of MT_GRAD_RING_SLOTS layer slots
-  float* grad_head = nullptr;     // [final norm | LM head] gradients: inside grad, or own buffer
+  // Host gradients, gsz bytes per element (4: fp32; 2: bf16 with MT_FLAG_BF16_GRADS).
+  int gsz = 4;
+  uint8_t* grad = nullptr;        // pinned gradient arena (not with MT_FLAG_GRAD_RING)
+  uint8_t* ring = nullptr;        // pinned gradient ring of MT_GRAD_RING_SLOTS layer slots
+  uint8_t* grad_head = nullptr;   // [final norm | LM head] gradients: inside grad, or own buffer
   size_t layer_f = 0;             // floats of one layer's gradient block
   uint16_t* bf_layers = nullptr;  // pinned bf16 layer blocks
   uint16_t* bf_embed = nullptr;   // pinned bf16 embedding (read by the GPU in place)
@@ -127,6 +129,8 @@ struct mt_ctx {
   cudaStream_t s_h2d = nullptr, s_comp = nullptr, s_d2h = nullptr;
   uint16_t* wslot[2] = {nullptr, nullptr};
   float* gslot[2] = {nullptr, nullptr};
+  uint16_t* gslot16[2] = {nullptr, nullptr};  // MT_FLAG_BF16_GRADS: bf16 copies offloaded instead
+  uint16_t* d_head_g16 = nullptr;
   uint16_t* d_head_w = nullptr;  // [gf | Whead] bf16
   float* d_head_g = nullptr;     // [dgf | dWhead] fp32
   float* xb = nullptr;           // boundary activations [(L+1), T, d]
@@ -166,7 +170,7 @@ struct mt_ctx {
   std::vector<Job> deferred;
   std::vector<char> prev_pending;
   int defer_layers = 0;
-  float* defer_g = nullptr;
+  uint8_t* defer_g = nullptr;
   int overlap_threads = 0;
   struct JobTime {
     int kind, layer;
@@ -458,7 +462,8 @@ bool wait_event(mt_ctx* c, cudaEvent_t e) {
 struct Seg {
   size_t off, n;       // floats in the arena
   uint16_t* bf;        // bf16 destination of element 0
-  const float* g;      // gradient of element 0; nullptr: zero gradient
+  const float* g;      // fp32 gradient of element 0; both null: zero gradient
+  const uint16_t* g16 = nullptr;  // bf16 gradient of element 0 (MT_FLAG_BF16_GRADS)
 };
 
 // AdamW step t over the segments. threads > 0 caps the threads that work on
@@ -472,20 +477,25 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs, int t, int threads 
     size_t off, n;
     uint16_t* bf;
     const float* g;
+    const uint16_t* g16;
   };
   std::vector<Task> tasks;
-  size_t total = 0;
+  double bytes = 0;  // host DRAM bytes: p, m, v read and written, bf16 copy written, gradient read
   for (const Seg& sg : segs) {
     for (size_t i = 0; i < sg.n; i += chunk)
-      tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf ? sg.bf + i : nullptr, sg.g ? sg.g + i : nullptr});
-    total += sg.n;
+      tasks.push_back({sg.off + i, std::min(chunk, sg.n - i), sg.bf ? sg.bf + i : nullptr, sg.g ? sg.g + i : nullptr,
+                       sg.g16 ? sg.g16 + i : nullptr});
+    bytes += (26.0 + (sg.g ? 4.0 : sg.g16 ? 2.0 : 0.0)) * sg.n;
   }
   if (tasks.empty()) return;
   const double t0 = now_s();
   if (c->adamw_first == 0) c->adamw_first = t0;
   auto one = [&](size_t i) {
     const Task& k = tasks[i];
-    adamw_chunk(c->arena + k.off, k.g, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
+    if (k.g16)
+      adamw_chunk_bf16g(c->arena + k.off, k.g16, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
+    else
+      adamw_chunk(c->arena + k.off, k.g, c->m + k.off, c->v + k.off, k.bf, k.n, h, t);
   };
   if (threads <= 0 || threads >= c->pool->size()) {
     c->pool->run((int)tasks.size(), [&](int i) { one((size_t)i); });
@@ -497,7 +507,7 @@ void adamw_segments(mt_ctx* c, const std::vector<Seg>& segs, int t, int threads 
   }
   c->adamw_last = now_s();
   c->adamw_s += c->adamw_last - t0;
-  c->adamw_bytes += 30.0 * total;
+  c->adamw_bytes += bytes;
 }
 
 void run_job_body(mt_ctx* c, const Job& j);
@@ -514,21 +524,28 @@ void run_job(mt_ctx* c, const Job& j) {
   c->job_times.push_back({(int)j.kind, j.layer, t0, now_s()});
 }
 
+// Segment of n arena floats from `off` whose host gradient starts at g
+// (gsz bytes per element).
+Seg grad_seg(mt_ctx* c, size_t off, size_t n, uint16_t* bf, const uint8_t* g) {
+  if (c->gsz == 2) return Seg{off, n, bf, nullptr, reinterpret_cast<const uint16_t*>(g)};
+  return Seg{off, n, bf, reinterpret_cast<const float*>(g)};
+}
+
 // AdamW segments of decoder layer l (gradient block g) or, for l < 0, of the
 // final norm and LM head (gradients in grad_head).
-std::vector<Seg> layer_or_head_segs(mt_ctx* c, int l, const float* g) {
+std::vector<Seg> layer_or_head_segs(mt_ctx* c, int l, const uint8_t* g) {
   const Layout& y = c->lay;
   std::vector<Seg> segs;
   if (l >= 0) {
     uint16_t* blk = c->bf_layers + (size_t)l * y.bf_layer;
     for (int tid = 0; tid < kLayerTensors; ++tid) {
       const TRef& r = y.t(l, tid);
-      segs.push_back({r.off, r.n, blk + y.bf_of(tid), g + (r.off - y.layer_begin(l))});
+      segs.push_back(grad_seg(c, r.off, r.n, blk + y.bf_of(tid), g + (r.off - y.layer_begin(l)) * c->gsz));
     }
   } else {
-    segs.push_back({y.final_norm.off, y.final_norm.n, c->bf_head, c->grad_head});
-    segs.push_back({y.head.off, y.head.n, c->bf_head + align_up(y.sh.d, 128),
-                    c->grad_head + (y.head.off - y.final_norm.off)});
+    segs.push_back(grad_seg(c, y.final_norm.off, y.final_norm.n, c->bf_head, c->grad_head));
+    segs.push_back(grad_seg(c, y.head.off, y.head.n, c->bf_head + align_up(y.sh.d, 128),
+                            c->grad_head + (y.head.off - y.final_norm.off) * c->gsz));
   }
   return segs;
 }
@@ -593,13 +610,14 @@ void run_job_body(mt_ctx* c, const Job& j) {
     // gradient arena, put last step's touched rows back to zero and scatter
     // this step's rows in (every other row's stored gradient is 0). The update
     // reads them from the staging rows.
-    float* ge = c->grad ? c->grad + y.embed.off : nullptr;
-    const size_t d = s.d;
+    uint8_t* ge = c->grad ? c->grad + y.embed.off * c->gsz : nullptr;
+    const size_t d = s.d, gsz = c->gsz;
     const int nt = c->pool->size() * 4;
     if (ge) {
       const size_t np = c->prev_uniq.size();
       c->pool->run(nt, [&](int i) {
-        for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k) memset(ge + (size_t)c->prev_uniq[k] * d, 0, d * 4);
+        for (size_t k = np * i / nt; k < np * (i + 1) / nt; ++k)
+          memset(ge + (size_t)c->prev_uniq[k] * d * gsz, 0, d * gsz);
       });
     }
     c->prev_uniq = c->uniq;
@@ -608,11 +626,17 @@ void run_job_body(mt_ctx* c, const Job& j) {
     c->pool->run(nt, [&](int i) {
       bool b = false;
       for (size_t u = nu * i / nt; u < nu * (i + 1) / nt; ++u) {
-        const float* src = c->emb_rows_h + u * d;
+        float* src = c->emb_rows_h + u * d;
+        if (gsz == 2)  // bf16 gradients: these rows are rounded once too, here on the host
+          for (size_t k = 0; k < d; ++k) {
+            const uint32_t w = (uint32_t)bf16_rne(src[k]) << 16;
+            memcpy(src + k, &w, 4);
+          }
         float acc = 0.f;
         for (size_t k = 0; k < d; ++k) acc += src[k] * 0.f;  // NaN or Inf anywhere makes acc NaN
         b |= !(acc == 0.f);
-        if (ge) memcpy(ge + (size_t)c->uniq[u] * d, src, d * sizeof(float));
+        if (ge && gsz == 4) memcpy(ge + (size_t)c->uniq[u] * d * 4, src, d * 4);
+        if (ge && gsz == 2) bf16_round_chunk(src, reinterpret_cast<uint16_t*>(ge + (size_t)c->uniq[u] * d * 2), d);
       }
       bad[i] = b;
     });
@@ -795,11 +819,11 @@ int issue_head_load(mt_ctx* c) {
 // jobs finish in backward order, so that is when layer_jobs_done passes it.
 int offload_layer(mt_ctx* c, int l, int k) {
   const Layout& y = c->lay;
-  const size_t b = y.layer_begin(l), e = y.layer_end(l);
+  const size_t b = y.layer_begin(l), e = y.layer_end(l), gsz = c->gsz;
   const int nd = c->defer_layers;
-  float* dst = c->grad ? c->grad + b
-               : k < nd ? c->defer_g + (size_t)k * c->layer_f
-                        : c->ring + (size_t)((k - nd) % MT_GRAD_RING_SLOTS) * c->layer_f;
+  uint8_t* dst = c->grad ? c->grad + b * gsz
+                 : k < nd ? c->defer_g + (size_t)k * c->layer_f * gsz
+                          : c->ring + (size_t)((k - nd) % MT_GRAD_RING_SLOTS) * c->layer_f * gsz;
   if (!c->grad && k >= nd + MT_GRAD_RING_SLOTS) {
     std::unique_lock<std::mutex> lk(c->opt_mu);
     const int need = k - MT_GRAD_RING_SLOTS + 1;
@@ -807,10 +831,15 @@ int offload_layer(mt_ctx* c, int l, int k) {
                                  [&] { return c->layer_jobs_done >= need; }))
       return set_err(c, MT_ERR_TIMEOUT, "gradient ring: no slot was released within the wait limit");
   }
+  const void* src = c->gslot[k & 1];
+  if (gsz == 2) {  // bf16 offload: round the checked fp32 gradients on the GPU (RNE)
+    KL(launch_cast_f32_bf16(c->gslot[k & 1], c->gslot16[k & 1], (int64_t)(e - b), c->s_comp), 1);
+    src = c->gslot16[k & 1];
+  }
   CK(cudaEventRecord(c->ev_gready[k], c->s_comp));
   CK(cudaStreamWaitEvent(c->s_d2h, c->ev_gready[k], 0));
   CK(cudaEventRecord(c->ev_d2h_start[k], c->s_d2h));
-  CK(cudaMemcpyAsync(dst, c->gslot[k & 1], (e - b) * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  CK(cudaMemcpyAsync(dst, src, (e - b) * gsz, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaMemcpyAsync(c->flags_h + l, c->d_flags + l, 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaEventRecord(c->ev_gdrained[k], c->s_d2h));
   Job j{Job::LAYER, l, c->ev_gdrained[k], l, dst};
@@ -847,11 +876,16 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         CK(cudaEventRecord(c->ev_fwd_end, sc));
         CK(cudaStreamWaitEvent(sc, c->ev_head_wready, 0));
         CKM(head_step(c, gin));
+        const size_t n = y.head.off + y.head.n - y.final_norm.off;
+        const void* hsrc = c->d_head_g;
+        if (c->gsz == 2) {
+          KL(launch_cast_f32_bf16(c->d_head_g, c->d_head_g16, (int64_t)n, sc), 1);
+          hsrc = c->d_head_g16;
+        }
         CK(cudaEventRecord(c->ev_head_gready, sc));
         CK(cudaStreamWaitEvent(c->s_d2h, c->ev_head_gready, 0));
         CK(cudaEventRecord(c->ev_head_d2h_start, c->s_d2h));
-        const size_t n = y.head.off + y.head.n - y.final_norm.off;
-        CK(cudaMemcpyAsync(c->grad_head, c->d_head_g, n * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+        CK(cudaMemcpyAsync(c->grad_head, hsrc, n * c->gsz, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaMemcpyAsync(c->flags_h + L, c->d_flags + L, 4, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaEventRecord(c->ev_head_drained, c->s_d2h));
         Job hj{Job::HEAD, -1, c->ev_head_drained, L};
@@ -927,8 +961,8 @@ void collect_stats(mt_ctx* c) {
   st.h2d_bytes = (double)c->load_seq.size() * y.bf_layer * 2 +
                  (double)(align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d) * 2 + 4.0 * (4 * y.sh.T + 1) +
                  (double)y.sh.T * y.sh.d * 2;  // embedding rows read in place
-  st.d2h_bytes = 4.0 * (y.head.off + y.head.n - y.final_norm.off) + 4.0 * c->uniq.size() * y.sh.d + 8.0;
-  for (int l = 0; l < L; ++l) st.d2h_bytes += 4.0 * (y.layer_end(l) - y.layer_begin(l));
+  st.d2h_bytes = (double)c->gsz * (y.head.off + y.head.n - y.final_norm.off) + 4.0 * c->uniq.size() * y.sh.d + 12.0;
+  for (int l = 0; l < L; ++l) st.d2h_bytes += (double)c->gsz * (y.layer_end(l) - y.layer_begin(l));
   st.adamw_ms = c->adamw_s * 1e3;
   st.adamw_bytes = c->adamw_bytes;
   st.gemm_flops = st.gemm_ms = st.attn_flops = st.attn_ms = 0;
@@ -951,7 +985,7 @@ void collect_stats(mt_ctx* c) {
 // ---------------------------------------------------------------------------
 // Create / destroy helpers.
 // ---------------------------------------------------------------------------
-size_t device_bytes(const Layout& y, int Tc) {
+size_t device_bytes(const Layout& y, int Tc, bool g16) {
   const Shapes& s = y.sh;
   const size_t T = s.T, d = s.d, F = s.F, V = s.V;
   const size_t A = 256;
@@ -964,6 +998,11 @@ size_t device_bytes(const Layout& y, int Tc) {
   add(lay_f * 4);
   add((align_up(d, 128) + V * d) * 2);                     // head weights
   add((y.head.off - y.final_norm.off + V * d) * 4);         // head grads
+  if (g16) {                                                // bf16 offload copies
+    add(lay_f * 2);
+    add(lay_f * 2);
+    add((y.head.off - y.final_norm.off + V * d) * 2);
+  }
   add((size_t)(s.L + 1) * T * d * 4);                       // boundary activations
   add(T * d * 2);                                           // u
   add(T * (size_t)s.Nqkv * 2);                              // qkv
@@ -1083,7 +1122,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   if (major != 10 || minor != 0) return set_err(nullptr, MT_ERR_CUDA, "this library runs on sm_100 (B200) only");
 
   const int Tc = logits_chunk(s);
-  const size_t need = device_bytes(y, Tc);
+  const size_t need = device_bytes(y, Tc, (cfg->flags & MT_FLAG_BF16_GRADS) != 0);
   size_t free_b = 0, total_b = 0;
   if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaMemGetInfo failed");
   if (need + ((size_t)256 << 20) > free_b) {
@@ -1097,6 +1136,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->lay = y;
   c->device = cfg->device;
   c->Tc = Tc;
+  c->gsz = (cfg->flags & MT_FLAG_BF16_GRADS) ? 2 : 4;
+  const size_t gsz = c->gsz;
   int nthreads = cfg->host_threads;
   if (nthreads <= 0) nthreads = std::max(1, (int)std::thread::hardware_concurrency() - 1);
   c->pool = new ThreadPool(nthreads - 1);
@@ -1129,18 +1170,18 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     if (n > 0) c->overlap_threads = std::min(n, c->pool->size());
   }
   if (cfg->flags & MT_FLAG_GRAD_RING) {
-    if (cudaHostAlloc(reinterpret_cast<void**>(&c->ring), (size_t)MT_GRAD_RING_SLOTS * c->layer_f * 4,
+    if (cudaHostAlloc(reinterpret_cast<void**>(&c->ring), (size_t)MT_GRAD_RING_SLOTS * c->layer_f * gsz,
                       cudaHostAllocPortable) != cudaSuccess ||
-        cudaHostAlloc(reinterpret_cast<void**>(&c->grad_head), head_f * 4, cudaHostAllocPortable) != cudaSuccess)
+        cudaHostAlloc(reinterpret_cast<void**>(&c->grad_head), head_f * gsz, cudaHostAllocPortable) != cudaSuccess)
       return fail(MT_ERR_PIN, "pinned gradient ring allocation failed");
     if (c->defer_layers > 0 && cudaHostAlloc(reinterpret_cast<void**>(&c->defer_g),
-                                             (size_t)c->defer_layers * c->layer_f * 4,
+                                             (size_t)c->defer_layers * c->layer_f * gsz,
                                              cudaHostAllocPortable) != cudaSuccess)
       return fail(MT_ERR_PIN, "pinned deferred-layer gradient allocation failed");
   } else {
-    if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * 4, cudaHostAllocPortable) != cudaSuccess)
+    if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * gsz, cudaHostAllocPortable) != cudaSuccess)
       return fail(MT_ERR_PIN, "pinned gradient arena allocation failed");
-    c->grad_head = c->grad + y.final_norm.off;
+    c->grad_head = c->grad + y.final_norm.off * gsz;
   }
   if (cudaHostAlloc(reinterpret_cast<void**>(&c->bf_layers), (size_t)s.L * y.bf_layer * 2, cudaHostAllocPortable) !=
           cudaSuccess ||
@@ -1175,15 +1216,16 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) {
     memset(c->m + b, 0, (e - b) * 4);
     memset(c->v + b, 0, (e - b) * 4);
-    if (c->grad) memset(c->grad + b, 0, (e - b) * 4);
+    if (c->grad) memset(c->grad + b * gsz, 0, (e - b) * gsz);
   });
   if (c->ring) {
     const size_t nr = (size_t)MT_GRAD_RING_SLOTS * c->layer_f;
-    parallel_ranges(*c->pool, nr, [&](size_t b, size_t e) { memset(c->ring + b, 0, (e - b) * 4); });
+    parallel_ranges(*c->pool, nr, [&](size_t b, size_t e) { memset(c->ring + b * gsz, 0, (e - b) * gsz); });
     if (c->defer_g)
       parallel_ranges(*c->pool, (size_t)c->defer_layers * c->layer_f,
-                      [&](size_t b, size_t e) { memset(c->defer_g + b, 0, (e - b) * 4); });
-    parallel_ranges(*c->pool, head_f, [&](size_t b, size_t e) { memset(c->grad_head + b, 0, (e - b) * 4); });
+                      [&](size_t b, size_t e) { memset(c->defer_g + b * gsz, 0, (e - b) * gsz); });
+    parallel_ranges(*c->pool, head_f,
+                    [&](size_t b, size_t e) { memset(c->grad_head + b * gsz, 0, (e - b) * gsz); });
   }
   // bf16 streaming copies
   for (int l = 0; l < s.L; ++l) {
@@ -1220,6 +1262,11 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->gslot[1] = (float*)carve(lay_f * 4);
   c->d_head_w = (uint16_t*)carve(head_bf * 2);
   c->d_head_g = (float*)carve((y.head.off - y.final_norm.off + V * d) * 4);
+  if (gsz == 2) {
+    c->gslot16[0] = (uint16_t*)carve(lay_f * 2);
+    c->gslot16[1] = (uint16_t*)carve(lay_f * 2);
+    c->d_head_g16 = (uint16_t*)carve((y.head.off - y.final_norm.off + V * d) * 2);
+  }
   c->xb = (float*)carve((size_t)(s.L + 1) * T * d * 4);
   c->u_b = (uint16_t*)carve(T * d * 2);
   c->qkv_b = (uint16_t*)carve(T * (size_t)s.Nqkv * 2);
@@ -1475,7 +1522,17 @@ extern "C" int mt_get_grads(mt_ctx* c, float* dst, size_t bytes) {
   if (!c || !dst) return MT_ERR_ARG;
   if (!c->grad) return set_err(c, MT_ERR_CONFIG, "created with MT_FLAG_GRAD_RING: no gradient arena is kept");
   if (bytes < c->lay.total * 4) return set_err(c, MT_ERR_ARG, "destination smaller than the arena");
-  memcpy(dst, c->grad, c->lay.total * 4);
+  if (c->gsz == 4) {
+    memcpy(dst, c->grad, c->lay.total * 4);
+  } else {  // bf16 gradients widen exactly to fp32
+    const uint16_t* g = reinterpret_cast<const uint16_t*>(c->grad);
+    parallel_ranges(*c->pool, c->lay.total, [&](size_t b, size_t e) {
+      for (size_t i = b; i < e; ++i) {
+        const uint32_t u = (uint32_t)g[i] << 16;
+        memcpy(dst + i, &u, 4);
+      }
+    });
+  }
   return MT_OK;
 }
 
@@ -1589,7 +1646,7 @@ extern "C" int mt_get_stream(mt_ctx* c, void** stream) {
 extern "C" size_t mt_device_bytes(const mt_config* cfg) {
   if (validate_config(cfg, nullptr) != MT_OK) return 0;
   const Layout y = make_layout(*cfg);
-  return device_bytes(y, logits_chunk(y.sh));
+  return device_bytes(y, logits_chunk(y.sh), (cfg->flags & MT_FLAG_BF16_GRADS) != 0);
 }
 
 namespace {

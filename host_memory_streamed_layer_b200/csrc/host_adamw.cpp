@@ -26,11 +26,26 @@ uint16_t bf16_rne(float x) {
 
 namespace {
 
-void adamw_scalar(float* p, const float* g, float* m, float* v, uint16_t* pb, size_t n, float decay, float b1,
+inline float bf16_to_f32(uint16_t h) {
+  const uint32_t u = (uint32_t)h << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return f;
+}
+
+// G is the gradient's element type: float, or uint16_t holding bf16 bits.
+template <typename G>
+void adamw_scalar(float* p, const G* g, float* m, float* v, uint16_t* pb, size_t n, float decay, float b1,
                   float b2, float step, float inv_sqrt_bc2, float eps) {
   const float c1 = 1.f - b1, c2 = 1.f - b2;
   for (size_t i = 0; i < n; ++i) {
-    const float gi = g ? g[i] : 0.f;
+    float gi = 0.f;
+    if (g) {
+      if constexpr (sizeof(G) == 2)
+        gi = bf16_to_f32(g[i]);
+      else
+        gi = g[i];
+    }
     const float mi = b1 * m[i] + c1 * gi;
     const float vi = b2 * v[i] + c2 * gi * gi;
     const float pi = p[i] * decay - step * mi / (sqrtf(vi) * inv_sqrt_bc2 + eps);
@@ -58,8 +73,9 @@ __attribute__((target("avx512f,avx512bw"))) inline __m256i bf16x16_rne(__m512 x)
 // HAS_G = false is the update of a zero gradient (embedding rows no token of
 // the batch touches): the moments only decay and no gradient is read; the
 // result is bit-identical to reading zeros (b m + 0 rounds like b m).
-template <bool HAS_G>
-__attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const float* g, float* m, float* v,
+// G = uint16_t reads a bf16 gradient (exactly widened to fp32).
+template <bool HAS_G, typename G = float>
+__attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const G* g, float* m, float* v,
                                                               uint16_t* pb, size_t n, float decay, float b1, float b2,
                                                               float step, float inv_sqrt_bc2, float eps) {
   const bool nt = pb && ((reinterpret_cast<uintptr_t>(pb) & 31) == 0);
@@ -71,7 +87,12 @@ __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const fl
   for (; i + 16 <= n; i += 16) {
     __m512 mi, vi;
     if (HAS_G) {
-      const __m512 gi = _mm512_loadu_ps(g + i);
+      __m512 gi;
+      if constexpr (sizeof(G) == 2)
+        gi = _mm512_castsi512_ps(_mm512_slli_epi32(
+            _mm512_cvtepu16_epi32(_mm256_loadu_si256(reinterpret_cast<const __m256i*>(g + i))), 16));
+      else
+        gi = _mm512_loadu_ps(reinterpret_cast<const float*>(g) + i);
       mi = _mm512_fmadd_ps(vb1, _mm512_loadu_ps(m + i), _mm512_mul_ps(vc1, gi));
       vi = _mm512_fmadd_ps(vb2, _mm512_loadu_ps(v + i), _mm512_mul_ps(vc2, _mm512_mul_ps(gi, gi)));
     } else {
@@ -91,8 +112,8 @@ __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const fl
   }
   if (nt) _mm_sfence();
   if (i < n)
-    adamw_scalar(p + i, HAS_G ? g + i : nullptr, m + i, v + i, pb ? pb + i : nullptr, n - i, decay, b1, b2, step,
-                 inv_sqrt_bc2, eps);
+    adamw_scalar<G>(p + i, HAS_G ? g + i : nullptr, m + i, v + i, pb ? pb + i : nullptr, n - i, decay, b1, b2, step,
+                    inv_sqrt_bc2, eps);
 }
 
 __attribute__((target("avx512f,avx512bw"))) void round_avx512(const float* x, uint16_t* out, size_t n) {
@@ -123,9 +144,23 @@ void adamw_chunk(float* p, const float* g, float* m, float* v, uint16_t* pb, siz
   if (adamw_uses_avx512() && g)
     adamw_avx512<true>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
   else if (adamw_uses_avx512())
-    adamw_avx512<false>(p, nullptr, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
+    adamw_avx512<false>(p, (const float*)nullptr, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
   else
-    adamw_scalar(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
+    adamw_scalar<float>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
+}
+
+void adamw_chunk_bf16g(float* p, const uint16_t* g, float* m, float* v, uint16_t* pb, size_t n, const AdamHyper& h,
+                       int t) {
+  if (!g) return adamw_chunk(p, nullptr, m, v, pb, n, h, t);
+  const double bc1 = 1.0 - pow((double)h.beta1, t);
+  const double bc2 = 1.0 - pow((double)h.beta2, t);
+  const float decay = 1.f - h.lr * h.wd;
+  const float step = (float)(h.lr / bc1);
+  const float inv_sqrt_bc2 = (float)(1.0 / sqrt(bc2));
+  if (adamw_uses_avx512())
+    adamw_avx512<true, uint16_t>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
+  else
+    adamw_scalar<uint16_t>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
 }
 
 void bf16_round_chunk(const float* x, uint16_t* out, size_t n) {

@@ -31,6 +31,10 @@ struct AdamHyper {
 // g == nullptr means a zero gradient (nothing is read).
 void adamw_chunk(float* p, const float* g, float* m, float* v, uint16_t* pb, size_t n, const AdamHyper& h, int t);
 
+// The same step with a bf16 gradient (bit patterns, widened exactly to fp32).
+void adamw_chunk_bf16g(float* p, const uint16_t* g, float* m, float* v, uint16_t* pb, size_t n, const AdamHyper& h,
+                       int t);
+
 // Round-to-nearest-even fp32 -> bf16 over n elements (NaN stays NaN).
 void bf16_round_chunk(const float* x, uint16_t* out, size_t n);
 uint16_t bf16_rne(float x);

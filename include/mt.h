@@ -88,6 +88,19 @@ extern "C" {
  * deferred layers keep their gradients in MT_DEFER_LAYERS extra pinned
  * layer-sized buffers. Ignored with MT_FLAG_NO_UPDATE. */
 #define MT_FLAG_DEFER_UPDATES 0x10u
+/* Offload gradients in bf16 instead of fp32: after its finite check on the
+ * GPU, each layer's (and the LM head's) fp32 gradient is rounded to bf16
+ * (nearest even) and only the bf16 copy crosses the link and sits in host
+ * memory; the host AdamW widens it exactly and keeps the fp32 master and
+ * moments. It halves the gradient bytes over the link (4 -> 2 per parameter)
+ * and in host memory, and cuts the optimizer's host DRAM traffic from 30 to
+ * 28 bytes per parameter, at the cost of one more rounding of every gradient
+ * (relative error <= 2^-9 per element). The embedding-gradient rows cross
+ * the link in fp32 and are rounded the same way on the host. mt_get_grads
+ * returns the bf16 values widened to fp32, exactly what the update used. A measured
+ * link-versus-accuracy variant: the method's own design offloads the
+ * gradients in full precision (MegaTrain abstract: full-precision training). */
+#define MT_FLAG_BF16_GRADS 0x20u
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0
