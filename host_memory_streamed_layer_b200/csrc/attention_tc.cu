@@ -9,16 +9,20 @@
 //               O_j is done; one 64-column x 128-row, 128-byte-swizzled box
 //               shape serves Q, K and V)
 //   warp 1      MMA issuer: S_j = Q K_j^T (128 x 128 x hd) into one of two
-//               tensor-memory S buffers, then O_j = P_j V_j (128 x hd x 128)
-//               into one of two tensor-memory O buffers; S_{j+1} is issued
-//               before O_j so the tensor core works while softmax runs
+//               tensor-memory S buffers, then O += P_j V_j (128 x hd x 128)
+//               into the one tensor-memory O accumulator; S_{j+1} is issued
+//               before P_j V_j so the tensor core works while softmax runs
 //   warps 2..9  softmax: two warpgroups; in each, thread r owns query row r
-//               (its tensor-memory lane). Both read the whole S_j row for the
-//               row max; warpgroup g then computes exp2, the partial row sum
-//               and the bf16 P for keys [64g, 64g+64) (one 128-byte-swizzled
-//               K-major sub-tile of the A operand of the next MMA) and
-//               accumulates O columns [g hd/2, (g+1) hd/2) in registers, one
-//               block behind, with the online-softmax correction
+//               (its tensor-memory lane). Both load the whole S_j row in one
+//               batch for the row max; warpgroup g then computes exp2, the
+//               partial row sum and the bf16 P for keys [64g, 64g+64) (one
+//               128-byte-swizzled K-major sub-tile of the A operand of the
+//               next MMA) from the registers it already holds. The running
+//               maximum is raised lazily: only when a row's maximum grows by
+//               more than 2^8 (in exp2 units) are the row's O columns rescaled
+//               in tensor memory (after the previous P V has landed), so the
+//               probabilities stay below 256 and, on most blocks, O is never
+//               read back until the end
 //
 // Every mbarrier wait is bounded (mt_common.cuh); on expiry the kernel records
 // an error code, drains its copies and MMAs (bounded) and returns.
@@ -49,8 +53,12 @@ struct FaCfg {
   static constexpr int SMEM = 1024 + OFF_BAR + 256;
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;    // S buffers at columns 0 and 128
-  static constexpr uint32_t O_COL = 256;  // O buffers at 256 and 256 + HD
+  static constexpr uint32_t O_COL = 256;  // the O accumulator, HD columns
 };
+
+// A row's running maximum is raised only when its block maximum exceeds it by
+// more than this many units of exp2 (probabilities then stay <= 2^8).
+constexpr float kRescaleLog2 = 8.0f;
 
 struct FaParams {
   __nv_bfloat16* O;
@@ -77,6 +85,21 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Element-wise fp32 add of a shared-memory tile into global memory by the TMA
+// engine (tensor map m, tile origin {c0 inner, c1 outer}); asynchronous, in a
+// bulk async-group of the issuing thread. No multicast.
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
+  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)),
+               "r"(smem_u32(src)), "r"(c0), "r"(c1)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until the source of every committed bulk operation has been read.
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until every committed bulk operation has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 template <int HD>
 __global__ void __launch_bounds__(FA_THREADS, 1)
     k_flash_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -97,8 +120,7 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
   uint64_t* s_full = bar + 9;    // [2]
   uint64_t* s_empty = bar + 11;  // [2]
   uint64_t* p_full = bar + 13;   // [2]
-  uint64_t* o_full = bar + 15;   // [2]
-  uint64_t* o_empty = bar + 17;  // [2]
+  uint64_t* o_full = bar + 15;   // [2]  P_j V_j (and every earlier MMA) done, j mod 2
   uint64_t* drain = bar + 19;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 20);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 21);
@@ -122,7 +144,6 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       mbar_init(&s_empty[i], 8);
       mbar_init(&p_full[i], 8);
       mbar_init(&o_full[i], 1);
-      mbar_init(&o_empty[i], 8);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -196,18 +217,19 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
       bool ok = mbar_wait(q_full, 0) && !*abort_flag;
       bool issued = false;
+      // O += P_i V_i. The softmax warps signal p_full only after any rescale
+      // of O that block i needs, so the accumulator is never read and
+      // written at once.
       auto issue_pv = [&](int i) -> bool {
         const int pb = i & 1;
         const uint32_t ph = (i >> 1) & 1;
-        if (*abort_flag || !mbar_wait(&v_full[pb], ph) || !mbar_wait(&p_full[pb], ph) ||
-            !mbar_wait(&o_empty[pb], ph ^ 1))
-          return false;
+        if (*abort_flag || !mbar_wait(&v_full[pb], ph) || !mbar_wait(&p_full[pb], ph)) return false;
         tc_fence_after();
         const uint64_t aP = dP0 + ((pb * C::P_BYTES) >> 4), bV = dV0 + (((i & 1) * C::KV_BYTES) >> 4);
 #pragma unroll
         for (int kk = 0; kk < FA_BKV / 16; ++kk)
-          umma_bf16(tmem + C::O_COL + pb * HD, aP + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), bV + ((kk * 2048) >> 4),
-                    idesc_o, kk != 0);
+          umma_bf16(tmem + C::O_COL, aP + (((kk >> 2) * 16384 + (kk & 3) * 32) >> 4), bV + ((kk * 2048) >> 4),
+                    idesc_o, (i | kk) != 0);
         umma_commit(&o_full[pb]);
         umma_commit(&v_empty[pb]);
         return true;
@@ -251,30 +273,10 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // query row inside the tile == tensor-memory lane
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t obase = tmem + lane_base + C::O_COL + wg * HH;  // this warpgroup's O columns
     const float sl2 = p.scale * 1.4426950408889634f;
-    float o[HH];
-#pragma unroll
-    for (int i = 0; i < HH; ++i) o[i] = 0.f;
-    float m = -INFINITY, l = 0.f, corr_prev = 0.f;
+    float m = -INFINITY, l = 0.f;  // running (lazily raised) row maximum, this half's row sum
     bool ok = true;
-
-    auto accumulate_o = [&](int i, float corr) -> bool {
-      const int ob = i & 1;
-      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[ob], (i >> 1) & 1)) return false;
-      tc_fence_after();
-#pragma unroll
-      for (int c = 0; c < HH / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem + lane_base + C::O_COL + ob * HD + wg * HH + c * 16, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 16; ++e) o[c * 16 + e] = o[c * 16 + e] * corr + __uint_as_float(v[e]);
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&o_empty[ob]);
-      return true;
-    };
 
     for (int j = 0; j < nkv; ++j) {
       const int sb = j & 1;
@@ -285,60 +287,85 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       }
       tc_fence_after();
       const uint32_t sbase = tmem + lane_base + C::S_COL + sb * FA_BKV;
+      // The whole row in one batch: this warpgroup's 64 keys (kept for the
+      // exponentials) and the other 64 (for the maximum only).
+      uint32_t v[64], w[64];
+      tmem_ld_32x32b_x32(sbase + wg * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+      tmem_ld_32x32b_x32(sbase + wg * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+      tmem_ld_32x32b_x32(sbase + (wg ^ 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(w));
+      tmem_ld_32x32b_x32(sbase + (wg ^ 1) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(w + 32));
+      tmem_ld_wait();
+      // The causal mask only touches the diagonal block (j == nkv - 1): row r
+      // sees keys [0, r] of it.
+      const bool diag = j == nkv - 1;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const int cv = wg * 64 + e, cw = (wg ^ 1) * 64 + e;
+        if (!diag || cv <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
+        if (!diag || cw <= r) mx = fmaxf(mx, __uint_as_float(w[e]));
+      }
+      // Lazy maximum: raise it (and rescale O and l) only when the block's
+      // maximum exceeds the running one by more than 2^kRescaleLog2.
+      const bool raise = (m == -INFINITY) || (mx - m) * sl2 > kRescaleLog2;
+      const float corr = (raise && m != -INFINITY) ? ex2((m - mx) * sl2) : 1.f;
+      if (raise) m = mx;
+      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+        // O holds blocks < j scaled by the old maximum: once P_{j-1} V_{j-1}
+        // has landed, multiply this warpgroup's columns of the raised rows.
+        const int pj = j - 1;
+        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[pj & 1], (pj >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < HH / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld_32x32b_x32(obase + c * 32, o);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint32_t t8[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) t8[u] = __float_as_uint(__uint_as_float(o[e + u]) * corr);
+            tmem_st_32x32b_x8(obase + c * 32 + e, t8);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+      }
+      l *= corr;
+      // The P buffer of this block was last read by P_{j-2} V_{j-2}.
+      if (j >= 2) {
+        const int pj = j - 2;
+        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[pj & 1], (pj >> 1) & 1)) {
+          ok = false;
+          break;
+        }
+      }
+      // this warpgroup's 64 keys -> probabilities, partial row sum, bf16 P
+      // into swizzle sub-tile wg of the A operand
       uint8_t* prow = sP + sb * C::P_BYTES + wg * 16384 + r * 128;
-      float corr, rs;
-      // The causal mask only touches the diagonal block: the other blocks run
-      // an instantiation without any per-element test.
-      auto block = [&](auto diag_tag) {
-        constexpr bool DIAG = decltype(diag_tag)::value;
-        // pass 1: row max of the visible scores (whole row)
-        float mx = -INFINITY;
+      const float mb = m * sl2;
+      float rs = 0.f;
 #pragma unroll
-        for (int c = 0; c < FA_BKV / 16; ++c) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(sbase + c * 16, v);
-          tmem_ld_wait();
+      for (int chunk = 0; chunk < 8; ++chunk) {  // 16-byte chunks of 8 keys
+        uint32_t pk[4];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x = __uint_as_float(v[e]);
-            if (!DIAG || c * 16 + e <= r) mx = fmaxf(mx, x);
-          }
+        for (int e = 0; e < 8; e += 2) {
+          const int k = chunk * 8 + e;
+          const int col = wg * 64 + k;
+          float p0 = ex2(fmaf(__uint_as_float(v[k]), sl2, -mb));
+          float p1 = ex2(fmaf(__uint_as_float(v[k + 1]), sl2, -mb));
+          if (diag && col > r) p0 = 0.f;
+          if (diag && col + 1 > r) p1 = 0.f;
+          rs += p0 + p1;
+          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        const float mnew = fmaxf(m, mx);
-        corr = (m == -INFINITY) ? 0.f : ex2((m - mnew) * sl2);
-        const float mb = mnew * sl2;
-        m = mnew;
-        // pass 2: this warpgroup's 64 keys -> probabilities, partial row sum,
-        // bf16 P into swizzle sub-tile wg of the A operand
-        rs = 0.f;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(sbase + wg * 64 + c * 16, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {  // two 16-byte chunks of 8 keys
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-              const int col = wg * 64 + c * 16 + q * 8 + e;
-              float p0 = ex2(fmaf(__uint_as_float(v[q * 8 + e]), sl2, -mb));
-              float p1 = ex2(fmaf(__uint_as_float(v[q * 8 + e + 1]), sl2, -mb));
-              if (DIAG && col > r) p0 = 0.f;
-              if (DIAG && col + 1 > r) p1 = 0.f;
-              rs += p0 + p1;
-              pk[e >> 1] = pack_bf16x2(p0, p1);
-            }
-            const int chunk = c * 2 + q;  // 0..7 inside the 64-key sub-tile
-            *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
-        }
-      };
-      if (j == nkv - 1)
-        block(std::true_type{});
-      else
-        block(std::false_type{});
-      l = l * corr + rs;
+        *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += rs;
       tc_fence_before();
       fence_proxy_async_smem();
       __syncwarp();
@@ -346,13 +373,11 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
         mbar_arrive(&s_empty[sb]);
         mbar_arrive(&p_full[sb]);
       }
-      if (j >= 1 && !accumulate_o(j - 1, corr_prev)) {
-        ok = false;
-        break;
-      }
-      corr_prev = corr;
     }
-    if (ok && !accumulate_o(nkv - 1, corr_prev)) ok = false;
+    // the last P V
+    if (ok && (__any_sync(0xffffffffu, *abort_flag) ||
+               !mbar_wait_warp(&o_full[(nkv - 1) & 1], ((nkv - 1) >> 1) & 1)))
+      ok = false;
     if (!ok) {
       record_error(p.err, DEV_TIMEOUT_EPILOGUE);
       *abort_flag = 1;
@@ -363,22 +388,29 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
     if (ok) lsum[wg * FA_BQ + r] = l;
     asm volatile("bar.sync 1, 256;" ::: "memory");
     if (ok) {
+      tc_fence_after();
       const float lt = l + lsum[(wg ^ 1) * FA_BQ + r];
       const int qi = q0 + r;
-      if (qi < p.s) {
-        const float inv = 1.f / lt;
-        __nv_bfloat16* orow = p.O + (int64_t)(row0 + qi) * p.ldo + h * HD + wg * HH;
+      const float inv = 1.f / lt;
+      __nv_bfloat16* orow = p.O + (int64_t)(row0 + qi) * p.ldo + h * HD + wg * HH;
 #pragma unroll
-        for (int c = 0; c < HH / 8; ++c) {
-          uint4 w;
-          w.x = pack_bf16x2(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-          w.y = pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-          w.z = pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-          w.w = pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-          reinterpret_cast<uint4*>(orow)[c] = w;
+      for (int c = 0; c < HH / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(obase + c * 32, o);  // warp-collective: every lane loads
+        tmem_ld_wait();
+        if (qi < p.s) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 t;
+            t.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv, __uint_as_float(o[e + 1]) * inv);
+            t.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            t.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            t.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 32 + e)[0] = t;
+          }
         }
-        if (wg == 0) p.LSE[((int64_t)b * p.H + h) * p.s + qi] = m * p.scale + logf(lt);
       }
+      if (wg == 0 && qi < p.s) p.LSE[((int64_t)b * p.H + h) * p.s + qi] = m * p.scale + logf(lt);
     }
   }
 
@@ -440,8 +472,10 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
 //          as their A operand; dS^T also into a 128-byte-swizzled shared tile)
 //   dV  += P^T dO,  dK += dS^T Q              (128 keys x hd, TMEM, A from TMEM)
 //   dQ^T = K^T dS^T                            (hd x 128 queries, into the
-//          dP^T columns), read out one head column per thread and added to
-//          the fp32 dQ accumulator with global reductions from registers
+//          dP^T columns), read out one head column per thread, staged as two
+//          64-query fp32 halves in the (then free) dS^T tile and added to the
+//          fp32 dQ accumulator by TMA bulk tensor reductions, which the L2
+//          performs while the warps go on with the next block's exponentials
 // Every product is N = 128 wide: 64-wide products run the tensor core at
 // little more than half rate (55 instead of 32 cycles per 128 x 64 x 16 MMA,
 // measured), which bounded the 64-query form of this kernel.
@@ -483,6 +517,7 @@ struct FbParams {
   const float* rsin;
   int* err;
   int vec_lse;  // LSE and D rows start 16-byte aligned: s % 4 == 0 and aligned bases
+  int T;        // tokens of all sequences: rows of the dQ accumulator
 };
 
 // Start-address step (address / 16) of k-step kk (16 elements of the
@@ -494,7 +529,7 @@ __device__ __forceinline__ uint32_t km_step(int kk) {
 __global__ void __launch_bounds__(FB_THREADS, 1)
     k_flash_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   FbParams p) {
+                   const __grid_constant__ CUtensorMap tmDQ, FbParams p) {
   using C = FbCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -515,6 +550,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   uint64_t* drain = bar + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12);
+  uint64_t* stage_full = bar + 13;  // [2] a 64-query half of dQ staged (8 warps each)
+  uint64_t* stage_free = bar + 15;  // the TMA has read a staged half (twice per block)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -538,12 +575,16 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     mbar_init(mma_done, 1);
     mbar_init(dq_empty, FB_GWARPS);
     mbar_init(drain, 1);
+    mbar_init(&stage_full[0], FB_GWARPS / 2);
+    mbar_init(&stage_full[1], FB_GWARPS / 2);
+    mbar_init(stage_free, 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmO);
+    tma_prefetch_desc(&tmDQ);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -683,23 +724,52 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     bool ok = true;
 
     // dQ^T of an iteration (complete: the caller waited for mma_done): this
-    // warp's 32 query columns for head column r, added to the fp32 dQ
-    // accumulator with reductions from registers (a warp's 32 lanes are 32
-    // consecutive head columns of one query row: 128 coalesced bytes).
-    auto flush_dq = [&](int hq, int q0) {
+    // warp's 32 query columns for head column r, scaled and written into the
+    // staging tile (the dS^T tile, which the dQ MMA has finished reading) as
+    // fp32 rows [query][head column] of its 64-query half; warp 2's lane 0
+    // hands each staged half to the TMA engine as one bulk tensor reduction
+    // into the fp32 dQ accumulator and releases the tile once the TMA has read
+    // it. Rows past the sequence end carry exact zeros (their dS is 0), so the
+    // add leaves whatever they overlap unchanged. Every wait is bounded;
+    // returns false after a wait ran out.
+    int nflush = 0;
+    auto flush_dq = [&](int hq, int q0) -> bool {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lane_base + C::C_DP + qg * FB_QW, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_empty);
-      const int qf = q0 + qg * FB_QW;
-      float* dst = p.dQacc + (int64_t)(row0 + qf) * p.ldqa + (int64_t)hq * FB_HD + r;
+      const int half = qg >> 1;
+      if (half == 1 && !mbar_wait_warp(stage_free, 0)) return false;  // the TMA has read half 0
+      float* stg = reinterpret_cast<float*>(sdSt) + (qg & 1) * 32 * FB_HD + r;
 #pragma unroll
-      for (int e = 0; e < FB_QW; ++e)
-        if (qf + e < p.s)
-          asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + (int64_t)e * p.ldqa), "f"(__uint_as_float(v[e]) * p.scale)
-                       : "memory");
+      for (int e = 0; e < FB_QW; ++e) stg[e * FB_HD] = __uint_as_float(v[e]) * p.scale;
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&stage_full[half]);
+      const uint32_t par = (uint32_t)(nflush & 1);
+      ++nflush;
+      if (warp == 2) {
+        int good = 1;
+        if (lane == 0) {
+          for (int h2 = 0; h2 < 2; ++h2) {
+            if (!mbar_wait(&stage_full[h2], par)) {
+              good = 0;
+              break;
+            }
+            // (a half that starts past the last token has nothing to add)
+            if (row0 + q0 + 64 * h2 < p.T) {
+              tma_reduce_add_2d(&tmDQ, sdSt, hq * FB_HD, row0 + q0 + 64 * h2);
+              bulk_commit_group();
+              bulk_wait_read_all();
+            }
+            mbar_arrive(stage_free);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, good, 0)) return false;
+      }
+      return true;
     };
 
     int h = kvh * group, qb = qb_first;  // head and query block of iteration it
@@ -718,7 +788,13 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           break;
         }
         tc_fence_after();
-        flush_dq(h_prev, q0_prev);
+        // the staging tile is this iteration's dS^T tile: wait until the TMA
+        // has read the second half too
+        if (!flush_dq(h_prev, q0_prev) || !mbar_wait_warp(stage_free, 1)) {
+          record_error(p.err, 420 + (it & 15));
+          ok = false;
+          break;
+        }
       }
       const int qc = q0 + qg * FB_QW;  // first query of this warp's columns
       const float* lse = p.LSE + ((int64_t)b * p.H + hq) * p.s + qc;
@@ -812,7 +888,10 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         ok = false;
       } else {
         tc_fence_after();
-        flush_dq(h_prev, q0_prev);
+        if (!flush_dq(h_prev, q0_prev)) {
+          record_error(p.err, 460);
+          ok = false;
+        }
       }
     }
     if (!ok) {
@@ -880,6 +959,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     }
   }
 
+  // the dQ reductions this CTA handed to the TMA complete before it exits
+  if (warp == 2 && lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -902,17 +983,21 @@ int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
     attr = true;
   }
   const int64_t T = (int64_t)a.b * a.s;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv, mo, mdq;
+  // dQ accumulator: fp32 [T, ldqa], tiles of 64 query rows x 128 head columns
+  // (the TMA reduction needs a 16-byte aligned base and a pitch of 4 floats)
+  if ((reinterpret_cast<uintptr_t>(a.dq_acc) & 15) || (a.ldqa % 4) || a.ldqa < (int64_t)a.H * FB_HD) return MT_ERR_ARG;
   if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * FB_HD, T, a.ldqkv, FB_BQ) ||
       !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
       !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
-      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ))
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ) ||
+      !make_tensor_map_2d_f32(&mdq, a.dq_acc, (int64_t)a.H * FB_HD, T, a.ldqa, FB_HD, FB_BQ / 2))
     return MT_ERR_ARG;
   const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
-             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
+             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0, (int)T};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
-  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
+  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, p);
   return launch_status();
 }
 

@@ -171,3 +171,37 @@ extern "C" size_t mt_host_state_bytes(const mt_config* cfg) {
   const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
   return common + ((size_t)(MT_GRAD_RING_SLOTS + mt::defer_layer_count(*cfg)) * layer_f + head_f) * gsz;
 }
+
+extern "C" int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard* out) {
+  if (!out || world < 1 || world > 1024 || rank < 0 || rank >= world) return MT_ERR_ARG;
+  if (mt::validate_config(cfg, nullptr) != MT_OK) return MT_ERR_CONFIG;
+  if (cfg->d % 128) return MT_ERR_CONFIG;  // fp32 and bf16 block offsets coincide only then
+  const mt::Layout y = mt::make_layout(*cfg);
+  const size_t lb = y.layer_begin(0), le = y.layer_end(0);
+  // The fp32 arena block of a layer and its bf16 streamed block must hold
+  // every tensor at the same element offset, so that one element range is one
+  // rank's share of the weights, of the gradients and of the update alike.
+  if (le - lb != y.bf_layer) return MT_ERR_CONFIG;
+  for (int tid = 0; tid < mt::kLayerTensors; ++tid)
+    if (y.t(0, tid).off - lb != y.bf_of(tid)) return MT_ERR_CONFIG;
+  const size_t head_elems = y.head.off + y.head.n - y.final_norm.off;
+  if (y.head.off - y.final_norm.off != (size_t)((cfg->d + 127) / 128 * 128)) return MT_ERR_CONFIG;
+  auto chunk = [&](size_t n) { return (n + (size_t)world * 128 - 1) / ((size_t)world * 128) * 128; };
+  auto part = [&](size_t n, size_t c, uint64_t* b, uint64_t* e) {
+    *b = std::min(n, (size_t)rank * c);
+    *e = std::min(n, (size_t)(rank + 1) * c);
+  };
+  memset(out, 0, sizeof(*out));
+  out->world = world;
+  out->rank = rank;
+  out->layer_elems = le - lb;
+  out->layer_chunk = chunk(le - lb);
+  part(le - lb, out->layer_chunk, &out->layer_begin, &out->layer_end);
+  out->head_elems = head_elems;
+  out->head_chunk = chunk(head_elems);
+  part(head_elems, out->head_chunk, &out->head_begin, &out->head_end);
+  const int rows = (cfg->V + world - 1) / world;
+  out->embed_row_begin = std::min(cfg->V, rank * rows);
+  out->embed_row_end = std::min(cfg->V, (rank + 1) * rows);
+  return MT_OK;
+}

@@ -338,6 +338,25 @@ def mt_get_stream(ctx: int) -> int:
     return st.value or 0
 
 
+class mt_shard(ctypes.Structure):
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32)] + \
+        [(n, ctypes.c_uint64) for n in ("layer_elems", "layer_chunk", "layer_begin", "layer_end",
+                                         "head_elems", "head_chunk", "head_begin", "head_end")] + \
+        [("embed_row_begin", ctypes.c_int32), ("embed_row_end", ctypes.c_int32)]
+
+    def as_dict(self):
+        return {n: getattr(self, n) for n, _ in self._fields_}
+
+
+_sig("mt_shard_plan", c_int, _cfgp, c_int, c_int, ctypes.POINTER(mt_shard))
+
+
+def mt_shard_plan(cfg: mt_config, world: int, rank: int) -> dict:
+    sp = mt_shard()
+    _check(lib.mt_shard_plan(ctypes.byref(cfg), world, rank, ctypes.byref(sp)), "mt_shard_plan")
+    return sp.as_dict()
+
+
 def mt_device_bytes(cfg: mt_config) -> int:
     return lib.mt_device_bytes(ctypes.byref(cfg))
 

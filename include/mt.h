@@ -198,6 +198,33 @@ size_t mt_host_state_bytes(const mt_config* cfg);
  * Only the boundary activations grow with L. No GPU needed. */
 size_t mt_device_bytes(const mt_config* cfg);
 
+/* Partition of the training state over `world` GPUs of one host that each
+ * train their own micro-batch through the same streamed layers (data-parallel
+ * sharded streaming: each GPU loads 1/world of every layer over its host link
+ * and all-gathers the rest from its peers, reduce-scatters the fp32 gradients
+ * and offloads only its own part, whose host AdamW it runs; the collectives
+ * are the all-gather and reduce-scatter that the pages contrast with
+ * MegaTrain's single-GPU streaming: intelligentliving.co, "Balancing Reduced
+ * Collective Communication with Weight Streaming Latency").
+ * A layer block (the floats of one decoder layer, from its attention-norm gain
+ * to the end of Wdown) holds every tensor at the same element offset in the
+ * fp32 arena and in the bf16 streamed block, so one element range is a rank's
+ * share of the weights it loads, of the summed gradients it receives and of
+ * the parameters it updates. Ranks own consecutive chunks of
+ * layer_chunk = ceil(layer_elems / (world * 128)) * 128 elements (256-byte
+ * aligned in bf16; the device slots are padded to world * layer_chunk, the
+ * last ranges clipped, possibly empty); the [final-norm gain | LM head] block
+ * is split the same way, and the embedding by rows. Requires d % 128 == 0
+ * (MT_ERR_CONFIG otherwise); MT_ERR_ARG for world < 1 or rank outside
+ * [0, world). Host-side arithmetic only. */
+typedef struct mt_shard {
+  int32_t world, rank;
+  uint64_t layer_elems, layer_chunk, layer_begin, layer_end; /* elements of a layer block; this rank's [begin, end) */
+  uint64_t head_elems, head_chunk, head_begin, head_end;     /* elements of the [final gain | head] block */
+  int32_t embed_row_begin, embed_row_end;                    /* embedding rows this rank updates */
+} mt_shard;
+int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard* out);
+
 /* Creates a context on cfg->device: the host-resident state and the small,
  * fixed device footprint of MegaTrain's memory-centric design (MegaTrain
  * abstract: GPUs are transient compute engines; saify.me, "The memory-centric
