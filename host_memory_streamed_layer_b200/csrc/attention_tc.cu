@@ -551,7 +551,10 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12);
   uint64_t* stage_full = bar + 13;  // [2] a 64-query half of dQ staged (8 warps each)
-  uint64_t* stage_free = bar + 15;  // the TMA has read a staged half (twice per block)
+  uint64_t* stage_free = bar + 15;  // [2] the TMA has read staged half 0 / half 1
+  // (each of the four completes exactly once per flush of dQ: flush f waits
+  // for parity f mod 2, never ambiguous because no barrier can run a phase
+  // ahead of a warp that has not taken part in the flush)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -577,7 +580,8 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     mbar_init(drain, 1);
     mbar_init(&stage_full[0], FB_GWARPS / 2);
     mbar_init(&stage_full[1], FB_GWARPS / 2);
-    mbar_init(stage_free, 1);
+    mbar_init(&stage_free[0], 1);
+    mbar_init(&stage_free[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmQ);
@@ -741,15 +745,15 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_empty);
       const int half = qg >> 1;
-      if (half == 1 && !mbar_wait_warp(stage_free, 0)) return false;  // the TMA has read half 0
+      const uint32_t par = (uint32_t)(nflush & 1);
+      ++nflush;
+      if (half == 1 && !mbar_wait_warp(&stage_free[0], par)) return false;  // the TMA has read half 0
       float* stg = reinterpret_cast<float*>(sdSt) + (qg & 1) * 32 * FB_HD + r;
 #pragma unroll
       for (int e = 0; e < FB_QW; ++e) stg[e * FB_HD] = __uint_as_float(v[e]) * p.scale;
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&stage_full[half]);
-      const uint32_t par = (uint32_t)(nflush & 1);
-      ++nflush;
       if (warp == 2) {
         int good = 1;
         if (lane == 0) {
@@ -764,7 +768,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
               bulk_commit_group();
               bulk_wait_read_all();
             }
-            mbar_arrive(stage_free);
+            mbar_arrive(&stage_free[h2]);
           }
         }
         if (!__shfl_sync(0xffffffffu, good, 0)) return false;
@@ -790,7 +794,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         tc_fence_after();
         // the staging tile is this iteration's dS^T tile: wait until the TMA
         // has read the second half too
-        if (!flush_dq(h_prev, q0_prev) || !mbar_wait_warp(stage_free, 1)) {
+        if (!flush_dq(h_prev, q0_prev) || !mbar_wait_warp(&stage_free[1], (uint32_t)((nflush - 1) & 1))) {
           record_error(p.err, 420 + (it & 15));
           ok = false;
           break;
