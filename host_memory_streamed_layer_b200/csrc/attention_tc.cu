@@ -85,21 +85,6 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// Element-wise fp32 add of a shared-memory tile into global memory by the TMA
-// engine (tensor map m, tile origin {c0 inner, c1 outer}); asynchronous, in a
-// bulk async-group of the issuing thread. No multicast.
-__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, const void* src, int c0, int c1) {
-  asm volatile("cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(m)),
-               "r"(smem_u32(src)), "r"(c0), "r"(c1)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-// Waits until the source of every committed bulk operation has been read.
-__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-// Waits until every committed bulk operation has completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
 template <int HD>
 __global__ void __launch_bounds__(FA_THREADS, 1)
     k_flash_fwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -295,75 +280,75 @@ __global__ void __launch_bounds__(FA_THREADS, 1)
       tmem_ld_32x32b_x32(sbase + (wg ^ 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(w));
       tmem_ld_32x32b_x32(sbase + (wg ^ 1) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(w + 32));
       tmem_ld_wait();
-      // The causal mask only touches the diagonal block (j == nkv - 1): row r
-      // sees keys [0, r] of it.
-      const bool diag = j == nkv - 1;
-      float mx = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < 64; ++e) {
-        const int cv = wg * 64 + e, cw = (wg ^ 1) * 64 + e;
-        if (!diag || cv <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
-        if (!diag || cw <= r) mx = fmaxf(mx, __uint_as_float(w[e]));
-      }
-      // Lazy maximum: raise it (and rescale O and l) only when the block's
-      // maximum exceeds the running one by more than 2^kRescaleLog2.
-      const bool raise = (m == -INFINITY) || (mx - m) * sl2 > kRescaleLog2;
-      const float corr = (raise && m != -INFINITY) ? ex2((m - mx) * sl2) : 1.f;
-      if (raise) m = mx;
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
-        // O holds blocks < j scaled by the old maximum: once P_{j-1} V_{j-1}
-        // has landed, multiply this warpgroup's columns of the raised rows.
-        const int pj = j - 1;
-        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[pj & 1], (pj >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int c = 0; c < HH / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld_32x32b_x32(obase + c * 32, o);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; e += 8) {
-            uint32_t t8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) t8[u] = __float_as_uint(__uint_as_float(o[e + u]) * corr);
-            tmem_st_32x32b_x8(obase + c * 32 + e, t8);
-          }
-        }
-        tmem_st_wait();
-        tc_fence_before();
-      }
-      l *= corr;
-      // The P buffer of this block was last read by P_{j-2} V_{j-2}.
-      if (j >= 2) {
-        const int pj = j - 2;
-        if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[pj & 1], (pj >> 1) & 1)) {
-          ok = false;
-          break;
-        }
-      }
-      // this warpgroup's 64 keys -> probabilities, partial row sum, bf16 P
-      // into swizzle sub-tile wg of the A operand
-      uint8_t* prow = sP + sb * C::P_BYTES + wg * 16384 + r * 128;
-      const float mb = m * sl2;
+      // The causal mask only touches the diagonal block (j == nkv - 1, row r
+      // sees keys [0, r] of it): the other blocks run an instantiation without
+      // any per-element test.
       float rs = 0.f;
+      auto block = [&](auto diag_tag) -> bool {
+        constexpr bool DIAG = decltype(diag_tag)::value;
+        float mx = -INFINITY;
 #pragma unroll
-      for (int chunk = 0; chunk < 8; ++chunk) {  // 16-byte chunks of 8 keys
-        uint32_t pk[4];
-#pragma unroll
-        for (int e = 0; e < 8; e += 2) {
-          const int k = chunk * 8 + e;
-          const int col = wg * 64 + k;
-          float p0 = ex2(fmaf(__uint_as_float(v[k]), sl2, -mb));
-          float p1 = ex2(fmaf(__uint_as_float(v[k + 1]), sl2, -mb));
-          if (diag && col > r) p0 = 0.f;
-          if (diag && col + 1 > r) p1 = 0.f;
-          rs += p0 + p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 64; ++e) {
+          if (!DIAG || wg * 64 + e <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
+          if (!DIAG || (wg ^ 1) * 64 + e <= r) mx = fmaxf(mx, __uint_as_float(w[e]));
         }
-        *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        // Lazy maximum: raise it (and rescale O and l) only when the block's
+        // maximum exceeds the running one by more than 2^kRescaleLog2.
+        const bool raise = (m == -INFINITY) || (mx - m) * sl2 > kRescaleLog2;
+        const float corr = (raise && m != -INFINITY) ? ex2((m - mx) * sl2) : 1.f;
+        if (raise) m = mx;
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          // O holds blocks < j scaled by the old maximum: once P_{j-1} V_{j-1}
+          // has landed, multiply this warpgroup's columns of the raised rows.
+          const int pj = j - 1;
+          if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[pj & 1], (pj >> 1) & 1)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < HH / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(obase + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t t8[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) t8[u] = __float_as_uint(__uint_as_float(o[e + u]) * corr);
+              tmem_st_32x32b_x8(obase + c * 32 + e, t8);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+        }
+        l *= corr;
+        // The P buffer of this block was last read by P_{j-2} V_{j-2}.
+        if (j >= 2) {
+          const int pj = j - 2;
+          if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&o_full[pj & 1], (pj >> 1) & 1)) return false;
+        }
+        // this warpgroup's 64 keys -> probabilities, partial row sum, bf16 P
+        // into swizzle sub-tile wg of the A operand
+        uint8_t* prow = sP + sb * C::P_BYTES + wg * 16384 + r * 128;
+        const float mb = m * sl2;
+#pragma unroll
+        for (int chunk = 0; chunk < 8; ++chunk) {  // 16-byte chunks of 8 keys
+          uint32_t pk[4];
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) {
+            const int k = chunk * 8 + e;
+            float p0 = ex2(fmaf(__uint_as_float(v[k]), sl2, -mb));
+            float p1 = ex2(fmaf(__uint_as_float(v[k + 1]), sl2, -mb));
+            if (DIAG && wg * 64 + k > r) p0 = 0.f;
+            if (DIAG && wg * 64 + k + 1 > r) p1 = 0.f;
+            rs += p0 + p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+        return true;
+      };
+      if (!(j == nkv - 1 ? block(std::true_type{}) : block(std::false_type{}))) {
+        ok = false;
+        break;
       }
       l += rs;
       tc_fence_before();
@@ -472,10 +457,8 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
 //          as their A operand; dS^T also into a 128-byte-swizzled shared tile)
 //   dV  += P^T dO,  dK += dS^T Q              (128 keys x hd, TMEM, A from TMEM)
 //   dQ^T = K^T dS^T                            (hd x 128 queries, into the
-//          dP^T columns), read out one head column per thread, staged as two
-//          64-query fp32 halves in the (then free) dS^T tile and added to the
-//          fp32 dQ accumulator by TMA bulk tensor reductions, which the L2
-//          performs while the warps go on with the next block's exponentials
+//          dP^T columns), read out one head column per thread and added to
+//          the fp32 dQ accumulator with global reductions from registers
 // Every product is N = 128 wide: 64-wide products run the tensor core at
 // little more than half rate (55 instead of 32 cycles per 128 x 64 x 16 MMA,
 // measured), which bounded the 64-query form of this kernel.
@@ -517,7 +500,6 @@ struct FbParams {
   const float* rsin;
   int* err;
   int vec_lse;  // LSE and D rows start 16-byte aligned: s % 4 == 0 and aligned bases
-  int T;        // tokens of all sequences: rows of the dQ accumulator
 };
 
 // Start-address step (address / 16) of k-step kk (16 elements of the
@@ -529,7 +511,7 @@ __device__ __forceinline__ uint32_t km_step(int kk) {
 __global__ void __launch_bounds__(FB_THREADS, 1)
     k_flash_bwd_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const __grid_constant__ CUtensorMap tmDQ, FbParams p) {
+                   FbParams p) {
   using C = FbCfg;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -550,11 +532,6 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
   uint64_t* drain = bar + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 11);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 12);
-  uint64_t* stage_full = bar + 13;  // [2] a 64-query half of dQ staged (8 warps each)
-  uint64_t* stage_free = bar + 15;  // [2] the TMA has read staged half 0 / half 1
-  // (each of the four completes exactly once per flush of dQ: flush f waits
-  // for parity f mod 2, never ambiguous because no barrier can run a phase
-  // ahead of a warp that has not taken part in the flush)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
@@ -578,17 +555,12 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     mbar_init(mma_done, 1);
     mbar_init(dq_empty, FB_GWARPS);
     mbar_init(drain, 1);
-    mbar_init(&stage_full[0], FB_GWARPS / 2);
-    mbar_init(&stage_full[1], FB_GWARPS / 2);
-    mbar_init(&stage_free[0], 1);
-    mbar_init(&stage_free[1], 1);
     *abort_flag = 0;
     fence_mbarrier_init();
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmO);
-    tma_prefetch_desc(&tmDQ);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, 512);
@@ -728,52 +700,23 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     bool ok = true;
 
     // dQ^T of an iteration (complete: the caller waited for mma_done): this
-    // warp's 32 query columns for head column r, scaled and written into the
-    // staging tile (the dS^T tile, which the dQ MMA has finished reading) as
-    // fp32 rows [query][head column] of its 64-query half; warp 2's lane 0
-    // hands each staged half to the TMA engine as one bulk tensor reduction
-    // into the fp32 dQ accumulator and releases the tile once the TMA has read
-    // it. Rows past the sequence end carry exact zeros (their dS is 0), so the
-    // add leaves whatever they overlap unchanged. Every wait is bounded;
-    // returns false after a wait ran out.
-    int nflush = 0;
-    auto flush_dq = [&](int hq, int q0) -> bool {
+    // warp's 32 query columns for head column r, added to the fp32 dQ
+    // accumulator with reductions from registers (a warp's 32 lanes are 32
+    // consecutive head columns of one query row: 128 coalesced bytes).
+    auto flush_dq = [&](int hq, int q0) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lane_base + C::C_DP + qg * FB_QW, v);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(dq_empty);
-      const int half = qg >> 1;
-      const uint32_t par = (uint32_t)(nflush & 1);
-      ++nflush;
-      if (half == 1 && !mbar_wait_warp(&stage_free[0], par)) return false;  // the TMA has read half 0
-      float* stg = reinterpret_cast<float*>(sdSt) + (qg & 1) * 32 * FB_HD + r;
+      const int qf = q0 + qg * FB_QW;
+      float* dst = p.dQacc + (int64_t)(row0 + qf) * p.ldqa + (int64_t)hq * FB_HD + r;
 #pragma unroll
-      for (int e = 0; e < FB_QW; ++e) stg[e * FB_HD] = __uint_as_float(v[e]) * p.scale;
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&stage_full[half]);
-      if (warp == 2) {
-        int good = 1;
-        if (lane == 0) {
-          for (int h2 = 0; h2 < 2; ++h2) {
-            if (!mbar_wait(&stage_full[h2], par)) {
-              good = 0;
-              break;
-            }
-            // (a half that starts past the last token has nothing to add)
-            if (row0 + q0 + 64 * h2 < p.T) {
-              tma_reduce_add_2d(&tmDQ, sdSt, hq * FB_HD, row0 + q0 + 64 * h2);
-              bulk_commit_group();
-              bulk_wait_read_all();
-            }
-            mbar_arrive(&stage_free[h2]);
-          }
-        }
-        if (!__shfl_sync(0xffffffffu, good, 0)) return false;
-      }
-      return true;
+      for (int e = 0; e < FB_QW; ++e)
+        if (qf + e < p.s)
+          asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst + (int64_t)e * p.ldqa), "f"(__uint_as_float(v[e]) * p.scale)
+                       : "memory");
     };
 
     int h = kvh * group, qb = qb_first;  // head and query block of iteration it
@@ -792,13 +735,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           break;
         }
         tc_fence_after();
-        // the staging tile is this iteration's dS^T tile: wait until the TMA
-        // has read the second half too
-        if (!flush_dq(h_prev, q0_prev) || !mbar_wait_warp(&stage_free[1], (uint32_t)((nflush - 1) & 1))) {
-          record_error(p.err, 420 + (it & 15));
-          ok = false;
-          break;
-        }
+        flush_dq(h_prev, q0_prev);
       }
       const int qc = q0 + qg * FB_QW;  // first query of this warp's columns
       const float* lse = p.LSE + ((int64_t)b * p.H + hq) * p.s + qc;
@@ -892,10 +829,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         ok = false;
       } else {
         tc_fence_after();
-        if (!flush_dq(h_prev, q0_prev)) {
-          record_error(p.err, 460);
-          ok = false;
-        }
+        flush_dq(h_prev, q0_prev);
       }
     }
     if (!ok) {
@@ -963,8 +897,6 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     }
   }
 
-  // the dQ reductions this CTA handed to the TMA complete before it exits
-  if (warp == 2 && lane == 0) bulk_wait_all();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -987,21 +919,17 @@ int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
     attr = true;
   }
   const int64_t T = (int64_t)a.b * a.s;
-  CUtensorMap mq, mk, mv, mo, mdq;
-  // dQ accumulator: fp32 [T, ldqa], tiles of 64 query rows x 128 head columns
-  // (the TMA reduction needs a 16-byte aligned base and a pitch of 4 floats)
-  if ((reinterpret_cast<uintptr_t>(a.dq_acc) & 15) || (a.ldqa % 4) || a.ldqa < (int64_t)a.H * FB_HD) return MT_ERR_ARG;
+  CUtensorMap mq, mk, mv, mo;
   if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * FB_HD, T, a.ldqkv, FB_BQ) ||
       !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
       !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
-      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ) ||
-      !make_tensor_map_2d_f32(&mdq, a.dq_acc, (int64_t)a.H * FB_HD, T, a.ldqa, FB_HD, FB_BQ / 2))
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ))
     return MT_ERR_ARG;
   const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
-             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0, (int)T};
+             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
-  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, mdq, p);
+  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
 
