@@ -64,6 +64,8 @@ def parse():
     ap.add_argument("--grads", default="ring", choices=["ring", "arena"],
                     help="host gradients: ring of layer slots (14 B/param of host memory) or a full arena (18)")
     ap.add_argument("--host-threads", type=int, default=0, help="host optimizer threads per replica (0: cores / N)")
+    ap.add_argument("--offload-acts", action="store_true",
+                    help="keep the boundary activations in pinned host memory (MT_FLAG_OFFLOAD_ACTS)")
     ap.add_argument("--grad-dtype", default="fp32", choices=["fp32", "bf16"],
                     help="dtype of the offloaded gradients (bf16: MT_FLAG_BF16_GRADS, a measured variant)")
     ap.add_argument("--no-defer", action="store_true",
@@ -587,7 +589,8 @@ def main():
     # (MT_FLAG_DEFER_UPDATES), when the host optimizer is otherwise idle.
     cfg.flags = (mt.MT_FLAG_KERNEL_TIMING | (mt.MT_FLAG_GRAD_RING if args.grads == "ring" else 0) |
                  (0 if args.no_defer else mt.MT_FLAG_DEFER_UPDATES) |
-                 (mt.MT_FLAG_BF16_GRADS if args.grad_dtype == "bf16" else 0))
+                 (mt.MT_FLAG_BF16_GRADS if args.grad_dtype == "bf16" else 0) |
+                 (mt.MT_FLAG_OFFLOAD_ACTS if args.offload_acts else 0))
     ncpu = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cfg.host_threads = args.host_threads or max(1, ncpu // world)
 
@@ -700,6 +703,7 @@ def main():
                        "deferred_updates": (None if args.no_defer else
                                             f"LM head + last {defer_layers(sh)} layer(s) updated during the next "
                                             "forward sweep; the timed region ends after mt_flush"),
+                       "boundary_activations": "pinned host memory" if args.offload_acts else "HBM",
                        "grads": (f"{args.grad_dtype} gradients offloaded; " +
                                  (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
                                   if args.grads == "ring" else "full gradient arena in pinned host memory"))},

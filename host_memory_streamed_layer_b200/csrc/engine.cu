@@ -133,7 +133,12 @@ struct mt_ctx {
   uint16_t* d_head_g16 = nullptr;
   uint16_t* d_head_w = nullptr;  // [gf | Whead] bf16
   float* d_head_g = nullptr;     // [dgf | dWhead] fp32
-  float* xb = nullptr;           // boundary activations [(L+1), T, d]
+  float* xb = nullptr;           // boundary activations [(L+1), T, d], or 3 slots with MT_FLAG_OFFLOAD_ACTS
+  // MT_FLAG_OFFLOAD_ACTS: x_0 .. x_{L-3} in pinned host memory, moved on their
+  // own stream; per boundary l: offloaded (or copied to slot 2), brought back
+  float* xh = nullptr;
+  cudaStream_t s_act = nullptr;
+  std::vector<cudaEvent_t> ev_xready, ev_xout, ev_xin, ev_bwdone;
   uint16_t *u_b, *qkv_b, *ao_b, *w_b, *gu_b, *act_b, *gxb, *dact_b, *dgu_b, *dhb, *dao_b, *dqkv_b, *n_b, *dz_b;
   float *lse, *h_f, *r1, *r2, *gx0, *gx1, *tmp_f, *dh_f, *dvec, *dqacc, *rms_part, *rf, *logits, *rowloss;
   int32_t *d_tok, *d_lab, *d_offs, *d_pos, *d_flags, *d_err;
@@ -314,15 +319,36 @@ int check_finite(mt_ctx* c, const float* g, size_t n, int idx) {
 }
 
 // ---------------------------------------------------------------------------
-// Layer forward from x = xb[l] with the weights of `slot`. With keep_out the
-// layer output goes to xb[l+1]; otherwise (recompute) the down projection is
-// skipped, since the backward only needs the intermediates.
+// Boundary activations on the device. Resident: x_l at xb[l]. With
+// MT_FLAG_OFFLOAD_ACTS three [T, d] slots: the forward alternates slots 0 and
+// 1 (x_l in slot l mod 2, so x_L also follows that rule); in the backward, x_{L-1} is
+// still in its forward slot and x_l for l <= L-2 (brought back from host
+// memory, x_{L-2} by a device copy) alternates between slot 2 and slot
+// (L-1) mod 2, so that x_{l-1} can load while layer l runs.
 // ---------------------------------------------------------------------------
-int layer_fwd(mt_ctx* c, int l, int slot, bool keep_out) {
+bool offload_acts(const mt_ctx* c) { return (c->cfg.flags & MT_FLAG_OFFLOAD_ACTS) != 0; }
+
+float* x_fwd(mt_ctx* c, int l) {
+  const size_t n = (size_t)c->lay.sh.T * c->lay.sh.d;
+  return c->xb + (offload_acts(c) ? (size_t)(l & 1) : (size_t)l) * n;
+}
+
+float* x_bwd(mt_ctx* c, int l) {
+  const int L = c->lay.sh.L;
+  if (!offload_acts(c) || l == L - 1) return x_fwd(c, l);
+  const size_t n = (size_t)c->lay.sh.T * c->lay.sh.d;
+  return c->xb + (size_t)(((L - 2 - l) % 2 == 0) ? 2 : ((L - 1) & 1)) * n;
+}
+
+// ---------------------------------------------------------------------------
+// Layer forward from x with the weights of `slot`. With xo the layer output
+// goes there; otherwise (recompute) the down projection is skipped, since the
+// backward only needs the intermediates.
+// ---------------------------------------------------------------------------
+int layer_fwd(mt_ctx* c, int l, int slot, const float* x, float* xo) {
   const Shapes& s = c->lay.sh;
   const Layout& y = c->lay;
   const uint16_t* W = c->wslot[slot];
-  const float* x = c->xb + (size_t)l * s.T * s.d;
   cudaStream_t st = c->s_comp;
   KL(launch_rmsnorm_fwd(x, W + y.bf_g1, c->u_b, c->r1, s.T, s.d, c->cfg.norm_eps, st), 1);
   {
@@ -350,22 +376,19 @@ int layer_fwd(mt_ctx* c, int l, int slot, bool keep_out) {
   KL(launch_rmsnorm_fwd(c->h_f, W + y.bf_g2, c->w_b, c->r2, s.T, s.d, c->cfg.norm_eps, st), 1);
   CKM(gemm(c, gd_fwd(c->w_b, s.d, W + y.bf_gu, s.d, c->gu_b, 2 * s.F, EPI_BF16, nullptr, s.T, 2 * s.F, s.d)));
   KL(launch_swiglu_fwd(c->gu_b, c->act_b, s.T, s.F, st), 1);
-  if (keep_out) {
-    float* xo = c->xb + (size_t)(l + 1) * s.T * s.d;
-    CKM(gemm(c, gd_fwd(c->act_b, s.F, W + y.bf_d, s.F, xo, s.d, EPI_F32_ADD, c->h_f, s.T, s.d, s.F)));
-  }
+  if (xo) CKM(gemm(c, gd_fwd(c->act_b, s.F, W + y.bf_d, s.F, xo, s.d, EPI_F32_ADD, c->h_f, s.T, s.d, s.F)));
   return MT_OK;
 }
 
-// Layer backward: gin = dL/dx_{l+1} (fp32), writes gout = dL/dx_l and the
-// layer's fp32 gradients into grad slot gs (arena layout of the layer).
-int layer_bwd(mt_ctx* c, int l, int slot, float* gs, const float* gin, float* gout) {
+// Layer backward from its input x: gin = dL/dx_{l+1} (fp32), writes gout =
+// dL/dx_l and the layer's fp32 gradients into grad slot gs (arena layout of
+// the layer).
+int layer_bwd(mt_ctx* c, int l, int slot, const float* x, float* gs, const float* gin, float* gout) {
   const Shapes& s = c->lay.sh;
   const Layout& y = c->lay;
   const uint16_t* W = c->wslot[slot];
   const size_t base = y.layer_begin(l);
   auto G = [&](int tid) { return gs + (y.t(l, tid).off - base); };
-  const float* x = c->xb + (size_t)l * s.T * s.d;
   cudaStream_t st = c->s_comp;
   const int T = s.T, d = s.d, F = s.F;
 
@@ -429,7 +452,7 @@ int head_step(mt_ctx* c, float* gout) {
   const uint16_t* Wh = c->d_head_w + align_up(d, 128);
   float* dgf = c->d_head_g;
   float* dWh = c->d_head_g + gf_pad;
-  const float* xL = c->xb + (size_t)s.L * T * d;
+  const float* xL = x_fwd(c, s.L);
   KL(launch_rmsnorm_fwd(xL, gf, c->n_b, c->rf, T, d, c->cfg.norm_eps, st), 1);
   for (int t0 = 0; t0 < T; t0 += c->Tc) {
     const int tc = std::min(c->Tc, T - t0);
@@ -848,6 +871,35 @@ int offload_layer(mt_ctx* c, int l, int k) {
   return MT_OK;
 }
 
+// MT_FLAG_OFFLOAD_ACTS, forward: x_l (just written on the compute stream)
+// leaves the slot that x_{l+2} takes: to host memory for l <= L-3, by a device
+// copy into slot 2 for l = L-2 (the first layer recomputed). ev_xout[l]: done.
+int stash_act(mt_ctx* c, int l) {
+  const int L = c->lay.sh.L;
+  if (!offload_acts(c) || l > L - 2) return MT_OK;
+  const size_t n = (size_t)c->lay.sh.T * c->lay.sh.d;
+  CK(cudaEventRecord(c->ev_xready[l], c->s_comp));
+  CK(cudaStreamWaitEvent(c->s_act, c->ev_xready[l], 0));
+  if (l == L - 2)
+    CK(cudaMemcpyAsync(x_bwd(c, l), x_fwd(c, l), n * 4, cudaMemcpyDeviceToDevice, c->s_act));
+  else
+    CK(cudaMemcpyAsync(c->xh + (size_t)l * n, x_fwd(c, l), n * 4, cudaMemcpyDeviceToHost, c->s_act));
+  CK(cudaEventRecord(c->ev_xout[l], c->s_act));
+  return MT_OK;
+}
+
+// Backward: x_l (l <= L-3) back from host memory into its backward slot, once
+// the slot's last user, layer l+2's backward, is done. ev_xin[l]: landed.
+int fetch_act(mt_ctx* c, int l) {
+  const int L = c->lay.sh.L;
+  if (!offload_acts(c) || l < 0 || l > L - 3) return MT_OK;
+  const size_t n = (size_t)c->lay.sh.T * c->lay.sh.d;
+  CK(cudaStreamWaitEvent(c->s_act, c->ev_bwdone[l + 2], 0));
+  CK(cudaMemcpyAsync(x_bwd(c, l), c->xh + (size_t)l * n, n * 4, cudaMemcpyHostToDevice, c->s_act));
+  CK(cudaEventRecord(c->ev_xin[l], c->s_act));
+  return MT_OK;
+}
+
 int enqueue_step(mt_ctx* c, int n_unique) {
   const Layout& y = c->lay;
   const Shapes& s = y.sh;
@@ -858,7 +910,8 @@ int enqueue_step(mt_ctx* c, int n_unique) {
   CK(cudaEventRecord(c->ev_step_start, sc));
   CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));  // error word of this step's kernels
   CK(cudaMemcpyAsync(c->d_tok, c->stage_i, (size_t)(4 * T + 1) * 4, cudaMemcpyHostToDevice, sc));
-  KL(launch_embed_fwd(c->d_tok, c->bf_embed_dev, c->xb, T, d, sc), 1);
+  KL(launch_embed_fwd(c->d_tok, c->bf_embed_dev, x_fwd(c, 0), T, d, sc), 1);
+  CKM(stash_act(c, 0));
   CKM(issue_load(c, 0));
   if (nloads > 1) CKM(issue_load(c, 1));
   if (L == 1) CKM(issue_head_load(c));
@@ -871,7 +924,10 @@ int enqueue_step(mt_ctx* c, int n_unique) {
     CK(cudaStreamWaitEvent(sc, c->ev_wready[i], 0));
     if (i < L) {
       const int l = i;
-      CKM(layer_fwd(c, l, slot, true));
+      // with offloaded activations x_{l+1} takes the slot of x_{l-1}
+      if (offload_acts(c) && l >= 1) CK(cudaStreamWaitEvent(sc, c->ev_xout[l - 1], 0));
+      CKM(layer_fwd(c, l, slot, x_fwd(c, l), x_fwd(c, l + 1)));
+      CKM(stash_act(c, l + 1));
       if (l == L - 1) {
         CK(cudaEventRecord(c->ev_fwd_end, sc));
         CK(cudaStreamWaitEvent(sc, c->ev_head_wready, 0));
@@ -893,18 +949,27 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         push_job(c, hj);
         CK(cudaEventRecord(c->ev_head_end, sc));
         // backward of the last layer: its intermediates are still in the workspace
-        CKM(layer_bwd(c, l, slot, c->gslot[0], gin, gout));
+        CKM(layer_bwd(c, l, slot, x_bwd(c, l), c->gslot[0], gin, gout));
         CKM(offload_layer(c, l, 0));
         std::swap(gin, gout);
+        if (offload_acts(c)) {
+          CK(cudaEventRecord(c->ev_bwdone[l], sc));
+          CKM(fetch_act(c, l - 2));
+        }
       }
     } else {
       const int k = i - (L - 1);  // backward index: layer L-1-k
       const int l = L - 1 - k;
       if (k >= 2) CK(cudaStreamWaitEvent(sc, c->ev_gdrained[k - 2], 0));
-      CKM(layer_fwd(c, l, slot, false));
-      CKM(layer_bwd(c, l, slot, c->gslot[k & 1], gin, gout));
+      if (offload_acts(c)) CK(cudaStreamWaitEvent(sc, l == L - 2 ? c->ev_xout[l] : c->ev_xin[l], 0));
+      CKM(layer_fwd(c, l, slot, x_bwd(c, l), nullptr));
+      CKM(layer_bwd(c, l, slot, x_bwd(c, l), c->gslot[k & 1], gin, gout));
       CKM(offload_layer(c, l, k));
       std::swap(gin, gout);
+      if (offload_acts(c)) {
+        CK(cudaEventRecord(c->ev_bwdone[l], sc));
+        CKM(fetch_act(c, l - 2));
+      }
     }
     CK(cudaEventRecord(c->ev_slotfree[i], sc));
     // The head's weights follow the last forward load on the H2D stream, ahead
@@ -958,10 +1023,12 @@ void collect_stats(mt_ctx* c) {
   st.d2h_ms = d2h;
   st.wait_weights_ms = wait;
   const Layout& y = c->lay;
-  st.h2d_bytes = (double)c->load_seq.size() * y.bf_layer * 2 +
+  const double act_bytes = offload_acts(c) && L >= 3 ? 4.0 * (L - 2) * y.sh.T * y.sh.d : 0.0;
+  st.h2d_bytes = act_bytes + (double)c->load_seq.size() * y.bf_layer * 2 +
                  (double)(align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d) * 2 + 4.0 * (4 * y.sh.T + 1) +
                  (double)y.sh.T * y.sh.d * 2;  // embedding rows read in place
-  st.d2h_bytes = (double)c->gsz * (y.head.off + y.head.n - y.final_norm.off) + 4.0 * c->uniq.size() * y.sh.d + 12.0;
+  st.d2h_bytes = act_bytes + (double)c->gsz * (y.head.off + y.head.n - y.final_norm.off) +
+                 4.0 * c->uniq.size() * y.sh.d + 12.0;
   for (int l = 0; l < L; ++l) st.d2h_bytes += (double)c->gsz * (y.layer_end(l) - y.layer_begin(l));
   st.adamw_ms = c->adamw_s * 1e3;
   st.adamw_bytes = c->adamw_bytes;
@@ -985,7 +1052,7 @@ void collect_stats(mt_ctx* c) {
 // ---------------------------------------------------------------------------
 // Create / destroy helpers.
 // ---------------------------------------------------------------------------
-size_t device_bytes(const Layout& y, int Tc, bool g16) {
+size_t device_bytes(const Layout& y, int Tc, bool g16, bool offload) {
   const Shapes& s = y.sh;
   const size_t T = s.T, d = s.d, F = s.F, V = s.V;
   const size_t A = 256;
@@ -1003,7 +1070,7 @@ size_t device_bytes(const Layout& y, int Tc, bool g16) {
     add(lay_f * 2);
     add((y.head.off - y.final_norm.off + V * d) * 2);
   }
-  add((size_t)(s.L + 1) * T * d * 4);                       // boundary activations
+  add((size_t)(offload ? std::min(s.L + 1, 3) : s.L + 1) * T * d * 4);  // boundary activations
   add(T * d * 2);                                           // u
   add(T * (size_t)s.Nqkv * 2);                              // qkv
   add(T * (size_t)s.Hd * 2);                                // attention output
@@ -1063,7 +1130,7 @@ void free_all(mt_ctx* c) {
     c->opt_thread.join();
   }
   cudaSetDevice(c->device);
-  for (cudaStream_t s : {c->s_h2d, c->s_comp, c->s_d2h})
+  for (cudaStream_t s : {c->s_h2d, c->s_comp, c->s_d2h, c->s_act})
     if (s) cudaStreamSynchronize(s);
   auto kill = [](std::vector<cudaEvent_t>& v) {
     for (auto e : v)
@@ -1078,6 +1145,10 @@ void free_all(mt_ctx* c) {
   kill(c->ev_d2h_start);
   kill(c->ev_gdrained);
   kill(c->ev_timing);
+  kill(c->ev_xready);
+  kill(c->ev_xout);
+  kill(c->ev_xin);
+  kill(c->ev_bwdone);
   for (cudaEvent_t e : {c->ev_head_h2d_start, c->ev_head_wready, c->ev_head_gready, c->ev_head_d2h_start,
                         c->ev_head_drained, c->ev_emb_ready, c->ev_emb_d2h_start, c->ev_emb_drained,
                         c->ev_step_start, c->ev_fwd_end, c->ev_head_end, c->ev_bwd_end, c->ev_step_end})
@@ -1086,11 +1157,12 @@ void free_all(mt_ctx* c) {
   if (c->s_comp) cudaStreamDestroy(c->s_comp);
   if (c->s_h2d && c->s_h2d != c->s_comp) cudaStreamDestroy(c->s_h2d);
   if (c->s_d2h && c->s_d2h != c->s_comp && c->s_d2h != c->s_h2d) cudaStreamDestroy(c->s_d2h);
+  if (c->s_act && c->s_act != c->s_comp) cudaStreamDestroy(c->s_act);
   if (c->dmem) cudaFree(c->dmem);
   for (void* p : {(void*)c->grad, (void*)c->ring, (void*)c->defer_g, (void*)(c->grad ? nullptr : c->grad_head),
                   (void*)c->bf_layers,
                   (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h, (void*)c->stage_i, (void*)c->flags_h,
-                  (void*)c->misc_h})
+                  (void*)c->misc_h, (void*)c->xh})
     if (p) cudaFreeHost(p);
   free(c->m);
   free(c->v);
@@ -1122,7 +1194,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   if (major != 10 || minor != 0) return set_err(nullptr, MT_ERR_CUDA, "this library runs on sm_100 (B200) only");
 
   const int Tc = logits_chunk(s);
-  const size_t need = device_bytes(y, Tc, (cfg->flags & MT_FLAG_BF16_GRADS) != 0);
+  const size_t need =
+      device_bytes(y, Tc, (cfg->flags & MT_FLAG_BF16_GRADS) != 0, (cfg->flags & MT_FLAG_OFFLOAD_ACTS) != 0);
   size_t free_b = 0, total_b = 0;
   if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaMemGetInfo failed");
   if (need + ((size_t)256 << 20) > free_b) {
@@ -1198,6 +1271,10 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     return fail(MT_ERR_PIN, "pinned host allocation failed");
   if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->bf_embed_dev), c->bf_embed, 0) != cudaSuccess)
     return fail(MT_ERR_PIN, "embedding table not mapped for device access");
+  if ((cfg->flags & MT_FLAG_OFFLOAD_ACTS) && s.L >= 3 &&
+      cudaHostAlloc(reinterpret_cast<void**>(&c->xh), (size_t)(s.L - 2) * s.T * s.d * 4, cudaHostAllocPortable) !=
+          cudaSuccess)
+    return fail(MT_ERR_PIN, "pinned boundary-activation allocation failed");
   // Initialise (owned arena from seed), zero moments and gradients (parallel first touch).
   if (c->arena_owned) {
     auto fill = [&](const TRef& r, uint64_t key, bool gain) {
@@ -1267,7 +1344,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     c->gslot16[1] = (uint16_t*)carve(lay_f * 2);
     c->d_head_g16 = (uint16_t*)carve((y.head.off - y.final_norm.off + V * d) * 2);
   }
-  c->xb = (float*)carve((size_t)(s.L + 1) * T * d * 4);
+  c->xb = (float*)carve((size_t)((cfg->flags & MT_FLAG_OFFLOAD_ACTS) ? std::min(s.L + 1, 3) : s.L + 1) * T * d * 4);
   c->u_b = (uint16_t*)carve(T * d * 2);
   c->qkv_b = (uint16_t*)carve(T * (size_t)s.Nqkv * 2);
   c->ao_b = (uint16_t*)carve(T * (size_t)s.Hd * 2);
@@ -1324,11 +1401,12 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   if (cfg->flags & MT_FLAG_SERIALIZE) {
     if (cudaStreamCreateWithFlags(&c->s_comp, cudaStreamNonBlocking) != cudaSuccess)
       return fail(MT_ERR_CUDA, "stream");
-    c->s_h2d = c->s_d2h = c->s_comp;
+    c->s_h2d = c->s_d2h = c->s_act = c->s_comp;
   } else {
     if (cudaStreamCreateWithFlags(&c->s_comp, cudaStreamNonBlocking) != cudaSuccess ||
         cudaStreamCreateWithFlags(&c->s_h2d, cudaStreamNonBlocking) != cudaSuccess ||
-        cudaStreamCreateWithFlags(&c->s_d2h, cudaStreamNonBlocking) != cudaSuccess)
+        cudaStreamCreateWithFlags(&c->s_d2h, cudaStreamNonBlocking) != cudaSuccess ||
+        ((cfg->flags & MT_FLAG_OFFLOAD_ACTS) && cudaStreamCreateWithFlags(&c->s_act, cudaStreamNonBlocking) != cudaSuccess))
       return fail(MT_ERR_CUDA, "stream");
   }
   // weight loads: 0..L-1 then L-2..0 (layer L-1 stays resident over the turn)
@@ -1344,6 +1422,9 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   bool ok = mk(c->ev_wready, nloads) && mk(c->ev_compready, nloads) && mk(c->ev_h2d_start, nloads) &&
             mk(c->ev_slotfree, nloads) && mk(c->ev_gready, s.L) && mk(c->ev_d2h_start, s.L) &&
             mk(c->ev_gdrained, s.L);
+  if (cfg->flags & MT_FLAG_OFFLOAD_ACTS)
+    ok = ok && mk(c->ev_xready, s.L + 1) && mk(c->ev_xout, s.L + 1) && mk(c->ev_xin, s.L + 1) &&
+         mk(c->ev_bwdone, s.L + 1);
   for (cudaEvent_t* e : {&c->ev_head_h2d_start, &c->ev_head_wready, &c->ev_head_gready, &c->ev_head_d2h_start,
                          &c->ev_head_drained, &c->ev_emb_ready, &c->ev_emb_d2h_start, &c->ev_emb_drained,
                          &c->ev_step_start, &c->ev_fwd_end, &c->ev_head_end, &c->ev_bwd_end, &c->ev_step_end})
@@ -1468,11 +1549,11 @@ extern "C" int mt_layer_fwd_bwd(mt_ctx* c, int l, const float* x_in, const float
   CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));
   // the layer's streamed bf16 weights into slot 0, x_l into its boundary slot
   CK(cudaMemcpyAsync(c->wslot[0], c->bf_layers + (size_t)l * y.bf_layer, y.bf_layer * 2, cudaMemcpyHostToDevice, sc));
-  CK(cudaMemcpyAsync(c->xb + (size_t)l * n, x_in, n * 4, cudaMemcpyHostToDevice, sc));
+  CK(cudaMemcpyAsync(x_fwd(c, l), x_in, n * 4, cudaMemcpyHostToDevice, sc));
   CK(cudaMemcpyAsync(c->gx0, dx_out, n * 4, cudaMemcpyHostToDevice, sc));
-  CKM(layer_fwd(c, l, 0, true));
-  CKM(layer_bwd(c, l, 0, c->gslot[0], c->gx0, c->gx1));
-  CK(cudaMemcpyAsync(x_out, c->xb + (size_t)(l + 1) * n, n * 4, cudaMemcpyDeviceToHost, sc));
+  CKM(layer_fwd(c, l, 0, x_fwd(c, l), x_fwd(c, l + 1)));
+  CKM(layer_bwd(c, l, 0, x_fwd(c, l), c->gslot[0], c->gx0, c->gx1));
+  CK(cudaMemcpyAsync(x_out, x_fwd(c, l + 1), n * 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaMemcpyAsync(dx_in, c->gx1, n * 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaMemcpyAsync(grads, c->gslot[0], c->layer_f * 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
@@ -1503,7 +1584,7 @@ extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* label
   const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
   CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));
   CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, head_bf * 2, cudaMemcpyHostToDevice, sc));
-  CK(cudaMemcpyAsync(c->xb + (size_t)s.L * n, x_L, n * 4, cudaMemcpyHostToDevice, sc));
+  CK(cudaMemcpyAsync(x_fwd(c, s.L), x_L, n * 4, cudaMemcpyHostToDevice, sc));
   CK(cudaMemcpyAsync(c->d_lab, labels, (size_t)s.T * 4, cudaMemcpyHostToDevice, sc));
   CKM(head_step(c, c->gx0));
   CK(cudaMemcpyAsync(c->misc_h, c->d_loss, 4, cudaMemcpyDeviceToHost, sc));
@@ -1646,7 +1727,8 @@ extern "C" int mt_get_stream(mt_ctx* c, void** stream) {
 extern "C" size_t mt_device_bytes(const mt_config* cfg) {
   if (validate_config(cfg, nullptr) != MT_OK) return 0;
   const Layout y = make_layout(*cfg);
-  return device_bytes(y, logits_chunk(y.sh), (cfg->flags & MT_FLAG_BF16_GRADS) != 0);
+  return device_bytes(y, logits_chunk(y.sh), (cfg->flags & MT_FLAG_BF16_GRADS) != 0,
+                      (cfg->flags & MT_FLAG_OFFLOAD_ACTS) != 0);
 }
 
 namespace {

@@ -166,10 +166,13 @@ extern "C" size_t mt_host_state_bytes(const mt_config* cfg) {
   const size_t bf = (size_t)y.sh.L * y.bf_layer + 2 * (size_t)y.sh.V * y.sh.d + y.sh.d + 256;
   const size_t common = P * 4 * 2 + bf * 2 + (size_t)y.sh.T * y.sh.d * 4;  // m, v; bf16 copy; embedding staging
   const size_t gsz = (cfg->flags & MT_FLAG_BF16_GRADS) ? 2 : 4;           // bytes per host gradient element
-  if (!(cfg->flags & MT_FLAG_GRAD_RING)) return common + P * gsz;        // whole gradient arena
+  const size_t acts = ((cfg->flags & MT_FLAG_OFFLOAD_ACTS) && y.sh.L >= 3)  // x_0 .. x_{L-3}, fp32
+                          ? (size_t)(y.sh.L - 2) * y.sh.T * y.sh.d * 4
+                          : 0;
+  if (!(cfg->flags & MT_FLAG_GRAD_RING)) return acts + common + P * gsz;  // whole gradient arena
   const size_t layer_f = y.layer_end(0) - y.layer_begin(0);
   const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
-  return common + ((size_t)(MT_GRAD_RING_SLOTS + mt::defer_layer_count(*cfg)) * layer_f + head_f) * gsz;
+  return acts + common + ((size_t)(MT_GRAD_RING_SLOTS + mt::defer_layer_count(*cfg)) * layer_f + head_f) * gsz;
 }
 
 extern "C" int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard* out) {

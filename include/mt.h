@@ -101,6 +101,18 @@ extern "C" {
  * link-versus-accuracy variant: the method's own design offloads the
  * gradients in full precision (MegaTrain abstract: full-precision training). */
 #define MT_FLAG_BF16_GRADS 0x20u
+/* Keep the layer-boundary activations in pinned host memory instead of HBM:
+ * during the forward, x_0 .. x_{L-3} (fp32 [b*s, d] each) are copied to host
+ * memory on a stream of their own as soon as they are produced, x_{L-2} moves
+ * to a third device slot, and in the backward each x_l returns to the device
+ * while layer l+1 computes. The device then holds three boundary slots
+ * instead of L+1 (mt_device_bytes), which is what lets the context grow
+ * (MegaTrain abstract: 7B at 512k tokens on one GH200; saify.me, "Who this is
+ * actually for": ultra-long context as a side effect of the layer-wise
+ * design), at the cost of 2 (L-2) b s d 4 bytes more over the host link per
+ * step and (L-2) b s d 4 bytes of pinned host memory (mt_host_state_bytes).
+ * The arithmetic is unchanged: every copy is exact. */
+#define MT_FLAG_OFFLOAD_ACTS 0x40u
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0
@@ -185,7 +197,10 @@ int mt_tensor_offset(const mt_config* cfg, int layer, int tensor_id, size_t* off
  * the embedding-gradient rows, plus the fp32 gradients: the whole gradient
  * arena (4 B/param), or with MT_FLAG_GRAD_RING in cfg->flags the ring of
  * MT_GRAD_RING_SLOTS layer slots and the final-norm + LM-head gradient (and,
- * with MT_FLAG_DEFER_UPDATES too, MT_DEFER_LAYERS more layer slots). */
+ * with MT_FLAG_DEFER_UPDATES too, MT_DEFER_LAYERS more layer slots); with
+ * MT_FLAG_BF16_GRADS the gradient buffers are bf16 (2 B per element); with
+ * MT_FLAG_OFFLOAD_ACTS also the (L-2) offloaded fp32 [b*s, d] boundary
+ * activations. */
 size_t mt_host_state_bytes(const mt_config* cfg);
 
 /* Device bytes mt_create allocates for cfg, in one allocation, 0 for a bad

@@ -333,3 +333,22 @@ def test_device_bytes_grow_only_by_the_boundary_activations():
         assert sizes[1] > 2 * 2 * P_layer + 2 * 4 * P_layer + 3 * T * d * 4
     bad = arena.config(dict(L=2, d=100, H=2, Hkv=2, F=64, V=64, b=1, s=8))
     assert mt.mt_device_bytes(bad) == 0
+
+
+def test_offloaded_activations_keep_three_device_slots():
+    """MT_FLAG_OFFLOAD_ACTS: the device footprint no longer grows with L (three
+    boundary slots), and the host state grows by the L-2 offloaded fp32
+    [b*s, d] boundary activations."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    base = dict(d=1024, H=8, Hkv=8, F=2752, V=4096, b=4, s=1024)
+    T, d = base["b"] * base["s"], base["d"]
+    dev, host = [], []
+    for L in (3, 6, 40):
+        cfg = arena.config(dict(base, L=L))
+        plain_dev, plain_host = mt.mt_device_bytes(cfg), mt.mt_host_state_bytes(cfg)
+        cfg.flags = mt.MT_FLAG_OFFLOAD_ACTS
+        dev.append(mt.mt_device_bytes(cfg))
+        host.append(mt.mt_host_state_bytes(cfg))
+        assert plain_dev - dev[-1] == (L + 1 - 3) * T * d * 4
+        assert host[-1] - plain_host == (L - 2) * T * d * 4
+    assert dev[0] == dev[1] == dev[2]

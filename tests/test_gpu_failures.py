@@ -234,3 +234,15 @@ def test_device_footprint_is_the_documented_one_and_flat_in_layers():
     b2 = mt.mt_device_bytes(arena.config(dict(base, L=2)))
     b6 = mt.mt_device_bytes(arena.config(dict(base, L=6)))
     assert b6 - b2 == extra
+    # with the boundary activations offloaded the footprint is flat in L
+    cfg = arena.config(dict(base, L=6))
+    cfg.flags = mt.MT_FLAG_OFFLOAD_ACTS
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    ctx = mt.mt_create(cfg)
+    try:
+        delta = free0 - torch.cuda.mem_get_info()[0]
+    finally:
+        mt.mt_destroy(ctx)
+    assert abs(delta - mt.mt_device_bytes(cfg)) <= (32 << 20)
+    assert abs(delta - deltas[2]) <= (32 << 20)  # three boundary slots, as the resident 2-layer context

@@ -215,6 +215,59 @@ def test_checkpoint_resume_continues_the_trajectory():
     assert rel(P2b, P2) <= 1e-5
 
 
+@pytest.mark.parametrize("name,shape,flags", [
+    ("gqa_ragged", SHAPES["gqa_ragged"], 0),
+    ("five_layers", dict(L=5, d=256, H=4, Hkv=2, F=688, V=1024, b=2, s=128), 0),
+    ("five_layers_ring_defer", dict(L=5, d=256, H=4, Hkv=2, F=688, V=1024, b=2, s=128), 0x8 | 0x10),
+    ("long_context", dict(L=4, d=1024, H=8, Hkv=8, F=2816, V=4096, b=1, s=16384), 0x8),
+])
+def test_offloaded_activations_give_the_resident_result(name, shape, flags):
+    """MT_FLAG_OFFLOAD_ACTS: the boundary activations go to host memory in the
+    forward and return for each layer's recompute; the copies are exact, so
+    two steps match the resident run (loss to 1e-5, every gradient and the
+    updated master to the run-to-run noise of the attention's dQ reductions),
+    and the first step's loss and gradients match the oracle."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    c = oracle.OracleConfig(**shape)
+    runs = {}
+    for off in (0, mt.MT_FLAG_OFFLOAD_ACTS):
+        cfg = arena.config(shape)
+        cfg.flags = flags | off
+        cfg.host_threads = 4
+        A = arena.pack(cfg, synth.init_weights(shape, 0))
+        ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+        out = []
+        try:
+            for step in range(2):
+                tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, step)
+                loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+                G = None
+                if not flags & mt.MT_FLAG_GRAD_RING:
+                    G = np.empty_like(A)
+                    mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
+                out.append((loss, G))
+            mt.mt_flush(ctx)
+            st = mt.mt_get_stats(ctx)
+        finally:
+            mt.mt_destroy(ctx)
+        runs[off] = (out, A.copy(), st)
+    res, off = runs[0], runs[mt.MT_FLAG_OFFLOAD_ACTS]
+    for (la, Ga), (lb, Gb) in zip(res[0], off[0]):
+        assert abs(la - lb) <= 1e-5
+        if Ga is not None:
+            A_, B_ = oracle.unpack_arena(Ga, c), oracle.unpack_arena(Gb, c)
+            assert max(rel(B_[k], A_[k]) for k in A_) <= 1e-4
+    assert rel(off[1], res[1]) <= 1e-3
+    # the extra link traffic of the offload is accounted for
+    T, d, L = shape["b"] * shape["s"], shape["d"], shape["L"]
+    assert off[2]["h2d_bytes"] - res[2]["h2d_bytes"] == pytest.approx(4.0 * (L - 2) * T * d)
+    if name == "gqa_ragged":
+        r = oracle_steps(shape, 1)[0]
+        assert abs(off[0][0][0] - r["loss"]) <= 1e-2
+        G = oracle.unpack_arena(off[0][0][1], c)
+        assert max(rel(G[k], r["G"][k]) for k in r["G"]) <= 2e-2
+
+
 def test_bf16_gradient_offload_stays_within_the_bars():
     """MT_FLAG_BF16_GRADS: every gradient is rounded once to bf16 before it
     leaves the GPU (the embedding rows on the host). The gradients the library
