@@ -51,6 +51,11 @@ class OracleConfig:
     beta2: float = 0.95
     adam_eps: float = 1e-8
     wd: float = 0.1
+    # Tied embeddings (one of the decoder variants the pages list as
+    # supported: saify.me, "Who this is actually for"): the LM head is the
+    # embedding table itself, z = n E^T, so E's gradient is the sum of the
+    # gather's and the head's; the arena has no separate LM-head tensor.
+    tied: bool = False
 
     @property
     def hd(self) -> int:
@@ -79,7 +84,8 @@ def _layer_tensors(c: OracleConfig):
 def arena_layout(c: OracleConfig):
     """List of (layer, tensor id, offset in floats, shape) in arena order:
     embedding, then each layer's nine tensors, then the final norm and the
-    untied LM head. Offsets are rounded up to 64 floats (256 bytes)."""
+    untied LM head (none when tied). Offsets are rounded up to 64 floats (256
+    bytes)."""
     out = []
     off = 0
 
@@ -94,7 +100,8 @@ def arena_layout(c: OracleConfig):
         for tid, shape in _layer_tensors(c):
             put(l, tid, shape)
     put(-1, FINAL_NORM, (c.d,))
-    put(-1, LM_HEAD, (c.V, c.d))
+    if not c.tied:
+        put(-1, LM_HEAD, (c.V, c.d))
     return out, off
 
 
@@ -404,17 +411,19 @@ def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
         W = {tid: weights[(l, tid)] for tid in range(9)}
         x, cache = layer_fwd(x, W, c, cos, sin)
         caches.append(cache)
+    Whead = E if c.tied else weights[(-1, LM_HEAD)]
     loss, dx, dgf, dWhead = head_ce_fwd_bwd(
-        x.reshape(T, c.d), weights[(-1, FINAL_NORM)], weights[(-1, LM_HEAD)],
-        labels.reshape(T), c.norm_eps)
-    grads = {(-1, FINAL_NORM): dgf, (-1, LM_HEAD): dWhead}
+        x.reshape(T, c.d), weights[(-1, FINAL_NORM)], Whead, labels.reshape(T), c.norm_eps)
+    grads = {(-1, FINAL_NORM): dgf}
+    if not c.tied:
+        grads[(-1, LM_HEAD)] = dWhead
     dx = dx.reshape(b, s, c.d)
     for l in reversed(range(c.L)):
         W = {tid: weights[(l, tid)] for tid in range(9)}
         dx, G = layer_bwd(dx, W, caches[l], c, cos, sin)
         for tid, g in G.items():
             grads[(l, tid)] = g
-    dE = np.zeros_like(E)
+    dE = dWhead.copy() if c.tied else np.zeros_like(E)  # tied: the head's share of E's gradient
     np.add.at(dE, tokens.reshape(T), dx.reshape(T, c.d))
     grads[(-1, EMBED)] = dE
     return loss, grads

@@ -82,5 +82,6 @@ def init_weights(cfg: dict, seed: int) -> dict:
         for tid, shape in layer_shapes(d, H, Hkv, F, hd):
             out[(l, tid)] = init_tensor(seed, l, tid, shape)
     out[(-1, FINAL_NORM)] = init_tensor(seed, -1, FINAL_NORM, (d,))
-    out[(-1, LM_HEAD)] = init_tensor(seed, -1, LM_HEAD, (V, d))
+    if not cfg.get("tied", False):  # tied embeddings: the head is the embedding table
+        out[(-1, LM_HEAD)] = init_tensor(seed, -1, LM_HEAD, (V, d))
     return out

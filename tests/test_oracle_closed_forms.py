@@ -379,3 +379,31 @@ def test_host_state_sizing_matches_pages():
     bytes_per_param = 3 * np.dtype(np.float32).itemsize
     assert bytes_per_param == gold["host_state_bytes_per_param"]
     assert gold["largest_model_params"] * bytes_per_param <= gold["largest_model_host_ram_bytes"]
+
+
+def test_tied_gradient_is_the_untied_pair_summed():
+    """With the untied head set equal to the embedding, every gradient is the
+    same as in the tied model except the table's, which is the untied
+    embedding gradient plus the untied head gradient; the arena loses exactly
+    the head tensor."""
+    import numpy as np
+    import oracle
+    import synth
+    from oracle.model import EMBED, LM_HEAD
+    shape = dict(L=1, d=32, H=2, Hkv=1, F=48, V=40, b=2, s=12)
+    untied = oracle.OracleConfig(**shape)
+    tied = oracle.OracleConfig(**shape, tied=True)
+    W = {k: v.astype(np.float64) for k, v in synth.init_weights({**shape, "tied": True}, 2).items()}
+    Wu = dict(W)
+    Wu[(-1, LM_HEAD)] = W[(-1, EMBED)].copy()
+    tok, lab = synth.tokens_labels(2, 12, 40, 5)
+    lt, Gt = oracle.train_step_grads(W, tok, lab, tied)
+    lu, Gu = oracle.train_step_grads(Wu, tok, lab, untied)
+    assert lt == lu
+    for k in Gt:
+        want = Gu[k] + (Gu[(-1, LM_HEAD)] if k == (-1, EMBED) else 0)
+        assert np.allclose(Gt[k], want, rtol=1e-13, atol=1e-16), k  # same sums, another order
+    layout_t, n_t = oracle.arena_layout(tied)
+    layout_u, n_u = oracle.arena_layout(untied)
+    assert [x[:2] for x in layout_t] == [x[:2] for x in layout_u if x[:2] != (-1, LM_HEAD)]
+    assert n_u - n_t == 40 * 32

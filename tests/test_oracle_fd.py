@@ -106,3 +106,30 @@ def test_fd_on_tiny_workload_shape():
             an = G[key].reshape(-1)[i]
             scale = max(abs(fd), 1e-2 * np.abs(G[key]).max(), 1e-12)
             assert abs(fd - an) <= 1e-6 * scale, (key, i, fd, an)
+
+
+def test_tied_embeddings_match_central_differences():
+    """Tied embeddings: the LM head is the embedding table, so the derivative
+    of the loss with respect to one table entry covers both uses (gather and
+    head). Rows the batch does not gather still get the head's share."""
+    c = oracle.OracleConfig(L=1, d=32, H=4, Hkv=2, F=40, V=50, b=2, s=8, tied=True)
+    W = _weights(c, 3)
+    del W[(-1, LM_HEAD)]
+    rng = np.random.default_rng(11)
+    tok = rng.integers(0, c.V, (c.b, c.s))
+    lab = rng.integers(0, c.V, (c.b, c.s))
+    tok[1, :3] = tok[0, 0]
+    _, G = oracle.train_step_grads(W, tok, lab, c)
+    assert (-1, LM_HEAD) not in G
+    used = np.unique(tok)
+    unused = np.setdiff1d(np.arange(c.V), used)[:4]
+    flat = W[(-1, EMBED)].reshape(-1)
+    rows = np.concatenate([used[:5], unused])
+    h = 1e-4
+    for r in rows:
+        for j in rng.choice(c.d, 4, replace=False):
+            i = r * c.d + j
+            fd = _fd5(W, flat, i, h, tok, lab, c)
+            an = G[(-1, EMBED)].reshape(-1)[i]
+            scale = max(abs(fd), 1e-3 * np.abs(G[(-1, EMBED)]).max(), 1e-9)
+            assert abs(fd - an) <= 1e-6 * scale + 1e-10, (r, j, fd, an)

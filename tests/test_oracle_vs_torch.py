@@ -39,7 +39,7 @@ def _torch_step(W, tok, lab, c):
         m = F.rms_norm(h, (c.d,), w(MLP_NORM), c.norm_eps)
         x = h + (F.silu(m @ w(WGATE).T) * (m @ w(WUP).T)) @ w(WDOWN).T
     n = F.rms_norm(x, (c.d,), Wt[(-1, FINAL_NORM)], c.norm_eps)
-    z = n @ Wt[(-1, LM_HEAD)].T
+    z = n @ Wt[(-1, EMBED) if c.tied else (-1, LM_HEAD)].T  # tied: one parameter, two uses
     loss = F.cross_entropy(z.reshape(-1, c.V), torch.tensor(lab).reshape(-1).long())
     loss.backward()
     return loss.item(), {k: v.grad.numpy() for k, v in Wt.items()}
@@ -77,6 +77,24 @@ def test_tiny_workload_matches_torch():
     c = oracle.OracleConfig(**cfg)
     W = {k: v.astype(np.float64) for k, v in synth.init_weights(cfg, 0).items()}
     tok, lab = synth.tokens_labels(c.b, c.s, c.V, 0)
+    loss, G = oracle.train_step_grads(W, tok, lab, c)
+    tloss, TG = _torch_step(W, tok, lab, c)
+    assert abs(loss - tloss) <= 1e-12 * abs(tloss)
+    for k in W:
+        assert _rel(G[k], TG[k]) <= 1e-10, k
+
+
+def test_tied_embeddings_match_torch():
+    """Tied embeddings: torch autograd accumulates both uses of the one table
+    parameter; the oracle adds the head's gradient to the gather's."""
+    shape = dict(L=2, d=64, H=4, Hkv=2, F=96, V=80, b=2, s=16, tied=True)
+    c = oracle.OracleConfig(**shape)
+    W = {k: v.astype(np.float64) * (1 if k[1] in (ATTN_NORM, MLP_NORM, FINAL_NORM) else 10)
+         for k, v in synth.init_weights(shape, 9).items()}
+    assert (-1, LM_HEAD) not in W
+    rng = np.random.default_rng(4)
+    tok = rng.integers(0, c.V, (c.b, c.s))
+    lab = rng.integers(0, c.V, (c.b, c.s))
     loss, G = oracle.train_step_grads(W, tok, lab, c)
     tloss, TG = _torch_step(W, tok, lab, c)
     assert abs(loss - tloss) <= 1e-12 * abs(tloss)
