@@ -105,10 +105,11 @@ struct mt_ctx {
   uint8_t* grad = nullptr;        // pinned gradient arena (not with MT_FLAG_GRAD_RING)
   uint8_t* ring = nullptr;        // pinned gradient ring of MT_GRAD_RING_SLOTS layer slots
   uint8_t* grad_head = nullptr;   // [final norm | LM head] gradients: inside grad, or own buffer
+  bool grad_head_owned = false;   // own pinned buffer (gradient ring, or tied embeddings)
   size_t layer_f = 0;             // floats of one layer's gradient block
   uint16_t* bf_layers = nullptr;  // pinned bf16 layer blocks
   uint16_t* bf_embed = nullptr;   // pinned bf16 embedding (read by the GPU in place)
-  uint16_t* bf_head = nullptr;    // pinned bf16 [final norm | LM head]
+  uint16_t* bf_head = nullptr;    // pinned bf16 [final norm | LM head] ([final norm] when tied)
   uint16_t* bf_embed_dev = nullptr;  // device alias of bf_embed
   float* emb_rows_h = nullptr;    // pinned embedding-gradient rows [T, d]
   int32_t* stage_i = nullptr;     // pinned: tokens[T] labels[T] offs[T+1] pos[T]
@@ -447,7 +448,7 @@ int head_step(mt_ctx* c, float* gout) {
   const Shapes& s = c->lay.sh;
   const int T = s.T, d = s.d, V = s.V;
   cudaStream_t st = c->s_comp;
-  const size_t gf_pad = c->lay.head.off - c->lay.final_norm.off;  // floats between dgf and dWhead
+  const size_t gf_pad = c->lay.gf_pad;  // floats between dgf and dWhead
   const uint16_t* gf = c->d_head_w;
   const uint16_t* Wh = c->d_head_w + align_up(d, 128);
   float* dgf = c->d_head_g;
@@ -464,7 +465,7 @@ int head_step(mt_ctx* c, float* gout) {
   }
   KL(launch_sum_all(c->rowloss, T, c->d_loss, 0, st), 1);
   KL(launch_rmsnorm_bwd(xL, gf, c->rf, c->tmp_f, nullptr, gout, nullptr, c->rms_part, dgf, T, d, st), 2);
-  return check_finite(c, c->d_head_g, gf_pad + (size_t)V * d, s.L);
+  return check_finite(c, c->d_head_g, c->lay.head_block, s.L);
 }
 
 // ---------------------------------------------------------------------------
@@ -567,8 +568,10 @@ std::vector<Seg> layer_or_head_segs(mt_ctx* c, int l, const uint8_t* g) {
     }
   } else {
     segs.push_back(grad_seg(c, y.final_norm.off, y.final_norm.n, c->bf_head, c->grad_head));
-    segs.push_back(grad_seg(c, y.head.off, y.head.n, c->bf_head + align_up(y.sh.d, 128),
-                            c->grad_head + (y.head.off - y.final_norm.off) * c->gsz));
+    // (tied: the table's update waits for the gathered rows' gradient, in the EMBED job)
+    if (!y.tied)
+      segs.push_back(grad_seg(c, y.head.off, y.head.n, c->bf_head + align_up(y.sh.d, 128),
+                              c->grad_head + y.gf_pad * c->gsz));
   }
   return segs;
 }
@@ -633,7 +636,8 @@ void run_job_body(mt_ctx* c, const Job& j) {
     // gradient arena, put last step's touched rows back to zero and scatter
     // this step's rows in (every other row's stored gradient is 0). The update
     // reads them from the staging rows.
-    uint8_t* ge = c->grad ? c->grad + y.embed.off * c->gsz : nullptr;
+    // (tied embeddings: the rows go into the head's dense table gradient below)
+    uint8_t* ge = (c->grad && !y.tied) ? c->grad + y.embed.off * c->gsz : nullptr;
     const size_t d = s.d, gsz = c->gsz;
     const int nt = c->pool->size() * 4;
     if (ge) {
@@ -668,6 +672,24 @@ void run_job_body(mt_ctx* c, const Job& j) {
     int32_t dev_err = 0;  // device error word as of the embedding backward
     memcpy(&dev_err, c->misc_h + 2, 4);
     if (dev_err != 0) c->flags_h[j.flag_index] |= kFlagDeviceError;
+    if (y.tied) {
+      // The table's gradient: the head's dense V x d part plus the gathered
+      // rows (distinct rows per task, so no two threads add to one row).
+      float* gh = reinterpret_cast<float*>(c->grad_head) + y.gf_pad;
+      c->pool->run(nt, [&](int i) {
+        for (size_t u = nu * i / nt; u < nu * (i + 1) / nt; ++u) {
+          float* row = gh + (size_t)c->uniq[u] * d;
+          const float* src = c->emb_rows_h + u * d;
+          for (size_t k = 0; k < d; ++k) row[k] += src[k];
+        }
+      });
+      if (c->grad) {  // the gradient arena reports the table's and the final gain's gradients
+        parallel_ranges(*c->pool, y.embed.n, [&](size_t b, size_t e) {
+          memcpy(reinterpret_cast<float*>(c->grad) + y.embed.off + b, gh + b, (e - b) * 4);
+        });
+        memcpy(reinterpret_cast<float*>(c->grad) + y.final_norm.off, c->grad_head, d * 4);
+      }
+    }
   }
   if (!passes_checks(c, c->flags_h[j.flag_index])) return;
   if (c->cfg.flags & MT_FLAG_NO_UPDATE) return;
@@ -684,6 +706,8 @@ void run_job_body(mt_ctx* c, const Job& j) {
   std::vector<Seg> segs;
   if (j.kind == Job::LAYER || j.kind == Job::HEAD) {
     segs = layer_or_head_segs(c, j.kind == Job::HEAD ? -1 : j.layer, j.g);
+  } else if (y.tied) {  // EMBED, tied: one dense update of the whole table
+    segs.push_back({y.embed.off, y.embed.n, c->bf_embed, reinterpret_cast<const float*>(c->grad_head) + y.gf_pad});
   } else {
     for (size_t u = 0; u < c->uniq.size(); ++u) {
       const size_t r = (size_t)c->uniq[u];
@@ -691,7 +715,7 @@ void run_job_body(mt_ctx* c, const Job& j) {
     }
   }
   adamw_segments(c, segs, c->step);
-  if (j.kind == Job::EMBED && (c->cfg.flags & MT_FLAG_DEFER_UPDATES)) {
+  if (j.kind == Job::EMBED && (c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !y.tied) {
     // The step's last job: every gradient passed its checks, so the
     // zero-gradient update of the rows it did not touch is due. It runs with
     // the next step (or at the next flush), overlapping its GPU work.
@@ -825,11 +849,23 @@ int issue_load(mt_ctx* c, int i) {
   return MT_OK;
 }
 
+// [final gain | LM head] bf16 into the device head block; with tied
+// embeddings the head part is the streamed embedding table.
+int copy_head_weights(mt_ctx* c, cudaStream_t st) {
+  const size_t g = align_up(c->lay.sh.d, 128), n = (size_t)c->lay.sh.V * c->lay.sh.d;
+  if (c->lay.tied) {
+    CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, g * 2, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(c->d_head_w + g, c->bf_embed, n * 2, cudaMemcpyHostToDevice, st));
+  } else {
+    CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, (g + n) * 2, cudaMemcpyHostToDevice, st));
+  }
+  return MT_OK;
+}
+
 int issue_head_load(mt_ctx* c) {
-  const size_t n = align_up(c->lay.sh.d, 128) + (size_t)c->lay.sh.V * c->lay.sh.d;
   CKM(await_deferred(c, c->lay.sh.L));
   CK(cudaEventRecord(c->ev_head_h2d_start, c->s_h2d));
-  CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, n * 2, cudaMemcpyHostToDevice, c->s_h2d));
+  CKM(copy_head_weights(c, c->s_h2d));
   CK(cudaEventRecord(c->ev_head_wready, c->s_h2d));
   return MT_OK;
 }
@@ -932,7 +968,7 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         CK(cudaEventRecord(c->ev_fwd_end, sc));
         CK(cudaStreamWaitEvent(sc, c->ev_head_wready, 0));
         CKM(head_step(c, gin));
-        const size_t n = y.head.off + y.head.n - y.final_norm.off;
+        const size_t n = y.head_block;
         const void* hsrc = c->d_head_g;
         if (c->gsz == 2) {
           KL(launch_cast_f32_bf16(c->d_head_g, c->d_head_g16, (int64_t)n, sc), 1);
@@ -991,7 +1027,8 @@ int enqueue_step(mt_ctx* c, int n_unique) {
   c->flags_h[L + 1] = 0;
   push_job(c, Job{Job::EMBED, -1, c->ev_emb_drained, L + 1});
   // Without deferral the untouched rows' update follows the step's last check.
-  if (!(c->cfg.flags & MT_FLAG_DEFER_UPDATES)) push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, L + 1});
+  // (tied embeddings: every row has a head gradient, so the EMBED job updates them all)
+  if (!(c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !y.tied) push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, L + 1});
   CK(cudaMemcpyAsync(c->misc_h, c->d_loss, 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaEventRecord(c->ev_step_end, sc));
@@ -1027,7 +1064,7 @@ void collect_stats(mt_ctx* c) {
   st.h2d_bytes = act_bytes + (double)c->load_seq.size() * y.bf_layer * 2 +
                  (double)(align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d) * 2 + 4.0 * (4 * y.sh.T + 1) +
                  (double)y.sh.T * y.sh.d * 2;  // embedding rows read in place
-  st.d2h_bytes = act_bytes + (double)c->gsz * (y.head.off + y.head.n - y.final_norm.off) +
+  st.d2h_bytes = act_bytes + (double)c->gsz * y.head_block +
                  4.0 * c->uniq.size() * y.sh.d + 12.0;
   for (int l = 0; l < L; ++l) st.d2h_bytes += (double)c->gsz * (y.layer_end(l) - y.layer_begin(l));
   st.adamw_ms = c->adamw_s * 1e3;
@@ -1063,12 +1100,12 @@ size_t device_bytes(const Layout& y, int Tc, bool g16, bool offload) {
   const size_t lay_f = y.layer_end(0) - y.layer_begin(0);
   add(lay_f * 4);
   add(lay_f * 4);
-  add((align_up(d, 128) + V * d) * 2);                     // head weights
-  add((y.head.off - y.final_norm.off + V * d) * 4);         // head grads
+  add((align_up(d, 128) + V * d) * 2);                     // head weights (or the tied table)
+  add(y.head_block * 4);                                    // head grads
   if (g16) {                                                // bf16 offload copies
     add(lay_f * 2);
     add(lay_f * 2);
-    add((y.head.off - y.final_norm.off + V * d) * 2);
+    add(y.head_block * 2);
   }
   add((size_t)(offload ? std::min(s.L + 1, 3) : s.L + 1) * T * d * 4);  // boundary activations
   add(T * d * 2);                                           // u
@@ -1159,7 +1196,7 @@ void free_all(mt_ctx* c) {
   if (c->s_d2h && c->s_d2h != c->s_comp && c->s_d2h != c->s_h2d) cudaStreamDestroy(c->s_d2h);
   if (c->s_act && c->s_act != c->s_comp) cudaStreamDestroy(c->s_act);
   if (c->dmem) cudaFree(c->dmem);
-  for (void* p : {(void*)c->grad, (void*)c->ring, (void*)c->defer_g, (void*)(c->grad ? nullptr : c->grad_head),
+  for (void* p : {(void*)c->grad, (void*)c->ring, (void*)c->defer_g, (void*)(c->grad_head_owned ? c->grad_head : nullptr),
                   (void*)c->bf_layers,
                   (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h, (void*)c->stage_i, (void*)c->flags_h,
                   (void*)c->misc_h, (void*)c->xh})
@@ -1230,8 +1267,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   if (posix_memalign(reinterpret_cast<void**>(&c->m), 64, y.total * 4) ||
       posix_memalign(reinterpret_cast<void**>(&c->v), 64, y.total * 4))
     return fail(MT_ERR_NOMEM, "host moment allocation failed");
-  const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
-  const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
+  const size_t head_bf = align_up(s.d, 128) + (y.tied ? 0 : (size_t)s.V * s.d);  // host bf16 head block
+  const size_t head_f = y.head_block;
   c->layer_f = y.layer_end(0) - y.layer_begin(0);
   for (int l = 1; l < s.L; ++l)
     if (y.layer_end(l) - y.layer_begin(l) != c->layer_f) return fail(MT_ERR_CONFIG, "layer blocks differ in size");
@@ -1254,8 +1291,14 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   } else {
     if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad), y.total * gsz, cudaHostAllocPortable) != cudaSuccess)
       return fail(MT_ERR_PIN, "pinned gradient arena allocation failed");
-    c->grad_head = c->grad + y.final_norm.off * gsz;
+    if (y.tied) {  // the arena has no LM-head tensor: the head's gradient block is separate
+      if (cudaHostAlloc(reinterpret_cast<void**>(&c->grad_head), head_f * gsz, cudaHostAllocPortable) != cudaSuccess)
+        return fail(MT_ERR_PIN, "pinned head-gradient allocation failed");
+    } else {
+      c->grad_head = c->grad + y.final_norm.off * gsz;
+    }
   }
+  c->grad_head_owned = (cfg->flags & MT_FLAG_GRAD_RING) || y.tied;
   if (cudaHostAlloc(reinterpret_cast<void**>(&c->bf_layers), (size_t)s.L * y.bf_layer * 2, cudaHostAllocPortable) !=
           cudaSuccess ||
       cudaHostAlloc(reinterpret_cast<void**>(&c->bf_embed), (size_t)s.V * s.d * 2,
@@ -1288,7 +1331,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
       for (int tid = 0; tid < kLayerTensors; ++tid)
         fill(y.t(l, tid), seed ^ (((uint64_t)(l + 1) << 8) | tid), tid == MT_T_ATTN_NORM || tid == MT_T_MLP_NORM);
     fill(y.final_norm, seed ^ 0x1001, true);
-    fill(y.head, seed ^ 0x1002, false);
+    if (!y.tied) fill(y.head, seed ^ 0x1002, false);
   }
   parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) {
     memset(c->m + b, 0, (e - b) * 4);
@@ -1301,9 +1344,9 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     if (c->defer_g)
       parallel_ranges(*c->pool, (size_t)c->defer_layers * c->layer_f,
                       [&](size_t b, size_t e) { memset(c->defer_g + b * gsz, 0, (e - b) * gsz); });
-    parallel_ranges(*c->pool, head_f,
-                    [&](size_t b, size_t e) { memset(c->grad_head + b * gsz, 0, (e - b) * gsz); });
   }
+  if (c->grad_head_owned)
+    parallel_ranges(*c->pool, head_f, [&](size_t b, size_t e) { memset(c->grad_head + b * gsz, 0, (e - b) * gsz); });
   // bf16 streaming copies
   for (int l = 0; l < s.L; ++l) {
     uint16_t* blk = c->bf_layers + (size_t)l * y.bf_layer;
@@ -1319,7 +1362,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   memset(c->bf_head, 0, head_bf * 2);
   bf16_round_chunk(c->arena + y.final_norm.off, c->bf_head, s.d);
   uint16_t* bhw = c->bf_head + align_up(s.d, 128);
-  parallel_ranges(*c->pool, y.head.n,
+  parallel_ranges(*c->pool, y.head.n,  // (nothing when tied)
                   [&](size_t b, size_t e) { bf16_round_chunk(c->arena + y.head.off + b, bhw + b, e - b); });
 
   // device memory: one allocation carved into buffers
@@ -1337,12 +1380,12 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   const size_t lay_f = y.layer_end(0) - y.layer_begin(0);
   c->gslot[0] = (float*)carve(lay_f * 4);
   c->gslot[1] = (float*)carve(lay_f * 4);
-  c->d_head_w = (uint16_t*)carve(head_bf * 2);
-  c->d_head_g = (float*)carve((y.head.off - y.final_norm.off + V * d) * 4);
+  c->d_head_w = (uint16_t*)carve((align_up(d, 128) + V * d) * 2);
+  c->d_head_g = (float*)carve(y.head_block * 4);
   if (gsz == 2) {
     c->gslot16[0] = (uint16_t*)carve(lay_f * 2);
     c->gslot16[1] = (uint16_t*)carve(lay_f * 2);
-    c->d_head_g16 = (uint16_t*)carve((y.head.off - y.final_norm.off + V * d) * 2);
+    c->d_head_g16 = (uint16_t*)carve(y.head_block * 2);
   }
   c->xb = (float*)carve((size_t)((cfg->flags & MT_FLAG_OFFLOAD_ACTS) ? std::min(s.L + 1, 3) : s.L + 1) * T * d * 4);
   c->u_b = (uint16_t*)carve(T * d * 2);
@@ -1570,7 +1613,7 @@ extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* label
   if (!x_L || !labels || !loss_out || !dx_L || !grads) return set_err(c, MT_ERR_ARG, "NULL argument");
   const Layout& y = c->lay;
   const Shapes& s = y.sh;
-  const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
+  const size_t head_f = y.head_block;
   if (grads_bytes < head_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than the final-norm + head block");
   for (int t = 0; t < s.T; ++t)
     if (labels[t] < 0 || labels[t] >= s.V) return set_err(c, MT_ERR_ARG, "label outside [0, V)");
@@ -1581,9 +1624,8 @@ extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* label
   c->timing_used = 0;
   c->timed.clear();
   c->err.clear();
-  const size_t head_bf = align_up(s.d, 128) + (size_t)s.V * s.d;
   CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));
-  CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, head_bf * 2, cudaMemcpyHostToDevice, sc));
+  CKM(copy_head_weights(c, sc));
   CK(cudaMemcpyAsync(x_fwd(c, s.L), x_L, n * 4, cudaMemcpyHostToDevice, sc));
   CK(cudaMemcpyAsync(c->d_lab, labels, (size_t)s.T * 4, cudaMemcpyHostToDevice, sc));
   CKM(head_step(c, c->gx0));

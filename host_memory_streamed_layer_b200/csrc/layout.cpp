@@ -34,6 +34,8 @@ int validate_config(const mt_config* c, std::string* why) {
       !(c->beta2 >= 0 && c->beta2 < 1) || !(c->adam_eps > 0) || !(c->wd >= 0))
     return fail(MT_ERR_CONFIG, "hyper-parameter out of range");
   if (c->host_threads < 0) return fail(MT_ERR_CONFIG, "host_threads must be >= 0");
+  if ((c->flags & MT_FLAG_TIED_EMBED) && (c->flags & MT_FLAG_BF16_GRADS))
+    return fail(MT_ERR_CONFIG, "tied embeddings take their gradients in fp32 (no MT_FLAG_BF16_GRADS)");
   return MT_OK;
 }
 
@@ -74,8 +76,14 @@ Layout make_layout(const mt_config& c) {
     t[MT_T_WDOWN] = put(d * F);
   }
   y.final_norm = put(d);
-  y.head = put(V * d);
+  y.tied = (c.flags & MT_FLAG_TIED_EMBED) != 0;
+  if (y.tied)
+    y.head = TRef{off, 0};
+  else
+    y.head = put(V * d);
   y.total = off;
+  y.gf_pad = round_up(d, 64);
+  y.head_block = y.gf_pad + V * d;
   // bf16 block (128 elements = 256 bytes alignment)
   size_t b = 0;
   auto bput = [&](size_t n) {
@@ -139,7 +147,7 @@ extern "C" int mt_tensor_offset(const mt_config* cfg, int layer, int tid, size_t
       r = y.embed;
     else if (tid == MT_T_FINAL_NORM)
       r = y.final_norm;
-    else if (tid == MT_T_LM_HEAD)
+    else if (tid == MT_T_LM_HEAD && !y.tied)
       r = y.head;
     else
       return MT_ERR_ARG;
@@ -163,22 +171,23 @@ extern "C" size_t mt_host_state_bytes(const mt_config* cfg) {
   if (mt::validate_config(cfg, nullptr) != MT_OK) return 0;
   mt::Layout y = mt::make_layout(*cfg);
   const size_t P = y.total;
-  const size_t bf = (size_t)y.sh.L * y.bf_layer + 2 * (size_t)y.sh.V * y.sh.d + y.sh.d + 256;
+  const size_t bf = (size_t)y.sh.L * y.bf_layer + (y.tied ? 1 : 2) * (size_t)y.sh.V * y.sh.d + y.sh.d + 256;
   const size_t common = P * 4 * 2 + bf * 2 + (size_t)y.sh.T * y.sh.d * 4;  // m, v; bf16 copy; embedding staging
   const size_t gsz = (cfg->flags & MT_FLAG_BF16_GRADS) ? 2 : 4;           // bytes per host gradient element
   const size_t acts = ((cfg->flags & MT_FLAG_OFFLOAD_ACTS) && y.sh.L >= 3)  // x_0 .. x_{L-3}, fp32
                           ? (size_t)(y.sh.L - 2) * y.sh.T * y.sh.d * 4
                           : 0;
-  if (!(cfg->flags & MT_FLAG_GRAD_RING)) return acts + common + P * gsz;  // whole gradient arena
+  const size_t head_own = y.tied ? y.head_block * 4 : 0;                  // tied: the head's gradient block
+  if (!(cfg->flags & MT_FLAG_GRAD_RING)) return acts + common + P * gsz + head_own;  // whole gradient arena
   const size_t layer_f = y.layer_end(0) - y.layer_begin(0);
-  const size_t head_f = y.head.off + y.head.n - y.final_norm.off;
-  return acts + common + ((size_t)(MT_GRAD_RING_SLOTS + mt::defer_layer_count(*cfg)) * layer_f + head_f) * gsz;
+  return acts + common + ((size_t)(MT_GRAD_RING_SLOTS + mt::defer_layer_count(*cfg)) * layer_f + y.head_block) * gsz;
 }
 
 extern "C" int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard* out) {
   if (!out || world < 1 || world > 1024 || rank < 0 || rank >= world) return MT_ERR_ARG;
   if (mt::validate_config(cfg, nullptr) != MT_OK) return MT_ERR_CONFIG;
   if (cfg->d % 128) return MT_ERR_CONFIG;  // fp32 and bf16 block offsets coincide only then
+  if (cfg->flags & MT_FLAG_TIED_EMBED) return MT_ERR_CONFIG;  // one table, two owners: not partitioned
   const mt::Layout y = mt::make_layout(*cfg);
   const size_t lb = y.layer_begin(0), le = y.layer_end(0);
   // The fp32 arena block of a layer and its bf16 streamed block must hold

@@ -35,8 +35,12 @@ struct Shapes {
 
 struct Layout {
   Shapes sh{};
-  // fp32 arena, in floats
+  // fp32 arena, in floats (head.n == 0 with tied embeddings: the table is the head)
   TRef embed, final_norm, head;
+  bool tied = false;
+  // [final-norm gain | LM head] gradient block (device and host buffers, also
+  // when tied): the gain padded to gf_pad floats, then V*d
+  size_t gf_pad = 0, head_block = 0;
   std::vector<TRef> layer;  // L * kLayerTensors
   size_t total = 0;
   size_t layer_begin(int l) const { return layer[(size_t)l * kLayerTensors].off; }

@@ -186,6 +186,7 @@ MT_FLAG_SERIALIZE, MT_FLAG_KERNEL_TIMING, MT_FLAG_NO_UPDATE, MT_FLAG_GRAD_RING =
 MT_FLAG_DEFER_UPDATES = 0x10
 MT_FLAG_BF16_GRADS = 0x20
 MT_FLAG_OFFLOAD_ACTS = 0x40
+MT_FLAG_TIED_EMBED = 0x80
 MT_GRAD_RING_SLOTS = 3
 MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
 MT_T_EMBED, MT_T_FINAL_NORM, MT_T_LM_HEAD = 100, 101, 102

@@ -113,6 +113,16 @@ extern "C" {
  * step and (L-2) b s d 4 bytes of pinned host memory (mt_host_state_bytes).
  * The arithmetic is unchanged: every copy is exact. */
 #define MT_FLAG_OFFLOAD_ACTS 0x40u
+/* Tied embeddings: the LM head is the embedding table (z = n E^T), one of the
+ * decoder variants the pages list as supported (saify.me, "Who this is
+ * actually for": "The repo supports many architectures"). The arena has no
+ * LM-head tensor (mt_arena_bytes shrinks by V*d floats; mt_tensor_offset
+ * refuses MT_T_LM_HEAD); the head streams the bf16 table each step, and the
+ * table's gradient is the head's dense V x d gradient plus the gathered rows'.
+ * It is updated with one dense AdamW in the step's last host job, after every
+ * gradient of the step has been checked. Not with MT_FLAG_BF16_GRADS, and not
+ * partitioned by mt_shard_plan (MT_ERR_CONFIG). */
+#define MT_FLAG_TIED_EMBED 0x80u
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0

@@ -352,3 +352,27 @@ def test_offloaded_activations_keep_three_device_slots():
         assert plain_dev - dev[-1] == (L + 1 - 3) * T * d * 4
         assert host[-1] - plain_host == (L - 2) * T * d * 4
     assert dev[0] == dev[1] == dev[2]
+
+
+def test_tied_embeddings_layout():
+    """MT_FLAG_TIED_EMBED: the arena loses exactly the LM-head tensor (the
+    oracle's tied layout matches the library's offsets), MT_T_LM_HEAD is
+    refused, and the combinations the flag does not support are refused."""
+    import oracle
+    from host_memory_streamed_layer_b200 import arena, mt
+    shape = dict(L=3, d=256, H=4, Hkv=2, F=688, V=1000, b=2, s=64)
+    cfg = arena.config(shape)
+    untied = mt.mt_arena_bytes(cfg)
+    cfg.flags = mt.MT_FLAG_TIED_EMBED
+    assert untied - mt.mt_arena_bytes(cfg) == 4 * shape["V"] * shape["d"]
+    c = oracle.OracleConfig(**shape, tied=True)
+    layout, total = oracle.arena_layout(c)
+    assert total * 4 == mt.mt_arena_bytes(cfg)
+    for layer, tid, off, shp in layout:
+        assert mt.mt_tensor_offset(cfg, layer, tid) == (off, int(np.prod(shp)))
+    with pytest.raises(mt.MTError):
+        mt.mt_tensor_offset(cfg, -1, mt.MT_T_LM_HEAD)
+    with pytest.raises(mt.MTError):
+        mt.mt_shard_plan(cfg, 2, 0)
+    cfg.flags = mt.MT_FLAG_TIED_EMBED | mt.MT_FLAG_BF16_GRADS
+    assert mt.mt_arena_bytes(cfg) == 0

@@ -268,6 +268,70 @@ def test_offloaded_activations_give_the_resident_result(name, shape, flags):
         assert max(rel(G[k], r["G"][k]) for k in r["G"]) <= 2e-2
 
 
+def _tied_run(shape, flags, nsteps, seed=0):
+    from host_memory_streamed_layer_b200 import arena, mt
+    cfg = arena.config(shape)
+    cfg.flags = flags | mt.MT_FLAG_TIED_EMBED
+    cfg.host_threads = 4
+    A = arena.pack(cfg, synth.init_weights({**shape, "tied": True}, seed))
+    ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+    out = []
+    try:
+        for step in range(nsteps):
+            tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], seed, step)
+            before = A.copy()
+            loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+            G = None
+            if not flags & mt.MT_FLAG_GRAD_RING:
+                G = np.empty_like(A)
+                mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
+            mt.mt_flush(ctx)
+            out.append(dict(before=before, loss=loss, G=G, P=A.copy()))
+    finally:
+        mt.mt_destroy(ctx)
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny", "gqa_ragged", "hd128"])
+def test_tied_embeddings_match_oracle(name):
+    """MT_FLAG_TIED_EMBED: the head reads the streamed embedding table, and
+    the table's gradient is the head's plus the gathered rows'. One step
+    against the oracle's tied model: loss, every gradient (no LM-head tensor),
+    the host AdamW on the engine's gradients (1e-6) and the end-to-end update
+    (the same 5e-3 bar as the untied model)."""
+    shape = SHAPES[name]
+    c = oracle.OracleConfig(**shape, tied=True)
+    g = _tied_run(shape, 0, 1)[0]
+    W = {k: oracle.bf16_round(v.astype(np.float32))
+         for k, v in oracle.unpack_arena(g["before"], c).items()}
+    assert (-1, 102) not in W
+    rloss, RG = oracle.train_step_grads(W, *synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, 0), c)
+    assert abs(g["loss"] - rloss) <= 1e-2
+    G = oracle.unpack_arena(g["G"], c)
+    assert max(rel(G[k], RG[k]) for k in RG) <= 2e-2, {k: rel(G[k], RG[k]) for k in RG}
+    p, _, _ = oracle.adamw_update(g["before"].astype(np.float64), g["G"].astype(np.float64), 0.0, 0.0, 1, **HYP)
+    assert rel(g["P"].astype(np.float64), p) <= 1e-6
+    P, before = oracle.unpack_arena(g["P"], c), oracle.unpack_arena(g["before"], c)
+    num = den = 0.0
+    for k in before:
+        po, _, _ = oracle.adamw_update(before[k], RG[k], 0 * before[k], 0 * before[k], 1, **HYP)
+        num += float(np.sum((P[k] - po) ** 2))
+        den += float(np.sum(po ** 2))
+    assert math.sqrt(num / den) <= 5e-3, math.sqrt(num / den)
+
+
+def test_tied_embeddings_with_ring_and_deferral():
+    """Tied embeddings with the gradient ring and deferred updates follow the
+    plain tied run for three steps (same losses, same master)."""
+    from host_memory_streamed_layer_b200 import mt
+    shape = dict(L=5, d=256, H=4, Hkv=2, F=688, V=1024, b=2, s=128)
+    base = _tied_run(shape, 0, 3)
+    alt = _tied_run(shape, mt.MT_FLAG_GRAD_RING | mt.MT_FLAG_DEFER_UPDATES, 3)
+    for a, b in zip(base, alt):
+        assert abs(a["loss"] - b["loss"]) <= 1e-4
+        assert rel(b["P"], a["P"]) <= 2e-3
+
+
 def test_bf16_gradient_offload_stays_within_the_bars():
     """MT_FLAG_BF16_GRADS: every gradient is rounded once to bf16 before it
     leaves the GPU (the embedding rows on the host). The gradients the library
