@@ -160,7 +160,7 @@ def test_embedding_fwd_exact_and_bwd():
     assert np.allclose(np64(rows), ref[uniq], rtol=1e-5, atol=1e-5)
 
 
-@pytest.mark.parametrize("T,V", [(64, 1024), (9, 32000), (3, 152064)])
+@pytest.mark.parametrize("T,V", [(64, 1024), (9, 32000), (2, 49152), (2, 49160), (3, 152064)])
 def test_softmax_ce(T, V):
     mt = _mt()
     rng = np.random.default_rng(V)
