@@ -126,6 +126,68 @@ def test_attention_full_shape_sampled(impl):
     assert np.linalg.norm(gv - rdv[0, -16:, 0]) <= 2e-2 * np.linalg.norm(rdv[0, -16:, 0])
 
 
+@pytest.mark.parametrize("impl", ["mma", "tc"])
+def test_attention_whole_heads_full_length(impl):
+    """Every row of two whole heads at the full 2048-token length, element by
+    element (per-row relative L2): o, the log-sum-exp, dq, dk and dv against
+    the oracle's attention of the whole sequence. Each query row's last key
+    block is the masked diagonal one and its earlier blocks run the mask-free
+    instantiation, and each key row is seen by both kinds, so both are covered
+    at full length. GQA (4 query heads per KV head) is on, so dk and dv sum
+    over a group."""
+    mt = _mt()
+    Hkv = H // 4
+    g = torch.Generator(device=DEV).manual_seed(11)
+    ld = (H + 2 * Hkv) * HD
+    qkv = torch.randn(T, ld, device=DEV, generator=g).to(torch.bfloat16)
+    o = torch.empty(T, H * HD, device=DEV, dtype=torch.bfloat16)
+    lse = torch.empty(B, H, S, device=DEV)
+    p = qkv.data_ptr()
+    pk, pv = p + 2 * H * HD, p + 2 * (H + Hkv) * HD
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    fwd = mt.mt_k_attn_fwd_tc if impl == "tc" else mt.mt_k_attn_fwd
+    fwd(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, Hkv, HD, 0,
+        *([err.data_ptr()] if impl == "tc" else []))
+    do = torch.randn(T, H * HD, device=DEV, generator=g).to(torch.bfloat16)
+    dvec = torch.empty(B, H, S, device=DEV)
+    dqa = torch.empty(T, H * HD, device=DEV)
+    dqkv = torch.empty(T, ld, device=DEV, dtype=torch.bfloat16)
+    dp = dqkv.data_ptr()
+    bwd = mt.mt_k_attn_bwd_tc if impl == "tc" else mt.mt_k_attn_bwd
+    kw = {"dev_err": err.data_ptr()} if impl == "tc" else {}
+    bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(), dvec.data_ptr(), dqa.data_ptr(),
+        H * HD, dp, ld, dp + 2 * H * HD, dp + 2 * (H + Hkv) * HD, ld, B, S, H, Hkv, HD, **kw)
+    torch.cuda.synchronize()
+    assert err.item() == 0
+
+    def rows_close(got, ref, tol, floor):
+        num = np.linalg.norm(got - ref, axis=-1)
+        den = np.linalg.norm(ref, axis=-1)
+        assert np.all(num <= tol * den + floor), float(np.max(num / (den + 1e-30)))
+
+    X = qkv.double().cpu().numpy()
+    dO = do.double().cpu().numpy()
+    G = dqkv.double().cpu().numpy()
+    O = o.double().cpu().numpy()
+    for bi, kvh in [(2, 1), (6, 3)]:
+        rows = slice(bi * S, (bi + 1) * S)
+        k = X[rows, (H + kvh) * HD:(H + kvh + 1) * HD][None, :, None]
+        v = X[rows, (H + Hkv + kvh) * HD:(H + Hkv + kvh + 1) * HD][None, :, None]
+        dk = np.zeros((S, HD))
+        dv = np.zeros((S, HD))
+        for h in range(kvh * 4, kvh * 4 + 4):
+            q = X[rows, h * HD:(h + 1) * HD][None, :, None]
+            ro, P = oracle.attention_fwd(q, k, v)
+            rows_close(O[rows, h * HD:(h + 1) * HD], ro[0, :, 0], 1e-2, 1e-3)
+            assert np.max(np.abs(lse[bi, h].double().cpu().numpy() - oracle.attention_lse(q, k)[0, 0])) < 1e-3
+            rdq, rdk, rdv = oracle.attention_bwd(q, k, v, P, dO[rows, h * HD:(h + 1) * HD][None, :, None])
+            rows_close(G[rows, h * HD:(h + 1) * HD], rdq[0, :, 0], 2e-2, 1e-3)
+            dk += rdk[0, :, 0]
+            dv += rdv[0, :, 0]
+        rows_close(G[rows, (H + kvh) * HD:(H + kvh + 1) * HD], dk, 2e-2, 1e-3)
+        rows_close(G[rows, (H + Hkv + kvh) * HD:(H + Hkv + kvh + 1) * HD], dv, 2e-2, 1e-3)
+
+
 def test_full_step_properties():
     from host_memory_streamed_layer_b200 import arena, mt
     cfg = arena.config(SH)
