@@ -66,6 +66,11 @@ def parse():
     ap.add_argument("--host-threads", type=int, default=0, help="host optimizer threads per replica (0: cores / N)")
     ap.add_argument("--offload-acts", action="store_true",
                     help="keep the boundary activations in pinned host memory (MT_FLAG_OFFLOAD_ACTS)")
+    ap.add_argument("--shard", action="store_true",
+                    help="sharded streaming over the N ranks (mt_create_sharded): each loads, offloads and updates "
+                         "1/N of the state, all-gather / reduce-scatter over NCCL; implies --no-defer")
+    ap.add_argument("--stash-attn", action="store_true",
+                    help="keep each layer's attention output for its backward (MT_FLAG_STASH_ATTN)")
     ap.add_argument("--grad-dtype", default="fp32", choices=["fp32", "bf16"],
                     help="dtype of the offloaded gradients (bf16: MT_FLAG_BF16_GRADS, a measured variant)")
     ap.add_argument("--no-defer", action="store_true",
@@ -127,18 +132,19 @@ def workload_desc(name, sh):
             f"bf16 weights streamed per layer")
 
 
-def flops_per_step(sh):
+def flops_per_step(sh, stash=False):
     """Model FLOPs (6 N T with causal attention) and the FLOPs this schedule
-    executes (forward, recompute without the down projection, backward,
-    flash-attention backward recompute, LM head)."""
+    executes (forward, recompute without the down projection, and without the
+    attention with stash (MT_FLAG_STASH_ATTN), backward, flash-attention
+    backward recompute, LM head)."""
     L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
     hd = d // H
     T = b * s
     Pm = d * (H + 2 * Hkv) * hd + d * H * hd + 3 * d * F
     A = 2.0 * b * s * s * H * hd  # causal attention forward (QK^T and PV over the visible half)
     model = L * (6.0 * T * Pm + 3 * A) + 6.0 * T * V * d
-    executed = L * (2.0 * T * Pm + A) + (L - 1) * (2.0 * T * (Pm - d * F) + A) + L * (4.0 * T * Pm + 2.5 * A) \
-        + 6.0 * T * V * d
+    executed = L * (2.0 * T * Pm + A) + (L - 1) * (2.0 * T * (Pm - d * F) + (0 if stash else A)) \
+        + L * (4.0 * T * Pm + 2.5 * A) + 6.0 * T * V * d
     return model, executed
 
 
@@ -444,7 +450,7 @@ def write_timeline(tl, path, workload):
 
 
 def step_bounds(sh, *, peak_tflops, link, host_gbs, h2d_bytes, d2h_bytes, update_bytes, n_unique,
-                deferred_layers=None):
+                deferred_layers=None, stash=False):
     """Phase bound of this method's dependency structure (seconds).
 
     The forward sweep and head (GPU compute or weight H2D, whichever is slower)
@@ -460,7 +466,7 @@ def step_bounds(sh, *, peak_tflops, link, host_gbs, h2d_bytes, d2h_bytes, update
     is read by every H2D and written by every D2H) to the optimizer's at the
     same rate, and measured steps beat it where DMA and CPU traffic together
     draw more from host DRAM than the CPU alone."""
-    f_fl, b_fl = phase_flops(sh)
+    f_fl, b_fl = phase_flops(sh, stash)
     L = sh["L"]
     peak = peak_tflops * 1e12
     h2d_fwd = h2d_bytes * L / (2 * L - 1)
@@ -501,15 +507,16 @@ def head_params(sh):
     return sh["d"] + sh["V"] * sh["d"]
 
 
-def phase_flops(sh):
-    """(forward + head FLOPs, backward-phase FLOPs) of the schedule."""
+def phase_flops(sh, stash=False):
+    """(forward + head FLOPs, backward-phase FLOPs) of the schedule (stash: the
+    recompute runs no attention forward)."""
     L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
     hd = d // H
     T = b * s
     Pm = d * (H + 2 * Hkv) * hd + d * H * hd + 3 * d * F
     A = 2.0 * b * s * s * H * hd
     fwd = L * (2.0 * T * Pm + A) + 6.0 * T * V * d
-    bwd = (L - 1) * (2.0 * T * (Pm - d * F) + A) + L * (4.0 * T * Pm + 2.5 * A)
+    bwd = (L - 1) * (2.0 * T * (Pm - d * F) + (0 if stash else A)) + L * (4.0 * T * Pm + 2.5 * A)
     return fwd, bwd
 
 
@@ -580,7 +587,9 @@ def main():
     sh = synth.WORKLOADS[args.workload]
     T = sh["b"] * sh["s"]
     cfg = arena.config(sh)
-    cfg.seed = 1234 + rank
+    if args.shard:
+        args.no_defer = True  # the sharded engine runs every update inside its step
+    cfg.seed = 1234 if args.shard else 1234 + rank  # one model over the ranks, or N replicas
     cfg.device = local
     # Gradients stream through a ring of host slots (14 instead of 18 B/param of
     # host memory): the 14B workload then fits a ~200 GB host, and so do eight
@@ -590,7 +599,8 @@ def main():
     cfg.flags = (mt.MT_FLAG_KERNEL_TIMING | (mt.MT_FLAG_GRAD_RING if args.grads == "ring" else 0) |
                  (0 if args.no_defer else mt.MT_FLAG_DEFER_UPDATES) |
                  (mt.MT_FLAG_BF16_GRADS if args.grad_dtype == "bf16" else 0) |
-                 (mt.MT_FLAG_OFFLOAD_ACTS if args.offload_acts else 0))
+                 (mt.MT_FLAG_OFFLOAD_ACTS if args.offload_acts else 0) |
+                 (mt.MT_FLAG_STASH_ATTN if args.stash_attn else 0))
     ncpu = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     cfg.host_threads = args.host_threads or max(1, ncpu // world)
 
@@ -614,7 +624,15 @@ def main():
     host_bw = host_optimizer_bandwidth(mt, cfg.host_threads) if rank == 0 else None
     # independent host-DRAM ceiling: STREAM triad (12 B/element, non-temporal stores)
     triad = mt.mt_host_triad_gbs(1 << 28, cfg.host_threads) if rank == 0 else None
-    ctx = mt.mt_create(cfg)
+    if args.shard:
+        nccl_id = mt.mt_shard_id() if rank == 0 else bytes(mt.MT_SHARD_ID_BYTES)
+        if dist is not None:
+            box = [nccl_id]
+            dist.broadcast_object_list(box, src=0)
+            nccl_id = box[0]
+        ctx = mt.mt_create_sharded(cfg, 0, 0, world, rank, nccl_id)
+    else:
+        ctx = mt.mt_create(cfg)
     try:
         n_e2e = max(3, (args.steps + 1) // 2)
         nsteps = args.warmup + args.steps + n_e2e
@@ -670,7 +688,7 @@ def main():
 
     if rank == 0:
         P, ptype = peaks()
-        model_f, exec_f = flops_per_step(sh)
+        model_f, exec_f = flops_per_step(sh, args.stash_attn)
         K = args.steps
         value = weak_value(T, world, K, t_dev)
         ms = t_dev / K * 1e3
@@ -688,7 +706,7 @@ def main():
         t_d2h = d2h_b / (link["d2h_gbs"] * 1e9)
         sb = step_bounds(sh, peak_tflops=peak, link=link, host_gbs=host_bw, h2d_bytes=h2d_b, d2h_bytes=d2h_b,
                          update_bytes=mean("adamw_bytes"), n_unique=n_uniq,
-                         deferred_layers=None if args.no_defer else defer_layers(sh))
+                         deferred_layers=None if args.no_defer else defer_layers(sh), stash=args.stash_attn)
         host_bytes, upd_fwd, upd_bwd = sb["update_bytes"], sb["update_bytes_fwd"], sb["update_bytes_bwd"]
         t_fwd_b, t_bwd_b, t_host_b, t_bound = sb["fwd"], sb["bwd"], sb["host_bwd"], sb["bound"]
         t_model, dram_fwd, dram_bwd = sb["model"], sb["dram_fwd"], sb["dram_bwd"]
@@ -698,12 +716,16 @@ def main():
             "dtype": "bf16", "data": "synthetic (uniform random tokens from seed, N(0,0.02) weights)",
             "config": {"workload": workload_desc(args.workload, sh), "workload_choice": wnote,
                        "global_batch": sh["b"] * world,
-                       "seq_len": sh["s"], "parallelism": "replicas" if world > 1 else "single GPU",
+                       "seq_len": sh["s"],
+                       "parallelism": (f"sharded streaming over {world} rank(s) (NCCL all-gather / reduce-scatter)"
+                                       if args.shard else "replicas" if world > 1 else "single GPU"),
                        "l2": "no flush needed: every step streams all weights (>1 GB) through HBM from host",
                        "deferred_updates": (None if args.no_defer else
                                             f"LM head + last {defer_layers(sh)} layer(s) updated during the next "
                                             "forward sweep; the timed region ends after mt_flush"),
                        "boundary_activations": "pinned host memory" if args.offload_acts else "HBM",
+                       "attention_recompute": ("none: O and LSE kept per layer (MT_FLAG_STASH_ATTN)"
+                                               if args.stash_attn else "in each layer's recompute"),
                        "grads": (f"{args.grad_dtype} gradients offloaded; " +
                                  (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
                                   if args.grads == "ring" else "full gradient arena in pinned host memory"))},

@@ -434,12 +434,390 @@ int launch_fa(const AttnArgs& a, cudaStream_t st, int* err) {
 
 }  // namespace
 
+// ===========================================================================
+// Forward, head_dim 128, two query tiles per CTA in ping-pong.
+//
+// A CTA takes 256 consecutive queries of one head as tiles A and B (128 rows
+// each) and streams the key blocks both need. Each tile has its own softmax
+// warpgroup, whose thread r owns row r of the tile for all 128 keys of a
+// block, and its own tensor memory: S (128 columns, over which the thread
+// writes its bf16 P in place, the A operand of P V) and O (128 columns). While
+// one warpgroup turns S into P, the tensor core runs the other tile's
+// products, so the MMAs and the softmax of the two tiles overlap:
+//   warp 0   TMA producer: Q_A, Q_B once, then K_j and V_j per 128-key block
+//            into two-stage rings
+//   warp 1   MMA issuer: S_A(0), S_B(0); per block j: O_A += P_A(j) V_j,
+//            S_A(j+1) once that P V is done (it reads the S_A columns),
+//            O_B += P_B(j) V_j, S_B(j+1)
+//   warps 2..5 / 6..9  softmax of tile A / tile B: row max, lazy rescale of O
+//            in tensor memory (only when a row's maximum grows by more than
+//            2^8 in exp2 units), exp2, row sum, bf16 P into tensor memory
+// Tile A needs key blocks 0 .. 2p, tile B 0 .. 2p + 1 (p the CTA's pair of
+// tiles); a tile B wholly past the sequence end does nothing. Shared memory:
+// Q_A, Q_B, two K and two V stages (192 KB); no P tile.
+// ===========================================================================
+namespace {
+
+constexpr int PP_THREADS = 320;  // producer, MMA, two softmax warpgroups
+
+struct PpCfg {
+  static constexpr int TILE = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16 (two 64-column swizzle sub-tiles)
+  static constexpr int OFF_QA = 0;
+  static constexpr int OFF_QB = TILE;
+  static constexpr int OFF_K = 2 * TILE;  // [2]
+  static constexpr int OFF_V = 4 * TILE;  // [2]
+  static constexpr int OFF_BAR = 6 * TILE;
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  // tensor-memory columns of tile t: S (and P over it) and O
+  __host__ __device__ static constexpr uint32_t c_s(int t) { return t ? 128u : 0u; }
+  __host__ __device__ static constexpr uint32_t c_o(int t) { return t ? 384u : 256u; }
+};
+
+__global__ void __launch_bounds__(PP_THREADS, 1)
+    k_flash_fwd_pp(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, FaParams p) {
+  using C = PpCfg;
+  constexpr int HD = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ[2] = {smem + C::OFF_QA, smem + C::OFF_QB};
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* q_full = bar + 0;
+  uint64_t* k_full = bar + 1;    // [2]
+  uint64_t* k_empty = bar + 3;   // [2]
+  uint64_t* v_full = bar + 5;    // [2]
+  uint64_t* v_empty = bar + 7;   // [2]
+  uint64_t* s_full = bar + 9;    // [2 tiles] S of the tile's current block in tensor memory
+  uint64_t* p_full = bar + 11;   // [2 tiles] P written (and any O rescale done), 4 warps each
+  uint64_t* pv_done = bar + 13;  // [2 tiles] the tile's P V (and every earlier MMA) done
+  uint64_t* drain = bar + 15;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 16);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 17);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pair = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.H / p.Hkv);
+  const int q0 = pair * 256;
+  const int row0 = b * p.s;
+  // key blocks each tile needs (0 for a tile wholly past the sequence end)
+  int nkv_t[2];
+  nkv_t[0] = 2 * pair + 1;
+  nkv_t[1] = (q0 + 128 < p.s) ? 2 * pair + 2 : 0;
+  const int nkv = nkv_t[1] > 0 ? nkv_t[1] : nkv_t[0];
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 4);
+      mbar_init(&pv_done[i], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
+      bool ok = true;
+      const int nq = nkv_t[1] > 0 ? 2 : 1;
+      mbar_arrive_expect_tx(q_full, nq * C::TILE);
+      for (int t = 0; t < nq; ++t)
+        for (int c = 0; c < 2; ++c) tma_load_2d(sQ[t] + c * 16384, &tmQ, q_full, h * HD + c * 64, row0 + q0 + 128 * t);
+      for (int j = 0; j < nkv; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        const int r = row0 + j * 128;
+        if (*abort_flag || !mbar_wait(&k_empty[st], ph ^ 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[st], C::TILE);
+        for (int c = 0; c < 2; ++c) tma_load_2d(sK + st * C::TILE + c * 16384, &tmK, &k_full[st], kvh * HD + c * 64, r);
+        k_last[st] = (int)ph;
+        if (*abort_flag || !mbar_wait(&v_empty[st], ph ^ 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&v_full[st], C::TILE);
+        for (int c = 0; c < 2; ++c) tma_load_2d(sV + st * C::TILE + c * 16384, &tmV, &v_full[st], kvh * HD + c * 64, r);
+        v_last[st] = (int)ph;
+      }
+      if (!ok) {
+        record_error(p.err, DEV_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+        // let every issued copy land before the CTA's shared memory goes away
+        if (!mbar_wait(q_full, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        for (int s2 = 0; s2 < 2; ++s2) {
+          if (k_last[s2] >= 0 && !mbar_wait(&k_full[s2], (uint32_t)k_last[s2])) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+          if (v_last[s2] >= 0 && !mbar_wait(&v_full[s2], (uint32_t)v_last[s2])) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, 128, false, false);  // S = Q K^T
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, HD, false, true);    // O += P V, P from tensor memory
+      const uint64_t dQ0[2] = {sdesc_sw128(smem_u32(sQ[0]), 16, 1024), sdesc_sw128(smem_u32(sQ[1]), 16, 1024)};
+      const uint64_t dK0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+      const uint64_t dV0 = sdesc_sw128(smem_u32(sV), 16384, 1024);
+      bool ok = mbar_wait(q_full, 0) && !*abort_flag;
+      bool issued = false;
+      // S_t(j) = Q_t K_j^T; K_j is released once every tile that uses it has its S.
+      auto issue_s = [&](int t, int j) -> bool {
+        const int st = j & 1;
+        if (*abort_flag || !mbar_wait(&k_full[st], (j >> 1) & 1)) return false;
+        // the S columns hold P_t(j - 1) until its P V is done
+        if (j > 0 && !mbar_wait(&pv_done[t], (j - 1) & 1)) return false;
+        tc_fence_after();
+        const uint64_t bK = dK0 + ((st * C::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t step = ((kk >> 2) * 16384 + (kk & 3) * 32) >> 4;
+          umma_bf16(tmem + C::c_s(t), dQ0[t] + step, bK + step, idesc_s, kk != 0);
+        }
+        issued = true;
+        umma_commit(&s_full[t]);
+        const bool last_user = (t == 1) || nkv_t[1] <= j;
+        if (last_user) umma_commit(&k_empty[st]);
+        return true;
+      };
+      // O_t += P_t(j) V_j; V_j is released after its last user.
+      auto issue_pv = [&](int t, int j) -> bool {
+        const int st = j & 1;
+        if (*abort_flag || !mbar_wait(&v_full[st], (j >> 1) & 1) || !mbar_wait(&p_full[t], j & 1)) return false;
+        tc_fence_after();
+        const uint64_t bV = dV0 + ((st * C::TILE) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_bf16_ts(tmem + C::c_o(t), tmem + C::c_s(t) + 8 * kk, bV + ((kk * 2048) >> 4), idesc_o, (j | kk) != 0);
+        umma_commit(&pv_done[t]);
+        const bool last_user = (t == 1) || nkv_t[1] <= j;
+        if (last_user) umma_commit(&v_empty[st]);
+        return true;
+      };
+      if (ok) ok = issue_s(0, 0);
+      if (ok && nkv_t[1] > 0) ok = issue_s(1, 0);
+      for (int j = 0; j < nkv && ok; ++j) {
+        if (j < nkv_t[0] && !issue_pv(0, j)) ok = false;
+        if (ok && j + 1 < nkv_t[0] && !issue_s(0, j + 1)) ok = false;
+        if (ok && j < nkv_t[1] && !issue_pv(1, j)) ok = false;
+        if (ok && j + 1 < nkv_t[1] && !issue_s(1, j + 1)) ok = false;
+      }
+      if (!ok) {
+        record_error(p.err, DEV_TIMEOUT_MMA);
+        *abort_flag = 1;
+      }
+      if (issued) {  // every MMA issued here completes before tensor memory is freed
+        umma_commit(drain);
+        if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+      }
+    }
+  } else {
+    // ---------------- softmax of tile t (warps 2..5: A, 6..9: B) ----------------
+    const int t = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // query row of the tile == tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const uint32_t sbase = tmem + lane_base + C::c_s(t);
+    const uint32_t obase = tmem + lane_base + C::c_o(t);
+    const int n_t = nkv_t[t];
+    const float sl2 = p.scale * 1.4426950408889634f;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_t; ++j) {
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&s_full[t], j & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // The causal mask touches only the tile's diagonal block (its last one):
+      // row r sees keys [0, r] of it; the other blocks need no test. Half a
+      // row (64 scores) is held at a time: both halves for the maximum, then
+      // the second half's probabilities are packed (32 registers) before the
+      // first half is read again, because P over keys [0, 64) overwrites the
+      // S columns [0, 32) and P over [64, 128) the columns [32, 64).
+      auto block = [&](auto diag_tag) -> bool {
+        constexpr bool DIAG = decltype(diag_tag)::value;
+        uint32_t v[64];
+        float mx = -INFINITY;
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld_32x32b_x32(sbase + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld_32x32b_x32(sbase + hf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (!DIAG || hf * 64 + e <= r) mx = fmaxf(mx, __uint_as_float(v[e]));
+        }
+        const bool raise = (m == -INFINITY) || (mx - m) * sl2 > kRescaleLog2;
+        const float corr = (raise && m != -INFINITY) ? ex2((m - mx) * sl2) : 1.f;
+        if (raise) m = mx;
+        if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          // O holds blocks < j at the old maximum: once P(j-1) V has landed,
+          // rescale the raised rows (the others multiply by 1)
+          if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&pv_done[t], (j - 1) & 1)) return false;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld_32x32b_x32(obase + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t t8[8];
+#pragma unroll
+              for (int u = 0; u < 8; ++u) t8[u] = __float_as_uint(__uint_as_float(o[e + u]) * corr);
+              tmem_st_32x32b_x8(obase + c * 32 + e, t8);
+            }
+          }
+          tmem_st_wait();
+        }
+        l *= corr;
+        const float mb = m * sl2;
+        float rs = 0.f;
+        // probabilities of keys [64 hf, 64 hf + 64) from v, as bf16 pairs
+        auto probs = [&](int hf, uint32_t (&pk)[32]) {
+#pragma unroll
+          for (int e = 0; e < 64; e += 2) {
+            const int k = hf * 64 + e;
+            float p0 = ex2(fmaf(__uint_as_float(v[e]), sl2, -mb));
+            float p1 = ex2(fmaf(__uint_as_float(v[e + 1]), sl2, -mb));
+            if (DIAG && k > r) p0 = 0.f;
+            if (DIAG && k + 1 > r) p1 = 0.f;
+            rs += p0 + p1;
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
+        };
+        uint32_t hi[32], lo[32];
+        probs(1, hi);  // v still holds keys [64, 128)
+        tmem_ld_32x32b_x32(sbase, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld_32x32b_x32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld_wait();
+        probs(0, lo);
+        // key k in column k / 2, even k in the low half (the A-operand layout)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_st_32x32b_x8(sbase + c * 8, *reinterpret_cast<const uint32_t(*)[8]>(lo + 8 * c));
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_st_32x32b_x8(sbase + 32 + c * 8, *reinterpret_cast<const uint32_t(*)[8]>(hi + 8 * c));
+        l += rs;
+        return true;
+      };
+      if (!(j == n_t - 1 ? block(std::true_type{}) : block(std::false_type{}))) {
+        ok = false;
+        break;
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
+    }
+    if (ok && n_t > 0 &&
+        (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&pv_done[t], (n_t - 1) & 1)))
+      ok = false;
+    if (!ok) {
+      record_error(p.err, DEV_TIMEOUT_EPILOGUE);
+      *abort_flag = 1;
+    } else if (n_t > 0) {
+      tc_fence_after();
+      const int qi = q0 + 128 * t + r;
+      const float inv = 1.f / l;
+      __nv_bfloat16* orow = p.O + (int64_t)(row0 + qi) * p.ldo + h * HD;
+#pragma unroll 1
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld_32x32b_x32(obase + c * 32, o);  // warp-collective: every lane loads
+        tmem_ld_wait();
+        if (qi < p.s) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[e + 0]) * inv, __uint_as_float(o[e + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[e + 4]) * inv, __uint_as_float(o[e + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[e + 6]) * inv, __uint_as_float(o[e + 7]) * inv);
+            reinterpret_cast<uint4*>(orow + c * 32 + e)[0] = w;
+          }
+        }
+      }
+      if (qi < p.s) p.LSE[((int64_t)b * p.H + h) * p.s + qi] = m * p.scale + logf(l);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+int launch_fa_pp(const AttnArgs& a, cudaStream_t st, int* err) {
+  using C = PpCfg;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_flash_fwd_pp, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return MT_ERR_CUDA;
+    attr = true;
+  }
+  const int64_t T = (int64_t)a.b * a.s;
+  CUtensorMap mq, mk, mv;
+  if (!fa_map(&mq, a.q, (int64_t)a.H * 128, T, a.ldqkv) || !fa_map(&mk, a.k, (int64_t)a.Hkv * 128, T, a.ldqkv) ||
+      !fa_map(&mv, a.v, (int64_t)a.Hkv * 128, T, a.ldqkv))
+    return MT_ERR_ARG;
+  FaParams p{(__nv_bfloat16*)a.o, a.ldo, a.lse, a.s, a.H, a.Hkv, a.scale, err};
+  dim3 grid((a.s + 255) / 256, a.H, a.b);
+  k_flash_fwd_pp<<<grid, PP_THREADS, C::SMEM, st>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+}  // namespace
+
+namespace {
+int g_fa_variant = 0;  // 0 automatic, 1 one query tile per CTA, 2 two tiles in ping-pong
+}
+
+int attention_fwd_variant(int v) {
+  const int was = g_fa_variant;
+  g_fa_variant = v;
+  return was;
+}
+
 int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   if (a.b <= 0 || a.s <= 0) return MT_OK;
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.o) || (a.ldqkv % 8) || (a.ldo % 8)) return MT_ERR_ARG;
   if (a.hd == 64) return launch_fa<64>(a, st, err);
-  if (a.hd == 128) return launch_fa<128>(a, st, err);
+  // head dim 128: two query tiles per CTA from 8192 tokens on (measured on
+  // B200: 939 against 903 TFLOP/s at s = 16384, but 536 against 562 at
+  // s = 2048, where the pairs' short rows leave their prologue and epilogue
+  // exposed)
+  if (a.hd == 128) {
+    const int v = g_fa_variant ? g_fa_variant : (a.s >= 8192 ? 2 : 1);
+    return v == 2 ? launch_fa_pp(a, st, err) : launch_fa<128>(a, st, err);
+  }
   return MT_ERR_CONFIG;
 }
 
@@ -702,7 +1080,10 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     // dQ^T of an iteration (complete: the caller waited for mma_done): this
     // warp's 32 query columns for head column r, added to the fp32 dQ
     // accumulator with reductions from registers (a warp's 32 lanes are 32
-    // consecutive head columns of one query row: 128 coalesced bytes).
+    // consecutive head columns of one query row: 128 coalesced bytes, whole
+    // 32-byte sectors; the reductions are bound by L2 sector operations, and
+    // a row-per-thread form with 16-byte vector reductions, which touches
+    // half-sectors, measured 13-19 % slower).
     auto flush_dq = [&](int hq, int q0) {
       uint32_t v[32];
       tmem_ld_32x32b_x32(tmem + lane_base + C::C_DP + qg * FB_QW, v);

@@ -402,74 +402,6 @@ __global__ void __launch_bounds__(256) k_softmax_ce(const float* __restrict__ z,
   }
 }
 
-// The same cross-entropy with the logit row read from HBM once: rows of up to
-// kCeSmemFloats floats are staged in shared memory while their maximum is
-// taken, then the exponentials' sum and dz are computed from there (6 V bytes
-// of DRAM traffic per row instead of 10 V). 512 threads; each thread keeps
-// four 16-byte loads in flight to cover the latency with one CTA per SM.
-constexpr int kCeSmemFloats = 48 * 1024;  // 192 KB
-
-__global__ void __launch_bounds__(512) k_softmax_ce_smem(const float* __restrict__ z, int64_t ldz,
-                                                         const int* __restrict__ labels, bf16* __restrict__ dz,
-                                                         int64_t lddz, float* __restrict__ row_loss, int V,
-                                                         float scale) {
-  extern __shared__ float4 srow[];
-  __shared__ float sh[16];
-  const int row = blockIdx.x;
-  const float4* zr = reinterpret_cast<const float4*>(z + (int64_t)row * ldz);
-  const int n4 = V >> 2;
-  // load + maximum
-  float m = -INFINITY;
-  for (int i0 = threadIdx.x; i0 < n4; i0 += 4 * 512) {
-    float4 v[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (i0 + u * 512 < n4) v[u] = zr[i0 + u * 512];
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      if (i0 + u * 512 < n4) {
-        srow[i0 + u * 512] = v[u];
-        m = fmaxf(m, fmaxf(fmaxf(v[u].x, v[u].y), fmaxf(v[u].z, v[u].w)));
-      }
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  if (l == 0) sh[w] = m;
-  __syncthreads();
-  float M = sh[0];
-#pragma unroll
-  for (int i = 1; i < 16; ++i) M = fmaxf(M, sh[i]);
-  __syncthreads();
-  // sum of exponentials (each thread re-reads the elements it staged)
-  float sum = 0.f;
-  for (int i = threadIdx.x; i < n4; i += 512) {
-    const float4 v = srow[i];
-    sum += expf(v.x - M) + expf(v.y - M) + expf(v.z - M) + expf(v.w - M);
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (l == 0) sh[w] = sum;
-  __syncthreads();
-  float S = 0.f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) S += sh[i];
-  const float lse = M + logf(S);
-  const int y = labels[row];
-  if (threadIdx.x == 0) row_loss[row] = lse - reinterpret_cast<const float*>(srow)[y];
-  bf16* dr = dz + (int64_t)row * lddz;
-  for (int i = threadIdx.x; i < n4; i += 512) {
-    const float4 v = srow[i];
-    const int j = 4 * i;
-    float p0 = expf(v.x - lse), p1 = expf(v.y - lse), p2 = expf(v.z - lse), p3 = expf(v.w - lse);
-    if (y == j) p0 -= 1.f;
-    if (y == j + 1) p1 -= 1.f;
-    if (y == j + 2) p2 -= 1.f;
-    if (y == j + 3) p3 -= 1.f;
-    store_bf16x4(dr + j, p0 * scale, p1 * scale, p2 * scale, p3 * scale);
-  }
-}
-
 // Sum of n floats by one block, fixed order (per-thread strided, then a tree).
 __global__ void k_sum_all(const float* __restrict__ v, int n, float* __restrict__ out, int accumulate) {
   __shared__ float sh[8];
@@ -561,18 +493,6 @@ int launch_embed_bwd(const int* offs, const int* pos, int n_unique, const float*
 int launch_softmax_ce(const float* z, int64_t ldz, const int* labels, void* dz, int64_t lddz, float* row_loss,
                       int Tc, int V, float scale, cudaStream_t st) {
   if (Tc <= 0) return MT_OK;
-  if (V <= kCeSmemFloats) {  // the row fits in shared memory: one read of the logits
-    static bool attr = false;
-    const int smem = V * 4;
-    if (!attr) {
-      if (cudaFuncSetAttribute(k_softmax_ce_smem, cudaFuncAttributeMaxDynamicSharedMemorySize, kCeSmemFloats * 4) !=
-          cudaSuccess)
-        return MT_ERR_CUDA;
-      attr = true;
-    }
-    k_softmax_ce_smem<<<Tc, 512, smem, st>>>(z, ldz, labels, (bf16*)dz, lddz, row_loss, V, scale);
-    return launch_status();
-  }
   k_softmax_ce<<<Tc, 256, 0, st>>>(z, ldz, labels, (bf16*)dz, lddz, row_loss, V, scale);
   return launch_status();
 }

@@ -39,6 +39,7 @@
 #include "host_adamw.h"
 #include "layout.h"
 #include "mt_internal.h"
+#include "nccl_dl.h"
 
 namespace mt {
 
@@ -193,6 +194,19 @@ struct mt_ctx {
   mt_stats stats{};
   int64_t launches = 0;
   std::vector<int> load_seq;  // layer of each weight load
+
+  // ---- sharded streaming (mt_create_sharded) ----
+  // Two communicators over the same ranks: the H2D stream's all-gathers and
+  // the compute stream's reductions, so that each communicator's collectives
+  // run on one stream in one program order on every rank.
+  const NcclApi* nccl = nullptr;
+  ncclComm_t comm_h2d = nullptr, comm_comp = nullptr;
+  mt_shard plan{};              // this rank's element ranges (world 1, everything: unsharded)
+  uint16_t* d_embed_w = nullptr;  // bf16 embedding table on the device, [world * rows, d]
+  float* d_embed_g = nullptr;     // dense embedding gradient, [world * rows, d]
+  int32_t* d_uid = nullptr;       // unique token ids of the step, [T]
+  float* emb_own_h = nullptr;     // pinned: this rank's rows of the mean embedding gradient
+  cudaEvent_t ev_embw = nullptr;  // embedding table all-gathered
 };
 
 namespace mteng {
@@ -216,6 +230,30 @@ int set_err(mt_ctx* c, int code, const std::string& m) {
     int r_ = (call);            \
     if (r_ != MT_OK) return r_; \
   } while (0)
+#define NK(call)                                                                                       \
+  do {                                                                                                 \
+    ncclResult_t e_ = (c->nccl->call);                                                                 \
+    if (e_ != ncclSuccess)                                                                             \
+      return set_err(c, MT_ERR_CUDA, std::string("nccl") + #call + ": " + c->nccl->GetErrorString(e_)); \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// Sharded streaming: rank r of `world` owns elements [begin, end) of every
+// layer block and of the [final gain | LM head] block, and embedding rows
+// [row_begin, row_end). Each loads only its own part over the host link and
+// all-gathers the rest; the gradients are averaged over the ranks with a
+// reduce-scatter that leaves each rank its own part, which it checks,
+// offloads and updates. Device blocks are padded to world * chunk elements.
+// ---------------------------------------------------------------------------
+bool sharded(const mt_ctx* c) { return c->comm_comp != nullptr; }
+
+size_t embed_rows_chunk(const mt_shard& p, int V) { return (size_t)((V + p.world - 1) / p.world); }
+
+// Reduce-scatter (mean over ranks) of a padded fp32 block on the compute
+// stream: rank r's chunk ends up at blk + r * chunk. Then the finite check of
+// that chunk into flag `idx`, and the flag's maximum over the ranks, so that
+// every rank takes the same skip decision.
+int reduce_own_chunk(mt_ctx* c, float* blk, size_t chunk, size_t own_begin, size_t own_end, int idx);
 
 // ---------------------------------------------------------------------------
 // Kernel wrappers with launch counting and optional event timing.
@@ -319,6 +357,25 @@ int check_finite(mt_ctx* c, const float* g, size_t n, int idx) {
   return MT_OK;
 }
 
+int reduce_own_chunk(mt_ctx* c, float* blk, size_t chunk, size_t own_begin, size_t own_end, int idx) {
+  NK(ReduceScatter(blk, blk + (size_t)c->plan.rank * chunk, chunk, ncclFloat32, ncclAvg, c->comm_comp, c->s_comp));
+  CKM(check_finite(c, blk + own_begin, own_end - own_begin, idx));
+  NK(AllReduce(c->d_flags + idx, c->d_flags + idx, 1, ncclInt32, ncclMax, c->comm_comp, c->s_comp));
+  return MT_OK;
+}
+
+// Rows of the step's unique tokens (row u for token uid[u]) into a zeroed
+// dense [rows, d] gradient; d is a multiple of 4.
+__global__ void k_scatter_rows(const float* __restrict__ rows, const int32_t* __restrict__ uid, int n,
+                               float* __restrict__ dst, int d) {
+  const int d4 = d / 4;
+  for (int u = blockIdx.x; u < n; u += gridDim.x) {
+    const float4* src = reinterpret_cast<const float4*>(rows + (size_t)u * d);
+    float4* out = reinterpret_cast<float4*>(dst + (size_t)uid[u] * d);
+    for (int i = threadIdx.x; i < d4; i += blockDim.x) out[i] = src[i];
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Boundary activations on the device. Resident: x_l at xb[l]. With
 // MT_FLAG_OFFLOAD_ACTS three [T, d] slots: the forward alternates slots 0 and
@@ -341,10 +398,28 @@ float* x_bwd(mt_ctx* c, int l) {
   return c->xb + (size_t)(((L - 2 - l) % 2 == 0) ? 2 : ((L - 1) & 1)) * n;
 }
 
+// Attention output O [T, H hd] (bf16) and log-sum-exp [b, H, s] of layer l:
+// one buffer for every layer, or with MT_FLAG_STASH_ATTN one per layer, kept
+// from the forward sweep to the layer's backward, so that the recompute runs
+// no attention forward.
+bool stash_attn(const mt_ctx* c) { return (c->cfg.flags & MT_FLAG_STASH_ATTN) != 0; }
+
+uint16_t* ao_of(mt_ctx* c, int l) {
+  const Shapes& s = c->lay.sh;
+  return c->ao_b + (stash_attn(c) ? (size_t)l * s.T * s.Hd : 0);
+}
+
+float* lse_of(mt_ctx* c, int l) {
+  const Shapes& s = c->lay.sh;
+  return c->lse + (stash_attn(c) ? (size_t)l * s.b * s.H * s.s : 0);
+}
+
 // ---------------------------------------------------------------------------
 // Layer forward from x with the weights of `slot`. With xo the layer output
 // goes there; otherwise (recompute) the down projection is skipped, since the
-// backward only needs the intermediates.
+// backward only needs the intermediates, and with MT_FLAG_STASH_ATTN so is the
+// attention, whose output the forward sweep kept (the forward is
+// deterministic: the kept O and LSE are the ones a recompute would produce).
 // ---------------------------------------------------------------------------
 int layer_fwd(mt_ctx* c, int l, int slot, const float* x, float* xo) {
   const Shapes& s = c->lay.sh;
@@ -363,17 +438,17 @@ int layer_fwd(mt_ctx* c, int l, int slot, const float* x, float* xo) {
   a.k = c->qkv_b + s.Hd;
   a.v = c->qkv_b + s.Hd + s.Hkv * s.hd;
   a.ldqkv = s.Nqkv;
-  a.o = c->ao_b;
+  a.o = ao_of(c, l);
   a.ldo = s.Hd;
-  a.lse = c->lse;
+  a.lse = lse_of(c, l);
   a.b = s.b;
   a.s = s.s;
   a.H = s.H;
   a.Hkv = s.Hkv;
   a.hd = s.hd;
   a.scale = 1.0f / sqrtf((float)s.hd);
-  CKM(attn(c, a, false));
-  CKM(gemm(c, gd_fwd(c->ao_b, s.Hd, W + y.bf_o, s.Hd, c->h_f, s.d, EPI_F32_ADD, x, s.T, s.d, s.Hd)));
+  if (xo || !stash_attn(c)) CKM(attn(c, a, false));
+  CKM(gemm(c, gd_fwd(ao_of(c, l), s.Hd, W + y.bf_o, s.Hd, c->h_f, s.d, EPI_F32_ADD, x, s.T, s.d, s.Hd)));
   KL(launch_rmsnorm_fwd(c->h_f, W + y.bf_g2, c->w_b, c->r2, s.T, s.d, c->cfg.norm_eps, st), 1);
   CKM(gemm(c, gd_fwd(c->w_b, s.d, W + y.bf_gu, s.d, c->gu_b, 2 * s.F, EPI_BF16, nullptr, s.T, 2 * s.F, s.d)));
   KL(launch_swiglu_fwd(c->gu_b, c->act_b, s.T, s.F, st), 1);
@@ -405,7 +480,7 @@ int layer_bwd(mt_ctx* c, int l, int slot, const float* x, float* gs, const float
                         T, d, st),
      2);
   // output projection
-  CKM(gemm(c, gd_dw(c->dhb, d, c->ao_b, s.Hd, G(MT_T_WO), s.Hd, EPI_F32, d, s.Hd, T)));
+  CKM(gemm(c, gd_dw(c->dhb, d, ao_of(c, l), s.Hd, G(MT_T_WO), s.Hd, EPI_F32, d, s.Hd, T)));
   CKM(gemm(c, gd_dx(c->dhb, d, W + y.bf_o, s.Hd, c->dao_b, s.Hd, EPI_BF16, T, s.Hd, d)));
   // attention
   AttnArgs a{};
@@ -413,9 +488,9 @@ int layer_bwd(mt_ctx* c, int l, int slot, const float* x, float* gs, const float
   a.k = c->qkv_b + s.Hd;
   a.v = c->qkv_b + s.Hd + s.Hkv * s.hd;
   a.ldqkv = s.Nqkv;
-  a.o = c->ao_b;
+  a.o = ao_of(c, l);
   a.ldo = s.Hd;
-  a.lse = c->lse;
+  a.lse = lse_of(c, l);
   a.dout = c->dao_b;
   a.dvec = c->dvec;
   a.dq_acc = c->dqacc;
@@ -440,6 +515,8 @@ int layer_bwd(mt_ctx* c, int l, int slot, const float* x, float* gs, const float
   KL(launch_rmsnorm_bwd(x, W + y.bf_g1, c->r1, c->tmp_f, c->dh_f, gout, nullptr, c->rms_part, G(MT_T_ATTN_NORM), T,
                         d, st),
      2);
+  if (sharded(c))
+    return reduce_own_chunk(c, gs, c->plan.layer_chunk, c->plan.layer_begin, c->plan.layer_end, l);
   return check_finite(c, gs, y.layer_end(l) - base, l);
 }
 
@@ -464,7 +541,10 @@ int head_step(mt_ctx* c, float* gout) {
     CKM(gemm(c, gd_dx(c->dz_b, V, Wh, d, c->tmp_f + (size_t)t0 * d, d, EPI_F32, tc, d, V)));
   }
   KL(launch_sum_all(c->rowloss, T, c->d_loss, 0, st), 1);
+  if (sharded(c)) NK(AllReduce(c->d_loss, c->d_loss, 1, ncclFloat32, ncclAvg, c->comm_comp, st));
   KL(launch_rmsnorm_bwd(xL, gf, c->rf, c->tmp_f, nullptr, gout, nullptr, c->rms_part, dgf, T, d, st), 2);
+  if (sharded(c))
+    return reduce_own_chunk(c, c->d_head_g, c->plan.head_chunk, c->plan.head_begin, c->plan.head_end, s.L);
   return check_finite(c, c->d_head_g, c->lay.head_block, s.L);
 }
 
@@ -573,7 +653,20 @@ std::vector<Seg> layer_or_head_segs(mt_ctx* c, int l, const uint8_t* g) {
       segs.push_back(grad_seg(c, y.head.off, y.head.n, c->bf_head + align_up(y.sh.d, 128),
                               c->grad_head + y.gf_pad * c->gsz));
   }
-  return segs;
+  if (!sharded(c)) return segs;
+  // Sharded: only this rank's elements [lo, hi) of the block (offsets from the
+  // block's first arena float); the other ranks update the rest.
+  const size_t base = l >= 0 ? y.layer_begin(l) : y.final_norm.off;
+  const size_t lo = base + (l >= 0 ? c->plan.layer_begin : c->plan.head_begin);
+  const size_t hi = base + (l >= 0 ? c->plan.layer_end : c->plan.head_end);
+  std::vector<Seg> mine;
+  for (const Seg& sg : segs) {
+    const size_t b = std::max(sg.off, lo), e = std::min(sg.off + sg.n, hi);
+    if (b >= e) continue;
+    const size_t k = b - sg.off;
+    mine.push_back(Seg{b, e - b, sg.bf ? sg.bf + k : nullptr, sg.g ? sg.g + k : nullptr, sg.g16 ? sg.g16 + k : nullptr});
+  }
+  return mine;
 }
 
 // Segments of the zero-gradient update of every embedding row not listed in
@@ -631,7 +724,16 @@ void run_job_body(mt_ctx* c, const Job& j) {
     adamw_segments(c, untouched_segs(c, c->uniq), c->step);
     return;
   }
-  if (j.kind == Job::EMBED) {
+  if (j.kind == Job::EMBED && sharded(c)) {
+    // This rank's rows of the mean dense gradient, checked on the device (the
+    // flag came back with them, its maximum over the ranks): the gradient
+    // arena reports them, the update below reads them from the staging rows.
+    const size_t d = s.d, rb = (size_t)c->plan.embed_row_begin, re = (size_t)c->plan.embed_row_end;
+    if (c->grad)
+      parallel_ranges(*c->pool, (re - rb) * d, [&](size_t b, size_t e) {
+        memcpy(reinterpret_cast<float*>(c->grad) + y.embed.off + rb * d + b, c->emb_own_h + b, (e - b) * 4);
+      });
+  } else if (j.kind == Job::EMBED) {
     // Touched rows: check this step's gradient rows for NaN/Inf and, with a
     // gradient arena, put last step's touched rows back to zero and scatter
     // this step's rows in (every other row's stored gradient is 0). The update
@@ -708,6 +810,9 @@ void run_job_body(mt_ctx* c, const Job& j) {
     segs = layer_or_head_segs(c, j.kind == Job::HEAD ? -1 : j.layer, j.g);
   } else if (y.tied) {  // EMBED, tied: one dense update of the whole table
     segs.push_back({y.embed.off, y.embed.n, c->bf_embed, reinterpret_cast<const float*>(c->grad_head) + y.gf_pad});
+  } else if (sharded(c)) {  // EMBED, sharded: this rank's rows, dense (untouched rows have zero gradient)
+    const size_t rb = (size_t)c->plan.embed_row_begin, re = (size_t)c->plan.embed_row_end;
+    if (re > rb) segs.push_back({y.embed.off + rb * s.d, (re - rb) * s.d, c->bf_embed + rb * s.d, c->emb_own_h});
   } else {
     for (size_t u = 0; u < c->uniq.size(); ++u) {
       const size_t r = (size_t)c->uniq[u];
@@ -843,8 +948,17 @@ int issue_load(mt_ctx* c, int i) {
   if (i < y.sh.L && i >= y.sh.L - c->defer_layers) CKM(await_deferred(c, i));  // forward load of a deferred layer
   if (i >= 2) CK(cudaStreamWaitEvent(c->s_h2d, c->ev_slotfree[i - 2], 0));
   CK(cudaEventRecord(c->ev_h2d_start[i], c->s_h2d));
-  CK(cudaMemcpyAsync(c->wslot[slot], c->bf_layers + (size_t)c->load_seq[i] * y.bf_layer, y.bf_layer * 2,
-                     cudaMemcpyHostToDevice, c->s_h2d));
+  const uint16_t* src = c->bf_layers + (size_t)c->load_seq[i] * y.bf_layer;
+  if (sharded(c)) {  // this rank's part over the host link, the rest from the peers
+    const mt_shard& p = c->plan;
+    if (p.layer_end > p.layer_begin)
+      CK(cudaMemcpyAsync(c->wslot[slot] + p.layer_begin, src + p.layer_begin, (p.layer_end - p.layer_begin) * 2,
+                         cudaMemcpyHostToDevice, c->s_h2d));
+    NK(AllGather(c->wslot[slot] + (size_t)p.rank * p.layer_chunk, c->wslot[slot], p.layer_chunk, ncclBfloat16,
+                 c->comm_h2d, c->s_h2d));
+  } else {
+    CK(cudaMemcpyAsync(c->wslot[slot], src, y.bf_layer * 2, cudaMemcpyHostToDevice, c->s_h2d));
+  }
   CK(cudaEventRecord(c->ev_wready[i], c->s_h2d));
   return MT_OK;
 }
@@ -853,7 +967,14 @@ int issue_load(mt_ctx* c, int i) {
 // embeddings the head part is the streamed embedding table.
 int copy_head_weights(mt_ctx* c, cudaStream_t st) {
   const size_t g = align_up(c->lay.sh.d, 128), n = (size_t)c->lay.sh.V * c->lay.sh.d;
-  if (c->lay.tied) {
+  if (sharded(c)) {  // (on the H2D stream: its communicator)
+    const mt_shard& p = c->plan;
+    if (p.head_end > p.head_begin)
+      CK(cudaMemcpyAsync(c->d_head_w + p.head_begin, c->bf_head + p.head_begin, (p.head_end - p.head_begin) * 2,
+                         cudaMemcpyHostToDevice, st));
+    NK(AllGather(c->d_head_w + (size_t)p.rank * p.head_chunk, c->d_head_w, p.head_chunk, ncclBfloat16, c->comm_h2d,
+                 st));
+  } else if (c->lay.tied) {
     CK(cudaMemcpyAsync(c->d_head_w, c->bf_head, g * 2, cudaMemcpyHostToDevice, st));
     CK(cudaMemcpyAsync(c->d_head_w + g, c->bf_embed, n * 2, cudaMemcpyHostToDevice, st));
   } else {
@@ -895,10 +1016,15 @@ int offload_layer(mt_ctx* c, int l, int k) {
     KL(launch_cast_f32_bf16(c->gslot[k & 1], c->gslot16[k & 1], (int64_t)(e - b), c->s_comp), 1);
     src = c->gslot16[k & 1];
   }
+  // the part of the block that crosses the link: all of it, or this rank's own
+  const size_t ob = sharded(c) ? c->plan.layer_begin : 0;
+  const size_t on = sharded(c) ? c->plan.layer_end - c->plan.layer_begin : e - b;
   CK(cudaEventRecord(c->ev_gready[k], c->s_comp));
   CK(cudaStreamWaitEvent(c->s_d2h, c->ev_gready[k], 0));
   CK(cudaEventRecord(c->ev_d2h_start[k], c->s_d2h));
-  CK(cudaMemcpyAsync(dst, src, (e - b) * gsz, cudaMemcpyDeviceToHost, c->s_d2h));
+  if (on > 0)
+    CK(cudaMemcpyAsync(dst + ob * gsz, static_cast<const uint8_t*>(src) + ob * gsz, on * gsz, cudaMemcpyDeviceToHost,
+                       c->s_d2h));
   CK(cudaMemcpyAsync(c->flags_h + l, c->d_flags + l, 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaEventRecord(c->ev_gdrained[k], c->s_d2h));
   Job j{Job::LAYER, l, c->ev_gdrained[k], l, dst};
@@ -945,8 +1071,21 @@ int enqueue_step(mt_ctx* c, int n_unique) {
 
   CK(cudaEventRecord(c->ev_step_start, sc));
   CK(cudaMemsetAsync(c->d_err, 0, sizeof(int32_t), sc));  // error word of this step's kernels
-  CK(cudaMemcpyAsync(c->d_tok, c->stage_i, (size_t)(4 * T + 1) * 4, cudaMemcpyHostToDevice, sc));
-  KL(launch_embed_fwd(c->d_tok, c->bf_embed_dev, x_fwd(c, 0), T, d, sc), 1);
+  CK(cudaMemcpyAsync(c->d_tok, c->stage_i, (size_t)(5 * T + 1) * 4, cudaMemcpyHostToDevice, sc));
+  if (sharded(c)) {
+    // The embedding table lives on the device: this rank's rows (updated on
+    // the host in the last step) over the link, the rest from the peers.
+    const mt_shard& p = c->plan;
+    const size_t rows = embed_rows_chunk(p, s.V), rb = (size_t)p.embed_row_begin, re = (size_t)p.embed_row_end;
+    if (re > rb)
+      CK(cudaMemcpyAsync(c->d_embed_w + rb * d, c->bf_embed + rb * d, (re - rb) * d * 2, cudaMemcpyHostToDevice,
+                         c->s_h2d));
+    NK(AllGather(c->d_embed_w + (size_t)p.rank * rows * d, c->d_embed_w, rows * d, ncclBfloat16, c->comm_h2d,
+                 c->s_h2d));
+    CK(cudaEventRecord(c->ev_embw, c->s_h2d));
+    CK(cudaStreamWaitEvent(sc, c->ev_embw, 0));
+  }
+  KL(launch_embed_fwd(c->d_tok, sharded(c) ? c->d_embed_w : c->bf_embed_dev, x_fwd(c, 0), T, d, sc), 1);
   CKM(stash_act(c, 0));
   CKM(issue_load(c, 0));
   if (nloads > 1) CKM(issue_load(c, 1));
@@ -977,7 +1116,10 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         CK(cudaEventRecord(c->ev_head_gready, sc));
         CK(cudaStreamWaitEvent(c->s_d2h, c->ev_head_gready, 0));
         CK(cudaEventRecord(c->ev_head_d2h_start, c->s_d2h));
-        CK(cudaMemcpyAsync(c->grad_head, hsrc, n * c->gsz, cudaMemcpyDeviceToHost, c->s_d2h));
+        const size_t hb = sharded(c) ? c->plan.head_begin : 0, he = sharded(c) ? c->plan.head_end : n;
+        if (he > hb)
+          CK(cudaMemcpyAsync(c->grad_head + hb * c->gsz, static_cast<const uint8_t*>(hsrc) + hb * c->gsz,
+                             (he - hb) * c->gsz, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaMemcpyAsync(c->flags_h + L, c->d_flags + L, 4, cudaMemcpyDeviceToHost, c->s_d2h));
         CK(cudaEventRecord(c->ev_head_drained, c->s_d2h));
         Job hj{Job::HEAD, -1, c->ev_head_drained, L};
@@ -1018,17 +1160,38 @@ int enqueue_step(mt_ctx* c, int n_unique) {
   CK(cudaEventRecord(c->ev_bwd_end, sc));
   // embedding gradient rows, in token order per unique id
   KL(launch_embed_bwd(c->d_offs, c->d_pos, n_unique, gin, c->tmp_f, d, sc), 1);
-  CK(cudaEventRecord(c->ev_emb_ready, sc));
-  CK(cudaStreamWaitEvent(c->s_d2h, c->ev_emb_ready, 0));
-  CK(cudaEventRecord(c->ev_emb_d2h_start, c->s_d2h));
-  CK(cudaMemcpyAsync(c->emb_rows_h, c->tmp_f, (size_t)n_unique * d * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  if (sharded(c)) {
+    // dense [world * rows, d] gradient, averaged over the ranks by rows
+    const mt_shard& p = c->plan;
+    const size_t rows = embed_rows_chunk(p, s.V), rb = (size_t)p.embed_row_begin, re = (size_t)p.embed_row_end;
+    CK(cudaMemsetAsync(c->d_embed_g, 0, (size_t)p.world * rows * d * 4, sc));
+    if (n_unique > 0) {
+      k_scatter_rows<<<std::min(n_unique, 1184), 128, 0, sc>>>(c->tmp_f, c->d_uid, n_unique, c->d_embed_g, d);
+      CK(cudaGetLastError());
+      c->launches += 1;
+    }
+    CKM(reduce_own_chunk(c, c->d_embed_g, rows * d, rb * d, re * d, L + 1));
+    CK(cudaEventRecord(c->ev_emb_ready, sc));
+    CK(cudaStreamWaitEvent(c->s_d2h, c->ev_emb_ready, 0));
+    CK(cudaEventRecord(c->ev_emb_d2h_start, c->s_d2h));
+    if (re > rb)
+      CK(cudaMemcpyAsync(c->emb_own_h, c->d_embed_g + rb * d, (re - rb) * d * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+    CK(cudaMemcpyAsync(c->flags_h + L + 1, c->d_flags + L + 1, 4, cudaMemcpyDeviceToHost, c->s_d2h));
+  } else {
+    CK(cudaEventRecord(c->ev_emb_ready, sc));
+    CK(cudaStreamWaitEvent(c->s_d2h, c->ev_emb_ready, 0));
+    CK(cudaEventRecord(c->ev_emb_d2h_start, c->s_d2h));
+    CK(cudaMemcpyAsync(c->emb_rows_h, c->tmp_f, (size_t)n_unique * d * 4, cudaMemcpyDeviceToHost, c->s_d2h));
+    c->flags_h[L + 1] = 0;  // set by the host's own check of the rows
+  }
   CK(cudaMemcpyAsync(c->misc_h + 2, c->d_err, 4, cudaMemcpyDeviceToHost, c->s_d2h));
   CK(cudaEventRecord(c->ev_emb_drained, c->s_d2h));
-  c->flags_h[L + 1] = 0;
   push_job(c, Job{Job::EMBED, -1, c->ev_emb_drained, L + 1});
   // Without deferral the untouched rows' update follows the step's last check.
-  // (tied embeddings: every row has a head gradient, so the EMBED job updates them all)
-  if (!(c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !y.tied) push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, L + 1});
+  // (tied embeddings: every row has a head gradient, so the EMBED job updates
+  // them all; sharded: the EMBED job's dense rows include them)
+  if (!(c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !y.tied && !sharded(c))
+    push_job(c, Job{Job::EMBED_UNTOUCHED, -1, nullptr, L + 1});
   CK(cudaMemcpyAsync(c->misc_h, c->d_loss, 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaMemcpyAsync(c->misc_h + 1, c->d_err, 4, cudaMemcpyDeviceToHost, sc));
   CK(cudaEventRecord(c->ev_step_end, sc));
@@ -1061,12 +1224,19 @@ void collect_stats(mt_ctx* c) {
   st.wait_weights_ms = wait;
   const Layout& y = c->lay;
   const double act_bytes = offload_acts(c) && L >= 3 ? 4.0 * (L - 2) * y.sh.T * y.sh.d : 0.0;
-  st.h2d_bytes = act_bytes + (double)c->load_seq.size() * y.bf_layer * 2 +
-                 (double)(align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d) * 2 + 4.0 * (4 * y.sh.T + 1) +
-                 (double)y.sh.T * y.sh.d * 2;  // embedding rows read in place
-  st.d2h_bytes = act_bytes + (double)c->gsz * y.head_block +
-                 4.0 * c->uniq.size() * y.sh.d + 12.0;
-  for (int l = 0; l < L; ++l) st.d2h_bytes += (double)c->gsz * (y.layer_end(l) - y.layer_begin(l));
+  if (sharded(c)) {  // this rank's parts only; the rest crosses NVLink
+    const mt_shard& p = c->plan;
+    const double lay = (double)(p.layer_end - p.layer_begin), head = (double)(p.head_end - p.head_begin);
+    const double rows = (double)(p.embed_row_end - p.embed_row_begin) * y.sh.d;
+    st.h2d_bytes = act_bytes + (double)c->load_seq.size() * lay * 2 + head * 2 + rows * 2 + 4.0 * (5 * y.sh.T + 1);
+    st.d2h_bytes = act_bytes + 4.0 * (head + rows + (double)L * lay) + 4.0 * (L + 4);
+  } else {
+    st.h2d_bytes = act_bytes + (double)c->load_seq.size() * y.bf_layer * 2 +
+                   (double)(align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d) * 2 + 4.0 * (5 * y.sh.T + 1) +
+                   (double)y.sh.T * y.sh.d * 2;  // embedding rows read in place
+    st.d2h_bytes = act_bytes + (double)c->gsz * y.head_block + 4.0 * c->uniq.size() * y.sh.d + 12.0;
+    for (int l = 0; l < L; ++l) st.d2h_bytes += (double)c->gsz * (y.layer_end(l) - y.layer_begin(l));
+  }
   st.adamw_ms = c->adamw_s * 1e3;
   st.adamw_bytes = c->adamw_bytes;
   st.gemm_flops = st.gemm_ms = st.attn_flops = st.attn_ms = 0;
@@ -1089,19 +1259,40 @@ void collect_stats(mt_ctx* c) {
 // ---------------------------------------------------------------------------
 // Create / destroy helpers.
 // ---------------------------------------------------------------------------
-size_t device_bytes(const Layout& y, int Tc, bool g16, bool offload) {
+// Elements of a device weight / gradient slot and of the device head block:
+// the blocks themselves, or padded to world * chunk when sharded.
+size_t slot_elems(const Layout& y, const mt_shard* p) {
+  return p ? (size_t)p->world * p->layer_chunk : y.bf_layer;
+}
+size_t gslot_elems(const Layout& y, const mt_shard* p) {
+  return p ? (size_t)p->world * p->layer_chunk : y.layer_end(0) - y.layer_begin(0);
+}
+size_t head_w_elems(const Layout& y, const mt_shard* p) {
+  return p ? (size_t)p->world * p->head_chunk : align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d;
+}
+size_t head_g_elems(const Layout& y, const mt_shard* p) {
+  return p ? (size_t)p->world * p->head_chunk : y.head_block;
+}
+
+size_t device_bytes(const Layout& y, int Tc, uint32_t flags, const mt_shard* plan = nullptr) {
+  const bool g16 = (flags & MT_FLAG_BF16_GRADS) != 0, offload = (flags & MT_FLAG_OFFLOAD_ACTS) != 0;
+  const size_t n_attn = (flags & MT_FLAG_STASH_ATTN) ? (size_t)y.sh.L : 1;  // O / LSE buffers
   const Shapes& s = y.sh;
   const size_t T = s.T, d = s.d, F = s.F, V = s.V;
   const size_t A = 256;
   size_t b = 0;
   auto add = [&](size_t bytes) { b += align_up(bytes, A); };
-  add(y.bf_layer * 2);
-  add(y.bf_layer * 2);
+  add(slot_elems(y, plan) * 2);
+  add(slot_elems(y, plan) * 2);
   const size_t lay_f = y.layer_end(0) - y.layer_begin(0);
-  add(lay_f * 4);
-  add(lay_f * 4);
-  add((align_up(d, 128) + V * d) * 2);                     // head weights (or the tied table)
-  add(y.head_block * 4);                                    // head grads
+  add(gslot_elems(y, plan) * 4);
+  add(gslot_elems(y, plan) * 4);
+  add(head_w_elems(y, plan) * 2);                           // head weights (or the tied table)
+  add(head_g_elems(y, plan) * 4);                           // head grads
+  if (plan) {                                               // embedding table and its dense gradient
+    add((size_t)plan->world * embed_rows_chunk(*plan, s.V) * d * 2);
+    add((size_t)plan->world * embed_rows_chunk(*plan, s.V) * d * 4);
+  }
   if (g16) {                                                // bf16 offload copies
     add(lay_f * 2);
     add(lay_f * 2);
@@ -1110,8 +1301,8 @@ size_t device_bytes(const Layout& y, int Tc, bool g16, bool offload) {
   add((size_t)(offload ? std::min(s.L + 1, 3) : s.L + 1) * T * d * 4);  // boundary activations
   add(T * d * 2);                                           // u
   add(T * (size_t)s.Nqkv * 2);                              // qkv
-  add(T * (size_t)s.Hd * 2);                                // attention output
-  add((size_t)s.b * s.H * s.s * 4);                         // lse
+  add(n_attn * T * (size_t)s.Hd * 2);                       // attention output
+  add(n_attn * s.b * s.H * (size_t)s.s * 4);                // lse
   add(T * d * 4);                                           // h
   add(T * 4);                                               // r1
   add(T * 4);                                               // r2
@@ -1136,7 +1327,7 @@ size_t device_bytes(const Layout& y, int Tc, bool g16, bool offload) {
   add((size_t)Tc * V * 4);                                  // logits
   add((size_t)Tc * V * 2);                                  // dz
   add(T * 4);                                               // row loss
-  add((4 * T + 1) * 4);                                     // tokens, labels, offs, pos
+  add((5 * T + 1) * 4);                                     // tokens, labels, offs, pos, unique ids
   add((size_t)(s.L + 2) * 4);                               // flags
   add(4);                                                   // error word
   add((size_t)s.s * (s.hd / 2) * 4 * 2);                    // cos, sin
@@ -1190,6 +1381,9 @@ void free_all(mt_ctx* c) {
                         c->ev_head_drained, c->ev_emb_ready, c->ev_emb_d2h_start, c->ev_emb_drained,
                         c->ev_step_start, c->ev_fwd_end, c->ev_head_end, c->ev_bwd_end, c->ev_step_end})
     if (e) cudaEventDestroy(e);
+  if (c->ev_embw) cudaEventDestroy(c->ev_embw);
+  if (c->comm_h2d) c->nccl->CommDestroy(c->comm_h2d);
+  if (c->comm_comp) c->nccl->CommDestroy(c->comm_comp);
   // In serialized mode the three handles are one stream: destroy each once.
   if (c->s_comp) cudaStreamDestroy(c->s_comp);
   if (c->s_h2d && c->s_h2d != c->s_comp) cudaStreamDestroy(c->s_h2d);
@@ -1199,7 +1393,7 @@ void free_all(mt_ctx* c) {
   for (void* p : {(void*)c->grad, (void*)c->ring, (void*)c->defer_g, (void*)(c->grad_head_owned ? c->grad_head : nullptr),
                   (void*)c->bf_layers,
                   (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h, (void*)c->stage_i, (void*)c->flags_h,
-                  (void*)c->misc_h, (void*)c->xh})
+                  (void*)c->misc_h, (void*)c->xh, (void*)c->emb_own_h})
     if (p) cudaFreeHost(p);
   free(c->m);
   free(c->v);
@@ -1208,7 +1402,10 @@ void free_all(mt_ctx* c) {
   delete c;
 }
 
-int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx** out) {
+// world == 0: an unsharded context; else rank `rank` of a sharded one whose
+// NCCL unique id is `id`.
+int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx** out, int world = 0, int rank = 0,
+                const void* id = nullptr) {
   mt_ctx* c = nullptr;
   std::string why;
   int r = validate_config(cfg, &why);
@@ -1217,6 +1414,18 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   *out = nullptr;
   Layout y = make_layout(*cfg);
   const Shapes& s = y.sh;
+  mt_shard plan{};
+  const NcclApi* nccl = nullptr;
+  if (world > 0) {
+    if (!id) return set_err(nullptr, MT_ERR_ARG, "sharded context without an NCCL id");
+    if (cfg->flags & (MT_FLAG_DEFER_UPDATES | MT_FLAG_TIED_EMBED | MT_FLAG_BF16_GRADS))
+      return set_err(nullptr, MT_ERR_CONFIG,
+                     "sharded streaming runs without MT_FLAG_DEFER_UPDATES, MT_FLAG_TIED_EMBED and MT_FLAG_BF16_GRADS");
+    r = mt_shard_plan(cfg, world, rank, &plan);
+    if (r != MT_OK) return set_err(nullptr, r, "no shard plan for this config (d must be a multiple of 128)");
+    nccl = nccl_api(&why);
+    if (!nccl) return set_err(nullptr, MT_ERR_CUDA, why);
+  }
   if (arena) {
     if (arena_bytes < y.total * 4) return set_err(nullptr, MT_ERR_ARENA, "arena smaller than mt_arena_bytes(cfg)");
     if (reinterpret_cast<uintptr_t>(arena) & 255) return set_err(nullptr, MT_ERR_ARENA, "arena not 256-byte aligned");
@@ -1231,8 +1440,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   if (major != 10 || minor != 0) return set_err(nullptr, MT_ERR_CUDA, "this library runs on sm_100 (B200) only");
 
   const int Tc = logits_chunk(s);
-  const size_t need =
-      device_bytes(y, Tc, (cfg->flags & MT_FLAG_BF16_GRADS) != 0, (cfg->flags & MT_FLAG_OFFLOAD_ACTS) != 0);
+  const size_t need = device_bytes(y, Tc, cfg->flags, world > 0 ? &plan : nullptr);
   size_t free_b = 0, total_b = 0;
   if (cudaMemGetInfo(&free_b, &total_b) != cudaSuccess) return set_err(nullptr, MT_ERR_CUDA, "cudaMemGetInfo failed");
   if (need + ((size_t)256 << 20) > free_b) {
@@ -1244,6 +1452,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c = new mt_ctx();
   c->cfg = *cfg;
   c->lay = y;
+  c->plan = plan;
+  c->nccl = nccl;
   c->device = cfg->device;
   c->Tc = Tc;
   c->gsz = (cfg->flags & MT_FLAG_BF16_GRADS) ? 2 : 4;
@@ -1306,7 +1516,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
       cudaHostAlloc(reinterpret_cast<void**>(&c->bf_head), head_bf * 2, cudaHostAllocPortable) != cudaSuccess ||
       cudaHostAlloc(reinterpret_cast<void**>(&c->emb_rows_h), (size_t)s.T * s.d * 4, cudaHostAllocPortable) !=
           cudaSuccess ||
-      cudaHostAlloc(reinterpret_cast<void**>(&c->stage_i), (size_t)(4 * s.T + 1) * 4, cudaHostAllocPortable) !=
+      cudaHostAlloc(reinterpret_cast<void**>(&c->stage_i), (size_t)(5 * s.T + 1) * 4, cudaHostAllocPortable) !=
           cudaSuccess ||
       cudaHostAlloc(reinterpret_cast<void**>(&c->flags_h), (size_t)(s.L + 2) * 4, cudaHostAllocPortable) !=
           cudaSuccess ||
@@ -1314,6 +1524,10 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     return fail(MT_ERR_PIN, "pinned host allocation failed");
   if (cudaHostGetDevicePointer(reinterpret_cast<void**>(&c->bf_embed_dev), c->bf_embed, 0) != cudaSuccess)
     return fail(MT_ERR_PIN, "embedding table not mapped for device access");
+  if (world > 0 &&
+      cudaHostAlloc(reinterpret_cast<void**>(&c->emb_own_h),
+                    std::max<size_t>(1, embed_rows_chunk(plan, s.V)) * s.d * 4, cudaHostAllocPortable) != cudaSuccess)
+    return fail(MT_ERR_PIN, "pinned embedding-row allocation failed");
   if ((cfg->flags & MT_FLAG_OFFLOAD_ACTS) && s.L >= 3 &&
       cudaHostAlloc(reinterpret_cast<void**>(&c->xh), (size_t)(s.L - 2) * s.T * s.d * 4, cudaHostAllocPortable) !=
           cudaSuccess)
@@ -1333,11 +1547,27 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     fill(y.final_norm, seed ^ 0x1001, true);
     if (!y.tied) fill(y.head, seed ^ 0x1002, false);
   }
-  parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) {
-    memset(c->m + b, 0, (e - b) * 4);
-    memset(c->v + b, 0, (e - b) * 4);
-    if (c->grad) memset(c->grad + b * gsz, 0, (e - b) * gsz);
-  });
+  if (world > 0) {
+    // Sharded: the moments are read and written on the rank's own ranges
+    // only, so only those pages are touched (the rest stay unbacked).
+    std::vector<std::pair<size_t, size_t>> own;
+    for (int l = 0; l < s.L; ++l) own.push_back({y.layer_begin(l) + plan.layer_begin, y.layer_begin(l) + plan.layer_end});
+    own.push_back({y.final_norm.off + plan.head_begin, y.final_norm.off + plan.head_end});
+    own.push_back({y.embed.off + (size_t)plan.embed_row_begin * s.d, y.embed.off + (size_t)plan.embed_row_end * s.d});
+    for (const auto& r : own)
+      parallel_ranges(*c->pool, r.second - r.first, [&](size_t b, size_t e) {
+        memset(c->m + r.first + b, 0, (e - b) * 4);
+        memset(c->v + r.first + b, 0, (e - b) * 4);
+      });
+    if (c->grad)
+      parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) { memset(c->grad + b * gsz, 0, (e - b) * gsz); });
+  } else {
+    parallel_ranges(*c->pool, y.total, [&](size_t b, size_t e) {
+      memset(c->m + b, 0, (e - b) * 4);
+      memset(c->v + b, 0, (e - b) * 4);
+      if (c->grad) memset(c->grad + b * gsz, 0, (e - b) * gsz);
+    });
+  }
   if (c->ring) {
     const size_t nr = (size_t)MT_GRAD_RING_SLOTS * c->layer_f;
     parallel_ranges(*c->pool, nr, [&](size_t b, size_t e) { memset(c->ring + b * gsz, 0, (e - b) * gsz); });
@@ -1375,13 +1605,19 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
     return r;
   };
   const size_t T = s.T, d = s.d, F = s.F, V = s.V;
-  c->wslot[0] = (uint16_t*)carve(y.bf_layer * 2);
-  c->wslot[1] = (uint16_t*)carve(y.bf_layer * 2);
+  const mt_shard* pp = world > 0 ? &plan : nullptr;
+  c->wslot[0] = (uint16_t*)carve(slot_elems(y, pp) * 2);
+  c->wslot[1] = (uint16_t*)carve(slot_elems(y, pp) * 2);
   const size_t lay_f = y.layer_end(0) - y.layer_begin(0);
-  c->gslot[0] = (float*)carve(lay_f * 4);
-  c->gslot[1] = (float*)carve(lay_f * 4);
-  c->d_head_w = (uint16_t*)carve((align_up(d, 128) + V * d) * 2);
-  c->d_head_g = (float*)carve(y.head_block * 4);
+  c->gslot[0] = (float*)carve(gslot_elems(y, pp) * 4);
+  c->gslot[1] = (float*)carve(gslot_elems(y, pp) * 4);
+  c->d_head_w = (uint16_t*)carve(head_w_elems(y, pp) * 2);
+  c->d_head_g = (float*)carve(head_g_elems(y, pp) * 4);
+  if (pp) {
+    const size_t rows = embed_rows_chunk(plan, s.V);
+    c->d_embed_w = (uint16_t*)carve((size_t)world * rows * d * 2);
+    c->d_embed_g = (float*)carve((size_t)world * rows * d * 4);
+  }
   if (gsz == 2) {
     c->gslot16[0] = (uint16_t*)carve(lay_f * 2);
     c->gslot16[1] = (uint16_t*)carve(lay_f * 2);
@@ -1390,8 +1626,9 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->xb = (float*)carve((size_t)((cfg->flags & MT_FLAG_OFFLOAD_ACTS) ? std::min(s.L + 1, 3) : s.L + 1) * T * d * 4);
   c->u_b = (uint16_t*)carve(T * d * 2);
   c->qkv_b = (uint16_t*)carve(T * (size_t)s.Nqkv * 2);
-  c->ao_b = (uint16_t*)carve(T * (size_t)s.Hd * 2);
-  c->lse = (float*)carve((size_t)s.b * s.H * s.s * 4);
+  const size_t n_attn = (cfg->flags & MT_FLAG_STASH_ATTN) ? (size_t)s.L : 1;
+  c->ao_b = (uint16_t*)carve(n_attn * T * (size_t)s.Hd * 2);
+  c->lse = (float*)carve(n_attn * s.b * s.H * (size_t)s.s * 4);
   c->h_f = (float*)carve(T * d * 4);
   c->r1 = (float*)carve(T * 4);
   c->r2 = (float*)carve(T * 4);
@@ -1416,7 +1653,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->logits = (float*)carve((size_t)Tc * V * 4);
   c->dz_b = (uint16_t*)carve((size_t)Tc * V * 2);
   c->rowloss = (float*)carve(T * 4);
-  c->d_tok = (int32_t*)carve((4 * T + 1) * 4);
+  c->d_tok = (int32_t*)carve((5 * T + 1) * 4);
+  c->d_uid = c->d_tok + 4 * T + 1;
   c->d_lab = c->d_tok + T;
   c->d_offs = c->d_tok + 2 * T;
   c->d_pos = c->d_tok + 3 * T + 1;
@@ -1473,6 +1711,25 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
                          &c->ev_step_start, &c->ev_fwd_end, &c->ev_head_end, &c->ev_bwd_end, &c->ev_step_end})
     ok = ok && cudaEventCreate(e) == cudaSuccess;
   if (!ok) return fail(MT_ERR_CUDA, "event creation failed");
+  if (world > 0) {
+    // Every rank joins here (NCCL's initialisation is collective); then the
+    // table the first step gathers from: the same bf16 copy on every rank.
+    if (cudaEventCreate(&c->ev_embw) != cudaSuccess) return fail(MT_ERR_CUDA, "event creation failed");
+    ncclUniqueId uid;
+    memcpy(&uid, id, sizeof(uid));
+    ncclResult_t e = nccl->CommInitRank(&c->comm_comp, world, uid, rank);
+    if (e != ncclSuccess) {
+      c->comm_comp = nullptr;
+      return fail(MT_ERR_CUDA, std::string("ncclCommInitRank: ") + nccl->GetErrorString(e));
+    }
+    e = nccl->CommSplit(c->comm_comp, 0, rank, &c->comm_h2d, nullptr);
+    if (e != ncclSuccess) {
+      c->comm_h2d = nullptr;
+      return fail(MT_ERR_CUDA, std::string("ncclCommSplit: ") + nccl->GetErrorString(e));
+    }
+    if (cudaMemcpy(c->d_embed_w, c->bf_embed, (size_t)s.V * s.d * 2, cudaMemcpyHostToDevice) != cudaSuccess)
+      return fail(MT_ERR_CUDA, "embedding table copy failed");
+  }
   if (const char* w = getenv("MT_WAIT_LIMIT_S")) {
     const double lim = atof(w);
     if (lim > 0) c->wait_limit_s = lim;
@@ -1491,6 +1748,34 @@ using namespace mteng;
 extern "C" int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, mt_ctx** out) {
   g_create_error.clear();
   return create_impl(cfg, host_param_arena, arena_bytes, out);
+}
+
+extern "C" int mt_shard_id(void* id_out) {
+  g_create_error.clear();
+  if (!id_out) return set_err(nullptr, MT_ERR_ARG, "id_out is NULL");
+  static_assert(sizeof(ncclUniqueId) == MT_SHARD_ID_BYTES, "NCCL unique id size");
+  std::string why;
+  const NcclApi* nccl = nccl_api(&why);
+  if (!nccl) return set_err(nullptr, MT_ERR_CUDA, why);
+  ncclUniqueId uid;
+  const ncclResult_t e = nccl->GetUniqueId(&uid);
+  if (e != ncclSuccess) return set_err(nullptr, MT_ERR_CUDA, std::string("ncclGetUniqueId: ") + nccl->GetErrorString(e));
+  memcpy(id_out, &uid, sizeof(uid));
+  return MT_OK;
+}
+
+extern "C" int mt_create_sharded(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, int world,
+                                 int rank, const void* id, mt_ctx** out) {
+  g_create_error.clear();
+  if (world < 1 || rank < 0 || rank >= world) return set_err(nullptr, MT_ERR_ARG, "rank outside [0, world)");
+  return create_impl(cfg, host_param_arena, arena_bytes, out, world, rank, id);
+}
+
+extern "C" size_t mt_device_bytes_sharded(const mt_config* cfg, int world) {
+  mt_shard p{};
+  if (mt_shard_plan(cfg, world, 0, &p) != MT_OK) return 0;
+  const Layout y = make_layout(*cfg);
+  return device_bytes(y, logits_chunk(y.sh), cfg->flags, &p);
 }
 
 extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* labels, float* loss_out) {
@@ -1523,6 +1808,8 @@ extern "C" int mt_train_step(mt_ctx* c, const int32_t* tokens, const int32_t* la
   const int n_unique = (int)c->uniq.size();
   offs[n_unique] = acc;
   for (int t = 0; t < T; ++t) pos[start[tokens[t]]++] = t;  // increasing t within each token
+  int32_t* uid = st + 4 * T + 1;  // the unique ids, for the sharded dense embedding gradient
+  for (int u = 0; u < n_unique; ++u) uid[u] = c->uniq[u];
 
   c->call_t0 = now_s();
   c->adamw_first = c->adamw_last = 0;
@@ -1582,6 +1869,7 @@ extern "C" int mt_layer_fwd_bwd(mt_ctx* c, int l, const float* x_in, const float
   const Shapes& s = y.sh;
   if (l < 0 || l >= s.L) return set_err(c, MT_ERR_ARG, "layer outside [0, L)");
   if (grads_bytes < c->layer_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than one layer's block");
+  if (sharded(c)) return set_err(c, MT_ERR_CONFIG, "single-layer calls are not available on a sharded context");
   flush_deferred(c);
   CK(cudaSetDevice(c->device));
   const size_t n = (size_t)s.T * s.d;
@@ -1615,6 +1903,7 @@ extern "C" int mt_head_fwd_bwd(mt_ctx* c, const float* x_L, const int32_t* label
   const Shapes& s = y.sh;
   const size_t head_f = y.head_block;
   if (grads_bytes < head_f * 4) return set_err(c, MT_ERR_ARG, "grads smaller than the final-norm + head block");
+  if (sharded(c)) return set_err(c, MT_ERR_CONFIG, "single-layer calls are not available on a sharded context");
   for (int t = 0; t < s.T; ++t)
     if (labels[t] < 0 || labels[t] >= s.V) return set_err(c, MT_ERR_ARG, "label outside [0, V)");
   flush_deferred(c);
@@ -1769,8 +2058,7 @@ extern "C" int mt_get_stream(mt_ctx* c, void** stream) {
 extern "C" size_t mt_device_bytes(const mt_config* cfg) {
   if (validate_config(cfg, nullptr) != MT_OK) return 0;
   const Layout y = make_layout(*cfg);
-  return device_bytes(y, logits_chunk(y.sh), (cfg->flags & MT_FLAG_BF16_GRADS) != 0,
-                      (cfg->flags & MT_FLAG_OFFLOAD_ACTS) != 0);
+  return device_bytes(y, logits_chunk(y.sh), cfg->flags);
 }
 
 namespace {

@@ -8,6 +8,8 @@
 
 #include <immintrin.h>
 #include <math.h>
+#include <pthread.h>
+#include <sched.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -74,10 +76,9 @@ __attribute__((target("avx512f,avx512bw"))) inline __m256i bf16x16_rne(__m512 x)
 // the batch touches): the moments only decay and no gradient is read; the
 // result is bit-identical to reading zeros (b m + 0 rounds like b m).
 // G = uint16_t reads a bf16 gradient (exactly widened to fp32).
-// NT_PMV streams p, m and v out with non-temporal stores as well (their lines
-// were just read, so the stores replace whole lines; this skips keeping them
-// in cache for a reuse that never comes within the step).
-template <bool HAS_G, typename G = float, bool NT_PMV = false>
+// p, m and v keep ordinary stores: their lines were just read, and streaming
+// them out with non-temporal stores measured slower on the B200 hosts' DRAM.
+template <bool HAS_G, typename G = float>
 __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const G* g, float* m, float* v,
                                                               uint16_t* pb, size_t n, float decay, float b1, float b2,
                                                               float step, float inv_sqrt_bc2, float eps) {
@@ -105,21 +106,15 @@ __attribute__((target("avx512f,avx512bw"))) void adamw_avx512(float* p, const G*
     const __m512 den = _mm512_fmadd_ps(_mm512_sqrt_ps(vi), vibc2, veps);
     const __m512 pi = _mm512_sub_ps(_mm512_mul_ps(_mm512_loadu_ps(p + i), vdec),
                                     _mm512_div_ps(_mm512_mul_ps(vstep, mi), den));
-    if (NT_PMV) {
-      _mm512_stream_ps(m + i, mi);
-      _mm512_stream_ps(v + i, vi);
-      _mm512_stream_ps(p + i, pi);
-    } else {
-      _mm512_storeu_ps(m + i, mi);
-      _mm512_storeu_ps(v + i, vi);
-      _mm512_storeu_ps(p + i, pi);
-    }
+    _mm512_storeu_ps(m + i, mi);
+    _mm512_storeu_ps(v + i, vi);
+    _mm512_storeu_ps(p + i, pi);
     if (nt)
       _mm256_stream_si256(reinterpret_cast<__m256i*>(pb + i), bf16x16_rne(pi));
     else if (pb)
       _mm256_storeu_si256(reinterpret_cast<__m256i*>(pb + i), bf16x16_rne(pi));
   }
-  if (nt || NT_PMV) _mm_sfence();
+  if (nt) _mm_sfence();
   if (i < n)
     adamw_scalar<G>(p + i, HAS_G ? g + i : nullptr, m + i, v + i, pb ? pb + i : nullptr, n - i, decay, b1, b2, step,
                     inv_sqrt_bc2, eps);
@@ -144,34 +139,14 @@ bool adamw_uses_avx512() {
   return yes;
 }
 
-// MT_ADAMW_NT=1: non-temporal stores of p, m and v too (64-byte aligned chunks
-// only). Read once per process.
-bool adamw_nt_pmv() {
-  static const bool yes = [] {
-    const char* e = getenv("MT_ADAMW_NT");
-    return e && e[0] == '1';
-  }();
-  return yes;
-}
-
-inline bool al64(const void* a, const void* b, const void* c) {
-  return ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b) | reinterpret_cast<uintptr_t>(c)) & 63) == 0;
-}
-
 void adamw_chunk(float* p, const float* g, float* m, float* v, uint16_t* pb, size_t n, const AdamHyper& h, int t) {
   const double bc1 = 1.0 - pow((double)h.beta1, t);
   const double bc2 = 1.0 - pow((double)h.beta2, t);
   const float decay = 1.f - h.lr * h.wd;
   const float step = (float)(h.lr / bc1);
   const float inv_sqrt_bc2 = (float)(1.0 / sqrt(bc2));
-  const bool ntp = adamw_nt_pmv() && al64(p, m, v);
-  if (adamw_uses_avx512() && g && ntp)
-    adamw_avx512<true, float, true>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
-  else if (adamw_uses_avx512() && g)
+  if (adamw_uses_avx512() && g)
     adamw_avx512<true>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
-  else if (adamw_uses_avx512() && ntp)
-    adamw_avx512<false, float, true>(p, (const float*)nullptr, m, v, pb, n, decay, h.beta1, h.beta2, step,
-                                     inv_sqrt_bc2, h.eps);
   else if (adamw_uses_avx512())
     adamw_avx512<false>(p, (const float*)nullptr, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
   else
@@ -186,9 +161,7 @@ void adamw_chunk_bf16g(float* p, const uint16_t* g, float* m, float* v, uint16_t
   const float decay = 1.f - h.lr * h.wd;
   const float step = (float)(h.lr / bc1);
   const float inv_sqrt_bc2 = (float)(1.0 / sqrt(bc2));
-  if (adamw_uses_avx512() && adamw_nt_pmv() && al64(p, m, v))
-    adamw_avx512<true, uint16_t, true>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
-  else if (adamw_uses_avx512())
+  if (adamw_uses_avx512())
     adamw_avx512<true, uint16_t>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
   else
     adamw_scalar<uint16_t>(p, g, m, v, pb, n, decay, h.beta1, h.beta2, step, inv_sqrt_bc2, h.eps);
@@ -203,8 +176,35 @@ void bf16_round_chunk(const float* x, uint16_t* out, size_t n) {
 }
 
 // ---------------------------------------------------------------------------
+// MT_PIN_THREADS=1: worker i runs on the (i+1)-th CPU the process may use
+// (the first is left to the calling thread), so that a worker keeps its core
+// and the pages it first touched stay near it. Read once per process.
+static bool pin_threads() {
+  static const bool yes = [] {
+    const char* e = getenv("MT_PIN_THREADS");
+    return e && e[0] == '1';
+  }();
+  return yes;
+}
+
 ThreadPool::ThreadPool(int workers) {
-  for (int i = 0; i < workers; ++i) workers_.emplace_back([this] { loop(); });
+  std::vector<int> cpus;
+  if (pin_threads()) {
+    cpu_set_t set;
+    CPU_ZERO(&set);
+    if (sched_getaffinity(0, sizeof(set), &set) == 0)
+      for (int c = 0; c < CPU_SETSIZE; ++c)
+        if (CPU_ISSET(c, &set)) cpus.push_back(c);
+  }
+  for (int i = 0; i < workers; ++i) {
+    workers_.emplace_back([this] { loop(); });
+    if (cpus.size() > 1) {
+      cpu_set_t one;
+      CPU_ZERO(&one);
+      CPU_SET(cpus[(size_t)(i + 1) % cpus.size()], &one);
+      pthread_setaffinity_np(workers_.back().native_handle(), sizeof(one), &one);
+    }
+  }
 }
 
 ThreadPool::~ThreadPool() {

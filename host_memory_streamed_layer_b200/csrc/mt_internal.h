@@ -48,6 +48,9 @@ struct GemmDesc {
 int gemm_bf16(const GemmDesc& g, cudaStream_t st, int* dev_err);
 // Kernel family for later GEMMs: 0 automatic, 1 single-CTA, 2 CTA pairs; returns the previous one.
 int gemm_variant(int v);
+// Forward attention kernel for head dim 128 in later calls (0 automatic, 1 one
+// query tile per CTA, 2 two tiles in ping-pong); returns the previous choice.
+int attention_fwd_variant(int v);
 // Main-loop wait limit (ns) of later single-CTA GEMM launches; returns the previous one.
 uint64_t gemm_wait_limit_ns(uint64_t ns);
 

@@ -1,7 +1,7 @@
 """Micro-benchmark of single hot-path kernels through the C ABI.
 
     python -m host_memory_streamed_layer_b200.kernel_bench gemm [--shape NAME] [--iters N]
-    python -m host_memory_streamed_layer_b200.kernel_bench attn [--fwd-only] [--iters N]
+    python -m host_memory_streamed_layer_b200.kernel_bench attn [--fwd-only] [--iters N] [--attn-shape B,S,H]
     python -m host_memory_streamed_layer_b200.kernel_bench rmsnorm_bwd [--iters N]
     python -m host_memory_streamed_layer_b200.kernel_bench elementwise [--iters N]
 
@@ -12,7 +12,9 @@ which is what an ncu capture of one launch wants. Shapes are those of the
 llama-1.3b workload (T = 8 x 2048 tokens, d 2048, FFN 5504, 16 heads); for
 the GEMMs, --workload NAME takes every GEMM shape of that workload's training
 step instead, and each result line carries the shape's launches per step
-(so per-shape ncu figures can be weighted into a per-launch step average).
+(so per-shape ncu figures can be weighted into a per-launch step average);
+for attention, --attn-shape B,S,H sets sequences, length and heads (head dim
+128, as many KV heads as query heads).
 """
 from __future__ import annotations
 
@@ -109,8 +111,9 @@ def bench_gemm(names, iters, warmup, table=None):
     return out
 
 
-def bench_attn(iters, warmup, fwd_only, impl="tc"):
+def bench_attn(iters, warmup, fwd_only, impl="tc", B=B, S=S, H=H):
     st = torch.cuda.current_stream().cuda_stream
+    T = B * S
     ld = 3 * H * HD
     qkv = torch.randn(T, ld, device="cuda").to(torch.bfloat16)
     o = torch.empty(T, H * HD, device="cuda", dtype=torch.bfloat16)
@@ -209,6 +212,9 @@ def main():
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--impl", default="tc", choices=["tc", "mma"])
     ap.add_argument("--workload", default=None, help="GEMMs: every shape of this workload's training step")
+    ap.add_argument("--attn-shape", default=f"{B},{S},{H}", help="attention: sequences,length,heads")
+    ap.add_argument("--attn-variant", default="auto", choices=["auto", "one", "pingpong"],
+                    help="attention forward kernel (head dim 128): automatic, one or two query tiles per CTA")
     a = ap.parse_args()
     if a.kernel == "gemm":
         table = None
@@ -218,7 +224,12 @@ def main():
         names = list(table or GEMMS) if a.shape == "all" else a.shape.split(",")
         res = bench_gemm(names, a.iters, a.warmup, table)
     elif a.kernel == "attn":
-        res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl)
+        ab, as_, ah = (int(x) for x in a.attn_shape.split(","))
+        mt.mt_k_attn_fwd_variant({"auto": mt.ATTN_AUTO, "one": mt.ATTN_ONE_TILE,
+                                  "pingpong": mt.ATTN_PINGPONG}[a.attn_variant])
+        res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl, ab, as_, ah)
+        for r in res:
+            r["shape"] = dict(b=ab, s=as_, heads=ah, hd=HD)
     elif a.kernel == "elementwise":
         res = bench_elementwise(a.iters, a.warmup)
     else:

@@ -53,6 +53,7 @@ def mt_k_gemm_bf16(A, lda, a_mn, B, ldb, b_mn, C, ldc, out_kind, R, ldr, M, N, K
 
 
 _sig("mt_k_gemm_variant", c_int, c_int)
+_sig("mt_k_attn_fwd_variant", c_int, c_int)
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
 
 
@@ -61,6 +62,18 @@ def mt_k_gemm_variant(variant: int) -> int:
     rc = lib.mt_k_gemm_variant(variant)
     if rc < 0:
         raise MTError(rc, "mt_k_gemm_variant")
+    return rc
+
+
+ATTN_AUTO, ATTN_ONE_TILE, ATTN_PINGPONG = 0, 1, 2
+
+
+def mt_k_attn_fwd_variant(variant: int) -> int:
+    """Selects the head-dim-128 attention forward kernel for later calls;
+    returns the previous choice."""
+    rc = lib.mt_k_attn_fwd_variant(variant)
+    if rc < 0:
+        raise MTError(rc, "mt_k_attn_fwd_variant")
     return rc
 
 
@@ -187,6 +200,7 @@ MT_FLAG_DEFER_UPDATES = 0x10
 MT_FLAG_BF16_GRADS = 0x20
 MT_FLAG_OFFLOAD_ACTS = 0x40
 MT_FLAG_TIED_EMBED = 0x80
+MT_FLAG_STASH_ATTN = 0x100
 MT_GRAD_RING_SLOTS = 3
 MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
 MT_T_EMBED, MT_T_FINAL_NORM, MT_T_LM_HEAD = 100, 101, 102
@@ -361,6 +375,38 @@ def mt_shard_plan(cfg: mt_config, world: int, rank: int) -> dict:
 
 def mt_device_bytes(cfg: mt_config) -> int:
     return lib.mt_device_bytes(ctypes.byref(cfg))
+
+
+MT_SHARD_ID_BYTES = 128
+_sig("mt_shard_id", c_int, c_void_p)
+_sig("mt_create_sharded", c_int, _cfgp, c_void_p, c_size_t, c_int, c_int, c_void_p, ctypes.POINTER(c_void_p))
+_sig("mt_device_bytes_sharded", c_size_t, _cfgp, c_int)
+
+
+def mt_shard_id() -> bytes:
+    """A fresh NCCL unique id for mt_create_sharded (one rank makes it; every
+    rank passes the same bytes)."""
+    buf = ctypes.create_string_buffer(MT_SHARD_ID_BYTES)
+    rc = lib.mt_shard_id(buf)
+    if rc != MT_OK:
+        raise MTError(rc, "mt_shard_id " + lib.mt_last_error(None).decode())
+    return buf.raw
+
+
+def mt_create_sharded(cfg: mt_config, arena_ptr: int, arena_bytes: int, world: int, rank: int, nccl_id: bytes) -> int:
+    """Context of rank `rank` of a sharded run; returns once every rank joined."""
+    if len(nccl_id) != MT_SHARD_ID_BYTES:
+        raise ValueError("nccl_id must be MT_SHARD_ID_BYTES bytes")
+    ctx = c_void_p()
+    buf = ctypes.create_string_buffer(bytes(nccl_id), MT_SHARD_ID_BYTES)
+    rc = lib.mt_create_sharded(ctypes.byref(cfg), arena_ptr or None, arena_bytes, world, rank, buf, ctypes.byref(ctx))
+    if rc != MT_OK:
+        raise MTError(rc, "mt_create_sharded " + lib.mt_last_error(None).decode())
+    return ctx.value
+
+
+def mt_device_bytes_sharded(cfg: mt_config, world: int) -> int:
+    return lib.mt_device_bytes_sharded(ctypes.byref(cfg), world)
 
 
 def mt_inject_host_stall(ctx: int, stream: int, ms: int):

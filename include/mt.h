@@ -123,6 +123,18 @@ extern "C" {
  * gradient of the step has been checked. Not with MT_FLAG_BF16_GRADS, and not
  * partitioned by mt_shard_plan (MT_ERR_CONFIG). */
 #define MT_FLAG_TIED_EMBED 0x80u
+/* Keep each layer's attention output O (bf16 [b*s, H*hd]) and log-sum-exp
+ * (fp32 [b, H, s]) on the device from the forward sweep to the layer's
+ * backward, so that the layer's recompute skips the attention forward. The
+ * pages' checkpointing keeps some intermediates and recomputes the rest
+ * (intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
+ * Optimizer Steps"); which ones is a memory-for-time choice, and at long
+ * context, where attention dominates the layer, this one saves one of the
+ * layer's two attention forwards (about a fifth of its attention work, the
+ * backward counting 2.5 forwards). Costs (L-1) (b s H hd 2 + b H s 4) bytes of HBM
+ * (mt_device_bytes). The results are unchanged: the attention forward is
+ * deterministic, so the kept O and LSE are those a recompute would give. */
+#define MT_FLAG_STASH_ATTN 0x100u
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0
@@ -220,7 +232,9 @@ size_t mt_host_state_bytes(const mt_config* cfg);
  * weights and gradients, the boundary activations x_0..x_L (fp32 [b*s, d]
  * each, the only per-layer state kept: intelligentliving.co, "Checkpointing,
  * Manual Gradients, and CPU-Side Optimizer Steps") and one layer's workspace.
- * Only the boundary activations grow with L. No GPU needed. */
+ * Only the boundary activations grow with L (three slots with
+ * MT_FLAG_OFFLOAD_ACTS), and with MT_FLAG_STASH_ATTN each layer's attention
+ * output and log-sum-exp. No GPU needed. */
 size_t mt_device_bytes(const mt_config* cfg);
 
 /* Partition of the training state over `world` GPUs of one host that each
@@ -263,6 +277,49 @@ int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard* out);
  * all device memory. Fails with MT_ERR_NOMEM before allocating if the device
  * budget does not fit. */
 int mt_create(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, mt_ctx** out);
+
+/* Bytes of the NCCL unique id that mt_create_sharded takes. */
+#define MT_SHARD_ID_BYTES 128
+/* Writes a fresh NCCL unique id (MT_SHARD_ID_BYTES bytes) to id_out. One rank
+ * calls it and hands the same bytes to every rank (a torch.distributed
+ * broadcast, for instance). NCCL is loaded at run time (libnccl.so.2, 2.18 or
+ * later); MT_ERR_CUDA if it cannot be loaded or fails, MT_ERR_ARG for NULL. */
+int mt_shard_id(void* id_out);
+
+/* mt_create for rank `rank` of `world` GPUs of one host that train
+ * data-parallel with sharded streaming (mt_shard_plan; intelligentliving.co,
+ * "Balancing Reduced Collective Communication with Weight Streaming
+ * Latency", names the all-gather and reduce-scatter used here). Every rank
+ * calls it with the same cfg, the same initial arena contents (or NULL and the
+ * same cfg->seed) and the id of mt_shard_id; the call returns once all ranks
+ * have joined (NCCL's initialisation is collective). Per step, each rank
+ *   - copies its own part of every bf16 layer block, of the [final gain | LM
+ *     head] block and its own embedding rows over its host link, and
+ *     all-gathers the rest from the peers over NVLink into its device slots;
+ *   - runs forward and backward on its own tokens (mt_train_step's tokens
+ *     and labels are the rank's micro-batch);
+ *   - averages every gradient block over the ranks with a reduce-scatter
+ *     that leaves it its own part (the embedding gradient as a dense
+ *     [V, d] block split by rows), checks that part for NaN/Inf with the
+ *     verdict shared by all ranks, offloads only that part and runs the host
+ *     AdamW on the matching elements of its arena.
+ * So per rank the host link carries 1/world of the weights and gradients and
+ * the host optimizer 1/world of the update. The returned loss is the mean over
+ * all ranks' tokens. The arena, the moments, mt_get_params / mt_get_grads /
+ * mt_get_opt_state hold current values on the rank's own ranges only.
+ * Collectives of the H2D stream and of the compute stream use two
+ * communicators, so each runs in one program order on every rank.
+ * Requires d % 128 == 0; MT_ERR_CONFIG with MT_FLAG_DEFER_UPDATES,
+ * MT_FLAG_TIED_EMBED or MT_FLAG_BF16_GRADS, and mt_layer_fwd_bwd /
+ * mt_head_fwd_bwd refuse a sharded context. world = 1 runs the same path
+ * with one rank (the collectives are copies). */
+int mt_create_sharded(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, int world, int rank,
+                      const void* id, mt_ctx** out);
+
+/* mt_device_bytes of a rank of a sharded context: slots padded to world
+ * chunks, plus the device embedding table (bf16) and its dense fp32
+ * gradient, [world * ceil(V / world), d] each. 0 for a bad cfg or world. */
+size_t mt_device_bytes_sharded(const mt_config* cfg, int world);
 
 /* One training step: tokens and labels are host int32 arrays of b*s ids in
  * [0, V), sequence-major. Runs forward, loss, backward and the host AdamW

@@ -192,6 +192,15 @@ int64_t mt_k_gemm_wait_limit_ns(int64_t ns);
  * family, or MT_ERR_ARG for another value (nothing changes). No GPU work. */
 int mt_k_gemm_variant(int variant);
 
+/* Selects the tcgen05 attention forward kernel for head dim 128 in later calls
+ * (mt_k_attn_fwd_tc and the engine): 0 automatic (the default: two query tiles
+ * per CTA from s = 8192 on, one below), 1 one 128-query tile per CTA, 2 two
+ * 128-query tiles per CTA in ping-pong, P kept in tensor memory. Both compute
+ * the same attention; this exists for measurement and tests. Returns the
+ * previous choice, or MT_ERR_ARG for another value (nothing changes). No GPU
+ * work. */
+int mt_k_attn_fwd_variant(int variant);
+
 /* Host AdamW over n fp32 elements, in place (HOST pointers, runs on the
  * calling thread; the engine runs the same routine across its worker pool):
  *   p <- p (1 - lr wd); m <- b1 m + (1-b1) g; v <- b2 v + (1-b2) g^2;

@@ -87,3 +87,18 @@ def test_deferred_layer_count_matches_the_library(monkeypatch, env):
     cfg.flags |= mt.MT_FLAG_DEFER_UPDATES
     layer_bytes = 4 * (mt.mt_tensor_offset(cfg, 1, 0)[0] - mt.mt_tensor_offset(cfg, 0, 0)[0])
     assert mt.mt_host_state_bytes(cfg) - ring == bench.defer_layers(sh) * layer_bytes
+
+
+def test_attention_stash_removes_the_recomputed_attention_forwards():
+    """With MT_FLAG_STASH_ATTN the schedule executes L-1 fewer causal attention
+    forwards (2 b s^2 H hd FLOPs each), all in the backward phase; the model
+    FLOPs do not change."""
+    sh = synth.WORKLOADS["llama-7b-128k"]
+    A = 2.0 * sh["b"] * sh["s"] ** 2 * sh["H"] * (sh["d"] // sh["H"])
+    f0, b0 = bench.phase_flops(sh)
+    f1, b1 = bench.phase_flops(sh, stash=True)
+    assert f1 == f0 and b0 - b1 == pytest.approx((sh["L"] - 1) * A)
+    m0, e0 = bench.flops_per_step(sh)
+    m1, e1 = bench.flops_per_step(sh, stash=True)
+    assert m1 == m0 and e0 - e1 == pytest.approx((sh["L"] - 1) * A)
+    assert e0 == pytest.approx(f0 + b0)

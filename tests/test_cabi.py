@@ -354,6 +354,28 @@ def test_offloaded_activations_keep_three_device_slots():
     assert dev[0] == dev[1] == dev[2]
 
 
+def test_attention_stash_adds_one_output_and_lse_per_layer():
+    """MT_FLAG_STASH_ATTN: the device keeps L attention outputs (bf16 [b*s, H*hd])
+    and log-sum-exp blocks (fp32 [b, H, s]) instead of one of each; host state
+    is unchanged. Sizes are 256-byte aligned like every other buffer."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    base = dict(d=1024, H=8, Hkv=2, F=2752, V=4096, b=3, s=1000)
+    T, Hd = base["b"] * base["s"], 1024
+
+    def al(n):
+        return (n + 255) // 256 * 256
+    for L in (1, 4, 32):
+        for extra in (0, mt.MT_FLAG_OFFLOAD_ACTS):
+            cfg = arena.config(dict(base, L=L))
+            cfg.flags = extra
+            plain_dev, plain_host = mt.mt_device_bytes(cfg), mt.mt_host_state_bytes(cfg)
+            cfg.flags = extra | mt.MT_FLAG_STASH_ATTN
+            grow = al(L * T * Hd * 2) - al(T * Hd * 2) + al(L * base["b"] * base["H"] * base["s"] * 4) \
+                - al(base["b"] * base["H"] * base["s"] * 4)
+            assert mt.mt_device_bytes(cfg) - plain_dev == grow
+            assert mt.mt_host_state_bytes(cfg) == plain_host
+
+
 def test_tied_embeddings_layout():
     """MT_FLAG_TIED_EMBED: the arena loses exactly the LM-head tensor (the
     oracle's tied layout matches the library's offsets), MT_T_LM_HEAD is

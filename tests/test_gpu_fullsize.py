@@ -126,7 +126,7 @@ def test_attention_full_shape_sampled(impl):
     assert np.linalg.norm(gv - rdv[0, -16:, 0]) <= 2e-2 * np.linalg.norm(rdv[0, -16:, 0])
 
 
-@pytest.mark.parametrize("impl", ["mma", "tc"])
+@pytest.mark.parametrize("impl", ["mma", "tc", "tc_pingpong"])
 def test_attention_whole_heads_full_length(impl):
     """Every row of two whole heads at the full 2048-token length, element by
     element (per-row relative L2): o, the log-sum-exp, dq, dk and dv against
@@ -145,16 +145,20 @@ def test_attention_whole_heads_full_length(impl):
     p = qkv.data_ptr()
     pk, pv = p + 2 * H * HD, p + 2 * (H + Hkv) * HD
     err = torch.zeros(1, dtype=torch.int32, device=DEV)
-    fwd = mt.mt_k_attn_fwd_tc if impl == "tc" else mt.mt_k_attn_fwd
-    fwd(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, Hkv, HD, 0,
-        *([err.data_ptr()] if impl == "tc" else []))
+    fwd = mt.mt_k_attn_fwd if impl == "mma" else mt.mt_k_attn_fwd_tc
+    was = mt.mt_k_attn_fwd_variant(mt.ATTN_PINGPONG if impl == "tc_pingpong" else mt.ATTN_ONE_TILE)
+    try:
+        fwd(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, Hkv, HD, 0,
+            *([] if impl == "mma" else [err.data_ptr()]))
+    finally:
+        mt.mt_k_attn_fwd_variant(was)
     do = torch.randn(T, H * HD, device=DEV, generator=g).to(torch.bfloat16)
     dvec = torch.empty(B, H, S, device=DEV)
     dqa = torch.empty(T, H * HD, device=DEV)
     dqkv = torch.empty(T, ld, device=DEV, dtype=torch.bfloat16)
     dp = dqkv.data_ptr()
-    bwd = mt.mt_k_attn_bwd_tc if impl == "tc" else mt.mt_k_attn_bwd
-    kw = {"dev_err": err.data_ptr()} if impl == "tc" else {}
+    bwd = mt.mt_k_attn_bwd if impl == "mma" else mt.mt_k_attn_bwd_tc
+    kw = {} if impl == "mma" else {"dev_err": err.data_ptr()}
     bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(), dvec.data_ptr(), dqa.data_ptr(),
         H * HD, dp, ld, dp + 2 * H * HD, dp + 2 * (H + Hkv) * HD, ld, B, S, H, Hkv, HD, **kw)
     torch.cuda.synchronize()

@@ -179,7 +179,7 @@ def test_softmax_ce(T, V):
 
 
 ATTN = [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 8, 1, 200, 1), (64, 2, 2, 1, 2), (128, 4, 4, 64, 1),
-        (128, 2, 2, 384, 2), (64, 4, 1, 300, 2)]
+        (128, 2, 2, 384, 2), (64, 4, 1, 300, 2), (128, 4, 2, 700, 2)]
 
 
 def _attn_inputs(hd, H, Hkv, s, b, seed):
@@ -194,10 +194,15 @@ def _attn_inputs(hd, H, Hkv, s, b, seed):
     return qkv, q, k, v, ld
 
 
-@pytest.mark.parametrize("impl", ["mma", "tc"])
+@pytest.mark.parametrize("impl", ["mma", "tc", "tc_pingpong"])
 @pytest.mark.parametrize("hd,H,Hkv,s,b", ATTN)
 def test_attention_fwd(hd, H, Hkv, s, b, impl):
+    """tc: the tcgen05 forward with one query tile per CTA; tc_pingpong: two
+    tiles per CTA in ping-pong (head dim 128, selected explicitly: the
+    automatic choice takes it only from 8192 tokens on)."""
     mt = _mt()
+    if impl == "tc_pingpong" and hd != 128:
+        pytest.skip("the two-tile forward is for head dim 128")
     qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, hd + s)
     T = b * s
     o = torch.empty(T, H * hd, dtype=torch.bfloat16, device=DEV)
@@ -208,8 +213,12 @@ def test_attention_fwd(hd, H, Hkv, s, b, impl):
         mt.mt_k_attn_fwd(p, p + 2 * H * hd, p + 2 * (H + Hkv) * hd, ld, o.data_ptr(), H * hd, lse.data_ptr(),
                          b, s, H, Hkv, hd)
     else:
-        mt.mt_k_attn_fwd_tc(p, p + 2 * H * hd, p + 2 * (H + Hkv) * hd, ld, o.data_ptr(), H * hd, lse.data_ptr(),
-                            b, s, H, Hkv, hd, 0, err.data_ptr())
+        was = mt.mt_k_attn_fwd_variant(mt.ATTN_PINGPONG if impl == "tc_pingpong" else mt.ATTN_ONE_TILE)
+        try:
+            mt.mt_k_attn_fwd_tc(p, p + 2 * H * hd, p + 2 * (H + Hkv) * hd, ld, o.data_ptr(), H * hd,
+                                lse.data_ptr(), b, s, H, Hkv, hd, 0, err.data_ptr())
+        finally:
+            mt.mt_k_attn_fwd_variant(was)
     sync()
     assert err.item() == 0
     ro, _ = oracle.attention_fwd(q, k, v)

@@ -215,22 +215,27 @@ def test_checkpoint_resume_continues_the_trajectory():
     assert rel(P2b, P2) <= 1e-5
 
 
+@pytest.mark.parametrize("extra", ["offload", "stash", "offload+stash"])
 @pytest.mark.parametrize("name,shape,flags", [
     ("gqa_ragged", SHAPES["gqa_ragged"], 0),
     ("five_layers", dict(L=5, d=256, H=4, Hkv=2, F=688, V=1024, b=2, s=128), 0),
     ("five_layers_ring_defer", dict(L=5, d=256, H=4, Hkv=2, F=688, V=1024, b=2, s=128), 0x8 | 0x10),
     ("long_context", dict(L=4, d=1024, H=8, Hkv=8, F=2816, V=4096, b=1, s=16384), 0x8),
 ])
-def test_offloaded_activations_give_the_resident_result(name, shape, flags):
+def test_offloaded_activations_give_the_resident_result(name, shape, flags, extra):
     """MT_FLAG_OFFLOAD_ACTS: the boundary activations go to host memory in the
-    forward and return for each layer's recompute; the copies are exact, so
-    two steps match the resident run (loss to 1e-5, every gradient and the
+    forward and return for each layer's recompute; the copies are exact.
+    MT_FLAG_STASH_ATTN: the recompute takes the forward's attention output and
+    log-sum-exp instead of running the attention again; the forward is
+    deterministic, so they are the recompute's. Either way (and both), two
+    steps match the plain run (first loss to 1e-5, every gradient and the
     updated master to the run-to-run noise of the attention's dQ reductions),
     and the first step's loss and gradients match the oracle."""
     from host_memory_streamed_layer_b200 import arena, mt
     c = oracle.OracleConfig(**shape)
     runs = {}
-    for off in (0, mt.MT_FLAG_OFFLOAD_ACTS):
+    var = (mt.MT_FLAG_OFFLOAD_ACTS if "offload" in extra else 0) | (mt.MT_FLAG_STASH_ATTN if "stash" in extra else 0)
+    for off in (0, var):
         cfg = arena.config(shape)
         cfg.flags = flags | off
         cfg.host_threads = 4
@@ -251,16 +256,27 @@ def test_offloaded_activations_give_the_resident_result(name, shape, flags):
         finally:
             mt.mt_destroy(ctx)
         runs[off] = (out, A.copy(), st)
-    res, off = runs[0], runs[mt.MT_FLAG_OFFLOAD_ACTS]
-    for (la, Ga), (lb, Gb) in zip(res[0], off[0]):
-        assert abs(la - lb) <= 1e-5
+    res, off = runs[0], runs[var]
+    for step, ((la, Ga), (lb, Gb)) in enumerate(zip(res[0], off[0])):
+        # the first forward is deterministic; the second runs on weights that
+        # carry the dQ reductions' order noise through one Adam step (at
+        # s = 16384 that moves the loss by a few 1e-6 relative)
+        assert abs(la - lb) <= (1e-5 if step == 0 else 1e-5 * max(1.0, abs(la)))
         if Ga is not None:
             A_, B_ = oracle.unpack_arena(Ga, c), oracle.unpack_arena(Gb, c)
             assert max(rel(B_[k], A_[k]) for k in A_) <= 1e-4
-    assert rel(off[1], res[1]) <= 1e-3
+    # Adam's first steps move each weight by about lr * sign(g): where a
+    # gradient lies within the dQ reductions' noise its sign can differ
+    # between two runs, so the masters differ by up to 2 lr there (1.4e-3
+    # relative seen at s = 16384); the end-to-end bar against the oracle
+    assert rel(off[1], res[1]) <= 5e-3
     # the extra link traffic of the offload is accounted for
     T, d, L = shape["b"] * shape["s"], shape["d"], shape["L"]
-    assert off[2]["h2d_bytes"] - res[2]["h2d_bytes"] == pytest.approx(4.0 * (L - 2) * T * d)
+    moved = 4.0 * (L - 2) * T * d if var & mt.MT_FLAG_OFFLOAD_ACTS else 0.0
+    assert off[2]["h2d_bytes"] - res[2]["h2d_bytes"] == pytest.approx(moved)
+    # the stash skips exactly the L-1 recomputed attention forwards of a step
+    skipped = L - 1 if var & mt.MT_FLAG_STASH_ATTN else 0
+    assert res[2]["kernel_launches"] - off[2]["kernel_launches"] == skipped
     if name == "gqa_ragged":
         r = oracle_steps(shape, 1)[0]
         assert abs(off[0][0][0] - r["loss"]) <= 1e-2
