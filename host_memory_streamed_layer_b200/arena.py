@@ -13,6 +13,8 @@ from . import mt
 
 def config(shape: dict, **hyper) -> "mt.mt_config":
     cfg = mt.mt_config_default(**{k: shape[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s")})
+    if shape.get("E"):
+        cfg.E, cfg.topk = shape["E"], shape.get("topk", 2)
     for k, v in hyper.items():
         setattr(cfg, k, v)
     return cfg

@@ -562,6 +562,18 @@ int attention_fwd(const AttnArgs& a, cudaStream_t st) {
   return MT_ERR_CONFIG;
 }
 
+namespace {
+int g_bwd_variant = 0;
+}
+
+int attention_bwd_variant(int v) {
+  const int was = g_bwd_variant;
+  g_bwd_variant = v;
+  return was;
+}
+
+int attention_bwd_kernels() { return g_bwd_variant == 2 ? 4 : 3; }
+
 int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   if (a.b <= 0 || a.s <= 0) return MT_OK;
   if (a.hd != 128) return MT_ERR_CONFIG;
@@ -569,9 +581,16 @@ int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   const int64_t nw = (int64_t)T * a.H;
   k_attn_bwd_pre<<<(int)((nw + 7) / 8), 256, 0, st>>>((const bf16*)a.o, (const bf16*)a.dout, a.ldo, a.dvec, T, a.s,
                                                       a.H, 128);
-  if (cudaMemsetAsync(a.dq_acc, 0, (size_t)T * a.ldqa * sizeof(float), st) != cudaSuccess) return MT_ERR_CUDA;
-  const int r = attention_bwd_tc_main(a, st, err);
-  if (r != MT_OK) return r;
+  const bool split = g_bwd_variant == 2;
+  if (split) {  // dK, dV without reductions; dQ written once per element by the query-major kernel
+    int r = attention_bwd_tc_main(a, st, err, true);
+    if (r == MT_OK) r = attention_bwd_dq_tc(a, st, err);
+    if (r != MT_OK) return r;
+  } else {
+    if (cudaMemsetAsync(a.dq_acc, 0, (size_t)T * a.ldqa * sizeof(float), st) != cudaSuccess) return MT_ERR_CUDA;
+    const int r = attention_bwd_tc_main(a, st, err, false);
+    if (r != MT_OK) return r;
+  }
   const int64_t nthr = (int64_t)T * a.H * (128 / 8);
   k_dq_cast<<<(int)((nthr + 255) / 256), 256, 0, st>>>(a.dq_acc, a.ldqa, (bf16*)a.dq, a.lddq, T, a.H, 128, a.s,
                                                        a.rope_cos, a.rope_sin);

@@ -810,12 +810,12 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   auto al16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; };
   if (!al16(a.q) || !al16(a.k) || !al16(a.v) || !al16(a.o) || (a.ldqkv % 8) || (a.ldo % 8)) return MT_ERR_ARG;
   if (a.hd == 64) return launch_fa<64>(a, st, err);
-  // head dim 128: two query tiles per CTA from 8192 tokens on (measured on
-  // B200: 939 against 903 TFLOP/s at s = 16384, but 536 against 562 at
-  // s = 2048, where the pairs' short rows leave their prologue and epilogue
-  // exposed)
+  // head dim 128: two query tiles per CTA above 8192 tokens (measured on
+  // B200, TFLOP/s one tile / two: 562 / 536 at s = 2048, 706 / 685 at 4096,
+  // 809 / 807 at 8192, 903 / 939 at 16384, 911 / 972 at 32768; with short rows
+  // the pairs' prologue and epilogue are exposed)
   if (a.hd == 128) {
-    const int v = g_fa_variant ? g_fa_variant : (a.s >= 8192 ? 2 : 1);
+    const int v = g_fa_variant ? g_fa_variant : (a.s > 8192 ? 2 : 1);
     return v == 2 ? launch_fa_pp(a, st, err) : launch_fa<128>(a, st, err);
   }
   return MT_ERR_CONFIG;
@@ -878,6 +878,7 @@ struct FbParams {
   const float* rsin;
   int* err;
   int vec_lse;  // LSE and D rows start 16-byte aligned: s % 4 == 0 and aligned bases
+  int skip_dq;  // dK and dV only: dQ comes from the query-major kernel (k_flash_bwd_dq)
 };
 
 // Start-address step (address / 16) of k-step kk (16 elements of the
@@ -1003,9 +1004,21 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       bool issued = false;
       bool ok = mbar_wait(kv_full, 0) && !*abort_flag;
       if (!ok) record_error(p.err, 200);
+      // dP^T(it) = V dO^T into the dP^T columns
+      auto issue_dp = [&](int it) {
+        const int st = it & 1;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < FB_HD / 16; ++kk)
+          umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
+      };
+      // With skip_dq the dP^T columns are free once the gradient warps have
+      // signalled p_full, so dP^T(it + 1) is issued right behind dV, dK(it),
+      // before the wait for them to finish: the tensor pipe stays queued.
+      bool dp_early = false;
       for (int it = 0; it < n_it && ok; ++it) {
         const int st = it & 1;
-        if (*abort_flag || !mbar_wait(&q_full[st], (it >> 1) & 1)) {
+        if (!dp_early && (*abort_flag || !mbar_wait(&q_full[st], (it >> 1) & 1))) {
           record_error(p.err, 210 + (it & 63));
           ok = false;
           break;
@@ -1021,16 +1034,15 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         for (int kk = 0; kk < FB_HD / 16; ++kk)
           umma_bf16(tmem + C::C_S, dK_km + km_step(kk), dQ_km + st * kStage + km_step(kk), id_s, kk != 0);
         issued = true;
-        // dP^T columns hold dQ^T of the previous iteration until it is read out
-        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1)) {
-          record_error(p.err, 250 + (it & 15));
-          ok = false;
-          break;
+        if (!dp_early) {
+          // dP^T columns hold dQ^T of the previous iteration until it is read out
+          if (it > 0 && !p.skip_dq && !mbar_wait(dq_empty, (it - 1) & 1)) {
+            record_error(p.err, 250 + (it & 15));
+            ok = false;
+            break;
+          }
+          issue_dp(it);
         }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < FB_HD / 16; ++kk)
-          umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
         umma_commit(s_full);
         if (*abort_flag || !mbar_wait(p_full, it & 1)) {
           record_error(p.err, 280 + (it & 15));
@@ -1050,11 +1062,23 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         }
         umma_commit(pdone);
         // dQ^T = K^T dS^T (K = 128 keys in 8 steps) into the dP^T columns
+        if (!p.skip_dq) {
 #pragma unroll
-        for (int kk = 0; kk < FB_BKV / 16; ++kk)
-          umma_bf16(tmem + C::C_DP, dK_mn + kk * kMn, ddSt_mn + kk * kMn, id_dq, kk != 0);
+          for (int kk = 0; kk < FB_BKV / 16; ++kk)
+            umma_bf16(tmem + C::C_DP, dK_mn + kk * kMn, ddSt_mn + kk * kMn, id_dq, kk != 0);
+        }
         umma_commit(mma_done);
         umma_commit(&q_empty[st]);
+        dp_early = false;
+        if (p.skip_dq && it + 1 < n_it) {
+          if (*abort_flag || !mbar_wait(&q_full[(it + 1) & 1], ((it + 1) >> 1) & 1)) {
+            record_error(p.err, 210 + ((it + 1) & 63));
+            ok = false;
+            break;
+          }
+          issue_dp(it + 1);
+          dp_early = true;
+        }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -1109,7 +1133,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         ++h;
       }
       // dQ^T of the previous iteration first: its columns take this iteration's dP^T
-      if (it > 0) {
+      if (it > 0 && !p.skip_dq) {
         if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1)) {
           record_error(p.err, 400 + (it & 63));
           ok = false;
@@ -1190,7 +1214,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         tmem_st_32x32b_x8(tmem + lane_base + C::C_S + qg * FB_QW + hf * 16 + 8, ds);
         // dS^T row r, queries [32 qg + 16 hf, +16): sub-tile qg / 2, 16-byte chunks 4 (qg % 2) + 2 hf, +1
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {
+        for (int c2 = 0; c2 < 2 && !p.skip_dq; ++c2) {
           const int chunk = 4 * (qg & 1) + 2 * hf + c2;
           const int off = (qg >> 1) * C::SUB + r * 128 + ((chunk ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(sdSt + off) = make_uint4(ds[4 * c2], ds[4 * c2 + 1], ds[4 * c2 + 2], ds[4 * c2 + 3]);
@@ -1204,13 +1228,20 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       h_prev = hq;
       q0_prev = q0;
     }
-    if (ok && n_it > 0) {
+    if (ok && n_it > 0 && !p.skip_dq) {
       if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (n_it - 1) & 1)) {
         record_error(p.err, 450);
         ok = false;
       } else {
         tc_fence_after();
         flush_dq(h_prev, q0_prev);
+      }
+    } else if (ok && n_it > 0) {  // dK and dV only: their last products must be done
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(pdone, (n_it - 1) & 1)) {
+        record_error(p.err, 451);
+        ok = false;
+      } else {
+        tc_fence_after();
       }
     }
     if (!ok) {
@@ -1288,9 +1319,332 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
 
 }  // namespace
 
+// ===========================================================================
+// dQ of the backward, query-major (head_dim 128), deterministic: one CTA per
+// (128-query block, query head, sequence) sums dQ over its key blocks
+// 0 .. qb in tensor memory and writes each element once, so no reductions
+// and one fixed summation order:
+//   S = Q K_j^T,  dP = dO V_j^T            (128 queries x 128 keys, TMEM)
+//   dS = exp2(S sl2 - LSE') (dP - D)       (8 gradient warps: one query row
+//        per thread, 64 keys per warp; bf16 dS written over the S columns it
+//        was computed from, the A operand of the next product)
+//   dQ += dS K_j                           (128 queries x hd, TMEM, A from TMEM)
+// S is double-buffered, so S_{j+1} runs while block j's gradients are
+// computed; dP is single (the gradient warps have read it when they signal).
+// Tensor memory: S [0,128) and [128,256), dP [256,384), dQ [384,512).
+// Shared memory: Q, dO, two K and two V stages (192 KB). dS of keys
+// [0, 64) sits in columns [0, 32) of its S buffer and of keys [64, 128) in
+// [64, 96): each warp overwrites only scores it has already read.
+// ===========================================================================
+namespace {
+
+constexpr int FQ_THREADS = 320;  // producer, MMA, 8 gradient warps
+
+struct FqCfg {
+  static constexpr int TILE = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16 as two 64-column sub-tiles
+  static constexpr int SUB = 128 * 128;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_DO = TILE;
+  static constexpr int OFF_K = 2 * TILE;  // [2]
+  static constexpr int OFF_V = 4 * TILE;  // [2]
+  static constexpr int OFF_BAR = 6 * TILE;
+  static constexpr int SMEM = 1024 + OFF_BAR + 256;
+  static constexpr uint32_t C_S = 0, C_DP = 256, C_DQ = 384;
+};
+
+struct FqParams {
+  const float* LSE;
+  const float* Dv;
+  float* dQacc;
+  int64_t ldqa;
+  int s, H, Hkv;
+  float scale;
+  int* err;
+};
+
+// Tensor-memory column of the A operand (dS) for k-step kk of S buffer sb.
+__device__ __forceinline__ uint32_t fq_a_col(int sb, int kk) {
+  return FqCfg::C_S + 128u * sb + (kk < 4 ? 8u * kk : 64u + 8u * (kk - 4));
+}
+
+__global__ void __launch_bounds__(FQ_THREADS, 1)
+    k_flash_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, FqParams p) {
+  using C = FqCfg;
+  constexpr int HD = 128;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sdO = smem + C::OFF_DO;
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* qd_full = bar + 0;
+  uint64_t* k_full = bar + 1;    // [2]
+  uint64_t* v_full = bar + 3;    // [2]
+  uint64_t* kv_empty = bar + 5;  // [2] K_j and V_j read by every product of block j
+  uint64_t* s_full = bar + 7;    // [2 S buffers] S_j and dP_j in tensor memory
+  uint64_t* p_full = bar + 9;    // dS_j written and dP_j read, 8 warps
+  uint64_t* dq_full = bar + 10;  // every dQ product done
+  uint64_t* drain = bar + 11;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 12);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 13);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = gridDim.x - 1 - blockIdx.x;  // longest rows first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.H / p.Hkv);
+  const int q0 = qb * 128;
+  const int row0 = b * p.s;
+  const int n = qb + 1;  // key blocks 0 .. qb
+
+  if (threadIdx.x == 0) {
+    mbar_init(qd_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&k_full[i], 1);
+      mbar_init(&v_full[i], 1);
+      mbar_init(&kv_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+    }
+    mbar_init(p_full, 8);
+    mbar_init(dq_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
+      bool ok = true;
+      mbar_arrive_expect_tx(qd_full, 2 * C::TILE);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_2d(sQ + c * C::SUB, &tmQ, qd_full, h * HD + c * 64, row0 + q0);
+        tma_load_2d(sdO + c * C::SUB, &tmO, qd_full, h * HD + c * 64, row0 + q0);
+      }
+      for (int j = 0; j < n; ++j) {
+        const int st = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        if (*abort_flag || !mbar_wait(&kv_empty[st], ph ^ 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&k_full[st], C::TILE);
+        for (int c = 0; c < 2; ++c) tma_load_2d(sK + st * C::TILE + c * C::SUB, &tmK, &k_full[st], kvh * HD + c * 64, row0 + j * 128);
+        k_last[st] = (int)ph;
+        mbar_arrive_expect_tx(&v_full[st], C::TILE);
+        for (int c = 0; c < 2; ++c) tma_load_2d(sV + st * C::TILE + c * C::SUB, &tmV, &v_full[st], kvh * HD + c * 64, row0 + j * 128);
+        v_last[st] = (int)ph;
+      }
+      if (!ok) {
+        record_error(p.err, DEV_TIMEOUT_PRODUCER);
+        *abort_flag = 1;
+        // let every issued copy land before the CTA's shared memory goes away
+        if (!mbar_wait(qd_full, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        for (int s2 = 0; s2 < 2; ++s2) {
+          if (k_last[s2] >= 0 && !mbar_wait(&k_full[s2], (uint32_t)k_last[s2])) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+          if (v_last[s2] >= 0 && !mbar_wait(&v_full[s2], (uint32_t)v_last[s2])) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t id_s = idesc_bf16_f32(128, 128, false, false);   // S, dP: both operands K-major
+      constexpr uint32_t id_dq = idesc_bf16_f32(128, HD, false, true);    // dQ += dS K: A in TMEM, K hd-major
+      const uint64_t dQd = sdesc_sw128(smem_u32(sQ), 16, 1024), dOd = sdesc_sw128(smem_u32(sdO), 16, 1024);
+      const uint64_t dKk = sdesc_sw128(smem_u32(sK), 16, 1024), dVk = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dKm = sdesc_sw128(smem_u32(sK), C::SUB, 1024);
+      constexpr uint32_t kStage = C::TILE >> 4, kMn = 2048 >> 4;
+      auto km = [](int kk) { return (uint32_t)(((kk >> 2) * C::SUB + (kk & 3) * 32) >> 4); };
+      bool ok = mbar_wait(qd_full, 0) && !*abort_flag;
+      bool issued = false;
+      auto issue_s = [&](int j) -> bool {
+        const int st = j & 1;
+        if (*abort_flag || !mbar_wait(&k_full[st], (j >> 1) & 1)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_bf16(tmem + C::C_S + 128u * (j & 1), dQd + km(kk), dKk + st * kStage + km(kk), id_s, kk != 0);
+        issued = true;
+        return true;
+      };
+      auto issue_dp = [&](int j) -> bool {
+        const int st = j & 1;
+        if (*abort_flag || !mbar_wait(&v_full[st], (j >> 1) & 1)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk)
+          umma_bf16(tmem + C::C_DP, dOd + km(kk), dVk + st * kStage + km(kk), id_s, kk != 0);
+        umma_commit(&s_full[j & 1]);  // S_j (issued earlier) and dP_j
+        return true;
+      };
+      if (ok) ok = issue_s(0) && issue_dp(0);
+      for (int j = 0; j < n && ok; ++j) {
+        const int st = j & 1;
+        // S buffer (j + 1) & 1 last held dS_{j-1}, read by a dQ product issued before
+        if (j + 1 < n && !issue_s(j + 1)) {
+          ok = false;
+          break;
+        }
+        if (*abort_flag || !mbar_wait(p_full, j & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          umma_bf16_ts(tmem + C::C_DQ, tmem + fq_a_col(j & 1, kk), dKm + st * kStage + kk * kMn, id_dq, (j | kk) != 0);
+        umma_commit(&kv_empty[st]);
+        // the gradient warps have read dP_j: dP_{j+1} may take its columns
+        if (j + 1 < n && !issue_dp(j + 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok) umma_commit(dq_full);
+      if (!ok) {
+        record_error(p.err, DEV_TIMEOUT_MMA);
+        *abort_flag = 1;
+      }
+      if (issued) {  // every MMA issued here completes before tensor memory is freed
+        umma_commit(drain);
+        if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+      }
+    }
+  } else {
+    // ---------------- gradient warps (2 .. 9) ----------------
+    const int wq = warp - 2;
+    const int half = wq >> 2;             // keys [64 half, 64 half + 64) of each block
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;    // query row of the block == tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int qi = q0 + r;
+    const float sl2 = p.scale * 1.4426950408889634f;
+    const int64_t vi = ((int64_t)b * p.H + h) * p.s + qi;
+    const float lse2 = qi < p.s ? __ldg(p.LSE + vi) * 1.4426950408889634f : 0.f;
+    const float dr = qi < p.s ? __ldg(p.Dv + vi) : 0.f;
+    bool ok = true;
+    for (int j = 0; j < n; ++j) {
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(&s_full[j & 1], (j >> 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sb = tmem + lane_base + C::C_S + 128u * (j & 1) + 64u * half;
+      const uint32_t db = tmem + lane_base + C::C_DP + 64u * half;
+      // The causal mask touches only the diagonal block (the last): query row
+      // r sees keys [0, r] of it.
+      auto chunk = [&](int c, auto diag_tag) {
+        constexpr bool DIAG = decltype(diag_tag)::value;
+        uint32_t sv[32], dv[32], ds[16];
+        tmem_ld_32x32b_x32(sb + 32 * c, sv);
+        tmem_ld_32x32b_x32(db + 32 * c, dv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float g[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int kl = 64 * half + 32 * c + e + u;
+            const float pr = ex2(fmaf(__uint_as_float(sv[e + u]), sl2, -lse2));
+            g[u] = (DIAG && kl > r) ? 0.f : pr * (__uint_as_float(dv[e + u]) - dr);
+          }
+          ds[e >> 1] = pack_bf16x2(g[0], g[1]);
+        }
+        // keys [64 half + 32 c, +32) -> columns 64 half + 16 c .. + 16 (key k in column k / 2
+        // within the half's 32 columns): scores this warp has already read
+        tmem_st_32x32b_x8(sb + 16 * c, *reinterpret_cast<const uint32_t(*)[8]>(ds));
+        tmem_st_32x32b_x8(sb + 16 * c + 8, *reinterpret_cast<const uint32_t(*)[8]>(ds + 8));
+      };
+      if (j == n - 1) {
+        chunk(0, std::true_type{});
+        chunk(1, std::true_type{});
+      } else {
+        chunk(0, std::false_type{});
+        chunk(1, std::false_type{});
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_full);
+    }
+    if (ok && (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(dq_full, 0))) ok = false;
+    if (!ok) {
+      record_error(p.err, DEV_TIMEOUT_EPILOGUE);
+      *abort_flag = 1;
+    } else {
+      tc_fence_after();
+      float* dst = p.dQacc + (int64_t)(row0 + qi) * p.ldqa + (int64_t)h * HD + 64 * half;
+#pragma unroll 1
+      for (int c = 0; c < 2; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + C::C_DQ + 64u * half + 32u * c, v);  // warp-collective
+        tmem_ld_wait();
+        if (qi < p.s) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + 32 * c + e) =
+                make_float4(__uint_as_float(v[e]) * p.scale, __uint_as_float(v[e + 1]) * p.scale,
+                            __uint_as_float(v[e + 2]) * p.scale, __uint_as_float(v[e + 3]) * p.scale);
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// dQ of the head_dim-128 backward by the query-major kernel: writes every
+// element of dq_acc's head columns once (scaled, before RoPE's transpose).
+// a.dvec must already hold D = rowsum(dO * O).
+int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* err) {
+  using C = FqCfg;
+  if (a.hd != 128) return MT_ERR_CONFIG;
+  if ((reinterpret_cast<uintptr_t>(a.dq_acc) & 15) || (a.ldqa % 4)) return MT_ERR_ARG;
+  static bool attr = false;
+  if (!attr) {
+    if (cudaFuncSetAttribute(k_flash_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+      return MT_ERR_CUDA;
+    attr = true;
+  }
+  const int64_t T = (int64_t)a.b * a.s;
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * 128, T, a.ldqkv, 128) ||
+      !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * 128, T, a.ldqkv, 128) ||
+      !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * 128, T, a.ldqkv, 128) ||
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * 128, T, a.ldo, 128))
+    return MT_ERR_ARG;
+  FqParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, a.s, a.H, a.Hkv, a.scale, err};
+  dim3 grid((a.s + 127) / 128, a.H, a.b);
+  k_flash_bwd_dq<<<grid, FQ_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
+  return launch_status();
+}
+
 // Backward with head_dim 128 on the tensor cores. a.dvec must already hold
-// D = rowsum(dO * O) and a.dq_acc must be zeroed; the caller casts dQ.
-int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
+// D = rowsum(dO * O) and, unless skip_dq, a.dq_acc must be zeroed; the caller
+// casts dQ. skip_dq: dK and dV only (dQ from attention_bwd_dq_tc).
+int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err, bool skip_dq) {
   using C = FbCfg;
   if (a.hd != FB_HD) return MT_ERR_CONFIG;
   static bool attr = false;
@@ -1308,7 +1662,7 @@ int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err) {
     return MT_ERR_ARG;
   const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
-             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
+             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0, skip_dq ? 1 : 0};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
   k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
   return launch_status();

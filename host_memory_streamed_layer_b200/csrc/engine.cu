@@ -310,7 +310,7 @@ int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
   int r = bwd ? (a.hd == 128 ? attention_bwd_tc(a, c->s_comp, c->d_err) : attention_bwd(a, c->s_comp))
               : attention_fwd_tc(a, c->s_comp, c->d_err);
   if (r != MT_OK) return set_err(c, r, "attention launch failed");
-  c->launches += bwd ? 4 : 1;
+  c->launches += bwd ? (a.hd == 128 ? attention_bwd_kernels() : 3) : 1;
   if (timing && e0 && e1) {
     cudaEventRecord(e1, c->s_comp);
     // causal attention: QK^T and PV over the visible half, per query head
@@ -1416,6 +1416,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   const Shapes& s = y.sh;
   mt_shard plan{};
   const NcclApi* nccl = nullptr;
+  if (cfg->E > 0) return set_err(nullptr, MT_ERR_CONFIG, "expert layers are not on the engine's path");
   if (world > 0) {
     if (!id) return set_err(nullptr, MT_ERR_ARG, "sharded context without an NCCL id");
     if (cfg->flags & (MT_FLAG_DEFER_UPDATES | MT_FLAG_TIED_EMBED | MT_FLAG_BF16_GRADS))

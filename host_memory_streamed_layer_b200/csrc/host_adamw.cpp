@@ -8,8 +8,6 @@
 
 #include <immintrin.h>
 #include <math.h>
-#include <pthread.h>
-#include <sched.h>
 #include <stdlib.h>
 #include <string.h>
 
@@ -176,35 +174,8 @@ void bf16_round_chunk(const float* x, uint16_t* out, size_t n) {
 }
 
 // ---------------------------------------------------------------------------
-// MT_PIN_THREADS=1: worker i runs on the (i+1)-th CPU the process may use
-// (the first is left to the calling thread), so that a worker keeps its core
-// and the pages it first touched stay near it. Read once per process.
-static bool pin_threads() {
-  static const bool yes = [] {
-    const char* e = getenv("MT_PIN_THREADS");
-    return e && e[0] == '1';
-  }();
-  return yes;
-}
-
 ThreadPool::ThreadPool(int workers) {
-  std::vector<int> cpus;
-  if (pin_threads()) {
-    cpu_set_t set;
-    CPU_ZERO(&set);
-    if (sched_getaffinity(0, sizeof(set), &set) == 0)
-      for (int c = 0; c < CPU_SETSIZE; ++c)
-        if (CPU_ISSET(c, &set)) cpus.push_back(c);
-  }
-  for (int i = 0; i < workers; ++i) {
-    workers_.emplace_back([this] { loop(); });
-    if (cpus.size() > 1) {
-      cpu_set_t one;
-      CPU_ZERO(&one);
-      CPU_SET(cpus[(size_t)(i + 1) % cpus.size()], &one);
-      pthread_setaffinity_np(workers_.back().native_handle(), sizeof(one), &one);
-    }
-  }
+  for (int i = 0; i < workers; ++i) workers_.emplace_back([this] { loop(); });
 }
 
 ThreadPool::~ThreadPool() {

@@ -30,6 +30,11 @@ extern "C" int mt_k_attn_fwd_variant(int variant) {
   return mt::attention_fwd_variant(variant);
 }
 
+extern "C" int mt_k_attn_bwd_variant(int variant) {
+  if (variant < 0 || variant > 2) return MT_ERR_ARG;
+  return mt::attention_bwd_variant(variant);
+}
+
 #include <cmath>
 
 namespace {

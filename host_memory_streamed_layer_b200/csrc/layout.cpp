@@ -34,6 +34,8 @@ int validate_config(const mt_config* c, std::string* why) {
       !(c->beta2 >= 0 && c->beta2 < 1) || !(c->adam_eps > 0) || !(c->wd >= 0))
     return fail(MT_ERR_CONFIG, "hyper-parameter out of range");
   if (c->host_threads < 0) return fail(MT_ERR_CONFIG, "host_threads must be >= 0");
+  if (c->E < 0 || c->E > 64) return fail(MT_ERR_CONFIG, "E (experts) must be in [0, 64]");
+  if (c->E > 0 && (c->topk < 1 || c->topk > c->E)) return fail(MT_ERR_CONFIG, "topk must be in [1, E]");
   if ((c->flags & MT_FLAG_TIED_EMBED) && (c->flags & MT_FLAG_BF16_GRADS))
     return fail(MT_ERR_CONFIG, "tied embeddings take their gradients in fp32 (no MT_FLAG_BF16_GRADS)");
   return MT_OK;
@@ -54,6 +56,9 @@ Layout make_layout(const mt_config& c) {
   s.T = c.b * c.s;
   s.Nqkv = (c.H + 2 * c.Hkv) * s.hd;
   s.Hd = c.H * s.hd;
+  s.E = c.E;
+  s.topk = c.E > 0 ? c.topk : 0;
+  const size_t Ee = c.E > 0 ? (size_t)c.E : 1;  // expert blocks of the MLP tensors
   size_t off = 0;
   auto put = [&](size_t n) {
     TRef r{off, n};
@@ -71,9 +76,10 @@ Layout make_layout(const mt_config& c) {
     t[MT_T_WV] = put((size_t)c.Hkv * s.hd * d);
     t[MT_T_WO] = put(d * (size_t)s.Hd);
     t[MT_T_MLP_NORM] = put(d);
-    t[MT_T_WGATE] = put(F * d);
-    t[MT_T_WUP] = put(F * d);
-    t[MT_T_WDOWN] = put(d * F);
+    t[MT_T_WGATE] = put(Ee * F * d);
+    t[MT_T_WUP] = put(Ee * F * d);
+    t[MT_T_WDOWN] = put(Ee * d * F);
+    t[MT_T_ROUTER] = put(c.E > 0 ? (size_t)c.E * d : 0);
   }
   y.final_norm = put(d);
   y.tied = (c.flags & MT_FLAG_TIED_EMBED) != 0;
@@ -95,8 +101,9 @@ Layout make_layout(const mt_config& c) {
   y.bf_qkv = bput((size_t)s.Nqkv * d);
   y.bf_o = bput(d * (size_t)s.Hd);
   y.bf_g2 = bput(d);
-  y.bf_gu = bput(2 * F * d);
-  y.bf_d = bput(d * F);
+  y.bf_gu = bput(2 * Ee * F * d);
+  y.bf_d = bput(Ee * d * F);
+  y.bf_r = bput(c.E > 0 ? (size_t)c.E * d : 0);
   y.bf_layer = b;
   return y;
 }
@@ -111,8 +118,9 @@ size_t Layout::bf_of(int tid) const {
     case MT_T_WO: return bf_o;
     case MT_T_MLP_NORM: return bf_g2;
     case MT_T_WGATE: return bf_gu;
-    case MT_T_WUP: return bf_gu + (size_t)sh.F * d;
+    case MT_T_WUP: return bf_gu + (size_t)(sh.E > 0 ? sh.E : 1) * sh.F * d;
     case MT_T_WDOWN: return bf_d;
+    case MT_T_ROUTER: return bf_r;
   }
   return 0;
 }
@@ -153,6 +161,7 @@ extern "C" int mt_tensor_offset(const mt_config* cfg, int layer, int tid, size_t
       return MT_ERR_ARG;
   } else {
     if (layer < 0 || layer >= cfg->L || tid < 0 || tid >= mt::kLayerTensors) return MT_ERR_ARG;
+    if (tid == MT_T_ROUTER && cfg->E == 0) return MT_ERR_ARG;  // dense MLP: no router
     r = y.t(layer, tid);
   }
   if (offset_floats) *offset_floats = r.off;
@@ -188,6 +197,7 @@ extern "C" int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard
   if (mt::validate_config(cfg, nullptr) != MT_OK) return MT_ERR_CONFIG;
   if (cfg->d % 128) return MT_ERR_CONFIG;  // fp32 and bf16 block offsets coincide only then
   if (cfg->flags & MT_FLAG_TIED_EMBED) return MT_ERR_CONFIG;  // one table, two owners: not partitioned
+  if (cfg->E > 0) return MT_ERR_CONFIG;  // expert layers: not partitioned
   const mt::Layout y = mt::make_layout(*cfg);
   const size_t lb = y.layer_begin(0), le = y.layer_end(0);
   // The fp32 arena block of a layer and its bf16 streamed block must hold

@@ -3,13 +3,16 @@
 // fp32 master arena (caller-visible, also the layout of the gradient arena):
 //   embedding [V,d]; per layer: attention-norm gain [d], Wq [H hd, d],
 //   Wk [Hkv hd, d], Wv [Hkv hd, d], Wo [d, H hd], MLP-norm gain [d],
-//   Wgate [F,d], Wup [F,d], Wdown [d,F]; final-norm gain [d]; LM head [V,d].
+//   Wgate [F,d], Wup [F,d], Wdown [d,F] (with E experts: [E,F,d], [E,F,d],
+//   [E,d,F], then the router [E,d]); final-norm gain [d]; LM head [V,d].
 //   Row-major [out, in], every tensor on a 256-byte boundary. With d a
 //   multiple of 64 no padding is needed, so Wq|Wk|Wv and Wgate|Wup are
 //   adjacent and one layer is one contiguous range.
 // bf16 layer block (host mirror and device weight slot), per layer:
 //   g1 [d] | Wqkv [(H+2Hkv) hd, d] | Wo [d, H hd] | g2 [d] | Wgu [2F, d] | Wd [d, F]
-//   each part on a 256-byte boundary.
+//   each part on a 256-byte boundary; with E experts Wgu holds every
+//   expert's gate rows [E F, d] then every expert's up rows, Wd [E d, F], and
+//   the router [E, d] follows.
 #pragma once
 
 #include <stddef.h>
@@ -22,7 +25,7 @@
 
 namespace mt {
 
-constexpr int kLayerTensors = 9;
+constexpr int kLayerTensors = 10;  // MT_T_ATTN_NORM .. MT_T_WDOWN, MT_T_ROUTER (empty without experts)
 
 struct TRef {
   size_t off = 0;  // elements
@@ -31,6 +34,7 @@ struct TRef {
 
 struct Shapes {
   int L, d, H, Hkv, F, V, b, s, hd, T, Nqkv, Hd;  // Hd = H * hd
+  int E = 0, topk = 0;                            // experts (0: dense MLP), experts per token
 };
 
 struct Layout {
@@ -50,7 +54,7 @@ struct Layout {
   }
   const TRef& t(int l, int tid) const { return layer[(size_t)l * kLayerTensors + tid]; }
   // bf16 layer block, in elements
-  size_t bf_g1 = 0, bf_qkv = 0, bf_o = 0, bf_g2 = 0, bf_gu = 0, bf_d = 0, bf_layer = 0;
+  size_t bf_g1 = 0, bf_qkv = 0, bf_o = 0, bf_g2 = 0, bf_gu = 0, bf_d = 0, bf_r = 0, bf_layer = 0;
   // bf16 offset of arena tensor tid inside the layer block
   size_t bf_of(int tid) const;
 };

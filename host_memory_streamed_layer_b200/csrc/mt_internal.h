@@ -97,7 +97,32 @@ int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
 // Backward on the tcgen05 tensor cores for head_dim 128 (same outputs as
 // attention_bwd); _main is the tensor-core kernel alone.
 int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
-int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* dev_err);
+int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* dev_err, bool skip_dq);
+// dQ of the head_dim-128 backward by the query-major kernel (no reductions).
+int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
+// Backward form for head_dim 128 in later calls (0 automatic, 1 fused: dQ by
+// reductions inside the key-major kernel, 2 split: dK/dV by the key-major
+// kernel, dQ by the query-major one, deterministic); returns the previous one.
+int attention_bwd_variant(int v);
+// Kernels one head_dim-128 backward launches in the current form.
+int attention_bwd_kernels();
+
+// Mixture-of-experts MLP (moe.cu). Router: logits [T, E], the topk experts
+// idx [T, k] and their gates [T, k] of the bf16 MLP input w [T, d] and router
+// Wr [E, d]. Gather: xe[slot] = w[row_of[slot]]. Combine: out = h + the
+// gated expert outputs ye (fp32 rows by slot). Dy: dye[slot] = gate dy (bf16)
+// and dgate = dy . ye. Router backward: dlogits, dWr [E, d] and the MLP
+// input's gradient dw [T, d] (router term plus the routed rows' dxe).
+int launch_moe_router(const void* w, const void* Wr, int T, int d, int E, int k, float* logits, int32_t* idx,
+                      float* gate, cudaStream_t st);
+int launch_moe_gather(const void* w, const int32_t* row_of, int rows, int d, void* xe, cudaStream_t st);
+int launch_moe_combine(const float* h, const float* ye, const int32_t* slot_of, const float* gate, int T, int k,
+                       int d, float* out, cudaStream_t st);
+int launch_moe_dy(const float* dy, const float* ye, const int32_t* slot_of, const float* gate, int T, int k, int d,
+                  void* dye, float* dgate, cudaStream_t st);
+int launch_moe_router_bwd(const float* gate, const float* dgate, const int32_t* idx, const void* w, const void* Wr,
+                          const float* dxe, const int32_t* slot_of, int T, int k, int d, int E, float* dlogits,
+                          float* dWr, float* dw, cudaStream_t st);
 
 int launch_rmsnorm_fwd(const float* x, const void* g, void* y, float* rstd, int T, int d, float eps, cudaStream_t st);
 int rmsnorm_bwd_blocks(int T);

@@ -215,6 +215,8 @@ def main():
     ap.add_argument("--attn-shape", default=f"{B},{S},{H}", help="attention: sequences,length,heads")
     ap.add_argument("--attn-variant", default="auto", choices=["auto", "one", "pingpong"],
                     help="attention forward kernel (head dim 128): automatic, one or two query tiles per CTA")
+    ap.add_argument("--attn-bwd", default="auto", choices=["auto", "fused", "split"],
+                    help="attention backward (head dim 128): dQ by reductions, or the deterministic split")
     a = ap.parse_args()
     if a.kernel == "gemm":
         table = None
@@ -227,6 +229,8 @@ def main():
         ab, as_, ah = (int(x) for x in a.attn_shape.split(","))
         mt.mt_k_attn_fwd_variant({"auto": mt.ATTN_AUTO, "one": mt.ATTN_ONE_TILE,
                                   "pingpong": mt.ATTN_PINGPONG}[a.attn_variant])
+        mt.mt_k_attn_bwd_variant({"auto": mt.ATTN_BWD_AUTO, "fused": mt.ATTN_BWD_FUSED,
+                                  "split": mt.ATTN_BWD_SPLIT}[a.attn_bwd])
         res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl, ab, as_, ah)
         for r in res:
             r["shape"] = dict(b=ab, s=as_, heads=ah, hd=HD)

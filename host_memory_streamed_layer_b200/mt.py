@@ -54,6 +54,7 @@ def mt_k_gemm_bf16(A, lda, a_mn, B, ldb, b_mn, C, ldc, out_kind, R, ldr, M, N, K
 
 _sig("mt_k_gemm_variant", c_int, c_int)
 _sig("mt_k_attn_fwd_variant", c_int, c_int)
+_sig("mt_k_attn_bwd_variant", c_int, c_int)
 GEMM_AUTO, GEMM_SINGLE, GEMM_PAIR = 0, 1, 2
 
 
@@ -74,6 +75,18 @@ def mt_k_attn_fwd_variant(variant: int) -> int:
     rc = lib.mt_k_attn_fwd_variant(variant)
     if rc < 0:
         raise MTError(rc, "mt_k_attn_fwd_variant")
+    return rc
+
+
+ATTN_BWD_AUTO, ATTN_BWD_FUSED, ATTN_BWD_SPLIT = 0, 1, 2
+
+
+def mt_k_attn_bwd_variant(variant: int) -> int:
+    """Selects the head-dim-128 attention backward form for later calls
+    (fused dQ reductions, or the deterministic split); returns the previous."""
+    rc = lib.mt_k_attn_bwd_variant(variant)
+    if rc < 0:
+        raise MTError(rc, "mt_k_attn_bwd_variant")
     return rc
 
 
@@ -203,6 +216,7 @@ MT_FLAG_TIED_EMBED = 0x80
 MT_FLAG_STASH_ATTN = 0x100
 MT_GRAD_RING_SLOTS = 3
 MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
+MT_T_ROUTER = 9
 MT_T_EMBED, MT_T_FINAL_NORM, MT_T_LM_HEAD = 100, 101, 102
 
 
@@ -213,7 +227,7 @@ class mt_config(ctypes.Structure):
                 ("rope_base", ctypes.c_float), ("lr", ctypes.c_float), ("beta1", ctypes.c_float),
                 ("beta2", ctypes.c_float), ("adam_eps", ctypes.c_float), ("wd", ctypes.c_float),
                 ("seed", ctypes.c_uint64), ("flags", ctypes.c_uint32), ("device", ctypes.c_int32),
-                ("host_threads", ctypes.c_int32)]
+                ("host_threads", ctypes.c_int32), ("E", ctypes.c_int32), ("topk", ctypes.c_int32)]
 
 
 class mt_stats(ctypes.Structure):

@@ -146,6 +146,15 @@ extern "C" {
 #define MT_T_WGATE 6
 #define MT_T_WUP 7
 #define MT_T_WDOWN 8
+/* Mixture-of-experts layers (E > 0; saify.me, "Who this is actually for",
+ * lists MoE variants among the supported families and gives no routing rule,
+ * so the plainest reading is taken): WGATE and WUP hold [E, F, d] (expert e's
+ * rows at e * F * d), WDOWN [E, d, F], and MT_T_ROUTER the router [E, d].
+ * Per token t of the MLP input w: logits = w Wr^T; the topk experts with the
+ * largest logits (ties to the lower index); gates = softmax of those logits;
+ * output = sum over them of gate * SwiGLU_e(w). Every routed token is
+ * computed (no capacity limit) and the loss has no auxiliary term. */
+#define MT_T_ROUTER 9
 #define MT_T_EMBED 100
 #define MT_T_FINAL_NORM 101
 #define MT_T_LM_HEAD 102
@@ -167,6 +176,8 @@ typedef struct mt_config {
   uint32_t flags;       /* MT_FLAG_* */
   int32_t device;       /* CUDA device ordinal */
   int32_t host_threads; /* host AdamW threads; 0 = all cores but one */
+  int32_t E;            /* experts per mixture-of-experts MLP; 0 = the dense SwiGLU MLP */
+  int32_t topk;         /* experts each token is routed to (1 <= topk <= E) when E > 0 */
 } mt_config;
 
 typedef struct mt_ctx mt_ctx;

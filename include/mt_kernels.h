@@ -194,12 +194,24 @@ int mt_k_gemm_variant(int variant);
 
 /* Selects the tcgen05 attention forward kernel for head dim 128 in later calls
  * (mt_k_attn_fwd_tc and the engine): 0 automatic (the default: two query tiles
- * per CTA from s = 8192 on, one below), 1 one 128-query tile per CTA, 2 two
+ * per CTA for s > 8192, one otherwise), 1 one 128-query tile per CTA, 2 two
  * 128-query tiles per CTA in ping-pong, P kept in tensor memory. Both compute
  * the same attention; this exists for measurement and tests. Returns the
  * previous choice, or MT_ERR_ARG for another value (nothing changes). No GPU
  * work. */
 int mt_k_attn_fwd_variant(int variant);
+
+/* Selects the form of the tcgen05 attention backward (mt_k_attn_bwd_tc and the
+ * engine) in later calls: 0 automatic (the default), 1 fused: one key-major
+ * kernel computes dK, dV and dQ, adding each key block's dQ into dq_acc with
+ * fp32 reductions (their order, and so dQ's last bits, vary from run to run),
+ * 2 split: the key-major kernel computes dK and dV only and a query-major
+ * kernel sums dQ over the key blocks in tensor memory and writes each element
+ * once (deterministic: the same inputs give the same bits; needs dq_acc
+ * 16-byte aligned and ldqa a multiple of 4, MT_ERR_ARG otherwise). Returns
+ * the previous choice, or MT_ERR_ARG for another value (nothing changes). No
+ * GPU work. */
+int mt_k_attn_bwd_variant(int variant);
 
 /* Host AdamW over n fp32 elements, in place (HOST pointers, runs on the
  * calling thread; the engine runs the same routine across its worker pool):

@@ -29,6 +29,7 @@ import numpy as np
 # Tensor ids of the arena layout (same numbering as the seeded input module,
 # restated here so the oracle depends on nothing outside numpy).
 ATTN_NORM, WQ, WK, WV, WO, MLP_NORM, WGATE, WUP, WDOWN = range(9)
+ROUTER = 9  # mixture-of-experts layers only
 EMBED, FINAL_NORM, LM_HEAD = 100, 101, 102
 
 ALIGN_FLOATS = 64  # every tensor of the fp32 arena starts on a 256-byte boundary
@@ -56,10 +57,20 @@ class OracleConfig:
     # embedding table itself, z = n E^T, so E's gradient is the sum of the
     # gather's and the head's; the arena has no separate LM-head tensor.
     tied: bool = False
+    # Mixture-of-experts MLP (another of the families the pages list as
+    # supported, saify.me, "Who this is actually for", with no routing rule
+    # given): E experts of SwiGLU width F per layer and top-k routing, the
+    # plainest reading (moe_fwd below). E = 0: the dense SwiGLU MLP.
+    E: int = 0
+    topk: int = 2
 
     @property
     def hd(self) -> int:
         return self.d // self.H
+
+    @property
+    def layer_tids(self):
+        return list(range(10 if self.E else 9))
 
 
 # ---------------------------------------------------------------------------
@@ -75,10 +86,16 @@ def _layer_tensors(c: OracleConfig):
         (WV, (c.Hkv * hd, c.d)),
         (WO, (c.d, c.H * hd)),
         (MLP_NORM, (c.d,)),
+    ] + ([
         (WGATE, (c.F, c.d)),
         (WUP, (c.F, c.d)),
         (WDOWN, (c.d, c.F)),
-    ]
+    ] if not c.E else [
+        (WGATE, (c.E, c.F, c.d)),  # expert e's gate rows at [e]
+        (WUP, (c.E, c.F, c.d)),
+        (WDOWN, (c.E, c.d, c.F)),
+        (ROUTER, (c.E, c.d)),
+    ])
 
 
 def arena_layout(c: OracleConfig):
@@ -301,11 +318,96 @@ def swiglu_bwd(gt, up, dact):
 
 
 # ---------------------------------------------------------------------------
+# Mixture-of-experts MLP. Reading (the pages name MoE variants but no rule):
+#   logits = w Wr^T                      [T, E]
+#   R_t    = the k experts with the largest logits (ties: lower index first)
+#   g_t    = softmax of logits_t over R_t (the gates sum to 1)
+#   y_t    = sum_{e in R_t} g_te * SwiGLU_e(w_t),
+#            SwiGLU_e(w) = (silu(w Wg_e^T) * (w Wu_e^T)) Wd_e^T
+# Every routed token is computed (no capacity limit, none dropped) and the
+# loss has no auxiliary balancing term: the pages state neither.
+# ---------------------------------------------------------------------------
+
+def moe_route(w: np.ndarray, Wr: np.ndarray, k: int):
+    """Router of moe_fwd. w: [T, d]. Returns (logits [T, E], idx [T, k] of the
+    k largest logits per row, largest first, ties to the lower index)."""
+    logits = w @ Wr.T
+    idx = np.argsort(-logits, axis=-1, kind="stable")[:, :k]
+    return logits, idx
+
+
+def moe_gates(logits: np.ndarray, idx: np.ndarray) -> np.ndarray:
+    """Softmax of each row's selected logits: g [T, k]."""
+    sel = np.take_along_axis(logits, idx, axis=-1)
+    sel = sel - sel.max(axis=-1, keepdims=True)
+    e = np.exp(sel)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def moe_fwd(w: np.ndarray, Wr, Wg, Wu, Wd, k: int, idx=None):
+    """w: [T, d]; Wr [E, d], Wg/Wu [E, F, d], Wd [E, d, F]. idx: a given
+    routing (e.g. one a GPU took where two logits were within rounding of
+    each other), else the router's. Returns (y [T, d], cache)."""
+    logits, r_idx = moe_route(w, Wr, k)
+    if idx is None:
+        idx = r_idx
+    g = moe_gates(logits, idx)
+    T, d = w.shape
+    E = Wr.shape[0]
+    y = np.zeros((T, d))
+    ye = np.zeros(idx.shape + (d,))  # each routed token's expert output, before its gate
+    parts = {}
+    for e in range(E):
+        t, j = np.nonzero(idx == e)
+        if t.size == 0:
+            continue
+        we = w[t]
+        gt = we @ Wg[e].T
+        up = we @ Wu[e].T
+        act = swiglu_fwd(gt, up)
+        out = act @ Wd[e].T
+        ye[t, j] = out
+        parts[e] = (t, j, gt, up, act)
+    for j in range(idx.shape[1]):  # fixed order over the k slots
+        y += g[:, j:j + 1] * ye[:, j]
+    return y, dict(w=w, logits=logits, idx=idx, g=g, ye=ye, parts=parts)
+
+
+def moe_bwd(dy: np.ndarray, Wr, Wg, Wu, Wd, cache: dict):
+    """Backward of moe_fwd for a fixed routing. Returns (dw [T, d], dWr, dWg,
+    dWu, dWd):
+      dg_tj   = dy_t . ye_tj ;  dlogit_te = g_te (dg_te - sum_j g_tj dg_tj), e in R_t
+      expert e, over its tokens: dye = g dy ; dWd_e = dye^T act ; dact = dye Wd_e ;
+      (dgt, dup) = SwiGLU backward ; dWg_e = dgt^T w ; dWu_e = dup^T w ;
+      dw += dgt Wg_e + dup Wu_e ;  router: dWr = dlogit^T w, dw += dlogit Wr."""
+    w, logits, idx, g, ye, parts = (cache[k] for k in ("w", "logits", "idx", "g", "ye", "parts"))
+    T, d = w.shape
+    E = Wr.shape[0]
+    dg = np.einsum("td,tjd->tj", dy, ye)
+    dsel = g * (dg - np.sum(g * dg, axis=-1, keepdims=True))
+    dlogits = np.zeros_like(logits)
+    np.put_along_axis(dlogits, idx, dsel, axis=-1)
+    dWr = dlogits.T @ w
+    dw = dlogits @ Wr
+    dWg, dWu, dWd = np.zeros_like(Wg), np.zeros_like(Wu), np.zeros_like(Wd)
+    for e, (t, j, gt, up, act) in parts.items():
+        dye = g[t, j][:, None] * dy[t]
+        dWd[e] = dye.T @ act
+        dact = dye @ Wd[e]
+        dgt, dup = swiglu_bwd(gt, up, dact)
+        dWg[e] = dgt.T @ w[t]
+        dWu[e] = dup.T @ w[t]
+        np.add.at(dw, t, dgt @ Wg[e] + dup @ Wu[e])
+    return dw, dWr, dWg, dWu, dWd
+
+
+# ---------------------------------------------------------------------------
 # One decoder layer.
 # ---------------------------------------------------------------------------
 
-def layer_fwd(x: np.ndarray, W: dict, c: OracleConfig, cos, sin):
-    """x: [b, s, d] -> (x_next, cache). W keys: ATTN_NORM, WQ, ..., WDOWN."""
+def layer_fwd(x: np.ndarray, W: dict, c: OracleConfig, cos, sin, routing=None):
+    """x: [b, s, d] -> (x_next, cache). W keys: ATTN_NORM, WQ, ..., WDOWN (and
+    ROUTER with experts; routing: a given [b*s, k] expert choice)."""
     b, s, d = x.shape
     hd = c.hd
     u, r1 = rmsnorm_fwd(x, W[ATTN_NORM], c.norm_eps)
@@ -318,12 +420,16 @@ def layer_fwd(x: np.ndarray, W: dict, c: OracleConfig, cos, sin):
     a = o.reshape(b, s, c.H * hd)
     h = x + a @ W[WO].T
     w, r2 = rmsnorm_fwd(h, W[MLP_NORM], c.norm_eps)
+    cache = dict(x=x, u=u, r1=r1, qr=qr, kr=kr, v=v, P=P, a=a, h=h, w=w, r2=r2)
+    if c.E:
+        y, cache["moe"] = moe_fwd(w.reshape(b * s, d), W[ROUTER], W[WGATE], W[WUP], W[WDOWN], c.topk,
+                                  idx=routing)
+        return h + y.reshape(b, s, d), cache
     gt = w @ W[WGATE].T
     up = w @ W[WUP].T
     act = swiglu_fwd(gt, up)
     x_next = h + act @ W[WDOWN].T
-    cache = dict(x=x, u=u, r1=r1, qr=qr, kr=kr, v=v, P=P, a=a, h=h, w=w, r2=r2,
-                 gt=gt, up=up, act=act)
+    cache.update(gt=gt, up=up, act=act)
     return x_next, cache
 
 
@@ -332,15 +438,21 @@ def layer_bwd(dxn: np.ndarray, W: dict, cache: dict, c: OracleConfig, cos, sin):
     b, s, d = dxn.shape
     hd = c.hd
     T = b * s
-    x, u, h, w, a, act = (cache[k] for k in ("x", "u", "h", "w", "a", "act"))
+    x, u, h, w, a = (cache[k] for k in ("x", "u", "h", "w", "a"))
     G = {}
-    # x' = h + act Wd^T
-    G[WDOWN] = dxn.reshape(T, d).T @ act.reshape(T, c.F)
-    dact = dxn @ W[WDOWN]
-    dgt, dup = swiglu_bwd(cache["gt"], cache["up"], dact)
-    G[WGATE] = dgt.reshape(T, c.F).T @ w.reshape(T, d)
-    G[WUP] = dup.reshape(T, c.F).T @ w.reshape(T, d)
-    dw = dgt @ W[WGATE] + dup @ W[WUP]
+    if c.E:
+        dwf, G[ROUTER], G[WGATE], G[WUP], G[WDOWN] = moe_bwd(dxn.reshape(T, d), W[ROUTER], W[WGATE], W[WUP],
+                                                             W[WDOWN], cache["moe"])
+        dw = dwf.reshape(b, s, d)
+    else:
+        act = cache["act"]
+        # x' = h + act Wd^T
+        G[WDOWN] = dxn.reshape(T, d).T @ act.reshape(T, c.F)
+        dact = dxn @ W[WDOWN]
+        dgt, dup = swiglu_bwd(cache["gt"], cache["up"], dact)
+        G[WGATE] = dgt.reshape(T, c.F).T @ w.reshape(T, d)
+        G[WUP] = dup.reshape(T, c.F).T @ w.reshape(T, d)
+        dw = dgt @ W[WGATE] + dup @ W[WUP]
     dh_norm, G[MLP_NORM] = rmsnorm_bwd(h, W[MLP_NORM], cache["r2"], dw)
     dh = dxn + dh_norm
     # h = x + a Wo^T
@@ -398,9 +510,11 @@ def head_ce_fwd_bwd(xL, gf, Whead, labels, eps):
 # ---------------------------------------------------------------------------
 
 def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
-                     c: OracleConfig):
+                     c: OracleConfig, routing=None):
     """weights: dict (layer, tensor id) -> float64 array, the values the forward
-    and backward use. tokens, labels: int [b, s]. Returns (loss, grads dict)."""
+    and backward use. tokens, labels: int [b, s]. routing: optional dict
+    layer -> [b*s, k] expert choice (mixture-of-experts layers), else each
+    router's own. Returns (loss, grads dict)."""
     b, s = tokens.shape
     T = b * s
     cos, sin = rope_tables(s, c.hd, c.rope_base)
@@ -408,8 +522,8 @@ def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
     x = E[tokens]  # [b, s, d]
     caches = []
     for l in range(c.L):
-        W = {tid: weights[(l, tid)] for tid in range(9)}
-        x, cache = layer_fwd(x, W, c, cos, sin)
+        W = {tid: weights[(l, tid)] for tid in c.layer_tids}
+        x, cache = layer_fwd(x, W, c, cos, sin, routing=(routing or {}).get(l))
         caches.append(cache)
     Whead = E if c.tied else weights[(-1, LM_HEAD)]
     loss, dx, dgf, dWhead = head_ce_fwd_bwd(
@@ -419,7 +533,7 @@ def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
         grads[(-1, LM_HEAD)] = dWhead
     dx = dx.reshape(b, s, c.d)
     for l in reversed(range(c.L)):
-        W = {tid: weights[(l, tid)] for tid in range(9)}
+        W = {tid: weights[(l, tid)] for tid in c.layer_tids}
         dx, G = layer_bwd(dx, W, caches[l], c, cos, sin)
         for tid, g in G.items():
             grads[(l, tid)] = g

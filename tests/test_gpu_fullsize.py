@@ -126,7 +126,7 @@ def test_attention_full_shape_sampled(impl):
     assert np.linalg.norm(gv - rdv[0, -16:, 0]) <= 2e-2 * np.linalg.norm(rdv[0, -16:, 0])
 
 
-@pytest.mark.parametrize("impl", ["mma", "tc", "tc_pingpong"])
+@pytest.mark.parametrize("impl", ["mma", "tc", "tc_pingpong", "tc_split"])
 def test_attention_whole_heads_full_length(impl):
     """Every row of two whole heads at the full 2048-token length, element by
     element (per-row relative L2): o, the log-sum-exp, dq, dk and dv against
@@ -159,8 +159,12 @@ def test_attention_whole_heads_full_length(impl):
     dp = dqkv.data_ptr()
     bwd = mt.mt_k_attn_bwd if impl == "mma" else mt.mt_k_attn_bwd_tc
     kw = {} if impl == "mma" else {"dev_err": err.data_ptr()}
-    bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(), dvec.data_ptr(), dqa.data_ptr(),
-        H * HD, dp, ld, dp + 2 * H * HD, dp + 2 * (H + Hkv) * HD, ld, B, S, H, Hkv, HD, **kw)
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT if impl == "tc_split" else mt.ATTN_BWD_FUSED)
+    try:
+        bwd(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(), dvec.data_ptr(), dqa.data_ptr(),
+            H * HD, dp, ld, dp + 2 * H * HD, dp + 2 * (H + Hkv) * HD, ld, B, S, H, Hkv, HD, **kw)
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
     torch.cuda.synchronize()
     assert err.item() == 0
 

@@ -199,7 +199,7 @@ def _attn_inputs(hd, H, Hkv, s, b, seed):
 def test_attention_fwd(hd, H, Hkv, s, b, impl):
     """tc: the tcgen05 forward with one query tile per CTA; tc_pingpong: two
     tiles per CTA in ping-pong (head dim 128, selected explicitly: the
-    automatic choice takes it only from 8192 tokens on)."""
+    automatic choice takes it only above 8192 tokens)."""
     mt = _mt()
     if impl == "tc_pingpong" and hd != 128:
         pytest.skip("the two-tile forward is for head dim 128")
@@ -228,12 +228,71 @@ def test_attention_fwd(hd, H, Hkv, s, b, impl):
     assert np.allclose(np64(lse), oracle.attention_lse(q, k), rtol=1e-4, atol=1e-4)
 
 
-@pytest.mark.parametrize("impl", ["mma", "tc"])
+def _bwd_form(mt, impl):
+    """The tensor-core backward's form for impl: tc (fused dQ reductions) or
+    tc_split (dK/dV key-major, dQ query-major, deterministic)."""
+    return mt.ATTN_BWD_SPLIT if impl == "tc_split" else mt.ATTN_BWD_FUSED
+
+
+@pytest.mark.parametrize("impl", ["mma", "tc", "tc_split"])
 @pytest.mark.parametrize("hd,H,Hkv,s,b", ATTN)
 def test_attention_bwd(hd, H, Hkv, s, b, impl):
-    if impl == "tc" and hd != 128:
+    if impl != "mma" and hd != 128:
         pytest.skip("tensor-core backward is for head_dim 128")
     mt = _mt()
+    if impl != "mma":
+        was = mt.mt_k_attn_bwd_variant(_bwd_form(mt, impl))
+        try:
+            _attention_bwd_case(mt, hd, H, Hkv, s, b, impl)
+        finally:
+            mt.mt_k_attn_bwd_variant(was)
+    else:
+        _attention_bwd_case(mt, hd, H, Hkv, s, b, impl)
+
+
+def test_split_attention_backward_is_bitwise_reproducible():
+    """The split form sums each dQ element in one fixed order (the query-major
+    kernel's key-block loop) and dK, dV in tensor memory: two runs on the same
+    inputs give the same bits, at a shape with many key blocks per query
+    block and GQA."""
+    mt = _mt()
+    hd, H, Hkv, s, b = 128, 8, 2, 1100, 2
+    qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, 3)
+    T = b * s
+    do = bf(np.random.default_rng(4).normal(size=(T, H * hd)))
+    o = torch.empty(T, H * hd, dtype=torch.bfloat16, device=DEV)
+    lse = torch.empty(b, H, s, device=DEV)
+    p = qkv.data_ptr()
+    pk, pv = p + 2 * H * hd, p + 2 * (H + Hkv) * hd
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    mt.mt_k_attn_fwd_tc(p, pk, pv, ld, o.data_ptr(), H * hd, lse.data_ptr(), b, s, H, Hkv, hd, 0, err.data_ptr())
+    outs = []
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT)
+    try:
+        for _ in range(2):
+            dvec = torch.empty(b, H, s, device=DEV)
+            dqa = torch.full((T, H * hd), float("nan"), device=DEV)  # every element must be written
+            dqkv = torch.zeros(T, ld, dtype=torch.bfloat16, device=DEV)
+            dp = dqkv.data_ptr()
+            mt.mt_k_attn_bwd_tc(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(), dvec.data_ptr(),
+                                dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd, dp + 2 * (H + Hkv) * hd, ld, b, s, H,
+                                Hkv, hd, dev_err=err.data_ptr())
+            sync()
+            outs.append((dqkv.cpu().clone(), dqa.cpu().clone()))
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
+    assert err.item() == 0
+    assert torch.isfinite(outs[0][1]).all()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    ro, P = oracle.attention_fwd(q, k, v)
+    rdq, rdk, rdv = oracle.attention_bwd(q, k, v, P, np64(do).reshape(b, s, H, hd))
+    g = outs[0][0].double().numpy()
+    assert rel_l2(g[:, :H * hd].reshape(b, s, H, hd), rdq) < 1e-2
+    assert rel_l2(g[:, H * hd:(H + Hkv) * hd].reshape(b, s, Hkv, hd), rdk) < 1e-2
+    assert rel_l2(g[:, (H + Hkv) * hd:].reshape(b, s, Hkv, hd), rdv) < 1e-2
+
+
+def _attention_bwd_case(mt, hd, H, Hkv, s, b, impl):
     qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, 7 * hd + s)
     T = b * s
     rng = np.random.default_rng(s)
@@ -308,14 +367,22 @@ def _qkv_rope_case(mt, hd, H, Hkv, s, b):
     assert np.all(np.abs(got - ref) <= bound)
 
 
-@pytest.mark.parametrize("impl", ["mma", "tc"])
+@pytest.mark.parametrize("impl", ["mma", "tc", "tc_split"])
 @pytest.mark.parametrize("hd,H,Hkv,s,b", [(64, 4, 4, 128, 2), (128, 4, 2, 100, 3), (128, 2, 1, 300, 2)])
 def test_attention_bwd_returns_pre_rope_gradients(hd, H, Hkv, s, b, impl):
-    if impl == "tc" and hd != 128:
-        pytest.skip("tensor-core backward is for head_dim 128")
     """With the RoPE tables the backward returns dL/d(pre-RoPE q, k): the
     oracle's attention backward followed by its rope_bwd."""
+    if impl != "mma" and hd != 128:
+        pytest.skip("tensor-core backward is for head_dim 128")
     mt = _mt()
+    was = mt.mt_k_attn_bwd_variant(_bwd_form(mt, impl))
+    try:
+        _pre_rope_case(mt, hd, H, Hkv, s, b, impl)
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
+
+
+def _pre_rope_case(mt, hd, H, Hkv, s, b, impl):
     qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, 11 * hd + s)
     T = b * s
     rng = np.random.default_rng(5 * s)

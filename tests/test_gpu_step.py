@@ -130,6 +130,29 @@ def test_serialized_and_no_update_modes():
     assert max(rel(Gn[k], Gb[k]) for k in Gb) <= 1e-3
 
 
+def test_split_attention_backward_makes_steps_bitwise_reproducible():
+    """With the split attention backward no reduction of the step depends on
+    timing: the GEMMs have no split-K, the normalisation, embedding and
+    loss reductions run in a fixed order, and dQ is summed in the query-major
+    kernel. Two pipelined runs and a serialized run (one stream) of two steps
+    then give the same bits: losses, every gradient and the updated master."""
+    arena, mt = _libs()
+    shape = SHAPES["hd128"]
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT)
+    try:
+        runs = [run_gpu(shape, 2), run_gpu(shape, 2), run_gpu(shape, 2, flags=mt.MT_FLAG_SERIALIZE)]
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
+    ref = runs[0]
+    for other in runs[1:]:
+        for a, b in zip(ref, other):
+            assert a["loss"] == b["loss"]
+            assert np.array_equal(a["G"], b["G"])
+            assert np.array_equal(a["P"], b["P"])
+    r = oracle_steps(shape, 1)[0]
+    assert abs(ref[0]["loss"] - r["loss"]) <= 1e-2
+
+
 def test_bad_tokens_rejected_before_device_work():
     arena, mt = _libs()
     shape = SHAPES["tiny"]
@@ -228,35 +251,49 @@ def test_offloaded_activations_give_the_resident_result(name, shape, flags, extr
     MT_FLAG_STASH_ATTN: the recompute takes the forward's attention output and
     log-sum-exp instead of running the attention again; the forward is
     deterministic, so they are the recompute's. Either way (and both), two
-    steps match the plain run (first loss to 1e-5, every gradient and the
-    updated master to the run-to-run noise of the attention's dQ reductions),
-    and the first step's loss and gradients match the oracle."""
+    steps match the plain run: bit for bit at head dim 128 (the split
+    attention backward leaves no order noise), else the first loss to 1e-5,
+    every gradient and the updated master to the run-to-run noise of the
+    attention's dQ reductions; the first step's loss and gradients match the
+    oracle."""
     from host_memory_streamed_layer_b200 import arena, mt
     c = oracle.OracleConfig(**shape)
     runs = {}
     var = (mt.MT_FLAG_OFFLOAD_ACTS if "offload" in extra else 0) | (mt.MT_FLAG_STASH_ATTN if "stash" in extra else 0)
-    for off in (0, var):
-        cfg = arena.config(shape)
-        cfg.flags = flags | off
-        cfg.host_threads = 4
-        A = arena.pack(cfg, synth.init_weights(shape, 0))
-        ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
-        out = []
-        try:
-            for step in range(2):
-                tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, step)
-                loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
-                G = None
-                if not flags & mt.MT_FLAG_GRAD_RING:
-                    G = np.empty_like(A)
-                    mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
-                out.append((loss, G))
-            mt.mt_flush(ctx)
-            st = mt.mt_get_stats(ctx)
-        finally:
-            mt.mt_destroy(ctx)
-        runs[off] = (out, A.copy(), st)
+    # Head dim 128 runs the deterministic split attention backward: with no
+    # order noise left the two runs must agree bit for bit. (Head dim 64 has
+    # only the reduction-based backward.)
+    exact = shape["d"] // shape["H"] == 128
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT if exact else mt.ATTN_BWD_AUTO)
+    try:
+        for off in (0, var):
+            cfg = arena.config(shape)
+            cfg.flags = flags | off
+            cfg.host_threads = 4
+            A = arena.pack(cfg, synth.init_weights(shape, 0))
+            ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+            out = []
+            try:
+                for step in range(2):
+                    tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, step)
+                    loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+                    G = None
+                    if not flags & mt.MT_FLAG_GRAD_RING:
+                        G = np.empty_like(A)
+                        mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
+                    out.append((loss, G))
+                mt.mt_flush(ctx)
+                st = mt.mt_get_stats(ctx)
+            finally:
+                mt.mt_destroy(ctx)
+            runs[off] = (out, A.copy(), st)
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
     res, off = runs[0], runs[var]
+    if exact:
+        for (la, Ga), (lb, Gb) in zip(res[0], off[0]):
+            assert la == lb and (Ga is None or np.array_equal(Ga, Gb))
+        assert np.array_equal(off[1], res[1])
     for step, ((la, Ga), (lb, Gb)) in enumerate(zip(res[0], off[0])):
         # the first forward is deterministic; the second runs on weights that
         # carry the dQ reductions' order noise through one Adam step (at
