@@ -31,6 +31,7 @@
 #include <chrono>
 #include <condition_variable>
 #include <deque>
+#include <functional>
 #include <mutex>
 #include <string>
 #include <thread>
@@ -207,6 +208,20 @@ struct mt_ctx {
   int32_t* d_uid = nullptr;       // unique token ids of the step, [T]
   float* emb_own_h = nullptr;     // pinned: this rank's rows of the mean embedding gradient
   cudaEvent_t ev_embw = nullptr;  // embedding table all-gathered
+
+  // ---- mixture-of-experts layers (E > 0) ----
+  // Routing of layer l, taken in its forward and reused by its recompute:
+  // slot_of[t k + j] (the routed row of token t's j-th expert) and row_of[slot]
+  // (the token of a routed row) on the device per layer, and each expert's
+  // row count on the host (the expert GEMMs' sizes).
+  float *moe_logits = nullptr, *moe_gate = nullptr, *moe_dgate = nullptr, *moe_dlogits = nullptr;
+  int32_t *moe_idx = nullptr, *moe_slot = nullptr, *moe_row = nullptr;
+  uint16_t *xe_b = nullptr, *dye_b = nullptr;
+  float *ye = nullptr, *dxe = nullptr;
+  int32_t* moe_idx_h = nullptr;    // pinned: per layer the experts each token chose [T k]
+  int32_t* moe_route_h = nullptr;  // pinned: per layer slot_of | row_of [2 T k]
+  std::vector<std::vector<int>> moe_count;  // [L][E]
+  cudaEvent_t ev_route = nullptr;
 };
 
 namespace mteng {
@@ -421,6 +436,134 @@ float* lse_of(mt_ctx* c, int l) {
 // attention, whose output the forward sweep kept (the forward is
 // deterministic: the kept O and LSE are the ones a recompute would produce).
 // ---------------------------------------------------------------------------
+// ---------------------------------------------------------------------------
+// Mixture-of-experts MLP of layer l from the bf16 MLP input w_b (expert
+// weights in the slot W). Routed rows are grouped by expert, tokens in
+// increasing order within an expert, so every expert product is one GEMM on
+// a contiguous block of rows. The forward sweep takes the routing: the
+// experts each token chose go to the host, which lays out the rows and keeps
+// each expert's row count (the GEMMs' sizes); the recompute reruns the router
+// (the same choices: the forward is deterministic) and reuses that layout.
+// ---------------------------------------------------------------------------
+bool wait_event(mt_ctx* c, cudaEvent_t e);
+
+void moe_dispatch(const int32_t* idx, int T, int k, int E, int32_t* slot_of, int32_t* row_of, std::vector<int>& cnt) {
+  std::fill(cnt.begin(), cnt.end(), 0);
+  const int Tk = T * k;
+  for (int p = 0; p < Tk; ++p) cnt[idx[p]]++;
+  std::vector<int> next(E, 0);
+  for (int e = 1; e < E; ++e) next[e] = next[e - 1] + cnt[e - 1];
+  for (int p = 0; p < Tk; ++p) {
+    const int sl = next[idx[p]]++;
+    slot_of[p] = sl;
+    row_of[sl] = p / k;
+  }
+}
+
+int moe_fwd(mt_ctx* c, int l, const uint16_t* W, float* xo) {
+  const Shapes& s = c->lay.sh;
+  const Layout& y = c->lay;
+  const int T = s.T, d = s.d, F = s.F, E = s.E, k = s.topk, Tk = T * k;
+  cudaStream_t st = c->s_comp;
+  const uint16_t* Wg = W + y.bf_gu;
+  const uint16_t* Wu = Wg + (size_t)E * F * d;
+  const uint16_t* Wd = W + y.bf_d;
+  int32_t* slot_of = c->moe_slot + (size_t)l * Tk;
+  int32_t* row_of = c->moe_row + (size_t)l * Tk;
+  KL(launch_moe_router(c->w_b, W + y.bf_r, T, d, E, k, c->moe_logits, c->moe_idx, c->moe_gate, st), 1);
+  if (xo) {
+    int32_t* ih = c->moe_idx_h + (size_t)l * Tk;
+    CK(cudaMemcpyAsync(ih, c->moe_idx, (size_t)Tk * 4, cudaMemcpyDeviceToHost, st));
+    CK(cudaEventRecord(c->ev_route, st));
+    if (!wait_event(c, c->ev_route)) return set_err(c, MT_ERR_TIMEOUT, "routing did not arrive within the wait limit");
+    for (int p = 0; p < Tk; ++p)
+      if (ih[p] < 0 || ih[p] >= E) return set_err(c, MT_ERR_DEVICE, "router chose no valid expert");
+    int32_t* hs = c->moe_route_h + (size_t)l * 2 * Tk;
+    moe_dispatch(ih, T, k, E, hs, hs + Tk, c->moe_count[l]);
+    CK(cudaMemcpyAsync(slot_of, hs, (size_t)Tk * 4, cudaMemcpyHostToDevice, st));
+    CK(cudaMemcpyAsync(row_of, hs + Tk, (size_t)Tk * 4, cudaMemcpyHostToDevice, st));
+  }
+  KL(launch_moe_gather(c->w_b, row_of, Tk, d, c->xe_b, st), 1);
+  const std::vector<int>& cnt = c->moe_count[l];
+  size_t off = 0;
+  for (int e = 0; e < E; ++e) {
+    const int n = cnt[e];
+    if (n == 0) continue;
+    // gate and up of expert e into the [rows, 2F] buffer's two halves
+    CKM(gemm(c, gd_fwd(c->xe_b + off * d, d, Wg + (size_t)e * F * d, d, c->gu_b + off * 2 * F, 2 * F, EPI_BF16,
+                       nullptr, n, F, d)));
+    CKM(gemm(c, gd_fwd(c->xe_b + off * d, d, Wu + (size_t)e * F * d, d, c->gu_b + off * 2 * F + F, 2 * F,
+                       EPI_BF16, nullptr, n, F, d)));
+    off += n;
+  }
+  KL(launch_swiglu_fwd(c->gu_b, c->act_b, Tk, F, st), 1);
+  off = 0;
+  for (int e = 0; e < E; ++e) {
+    const int n = cnt[e];
+    if (n == 0) continue;
+    CKM(gemm(c, gd_fwd(c->act_b + off * F, F, Wd + (size_t)e * d * F, F, c->ye + off * d, d, EPI_F32, nullptr, n, d,
+                       F)));
+    off += n;
+  }
+  if (xo) KL(launch_moe_combine(c->h_f, c->ye, slot_of, c->moe_gate, T, k, d, xo, st), 1);
+  return MT_OK;
+}
+
+// Backward of moe_fwd from gin = dL/d(MLP output): the expert, gate and router
+// weight gradients of layer l into Gw (the layer's gradient block at the
+// given tensor ids) and dL/dw (fp32) into c->tmp_f. An expert no token chose
+// gets zero gradients.
+int moe_bwd(mt_ctx* c, int l, const uint16_t* W, const float* gin, const std::function<float*(int)>& G) {
+  const Shapes& s = c->lay.sh;
+  const Layout& y = c->lay;
+  const int T = s.T, d = s.d, F = s.F, E = s.E, k = s.topk, Tk = T * k;
+  cudaStream_t st = c->s_comp;
+  const uint16_t* Wg = W + y.bf_gu;
+  const uint16_t* Wu = Wg + (size_t)E * F * d;
+  const uint16_t* Wd = W + y.bf_d;
+  const int32_t* slot_of = c->moe_slot + (size_t)l * Tk;
+  const std::vector<int>& cnt = c->moe_count[l];
+  KL(launch_moe_dy(gin, c->ye, slot_of, c->moe_gate, T, k, d, c->dye_b, c->moe_dgate, st), 1);
+  size_t off = 0;
+  for (int e = 0; e < E; ++e) {
+    const int n = cnt[e];
+    float* gWd = G(MT_T_WDOWN) + (size_t)e * d * F;
+    if (n == 0) {
+      CK(cudaMemsetAsync(gWd, 0, (size_t)d * F * 4, st));
+      continue;
+    }
+    CKM(gemm(c, gd_dw(c->dye_b + off * d, d, c->act_b + off * F, F, gWd, F, EPI_F32, d, F, n)));
+    CKM(gemm(c, gd_dx(c->dye_b + off * d, d, Wd + (size_t)e * d * F, F, c->dact_b + off * F, F, EPI_BF16, n, F, d)));
+    off += n;
+  }
+  KL(launch_swiglu_bwd(c->gu_b, c->dact_b, c->dgu_b, Tk, F, st), 1);
+  off = 0;
+  for (int e = 0; e < E; ++e) {
+    const int n = cnt[e];
+    float* gWg = G(MT_T_WGATE) + (size_t)e * F * d;
+    float* gWu = G(MT_T_WUP) + (size_t)e * F * d;
+    if (n == 0) {
+      CK(cudaMemsetAsync(gWg, 0, (size_t)F * d * 4, st));
+      CK(cudaMemsetAsync(gWu, 0, (size_t)F * d * 4, st));
+      continue;
+    }
+    const uint16_t* dg = c->dgu_b + off * 2 * F;
+    CKM(gemm(c, gd_dw(dg, 2 * F, c->xe_b + off * d, d, gWg, d, EPI_F32, F, d, n)));
+    CKM(gemm(c, gd_dw(dg + F, 2 * F, c->xe_b + off * d, d, gWu, d, EPI_F32, F, d, n)));
+    float* dx = c->dxe + off * d;
+    CKM(gemm(c, gd_dx(dg, 2 * F, Wg + (size_t)e * F * d, d, dx, d, EPI_F32, n, d, F)));
+    GemmDesc gu = gd_dx(dg + F, 2 * F, Wu + (size_t)e * F * d, d, dx, d, EPI_F32_ADD, n, d, F);
+    gu.R = dx;
+    gu.ldr = d;
+    CKM(gemm(c, gu));
+    off += n;
+  }
+  KL(launch_moe_router_bwd(c->moe_gate, c->moe_dgate, c->moe_idx, c->w_b, W + y.bf_r, c->dxe, slot_of, T, k, d, E,
+                           c->moe_dlogits, G(MT_T_ROUTER), c->tmp_f, st),
+     3);
+  return MT_OK;
+}
+
 int layer_fwd(mt_ctx* c, int l, int slot, const float* x, float* xo) {
   const Shapes& s = c->lay.sh;
   const Layout& y = c->lay;
@@ -450,6 +593,7 @@ int layer_fwd(mt_ctx* c, int l, int slot, const float* x, float* xo) {
   if (xo || !stash_attn(c)) CKM(attn(c, a, false));
   CKM(gemm(c, gd_fwd(ao_of(c, l), s.Hd, W + y.bf_o, s.Hd, c->h_f, s.d, EPI_F32_ADD, x, s.T, s.d, s.Hd)));
   KL(launch_rmsnorm_fwd(c->h_f, W + y.bf_g2, c->w_b, c->r2, s.T, s.d, c->cfg.norm_eps, st), 1);
+  if (s.E > 0) return moe_fwd(c, l, W, xo);
   CKM(gemm(c, gd_fwd(c->w_b, s.d, W + y.bf_gu, s.d, c->gu_b, 2 * s.F, EPI_BF16, nullptr, s.T, 2 * s.F, s.d)));
   KL(launch_swiglu_fwd(c->gu_b, c->act_b, s.T, s.F, st), 1);
   if (xo) CKM(gemm(c, gd_fwd(c->act_b, s.F, W + y.bf_d, s.F, xo, s.d, EPI_F32_ADD, c->h_f, s.T, s.d, s.F)));
@@ -468,14 +612,18 @@ int layer_bwd(mt_ctx* c, int l, int slot, const float* x, float* gs, const float
   cudaStream_t st = c->s_comp;
   const int T = s.T, d = s.d, F = s.F;
 
-  KL(launch_cast_f32_bf16(gin, c->gxb, (int64_t)T * d, st), 1);
-  // down projection
-  CKM(gemm(c, gd_dw(c->gxb, d, c->act_b, F, G(MT_T_WDOWN), F, EPI_F32, d, F, T)));
-  CKM(gemm(c, gd_dx(c->gxb, d, W + y.bf_d, F, c->dact_b, F, EPI_BF16, T, F, d)));
-  KL(launch_swiglu_bwd(c->gu_b, c->dact_b, c->dgu_b, T, F, st), 1);
-  // gate/up projections
-  CKM(gemm(c, gd_dw(c->dgu_b, 2 * F, c->w_b, d, G(MT_T_WGATE), d, EPI_F32, 2 * F, d, T)));
-  CKM(gemm(c, gd_dx(c->dgu_b, 2 * F, W + y.bf_gu, d, c->tmp_f, d, EPI_F32, T, d, 2 * F)));
+  if (s.E > 0) {
+    CKM(moe_bwd(c, l, W, gin, G));
+  } else {
+    KL(launch_cast_f32_bf16(gin, c->gxb, (int64_t)T * d, st), 1);
+    // down projection
+    CKM(gemm(c, gd_dw(c->gxb, d, c->act_b, F, G(MT_T_WDOWN), F, EPI_F32, d, F, T)));
+    CKM(gemm(c, gd_dx(c->gxb, d, W + y.bf_d, F, c->dact_b, F, EPI_BF16, T, F, d)));
+    KL(launch_swiglu_bwd(c->gu_b, c->dact_b, c->dgu_b, T, F, st), 1);
+    // gate/up projections
+    CKM(gemm(c, gd_dw(c->dgu_b, 2 * F, c->w_b, d, G(MT_T_WGATE), d, EPI_F32, 2 * F, d, T)));
+    CKM(gemm(c, gd_dx(c->dgu_b, 2 * F, W + y.bf_gu, d, c->tmp_f, d, EPI_F32, T, d, 2 * F)));
+  }
   KL(launch_rmsnorm_bwd(c->h_f, W + y.bf_g2, c->r2, c->tmp_f, gin, c->dh_f, c->dhb, c->rms_part, G(MT_T_MLP_NORM),
                         T, d, st),
      2);
@@ -1307,13 +1455,27 @@ size_t device_bytes(const Layout& y, int Tc, uint32_t flags, const mt_shard* pla
   add(T * 4);                                               // r1
   add(T * 4);                                               // r2
   add(T * d * 2);                                           // w
-  add(T * 2 * F * 2);                                       // gate|up
-  add(T * F * 2);                                           // act
+  const size_t R = s.E > 0 ? std::max(T, T * (size_t)s.topk) : T;  // MLP rows (routed rows with experts)
+  add(R * 2 * F * 2);                                       // gate|up
+  add(R * F * 2);                                           // act
   add(T * d * 4);                                           // gx0
   add(T * d * 4);                                           // gx1
   add(T * d * 2);                                           // gxb
-  add(T * F * 2);                                           // dact
-  add(T * 2 * F * 2);                                       // dgu
+  add(R * F * 2);                                           // dact
+  add(R * 2 * F * 2);                                       // dgu
+  if (s.E > 0) {
+    const size_t Tk = T * (size_t)s.topk, E = s.E;
+    add(T * E * 4);                  // logits
+    add(T * E * 4);                  // dlogits
+    add(Tk * 4);                     // idx
+    add(Tk * 4);                     // gate
+    add(Tk * 4);                     // dgate
+    add((size_t)s.L * Tk * 4 * 2);   // slot_of, row_of per layer
+    add(Tk * d * 2);                 // xe
+    add(Tk * d * 2);                 // dye
+    add(Tk * d * 4);                 // ye
+    add(Tk * d * 4);                 // dxe
+  }
   add(T * d * 4);                                           // tmp_f
   add(T * d * 4);                                           // dh
   add(T * d * 2);                                           // dhb
@@ -1382,6 +1544,7 @@ void free_all(mt_ctx* c) {
                         c->ev_step_start, c->ev_fwd_end, c->ev_head_end, c->ev_bwd_end, c->ev_step_end})
     if (e) cudaEventDestroy(e);
   if (c->ev_embw) cudaEventDestroy(c->ev_embw);
+  if (c->ev_route) cudaEventDestroy(c->ev_route);
   if (c->comm_h2d) c->nccl->CommDestroy(c->comm_h2d);
   if (c->comm_comp) c->nccl->CommDestroy(c->comm_comp);
   // In serialized mode the three handles are one stream: destroy each once.
@@ -1393,7 +1556,8 @@ void free_all(mt_ctx* c) {
   for (void* p : {(void*)c->grad, (void*)c->ring, (void*)c->defer_g, (void*)(c->grad_head_owned ? c->grad_head : nullptr),
                   (void*)c->bf_layers,
                   (void*)c->bf_embed, (void*)c->bf_head, (void*)c->emb_rows_h, (void*)c->stage_i, (void*)c->flags_h,
-                  (void*)c->misc_h, (void*)c->xh, (void*)c->emb_own_h})
+                  (void*)c->misc_h, (void*)c->xh, (void*)c->emb_own_h, (void*)c->moe_idx_h,
+                  (void*)c->moe_route_h})
     if (p) cudaFreeHost(p);
   free(c->m);
   free(c->v);
@@ -1416,7 +1580,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   const Shapes& s = y.sh;
   mt_shard plan{};
   const NcclApi* nccl = nullptr;
-  if (cfg->E > 0) return set_err(nullptr, MT_ERR_CONFIG, "expert layers are not on the engine's path");
+  if (cfg->E > 0 && world > 0) return set_err(nullptr, MT_ERR_CONFIG, "expert layers are not sharded");
   if (world > 0) {
     if (!id) return set_err(nullptr, MT_ERR_ARG, "sharded context without an NCCL id");
     if (cfg->flags & (MT_FLAG_DEFER_UPDATES | MT_FLAG_TIED_EMBED | MT_FLAG_BF16_GRADS))
@@ -1529,6 +1693,15 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
       cudaHostAlloc(reinterpret_cast<void**>(&c->emb_own_h),
                     std::max<size_t>(1, embed_rows_chunk(plan, s.V)) * s.d * 4, cudaHostAllocPortable) != cudaSuccess)
     return fail(MT_ERR_PIN, "pinned embedding-row allocation failed");
+  if (s.E > 0) {
+    const size_t Tk = (size_t)s.T * s.topk;
+    if (cudaHostAlloc(reinterpret_cast<void**>(&c->moe_idx_h), (size_t)s.L * Tk * 4, cudaHostAllocPortable) !=
+            cudaSuccess ||
+        cudaHostAlloc(reinterpret_cast<void**>(&c->moe_route_h), (size_t)s.L * Tk * 2 * 4, cudaHostAllocPortable) !=
+            cudaSuccess)
+      return fail(MT_ERR_PIN, "pinned routing allocation failed");
+    c->moe_count.assign(s.L, std::vector<int>(s.E, 0));
+  }
   if ((cfg->flags & MT_FLAG_OFFLOAD_ACTS) && s.L >= 3 &&
       cudaHostAlloc(reinterpret_cast<void**>(&c->xh), (size_t)(s.L - 2) * s.T * s.d * 4, cudaHostAllocPortable) !=
           cudaSuccess)
@@ -1634,13 +1807,28 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->r1 = (float*)carve(T * 4);
   c->r2 = (float*)carve(T * 4);
   c->w_b = (uint16_t*)carve(T * d * 2);
-  c->gu_b = (uint16_t*)carve(T * 2 * F * 2);
-  c->act_b = (uint16_t*)carve(T * F * 2);
+  const size_t R = s.E > 0 ? std::max(T, T * (size_t)s.topk) : T;
+  c->gu_b = (uint16_t*)carve(R * 2 * F * 2);
+  c->act_b = (uint16_t*)carve(R * F * 2);
   c->gx0 = (float*)carve(T * d * 4);
   c->gx1 = (float*)carve(T * d * 4);
   c->gxb = (uint16_t*)carve(T * d * 2);
-  c->dact_b = (uint16_t*)carve(T * F * 2);
-  c->dgu_b = (uint16_t*)carve(T * 2 * F * 2);
+  c->dact_b = (uint16_t*)carve(R * F * 2);
+  c->dgu_b = (uint16_t*)carve(R * 2 * F * 2);
+  if (s.E > 0) {
+    const size_t Tk = T * (size_t)s.topk, E = s.E;
+    c->moe_logits = (float*)carve(T * E * 4);
+    c->moe_dlogits = (float*)carve(T * E * 4);
+    c->moe_idx = (int32_t*)carve(Tk * 4);
+    c->moe_gate = (float*)carve(Tk * 4);
+    c->moe_dgate = (float*)carve(Tk * 4);
+    c->moe_slot = (int32_t*)carve((size_t)s.L * Tk * 4 * 2);
+    c->moe_row = c->moe_slot + (size_t)s.L * Tk;
+    c->xe_b = (uint16_t*)carve(Tk * d * 2);
+    c->dye_b = (uint16_t*)carve(Tk * d * 2);
+    c->ye = (float*)carve(Tk * d * 4);
+    c->dxe = (float*)carve(Tk * d * 4);
+  }
   c->tmp_f = (float*)carve(T * d * 4);
   c->dh_f = (float*)carve(T * d * 4);
   c->dhb = (uint16_t*)carve(T * d * 2);
@@ -1712,6 +1900,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
                          &c->ev_step_start, &c->ev_fwd_end, &c->ev_head_end, &c->ev_bwd_end, &c->ev_step_end})
     ok = ok && cudaEventCreate(e) == cudaSuccess;
   if (!ok) return fail(MT_ERR_CUDA, "event creation failed");
+  if (s.E > 0 && cudaEventCreateWithFlags(&c->ev_route, cudaEventDisableTiming) != cudaSuccess)
+    return fail(MT_ERR_CUDA, "event creation failed");
   if (world > 0) {
     // Every rank joins here (NCCL's initialisation is collective); then the
     // table the first step gathers from: the same bf16 copy on every rank.
@@ -1770,6 +1960,17 @@ extern "C" int mt_create_sharded(const mt_config* cfg, float* host_param_arena, 
   g_create_error.clear();
   if (world < 1 || rank < 0 || rank >= world) return set_err(nullptr, MT_ERR_ARG, "rank outside [0, world)");
   return create_impl(cfg, host_param_arena, arena_bytes, out, world, rank, id);
+}
+
+extern "C" int mt_get_routing(mt_ctx* c, int layer, int32_t* idx, size_t n) {
+  if (!c) return MT_ERR_ARG;
+  const Shapes& s = c->lay.sh;
+  if (s.E == 0) return set_err(c, MT_ERR_CONFIG, "no expert layers");
+  if (layer < 0 || layer >= s.L || !idx) return set_err(c, MT_ERR_ARG, "layer outside [0, L) or NULL");
+  const size_t Tk = (size_t)s.T * s.topk;
+  if (n < Tk) return set_err(c, MT_ERR_ARG, "idx smaller than b*s*topk");
+  memcpy(idx, c->moe_idx_h + (size_t)layer * Tk, Tk * 4);
+  return MT_OK;
 }
 
 extern "C" size_t mt_device_bytes_sharded(const mt_config* cfg, int world) {

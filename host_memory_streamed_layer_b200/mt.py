@@ -423,6 +423,17 @@ def mt_device_bytes_sharded(cfg: mt_config, world: int) -> int:
     return lib.mt_device_bytes_sharded(ctypes.byref(cfg), world)
 
 
+_sig("mt_get_routing", c_int, c_void_p, c_int, c_void_p, c_size_t)
+
+
+def mt_get_routing(ctx: int, layer: int, T: int, topk: int):
+    """The experts each of the T tokens chose in `layer`'s last forward, [T, topk]."""
+    import numpy as np
+    out = np.empty((T, topk), dtype=np.int32)
+    _check(lib.mt_get_routing(ctx, layer, out.ctypes.data, out.size), "mt_get_routing", ctx)
+    return out
+
+
 def mt_inject_host_stall(ctx: int, stream: int, ms: int):
     """Test aid: a host function sleeping ms milliseconds on one of the
     context's streams (0 prefetch, 1 compute, 2 offload)."""

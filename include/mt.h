@@ -332,6 +332,15 @@ int mt_create_sharded(const mt_config* cfg, float* host_param_arena, size_t aren
  * gradient, [world * ceil(V / world), d] each. 0 for a bad cfg or world. */
 size_t mt_device_bytes_sharded(const mt_config* cfg, int world);
 
+/* The experts each token chose in layer `layer`'s forward of the last step
+ * (mixture-of-experts layers, MT_T_ROUTER): idx[t * topk + j], t in [0, b*s)
+ * sequence-major, j in [0, topk) largest logit first. n counts int32
+ * elements (at least b*s*topk). The routing a forward took is the one its
+ * backward used, so a test can hand it to an independent model where two
+ * logits lie within rounding of each other. MT_ERR_CONFIG without experts,
+ * MT_ERR_ARG for a bad layer, NULL or short buffer. Host-side. */
+int mt_get_routing(mt_ctx* ctx, int layer, int32_t* idx, size_t n);
+
 /* One training step: tokens and labels are host int32 arrays of b*s ids in
  * [0, V), sequence-major. Runs forward, loss, backward and the host AdamW
  * update (bias correction from step 1), and writes the mean next-token

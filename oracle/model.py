@@ -510,11 +510,12 @@ def head_ce_fwd_bwd(xL, gf, Whead, labels, eps):
 # ---------------------------------------------------------------------------
 
 def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
-                     c: OracleConfig, routing=None):
+                     c: OracleConfig, routing=None, logits_out=None):
     """weights: dict (layer, tensor id) -> float64 array, the values the forward
     and backward use. tokens, labels: int [b, s]. routing: optional dict
     layer -> [b*s, k] expert choice (mixture-of-experts layers), else each
-    router's own. Returns (loss, grads dict)."""
+    router's own; logits_out: optional dict that receives each expert layer's
+    router logits [b*s, E]. Returns (loss, grads dict)."""
     b, s = tokens.shape
     T = b * s
     cos, sin = rope_tables(s, c.hd, c.rope_base)
@@ -525,6 +526,8 @@ def train_step_grads(weights: dict, tokens: np.ndarray, labels: np.ndarray,
         W = {tid: weights[(l, tid)] for tid in c.layer_tids}
         x, cache = layer_fwd(x, W, c, cos, sin, routing=(routing or {}).get(l))
         caches.append(cache)
+        if c.E and logits_out is not None:
+            logits_out[l] = cache["moe"]["logits"]
     Whead = E if c.tied else weights[(-1, LM_HEAD)]
     loss, dx, dgf, dWhead = head_ce_fwd_bwd(
         x.reshape(T, c.d), weights[(-1, FINAL_NORM)], Whead, labels.reshape(T), c.norm_eps)

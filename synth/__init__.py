@@ -31,6 +31,7 @@ HYPER = dict(norm_eps=1e-5, rope_base=10000.0, lr=1e-3, beta1=0.9, beta2=0.95,
 
 # Tensor ids used to key the weight streams. Per decoder layer:
 ATTN_NORM, WQ, WK, WV, WO, MLP_NORM, WGATE, WUP, WDOWN = range(9)
+ROUTER = 9  # mixture-of-experts layers
 # Model-level tensors use layer = -1:
 EMBED, FINAL_NORM, LM_HEAD = 100, 101, 102
 
@@ -58,8 +59,11 @@ def init_tensor(seed: int, layer: int, tid: int, shape) -> np.ndarray:
     return (rng.standard_normal(size=shape, dtype=np.float32) * np.float32(INIT_STD))
 
 
-def layer_shapes(d: int, H: int, Hkv: int, F: int, hd: int):
-    """(tensor id, shape) of one decoder layer, weights stored [out, in]."""
+def layer_shapes(d: int, H: int, Hkv: int, F: int, hd: int, E: int = 0):
+    """(tensor id, shape) of one decoder layer, weights stored [out, in]; with
+    E experts the MLP matrices are stacked per expert and a router follows."""
+    mlp = [(WGATE, (F, d)), (WUP, (F, d)), (WDOWN, (d, F))] if not E else \
+        [(WGATE, (E, F, d)), (WUP, (E, F, d)), (WDOWN, (E, d, F)), (ROUTER, (E, d))]
     return [
         (ATTN_NORM, (d,)),
         (WQ, (H * hd, d)),
@@ -67,10 +71,7 @@ def layer_shapes(d: int, H: int, Hkv: int, F: int, hd: int):
         (WV, (Hkv * hd, d)),
         (WO, (d, H * hd)),
         (MLP_NORM, (d,)),
-        (WGATE, (F, d)),
-        (WUP, (F, d)),
-        (WDOWN, (d, F)),
-    ]
+    ] + mlp
 
 
 def init_weights(cfg: dict, seed: int) -> dict:
@@ -79,7 +80,7 @@ def init_weights(cfg: dict, seed: int) -> dict:
     hd = d // H
     out = {(-1, EMBED): init_tensor(seed, -1, EMBED, (V, d))}
     for l in range(L):
-        for tid, shape in layer_shapes(d, H, Hkv, F, hd):
+        for tid, shape in layer_shapes(d, H, Hkv, F, hd, cfg.get("E", 0)):
             out[(l, tid)] = init_tensor(seed, l, tid, shape)
     out[(-1, FINAL_NORM)] = init_tensor(seed, -1, FINAL_NORM, (d,))
     if not cfg.get("tied", False):  # tied embeddings: the head is the embedding table
