@@ -398,3 +398,34 @@ def test_tied_embeddings_layout():
         mt.mt_shard_plan(cfg, 2, 0)
     cfg.flags = mt.MT_FLAG_TIED_EMBED | mt.MT_FLAG_BF16_GRADS
     assert mt.mt_arena_bytes(cfg) == 0
+
+
+def test_expert_layer_layout_matches_the_oracle():
+    """Expert layers (E > 0): the library's arena offsets and sizes are the
+    oracle's stacked-expert layout, the router exists only with experts, and
+    bad expert counts are refused; the bf16 layer block grows by the same
+    expert matrices (host state and device footprint follow)."""
+    import oracle
+    from host_memory_streamed_layer_b200 import arena, mt
+    sh = dict(L=3, d=256, H=2, Hkv=1, F=96, V=304, b=2, s=40, E=6, topk=2)
+    cfg = arena.config(sh)
+    layout, total = oracle.arena_layout(oracle.OracleConfig(**sh))
+    assert mt.mt_arena_bytes(cfg) == total * 4
+    for layer, tid, off, shape in layout:
+        assert mt.mt_tensor_offset(cfg, layer, tid) == (off, int(np.prod(shape)))
+    dense = arena.config(dict(sh, E=0))
+    with pytest.raises(mt.MTError):
+        mt.mt_tensor_offset(dense, 0, mt.MT_T_ROUTER)
+    for E, k in ((65, 1), (4, 0), (4, 5), (-1, 1)):
+        bad = arena.config(sh)
+        bad.E, bad.topk = E, k
+        assert mt.mt_arena_bytes(bad) == 0
+    per_layer = mt.mt_tensor_offset(cfg, 1, mt.MT_T_ATTN_NORM)[0] - mt.mt_tensor_offset(cfg, 0, mt.MT_T_ATTN_NORM)[0]
+    per_dense = (mt.mt_tensor_offset(dense, 1, mt.MT_T_ATTN_NORM)[0]
+                 - mt.mt_tensor_offset(dense, 0, mt.MT_T_ATTN_NORM)[0])
+    assert per_layer - per_dense == (6 - 1) * 3 * 96 * 256 + 6 * 256
+    assert mt.mt_host_state_bytes(cfg) > mt.mt_host_state_bytes(dense)
+    assert mt.mt_device_bytes(cfg) > mt.mt_device_bytes(dense)
+    with pytest.raises(mt.MTError) as e:  # expert layers are not partitioned
+        mt.mt_shard_plan(cfg, 2, 0)
+    assert e.value.code == -2
