@@ -126,8 +126,23 @@ def pick_workload(args, avail, world=1):
     return DEFAULT_ORDER[-1], "the smallest benchmark workload (none fits the host's free memory)"
 
 
+def mlp_active(sh):
+    """Matrix parameters a token runs through in one layer's MLP: the dense
+    SwiGLU, or topk experts' plus the router."""
+    E = sh.get("E", 0)
+    return 3 * sh["d"] * sh["F"] * (sh["topk"] if E else 1) + E * sh["d"]
+
+
+def recompute_skip(sh):
+    """Matrix parameters the recompute leaves out: the dense MLP's down
+    projection (the backward needs only its input); expert layers recompute
+    it (the gates' gradients need the experts' outputs)."""
+    return 0 if sh.get("E", 0) else sh["d"] * sh["F"]
+
+
 def workload_desc(name, sh):
-    return (f"{name}: {sh['L']} layers, d {sh['d']}, {sh['H']} heads ({sh['Hkv']} kv), SwiGLU {sh['F']}, "
+    experts = f", {sh['E']} experts top-{sh['topk']}" if sh.get("E", 0) else ""
+    return (f"{name}: {sh['L']} layers, d {sh['d']}, {sh['H']} heads ({sh['Hkv']} kv), SwiGLU {sh['F']}{experts}, "
             f"vocab {sh['V']}, {sh['b']} x {sh['s']} tokens per GPU; fp32 master + AdamW moments in host RAM, "
             f"bf16 weights streamed per layer")
 
@@ -140,10 +155,10 @@ def flops_per_step(sh, stash=False):
     L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
     hd = d // H
     T = b * s
-    Pm = d * (H + 2 * Hkv) * hd + d * H * hd + 3 * d * F
+    Pm = d * (H + 2 * Hkv) * hd + d * H * hd + mlp_active(sh)
     A = 2.0 * b * s * s * H * hd  # causal attention forward (QK^T and PV over the visible half)
     model = L * (6.0 * T * Pm + 3 * A) + 6.0 * T * V * d
-    executed = L * (2.0 * T * Pm + A) + (L - 1) * (2.0 * T * (Pm - d * F) + (0 if stash else A)) \
+    executed = L * (2.0 * T * Pm + A) + (L - 1) * (2.0 * T * (Pm - recompute_skip(sh)) + (0 if stash else A)) \
         + L * (4.0 * T * Pm + 2.5 * A) + 6.0 * T * V * d
     return model, executed
 
@@ -500,7 +515,9 @@ def defer_layers(sh):
 
 def layer_params(sh):
     hd = sh["d"] // sh["H"]
-    return sh["d"] * (sh["H"] + 2 * sh["Hkv"]) * hd + sh["d"] * sh["H"] * hd + 3 * sh["d"] * sh["F"] + 2 * sh["d"]
+    E = sh.get("E", 0)
+    mlp = (3 * sh["d"] * sh["F"] + sh["d"]) * E if E else 3 * sh["d"] * sh["F"]
+    return sh["d"] * (sh["H"] + 2 * sh["Hkv"]) * hd + sh["d"] * sh["H"] * hd + mlp + 2 * sh["d"]
 
 
 def head_params(sh):
@@ -513,10 +530,10 @@ def phase_flops(sh, stash=False):
     L, d, H, Hkv, F, V, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
     hd = d // H
     T = b * s
-    Pm = d * (H + 2 * Hkv) * hd + d * H * hd + 3 * d * F
+    Pm = d * (H + 2 * Hkv) * hd + d * H * hd + mlp_active(sh)
     A = 2.0 * b * s * s * H * hd
     fwd = L * (2.0 * T * Pm + A) + 6.0 * T * V * d
-    bwd = (L - 1) * (2.0 * T * (Pm - d * F) + (0 if stash else A)) + L * (4.0 * T * Pm + 2.5 * A)
+    bwd = (L - 1) * (2.0 * T * (Pm - recompute_skip(sh)) + (0 if stash else A)) + L * (4.0 * T * Pm + 2.5 * A)
     return fwd, bwd
 
 

@@ -23,6 +23,9 @@ WORKLOADS = {
     "llama-7b": dict(L=32, d=4096, H=32, Hkv=32, F=11008, V=32000, b=4, s=4096),
     "gqa-14b": dict(L=40, d=5120, H=40, Hkv=8, F=13824, V=152064, b=2, s=4096),
     "llama-7b-128k": dict(L=32, d=4096, H=32, Hkv=32, F=11008, V=32000, b=1, s=131072),
+    # mixture-of-experts decoder: 8 experts of SwiGLU width 1408, top-2 routing
+    # (2.2 B parameters, about 0.9 B active per token)
+    "moe-8x1408": dict(L=24, d=2048, H=16, Hkv=16, F=1408, V=32000, b=8, s=2048, E=8, topk=2),
 }
 
 # Hyper-parameters shared by every workload.
