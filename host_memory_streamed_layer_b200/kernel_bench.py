@@ -41,6 +41,8 @@ def step_gemms(sh):
     backward's input- and weight-gradient products per layer; the LM head per
     token chunk (chunks of at most ~4 GiB of fp32 logits + bf16 dz, multiples
     of 128 tokens)."""
+    if sh.get("E", 0):
+        raise ValueError("expert layers: their GEMM sizes follow the routing, not the shape")
     L, d, H, Hkv, Fh, Vh, b, s = (sh[k] for k in ("L", "d", "H", "Hkv", "F", "V", "b", "s"))
     hd = d // H
     Tt, Nqkv, Hd = b * s, (H + 2 * Hkv) * hd, H * hd

@@ -102,3 +102,22 @@ def test_attention_stash_removes_the_recomputed_attention_forwards():
     m1, e1 = bench.flops_per_step(sh, stash=True)
     assert m1 == m0 and e0 - e1 == pytest.approx((sh["L"] - 1) * A)
     assert e0 == pytest.approx(f0 + b0)
+
+
+def test_expert_workload_counts():
+    """Expert layers: the bench's parameter count is the arena's, a token's
+    MLP FLOPs count topk experts plus the router, and the recompute includes
+    the experts' down projections (the gates' gradients need their outputs)."""
+    from host_memory_streamed_layer_b200 import arena, mt
+    sh = synth.WORKLOADS["moe-8x1408"]
+    cfg = arena.config(sh)
+    n_layer = sum(mt.mt_tensor_offset(cfg, 0, t)[1] for t in range(10))
+    assert bench.layer_params(sh) == n_layer
+    d, F, E, k, L, T = sh["d"], sh["F"], sh["E"], sh["topk"], sh["L"], sh["b"] * sh["s"]
+    assert bench.mlp_active(sh) == 3 * d * F * k + E * d and bench.recompute_skip(sh) == 0
+    dense = {key: v for key, v in sh.items() if key not in ("E", "topk")}
+    m1, e1 = bench.flops_per_step(sh)
+    m0, e0 = bench.flops_per_step(dense)
+    assert m1 - m0 == pytest.approx(L * 6.0 * T * (bench.mlp_active(sh) - 3 * d * F))
+    f1, b1 = bench.phase_flops(sh)
+    assert e1 == pytest.approx(f1 + b1)
