@@ -365,7 +365,8 @@ def test_arena_layout_counts_and_alignment():
         c = oracle.OracleConfig(**cfg)
         layout, total = oracle.arena_layout(c)
         hd = c.d // c.H
-        per_layer = 2 * c.d + c.d * hd * (c.H + 2 * c.Hkv) + c.d * c.H * hd + 3 * c.F * c.d
+        mlp = (3 * c.F * c.d + c.d) * c.E if c.E else 3 * c.F * c.d  # experts: E SwiGLUs and the router
+        per_layer = 2 * c.d + c.d * hd * (c.H + 2 * c.Hkv) + c.d * c.H * hd + mlp
         params = 2 * c.V * c.d + c.d + c.L * per_layer
         assert sum(int(np.prod(s)) for *_, s in layout) == params
         assert all(off % 64 == 0 for _, _, off, _ in layout)
