@@ -1580,7 +1580,6 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   const Shapes& s = y.sh;
   mt_shard plan{};
   const NcclApi* nccl = nullptr;
-  if (cfg->E > 0 && world > 0) return set_err(nullptr, MT_ERR_CONFIG, "expert layers are not sharded");
   if (world > 0) {
     if (!id) return set_err(nullptr, MT_ERR_ARG, "sharded context without an NCCL id");
     if (cfg->flags & (MT_FLAG_DEFER_UPDATES | MT_FLAG_TIED_EMBED | MT_FLAG_BF16_GRADS))

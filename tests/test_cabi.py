@@ -426,6 +426,6 @@ def test_expert_layer_layout_matches_the_oracle():
     assert per_layer - per_dense == (6 - 1) * 3 * 96 * 256 + 6 * 256
     assert mt.mt_host_state_bytes(cfg) > mt.mt_host_state_bytes(dense)
     assert mt.mt_device_bytes(cfg) > mt.mt_device_bytes(dense)
-    with pytest.raises(mt.MTError) as e:  # expert layers are not partitioned
-        mt.mt_shard_plan(cfg, 2, 0)
-    assert e.value.code == -2
+    # expert layers partition like dense ones: their arena and bf16 offsets agree (d % 128 == 0)
+    p = mt.mt_shard_plan(cfg, 2, 1)
+    assert p["layer_elems"] == per_layer and p["layer_end"] == per_layer
