@@ -1385,6 +1385,11 @@ void collect_stats(mt_ctx* c) {
     st.d2h_bytes = act_bytes + (double)c->gsz * y.head_block + 4.0 * c->uniq.size() * y.sh.d + 12.0;
     for (int l = 0; l < L; ++l) st.d2h_bytes += (double)c->gsz * (y.layer_end(l) - y.layer_begin(l));
   }
+  if (y.sh.E > 0) {  // each layer's expert choices out and its row layout back, once per step
+    const double tk = (double)y.sh.T * y.sh.topk;
+    st.d2h_bytes += 4.0 * L * tk;
+    st.h2d_bytes += 8.0 * L * tk;
+  }
   st.adamw_ms = c->adamw_s * 1e3;
   st.adamw_bytes = c->adamw_bytes;
   st.gemm_flops = st.gemm_ms = st.attn_flops = st.attn_ms = 0;
