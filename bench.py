@@ -68,7 +68,7 @@ def parse():
                     help="keep the boundary activations in pinned host memory (MT_FLAG_OFFLOAD_ACTS)")
     ap.add_argument("--shard", action="store_true",
                     help="sharded streaming over the N ranks (mt_create_sharded): each loads, offloads and updates "
-                         "1/N of the state, all-gather / reduce-scatter over NCCL; implies --no-defer")
+                         "1/N of the state, all-gather / reduce-scatter over NCCL")
     ap.add_argument("--stash-attn", action="store_true",
                     help="keep each layer's attention output for its backward (MT_FLAG_STASH_ATTN)")
     ap.add_argument("--grad-dtype", default="fp32", choices=["fp32", "bf16"],
@@ -604,8 +604,6 @@ def main():
     sh = synth.WORKLOADS[args.workload]
     T = sh["b"] * sh["s"]
     cfg = arena.config(sh)
-    if args.shard:
-        args.no_defer = True  # the sharded engine runs every update inside its step
     cfg.seed = 1234 if args.shard else 1234 + rank  # one model over the ranks, or N replicas
     cfg.device = local
     # Gradients stream through a ring of host slots (14 instead of 18 B/param of

@@ -876,11 +876,22 @@ void run_job_body(mt_ctx* c, const Job& j) {
     // This rank's rows of the mean dense gradient, checked on the device (the
     // flag came back with them, its maximum over the ranks): the gradient
     // arena reports them, the update below reads them from the staging rows.
+    // With bf16 gradients the rows are rounded once, here on the host, as the
+    // unsharded path rounds its gathered rows.
     const size_t d = s.d, rb = (size_t)c->plan.embed_row_begin, re = (size_t)c->plan.embed_row_end;
-    if (c->grad)
-      parallel_ranges(*c->pool, (re - rb) * d, [&](size_t b, size_t e) {
-        memcpy(reinterpret_cast<float*>(c->grad) + y.embed.off + rb * d + b, c->emb_own_h + b, (e - b) * 4);
-      });
+    const size_t gsz = c->gsz;
+    parallel_ranges(*c->pool, (re - rb) * d, [&](size_t b, size_t e) {
+      float* src = c->emb_own_h + b;
+      if (gsz == 2)
+        for (size_t k = 0; k < e - b; ++k) {
+          const uint32_t w = (uint32_t)bf16_rne(src[k]) << 16;
+          memcpy(src + k, &w, 4);
+        }
+      if (c->grad && gsz == 4)
+        memcpy(reinterpret_cast<float*>(c->grad) + y.embed.off + rb * d + b, src, (e - b) * 4);
+      if (c->grad && gsz == 2)
+        bf16_round_chunk(src, reinterpret_cast<uint16_t*>(c->grad) + y.embed.off + rb * d + b, e - b);
+    });
   } else if (j.kind == Job::EMBED) {
     // Touched rows: check this step's gradient rows for NaN/Inf and, with a
     // gradient arena, put last step's touched rows back to zero and scatter
@@ -968,7 +979,7 @@ void run_job_body(mt_ctx* c, const Job& j) {
     }
   }
   adamw_segments(c, segs, c->step);
-  if (j.kind == Job::EMBED && (c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !y.tied) {
+  if (j.kind == Job::EMBED && (c->cfg.flags & MT_FLAG_DEFER_UPDATES) && !y.tied && !sharded(c)) {
     // The step's last job: every gradient passed its checks, so the
     // zero-gradient update of the rows it did not touch is due. It runs with
     // the next step (or at the next flush), overlapping its GPU work.
@@ -1587,9 +1598,8 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   const NcclApi* nccl = nullptr;
   if (world > 0) {
     if (!id) return set_err(nullptr, MT_ERR_ARG, "sharded context without an NCCL id");
-    if (cfg->flags & (MT_FLAG_DEFER_UPDATES | MT_FLAG_TIED_EMBED | MT_FLAG_BF16_GRADS))
-      return set_err(nullptr, MT_ERR_CONFIG,
-                     "sharded streaming runs without MT_FLAG_DEFER_UPDATES, MT_FLAG_TIED_EMBED and MT_FLAG_BF16_GRADS");
+    if (cfg->flags & MT_FLAG_TIED_EMBED)
+      return set_err(nullptr, MT_ERR_CONFIG, "sharded streaming runs without MT_FLAG_TIED_EMBED");
     r = mt_shard_plan(cfg, world, rank, &plan);
     if (r != MT_OK) return set_err(nullptr, r, "no shard plan for this config (d must be a multiple of 128)");
     nccl = nccl_api(&why);

@@ -320,9 +320,10 @@ int mt_shard_id(void* id_out);
  * mt_get_opt_state hold current values on the rank's own ranges only.
  * Collectives of the H2D stream and of the compute stream use two
  * communicators, so each runs in one program order on every rank.
- * Requires d % 128 == 0; MT_ERR_CONFIG with MT_FLAG_DEFER_UPDATES,
- * MT_FLAG_TIED_EMBED or MT_FLAG_BF16_GRADS, and mt_layer_fwd_bwd /
- * mt_head_fwd_bwd refuse a sharded context. world = 1 runs the same path
+ * Requires d % 128 == 0; MT_ERR_CONFIG with MT_FLAG_TIED_EMBED (the table
+ * would have two owners), and mt_layer_fwd_bwd / mt_head_fwd_bwd refuse a
+ * sharded context. Expert layers, deferred updates and bf16 gradients work
+ * as in an unsharded context (each rank routes its own tokens). world = 1 runs the same path
  * with one rank (the collectives are copies). */
 int mt_create_sharded(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, int world, int rank,
                       const void* id, mt_ctx** out);

@@ -53,6 +53,10 @@ def _run(shape, flags, nsteps, sharded):
         for step in range(nsteps):
             tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, step)
             loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+            # deferred updates (the unsharded engine defers the untouched
+            # embedding rows too; the sharded one updates its rows densely)
+            # are applied before the state is read
+            mt.mt_flush(ctx)
             G = None
             if not flags & mt.MT_FLAG_GRAD_RING:
                 G = np.empty_like(A)
@@ -64,13 +68,14 @@ def _run(shape, flags, nsteps, sharded):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("flags", [0, "ring", "offload+stash"])
+@pytest.mark.parametrize("flags", [0, "ring", "offload+stash", "defer+bf16+ring"])
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_one_rank_sharded_steps_match_the_plain_engine_and_the_oracle(name, flags):
     from host_memory_streamed_layer_b200 import mt
     shape = SHAPES[name]
     fl = {0: 0, "ring": mt.MT_FLAG_GRAD_RING,
-          "offload+stash": mt.MT_FLAG_OFFLOAD_ACTS | mt.MT_FLAG_STASH_ATTN}[flags]
+          "offload+stash": mt.MT_FLAG_OFFLOAD_ACTS | mt.MT_FLAG_STASH_ATTN,
+          "defer+bf16+ring": mt.MT_FLAG_DEFER_UPDATES | mt.MT_FLAG_BF16_GRADS | mt.MT_FLAG_GRAD_RING}[flags]
     # Head dim 128 runs the deterministic split attention backward: with one
     # rank every collective is a copy (the mean of one is the value) and the
     # dense zero-gradient rows update exactly like the untouched-row form, so
@@ -128,13 +133,13 @@ def test_one_rank_sharded_link_bytes_are_the_own_parts():
 
 def test_shard_id_and_refusals_without_a_gpu():
     """mt_shard_id gives MT_SHARD_ID_BYTES fresh bytes per call; a sharded
-    context refuses deferred updates, tied embeddings, bf16 gradients and
-    d % 128 != 0 before it touches a device, and bad ranks."""
+    context refuses tied embeddings and d % 128 != 0 before it touches a
+    device, and bad ranks."""
     from host_memory_streamed_layer_b200 import arena, mt
     a, b = mt.mt_shard_id(), mt.mt_shard_id()
     assert len(a) == len(b) == mt.MT_SHARD_ID_BYTES and a != b
     shape = SHAPES["hd128"]
-    for flag in (mt.MT_FLAG_DEFER_UPDATES, mt.MT_FLAG_TIED_EMBED, mt.MT_FLAG_BF16_GRADS):
+    for flag in (mt.MT_FLAG_TIED_EMBED,):
         cfg = arena.config(shape)
         cfg.flags = flag
         with pytest.raises(mt.MTError) as e:
