@@ -208,6 +208,10 @@ struct mt_ctx {
   int32_t* d_uid = nullptr;       // unique token ids of the step, [T]
   float* emb_own_h = nullptr;     // pinned: this rank's rows of the mean embedding gradient
   cudaEvent_t ev_embw = nullptr;  // embedding table all-gathered
+  // Floats from the start of d_head_g to the head's table gradient: the
+  // layout's gf_pad, or with tied embeddings on a sharded context past the
+  // padded [final gain] block that the reduce-scatter covers.
+  size_t head_g_split = 0;
 
   // ---- mixture-of-experts layers (E > 0) ----
   // Routing of layer l, taken in its forward and reused by its recompute:
@@ -377,6 +381,19 @@ int reduce_own_chunk(mt_ctx* c, float* blk, size_t chunk, size_t own_begin, size
   CKM(check_finite(c, blk + own_begin, own_end - own_begin, idx));
   NK(AllReduce(c->d_flags + idx, c->d_flags + idx, 1, ncclInt32, ncclMax, c->comm_comp, c->s_comp));
   return MT_OK;
+}
+
+// dst += src over n floats (n a multiple of 4, both 16-byte aligned).
+__global__ void k_add_f32(float* __restrict__ dst, const float* __restrict__ src, size_t n) {
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n / 4; i += (size_t)gridDim.x * blockDim.x) {
+    float4 a = reinterpret_cast<float4*>(dst)[i];
+    const float4 b = reinterpret_cast<const float4*>(src)[i];
+    a.x += b.x;
+    a.y += b.y;
+    a.z += b.z;
+    a.w += b.w;
+    reinterpret_cast<float4*>(dst)[i] = a;
+  }
 }
 
 // Rows of the step's unique tokens (row u for token uid[u]) into a zeroed
@@ -673,9 +690,10 @@ int head_step(mt_ctx* c, float* gout) {
   const Shapes& s = c->lay.sh;
   const int T = s.T, d = s.d, V = s.V;
   cudaStream_t st = c->s_comp;
-  const size_t gf_pad = c->lay.gf_pad;  // floats between dgf and dWhead
+  const size_t gf_pad = c->head_g_split;  // floats between dgf and dWhead
   const uint16_t* gf = c->d_head_w;
-  const uint16_t* Wh = c->d_head_w + align_up(d, 128);
+  // tied embeddings on a sharded context: the head reads the device table
+  const uint16_t* Wh = (sharded(c) && c->lay.tied) ? c->d_embed_w : c->d_head_w + align_up(d, 128);
   float* dgf = c->d_head_g;
   float* dWh = c->d_head_g + gf_pad;
   const float* xL = x_fwd(c, s.L);
@@ -892,6 +910,11 @@ void run_job_body(mt_ctx* c, const Job& j) {
       if (c->grad && gsz == 2)
         bf16_round_chunk(src, reinterpret_cast<uint16_t*>(c->grad) + y.embed.off + rb * d + b, e - b);
     });
+    // tied: the final gain's gradient came back in the head's own buffer; the
+    // gradient arena reports this rank's part of it
+    if (y.tied && c->grad && c->plan.head_end > c->plan.head_begin)
+      memcpy(c->grad + (y.final_norm.off + c->plan.head_begin) * gsz, c->grad_head + c->plan.head_begin * gsz,
+             (c->plan.head_end - c->plan.head_begin) * gsz);
   } else if (j.kind == Job::EMBED) {
     // Touched rows: check this step's gradient rows for NaN/Inf and, with a
     // gradient arena, put last step's touched rows back to zero and scatter
@@ -967,11 +990,11 @@ void run_job_body(mt_ctx* c, const Job& j) {
   std::vector<Seg> segs;
   if (j.kind == Job::LAYER || j.kind == Job::HEAD) {
     segs = layer_or_head_segs(c, j.kind == Job::HEAD ? -1 : j.layer, j.g);
-  } else if (y.tied) {  // EMBED, tied: one dense update of the whole table
-    segs.push_back({y.embed.off, y.embed.n, c->bf_embed, reinterpret_cast<const float*>(c->grad_head) + y.gf_pad});
   } else if (sharded(c)) {  // EMBED, sharded: this rank's rows, dense (untouched rows have zero gradient)
     const size_t rb = (size_t)c->plan.embed_row_begin, re = (size_t)c->plan.embed_row_end;
     if (re > rb) segs.push_back({y.embed.off + rb * s.d, (re - rb) * s.d, c->bf_embed + rb * s.d, c->emb_own_h});
+  } else if (y.tied) {  // EMBED, tied: one dense update of the whole table
+    segs.push_back({y.embed.off, y.embed.n, c->bf_embed, reinterpret_cast<const float*>(c->grad_head) + y.gf_pad});
   } else {
     for (size_t u = 0; u < c->uniq.size(); ++u) {
       const size_t r = (size_t)c->uniq[u];
@@ -1329,6 +1352,13 @@ int enqueue_step(mt_ctx* c, int n_unique) {
       CK(cudaGetLastError());
       c->launches += 1;
     }
+    if (y.tied) {  // the table's gradient is also the head's: add it before the ranks' mean
+      const size_t n = (size_t)s.V * d;
+      k_add_f32<<<(unsigned)std::min<size_t>((n / 4 + 255) / 256, 148 * 16), 256, 0, sc>>>(
+          c->d_embed_g, c->d_head_g + c->head_g_split, n);
+      CK(cudaGetLastError());
+      c->launches += 1;
+    }
     CKM(reduce_own_chunk(c, c->d_embed_g, rows * d, rb * d, re * d, L + 1));
     CK(cudaEventRecord(c->ev_emb_ready, sc));
     CK(cudaStreamWaitEvent(c->s_d2h, c->ev_emb_ready, 0));
@@ -1434,7 +1464,11 @@ size_t gslot_elems(const Layout& y, const mt_shard* p) {
 size_t head_w_elems(const Layout& y, const mt_shard* p) {
   return p ? (size_t)p->world * p->head_chunk : align_up(y.sh.d, 128) + (size_t)y.sh.V * y.sh.d;
 }
+size_t head_g_split(const Layout& y, const mt_shard* p) {
+  return (p && y.tied) ? std::max(y.gf_pad, (size_t)p->world * p->head_chunk) : y.gf_pad;
+}
 size_t head_g_elems(const Layout& y, const mt_shard* p) {
+  if (p && y.tied) return head_g_split(y, p) + (size_t)y.sh.V * y.sh.d;  // [gain, padded | table gradient]
   return p ? (size_t)p->world * p->head_chunk : y.head_block;
 }
 
@@ -1598,8 +1632,6 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   const NcclApi* nccl = nullptr;
   if (world > 0) {
     if (!id) return set_err(nullptr, MT_ERR_ARG, "sharded context without an NCCL id");
-    if (cfg->flags & MT_FLAG_TIED_EMBED)
-      return set_err(nullptr, MT_ERR_CONFIG, "sharded streaming runs without MT_FLAG_TIED_EMBED");
     r = mt_shard_plan(cfg, world, rank, &plan);
     if (r != MT_OK) return set_err(nullptr, r, "no shard plan for this config (d must be a multiple of 128)");
     nccl = nccl_api(&why);
@@ -1632,6 +1664,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   c->cfg = *cfg;
   c->lay = y;
   c->plan = plan;
+  c->head_g_split = head_g_split(y, world > 0 ? &plan : nullptr);
   c->nccl = nccl;
   c->device = cfg->device;
   c->Tc = Tc;

@@ -196,7 +196,6 @@ extern "C" int mt_shard_plan(const mt_config* cfg, int world, int rank, mt_shard
   if (!out || world < 1 || world > 1024 || rank < 0 || rank >= world) return MT_ERR_ARG;
   if (mt::validate_config(cfg, nullptr) != MT_OK) return MT_ERR_CONFIG;
   if (cfg->d % 128) return MT_ERR_CONFIG;  // fp32 and bf16 block offsets coincide only then
-  if (cfg->flags & MT_FLAG_TIED_EMBED) return MT_ERR_CONFIG;  // one table, two owners: not partitioned
   const mt::Layout y = mt::make_layout(*cfg);
   const size_t lb = y.layer_begin(0), le = y.layer_end(0);
   // The fp32 arena block of a layer and its bf16 streamed block must hold

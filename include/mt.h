@@ -120,8 +120,7 @@ extern "C" {
  * refuses MT_T_LM_HEAD); the head streams the bf16 table each step, and the
  * table's gradient is the head's dense V x d gradient plus the gathered rows'.
  * It is updated with one dense AdamW in the step's last host job, after every
- * gradient of the step has been checked. Not with MT_FLAG_BF16_GRADS, and not
- * partitioned by mt_shard_plan (MT_ERR_CONFIG). */
+ * gradient of the step has been checked. Not with MT_FLAG_BF16_GRADS. */
 #define MT_FLAG_TIED_EMBED 0x80u
 /* Keep each layer's attention output O (bf16 [b*s, H*hd]) and log-sum-exp
  * (fp32 [b, H, s]) on the device from the forward sweep to the layer's
@@ -320,10 +319,11 @@ int mt_shard_id(void* id_out);
  * mt_get_opt_state hold current values on the rank's own ranges only.
  * Collectives of the H2D stream and of the compute stream use two
  * communicators, so each runs in one program order on every rank.
- * Requires d % 128 == 0; MT_ERR_CONFIG with MT_FLAG_TIED_EMBED (the table
- * would have two owners), and mt_layer_fwd_bwd / mt_head_fwd_bwd refuse a
- * sharded context. Expert layers, deferred updates and bf16 gradients work
- * as in an unsharded context (each rank routes its own tokens). world = 1 runs the same path
+ * Requires d % 128 == 0; mt_layer_fwd_bwd / mt_head_fwd_bwd refuse a
+ * sharded context. Expert layers, deferred updates, bf16 gradients and tied
+ * embeddings work as in an unsharded context (each rank routes its own
+ * tokens; a tied head reads the device table and its dense gradient joins
+ * the rows' before the ranks' mean). world = 1 runs the same path
  * with one rank (the collectives are copies). */
 int mt_create_sharded(const mt_config* cfg, float* host_param_arena, size_t arena_bytes, int world, int rank,
                       const void* id, mt_ctx** out);

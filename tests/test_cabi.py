@@ -379,7 +379,8 @@ def test_attention_stash_adds_one_output_and_lse_per_layer():
 def test_tied_embeddings_layout():
     """MT_FLAG_TIED_EMBED: the arena loses exactly the LM-head tensor (the
     oracle's tied layout matches the library's offsets), MT_T_LM_HEAD is
-    refused, and the combinations the flag does not support are refused."""
+    refused, bf16 gradients are refused, and the shard plan's head block is
+    the final gain alone."""
     import oracle
     from host_memory_streamed_layer_b200 import arena, mt
     shape = dict(L=3, d=256, H=4, Hkv=2, F=688, V=1000, b=2, s=64)
@@ -394,8 +395,9 @@ def test_tied_embeddings_layout():
         assert mt.mt_tensor_offset(cfg, layer, tid) == (off, int(np.prod(shp)))
     with pytest.raises(mt.MTError):
         mt.mt_tensor_offset(cfg, -1, mt.MT_T_LM_HEAD)
-    with pytest.raises(mt.MTError):
-        mt.mt_shard_plan(cfg, 2, 0)
+    # sharded: the head block is the final gain alone (the table is split by rows)
+    p = mt.mt_shard_plan(cfg, 2, 1)
+    assert p["head_elems"] == shape["d"] and p["embed_row_end"] == shape["V"]
     cfg.flags = mt.MT_FLAG_TIED_EMBED | mt.MT_FLAG_BF16_GRADS
     assert mt.mt_arena_bytes(cfg) == 0
 

@@ -68,12 +68,12 @@ def _run(shape, flags, nsteps, sharded):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("flags", [0, "ring", "offload+stash", "defer+bf16+ring"])
+@pytest.mark.parametrize("flags", [0, "ring", "offload+stash", "defer+bf16+ring", "tied"])
 @pytest.mark.parametrize("name", list(SHAPES))
 def test_one_rank_sharded_steps_match_the_plain_engine_and_the_oracle(name, flags):
     from host_memory_streamed_layer_b200 import mt
-    shape = SHAPES[name]
-    fl = {0: 0, "ring": mt.MT_FLAG_GRAD_RING,
+    shape = dict(SHAPES[name], tied=flags == "tied")
+    fl = {0: 0, "ring": mt.MT_FLAG_GRAD_RING, "tied": mt.MT_FLAG_TIED_EMBED,
           "offload+stash": mt.MT_FLAG_OFFLOAD_ACTS | mt.MT_FLAG_STASH_ATTN,
           "defer+bf16+ring": mt.MT_FLAG_DEFER_UPDATES | mt.MT_FLAG_BF16_GRADS | mt.MT_FLAG_GRAD_RING}[flags]
     # Head dim 128 runs the deterministic split attention backward: with one
@@ -133,18 +133,11 @@ def test_one_rank_sharded_link_bytes_are_the_own_parts():
 
 def test_shard_id_and_refusals_without_a_gpu():
     """mt_shard_id gives MT_SHARD_ID_BYTES fresh bytes per call; a sharded
-    context refuses tied embeddings and d % 128 != 0 before it touches a
-    device, and bad ranks."""
+    context refuses d % 128 != 0 before it touches a device, and bad ranks."""
     from host_memory_streamed_layer_b200 import arena, mt
     a, b = mt.mt_shard_id(), mt.mt_shard_id()
     assert len(a) == len(b) == mt.MT_SHARD_ID_BYTES and a != b
     shape = SHAPES["hd128"]
-    for flag in (mt.MT_FLAG_TIED_EMBED,):
-        cfg = arena.config(shape)
-        cfg.flags = flag
-        with pytest.raises(mt.MTError) as e:
-            mt.mt_create_sharded(cfg, 0, 0, 2, 0, a)
-        assert e.value.code == -2  # MT_ERR_CONFIG
     with pytest.raises(mt.MTError) as e:
         mt.mt_create_sharded(arena.config(dict(shape, d=192, H=3, Hkv=3)), 0, 0, 2, 0, a)
     assert e.value.code == -2
