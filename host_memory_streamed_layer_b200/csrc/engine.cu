@@ -212,6 +212,7 @@ struct mt_ctx {
   // layout's gf_pad, or with tied embeddings on a sharded context past the
   // padded [final gain] block that the reduce-scatter covers.
   size_t head_g_split = 0;
+  size_t wslot_bytes = 0;  // bytes of a device weight slot (padded when sharded)
 
   // ---- mixture-of-experts layers (E > 0) ----
   // Routing of layer l, taken in its forward and reused by its recompute:
@@ -1244,6 +1245,14 @@ int fetch_act(mt_ctx* c, int l) {
   return MT_OK;
 }
 
+// MT_FLAG_POISON: gradient slot k & 1 filled with NaN before backward index
+// k writes it (its previous contents have drained to the host).
+int poison_grad(mt_ctx* c, int k) {
+  if (!(c->cfg.flags & MT_FLAG_POISON)) return MT_OK;
+  CK(cudaMemsetAsync(c->gslot[k & 1], 0xFF, c->layer_f * 4, c->s_comp));
+  return MT_OK;
+}
+
 int enqueue_step(mt_ctx* c, int n_unique) {
   const Layout& y = c->lay;
   const Shapes& s = y.sh;
@@ -1309,6 +1318,7 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         push_job(c, hj);
         CK(cudaEventRecord(c->ev_head_end, sc));
         // backward of the last layer: its intermediates are still in the workspace
+        CKM(poison_grad(c, 0));
         CKM(layer_bwd(c, l, slot, x_bwd(c, l), c->gslot[0], gin, gout));
         CKM(offload_layer(c, l, 0));
         std::swap(gin, gout);
@@ -1321,6 +1331,7 @@ int enqueue_step(mt_ctx* c, int n_unique) {
       const int k = i - (L - 1);  // backward index: layer L-1-k
       const int l = L - 1 - k;
       if (k >= 2) CK(cudaStreamWaitEvent(sc, c->ev_gdrained[k - 2], 0));
+      CKM(poison_grad(c, k));
       if (offload_acts(c)) CK(cudaStreamWaitEvent(sc, l == L - 2 ? c->ev_xout[l] : c->ev_xin[l], 0));
       CKM(layer_fwd(c, l, slot, x_bwd(c, l), nullptr));
       CKM(layer_bwd(c, l, slot, x_bwd(c, l), c->gslot[k & 1], gin, gout));
@@ -1331,6 +1342,7 @@ int enqueue_step(mt_ctx* c, int n_unique) {
         CKM(fetch_act(c, l - 2));
       }
     }
+    if (c->cfg.flags & MT_FLAG_POISON) CK(cudaMemsetAsync(c->wslot[slot], 0xFF, c->wslot_bytes, sc));
     CK(cudaEventRecord(c->ev_slotfree[i], sc));
     // The head's weights follow the last forward load on the H2D stream, ahead
     // of the first backward load. Issued here, after layer L-2's forward is
@@ -1827,6 +1839,7 @@ int create_impl(const mt_config* cfg, float* arena, size_t arena_bytes, mt_ctx**
   };
   const size_t T = s.T, d = s.d, F = s.F, V = s.V;
   const mt_shard* pp = world > 0 ? &plan : nullptr;
+  c->wslot_bytes = slot_elems(y, pp) * 2;
   c->wslot[0] = (uint16_t*)carve(slot_elems(y, pp) * 2);
   c->wslot[1] = (uint16_t*)carve(slot_elems(y, pp) * 2);
   const size_t lay_f = y.layer_end(0) - y.layer_begin(0);

@@ -214,6 +214,7 @@ MT_FLAG_BF16_GRADS = 0x20
 MT_FLAG_OFFLOAD_ACTS = 0x40
 MT_FLAG_TIED_EMBED = 0x80
 MT_FLAG_STASH_ATTN = 0x100
+MT_FLAG_POISON = 0x200
 MT_GRAD_RING_SLOTS = 3
 MT_T_ATTN_NORM, MT_T_WQ, MT_T_WK, MT_T_WV, MT_T_WO, MT_T_MLP_NORM, MT_T_WGATE, MT_T_WUP, MT_T_WDOWN = range(9)
 MT_T_ROUTER = 9

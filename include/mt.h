@@ -134,6 +134,14 @@ extern "C" {
  * (mt_device_bytes). The results are unchanged: the attention forward is
  * deterministic, so the kept O and LSE are those a recompute would give. */
 #define MT_FLAG_STASH_ATTN 0x100u
+/* Debug: fill every device weight slot with NaN (bf16 0xFFFF) as soon as the
+ * compute stream releases it and every gradient slot (fp32 0xFFFFFFFF) just
+ * before a layer's backward writes it, so that a read of a slot before its
+ * reload or write completes (a missing wait) turns the step's results into
+ * NaN instead of silently using stale data. Results are otherwise unchanged;
+ * costs one memset per load and per backward layer. (Race detection without
+ * a sanitizer, which this environment does not offer.) */
+#define MT_FLAG_POISON 0x200u
 
 /* Tensor ids inside a decoder layer and for model-level tensors (layer = -1). */
 #define MT_T_ATTN_NORM 0

@@ -663,3 +663,51 @@ def test_deferred_updates_follow_the_undeferred_trajectory(monkeypatch):
     for a, b in zip(ring["losses"], dfr["losses"]):
         assert abs(a - b) <= 1e-4
     assert rel(ring["P"], dfr["P"]) <= 2e-3
+
+
+@pytest.mark.parametrize("flags", [0, 0x8 | 0x10, 0x40 | 0x100])
+def test_poisoned_slots_and_host_stalls_leave_the_steps_unchanged(flags):
+    """Race checks without a sanitizer. MT_FLAG_POISON fills each weight slot
+    with NaN once the compute stream releases it and each gradient slot before
+    a backward writes it: a read before a reload or write completes would turn
+    the results into NaN. A host stall injected on the weight stream, then on
+    the gradient stream, delays copies without changing what any kernel reads.
+    With the split attention backward every reduction has a fixed order, so
+    all runs must agree bit for bit (plain, ring + deferral, offload + stash)."""
+    arena, mt = _libs()
+    shape = dict(SHAPES["hd128"], L=4)  # enough layers for offloaded boundaries and a recompute chain
+
+    def run(extra, stall=None):
+        cfg = arena.config(shape)
+        cfg.flags = flags | extra
+        cfg.host_threads = 4
+        A = arena.pack(cfg, synth.init_weights(shape, 0))
+        ctx = mt.mt_create(cfg, A.ctypes.data, A.nbytes)
+        out = []
+        try:
+            for step in range(2):
+                tok, lab = synth.tokens_labels(shape["b"], shape["s"], shape["V"], 0, step)
+                if stall is not None:
+                    mt.mt_inject_host_stall(ctx, stall[step], 60)
+                loss = mt.mt_train_step(ctx, tok.ctypes.data, lab.ctypes.data)
+                mt.mt_flush(ctx)
+                G = None
+                if not cfg.flags & mt.MT_FLAG_GRAD_RING:
+                    G = np.empty_like(A)
+                    mt.mt_get_grads(ctx, G.ctypes.data, G.nbytes)
+                out.append((loss, G, A.copy()))
+        finally:
+            mt.mt_destroy(ctx)
+        return out
+
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT)
+    try:
+        ref = run(0)
+        others = [run(mt.MT_FLAG_POISON), run(0, stall=(0, 2)), run(mt.MT_FLAG_POISON, stall=(2, 0))]
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
+    for other in others:
+        for (la, Ga, Pa), (lb, Gb, Pb) in zip(ref, other):
+            assert la == lb and np.isfinite(lb)
+            assert Ga is None or np.array_equal(Ga, Gb)
+            assert np.array_equal(Pa, Pb)
