@@ -69,6 +69,8 @@ def parse():
     ap.add_argument("--shard", action="store_true",
                     help="sharded streaming over the N ranks (mt_create_sharded): each loads, offloads and updates "
                          "1/N of the state, all-gather / reduce-scatter over NCCL")
+    ap.add_argument("--attn-bwd", default="auto", choices=["auto", "fused", "split"],
+                    help="attention backward: dQ by reductions (fused) or the deterministic split")
     ap.add_argument("--stash-attn", action="store_true",
                     help="keep each layer's attention output for its backward (MT_FLAG_STASH_ATTN)")
     ap.add_argument("--grad-dtype", default="fp32", choices=["fp32", "bf16"],
@@ -639,6 +641,8 @@ def main():
     host_bw = host_optimizer_bandwidth(mt, cfg.host_threads) if rank == 0 else None
     # independent host-DRAM ceiling: STREAM triad (12 B/element, non-temporal stores)
     triad = mt.mt_host_triad_gbs(1 << 28, cfg.host_threads) if rank == 0 else None
+    mt.mt_k_attn_bwd_variant({"auto": mt.ATTN_BWD_AUTO, "fused": mt.ATTN_BWD_FUSED,
+                              "split": mt.ATTN_BWD_SPLIT}[args.attn_bwd])
     if args.shard:
         nccl_id = mt.mt_shard_id() if rank == 0 else bytes(mt.MT_SHARD_ID_BYTES)
         if dist is not None:
@@ -741,6 +745,8 @@ def main():
                        "boundary_activations": "pinned host memory" if args.offload_acts else "HBM",
                        "attention_recompute": ("none: O and LSE kept per layer (MT_FLAG_STASH_ATTN)"
                                                if args.stash_attn else "in each layer's recompute"),
+                       "attention_backward": ("split: dK/dV key-major, dQ query-major, deterministic"
+                                              if args.attn_bwd == "split" else "fused: dQ by fp32 reductions"),
                        "grads": (f"{args.grad_dtype} gradients offloaded; " +
                                  (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
                                   if args.grads == "ring" else "full gradient arena in pinned host memory"))},
