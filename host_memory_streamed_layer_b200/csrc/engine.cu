@@ -330,7 +330,7 @@ int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
   int r = bwd ? (a.hd == 128 ? attention_bwd_tc(a, c->s_comp, c->d_err) : attention_bwd(a, c->s_comp))
               : attention_fwd_tc(a, c->s_comp, c->d_err);
   if (r != MT_OK) return set_err(c, r, "attention launch failed");
-  c->launches += bwd ? (a.hd == 128 ? attention_bwd_kernels() : 3) : 1;
+  c->launches += bwd ? (a.hd == 128 ? attention_bwd_kernels(a.s) : 3) : 1;
   if (timing && e0 && e1) {
     cudaEventRecord(e1, c->s_comp);
     // causal attention: QK^T and PV over the visible half, per query head

@@ -105,7 +105,7 @@ int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
 // kernel, dQ by the query-major one, deterministic); returns the previous one.
 int attention_bwd_variant(int v);
 // Kernels one head_dim-128 backward launches in the current form.
-int attention_bwd_kernels();
+int attention_bwd_kernels(int s);
 
 // Mixture-of-experts MLP (moe.cu). Router: logits [T, E], the topk experts
 // idx [T, k] and their gates [T, k] of the bf16 MLP input w [T, d] and router
