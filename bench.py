@@ -225,8 +225,8 @@ def oracle_sample_plan(sh):
     oracle forms the full s x s score matrix), the head 6 T V d, AdamW a
     constant per parameter."""
     hd = sh["d"] // sh["H"]
-    pm = sh["d"] * (sh["H"] + 2 * sh["Hkv"]) * hd + sh["d"] * sh["H"] * hd + 3 * sh["d"] * sh["F"]
-    s_smp = min(sh["s"], 2048 if pm < 1e8 else 512)
+    pm = sh["d"] * (sh["H"] + 2 * sh["Hkv"]) * hd + sh["d"] * sh["H"] * hd + mlp_active(sh)
+    s_smp = min(sh["s"], 2048 if pm < 1e8 and not sh.get("E", 0) else 512)  # (expert layers: slower per token)
     v_head = min(sh["V"], 32000)
     t_head = int(min(sh["b"] * sh["s"], max(64, 0.6e12 / (6.0 * v_head * sh["d"]) // 64 * 64)))
     p_layer = layer_params(sh)
@@ -253,7 +253,7 @@ class OracleSample:
         self.c = oracle.OracleConfig(**{**sh, "b": 1, "L": 1, "s": pl["s_smp"]})
         c, hd = self.c, self.c.d // self.c.H
         self.W = {tid: synth.init_tensor(seed, 0, tid, shp).astype(np.float64)
-                  for tid, shp in synth.layer_shapes(c.d, c.H, c.Hkv, c.F, hd)}
+                  for tid, shp in synth.layer_shapes(c.d, c.H, c.Hkv, c.F, hd, c.E)}
         rng = np.random.default_rng(seed)
         self.x = rng.normal(size=(1, c.s, c.d))
         self.dx = rng.normal(size=self.x.shape)
