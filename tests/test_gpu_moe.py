@@ -21,6 +21,8 @@ SHAPES = {
     # more experts than routed rows need: several experts get no token
     "sparse": dict(L=2, d=128, H=1, Hkv=1, F=64, V=256, b=1, s=8, E=16, topk=1),
     "ragged": dict(L=3, d=256, H=4, Hkv=2, F=96, V=304, b=3, s=37, E=6, topk=3),
+    # one layer, one token: two routed rows, one idle expert
+    "one_token": dict(L=1, d=128, H=1, Hkv=1, F=64, V=64, b=1, s=1, E=3, topk=2),
 }
 
 
