@@ -745,10 +745,8 @@ def main():
                        "boundary_activations": "pinned host memory" if args.offload_acts else "HBM",
                        "attention_recompute": ("none: O and LSE kept per layer (MT_FLAG_STASH_ATTN)"
                                                if args.stash_attn else "in each layer's recompute"),
-                       "attention_backward": ("split: dK/dV key-major, dQ query-major, deterministic"
-                                              if args.attn_bwd == "split" or (args.attn_bwd == "auto"
-                                                                              and sh["s"] >= 16384)
-                                              else "fused: dQ by fp32 reductions"),
+                       "attention_backward": ("fused: dQ by fp32 reductions" if args.attn_bwd == "fused"
+                                              else "split: dK/dV key-major, dQ query-major, deterministic"),
                        "grads": (f"{args.grad_dtype} gradients offloaded; " +
                                  (f"ring of {mt.MT_GRAD_RING_SLOTS} layer slots in pinned host memory"
                                   if args.grads == "ring" else "full gradient arena in pinned host memory"))},

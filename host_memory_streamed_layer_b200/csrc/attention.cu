@@ -572,7 +572,7 @@ int attention_bwd_variant(int v) {
   return was;
 }
 
-int attention_bwd_kernels(int s) { return (g_bwd_variant == 2 || (g_bwd_variant == 0 && s >= 16384)) ? 4 : 3; }
+int attention_bwd_kernels(int) { return g_bwd_variant == 1 ? 3 : 4; }
 
 int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   if (a.b <= 0 || a.s <= 0) return MT_OK;
@@ -581,11 +581,13 @@ int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   const int64_t nw = (int64_t)T * a.H;
   k_attn_bwd_pre<<<(int)((nw + 7) / 8), 256, 0, st>>>((const bf16*)a.o, (const bf16*)a.dout, a.ldo, a.dvec, T, a.s,
                                                       a.H, 128);
-  // automatic: the deterministic split form from 16384 tokens on, where it
-  // times the same as the fused one (one box: 8854 against 8988 us at 16384,
-  // 4345 against 4336 tokens/s in the 131072-token training step); below,
-  // the fused form (6-10 % faster at 2048)
-  const bool split = g_bwd_variant == 2 || (g_bwd_variant == 0 && a.s >= 16384);
+  // automatic: the deterministic split form, which is also the faster one at
+  // every length measured (B200, 16 or 32 heads of 128: 746 against 832 us at
+  // 8 x 2048, 2268 against 2671 at 4 x 4096, 7695 against 8979 at 16384);
+  // its query-major kernel stores dq_acc four floats at a time
+  const bool aligned = (reinterpret_cast<uintptr_t>(a.dq_acc) & 15) == 0 && a.ldqa % 4 == 0;
+  if (g_bwd_variant == 2 && !aligned) return MT_ERR_ARG;
+  const bool split = g_bwd_variant == 2 || (g_bwd_variant == 0 && aligned);
   if (split) {  // dK, dV without reductions; dQ written once per element by the query-major kernel
     int r = attention_bwd_tc_main(a, st, err, true);
     if (r == MT_OK) r = attention_bwd_dq_tc(a, st, err);

@@ -878,13 +878,78 @@ struct FbParams {
   const float* rsin;
   int* err;
   int vec_lse;  // LSE and D rows start 16-byte aligned: s % 4 == 0 and aligned bases
-  int skip_dq;  // dK and dV only: dQ comes from the query-major kernel (k_flash_bwd_dq)
 };
 
 // Start-address step (address / 16) of k-step kk (16 elements of the
 // contraction) inside a K-major 128-row tile made of two 64-column sub-tiles.
 __device__ __forceinline__ uint32_t km_step(int kk) {
   return (uint32_t)(((kk >> 2) * FbCfg::SUB + (kk & 3) * 32) >> 4);
+}
+
+// The CTA's dK and dV (tensor-memory columns C_DK and C_DV, fp32, one key
+// row per lane) out to global memory as bf16, by the 16 gradient warps.
+__device__ __forceinline__ void fb_store_dkdv(uint32_t tmem, uint32_t lane_base, int qg, int key, int row0,
+                                              int kvh, const FbParams& p) {
+  using C = FbCfg;
+  // tcgen05.ld is warp-collective: every lane loads, only keys inside the
+  // sequence store. Warps of query group 0 and 1 write dK (scaled,
+  // transposed RoPE; rotate-half pairs (i, i + 64) for i in [32 qg, 32 qg + 32)),
+  // groups 2 and 3 write dV columns [64 (qg - 2), 64 (qg - 2) + 64).
+  const bool store = key < p.s;
+  if (qg < 2) {
+    __nv_bfloat16* kr = p.dK + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
+    const float* cs = (p.rcos && store) ? p.rcos + (int64_t)key * (FB_HD / 2) : nullptr;
+    const float* sn = (p.rsin && store) ? p.rsin + (int64_t)key * (FB_HD / 2) : nullptr;
+#pragma unroll
+    for (int cc = 0; cc < 2; ++cc) {  // pairs (i, i + 64), 16 at a time
+      const int c = qg * 2 + cc;
+      uint32_t a[16], bb[16];
+      tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + c * 16, a);
+      tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + 64 + c * 16, bb);
+      tmem_ld_wait();
+      uint32_t w1[8], w2[8];
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        float y1[2], y2[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const float x1 = __uint_as_float(a[e + u]) * p.scale, x2 = __uint_as_float(bb[e + u]) * p.scale;
+          if (cs) {
+            const int i = c * 16 + e + u;
+            y1[u] = x1 * cs[i] + x2 * sn[i];
+            y2[u] = x2 * cs[i] - x1 * sn[i];
+          } else {
+            y1[u] = x1;
+            y2[u] = x2;
+          }
+        }
+        w1[e >> 1] = pack_bf16x2(y1[0], y1[1]);
+        w2[e >> 1] = pack_bf16x2(y2[0], y2[1]);
+      }
+      if (store) {
+        reinterpret_cast<uint4*>(kr + c * 16)[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+        reinterpret_cast<uint4*>(kr + c * 16)[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
+        reinterpret_cast<uint4*>(kr + 64 + c * 16)[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+        reinterpret_cast<uint4*>(kr + 64 + c * 16)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+      }
+    }
+  } else {
+    __nv_bfloat16* vr = p.dV + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
+#pragma unroll
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c = (qg - 2) * 4 + cc;
+      uint32_t v[16];
+      tmem_ld_32x32b_x16(tmem + lane_base + C::C_DV + c * 16, v);
+      tmem_ld_wait();
+      uint32_t w[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+      if (store) {
+        reinterpret_cast<uint4*>(vr + c * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        reinterpret_cast<uint4*>(vr + c * 16)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+  }
 }
 
 __global__ void __launch_bounds__(FB_THREADS, 1)
@@ -1004,21 +1069,9 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       bool issued = false;
       bool ok = mbar_wait(kv_full, 0) && !*abort_flag;
       if (!ok) record_error(p.err, 200);
-      // dP^T(it) = V dO^T into the dP^T columns
-      auto issue_dp = [&](int it) {
-        const int st = it & 1;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < FB_HD / 16; ++kk)
-          umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
-      };
-      // With skip_dq the dP^T columns are free once the gradient warps have
-      // signalled p_full, so dP^T(it + 1) is issued right behind dV, dK(it),
-      // before the wait for them to finish: the tensor pipe stays queued.
-      bool dp_early = false;
       for (int it = 0; it < n_it && ok; ++it) {
         const int st = it & 1;
-        if (!dp_early && (*abort_flag || !mbar_wait(&q_full[st], (it >> 1) & 1))) {
+        if (*abort_flag || !mbar_wait(&q_full[st], (it >> 1) & 1)) {
           record_error(p.err, 210 + (it & 63));
           ok = false;
           break;
@@ -1034,15 +1087,16 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         for (int kk = 0; kk < FB_HD / 16; ++kk)
           umma_bf16(tmem + C::C_S, dK_km + km_step(kk), dQ_km + st * kStage + km_step(kk), id_s, kk != 0);
         issued = true;
-        if (!dp_early) {
-          // dP^T columns hold dQ^T of the previous iteration until it is read out
-          if (it > 0 && !p.skip_dq && !mbar_wait(dq_empty, (it - 1) & 1)) {
-            record_error(p.err, 250 + (it & 15));
-            ok = false;
-            break;
-          }
-          issue_dp(it);
+        // dP^T columns hold dQ^T of the previous iteration until it is read out
+        if (it > 0 && !mbar_wait(dq_empty, (it - 1) & 1)) {
+          record_error(p.err, 250 + (it & 15));
+          ok = false;
+          break;
         }
+        // dP^T = V dO^T into the dP^T columns
+#pragma unroll
+        for (int kk = 0; kk < FB_HD / 16; ++kk)
+          umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
         umma_commit(s_full);
         if (*abort_flag || !mbar_wait(p_full, it & 1)) {
           record_error(p.err, 280 + (it & 15));
@@ -1062,23 +1116,11 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         }
         umma_commit(pdone);
         // dQ^T = K^T dS^T (K = 128 keys in 8 steps) into the dP^T columns
-        if (!p.skip_dq) {
 #pragma unroll
-          for (int kk = 0; kk < FB_BKV / 16; ++kk)
-            umma_bf16(tmem + C::C_DP, dK_mn + kk * kMn, ddSt_mn + kk * kMn, id_dq, kk != 0);
-        }
+        for (int kk = 0; kk < FB_BKV / 16; ++kk)
+          umma_bf16(tmem + C::C_DP, dK_mn + kk * kMn, ddSt_mn + kk * kMn, id_dq, kk != 0);
         umma_commit(mma_done);
         umma_commit(&q_empty[st]);
-        dp_early = false;
-        if (p.skip_dq && it + 1 < n_it) {
-          if (*abort_flag || !mbar_wait(&q_full[(it + 1) & 1], ((it + 1) >> 1) & 1)) {
-            record_error(p.err, 210 + ((it + 1) & 63));
-            ok = false;
-            break;
-          }
-          issue_dp(it + 1);
-          dp_early = true;
-        }
       }
       if (!ok) {
         *abort_flag = 1;
@@ -1133,7 +1175,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         ++h;
       }
       // dQ^T of the previous iteration first: its columns take this iteration's dP^T
-      if (it > 0 && !p.skip_dq) {
+      if (it > 0) {
         if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (it - 1) & 1)) {
           record_error(p.err, 400 + (it & 63));
           ok = false;
@@ -1214,7 +1256,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         tmem_st_32x32b_x8(tmem + lane_base + C::C_S + qg * FB_QW + hf * 16 + 8, ds);
         // dS^T row r, queries [32 qg + 16 hf, +16): sub-tile qg / 2, 16-byte chunks 4 (qg % 2) + 2 hf, +1
 #pragma unroll
-        for (int c2 = 0; c2 < 2 && !p.skip_dq; ++c2) {
+        for (int c2 = 0; c2 < 2; ++c2) {
           const int chunk = 4 * (qg & 1) + 2 * hf + c2;
           const int off = (qg >> 1) * C::SUB + r * 128 + ((chunk ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(sdSt + off) = make_uint4(ds[4 * c2], ds[4 * c2 + 1], ds[4 * c2 + 2], ds[4 * c2 + 3]);
@@ -1228,7 +1270,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       h_prev = hq;
       q0_prev = q0;
     }
-    if (ok && n_it > 0 && !p.skip_dq) {
+    if (ok && n_it > 0) {
       if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(mma_done, (n_it - 1) & 1)) {
         record_error(p.err, 450);
         ok = false;
@@ -1236,76 +1278,381 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         tc_fence_after();
         flush_dq(h_prev, q0_prev);
       }
-    } else if (ok && n_it > 0) {  // dK and dV only: their last products must be done
-      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(pdone, (n_it - 1) & 1)) {
-        record_error(p.err, 451);
-        ok = false;
-      } else {
-        tc_fence_after();
-      }
     }
     if (!ok) {
       *abort_flag = 1;
     } else if (n_it > 0) {
-      // tcgen05.ld is warp-collective: every lane loads, only keys inside the
-      // sequence store. Warps of query group 0 and 1 write dK (scaled,
-      // transposed RoPE; rotate-half pairs (i, i + 64) for i in [32 qg, 32 qg + 32)),
-      // groups 2 and 3 write dV columns [64 (qg - 2), 64 (qg - 2) + 64).
-      const bool store = key < p.s;
-      if (qg < 2) {
-        __nv_bfloat16* kr = p.dK + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
-        const float* cs = (p.rcos && store) ? p.rcos + (int64_t)key * (FB_HD / 2) : nullptr;
-        const float* sn = (p.rsin && store) ? p.rsin + (int64_t)key * (FB_HD / 2) : nullptr;
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {  // pairs (i, i + 64), 16 at a time
-          const int c = qg * 2 + cc;
-          uint32_t a[16], bb[16];
-          tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + c * 16, a);
-          tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + 64 + c * 16, bb);
-          tmem_ld_wait();
-          uint32_t w1[8], w2[8];
-#pragma unroll
-          for (int e = 0; e < 16; e += 2) {
-            float y1[2], y2[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const float x1 = __uint_as_float(a[e + u]) * p.scale, x2 = __uint_as_float(bb[e + u]) * p.scale;
-              if (cs) {
-                const int i = c * 16 + e + u;
-                y1[u] = x1 * cs[i] + x2 * sn[i];
-                y2[u] = x2 * cs[i] - x1 * sn[i];
-              } else {
-                y1[u] = x1;
-                y2[u] = x2;
-              }
-            }
-            w1[e >> 1] = pack_bf16x2(y1[0], y1[1]);
-            w2[e >> 1] = pack_bf16x2(y2[0], y2[1]);
-          }
-          if (store) {
-            reinterpret_cast<uint4*>(kr + c * 16)[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
-            reinterpret_cast<uint4*>(kr + c * 16)[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
-            reinterpret_cast<uint4*>(kr + 64 + c * 16)[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-            reinterpret_cast<uint4*>(kr + 64 + c * 16)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
-          }
+      fb_store_dkdv(tmem, lane_base, qg, key, row0, kvh, p);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+// ===========================================================================
+// dK and dV of the backward, key-major and pipelined (head_dim 128): the
+// key-major half of the deterministic split backward (dQ comes from
+// k_flash_bwd_dq). Same products as k_flash_bwd_tc without dQ^T, ordered for
+// a tensor core whose issue queue is only a few MMAs deep (the issuing thread
+// stalls until its MMAs are nearly done, so the issue order is the schedule):
+//   dP^T(n) = V dO^T         -> columns C_DP
+//   dV     += P^T(n) dO      (A = P^T, written by the gradient warps over the
+//                             S^T(n) scores they have read, as soon as their
+//                             exponentials are done: it does not wait for dP^T)
+//   S^T(n+1) = K Q^T         -> columns C_S (behind dV(n), which read them)
+//   dK     += dS^T(n) Q      (A = dS^T, written over the dP^T(n) values; the
+//                             gradient warps have had dV(n) and S^T(n+1) to
+//                             compute it)
+//   dP^T(n+1)                (behind dK(n), which read its columns)
+// Tensor memory is reused only behind the products that read it, which the
+// tensor core's in-order execution of one thread's MMAs makes safe, so the
+// issuing thread waits for nothing but operands: P^T(n), Q(n+1), dS^T(n),
+// dO(n+1). The gradient warps compute P^T(n+1) = exp(S^T - LSE) while dK(n)
+// and dP^T(n+1) run, and dS^T(n) while dV(n) and S^T(n+1) run. Each warp
+// writes a k-step's 16 queries of P^T (or dS^T) as 8 columns of bf16 pairs
+// inside the 32 score columns it has read itself: k-step kk at column
+// 32 (kk / 2) + 8 (kk % 2) of its buffer.
+// Tensor memory: dK [0,128), dV [128,256), S^T [256,384), dP^T [384,512).
+// Shared memory: K, V and two stages of Q and dO, 32 KB each (192 KB); Q and
+// dO of a stage have barriers of their own.
+// ===========================================================================
+namespace {
+
+struct FkCfg {
+  static constexpr int TILE = FbCfg::TILE;
+  static constexpr int SUB = FbCfg::SUB;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE;
+  static constexpr int OFF_Q = OFF_V + TILE;       // [2] stages
+  static constexpr int OFF_DO = OFF_Q + 2 * TILE;  // [2]
+  static constexpr int OFF_BAR = OFF_DO + 2 * TILE;
+  static constexpr int OFF_LD = OFF_BAR + 256;  // per gradient warp: 32 LSE' and 32 D values
+  static constexpr int SMEM = 1024 + OFF_LD + FB_GWARPS * 64 * 4;
+  static constexpr uint32_t C_DK = 0, C_DV = 128, C_S = 256, C_DP = 384;
+};
+
+// Column of k-step kk (16 queries) of P^T or dS^T inside its 128-column buffer.
+__device__ __forceinline__ uint32_t fk_a_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
+
+__global__ void __launch_bounds__(FB_THREADS, 1)
+    k_flash_bwd_kv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   FbParams p) {
+  using C = FkCfg;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = smem + C::OFF_K;
+  uint8_t* sV = smem + C::OFF_V;
+  uint8_t* sQ = smem + C::OFF_Q;
+  uint8_t* sdO = smem + C::OFF_DO;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  uint64_t* kv_full = bar + 0;
+  uint64_t* q_full = bar + 1;    // [2] Q of a stage landed
+  uint64_t* o_full = bar + 3;    // [2] dO of a stage landed
+  uint64_t* q_empty = bar + 5;   // [2] the stage's last products done
+  uint64_t* s_full = bar + 7;    // S^T(n) done
+  uint64_t* p_ready = bar + 8;   // P^T(n) written by every gradient warp
+  uint64_t* dp_full = bar + 9;   // dP^T(n) done
+  uint64_t* ds_ready = bar + 10; // dS^T(n) written by every gradient warp
+  uint64_t* kv_done = bar + 11;  // every product done
+  uint64_t* drain = bar + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 13);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bar + 14);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kvb = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
+  const int group = p.H / p.Hkv;
+  const int kv0 = kvb * FB_BKV;
+  const int row0 = b * p.s;
+  const int nqb = (p.s + FB_BQ - 1) / FB_BQ;
+  const int qb_first = kv0 / FB_BQ;
+  const int per_head = nqb - qb_first;
+  const int n_it = group * per_head;
+
+  if (threadIdx.x == 0) {
+    mbar_init(kv_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&o_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+    }
+    mbar_init(s_full, 1);
+    mbar_init(p_ready, FB_GWARPS);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_ready, FB_GWARPS);
+    mbar_init(kv_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int q_last[2] = {-1, -1};  // parity of the last loads into each stage
+      bool ok = true;
+      mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
+      for (int c = 0; c < 2; ++c) {
+        tma_load_2d(sK + c * C::SUB, &tmK, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+        tma_load_2d(sV + c * C::SUB, &tmV, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+      }
+      int h = kvh * group, qb = qb_first;  // head and query block of iteration it
+      for (int it = 0; it < n_it; ++it) {
+        const int st = it & 1;
+        const uint32_t ph = (it >> 1) & 1;
+        const int q0 = qb * FB_BQ, hq = h;
+        if (++qb == nqb) {
+          qb = qb_first;
+          ++h;
         }
-      } else {
-        __nv_bfloat16* vr = p.dV + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
+        if (*abort_flag || !mbar_wait(&q_empty[st], ph ^ 1)) {
+          record_error(p.err, 100 + (it & 63));
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&q_full[st], C::TILE);
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sQ + st * C::TILE + c * C::SUB, &tmQ, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
+        mbar_arrive_expect_tx(&o_full[st], C::TILE);
+        for (int c = 0; c < 2; ++c)
+          tma_load_2d(sdO + st * C::TILE + c * C::SUB, &tmO, &o_full[st], hq * FB_HD + c * 64, row0 + q0);
+        q_last[st] = (int)ph;
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        if (!mbar_wait(kv_full, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        for (int s2 = 0; s2 < 2; ++s2)
+          if (q_last[s2] >= 0 && (!mbar_wait(&q_full[s2], (uint32_t)q_last[s2]) ||
+                                  !mbar_wait(&o_full[s2], (uint32_t)q_last[s2])))
+            record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      constexpr uint32_t id_s = idesc_bf16_f32(FB_BKV, FB_BQ, false, false);  // keys x queries, K = hd
+      constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, FB_HD, false, true);  // keys x hd, K = queries (A in TMEM)
+      const uint64_t dK_km = sdesc_sw128(smem_u32(sK), 16, 1024), dV_km = sdesc_sw128(smem_u32(sV), 16, 1024);
+      const uint64_t dQ_km = sdesc_sw128(smem_u32(sQ), 16, 1024), dO_km = sdesc_sw128(smem_u32(sdO), 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), C::SUB, 1024), dO_mn = sdesc_sw128(smem_u32(sdO), C::SUB, 1024);
+      constexpr uint32_t kStage = C::TILE >> 4, kMn = 2048 >> 4;  // one stage; 16 rows of a 128-byte-row tile
+      bool issued = false;
+      bool ok = mbar_wait(kv_full, 0) && !*abort_flag;
+      if (!ok) record_error(p.err, 200);
+      // S^T(n) = K Q^T into the S^T columns, once Q(n) has landed
+      auto issue_s = [&](int n) -> bool {
+        const int st = n & 1;
+        if (*abort_flag || !mbar_wait(&q_full[st], (n >> 1) & 1)) return false;
+        tc_fence_after();
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int c = (qg - 2) * 4 + cc;
-          uint32_t v[16];
-          tmem_ld_32x32b_x16(tmem + lane_base + C::C_DV + c * 16, v);
-          tmem_ld_wait();
-          uint32_t w[8];
+        for (int kk = 0; kk < FB_HD / 16; ++kk)
+          umma_bf16(tmem + C::C_S, dK_km + km_step(kk), dQ_km + st * kStage + km_step(kk), id_s, kk != 0);
+        umma_commit(s_full);
+        issued = true;
+        return true;
+      };
+      // dP^T(n) = V dO^T into the dP^T columns, once dO(n) has landed
+      auto issue_dp = [&](int n) -> bool {
+        const int st = n & 1;
+        if (*abort_flag || !mbar_wait(&o_full[st], (n >> 1) & 1)) return false;
+        tc_fence_after();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
-          if (store) {
-            reinterpret_cast<uint4*>(vr + c * 16)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-            reinterpret_cast<uint4*>(vr + c * 16)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-          }
+        for (int kk = 0; kk < FB_HD / 16; ++kk)
+          umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
+        umma_commit(dp_full);
+        issued = true;
+        return true;
+      };
+      if (ok && !(issue_s(0) && issue_dp(0))) {
+        record_error(p.err, 210);
+        ok = false;
+      }
+      for (int n = 0; n < n_it && ok; ++n) {
+        const int st = n & 1;
+        const bool acc0 = n > 0;
+        // dV += P^T(n) dO(n): K = 128 queries in 8 steps
+        if (*abort_flag || !mbar_wait(p_ready, n & 1)) {
+          record_error(p.err, 220 + (n & 15));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < FB_BQ / 16; ++kk)
+          umma_bf16_ts(tmem + C::C_DV, tmem + C::C_S + fk_a_col(kk), dO_mn + st * kStage + kk * kMn, id_kv,
+                       acc0 || kk > 0);
+        if (n + 1 < n_it && !issue_s(n + 1)) {
+          record_error(p.err, 240 + (n & 15));
+          ok = false;
+          break;
+        }
+        // dK += dS^T(n) Q(n)
+        if (*abort_flag || !mbar_wait(ds_ready, n & 1)) {
+          record_error(p.err, 260 + (n & 15));
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < FB_BQ / 16; ++kk)
+          umma_bf16_ts(tmem + C::C_DK, tmem + C::C_DP + fk_a_col(kk), dQ_mn + st * kStage + kk * kMn, id_kv,
+                       acc0 || kk > 0);
+        umma_commit(&q_empty[st]);
+        if (n + 1 < n_it && !issue_dp(n + 1)) {
+          record_error(p.err, 280 + (n & 15));
+          ok = false;
+          break;
         }
       }
+      if (ok) umma_commit(kv_done);
+      if (!ok) {
+        *abort_flag = 1;
+        if (issued) {
+          umma_commit(drain);
+          if (!mbar_wait(drain, 0)) record_error(p.err, DEV_TIMEOUT_TEARDOWN);
+        }
+      }
+    }
+  } else {
+    // ---------------- gradient warps (2 .. 2 + FB_GWARPS) ----------------
+    // Warp w owns tensor-memory lane quarter w mod 4 (32 key rows) and query
+    // columns [32 qg, 32 qg + 32) of each block (k-steps 2 qg and 2 qg + 1).
+    const int qg = (warp - 2) >> 2;
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key row == tensor-memory lane
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const float sl2 = p.scale * 1.4426950408889634f;
+    const int key = kv0 + r;
+    // LSE' = LSE log2 e and D of this warp's 32 queries: lane i fetches
+    // query i's pair one iteration ahead; the warp's shared slot hands them
+    // to every lane (broadcast reads)
+    float* sld = reinterpret_cast<float*>(smem + C::OFF_LD) + (warp - 2) * 64;
+    auto fetch = [&](int hq_, int q0_, float& l, float& d) {
+      const int q = q0_ + qg * FB_QW + lane;
+      const int64_t i = ((int64_t)b * p.H + hq_) * p.s + q;
+      l = q < p.s ? __ldg(p.LSE + i) * 1.4426950408889634f : 0.f;
+      d = q < p.s ? __ldg(p.Dv + i) : 0.f;
+    };
+    const uint32_t s_cols = tmem + lane_base + C::C_S + qg * FB_QW;
+    const uint32_t dp_cols = tmem + lane_base + C::C_DP + qg * FB_QW;
+    bool ok = true;
+
+    int h = kvh * group, qb = qb_first;  // head and query block of iteration n
+    float pl, pd;
+    fetch(h, qb * FB_BQ, pl, pd);
+    for (int n = 0; n < n_it; ++n) {
+      const int q0 = qb * FB_BQ;
+      if (++qb == nqb) {
+        qb = qb_first;
+        ++h;
+      }
+      __syncwarp();
+      sld[lane] = pl;
+      sld[32 + lane] = pd;
+      __syncwarp();
+      if (n + 1 < n_it) fetch(h, qb * FB_BQ, pl, pd);
+      const int qc = q0 + qg * FB_QW;  // first query of this warp's columns
+      // Only blocks that touch the diagonal or a sequence end need the mask.
+      const bool need_mask = (qc < kv0 + FB_BKV) || (q0 + FB_BQ > p.s) || (kv0 + FB_BKV > p.s);
+      // P^T(n) = exp2(S^T sl2 - LSE'): this warp's 32 queries of key row r,
+      // kept in fp32 for dS^T and written as bf16 pairs over the scores
+      float pf[32];
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(s_full, n & 1)) {
+        record_error(p.err, 300 + (n & 63));
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        uint32_t sv[32];
+        tmem_ld_32x32b_x32(s_cols, sv);
+        tmem_ld_wait();
+        auto probs = [&](auto mask_tag) {
+          constexpr bool MASK = decltype(mask_tag)::value;
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 a4 = reinterpret_cast<const float4*>(sld)[i4];
+            const float lv[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int i = 4 * i4 + u, qi = qc + i;
+              const bool vis = !MASK || (key <= qi && qi < p.s && key < p.s);
+              pf[i] = vis ? ex2(fmaf(__uint_as_float(sv[i]), sl2, -lv[u])) : 0.f;
+            }
+          }
+        };
+        if (need_mask)
+          probs(std::true_type{});
+        else
+          probs(std::false_type{});
+        uint32_t pp[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) pp[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
+        tmem_st_32x32b_x8(s_cols, *reinterpret_cast<const uint32_t(*)[8]>(pp));
+        tmem_st_32x32b_x8(s_cols + 8, *reinterpret_cast<const uint32_t(*)[8]>(pp + 8));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(p_ready);
+      }
+      // dS^T(n) = P^T (dP^T - D), bf16 pairs over the dP^T values
+      if (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(dp_full, n & 1)) {
+        record_error(p.err, 340 + (n & 63));
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      {
+        uint32_t dv[32], ds[16];
+        tmem_ld_32x32b_x32(dp_cols, dv);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 d4 = reinterpret_cast<const float4*>(sld + 32)[e4];
+          const float dvv[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int u = 0; u < 4; u += 2) {
+            const int e = 4 * e4 + u;
+            ds[e >> 1] = pack_bf16x2(pf[e] * (__uint_as_float(dv[e]) - dvv[u]),
+                                     pf[e + 1] * (__uint_as_float(dv[e + 1]) - dvv[u + 1]));
+          }
+        }
+        tmem_st_32x32b_x8(dp_cols, *reinterpret_cast<const uint32_t(*)[8]>(ds));
+        tmem_st_32x32b_x8(dp_cols + 8, *reinterpret_cast<const uint32_t(*)[8]>(ds + 8));
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ds_ready);
+      }
+    }
+    if (ok && (__any_sync(0xffffffffu, *abort_flag) || !mbar_wait_warp(kv_done, 0))) {
+      record_error(p.err, 451);
+      ok = false;
+    }
+    if (!ok) {
+      *abort_flag = 1;
+    } else {
+      tc_fence_after();
+      fb_store_dkdv(tmem, lane_base, qg, key, row0, kvh, p);
     }
   }
 
@@ -1643,13 +1990,15 @@ int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* err) {
 
 // Backward with head_dim 128 on the tensor cores. a.dvec must already hold
 // D = rowsum(dO * O) and, unless skip_dq, a.dq_acc must be zeroed; the caller
-// casts dQ. skip_dq: dK and dV only (dQ from attention_bwd_dq_tc).
+// casts dQ. skip_dq: dK and dV only, by the pipelined key-major kernel (dQ
+// from attention_bwd_dq_tc); otherwise the fused kernel, dQ by reductions.
 int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err, bool skip_dq) {
   using C = FbCfg;
   if (a.hd != FB_HD) return MT_ERR_CONFIG;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(k_flash_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_flash_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
+        cudaFuncSetAttribute(k_flash_bwd_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, FkCfg::SMEM) != cudaSuccess)
       return MT_ERR_CUDA;
     attr = true;
   }
@@ -1662,9 +2011,12 @@ int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err, bool ski
     return MT_ERR_ARG;
   const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
-             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0, skip_dq ? 1 : 0};
+             a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
-  k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
+  if (skip_dq)
+    k_flash_bwd_kv<<<grid, FB_THREADS, FkCfg::SMEM, st>>>(mq, mk, mv, mo, p);
+  else
+    k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
 

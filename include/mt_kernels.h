@@ -202,14 +202,15 @@ int mt_k_gemm_variant(int variant);
 int mt_k_attn_fwd_variant(int variant);
 
 /* Selects the form of the tcgen05 attention backward (mt_k_attn_bwd_tc and the
- * engine) in later calls: 0 automatic (the default: split from s = 16384 on,
- * where both forms time the same, fused below), 1 fused: one key-major
+ * engine) in later calls: 0 automatic (the default: split, deterministic and
+ * the faster form at every length measured), 1 fused: one key-major
  * kernel computes dK, dV and dQ, adding each key block's dQ into dq_acc with
  * fp32 reductions (their order, and so dQ's last bits, vary from run to run),
  * 2 split: the key-major kernel computes dK and dV only and a query-major
  * kernel sums dQ over the key blocks in tensor memory and writes each element
  * once (deterministic: the same inputs give the same bits; needs dq_acc
- * 16-byte aligned and ldqa a multiple of 4, MT_ERR_ARG otherwise). Returns
+ * 16-byte aligned and ldqa a multiple of 4, MT_ERR_ARG before any GPU work
+ * otherwise). Returns
  * the previous choice, or MT_ERR_ARG for another value (nothing changes). No
  * GPU work. */
 int mt_k_attn_bwd_variant(int variant);
