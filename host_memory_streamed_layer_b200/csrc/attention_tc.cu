@@ -1607,8 +1607,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         uint32_t pp[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) pp[e] = pack_bf16x2(pf[2 * e], pf[2 * e + 1]);
-        tmem_st_32x32b_x8(s_cols, *reinterpret_cast<const uint32_t(*)[8]>(pp));
-        tmem_st_32x32b_x8(s_cols + 8, *reinterpret_cast<const uint32_t(*)[8]>(pp + 8));
+        tmem_st_32x32b_x16(s_cols, pp);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1636,8 +1635,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
                                      pf[e + 1] * (__uint_as_float(dv[e + 1]) - dvv[u + 1]));
           }
         }
-        tmem_st_32x32b_x8(dp_cols, *reinterpret_cast<const uint32_t(*)[8]>(ds));
-        tmem_st_32x32b_x8(dp_cols + 8, *reinterpret_cast<const uint32_t(*)[8]>(ds + 8));
+        tmem_st_32x32b_x16(dp_cols, ds);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -1914,8 +1912,7 @@ __global__ void __launch_bounds__(FQ_THREADS, 1)
         }
         // keys [64 half + 32 c, +32) -> columns 64 half + 16 c .. + 16 (key k in column k / 2
         // within the half's 32 columns): scores this warp has already read
-        tmem_st_32x32b_x8(sb + 16 * c, *reinterpret_cast<const uint32_t(*)[8]>(ds));
-        tmem_st_32x32b_x8(sb + 16 * c + 8, *reinterpret_cast<const uint32_t(*)[8]>(ds + 8));
+        tmem_st_32x32b_x16(sb + 16 * c, ds);
       };
       if (j == n - 1) {
         chunk(0, std::true_type{});
