@@ -572,22 +572,23 @@ int attention_bwd_variant(int v) {
   return was;
 }
 
-int attention_bwd_kernels(int) { return g_bwd_variant == 1 ? 3 : 4; }
+int attention_bwd_kernels(int hd) { return (g_bwd_variant == 1 && hd == 128) ? 3 : 4; }
 
 int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
   if (a.b <= 0 || a.s <= 0) return MT_OK;
-  if (a.hd != 128) return MT_ERR_CONFIG;
+  if (a.hd != 128 && a.hd != 64) return MT_ERR_CONFIG;
   const int T = a.b * a.s;
   const int64_t nw = (int64_t)T * a.H;
   k_attn_bwd_pre<<<(int)((nw + 7) / 8), 256, 0, st>>>((const bf16*)a.o, (const bf16*)a.dout, a.ldo, a.dvec, T, a.s,
-                                                      a.H, 128);
+                                                      a.H, a.hd);
   // automatic: the deterministic split form, which is also the faster one at
   // every length measured (B200, 16 or 32 heads of 128: 746 against 832 us at
   // 8 x 2048, 2268 against 2671 at 4 x 4096, 7695 against 8979 at 16384);
   // its query-major kernel stores dq_acc four floats at a time
   const bool aligned = (reinterpret_cast<uintptr_t>(a.dq_acc) & 15) == 0 && a.ldqa % 4 == 0;
-  if (g_bwd_variant == 2 && !aligned) return MT_ERR_ARG;
-  const bool split = g_bwd_variant == 2 || (g_bwd_variant == 0 && aligned);
+  // head dim 64 has the split form only
+  if ((g_bwd_variant == 2 || a.hd == 64) && !aligned) return MT_ERR_ARG;
+  const bool split = g_bwd_variant == 2 || a.hd == 64 || (g_bwd_variant == 0 && aligned);
   if (split) {  // dK, dV without reductions; dQ written once per element by the query-major kernel
     int r = attention_bwd_tc_main(a, st, err, true);
     if (r == MT_OK) r = attention_bwd_dq_tc(a, st, err);
@@ -597,8 +598,8 @@ int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* err) {
     const int r = attention_bwd_tc_main(a, st, err, false);
     if (r != MT_OK) return r;
   }
-  const int64_t nthr = (int64_t)T * a.H * (128 / 8);
-  k_dq_cast<<<(int)((nthr + 255) / 256), 256, 0, st>>>(a.dq_acc, a.ldqa, (bf16*)a.dq, a.lddq, T, a.H, 128, a.s,
+  const int64_t nthr = (int64_t)T * a.H * (a.hd / 8);
+  k_dq_cast<<<(int)((nthr + 255) / 256), 256, 0, st>>>(a.dq_acc, a.ldqa, (bf16*)a.dq, a.lddq, T, a.H, a.hd, a.s,
                                                        a.rope_cos, a.rope_sin);
   return launch_status();
 }

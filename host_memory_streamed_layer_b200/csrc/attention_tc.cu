@@ -888,24 +888,26 @@ __device__ __forceinline__ uint32_t km_step(int kk) {
 
 // The CTA's dK and dV (tensor-memory columns C_DK and C_DV, fp32, one key
 // row per lane) out to global memory as bf16, by the 16 gradient warps.
+template <int HD>
 __device__ __forceinline__ void fb_store_dkdv(uint32_t tmem, uint32_t lane_base, int qg, int key, int row0,
                                               int kvh, const FbParams& p) {
+  constexpr int HALF = HD / 2;
   using C = FbCfg;
   // tcgen05.ld is warp-collective: every lane loads, only keys inside the
   // sequence store. Warps of query group 0 and 1 write dK (scaled,
-  // transposed RoPE; rotate-half pairs (i, i + 64) for i in [32 qg, 32 qg + 32)),
-  // groups 2 and 3 write dV columns [64 (qg - 2), 64 (qg - 2) + 64).
+  // transposed RoPE; rotate-half pairs (i, i + HD/2) for i in [HD/4 qg, HD/4 (qg + 1))),
+  // groups 2 and 3 write dV columns [HD/2 (qg - 2), HD/2 (qg - 1)).
   const bool store = key < p.s;
   if (qg < 2) {
-    __nv_bfloat16* kr = p.dK + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
-    const float* cs = (p.rcos && store) ? p.rcos + (int64_t)key * (FB_HD / 2) : nullptr;
-    const float* sn = (p.rsin && store) ? p.rsin + (int64_t)key * (FB_HD / 2) : nullptr;
+    __nv_bfloat16* kr = p.dK + (int64_t)(row0 + key) * p.lddkv + kvh * HD;
+    const float* cs = (p.rcos && store) ? p.rcos + (int64_t)key * (HALF) : nullptr;
+    const float* sn = (p.rsin && store) ? p.rsin + (int64_t)key * (HALF) : nullptr;
 #pragma unroll
-    for (int cc = 0; cc < 2; ++cc) {  // pairs (i, i + 64), 16 at a time
-      const int c = qg * 2 + cc;
+    for (int cc = 0; cc < HD / 64; ++cc) {  // pairs (i, i + HD/2), 16 at a time
+      const int c = qg * (HD / 64) + cc;
       uint32_t a[16], bb[16];
       tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + c * 16, a);
-      tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + 64 + c * 16, bb);
+      tmem_ld_32x32b_x16(tmem + lane_base + C::C_DK + HALF + c * 16, bb);
       tmem_ld_wait();
       uint32_t w1[8], w2[8];
 #pragma unroll
@@ -929,15 +931,15 @@ __device__ __forceinline__ void fb_store_dkdv(uint32_t tmem, uint32_t lane_base,
       if (store) {
         reinterpret_cast<uint4*>(kr + c * 16)[0] = make_uint4(w1[0], w1[1], w1[2], w1[3]);
         reinterpret_cast<uint4*>(kr + c * 16)[1] = make_uint4(w1[4], w1[5], w1[6], w1[7]);
-        reinterpret_cast<uint4*>(kr + 64 + c * 16)[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
-        reinterpret_cast<uint4*>(kr + 64 + c * 16)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
+        reinterpret_cast<uint4*>(kr + HALF + c * 16)[0] = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+        reinterpret_cast<uint4*>(kr + HALF + c * 16)[1] = make_uint4(w2[4], w2[5], w2[6], w2[7]);
       }
     }
   } else {
-    __nv_bfloat16* vr = p.dV + (int64_t)(row0 + key) * p.lddkv + kvh * FB_HD;
+    __nv_bfloat16* vr = p.dV + (int64_t)(row0 + key) * p.lddkv + kvh * HD;
 #pragma unroll
-    for (int cc = 0; cc < 4; ++cc) {
-      const int c = (qg - 2) * 4 + cc;
+    for (int cc = 0; cc < HD / 32; ++cc) {
+      const int c = (qg - 2) * (HD / 32) + cc;
       uint32_t v[16];
       tmem_ld_32x32b_x16(tmem + lane_base + C::C_DV + c * 16, v);
       tmem_ld_wait();
@@ -1282,7 +1284,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     if (!ok) {
       *abort_flag = 1;
     } else if (n_it > 0) {
-      fb_store_dkdv(tmem, lane_base, qg, key, row0, kvh, p);
+      fb_store_dkdv<128>(tmem, lane_base, qg, key, row0, kvh, p);
     }
   }
 
@@ -1325,8 +1327,9 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
 // ===========================================================================
 namespace {
 
+template <int HD>
 struct FkCfg {
-  static constexpr int TILE = FbCfg::TILE;
+  static constexpr int TILE = 128 * HD * 2;  // 128 rows x HD bf16 as HD / 64 sub-tiles of 64 columns
   static constexpr int SUB = FbCfg::SUB;
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + TILE;
@@ -1341,11 +1344,12 @@ struct FkCfg {
 // Column of k-step kk (16 queries) of P^T or dS^T inside its 128-column buffer.
 __device__ __forceinline__ uint32_t fk_a_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
+template <int HD>
 __global__ void __launch_bounds__(FB_THREADS, 1)
     k_flash_bwd_kv(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                    FbParams p) {
-  using C = FkCfg;
+  using C = FkCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem + C::OFF_K;
@@ -1411,9 +1415,9 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       int q_last[2] = {-1, -1};  // parity of the last loads into each stage
       bool ok = true;
       mbar_arrive_expect_tx(kv_full, 2 * C::TILE);
-      for (int c = 0; c < 2; ++c) {
-        tma_load_2d(sK + c * C::SUB, &tmK, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
-        tma_load_2d(sV + c * C::SUB, &tmV, kv_full, kvh * FB_HD + c * 64, row0 + kv0);
+      for (int c = 0; c < HD / 64; ++c) {
+        tma_load_2d(sK + c * C::SUB, &tmK, kv_full, kvh * HD + c * 64, row0 + kv0);
+        tma_load_2d(sV + c * C::SUB, &tmV, kv_full, kvh * HD + c * 64, row0 + kv0);
       }
       int h = kvh * group, qb = qb_first;  // head and query block of iteration it
       for (int it = 0; it < n_it; ++it) {
@@ -1430,11 +1434,11 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
           break;
         }
         mbar_arrive_expect_tx(&q_full[st], C::TILE);
-        for (int c = 0; c < 2; ++c)
-          tma_load_2d(sQ + st * C::TILE + c * C::SUB, &tmQ, &q_full[st], hq * FB_HD + c * 64, row0 + q0);
+        for (int c = 0; c < HD / 64; ++c)
+          tma_load_2d(sQ + st * C::TILE + c * C::SUB, &tmQ, &q_full[st], hq * HD + c * 64, row0 + q0);
         mbar_arrive_expect_tx(&o_full[st], C::TILE);
-        for (int c = 0; c < 2; ++c)
-          tma_load_2d(sdO + st * C::TILE + c * C::SUB, &tmO, &o_full[st], hq * FB_HD + c * 64, row0 + q0);
+        for (int c = 0; c < HD / 64; ++c)
+          tma_load_2d(sdO + st * C::TILE + c * C::SUB, &tmO, &o_full[st], hq * HD + c * 64, row0 + q0);
         q_last[st] = (int)ph;
       }
       if (!ok) {
@@ -1450,7 +1454,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       constexpr uint32_t id_s = idesc_bf16_f32(FB_BKV, FB_BQ, false, false);  // keys x queries, K = hd
-      constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, FB_HD, false, true);  // keys x hd, K = queries (A in TMEM)
+      constexpr uint32_t id_kv = idesc_bf16_f32(FB_BKV, HD, false, true);  // keys x hd, K = queries (A in TMEM)
       const uint64_t dK_km = sdesc_sw128(smem_u32(sK), 16, 1024), dV_km = sdesc_sw128(smem_u32(sV), 16, 1024);
       const uint64_t dQ_km = sdesc_sw128(smem_u32(sQ), 16, 1024), dO_km = sdesc_sw128(smem_u32(sdO), 16, 1024);
       const uint64_t dQ_mn = sdesc_sw128(smem_u32(sQ), C::SUB, 1024), dO_mn = sdesc_sw128(smem_u32(sdO), C::SUB, 1024);
@@ -1464,7 +1468,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         if (*abort_flag || !mbar_wait(&q_full[st], (n >> 1) & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < FB_HD / 16; ++kk)
+        for (int kk = 0; kk < HD / 16; ++kk)
           umma_bf16(tmem + C::C_S, dK_km + km_step(kk), dQ_km + st * kStage + km_step(kk), id_s, kk != 0);
         umma_commit(s_full);
         issued = true;
@@ -1476,7 +1480,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
         if (*abort_flag || !mbar_wait(&o_full[st], (n >> 1) & 1)) return false;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < FB_HD / 16; ++kk)
+        for (int kk = 0; kk < HD / 16; ++kk)
           umma_bf16(tmem + C::C_DP, dV_km + km_step(kk), dO_km + st * kStage + km_step(kk), id_s, kk != 0);
         umma_commit(dp_full);
         issued = true;
@@ -1650,7 +1654,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
       *abort_flag = 1;
     } else {
       tc_fence_after();
-      fb_store_dkdv(tmem, lane_base, qg, key, row0, kvh, p);
+      fb_store_dkdv<HD>(tmem, lane_base, qg, key, row0, kvh, p);
     }
   }
 
@@ -1685,8 +1689,9 @@ namespace {
 
 constexpr int FQ_THREADS = 320;  // producer, MMA, 8 gradient warps
 
+template <int HD>
 struct FqCfg {
-  static constexpr int TILE = 128 * 128 * 2;  // 32 KB: 128 rows x 128 bf16 as two 64-column sub-tiles
+  static constexpr int TILE = 128 * HD * 2;  // 128 rows x HD bf16 as HD / 64 sub-tiles of 64 columns
   static constexpr int SUB = 128 * 128;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_DO = TILE;
@@ -1709,14 +1714,14 @@ struct FqParams {
 
 // Tensor-memory column of the A operand (dS) for k-step kk of S buffer sb.
 __device__ __forceinline__ uint32_t fq_a_col(int sb, int kk) {
-  return FqCfg::C_S + 128u * sb + (kk < 4 ? 8u * kk : 64u + 8u * (kk - 4));
+  return FqCfg<128>::C_S + 128u * sb + (kk < 4 ? 8u * kk : 64u + 8u * (kk - 4));
 }
 
+template <int HD>
 __global__ void __launch_bounds__(FQ_THREADS, 1)
     k_flash_bwd_dq(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO, FqParams p) {
-  using C = FqCfg;
-  constexpr int HD = 128;
+  using C = FqCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem + C::OFF_Q;
@@ -1776,7 +1781,7 @@ __global__ void __launch_bounds__(FQ_THREADS, 1)
       int k_last[2] = {-1, -1}, v_last[2] = {-1, -1};
       bool ok = true;
       mbar_arrive_expect_tx(qd_full, 2 * C::TILE);
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < HD / 64; ++c) {
         tma_load_2d(sQ + c * C::SUB, &tmQ, qd_full, h * HD + c * 64, row0 + q0);
         tma_load_2d(sdO + c * C::SUB, &tmO, qd_full, h * HD + c * 64, row0 + q0);
       }
@@ -1788,10 +1793,10 @@ __global__ void __launch_bounds__(FQ_THREADS, 1)
           break;
         }
         mbar_arrive_expect_tx(&k_full[st], C::TILE);
-        for (int c = 0; c < 2; ++c) tma_load_2d(sK + st * C::TILE + c * C::SUB, &tmK, &k_full[st], kvh * HD + c * 64, row0 + j * 128);
+        for (int c = 0; c < HD / 64; ++c) tma_load_2d(sK + st * C::TILE + c * C::SUB, &tmK, &k_full[st], kvh * HD + c * 64, row0 + j * 128);
         k_last[st] = (int)ph;
         mbar_arrive_expect_tx(&v_full[st], C::TILE);
-        for (int c = 0; c < 2; ++c) tma_load_2d(sV + st * C::TILE + c * C::SUB, &tmV, &v_full[st], kvh * HD + c * 64, row0 + j * 128);
+        for (int c = 0; c < HD / 64; ++c) tma_load_2d(sV + st * C::TILE + c * C::SUB, &tmV, &v_full[st], kvh * HD + c * 64, row0 + j * 128);
         v_last[st] = (int)ph;
       }
       if (!ok) {
@@ -1932,11 +1937,11 @@ __global__ void __launch_bounds__(FQ_THREADS, 1)
       *abort_flag = 1;
     } else {
       tc_fence_after();
-      float* dst = p.dQacc + (int64_t)(row0 + qi) * p.ldqa + (int64_t)h * HD + 64 * half;
+      float* dst = p.dQacc + (int64_t)(row0 + qi) * p.ldqa + (int64_t)h * HD + (HD / 2) * half;
 #pragma unroll 1
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < HD / 64; ++c) {
         uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + C::C_DQ + 64u * half + 32u * c, v);  // warp-collective
+        tmem_ld_32x32b_x32(tmem + lane_base + C::C_DQ + (HD / 2) * half + 32u * c, v);  // warp-collective
         tmem_ld_wait();
         if (qi < p.s) {
 #pragma unroll
@@ -1959,62 +1964,81 @@ __global__ void __launch_bounds__(FQ_THREADS, 1)
 
 }  // namespace
 
-// dQ of the head_dim-128 backward by the query-major kernel: writes every
+// dQ of the tensor-core backward (head dim 64 or 128) by the query-major kernel: writes every
 // element of dq_acc's head columns once (scaled, before RoPE's transpose).
 // a.dvec must already hold D = rowsum(dO * O).
-int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* err) {
-  using C = FqCfg;
-  if (a.hd != 128) return MT_ERR_CONFIG;
-  if ((reinterpret_cast<uintptr_t>(a.dq_acc) & 15) || (a.ldqa % 4)) return MT_ERR_ARG;
+namespace {
+template <int HD>
+int launch_bwd_dq(const AttnArgs& a, cudaStream_t st, int* err) {
+  using C = FqCfg<HD>;
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(k_flash_bwd_dq, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
+    if (cudaFuncSetAttribute(k_flash_bwd_dq<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess)
       return MT_ERR_CUDA;
     attr = true;
   }
   const int64_t T = (int64_t)a.b * a.s;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * 128, T, a.ldqkv, 128) ||
-      !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * 128, T, a.ldqkv, 128) ||
-      !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * 128, T, a.ldqkv, 128) ||
-      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * 128, T, a.ldo, 128))
+  if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * HD, T, a.ldqkv, 128) ||
+      !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * HD, T, a.ldqkv, 128) ||
+      !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * HD, T, a.ldqkv, 128) ||
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * HD, T, a.ldo, 128))
     return MT_ERR_ARG;
   FqParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, a.s, a.H, a.Hkv, a.scale, err};
   dim3 grid((a.s + 127) / 128, a.H, a.b);
-  k_flash_bwd_dq<<<grid, FQ_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
+  k_flash_bwd_dq<HD><<<grid, FQ_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
   return launch_status();
 }
+}  // namespace
 
-// Backward with head_dim 128 on the tensor cores. a.dvec must already hold
+int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* err) {
+  if (a.hd != 64 && a.hd != 128) return MT_ERR_CONFIG;
+  if ((reinterpret_cast<uintptr_t>(a.dq_acc) & 15) || (a.ldqa % 4)) return MT_ERR_ARG;
+  return a.hd == 128 ? launch_bwd_dq<128>(a, st, err) : launch_bwd_dq<64>(a, st, err);
+}
+
+// Key-major part of the tensor-core backward. a.dvec must already hold
 // D = rowsum(dO * O) and, unless skip_dq, a.dq_acc must be zeroed; the caller
-// casts dQ. skip_dq: dK and dV only, by the pipelined key-major kernel (dQ
-// from attention_bwd_dq_tc); otherwise the fused kernel, dQ by reductions.
-int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err, bool skip_dq) {
-  using C = FbCfg;
-  if (a.hd != FB_HD) return MT_ERR_CONFIG;
+// casts dQ. skip_dq: dK and dV only, by the pipelined key-major kernel (head
+// dim 64 or 128; dQ from attention_bwd_dq_tc); otherwise the fused kernel,
+// dQ by reductions (head dim 128).
+namespace {
+// The key-major kernel for head dim HD: the pipelined dK/dV-only one
+// (skip_dq), or the fused one with dQ by reductions (HD = 128 only).
+template <int HD>
+int launch_bwd_key_major(const AttnArgs& a, cudaStream_t st, int* err, bool skip_dq) {
   static bool attr = false;
   if (!attr) {
-    if (cudaFuncSetAttribute(k_flash_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) != cudaSuccess ||
-        cudaFuncSetAttribute(k_flash_bwd_kv, cudaFuncAttributeMaxDynamicSharedMemorySize, FkCfg::SMEM) != cudaSuccess)
+    if ((HD == 128 && cudaFuncSetAttribute(k_flash_bwd_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           FbCfg::SMEM) != cudaSuccess) ||
+        cudaFuncSetAttribute(k_flash_bwd_kv<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, FkCfg<HD>::SMEM) !=
+            cudaSuccess)
       return MT_ERR_CUDA;
     attr = true;
   }
   const int64_t T = (int64_t)a.b * a.s;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * FB_HD, T, a.ldqkv, FB_BQ) ||
-      !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
-      !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * FB_HD, T, a.ldqkv, FB_BKV) ||
-      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * FB_HD, T, a.ldo, FB_BQ))
+  if (!make_tensor_map_2d_bf16(&mq, a.q, (int64_t)a.H * HD, T, a.ldqkv, FB_BQ) ||
+      !make_tensor_map_2d_bf16(&mk, a.k, (int64_t)a.Hkv * HD, T, a.ldqkv, FB_BKV) ||
+      !make_tensor_map_2d_bf16(&mv, a.v, (int64_t)a.Hkv * HD, T, a.ldqkv, FB_BKV) ||
+      !make_tensor_map_2d_bf16(&mo, a.dout, (int64_t)a.H * HD, T, a.ldo, FB_BQ))
     return MT_ERR_ARG;
   const bool vec = (a.s % 4 == 0) && ((reinterpret_cast<uintptr_t>(a.lse) | reinterpret_cast<uintptr_t>(a.dvec)) & 15) == 0;
   FbParams p{a.lse, a.dvec, a.dq_acc, a.ldqa, (__nv_bfloat16*)a.dk, (__nv_bfloat16*)a.dv, a.lddkv, a.s, a.H, a.Hkv,
              a.scale, a.rope_cos, a.rope_sin, err, vec ? 1 : 0};
   dim3 grid((a.s + FB_BKV - 1) / FB_BKV, a.Hkv, a.b);
   if (skip_dq)
-    k_flash_bwd_kv<<<grid, FB_THREADS, FkCfg::SMEM, st>>>(mq, mk, mv, mo, p);
+    k_flash_bwd_kv<HD><<<grid, FB_THREADS, FkCfg<HD>::SMEM, st>>>(mq, mk, mv, mo, p);
   else
-    k_flash_bwd_tc<<<grid, FB_THREADS, C::SMEM, st>>>(mq, mk, mv, mo, p);
+    k_flash_bwd_tc<<<grid, FB_THREADS, FbCfg::SMEM, st>>>(mq, mk, mv, mo, p);
   return launch_status();
+}
+}  // namespace
+
+int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* err, bool skip_dq) {
+  if (a.hd == 128) return launch_bwd_key_major<128>(a, st, err, skip_dq);
+  if (a.hd == 64 && skip_dq) return launch_bwd_key_major<64>(a, st, err, true);
+  return MT_ERR_CONFIG;
 }
 
 }  // namespace mt

@@ -327,10 +327,10 @@ int attn(mt_ctx* c, AttnArgs& a, bool bwd) {
     e1 = timing_event(c);
     if (e0) cudaEventRecord(e0, c->s_comp);
   }
-  int r = bwd ? (a.hd == 128 ? attention_bwd_tc(a, c->s_comp, c->d_err) : attention_bwd(a, c->s_comp))
+  int r = bwd ? attention_bwd_tc(a, c->s_comp, c->d_err)
               : attention_fwd_tc(a, c->s_comp, c->d_err);
   if (r != MT_OK) return set_err(c, r, "attention launch failed");
-  c->launches += bwd ? (a.hd == 128 ? attention_bwd_kernels(a.s) : 3) : 1;
+  c->launches += bwd ? attention_bwd_kernels(a.hd) : 1;
   if (timing && e0 && e1) {
     cudaEventRecord(e1, c->s_comp);
     // causal attention: QK^T and PV over the visible half, per query head

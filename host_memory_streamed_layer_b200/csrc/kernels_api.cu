@@ -154,7 +154,7 @@ extern "C" int mt_k_attn_bwd_tc(const void* q, const void* k, const void* v, int
   if ((cos_tab == nullptr) != (sin_tab == nullptr)) return MT_ERR_ARG;
   if (!q || !k || !v || !o || !dout || !lse || !dvec || !dq_acc || !dq || !dk || !dv) return MT_ERR_ARG;
   if (b < 0 || s < 0 || H <= 0 || Hkv <= 0 || (H % Hkv)) return MT_ERR_ARG;
-  if (hd != 128) return MT_ERR_CONFIG;
+  if (hd != 128 && hd != 64) return MT_ERR_CONFIG;
   if (!al16(q) || !al16(k) || !al16(v) || !al16(o) || !al16(dout) || !al16(dq_acc) || (ldqkv % 8) || (ldo % 8) ||
       (ldqa % 4) || (lddq % 4) || (lddkv % 8) || ldqa < (int64_t)H * hd)
     return MT_ERR_ARG;

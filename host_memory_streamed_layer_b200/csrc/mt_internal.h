@@ -94,18 +94,20 @@ int attention_fwd(const AttnArgs& a, cudaStream_t st);
 int attention_bwd(const AttnArgs& a, cudaStream_t st);
 // Forward on the tcgen05 tensor cores (same outputs as attention_fwd).
 int attention_fwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
-// Backward on the tcgen05 tensor cores for head_dim 128 (same outputs as
-// attention_bwd); _main is the tensor-core kernel alone.
+// Backward on the tcgen05 tensor cores for head_dim 64 or 128 (same outputs
+// as attention_bwd); _main is the key-major tensor-core kernel alone.
 int attention_bwd_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
 int attention_bwd_tc_main(const AttnArgs& a, cudaStream_t st, int* dev_err, bool skip_dq);
-// dQ of the head_dim-128 backward by the query-major kernel (no reductions).
+// dQ of the tensor-core backward (head dim 64 or 128) by the query-major
+// kernel (no reductions).
 int attention_bwd_dq_tc(const AttnArgs& a, cudaStream_t st, int* dev_err);
-// Backward form for head_dim 128 in later calls (0 automatic, 1 fused: dQ by
-// reductions inside the key-major kernel, 2 split: dK/dV by the key-major
-// kernel, dQ by the query-major one, deterministic); returns the previous one.
+// Backward form in later calls (0 automatic, 1 fused: dQ by reductions
+// inside the key-major kernel, head dim 128 only, 2 split: dK/dV by the
+// key-major kernel, dQ by the query-major one, deterministic; head dim 64 is
+// always split); returns the previous one.
 int attention_bwd_variant(int v);
-// Kernels one head_dim-128 backward launches in the current form.
-int attention_bwd_kernels(int s);
+// Kernels one tensor-core backward of head dim hd launches in the current form.
+int attention_bwd_kernels(int hd);
 
 // Mixture-of-experts MLP (moe.cu). Router: logits [T, E], the topk experts
 // idx [T, k] and their gates [T, k] of the bf16 MLP input w [T, d] and router

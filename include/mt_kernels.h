@@ -144,10 +144,13 @@ int mt_k_attn_bwd(const void* q, const void* k, const void* v, int64_t ldqkv, co
                   const float* sin_tab, void* stream);
 
 /* The same backward (same arguments and outputs as mt_k_attn_bwd) on the
- * tcgen05 tensor cores, head_dim 128 only (MT_ERR_CONFIG otherwise): one CTA
+ * tcgen05 tensor cores, head_dim 64 or 128 (MT_ERR_CONFIG otherwise): one CTA
  * per 128-key block accumulates dK and dV in tensor memory over the group's
- * query heads and 128-query blocks; dQ goes through the fp32 accumulator.
- * q, k, v, o, dout 16-byte aligned; dev_err as for mt_k_attn_fwd_tc. */
+ * query heads and 128-query blocks; dQ goes through the fp32 accumulator,
+ * summed there by the query-major kernel (split form; head_dim 64 always) or
+ * by reductions (fused form, head_dim 128; mt_k_attn_bwd_variant).
+ * q, k, v, o, dout, dq_acc 16-byte aligned, ldqa a multiple of 4; dev_err as
+ * for mt_k_attn_fwd_tc. */
 int mt_k_attn_bwd_tc(const void* q, const void* k, const void* v, int64_t ldqkv, const void* o, const void* dout,
                      int64_t ldo, const float* lse, float* dvec, float* dq_acc, int64_t ldqa, void* dq, int64_t lddq,
                      void* dk, void* dv, int64_t lddkv, int b, int s, int H, int Hkv, int hd, const float* cos_tab,

@@ -237,8 +237,8 @@ def _bwd_form(mt, impl):
 @pytest.mark.parametrize("impl", ["mma", "tc", "tc_split"])
 @pytest.mark.parametrize("hd,H,Hkv,s,b", ATTN)
 def test_attention_bwd(hd, H, Hkv, s, b, impl):
-    if impl != "mma" and hd != 128:
-        pytest.skip("tensor-core backward is for head_dim 128")
+    if impl == "tc" and hd != 128:
+        pytest.skip("the fused tensor-core backward is for head_dim 128")
     mt = _mt()
     if impl != "mma":
         was = mt.mt_k_attn_bwd_variant(_bwd_form(mt, impl))
@@ -250,13 +250,13 @@ def test_attention_bwd(hd, H, Hkv, s, b, impl):
         _attention_bwd_case(mt, hd, H, Hkv, s, b, impl)
 
 
-def test_split_attention_backward_is_bitwise_reproducible():
+@pytest.mark.parametrize("hd,H,Hkv,s,b", [(128, 8, 2, 1100, 2), (64, 4, 1, 700, 2)])
+def test_split_attention_backward_is_bitwise_reproducible(hd, H, Hkv, s, b):
     """The split form sums each dQ element in one fixed order (the query-major
     kernel's key-block loop) and dK, dV in tensor memory: two runs on the same
-    inputs give the same bits, at a shape with many key blocks per query
-    block and GQA."""
+    inputs give the same bits, at shapes with many key blocks per query
+    block and GQA, for both head dims."""
     mt = _mt()
-    hd, H, Hkv, s, b = 128, 8, 2, 1100, 2
     qkv, q, k, v, ld = _attn_inputs(hd, H, Hkv, s, b, 3)
     T = b * s
     do = bf(np.random.default_rng(4).normal(size=(T, H * hd)))
@@ -372,8 +372,8 @@ def _qkv_rope_case(mt, hd, H, Hkv, s, b):
 def test_attention_bwd_returns_pre_rope_gradients(hd, H, Hkv, s, b, impl):
     """With the RoPE tables the backward returns dL/d(pre-RoPE q, k): the
     oracle's attention backward followed by its rope_bwd."""
-    if impl != "mma" and hd != 128:
-        pytest.skip("tensor-core backward is for head_dim 128")
+    if impl == "tc" and hd != 128:
+        pytest.skip("the fused tensor-core backward is for head_dim 128")
     mt = _mt()
     was = mt.mt_k_attn_bwd_variant(_bwd_form(mt, impl))
     try:
