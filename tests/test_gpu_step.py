@@ -130,15 +130,17 @@ def test_serialized_and_no_update_modes():
     assert max(rel(Gn[k], Gb[k]) for k in Gb) <= 1e-3
 
 
-def test_split_attention_backward_makes_steps_bitwise_reproducible():
-    """With the split attention backward no reduction of the step depends on
-    timing: the GEMMs have no split-K, the normalisation, embedding and
-    loss reductions run in a fixed order, and dQ is summed in the query-major
-    kernel. Two pipelined runs and a serialized run (one stream) of two steps
-    then give the same bits: losses, every gradient and the updated master."""
+@pytest.mark.parametrize("name", ["hd128", "tiny"])
+def test_default_steps_are_bitwise_reproducible(name):
+    """With the split attention backward (the automatic form, and the only one
+    for head dim 64) no reduction of the step depends on timing: the GEMMs
+    have no split-K, the normalisation, embedding and loss reductions run in
+    a fixed order, and dQ is summed in the query-major kernel. Two pipelined
+    runs and a serialized run (one stream) of two steps then give the same
+    bits: losses, every gradient and the updated master."""
     arena, mt = _libs()
-    shape = SHAPES["hd128"]
-    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT)
+    shape = SHAPES[name]
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_AUTO)
     try:
         runs = [run_gpu(shape, 2), run_gpu(shape, 2), run_gpu(shape, 2, flags=mt.MT_FLAG_SERIALIZE)]
     finally:
