@@ -1299,7 +1299,7 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
 }  // namespace
 
 // ===========================================================================
-// dK and dV of the backward, key-major and pipelined (head_dim 128): the
+// dK and dV of the backward, key-major and pipelined (head_dim 64 or 128): the
 // key-major half of the deterministic split backward (dQ comes from
 // k_flash_bwd_dq). Same products as k_flash_bwd_tc without dQ^T, ordered for
 // a tensor core whose issue queue is only a few MMAs deep (the issuing thread
@@ -1321,9 +1321,11 @@ __global__ void __launch_bounds__(FB_THREADS, 1)
 // writes a k-step's 16 queries of P^T (or dS^T) as 8 columns of bf16 pairs
 // inside the 32 score columns it has read itself: k-step kk at column
 // 32 (kk / 2) + 8 (kk % 2) of its buffer.
-// Tensor memory: dK [0,128), dV [128,256), S^T [256,384), dP^T [384,512).
-// Shared memory: K, V and two stages of Q and dO, 32 KB each (192 KB); Q and
-// dO of a stage have barriers of their own.
+// Tensor memory: dK [0,hd), dV [128,128+hd), S^T [256,384), dP^T [384,512).
+// Shared memory: K, V and two stages of Q and dO, 128 x hd bf16 each (192 KB
+// at hd 128); Q and dO of a stage have barriers of their own. Each gradient
+// warp also has a 256-byte slot through which its lanes hand the block's LSE
+// and D values (fetched one block ahead, one query per lane) to every lane.
 // ===========================================================================
 namespace {
 
