@@ -1,7 +1,7 @@
 """Micro-benchmark of single hot-path kernels through the C ABI.
 
     python -m host_memory_streamed_layer_b200.kernel_bench gemm [--shape NAME] [--iters N]
-    python -m host_memory_streamed_layer_b200.kernel_bench attn [--fwd-only] [--iters N] [--attn-shape B,S,H]
+    python -m host_memory_streamed_layer_b200.kernel_bench attn [--fwd-only] [--iters N] [--attn-shape B,S,H[,HD]]
     python -m host_memory_streamed_layer_b200.kernel_bench rmsnorm_bwd [--iters N]
     python -m host_memory_streamed_layer_b200.kernel_bench elementwise [--iters N]
 
@@ -13,8 +13,8 @@ llama-1.3b workload (T = 8 x 2048 tokens, d 2048, FFN 5504, 16 heads); for
 the GEMMs, --workload NAME takes every GEMM shape of that workload's training
 step instead, and each result line carries the shape's launches per step
 (so per-shape ncu figures can be weighted into a per-launch step average);
-for attention, --attn-shape B,S,H sets sequences, length and heads (head dim
-128, as many KV heads as query heads).
+for attention, --attn-shape B,S,H[,HD] sets sequences, length, heads and head
+dim (128 unless given; as many KV heads as query heads).
 """
 from __future__ import annotations
 
@@ -113,35 +113,35 @@ def bench_gemm(names, iters, warmup, table=None):
     return out
 
 
-def bench_attn(iters, warmup, fwd_only, impl="tc", B=B, S=S, H=H):
+def bench_attn(iters, warmup, fwd_only, impl="tc", B=B, S=S, H=H, hd=HD):
     st = torch.cuda.current_stream().cuda_stream
     T = B * S
-    ld = 3 * H * HD
+    ld = 3 * H * hd
     qkv = torch.randn(T, ld, device="cuda").to(torch.bfloat16)
-    o = torch.empty(T, H * HD, device="cuda", dtype=torch.bfloat16)
+    o = torch.empty(T, H * hd, device="cuda", dtype=torch.bfloat16)
     lse = torch.empty(B, H, S, device="cuda")
     p = qkv.data_ptr()
-    pk, pv = p + 2 * H * HD, p + 4 * H * HD
+    pk, pv = p + 2 * H * hd, p + 4 * H * hd
     if impl == "tc":
-        fwd = lambda: mt.mt_k_attn_fwd_tc(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, H, HD,  # noqa
+        fwd = lambda: mt.mt_k_attn_fwd_tc(p, pk, pv, ld, o.data_ptr(), H * hd, lse.data_ptr(), B, S, H, H, hd,  # noqa
                                           st)
     else:
-        fwd = lambda: mt.mt_k_attn_fwd(p, pk, pv, ld, o.data_ptr(), H * HD, lse.data_ptr(), B, S, H, H, HD, st)  # noqa
-    fl = 2.0 * B * H * S * S * HD
+        fwd = lambda: mt.mt_k_attn_fwd(p, pk, pv, ld, o.data_ptr(), H * hd, lse.data_ptr(), B, S, H, H, hd, st)  # noqa
+    fl = 2.0 * B * H * S * S * hd
     res = [{"kernel": f"attn_fwd_{impl}", "us": 0, "tflops": None}]
     sec = timed(fwd, iters, warmup)
     res[0].update(us=sec * 1e6, tflops=fl / sec / 1e12 if sec else None)
     if not fwd_only:
         fwd()
-        do = torch.randn(T, H * HD, device="cuda").to(torch.bfloat16)
+        do = torch.randn(T, H * hd, device="cuda").to(torch.bfloat16)
         dvec = torch.empty(B, H, S, device="cuda")
-        dqa = torch.empty(T, H * HD, device="cuda")
+        dqa = torch.empty(T, H * hd, device="cuda")
         dqkv = torch.empty(T, ld, device="cuda", dtype=torch.bfloat16)
         dp = dqkv.data_ptr()
         fn = mt.mt_k_attn_bwd_tc if impl == "tc" else mt.mt_k_attn_bwd
-        bwd = lambda: fn(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * HD, lse.data_ptr(),  # noqa
-                         dvec.data_ptr(), dqa.data_ptr(), H * HD, dp, ld, dp + 2 * H * HD,
-                         dp + 4 * H * HD, ld, B, S, H, H, HD, 0, 0, st)
+        bwd = lambda: fn(p, pk, pv, ld, o.data_ptr(), do.data_ptr(), H * hd, lse.data_ptr(),  # noqa
+                         dvec.data_ptr(), dqa.data_ptr(), H * hd, dp, ld, dp + 2 * H * hd,
+                         dp + 4 * H * hd, ld, B, S, H, H, hd, 0, 0, st)
         sec = timed(bwd, iters, warmup)
         res.append({"kernel": f"attn_bwd_{impl}", "us": sec * 1e6, "tflops": 2.5 * fl / sec / 1e12 if sec else None})
     return res
@@ -214,11 +214,12 @@ def main():
     ap.add_argument("--fwd-only", action="store_true")
     ap.add_argument("--impl", default="tc", choices=["tc", "mma"])
     ap.add_argument("--workload", default=None, help="GEMMs: every shape of this workload's training step")
-    ap.add_argument("--attn-shape", default=f"{B},{S},{H}", help="attention: sequences,length,heads")
+    ap.add_argument("--attn-shape", default=f"{B},{S},{H}",
+                    help="attention: sequences,length,heads[,head dim] (head dim 128 unless given)")
     ap.add_argument("--attn-variant", default="auto", choices=["auto", "one", "pingpong"],
                     help="attention forward kernel (head dim 128): automatic, one or two query tiles per CTA")
     ap.add_argument("--attn-bwd", default="auto", choices=["auto", "fused", "split"],
-                    help="attention backward (head dim 128): dQ by reductions, or the deterministic split")
+                    help="attention backward: dQ by reductions (head dim 128), or the deterministic split")
     a = ap.parse_args()
     if a.kernel == "gemm":
         table = None
@@ -228,14 +229,16 @@ def main():
         names = list(table or GEMMS) if a.shape == "all" else a.shape.split(",")
         res = bench_gemm(names, a.iters, a.warmup, table)
     elif a.kernel == "attn":
-        ab, as_, ah = (int(x) for x in a.attn_shape.split(","))
+        dims = [int(x) for x in a.attn_shape.split(",")]
+        ab, as_, ah = dims[:3]
+        ahd = dims[3] if len(dims) > 3 else HD
         mt.mt_k_attn_fwd_variant({"auto": mt.ATTN_AUTO, "one": mt.ATTN_ONE_TILE,
                                   "pingpong": mt.ATTN_PINGPONG}[a.attn_variant])
         mt.mt_k_attn_bwd_variant({"auto": mt.ATTN_BWD_AUTO, "fused": mt.ATTN_BWD_FUSED,
                                   "split": mt.ATTN_BWD_SPLIT}[a.attn_bwd])
-        res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl, ab, as_, ah)
+        res = bench_attn(a.iters, a.warmup, a.fwd_only, a.impl, ab, as_, ah, ahd)
         for r in res:
-            r["shape"] = dict(b=ab, s=as_, heads=ah, hd=HD)
+            r["shape"] = dict(b=ab, s=as_, heads=ah, hd=ahd)
     elif a.kernel == "elementwise":
         res = bench_elementwise(a.iters, a.warmup)
     else:
