@@ -82,8 +82,9 @@ ATTN_BWD_AUTO, ATTN_BWD_FUSED, ATTN_BWD_SPLIT = 0, 1, 2
 
 
 def mt_k_attn_bwd_variant(variant: int) -> int:
-    """Selects the head-dim-128 attention backward form for later calls
-    (fused dQ reductions, or the deterministic split); returns the previous."""
+    """Selects the tensor-core attention backward form for later calls:
+    automatic (the deterministic split), fused dQ reductions (head dim 128;
+    head dim 64 always runs split), or split; returns the previous choice."""
     rc = lib.mt_k_attn_bwd_variant(variant)
     if rc < 0:
         raise MTError(rc, "mt_k_attn_bwd_variant")
