@@ -364,10 +364,11 @@ int mt_get_routing(mt_ctx* ctx, int layer, int32_t* idx, size_t n);
  * after every check of the step has passed. The next step starts afresh (the
  * device error word is cleared at its start). With MT_FLAG_DEFER_UPDATES some
  * of this step's updates are still pending when it returns (see the flag).
- * Every reduction of a step runs in a fixed order (the attention backward in
- * its automatic, split form; mt_k_attn_bwd_variant), so the same arena,
- * tokens and labels give the same loss, gradients and parameters bit for bit,
- * pipelined or with MT_FLAG_SERIALIZE. */
+ * Every reduction of a step on one GPU runs in a fixed order (the attention
+ * backward in its automatic, split form; mt_k_attn_bwd_variant), so the same
+ * arena, tokens and labels give the same loss, gradients and parameters bit
+ * for bit, pipelined or with MT_FLAG_SERIALIZE (a sharded context adds the
+ * NCCL collectives' own summation order). */
 int mt_train_step(mt_ctx* ctx, const int32_t* tokens, const int32_t* labels, float* loss_out);
 
 /* Runs the updates that MT_FLAG_DEFER_UPDATES left pending, and returns when
