@@ -10,6 +10,7 @@
 #include <math.h>
 #include <stdlib.h>
 #include <string.h>
+#include <sys/mman.h>
 
 #include <chrono>
 #include <thread>
@@ -278,12 +279,32 @@ __attribute__((target("avx512f"))) void triad_avx512(float* a, const float* b, c
 }
 }  // namespace
 
+namespace {
+// Probe buffers allocated as the engine allocates its host state: anonymous
+// mappings advised onto transparent huge pages before their first touch.
+struct ProbeBuf {
+  void* p = nullptr;
+  size_t len = 0;
+  explicit ProbeBuf(size_t bytes) {
+    len = (bytes + (size_t(2) << 20) - 1) & ~((size_t(2) << 20) - 1);
+    void* got = mmap(nullptr, len, PROT_READ | PROT_WRITE, MAP_PRIVATE | MAP_ANONYMOUS, -1, 0);
+    if (got == MAP_FAILED) return;
+    madvise(got, len, MADV_HUGEPAGE);
+    p = got;
+  }
+  ~ProbeBuf() {
+    if (p) munmap(p, len);
+  }
+  ProbeBuf(const ProbeBuf&) = delete;
+  ProbeBuf& operator=(const ProbeBuf&) = delete;
+};
+}  // namespace
+
 extern "C" double mt_host_triad_gbs(size_t n, int threads) {
   if (n < (1u << 16)) return MT_ERR_ARG;
   if (threads <= 0) threads = std::max(1, (int)std::thread::hardware_concurrency() - 1);
-  float* a[3] = {};
-  for (auto& x : a)
-    if (posix_memalign(reinterpret_cast<void**>(&x), 64, n * 4)) x = nullptr;
+  ProbeBuf b0(n * 4), b1(n * 4), b2(n * 4);
+  float* a[3] = {static_cast<float*>(b0.p), static_cast<float*>(b1.p), static_cast<float*>(b2.p)};
   double best = 0;
   if (a[0] && a[1] && a[2]) {
     mt::ThreadPool pool(threads - 1);
@@ -309,18 +330,16 @@ extern "C" double mt_host_triad_gbs(size_t n, int threads) {
       best = std::max(best, 12.0 * n / sec / 1e9);
     }
   }
-  for (auto& x : a) free(x);
   return best > 0 ? best : MT_ERR_NOMEM;
 }
 
 extern "C" double mt_host_optimizer_gbs(size_t n, int threads) {
   if (n < (1u << 16)) return MT_ERR_ARG;
   if (threads <= 0) threads = std::max(1, (int)std::thread::hardware_concurrency() - 1);
-  float* a[4] = {};
-  uint16_t* pb = nullptr;
-  for (auto& x : a)
-    if (posix_memalign(reinterpret_cast<void**>(&x), 64, n * 4)) x = nullptr;
-  if (posix_memalign(reinterpret_cast<void**>(&pb), 64, n * 2)) pb = nullptr;
+  ProbeBuf b0(n * 4), b1(n * 4), b2(n * 4), b3(n * 4), b4(n * 2);
+  float* a[4] = {static_cast<float*>(b0.p), static_cast<float*>(b1.p), static_cast<float*>(b2.p),
+                 static_cast<float*>(b3.p)};
+  uint16_t* pb = static_cast<uint16_t*>(b4.p);
   double best = 0;
   if (a[0] && a[1] && a[2] && a[3] && pb) {
     mt::ThreadPool pool(threads - 1);
@@ -343,7 +362,5 @@ extern "C" double mt_host_optimizer_gbs(size_t n, int threads) {
       best = std::max(best, 30.0 * n / sec / 1e9);
     }
   }
-  for (auto& x : a) free(x);
-  free(pb);
   return best > 0 ? best : MT_ERR_NOMEM;
 }

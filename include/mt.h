@@ -490,7 +490,9 @@ int mt_get_stream(mt_ctx* ctx, void** stream);
  * arrays of n elements with `threads` threads (0 = all cores but one), best
  * of 3 passes, and returns GB/s counted as 30 bytes per element (read p, g,
  * m, v; write p, m, v and the bf16 copy). Allocates and frees its own host
- * buffers; no GPU needed. Returns a negative MT_ERR_* on failure. */
+ * buffers, on transparent huge pages where the host allows them, as the
+ * engine allocates its host state; no GPU needed. Returns a negative
+ * MT_ERR_* on failure. */
 double mt_host_optimizer_gbs(size_t n, int threads);
 
 /* Host DRAM ceiling independent of the optimizer: the STREAM triad
@@ -500,7 +502,8 @@ double mt_host_optimizer_gbs(size_t n, int threads);
  * write). The host AdamW's 30 bytes per parameter are judged against it
  * (intelligentliving.co, "Checkpointing, Manual Gradients, and CPU-Side
  * Optimizer Steps": CPU-side updates can become the slow step). Allocates
- * and frees its own host buffers; no GPU needed. Negative MT_ERR_* on failure. */
+ * and frees its own host buffers (huge pages where the host allows, like the
+ * engine's host state); no GPU needed. Negative MT_ERR_* on failure. */
 double mt_host_triad_gbs(size_t n, int threads);
 
 /* Applies pending deferred updates, waits for the context's streams, frees
