@@ -431,3 +431,36 @@ def test_expert_layer_layout_matches_the_oracle():
     # expert layers partition like dense ones: their arena and bf16 offsets agree (d % 128 == 0)
     p = mt.mt_shard_plan(cfg, 2, 1)
     assert p["layer_elems"] == per_layer and p["layer_end"] == per_layer
+
+
+def test_tensor_core_attention_backward_refusals_without_a_gpu():
+    """mt_k_attn_bwd_tc takes head dims 64 and 128 (MT_ERR_CONFIG otherwise)
+    and a dQ accumulator it can store four floats at a time (MT_ERR_ARG
+    otherwise), both refused before any device work; the form selector takes
+    0, 1 and 2 and returns the previous choice."""
+    mt = _mt()
+    from host_memory_streamed_layer_b200 import arena
+    buf = arena.aligned_empty(1 << 16)
+    p = buf.ctypes.data
+    b, s, H, Hkv = 1, 8, 2, 1
+
+    def call(hd, ldqa):
+        ld = (H + 2 * Hkv) * hd
+        return mt.mt_k_attn_bwd_tc(p, p, p, ld, p, p, H * hd, p, p, p, ldqa, p, ld, p, p, ld, b, s, H, Hkv, hd)
+    for hd in (32, 96, 256):
+        with pytest.raises(mt.MTError) as e:
+            call(hd, H * hd)
+        assert e.value.code == -2  # MT_ERR_CONFIG
+    for hd in (64, 128):
+        with pytest.raises(mt.MTError) as e:
+            call(hd, H * hd + 1)  # ldqa not a multiple of 4
+        assert e.value.code == -1  # MT_ERR_ARG
+    was = mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_SPLIT)
+    try:
+        assert mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_FUSED) == mt.ATTN_BWD_SPLIT
+        with pytest.raises(mt.MTError) as e:
+            mt.mt_k_attn_bwd_variant(3)
+        assert e.value.code == -1
+        assert mt.mt_k_attn_bwd_variant(mt.ATTN_BWD_AUTO) == mt.ATTN_BWD_FUSED
+    finally:
+        mt.mt_k_attn_bwd_variant(was)
